@@ -1,0 +1,197 @@
+"""fp64 CPU oracle for the Mamba-3 selective recurrence.
+
+TEST INFRASTRUCTURE ONLY: tests/, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` are the only
+callers.  The product package never imports this module, and this module
+imports nothing from the product package.
+
+The arithmetic lives in ``mamba3_oracle.c`` (plain C, fp64, pthreads over the
+independent (batch, head) units).  This file only compiles it with gcc,
+loads it with ctypes and marshals numpy arrays.
+
+Sources: the pages on the Mamba-3 paper -- "Mamba-3: 2x smaller state ..."
+(MarkTechPost, Korean translation) sections 1.1 (exponential-trapezoidal
+three-term update), 1.2 (complex state and the RoPE trick), 1.3 (MIMO rank-R
+input and output shapes).  The readout ``y = C^T h + D x`` is the standard SSM
+readout (the pages do not print it).
+
+Parity status of each entry point (what pins it) is listed in
+``tests/test_oracle_pins.py``; every function here is pinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mamba3_oracle.c")
+_LIB = os.path.join(_HERE, "libmamba3_oracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (fp64, -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-o", tmp, _SRC, "-lm", "-lpthread"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("batch", "seqlen", "nheads", "headdim", "dstate", "rank")]
+
+
+_P = ctypes.POINTER(ctypes.c_double)
+
+
+class _IO(ctypes.Structure):
+    _fields_ = [
+        (n, _P)
+        for n in (
+            "x", "B", "C", "theta", "dt", "lam", "A", "D",
+            "h0", "bprev0", "xprev0", "angle0",
+            "y", "h_out", "bprev_out", "xprev_out", "angle_out",
+        )
+    ]
+
+
+_lib = None
+
+
+def _bind(lib):
+    for name in ("m3o_scan_complex", "m3o_scan_rope"):
+        f = getattr(lib, name)
+        f.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_IO), ctypes.c_int,
+                      ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+        f.restype = ctypes.c_int
+    for name in ("m3o_scan_quadratic", "m3o_decode_step"):
+        f = getattr(lib, name)
+        f.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_IO), ctypes.c_int]
+        f.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+@dataclass
+class State:
+    """Decode state in the real frame rotated by -Phi (float64 numpy arrays).
+
+    h [b,H,N,P], b_prev [b,H,R,N], x_prev [b,H,R,P], angle [b,H,N/2].
+    """
+    h: np.ndarray
+    b_prev: np.ndarray
+    x_prev: np.ndarray
+    angle: np.ndarray
+
+    @staticmethod
+    def zeros(batch, nheads, headdim, dstate, rank) -> "State":
+        return State(
+            np.zeros((batch, nheads, dstate, headdim)),
+            np.zeros((batch, nheads, rank, dstate)),
+            np.zeros((batch, nheads, rank, headdim)),
+            np.zeros((batch, nheads, dstate // 2)),
+        )
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return a.ctypes.data_as(_P) if a is not None else None
+
+
+def _prepare(x, B, C, theta, dt, lam, A, D):
+    x, B, C, theta, dt, lam, A = map(_f64, (x, B, C, theta, dt, lam, A))
+    D = _f64(D) if D is not None else None
+    b, L, H, R, P = x.shape
+    N = B.shape[-1]
+    assert B.shape == (b, L, H, R, N) and C.shape == B.shape, "B/C must be [b,L,H,R,N]"
+    assert theta.shape == (b, L, H, N // 2), "theta must be [b,L,H,N/2]"
+    assert dt.shape == (b, L, H) and lam.shape == (b, L, H) and A.shape == (H,)
+    dims = _Dims(b, L, H, P, N, R)
+    return dims, (x, B, C, theta, dt, lam, A, D)
+
+
+def _run(fn_name, x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = None,
+         want_state=True, nthreads: Optional[int] = None, units=None):
+    lib = _load()
+    dims, arrs = _prepare(x, B, C, theta, dt, lam, A, D)
+    x, B, C, theta, dt, lam, A, D = arrs
+    b, L, H, R, P = x.shape
+    N = B.shape[-1]
+    y = np.zeros_like(x)
+    fin = State.zeros(b, H, P, N, R) if want_state else None
+    keep = [x, B, C, theta, dt, lam, A, D, y]
+    io = _IO()
+    io.x, io.B, io.C, io.theta, io.dt, io.lam, io.A, io.D = map(_ptr, (x, B, C, theta, dt, lam, A, D))
+    if init is not None:
+        ih, ib, ix, ia = (_f64(init.h), _f64(init.b_prev), _f64(init.x_prev), _f64(init.angle))
+        keep += [ih, ib, ix, ia]
+        io.h0, io.bprev0, io.xprev0, io.angle0 = map(_ptr, (ih, ib, ix, ia))
+    io.y = _ptr(y)
+    if fin is not None:
+        io.h_out, io.bprev_out, io.xprev_out, io.angle_out = map(
+            _ptr, (fin.h, fin.b_prev, fin.x_prev, fin.angle))
+    nt = nthreads if nthreads is not None else (os.cpu_count() or 1)
+    if fn_name in ("m3o_scan_complex", "m3o_scan_rope"):
+        if units is not None:
+            u = np.ascontiguousarray(np.asarray(units, dtype=np.int32))
+            keep.append(u)
+            rc = getattr(lib, fn_name)(ctypes.byref(dims), ctypes.byref(io), nt,
+                                       u.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), len(u))
+        else:
+            rc = getattr(lib, fn_name)(ctypes.byref(dims), ctypes.byref(io), nt, None, 0)
+    else:
+        rc = getattr(lib, fn_name)(ctypes.byref(dims), ctypes.byref(io), nt)
+    if rc != 0:
+        raise ValueError(f"{fn_name} rejected its arguments (rc={rc})")
+    return y, fin
+
+
+def scan_complex(x, B, C, theta, dt, lam, A, D=None, init=None, nthreads=None, units=None):
+    """The definition: explicit complex-diagonal state, sequential in t.
+
+    Returns (y [b,L,H,R,P], final State).  ``units`` optionally restricts the
+    work to a list of flattened (b*H + h) indices (others stay zero).
+    """
+    return _run("m3o_scan_complex", x, B, C, theta, dt, lam, A, D, init, True, nthreads, units)
+
+
+def scan_rope(x, B, C, theta, dt, lam, A, D=None, init=None, nthreads=None, units=None):
+    """Real state with B, C rotated by -Phi_t (the RoPE form)."""
+    return _run("m3o_scan_rope", x, B, C, theta, dt, lam, A, D, init, True, nthreads, units)
+
+
+def scan_quadratic(x, B, C, theta, dt, lam, A, D=None, init=None, nthreads=None):
+    """Materialised L x L masked-kernel form (brute force; tiny L only). Returns y."""
+    y, _ = _run("m3o_scan_quadratic", x, B, C, theta, dt, lam, A, D, init, False, nthreads)
+    return y
+
+
+def decode_step(state: State, x, B, C, theta, dt, lam, A, D=None, nthreads=None):
+    """One token continued from ``state``.
+
+    Per-token inputs are shaped without the L axis: x [b,H,R,P], B/C [b,H,R,N],
+    theta [b,H,N/2], dt/lam [b,H].  Returns (y [b,H,R,P], new State).
+    """
+    add = lambda a: _f64(a)[:, None]
+    y, fin = _run("m3o_decode_step", add(x), add(B), add(C), add(theta), add(dt), add(lam), A, D,
+                  state, True, nthreads)
+    return y[:, 0], fin
+
+
+__all__ = ["build", "State", "scan_complex", "scan_rope", "scan_quadratic", "decode_step"]

@@ -1,0 +1,65 @@
+"""The oracle's pins detect planted mistakes.
+
+Each case copies the oracle's C source, plants one plausible slip (a dropped
+term, a wrong sign, a conjugation or pairing swap), compiles the copy into a
+temporary library and checks that at least one pin of test_oracle_pins.py
+fails on it.  Everything runs on the CPU; the real oracle is untouched.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "mamba3_oracle.c")
+
+MUTATIONS = {
+    "drop_lag_term": ("(1.0 - lam) * dt * a[k] * u_prev[k * P + p]", "0.0 * u_prev[k * P + p]"),
+    "lag_without_pole": ("(1.0 - lam) * dt * a[k] * u_prev[k * P + p]", "(1.0 - lam) * dt * u_prev[k * P + p]"),
+    "lag_weight_lam": ("(1.0 - lam) * dt * a[k] * u_prev[k * P + p]", "lam * dt * a[k] * u_prev[k * P + p]"),
+    "rotation_sign": ("cexp(dt * (A + I * th[k]))", "cexp(dt * (A - I * th[k]))"),
+    "readout_no_conj": ("creal(conj(c) * Hs[k * P + p])", "creal(c * Hs[k * P + p])"),
+    "pair_swap": ("(Bt[r * N + 2 * k] + I * Bt[r * N + 2 * k + 1])", "(Bt[r * N + 2 * k + 1] + I * Bt[r * N + 2 * k])"),
+    "rope_sign": ("*o1 = -sin(phi) * v0 + cos(phi) * v1;", "*o1 = sin(phi) * v0 + cos(phi) * v1;"),
+    "quadratic_weight_next": ("(1.0 - io->lam[in]) * io->dt[in]", "(1.0 - io->lam[is]) * io->dt[is]"),
+    "mimo_rank_drop": ("for (int r = 0; r < R; ++r)\n          s += (Bt", "for (int r = 0; r < 1; ++r)\n          s += (Bt"),
+}
+
+PIN_FUNCS = [
+    lambda: [pins.test_time_invariant_equals_lfilter(l) for l in (0.0, 0.3, 0.5, 1.0)],
+    lambda: [pins.test_impulse_closed_form(f) for f in ("scan_complex", "scan_rope", "scan_quadratic")],
+    pins.test_lambda_one_is_exponential_euler,
+    pins.test_lambda_zero_is_pure_lag,
+    pins.test_theta_zero_is_real_ssm,
+    pins.test_parity_toy,
+    lambda: [pins.test_complex_equals_rope(r) for r in (1, 3)],
+    lambda: [pins.test_quadratic_equals_recurrence(r) for r in (1, 2)],
+    pins.test_mimo_is_superposition_of_siso,
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {name}"
+    mutated = src.replace(old, new, 1)
+    c = tmp_path / "mut.c"
+    so = tmp_path / "libmut.so"
+    c.write_text(mutated)
+    subprocess.check_call(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-o", str(so), str(c), "-lm", "-lpthread"])
+    saved = oracle._lib
+    oracle._lib = oracle._bind(ctypes.CDLL(str(so)))
+    try:
+        failed = 0
+        for f in PIN_FUNCS:
+            try:
+                f()
+            except AssertionError:
+                failed += 1
+        assert failed >= 1, f"no pin caught mutation {name}"
+    finally:
+        oracle._lib = saved
