@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the Mamba-3 recurrence on B200: prefill Mtokens/s and decode-step us.
+
+One JSON line on rank 0.  `value` is the chunked-prefill throughput on the
+SISO workload (batch 8, seqlen 2048, 64 heads, P 64, N 128, bf16 inputs, fp32
+state) summed over all ranks (weak scaling: every rank runs the full batch,
+no data-path collective).  A step is one `mamba3_scan_fwd` call over the
+batch, exporting the final state.  The decode step (batch 128, SISO and MIMO
+R=4, 1024 consecutive steps in one CUDA graph) is reported in the same line
+under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_recurrent_scan_b200 import workloads as wl  # noqa: E402
+
+PREFILL = wl.CONFIGS["siso_prefill_b8_l2048"]
+DECODE = [wl.CONFIGS["siso_decode_b128"], wl.CONFIGS["mimo4_decode_b128"]]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def esize(dt):
+    return torch.tensor([], dtype=dt).element_size()
+
+
+def prefill_bytes(w: wl.Workload, export_state=True) -> int:
+    """Algorithmic bytes of one prefill: every input read once, y written once,
+    the final state written once (A, D included)."""
+    s = esize(w.dtype)
+    th = w.token_heads
+    per_th = s * (2 * w.rank * w.headdim + 2 * w.rank * w.dstate + w.dstate // 2 + 2)
+    units = w.batch * w.nheads
+    state = 4 * units * (w.dstate * w.headdim + w.rank * w.dstate + w.rank * w.headdim + w.dstate // 2)
+    return th * per_th + (state if export_state else 0) + 8 * w.nheads
+
+
+def decode_bytes(w: wl.Workload) -> int:
+    """Algorithmic bytes of one decode step: the fp32 state read and written once,
+    the per-token inputs read once, y written once."""
+    s = esize(w.dtype)
+    units = w.batch * w.nheads
+    state = 4 * (w.dstate * w.headdim + w.rank * w.dstate + w.rank * w.headdim + w.dstate // 2)
+    io = s * (2 * w.rank * w.headdim + 2 * w.rank * w.dstate + w.dstate // 2 + 2)
+    return units * (2 * state + io) + 8 * w.nheads
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int, period_ms: int = 50):
+        self.device = device
+        self.period_ms = period_ms
+        self.proc = None
+
+    def start(self):
+        ident = []
+        try:
+            ident = [f"--id=GPU-{torch.cuda.get_device_properties(self.device).uuid}"]
+        except Exception:
+            pass
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *ident, f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __enter__(self):
+        return self.start()
+
+    def stop(self):
+        self.__exit__(None, None, None)
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- ranks
+def setup_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- our arm
+NAMES = ("x", "B", "C", "theta", "dt", "lam")
+
+
+def run_prefill(m3, args, world, rank, clk):
+    w = PREFILL
+    dev = torch.device("cuda")
+    inp = wl.make_inputs(w, seed=wl.BASE_SEED + rank, device=dev)
+    ins = [inp[n] for n in NAMES]
+    y = torch.empty_like(inp["x"])
+    fin = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
+    dims = m3.make_dims(inp["x"], inp["B"])
+    ws = torch.zeros(m3.mamba3_scan_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        m3.mamba3_scan_fwd(*ins, inp["A"], inp["D"], y=y, final_state=fin, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = m3.mamba3_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {m3.mamba3_status_string(status)}")
+
+    # timed region: events around every call (kernel duration) and around the whole loop
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.start()
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    launch_ms = max_over_ranks(launch_ms, world)
+    status = m3.mamba3_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {m3.mamba3_status_string(status)}")
+
+    # end to end through the same call with host buffers: pinned H2D of every
+    # input, the call, D2H of y, every step
+    host = {n: inp[n].cpu().pin_memory() for n in NAMES}
+    dev_in = {n: torch.empty_like(inp[n]) for n in NAMES}
+    yh = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = yh.numel() * yh.element_size()
+
+    def e2e_step():
+        for n in NAMES:
+            dev_in[n].copy_(host[n], non_blocking=True)
+        m3.mamba3_scan_fwd(*(dev_in[n] for n in NAMES), inp["A"], inp["D"], y=y, final_state=fin, workspace=ws,
+                           stream=stream)
+        yh.copy_(y, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    del host, dev_in
+    return dict(total_ms=total_ms, launch_ms=launch_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+                tokens=w.batch * w.seqlen, bytes=prefill_bytes(w))
+
+
+def run_decode(m3, w: wl.Workload, world, rank, steps):
+    """Seed the state with a 512-token prefill, then time `steps` decode steps
+    captured in one CUDA graph (per-step inputs pre-generated, larger than L2)."""
+    dev = torch.device("cuda")
+    pre = wl.make_inputs(w.with_(seqlen=w.prefill_tokens), seed=wl.BASE_SEED + rank, device=dev)
+    st = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
+    m3.mamba3_scan_fwd(*(pre[n] for n in NAMES), pre["A"], pre["D"], final_state=st)
+    A, D = pre["A"], pre["D"]
+    del pre
+    steps_in = wl.decode_inputs(w, steps, seed=wl.BASE_SEED + 1 + rank, device=dev)
+    ys = torch.empty((steps,) + steps_in["x"].shape[1:], dtype=w.dtype, device=dev)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    saved = st.clone()
+    with torch.cuda.stream(s):
+        for i in range(3):  # warm-up outside the graph
+            m3.mamba3_decode_step(st, *(steps_in[n][i] for n in NAMES), A, D, y=ys[i], stream=s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(steps):
+                m3.mamba3_decode_step(st, *(steps_in[n][i] for n in NAMES), A, D, y=ys[i], stream=s)
+    torch.cuda.synchronize()
+    times = []
+    for rep in range(3):
+        st.h.copy_(saved.h); st.b_prev.copy_(saved.b_prev); st.x_prev.copy_(saved.x_prev); st.angle.copy_(saved.angle)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        g.replay()
+        e1.record(s)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    us = max_over_ranks(min(times), world) * 1000.0 / steps
+    del g, steps_in, ys
+    torch.cuda.empty_cache()
+    return us
+
+
+def ours(args):
+    world, rank, local = setup_dist()
+    import linear_recurrent_scan_b200 as m3
+    m3.load_library()
+    peak, peak_kind = measured_peaks()
+    clk = ClockSampler(torch.cuda.current_device())
+    r = run_prefill(m3, args, world, rank, clk)
+    per_step_ms = r["total_ms"] / args.steps
+    tokens_all = r["tokens"] * world
+    value = tokens_all / (per_step_ms * 1e-3) / 1e6
+    achieved = r["bytes"] / (r["launch_ms"] * 1e-3) / 1e9
+    dec = {}
+    for w in DECODE:
+        us = run_decode(m3, w, world, rank, w.decode_steps)
+        gbs = decode_bytes(w) / (us * 1e-6) / 1e9
+        dec[w.name] = {"us_per_step": round(us, 2), "steps": w.decode_steps, "batch": w.batch, "rank": w.rank,
+                       "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                                    "frac": round(gbs / peak, 4), "traffic": None,
+                                    "bytes_per_step": decode_bytes(w)}}
+    clk.stop()
+    clocks = clk.summary()
+    clocks["window"] = "prefill timed steps through the decode graph replays"
+    e2e_value = tokens_all / (r["e2e_ms"] * 1e-3) / 1e6
+    out = {
+        "metric": "prefill Mtokens/s (SISO, batch 8, seqlen 2048) and decode step us at batch 128",
+        "value": round(value, 3),
+        "unit": "Mtokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(per_step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; distributions of the layer inputs, no dataset or weights)",
+        "config": {"workload": PREFILL.name, "batch": PREFILL.batch, "seqlen": PREFILL.seqlen,
+                   "nheads": PREFILL.nheads, "headdim": PREFILL.headdim, "dstate": PREFILL.dstate,
+                   "rank": PREFILL.rank, "state_dtype": "fp32", "parallelism": f"batch-sharded x{world} (weak)",
+                   "l2": "inputs (%.0f MB) larger than L2 (126 MB); no flush" % (r["bytes"] / 1e6)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                     "bytes_per_launch": r["bytes"], "launch_ms": round(r["launch_ms"], 4)},
+        "decode": dec,
+        "e2e": {"value": round(e2e_value, 3), "unit": "Mtokens/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        cpu = cpu_baseline(args)
+        if cpu is not None:
+            out["cpu_baseline"] = cpu
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- oracle arms
+class OracleSample:
+    """The fp64 oracle (as it stands, all host cores) on whole (batch, head)
+    units of the prefill workload, sized by a one-unit calibration."""
+
+    def __init__(self, target_s: float):
+        import oracle
+        self.oracle = oracle
+        w = PREFILL
+        self.threads = os.cpu_count() or 1
+        one_in = wl.to_f64({k: v for k, v in wl.make_inputs(w.with_(batch=1), device="cpu").items()})
+        t = time.perf_counter()
+        oracle.scan_complex(**one_in, units=[0], nthreads=1)
+        one = time.perf_counter() - t
+        units = int(target_s * self.threads / max(one, 1e-3))
+        self.units = max(1, min(units, w.batch * w.nheads))
+        batch = -(-self.units // w.nheads)
+        self.f = wl.to_f64(wl.make_inputs(w.with_(batch=batch), device="cpu"))
+
+    def run(self):
+        t = time.perf_counter()
+        self.oracle.scan_complex(**self.f, units=list(range(self.units)), nthreads=self.threads)
+        sec = time.perf_counter() - t
+        # tokens of the whole layer (all heads): units * L / H
+        return self.units * PREFILL.seqlen / PREFILL.nheads / sec / 1e6, sec
+
+    @property
+    def cores(self):
+        return min(self.threads, self.units)
+
+
+def cpu_baseline(args):
+    try:
+        o = OracleSample(target_s=12.0)
+        mtok, sec = o.run()
+    except Exception as e:  # the baseline is a report, never a reason to lose the line
+        return {"error": str(e)[:200]}
+    return {"value": round(mtok, 6), "unit": "Mtokens/s", "cores": o.cores, "kind": "oracle",
+            "sample": f"{o.units} of {PREFILL.batch * PREFILL.nheads} (batch, head) units of the prefill workload, "
+                      f"all {PREFILL.seqlen} tokens each, {sec:.1f} s"}
+
+
+def reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    times, vals = [], []
+    # each step a bounded sample (~3 s) so that warm-up + steps end in minutes
+    o = OracleSample(target_s=min(3.0, 150.0 / max(1, args.warmup + args.steps)))
+    units, threads = o.units, o.cores
+    for i in range(args.warmup + args.steps):
+        mtok, sec = o.run()
+        if i >= args.warmup:
+            times.append(sec)
+            vals.append(mtok)
+    value = statistics.median(vals)
+    out = {
+        "impl": "reference",
+        "metric": "prefill Mtokens/s (SISO, batch 8, seqlen 2048) and decode step us at batch 128",
+        "value": round(value, 6),
+        "unit": "Mtokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1000 * statistics.median(times), 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": PREFILL.name, "batch": PREFILL.batch, "seqlen": PREFILL.seqlen,
+                   "nheads": PREFILL.nheads, "headdim": PREFILL.headdim, "dstate": PREFILL.dstate,
+                   "rank": PREFILL.rank},
+        "cpu_baseline": {"value": round(value, 6), "unit": "Mtokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: {units} (batch, head) units x {PREFILL.seqlen} tokens on host cores"},
+        "e2e": {"value": round(value, 6), "unit": "Mtokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        reference(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,142 @@
+/*
+ * mamba3.h -- C ABI of the Mamba-3 selective-recurrence library (sm_100a).
+ *
+ * The layer's core computation, per (batch b, head h), token t = 1..L:
+ *
+ *   h_t = alpha_t h_{t-1} + beta_t B~_{t-1}^T x_{t-1} + gamma_t B~_t^T x_t
+ *   y_t = C~_t h_t + D_h x_t
+ *   alpha_t = exp(dt_t A_h),  beta_t = (1 - lam_t) dt_t alpha_t,  gamma_t = lam_t dt_t
+ *
+ * Sources (pages on the Mamba-3 paper, "Mamba-3: 2x smaller state ..." by
+ * MarkTechPost, Korean translation):
+ *   section 1.1  exponential-trapezoidal discretisation: the three-term update;
+ *   section 1.2  complex state via the RoPE trick: B~, C~ are B, C with each
+ *                adjacent pair (2k, 2k+1) rotated by -Phi_t,k where
+ *                Phi_t = Phi_0 + sum_{s<=t} dt_s theta_s (the angle accumulated
+ *                over time steps);
+ *   section 1.3  MIMO: B_t is N x R and x_t is P x R; B~_t^T x_t means
+ *                sum_r B~_t[r]^T x_t[r] and y_t has one P-vector per rank.
+ * The readout C~_t h_t + D x_t is the standard SSM readout (not printed on
+ * the pages).  A is one real scalar per head.
+ *
+ * Conventions (all entry points):
+ *  - Every pointer is a DEVICE pointer unless stated otherwise, owned by the
+ *    caller.  The library never allocates, frees or synchronises (except
+ *    mamba3_device_status, which synchronises the stream it is given); work
+ *    is enqueued on `stream` (a cudaStream_t passed as void*, NULL = legacy
+ *    default stream).
+ *  - Layouts are dense row-major with the last index fastest:
+ *      x, y      [batch, seqlen, nheads, rank, headdim]      (in_dtype)
+ *      B, C      [batch, seqlen, nheads, rank, dstate]       (in_dtype)
+ *      theta     [batch, seqlen, nheads, dstate/2]           (in_dtype)
+ *      dt, lam   [batch, seqlen, nheads]                     (in_dtype)
+ *      A, D      [nheads]                                    (float32)
+ *    For the decode step drop the seqlen axis.
+ *  - Every input and output pointer must be 16-byte aligned.
+ *  - Host-detectable errors return a negative status before anything is
+ *    enqueued.  No C++ exception crosses the ABI.  There is no CPU fallback:
+ *    without a CUDA device the calls return MAMBA3_ERR_CUDA.
+ */
+#ifndef MAMBA3_H
+#define MAMBA3_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define MAMBA3_API __attribute__((visibility("default")))
+#else
+#define MAMBA3_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MAMBA3_OK = 0,
+  MAMBA3_ERR_INVALID = -1,     /* null pointer, bad size, misaligned pointer */
+  MAMBA3_ERR_UNSUPPORTED = -2, /* valid arguments outside the compiled shapes */
+  MAMBA3_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required */
+  MAMBA3_ERR_CUDA = -4,        /* a CUDA runtime/driver call or launch failed */
+  MAMBA3_ERR_TIMEOUT = -5      /* a bounded on-device wait gave up (device status) */
+} mamba3_status;
+
+typedef enum { MAMBA3_F32 = 0, MAMBA3_BF16 = 1 } mamba3_dtype;
+
+typedef struct {
+  int batch;    /* b >= 1 */
+  int seqlen;   /* L >= 0 (ignored by mamba3_decode_step) */
+  int nheads;   /* H >= 1 */
+  int headdim;  /* P: multiple of 4 */
+  int dstate;   /* N: even */
+  int rank;     /* R: 1 (SISO) or 2, 4, 8 (MIMO) */
+  int chunk;    /* Q tokens per chunk for the prefill; 0 = library default */
+  mamba3_dtype in_dtype; /* dtype of x, B, C, theta, dt, lam and y */
+} mamba3_dims;
+
+/*
+ * Recurrent state of one layer (float32, device memory, caller-owned).
+ * It is what a decode step continues from and what a prefill exports:
+ *   h      [batch, nheads, dstate, headdim]  state in the frame rotated by -Phi
+ *                                            (row 2k = real, 2k+1 = imaginary part)
+ *   b_prev [batch, nheads, rank, dstate]     B~ of the last token (already rotated)
+ *   x_prev [batch, nheads, rank, headdim]    x of the last token
+ *   angle  [batch, nheads, dstate/2]         Phi of the last token, wrapped to [-pi, pi)
+ * A zero state (h = 0, b_prev = 0, x_prev = 0, angle = 0) is the start of a sequence.
+ */
+typedef struct {
+  float* h;
+  float* b_prev;
+  float* x_prev;
+  float* angle;
+} mamba3_state;
+
+/* Bytes of device workspace mamba3_scan_fwd needs for `dims` (>= 256; the
+ * first 256 bytes hold the device status word).  Returns 0 for invalid dims. */
+MAMBA3_API size_t mamba3_scan_workspace_bytes(const mamba3_dims* dims);
+
+/*
+ * Chunked prefill over a whole sequence (sections 1.1-1.3 above).
+ *   init         nullable: NULL = zero state; otherwise all four fields non-null.
+ *   D            nullable: NULL = no skip term.
+ *   final_state  nullable: NULL = do not export; otherwise all four fields
+ *                non-null.  It may alias `init` (in-place continuation).
+ *   workspace    device memory of at least mamba3_scan_workspace_bytes(dims);
+ *                its status word is reset by this call and read back with
+ *                mamba3_device_status.
+ * Numerics: float32 arithmetic and state; bf16 inputs feed bf16 tensor-core
+ * products with float32 accumulation.  y is written in in_dtype.
+ */
+MAMBA3_API int mamba3_scan_fwd(const mamba3_dims* dims, const void* x, const void* B, const void* C,
+                    const void* theta, const void* dt, const void* lam, const float* A,
+                    const float* D, const mamba3_state* init, void* y,
+                    const mamba3_state* final_state, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/*
+ * One decode step for every (batch, head), in place on `state`
+ * (section 1.3: the state is streamed once; the rank-R update and readout
+ * happen in registers).  Per-token inputs have no seqlen axis:
+ *   x [b,H,R,P], B/C [b,H,R,N], theta [b,H,N/2], dt/lam [b,H]; y [b,H,R,P].
+ * D nullable.  dims->seqlen and dims->chunk are ignored.
+ */
+MAMBA3_API int mamba3_decode_step(const mamba3_dims* dims, const mamba3_state* state, const void* x,
+                       const void* B, const void* C, const void* theta, const void* dt,
+                       const void* lam, const float* A, const float* D, void* y, void* stream);
+
+/* Synchronises `stream`, then returns the device status word that the last
+ * mamba3_scan_fwd on `workspace` left (MAMBA3_OK or MAMBA3_ERR_TIMEOUT), or
+ * MAMBA3_ERR_CUDA / MAMBA3_ERR_INVALID. */
+MAMBA3_API int mamba3_device_status(const void* workspace, void* stream);
+
+/* Static, human-readable text for a status code. */
+MAMBA3_API const char* mamba3_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+MAMBA3_API int mamba3_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA3_H */

@@ -1,0 +1,215 @@
+"""Mamba-3 selective recurrence on B200 (sm_100a): thin Python binding.
+
+The computation lives in ``libmamba3.so`` (hand-written CUDA, C ABI declared in
+``include/mamba3.h``).  This module only marshals torch tensors into the C
+calls: it checks shapes and dtypes, passes device pointers and the current
+CUDA stream, and raises on a non-zero status.  There is no CPU fallback; if
+the library has not been built the import of the C entry points fails.
+
+Entry points (same names as the C ABI):
+  mamba3_scan_workspace_bytes(dims)
+  mamba3_scan_fwd(x, B, C, theta, dt, lam, A, D=None, init=None, ...)
+  mamba3_decode_step(state, x, B, C, theta, dt, lam, A, D=None, ...)
+  mamba3_device_status(workspace)
+  mamba3_status_string(code)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmamba3.so")
+
+MAMBA3_OK = 0
+MAMBA3_ERR_INVALID = -1
+MAMBA3_ERR_UNSUPPORTED = -2
+MAMBA3_ERR_WORKSPACE = -3
+MAMBA3_ERR_CUDA = -4
+MAMBA3_ERR_TIMEOUT = -5
+MAMBA3_F32 = 0
+MAMBA3_BF16 = 1
+
+_DTYPES = {torch.float32: MAMBA3_F32, torch.bfloat16: MAMBA3_BF16}
+
+
+class Mamba3Error(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {mamba3_status_string(code)} (status {code})")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("seqlen", ctypes.c_int), ("nheads", ctypes.c_int),
+        ("headdim", ctypes.c_int), ("dstate", ctypes.c_int), ("rank", ctypes.c_int),
+        ("chunk", ctypes.c_int), ("in_dtype", ctypes.c_int),
+    ]
+
+
+class _CState(ctypes.Structure):
+    _fields_ = [("h", ctypes.c_void_p), ("b_prev", ctypes.c_void_p), ("x_prev", ctypes.c_void_p),
+                ("angle", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmamba3.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m linear_recurrent_scan_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, sz, i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    lib.mamba3_scan_workspace_bytes.argtypes = [ctypes.POINTER(Dims)]
+    lib.mamba3_scan_workspace_bytes.restype = sz
+    lib.mamba3_scan_fwd.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, vp, vp, vp, vp,
+                                    ctypes.POINTER(_CState), vp, ctypes.POINTER(_CState), vp, sz, vp]
+    lib.mamba3_scan_fwd.restype = i
+    lib.mamba3_decode_step.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(_CState), vp, vp, vp, vp, vp, vp,
+                                       vp, vp, vp, vp]
+    lib.mamba3_decode_step.restype = i
+    lib.mamba3_device_status.argtypes = [vp, vp]
+    lib.mamba3_device_status.restype = i
+    lib.mamba3_status_string.argtypes = [i]
+    lib.mamba3_status_string.restype = ctypes.c_char_p
+    lib.mamba3_version.argtypes = []
+    lib.mamba3_version.restype = i
+    _lib = lib
+    return lib
+
+
+@dataclass
+class State:
+    """Recurrent state (fp32 device tensors): h [b,H,N,P], b_prev [b,H,R,N],
+    x_prev [b,H,R,P], angle [b,H,N/2]."""
+    h: torch.Tensor
+    b_prev: torch.Tensor
+    x_prev: torch.Tensor
+    angle: torch.Tensor
+
+    @staticmethod
+    def zeros(batch, nheads, headdim, dstate, rank, device="cuda") -> "State":
+        z = lambda *s: torch.zeros(*s, dtype=torch.float32, device=device)
+        return State(z(batch, nheads, dstate, headdim), z(batch, nheads, rank, dstate),
+                     z(batch, nheads, rank, headdim), z(batch, nheads, dstate // 2))
+
+    def clone(self) -> "State":
+        return State(self.h.clone(), self.b_prev.clone(), self.x_prev.clone(), self.angle.clone())
+
+    def _c(self) -> _CState:
+        for t in (self.h, self.b_prev, self.x_prev, self.angle):
+            if t.dtype != torch.float32 or not t.is_contiguous():
+                raise ValueError("state tensors must be contiguous float32")
+        return _CState(self.h.data_ptr(), self.b_prev.data_ptr(), self.x_prev.data_ptr(), self.angle.data_ptr())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(code: int, where: str):
+    if code != MAMBA3_OK:
+        raise Mamba3Error(code, where)
+
+
+def make_dims(x: torch.Tensor, B: torch.Tensor, chunk: int = 0, decode: bool = False) -> Dims:
+    if decode:
+        b, H, R, P = x.shape
+        L = 1
+    else:
+        b, L, H, R, P = x.shape
+    if x.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    return Dims(b, L, H, P, B.shape[-1], R, chunk, _DTYPES[x.dtype])
+
+
+def mamba3_status_string(code: int) -> str:
+    return load_library().mamba3_status_string(code).decode()
+
+
+def mamba3_scan_workspace_bytes(dims: Dims) -> int:
+    return int(load_library().mamba3_scan_workspace_bytes(ctypes.byref(dims)))
+
+
+def _check_inputs(x, B, C, theta, dt, lam, A, D, decode):
+    lead = x.shape[:-2]
+    for name, t in (("x", x), ("B", B), ("C", C), ("theta", theta), ("dt", dt), ("lam", lam)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.dtype != x.dtype:
+            raise ValueError(f"{name} must have the dtype of x ({x.dtype})")
+        if t.device != x.device:
+            raise ValueError(f"{name} must be on the device of x")
+    if B.shape != C.shape or B.shape[:-1] != lead + (x.shape[-2],):
+        raise ValueError("B and C must be [..., R, N] with the leading shape of x")
+    if theta.shape != lead + (B.shape[-1] // 2,) or dt.shape != lead or lam.shape != lead:
+        raise ValueError("theta must be [..., N/2] and dt, lam [...] with the leading shape of x")
+    H = x.shape[-3]
+    for name, t in (("A", A), ("D", D)):
+        if t is not None and (t.dtype != torch.float32 or t.shape != (H,) or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous float32 tensor of shape [H]")
+
+
+def mamba3_scan_fwd(x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = None,
+                    y: Optional[torch.Tensor] = None, final_state: Optional[State] = None,
+                    workspace: Optional[torch.Tensor] = None, chunk: int = 0, stream=None):
+    """Chunked prefill. Shapes: x [b,L,H,R,P], B/C [b,L,H,R,N], theta [b,L,H,N/2],
+    dt/lam [b,L,H], A/D [H] fp32. Returns y (allocated if not given)."""
+    lib = load_library()
+    _check_inputs(x, B, C, theta, dt, lam, A, D, decode=False)
+    dims = make_dims(x, B, chunk)
+    if y is None:
+        y = torch.empty_like(x)
+    if workspace is None:
+        workspace = torch.empty(mamba3_scan_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
+    ci = init._c() if init is not None else None
+    cf = final_state._c() if final_state is not None else None
+    rc = lib.mamba3_scan_fwd(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam),
+                             _ptr(A), _ptr(D), ctypes.byref(ci) if ci is not None else None, _ptr(y),
+                             ctypes.byref(cf) if cf is not None else None, _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mamba3_scan_fwd")
+    return y
+
+
+def mamba3_decode_step(state: State, x, B, C, theta, dt, lam, A, D=None, y: Optional[torch.Tensor] = None,
+                       stream=None):
+    """One decode step in place on ``state``. Shapes: x [b,H,R,P], B/C [b,H,R,N],
+    theta [b,H,N/2], dt/lam [b,H]. Returns y [b,H,R,P]."""
+    lib = load_library()
+    _check_inputs(x, B, C, theta, dt, lam, A, D, decode=True)
+    dims = make_dims(x, B, decode=True)
+    if y is None:
+        y = torch.empty_like(x)
+    cs = state._c()
+    rc = lib.mamba3_decode_step(ctypes.byref(dims), ctypes.byref(cs), _ptr(x), _ptr(B), _ptr(C), _ptr(theta),
+                                _ptr(dt), _ptr(lam), _ptr(A), _ptr(D), _ptr(y), _stream(stream))
+    _check(rc, "mamba3_decode_step")
+    return y
+
+
+def mamba3_device_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(load_library().mamba3_device_status(_ptr(workspace), _stream(stream)))
+
+
+__all__ = [
+    "Dims", "State", "Mamba3Error", "load_library", "make_dims",
+    "mamba3_scan_workspace_bytes", "mamba3_scan_fwd", "mamba3_decode_step", "mamba3_device_status",
+    "mamba3_status_string",
+]

@@ -1,0 +1,43 @@
+// Internal launcher interface between the C ABI (mamba3_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/mamba3.h"
+
+namespace m3 {
+
+struct ScanArgs {
+  int batch, seqlen, nheads, P, N, R, Q;
+  mamba3_dtype dtype;
+  const void *x, *B, *C, *theta, *dt, *lam;
+  const float *A, *D;
+  const float *h0, *bprev0, *xprev0, *angle0;  // all null = zero state
+  void* y;
+  float *h_out, *bprev_out, *xprev_out, *angle_out;  // all null = no export
+  void* workspace;  // device status word at offset 0
+  size_t workspace_bytes;
+};
+
+struct DecodeArgs {
+  int batch, nheads, P, N, R;
+  mamba3_dtype dtype;
+  float *h, *bprev, *xprev, *angle;
+  const void *x, *B, *C, *theta, *dt, *lam;
+  const float *A, *D;
+  void* y;
+};
+
+// Each launcher returns MAMBA3_OK, MAMBA3_ERR_UNSUPPORTED (shape not compiled)
+// or MAMBA3_ERR_CUDA (launch failure).
+int decode_supported(const DecodeArgs& a);
+int launch_decode(const DecodeArgs& a, cudaStream_t s);
+
+int simt_scan_supported(const ScanArgs& a);
+int launch_scan_simt(const ScanArgs& a, cudaStream_t s);
+
+int tc_scan_supported(const ScanArgs& a);
+int launch_scan_tc(const ScanArgs& a, cudaStream_t s);
+
+}  // namespace m3

@@ -1,0 +1,144 @@
+// C ABI of the Mamba-3 recurrence library: argument validation and dispatch.
+// Every check runs on the host before anything is enqueued; the library never
+// allocates and never synchronises (except mamba3_device_status).
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int check_dims(const mamba3_dims* d, bool need_seqlen) {
+  if (!d) return MAMBA3_ERR_INVALID;
+  if (d->batch < 1 || d->nheads < 1 || d->headdim < 4 || d->dstate < 2) return MAMBA3_ERR_INVALID;
+  if (need_seqlen && d->seqlen < 0) return MAMBA3_ERR_INVALID;
+  if (d->headdim % 4 != 0 || d->dstate % 2 != 0) return MAMBA3_ERR_INVALID;
+  if (!(d->rank == 1 || d->rank == 2 || d->rank == 4 || d->rank == 8)) return MAMBA3_ERR_INVALID;
+  if (d->in_dtype != MAMBA3_F32 && d->in_dtype != MAMBA3_BF16) return MAMBA3_ERR_INVALID;
+  if (need_seqlen && d->chunk < 0) return MAMBA3_ERR_INVALID;
+  // every flattened index must fit comfortably in 64 bits and the grid in 31
+  const double tokens = (double)d->batch * (need_seqlen ? (d->seqlen > 0 ? d->seqlen : 1) : 1) * d->nheads;
+  const double row = (double)d->rank * (d->dstate > d->headdim ? d->dstate : d->headdim);
+  if (tokens * row > 9.0e15 || (double)d->batch * d->nheads > 2.0e9) return MAMBA3_ERR_INVALID;
+  if (d->dstate > 1024 || d->headdim > 1024) return MAMBA3_ERR_UNSUPPORTED;
+  return MAMBA3_OK;
+}
+
+int check_state(const mamba3_state* s) {
+  if (!s) return MAMBA3_OK;
+  if (!s->h || !s->b_prev || !s->x_prev || !s->angle) return MAMBA3_ERR_INVALID;
+  if (!aligned16(s->h) || !aligned16(s->b_prev) || !aligned16(s->x_prev) || !aligned4(s->angle))
+    return MAMBA3_ERR_INVALID;
+  return MAMBA3_OK;
+}
+
+int check_inputs(const void* x, const void* B, const void* C, const void* theta, const void* dt,
+                 const void* lam, const float* A, const float* D, const void* y) {
+  if (!x || !B || !C || !theta || !dt || !lam || !A || !y) return MAMBA3_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(theta) || !aligned16(y))
+    return MAMBA3_ERR_INVALID;
+  if (!aligned4(dt) || !aligned4(lam) || !aligned4(A) || (D && !aligned4(D))) return MAMBA3_ERR_INVALID;
+  return MAMBA3_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mamba3_version(void) { return 100; }
+
+const char* mamba3_status_string(int status) {
+  switch (status) {
+    case MAMBA3_OK: return "ok";
+    case MAMBA3_ERR_INVALID: return "invalid argument (null pointer, bad size or misaligned pointer)";
+    case MAMBA3_ERR_UNSUPPORTED: return "shape not supported by the compiled kernels";
+    case MAMBA3_ERR_WORKSPACE: return "workspace missing or too small";
+    case MAMBA3_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case MAMBA3_ERR_TIMEOUT: return "a bounded on-device wait gave up";
+  }
+  return "unknown status";
+}
+
+size_t mamba3_scan_workspace_bytes(const mamba3_dims* d) {
+  if (check_dims(d, true) != MAMBA3_OK) return 0;
+  return kStatusBytes;
+}
+
+int mamba3_scan_fwd(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                    const void* dt, const void* lam, const float* A, const float* D,
+                    const mamba3_state* init, void* y, const mamba3_state* final_state, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  int rc = check_dims(d, true);
+  if (rc) return rc;
+  if (d->seqlen > 0 && (rc = check_inputs(x, B, C, theta, dt, lam, A, D, y))) return rc;
+  if (d->seqlen == 0 && !A) return MAMBA3_ERR_INVALID;
+  if ((rc = check_state(init)) || (rc = check_state(final_state))) return rc;
+  if (!workspace || !aligned16(workspace)) return MAMBA3_ERR_WORKSPACE;
+  if (workspace_bytes < mamba3_scan_workspace_bytes(d)) return MAMBA3_ERR_WORKSPACE;
+
+  m3::ScanArgs a;
+  memset(&a, 0, sizeof(a));
+  a.batch = d->batch;
+  a.seqlen = d->seqlen;
+  a.nheads = d->nheads;
+  a.P = d->headdim;
+  a.N = d->dstate;
+  a.R = d->rank;
+  a.Q = d->chunk;
+  a.dtype = d->in_dtype;
+  a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.D = D;
+  if (init) { a.h0 = init->h; a.bprev0 = init->b_prev; a.xprev0 = init->x_prev; a.angle0 = init->angle; }
+  a.y = y;
+  if (final_state) {
+    a.h_out = final_state->h; a.bprev_out = final_state->b_prev;
+    a.xprev_out = final_state->x_prev; a.angle_out = final_state->angle;
+  }
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
+
+  const bool use_tc = m3::tc_scan_supported(a) == MAMBA3_OK;
+  if (!use_tc && (rc = m3::simt_scan_supported(a))) return rc;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  return use_tc ? m3::launch_scan_tc(a, s) : m3::launch_scan_simt(a, s);
+}
+
+int mamba3_decode_step(const mamba3_dims* d, const mamba3_state* state, const void* x, const void* B,
+                       const void* C, const void* theta, const void* dt, const void* lam, const float* A,
+                       const float* D, void* y, void* stream) {
+  int rc = check_dims(d, false);
+  if (rc) return rc;
+  if (!state) return MAMBA3_ERR_INVALID;
+  if ((rc = check_state(state))) return rc;
+  if ((rc = check_inputs(x, B, C, theta, dt, lam, A, D, y))) return rc;
+  m3::DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.batch = d->batch;
+  a.nheads = d->nheads;
+  a.P = d->headdim;
+  a.N = d->dstate;
+  a.R = d->rank;
+  a.dtype = d->in_dtype;
+  a.h = state->h; a.bprev = state->b_prev; a.xprev = state->x_prev; a.angle = state->angle;
+  a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.D = D; a.y = y;
+  if ((rc = m3::decode_supported(a))) return rc;
+  return m3::launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+
+int mamba3_device_status(const void* workspace, void* stream) {
+  if (!workspace) return MAMBA3_ERR_INVALID;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  m3::DeviceStatus st;
+  if (cudaMemcpy(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  return st.code;
+}
+
+}  // extern "C"

@@ -1,0 +1,161 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any CUDA call.
+
+Every call below either fails host validation (so nothing is ever enqueued,
+even on a machine with a GPU) or is skipped when a CUDA device is present.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import linear_recurrent_scan_b200 as m3
+from linear_recurrent_scan_b200 import build as m3build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    m3build.build()
+    return m3.load_library()
+
+
+def declared_symbols():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"MAMBA3_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_entry_points():
+    names = declared_symbols()
+    for n in ("mamba3_scan_fwd", "mamba3_decode_step", "mamba3_scan_workspace_bytes",
+              "mamba3_device_status", "mamba3_status_string", "mamba3_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", m3.LIB_PATH]).decode()
+    exported = set(re.findall(r"\sT\s(\w+)$", out, re.M))
+    missing = [n for n in declared_symbols() if n not in exported]
+    assert not missing, missing
+    for n in declared_symbols():
+        assert hasattr(lib, n)
+
+
+def test_no_driver_or_oracle_dependency(lib):
+    """The library links CUDA's runtime statically and never the oracle."""
+    out = subprocess.check_output(["ldd", m3.LIB_PATH]).decode()
+    assert "libcuda.so" not in out and "oracle" not in out
+
+
+def test_status_strings(lib):
+    assert m3.mamba3_status_string(0) == "ok"
+    for c in (-1, -2, -3, -4, -5):
+        assert m3.mamba3_status_string(c) != "unknown status"
+    assert m3.mamba3_status_string(17) == "unknown status"
+    assert lib.mamba3_version() >= 100
+
+
+def dims(**kw):
+    d = dict(batch=2, seqlen=64, nheads=3, headdim=16, dstate=16, rank=1, chunk=0, in_dtype=m3.MAMBA3_BF16)
+    d.update(kw)
+    return m3.Dims(**d)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(batch=0), dict(nheads=0), dict(headdim=6), dict(headdim=0), dict(dstate=15), dict(dstate=0),
+    dict(rank=3), dict(rank=0), dict(in_dtype=7), dict(seqlen=-1), dict(chunk=-2),
+])
+def test_workspace_bytes_rejects_bad_dims(lib, bad):
+    assert lib.mamba3_scan_workspace_bytes(ctypes.byref(dims(**bad))) == 0
+
+
+def test_workspace_bytes_valid(lib):
+    assert lib.mamba3_scan_workspace_bytes(ctypes.byref(dims())) >= 256
+    assert lib.mamba3_scan_workspace_bytes(None) == 0
+
+
+FAKE = 0x10000  # never dereferenced: every call using it fails validation first
+
+
+def scan(lib, d, ptrs=None, init=None, final=None, ws=FAKE, ws_bytes=1 << 20):
+    p = dict(x=FAKE, B=FAKE, C=FAKE, theta=FAKE, dt=FAKE, lam=FAKE, A=FAKE, D=None, y=FAKE)
+    p.update(ptrs or {})
+    return lib.mamba3_scan_fwd(ctypes.byref(d) if d is not None else None, p["x"], p["B"], p["C"], p["theta"],
+                               p["dt"], p["lam"], p["A"], p["D"], init, p["y"], final, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("name", ["x", "B", "C", "theta", "dt", "lam", "A", "y"])
+def test_scan_rejects_null_pointer(lib, name):
+    assert scan(lib, dims(), {name: None}) == m3.MAMBA3_ERR_INVALID
+
+
+@pytest.mark.parametrize("name", ["x", "B", "C", "theta", "y"])
+def test_scan_rejects_misaligned_pointer(lib, name):
+    assert scan(lib, dims(), {name: FAKE + 8}) == m3.MAMBA3_ERR_INVALID
+
+
+def test_scan_rejects_bad_dims_and_state(lib):
+    assert scan(lib, None) == m3.MAMBA3_ERR_INVALID
+    assert scan(lib, dims(rank=5)) == m3.MAMBA3_ERR_INVALID
+    half = m3._CState(FAKE, None, FAKE, FAKE)
+    assert scan(lib, dims(), init=ctypes.byref(half)) == m3.MAMBA3_ERR_INVALID
+    assert scan(lib, dims(), final=ctypes.byref(half)) == m3.MAMBA3_ERR_INVALID
+    mis = m3._CState(FAKE + 4, FAKE, FAKE, FAKE)
+    assert scan(lib, dims(), init=ctypes.byref(mis)) == m3.MAMBA3_ERR_INVALID
+
+
+def test_scan_rejects_workspace(lib):
+    assert scan(lib, dims(), ws=None) == m3.MAMBA3_ERR_WORKSPACE
+    assert scan(lib, dims(), ws_bytes=16) == m3.MAMBA3_ERR_WORKSPACE
+    assert scan(lib, dims(), ws=FAKE + 4) == m3.MAMBA3_ERR_WORKSPACE
+
+
+def test_scan_rejects_unsupported_shape(lib):
+    # a chunk whose rows do not fit the SIMT kernel and no tensor-core shape
+    assert scan(lib, dims(chunk=4096, in_dtype=m3.MAMBA3_F32)) == m3.MAMBA3_ERR_UNSUPPORTED
+    assert scan(lib, dims(dstate=4096)) == m3.MAMBA3_ERR_UNSUPPORTED
+
+
+def decode(lib, d, st=True, ptrs=None):
+    p = dict(x=FAKE, B=FAKE, C=FAKE, theta=FAKE, dt=FAKE, lam=FAKE, A=FAKE, D=None, y=FAKE)
+    p.update(ptrs or {})
+    cs = m3._CState(FAKE, FAKE, FAKE, FAKE) if st else None
+    return lib.mamba3_decode_step(ctypes.byref(d), ctypes.byref(cs) if cs is not None else None, p["x"], p["B"],
+                                  p["C"], p["theta"], p["dt"], p["lam"], p["A"], p["D"], p["y"], None)
+
+
+def test_decode_rejects(lib):
+    assert decode(lib, dims(), st=False) == m3.MAMBA3_ERR_INVALID
+    assert decode(lib, dims(), ptrs={"x": None}) == m3.MAMBA3_ERR_INVALID
+    assert decode(lib, dims(), ptrs={"B": FAKE + 2}) == m3.MAMBA3_ERR_INVALID
+    assert decode(lib, dims(headdim=12)) == m3.MAMBA3_ERR_UNSUPPORTED  # 128 % (P/4) != 0
+    assert decode(lib, dims(headdim=64, dstate=512)) == m3.MAMBA3_ERR_UNSUPPORTED
+
+
+def test_device_status_null(lib):
+    assert lib.mamba3_device_status(None, None) == m3.MAMBA3_ERR_INVALID
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_device_is_a_cuda_error(lib):
+    """No CPU fallback: with valid host arguments and no GPU the call fails in CUDA."""
+    assert scan(lib, dims()) == m3.MAMBA3_ERR_CUDA
+    assert decode(lib, dims()) == m3.MAMBA3_ERR_CUDA
+
+
+def test_python_binding_validates_shapes(lib):
+    x = torch.zeros(1, 4, 2, 1, 8, dtype=torch.bfloat16)
+    B = torch.zeros(1, 4, 2, 1, 16, dtype=torch.bfloat16)
+    th = torch.zeros(1, 4, 2, 7, dtype=torch.bfloat16)  # wrong: N/2 = 8
+    dt = torch.zeros(1, 4, 2, dtype=torch.bfloat16)
+    A = torch.zeros(2)
+    with pytest.raises(ValueError):
+        m3.mamba3_scan_fwd(x, B, B, th, dt, dt, A)
