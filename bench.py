@@ -269,9 +269,10 @@ def run_decode(m3, w: wl.Workload, world, rank, steps):
         torch.cuda.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(s)
-        g.replay()
-        e1.record(s)
+        with torch.cuda.stream(s):  # replay on the stream the events are recorded on
+            e0.record(s)
+            g.replay()
+            e1.record(s)
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1))
     us = max_over_ranks(min(times), world) * 1000.0 / steps

@@ -1,8 +1,657 @@
-// Tensor-core (tcgen05 + TMA) chunked prefill -- not built yet.
+// Chunked prefill of the Mamba-3 recurrence on the 5th-generation tensor
+// cores (tcgen05, accumulators in TMEM) fed by TMA (sm_100a, bf16 inputs).
+//
+// Method (derived from the three-term update of section 1.1, the RoPE trick of
+// section 1.2 and the MIMO shapes of section 1.3 of "Mamba-3: 2x smaller state
+// ..." (MarkTechPost, Korean translation)).  A chunk holds M = 128 rows, i.e.
+// Q = 128 / R tokens of R ranks each, row m = (token t = m / R, rank r = m % R).
+// With B~, C~ rotated by -Phi, the per-token log decay a_t = dt_t A, the
+// chunk-local cumulative sum cum_t, the trapezoid weight of column s
+//   w_s = lam_s dt_s + (1 - lam_{s+1}) dt_{s+1}
+// (the lagged term of step s+1 carries the same decay as the state, so it folds
+// into column s; at the end of the sequence the next token is absent) and the
+// carried state hbar (the state plus the next token's lagged term):
+//   S      = C~ B~^T                                         (M x M, K = N)
+//   P[m,j] = S[m,j] * { e^{cum_tm - cum_tj} w_tj  if t_j < t_m
+//                       lam_tm dt_tm               if t_j = t_m   (all rank pairs)
+//                       0                          if t_j > t_m }
+//   Y      = P X  +  diag(e^{cum_t}) C~ hbar_in  +  D X          (M x P)
+//   hbar_out = e^{cum_end} hbar_in + (diag(e^{cum_end - cum_t} w_t) B~)^T X
+// Every exponent is a difference of chunk-local sums, so nothing overflows.
+//
+// Design (one CTA per (batch, head), marching over the chunks; the state stays
+// on chip in fp32 registers of the epilogue warps):
+//   warp 0      TMA producer: B, C, X tiles of chunk c into a 2-stage ring
+//               (128-byte swizzle, the layout the MMA descriptors read).
+//   warp 1      TMEM allocator and single-thread MMA issuer.
+//   warps 2..5  "prep": decay scalars, accumulated angles (wrapped), RoPE of
+//               B and C in place in shared memory, then B~ scaled in place by
+//               e^{cum_end - cum_t} w_t for the state MMA.
+//   warps 6..9  "epilogue" (one TMEM lane per thread): mask S into P (bf16,
+//               shared memory), the state update hbar (fp32 registers) and its
+//               bf16 copy for the next chunk's inter-chunk MMA, and y.
+// MMAs per chunk: S = C~ B~^T; Yi = C~ hbar_in; Hacc = B~s^T X; Y = P X.
+// TMEM columns: S [0,128), Y [128,192), Yi x2 [192,320), Hacc x2 [320,448).
+// Every wait is bounded: on expiry the CTA raises an abort flag, reports
+// MAMBA3_ERR_TIMEOUT in the device status word, drains and returns.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace m3 {
-int tc_scan_supported(const ScanArgs&) { return MAMBA3_ERR_UNSUPPORTED; }
-int launch_scan_tc(const ScanArgs&, cudaStream_t) { return MAMBA3_ERR_UNSUPPORTED; }
+namespace {
+
+using namespace ptx;
+
+constexpr int kP = 64;          // head dim handled by this kernel
+constexpr int kM = 128;         // rows per chunk (MMA M)
+constexpr int kTile = 16384;    // one 128-row x 128-byte swizzled tile
+constexpr int kStages = 2;
+constexpr int kThreads = 320;   // 10 warps
+constexpr int kPrep0 = 64;      // first prep thread
+constexpr int kEpi0 = 192;      // first epilogue thread
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColY = 128, kColYi = 192, kColH = 320;
+
+enum Tag { kTagEmpty = 1, kTagFull, kTagPrep1, kTagPrep2, kTagSFull, kTagSFree, kTagAcc, kTagHb, kTagP, kTagY, kTagDrain };
+
+template <int N, int R>
+struct Cfg {
+  static constexpr int Q = kM / R;     // tokens per chunk
+  static constexpr int NKB = N / 64;   // 64-wide blocks of the state dimension
+  static constexpr int K2 = N / 2;     // rotation pairs
+  static constexpr int NPART = 128 / K2;
+  static constexpr int TP = Q / NPART; // tokens per prep thread in the angle scan
+  static constexpr int STAGE_BYTES = (2 * NKB + 1) * kTile;
+  static constexpr int OFF_B = 0, OFF_C = NKB * kTile, OFF_X = 2 * NKB * kTile;
+  static constexpr int OFF_P = kStages * STAGE_BYTES;  // masked scores, 2 tiles (K = 128)
+  static constexpr int OFF_H = OFF_P + 2 * kTile;      // hbar bf16, N rows x 128 bytes
+  static constexpr int OFF_SC = OFF_H + N * 128;       // scalars
+  // per stage scalar arrays (float, Q each): c2 (log2 cum), w, gam, ws (state scale), dt
+  static constexpr int SC_PER_STAGE = 5 * Q;
+  static constexpr int OFF_PART = OFF_SC + kStages * SC_PER_STAGE * 4;  // angle partials [NPART][K2]
+  static constexpr int OFF_PHI = OFF_PART + NPART * K2 * 4;            // running base angle [K2]
+  static constexpr int OFF_WARP = OFF_PHI + K2 * 4;                     // scan scratch [8]
+  static constexpr int OFF_BAR = (OFF_WARP + 32 + 7) & ~7;
+  static constexpr int NBAR = 16;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
+  static constexpr int SMEM = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = SMEM + 1024;       // slack for 1024-byte alignment
+  static_assert(TP >= 1 && TP * NPART == Q, "angle partition");
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+};
+
+// barrier slots
+enum Bar { bFull0 = 0, bFull1, bEmpty0, bEmpty1, bPrep1, bPrep2, bSFull, bSFree, bAcc, bHb, bPReady, bYFull, bDone };
+
+struct TcParams {
+  ScanArgs a;
+  int nchunks;
+};
+
+__device__ __forceinline__ size_t tok_index(const ScanArgs& a, int b, int t, int h) {
+  return ((size_t)b * a.seqlen + t) * a.nheads + h;
+}
+
+// byte offset of 16-byte chunk `c` (0..7) of row `row` inside a 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t swz(int row, int c) { return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4)); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(v);
+}
+
+// named barrier for the 128 prep threads (id 1)
+__device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+
+// named barrier over the 128 prep threads that also ORs a predicate across them,
+// so that every prep thread takes the same abort decision
+__device__ __forceinline__ bool prep_sync_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+// ------------------------------------------------------------------ prep warps
+// Decay scalars, accumulated angles, RoPE of B and C in place, then B~ scaled
+// in place for the state MMA.  Thread pt in [0,128).
+template <int N, int R>
+__device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh, float Ah,
+                                          uint64_t* bars, volatile int* abort_flag, DeviceStatus* status,
+                                          float* phi) {
+  using K = Cfg<N, R>;
+  constexpr int Q = K::Q, K2 = K::K2, TP = K::TP;
+  const int pt = threadIdx.x - kPrep0;
+  const int L = a.seqlen;
+  const __nv_bfloat16* DT = static_cast<const __nv_bfloat16*>(a.dt);
+  const __nv_bfloat16* LM = static_cast<const __nv_bfloat16*>(a.lam);
+  const __nv_bfloat16* TH = static_cast<const __nv_bfloat16*>(a.theta);
+  float* part_sum = reinterpret_cast<float*>(smem + K::OFF_PART);
+  float* warp_tot = reinterpret_cast<float*>(smem + K::OFF_WARP);
+  const size_t unit = (size_t)b * a.nheads + hh;
+  const int pk = pt % K2, part = pt / K2;
+
+  if (pt < K2) phi[pt] = a.angle0 ? a.angle0[unit * K2 + pt] : 0.f;
+  prep_sync();
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int s = c & 1, u = c >> 1;
+    const int t0 = c * Q;
+    float* sc = reinterpret_cast<float*>(smem + K::OFF_SC) + s * K::SC_PER_STAGE;
+    float *c2 = sc, *wv = sc + Q, *gm = sc + 2 * Q, *wsc = sc + 3 * Q, *dts = sc + 4 * Q;
+    uint8_t* st = smem + s * K::STAGE_BYTES;
+
+    // ---- decay scalars (thread = token) ----
+    float dt = 0.f, lm = 1.f, dtn = 0.f, lmn = 1.f;
+    if (pt < Q) {
+      const int tg = t0 + pt;
+      if (tg < L) {
+        const size_t i = tok_index(a, b, tg, hh);
+        dt = __bfloat162float(DT[i]);
+        lm = __bfloat162float(LM[i]);
+      }
+      if (tg + 1 < L) {
+        const size_t i = tok_index(a, b, tg + 1, hh);
+        dtn = __bfloat162float(DT[i]);
+        lmn = __bfloat162float(LM[i]);
+      }
+    }
+    // inclusive scan of dt*A*log2(e) over the chunk's tokens
+    float v = (pt < Q) ? dt * Ah * kLog2e : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float n = __shfl_up_sync(0xffffffffu, v, o);
+      if ((pt & 31) >= o) v += n;
+    }
+    mbar_wait(&bars[bFull0 + s], u & 1, abort_flag, status, kTagFull);
+    if ((pt & 31) == 31) warp_tot[pt >> 5] = v;
+    if (prep_sync_any(*abort_flag != 0)) return;  // one decision for all 128 prep threads
+    for (int w = 0; w < (pt >> 5); ++w) v += warp_tot[w];
+    if (pt < Q) {
+      const float gam = lm * dt;
+      c2[pt] = v;
+      gm[pt] = gam;
+      wv[pt] = gam + (1.f - lmn) * dtn;
+      dts[pt] = dt;
+    }
+    prep_sync();
+    const float c2end = c2[Q - 1];
+    if (pt < Q) wsc[pt] = wv[pt] * ex2(c2end - c2[pt]);
+
+    // ---- accumulated angles: thread = (pair pk, token part) ----
+    float inc[TP];
+    float loc = 0.f;
+#pragma unroll
+    for (int i = 0; i < TP; ++i) {
+      const int t = part * TP + i, tg = t0 + t;
+      const float th = (tg < L) ? __bfloat162float(TH[tok_index(a, b, tg, hh) * K2 + pk]) : 0.f;
+      inc[i] = dts[t] * th;
+      loc += inc[i];
+    }
+    part_sum[part * K2 + pk] = loc;
+    const float base = phi[pk];
+    prep_sync();
+    float run = base;
+    for (int p2 = 0; p2 < part; ++p2) run += part_sum[p2 * K2 + pk];
+    // rotate pair pk of every row of this part's tokens by -angle
+    const int kb = (2 * pk) / 64;
+    const int e = (2 * pk) % 64;  // element inside the 64-wide block
+    const int cidx = e >> 3, within = (e & 7) * 2;
+    const bool last_chunk = (c == nchunks - 1);
+#pragma unroll
+    for (int i = 0; i < TP; ++i) {
+      run += inc[i];
+      const int t = part * TP + i;
+      float sn, cs;
+      __sincosf(wrap_angle(run), &sn, &cs);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int row = t * R + r;
+        const uint32_t off = kb * kTile + swz(row, cidx) + within;
+        uint32_t* pb = reinterpret_cast<uint32_t*>(st + K::OFF_B + off);
+        uint32_t* pc = reinterpret_cast<uint32_t*>(st + K::OFF_C + off);
+        const float2 bv = unpack_bf16(*pb), cv = unpack_bf16(*pc);
+        const float b0 = cs * bv.x + sn * bv.y, b1 = -sn * bv.x + cs * bv.y;
+        *pb = pack_bf16(b0, b1);
+        *pc = pack_bf16(cs * cv.x + sn * cv.y, -sn * cv.x + cs * cv.y);
+        if (last_chunk && t0 + t == L - 1 && a.bprev_out) {
+          a.bprev_out[(unit * R + r) * N + 2 * pk] = b0;
+          a.bprev_out[(unit * R + r) * N + 2 * pk + 1] = b1;
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&bars[bPrep1]);
+    if (part == 0) {
+      float tot = base;
+      for (int p2 = 0; p2 < K::NPART; ++p2) tot += part_sum[p2 * K2 + pk];
+      phi[pk] = wrap_angle(tot);
+    }
+    if (last_chunk && a.xprev_out && L > 0) {
+      const __nv_bfloat16* xl = static_cast<const __nv_bfloat16*>(a.x) + tok_index(a, b, L - 1, hh) * R * kP;
+      for (int i = pt; i < R * kP; i += 128) a.xprev_out[unit * R * kP + i] = __bfloat162float(xl[i]);
+    }
+
+    // ---- B~ scaled in place by e^{cum_end - cum_t} w_t once S has read it ----
+    mbar_wait(&bars[bSFull], c & 1, abort_flag, status, kTagSFull);
+    if (prep_sync_any(*abort_flag != 0)) return;
+    {
+      const int row = pt;
+      const float f = wsc[row / R];
+#pragma unroll
+      for (int kb2 = 0; kb2 < K::NKB; ++kb2) {
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint4* p = reinterpret_cast<uint4*>(st + K::OFF_B + kb2 * kTile + swz(row, c8));
+          uint4 q = *p;
+          float2 f0 = unpack_bf16(q.x), f1 = unpack_bf16(q.y), f2 = unpack_bf16(q.z), f3 = unpack_bf16(q.w);
+          q.x = pack_bf16(f * f0.x, f * f0.y);
+          q.y = pack_bf16(f * f1.x, f * f1.y);
+          q.z = pack_bf16(f * f2.x, f * f2.y);
+          q.w = pack_bf16(f * f3.x, f * f3.y);
+          *p = q;
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&bars[bPrep2]);
+  }
+  if (pt < K2 && a.angle_out) a.angle_out[unit * K2 + pt] = phi[pt];
+}
+
+// ------------------------------------------------------------------ epilogue warps
+// One TMEM lane per thread: row m = 32 (warp % 4) + lane of S, Y, Yi; state
+// row n of Hacc / hbar (for N = 64 the M = 64 accumulator uses lanes 0..15 of
+// each 32-lane quadrant).
+template <int N, int R>
+__device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh, float Ah,
+                                         uint64_t* bars, volatile int* abort_flag, DeviceStatus* status,
+                                         uint32_t tmem) {
+  using K = Cfg<N, R>;
+  constexpr int Q = K::Q;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quad = warp & 3;
+  const int m = quad * 32 + lane;        // chunk row of S, Y, Yi, P
+  const int tm = m / R, rm = m % R;      // token and rank of row m
+  const int n = (N == 128) ? m : (lane < 16 ? quad * 16 + lane : -1);  // state row of hbar
+  const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+  const int L = a.seqlen;
+  const size_t unit = (size_t)b * a.nheads + hh;
+  const float Dh = a.D ? a.D[hh] : 0.f;
+  uint8_t* Pt = smem + K::OFF_P;
+  uint8_t* Hs = smem + K::OFF_H;
+
+  // ---- initial carried state hbar_0 = h_0 + (1 - lam_1) dt_1 B~_0^T x_0 ----
+  float hb[kP];
+#pragma unroll
+  for (int p = 0; p < kP; ++p) hb[p] = 0.f;
+  if (n >= 0 && a.h0 != nullptr && L > 0) {
+    const size_t i0 = tok_index(a, b, 0, hh);
+    const float mu1 = (1.f - __bfloat162float(static_cast<const __nv_bfloat16*>(a.lam)[i0])) *
+                      __bfloat162float(static_cast<const __nv_bfloat16*>(a.dt)[i0]);
+    const float* h0 = a.h0 + (unit * N + n) * kP;
+#pragma unroll
+    for (int p = 0; p < kP; ++p) hb[p] = h0[p];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float bp = mu1 * a.bprev0[(unit * R + r) * N + n];
+      const float* xp = a.xprev0 + (unit * R + r) * kP;
+#pragma unroll
+      for (int p = 0; p < kP; ++p) hb[p] += bp * xp[p];
+    }
+  }
+  auto store_hbar_bf16 = [&]() {
+    if (n >= 0) {
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint4 q;
+        q.x = pack_bf16(hb[8 * c8 + 0], hb[8 * c8 + 1]);
+        q.y = pack_bf16(hb[8 * c8 + 2], hb[8 * c8 + 3]);
+        q.z = pack_bf16(hb[8 * c8 + 4], hb[8 * c8 + 5]);
+        q.w = pack_bf16(hb[8 * c8 + 6], hb[8 * c8 + 7]);
+        *reinterpret_cast<uint4*>(Hs + swz(n, c8)) = q;
+      }
+    }
+  };
+  store_hbar_bf16();
+  fence_proxy_async_smem();
+  mbar_arrive(&bars[bHb]);
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int s = c & 1;
+    const int t0 = c * Q;
+    const float* sc = reinterpret_cast<const float*>(smem + K::OFF_SC) + s * K::SC_PER_STAGE;
+    const float *c2 = sc, *wv = sc + Q, *gm = sc + 2 * Q;
+
+    // ---- mask S into P ----
+    mbar_wait(&bars[bPrep1], c & 1, abort_flag, status, kTagPrep1);
+    mbar_wait(&bars[bSFull], c & 1, abort_flag, status, kTagSFull);
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
+    tc_fence_after();
+    const float my_c2 = c2[tm];
+    const float my_gam = gm[tm];
+    const float my_e = ex2(my_c2);
+    const float e_end = ex2(c2[Q - 1]);
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+      float sv[32];
+      if (blk <= quad) {  // warp-uniform: columns past the warp's last token are all zero
+        tmem_ld32(tmem + lane_base + kColS + 32 * blk, sv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int tj = (32 * blk + jj) / R;
+          float kf;
+          if (tj < tm)
+            kf = ex2(my_c2 - c2[tj]) * wv[tj];
+          else if (tj == tm)
+            kf = my_gam;
+          else
+            kf = 0.f;
+          sv[jj] *= kf;
+        }
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) sv[jj] = 0.f;
+      }
+      // columns 32*blk .. +31 live in k-block blk/2, 16-byte chunks 4*(blk&1) .. +3
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint4 q;
+        q.x = pack_bf16(sv[8 * q4 + 0], sv[8 * q4 + 1]);
+        q.y = pack_bf16(sv[8 * q4 + 2], sv[8 * q4 + 3]);
+        q.z = pack_bf16(sv[8 * q4 + 4], sv[8 * q4 + 5]);
+        q.w = pack_bf16(sv[8 * q4 + 6], sv[8 * q4 + 7]);
+        *reinterpret_cast<uint4*>(Pt + (blk >> 1) * kTile + swz(m, 4 * (blk & 1) + q4)) = q;
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(&bars[bSFree]);
+    fence_proxy_async_smem();
+    mbar_arrive(&bars[bPReady]);
+
+    // ---- state update hbar = e^{cum_end} hbar + Hacc ----
+    mbar_wait(&bars[bAcc], c & 1, abort_flag, status, kTagAcc);
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
+    tc_fence_after();
+    {
+      float acc[32];
+      const uint32_t cH = kColH + (c & 1) * 64;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        tmem_ld32(tmem + lane_base + cH + 32 * half, acc);
+        tmem_ld_wait();
+#pragma unroll
+        for (int p = 0; p < 32; ++p) hb[32 * half + p] = e_end * hb[32 * half + p] + acc[p];
+      }
+    }
+    store_hbar_bf16();
+    if (c == nchunks - 1 && a.h_out != nullptr && n >= 0) {
+      float* ho = a.h_out + (unit * N + n) * kP;
+#pragma unroll
+      for (int p = 0; p < kP; p += 4) *reinterpret_cast<float4*>(ho + p) = make_float4(hb[p], hb[p + 1], hb[p + 2], hb[p + 3]);
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&bars[bHb]);
+
+    // ---- y = Y + e^{cum_t} Yi + D x ----
+    mbar_wait(&bars[bYFull], c & 1, abort_flag, status, kTagY);
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
+    tc_fence_after();
+    const int tg = t0 + tm;
+    const size_t row = tok_index(a, b, tg < L ? tg : 0, hh) * R + rm;
+    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.x) + row * kP);
+    uint4* yr = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) + row * kP);
+    const uint32_t cYi = kColYi + (c & 1) * 64;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float yv[32], yi[32];
+      tmem_ld32(tmem + lane_base + kColY + 32 * half, yv);
+      tmem_ld32(tmem + lane_base + cYi + 32 * half, yi);
+      tmem_ld_wait();
+      if (tg < L) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 xq = xr[4 * half + q4];
+          const float2 x0 = unpack_bf16(xq.x), x1 = unpack_bf16(xq.y), x2 = unpack_bf16(xq.z), x3 = unpack_bf16(xq.w);
+          const int o = 8 * q4;
+          uint4 q;
+          q.x = pack_bf16(yv[o + 0] + my_e * yi[o + 0] + Dh * x0.x, yv[o + 1] + my_e * yi[o + 1] + Dh * x0.y);
+          q.y = pack_bf16(yv[o + 2] + my_e * yi[o + 2] + Dh * x1.x, yv[o + 3] + my_e * yi[o + 3] + Dh * x1.y);
+          q.z = pack_bf16(yv[o + 4] + my_e * yi[o + 4] + Dh * x2.x, yv[o + 5] + my_e * yi[o + 5] + Dh * x2.y);
+          q.w = pack_bf16(yv[o + 6] + my_e * yi[o + 6] + Dh * x3.x, yv[o + 7] + my_e * yi[o + 7] + Dh * x3.y);
+          yr[4 * half + q4] = q;
+        }
+      }
+    }
+    tc_fence_before();
+  }
+}
+
+template <int N, int R>
+__global__ void __launch_bounds__(kThreads, 1)
+    scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
+                   const __grid_constant__ CUtensorMap tmX, const TcParams prm) {
+  using K = Cfg<N, R>;
+  constexpr int Q = K::Q;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const ScanArgs& a = prm.a;
+  const int nchunks = prm.nchunks;
+  const int unit = blockIdx.x;
+  const int b = unit / a.nheads, hh = unit % a.nheads;
+  const int L = a.seqlen;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + K::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::OFF_MISC + 4);
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.workspace);
+  float* phi = reinterpret_cast<float*>(smem + K::OFF_PHI);
+  const float Ah = a.A[hh];
+
+  if (tid == 0) {
+    mbar_init(&bars[bFull0], 1);
+    mbar_init(&bars[bFull1], 1);
+    mbar_init(&bars[bEmpty0], 1);
+    mbar_init(&bars[bEmpty1], 1);
+    mbar_init(&bars[bPrep1], 128);
+    mbar_init(&bars[bPrep2], 128);
+    mbar_init(&bars[bSFull], 1);
+    mbar_init(&bars[bSFree], 128);
+    mbar_init(&bars[bAcc], 1);
+    mbar_init(&bars[bHb], 128);
+    mbar_init(&bars[bPReady], 128);
+    mbar_init(&bars[bYFull], 1);
+    mbar_init(&bars[bDone], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
+    prefetch_tmap(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1, u = c >> 1;
+        if (!mbar_wait(&bars[bEmpty0 + s], (u & 1) ^ 1, abort_flag, status, kTagEmpty)) break;
+        uint8_t* st = smem + s * K::STAGE_BYTES;
+        mbar_arrive_expect_tx(&bars[bFull0 + s], K::STAGE_BYTES);
+        const int t0 = c * Q;
+#pragma unroll
+        for (int kb = 0; kb < K::NKB; ++kb) {
+          tma_load_5d(st + K::OFF_B + kb * kTile, &tmB, &bars[bFull0 + s], kb * 64, 0, hh, t0, b);
+          tma_load_5d(st + K::OFF_C + kb * kTile, &tmC, &bars[bFull0 + s], kb * 64, 0, hh, t0, b);
+        }
+        tma_load_5d(st + K::OFF_X, &tmX, &bars[bFull0 + s], 0, 0, hh, t0, b);
+        issued = c + 1;
+      }
+      // drain: never leave this CTA with bulk copies still landing in its smem
+      for (int c = issued - 2; c < issued; ++c)
+        if (c >= 0) mbar_wait(&bars[bFull0 + (c & 1)], (c >> 1) & 1, abort_flag, status, kTagDrain, 400000000LL);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t iS = idesc_bf16(kM, kM, 0, 0);     // S = C~ B~^T
+      const uint32_t iYi = idesc_bf16(kM, kP, 0, 1);    // Yi = C~ hbar
+      const uint32_t iH = idesc_bf16(N, kP, 1, 1);      // Hacc = B~s^T X
+      const uint32_t iY = idesc_bf16(kM, kP, 0, 1);     // Y = P X
+      const uint32_t sbase = smem_u32(smem);
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1;
+        const uint32_t st = sbase + s * K::STAGE_BYTES;
+        const uint32_t cB = st + K::OFF_B, cC = st + K::OFF_C, cX = st + K::OFF_X;
+        if (!mbar_wait(&bars[bPrep1], c & 1, abort_flag, status, kTagPrep1)) break;
+        if (c > 0 && !mbar_wait(&bars[bSFree], (c - 1) & 1, abort_flag, status, kTagSFree)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < N / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
+          mma_bf16_ss(tmem + kColS, smem_desc_sw128(cC + off, 16, 1024), smem_desc_sw128(cB + off, 16, 1024), iS,
+                      kk > 0);
+        }
+        mma_commit(&bars[bSFull]);
+        if (!mbar_wait(&bars[bPrep2], c & 1, abort_flag, status, kTagPrep2)) break;
+        if (!mbar_wait(&bars[bHb], c & 1, abort_flag, status, kTagHb)) break;
+        tc_fence_after();
+        const uint32_t cYi = kColYi + (c & 1) * 64, cH = kColH + (c & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < N / 16; ++kk) {
+          const uint32_t offa = (kk >> 2) * kTile + (kk & 3) * 32;
+          mma_bf16_ss(tmem + cYi, smem_desc_sw128(cC + offa, 16, 1024),
+                      smem_desc_sw128(sbase + K::OFF_H + kk * 2048, N * 128, 1024), iYi, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kM / 16; ++kk) {
+          mma_bf16_ss(tmem + cH, smem_desc_sw128(cB + kk * 2048, kTile, 1024),
+                      smem_desc_sw128(cX + kk * 2048, kTile, 1024), iH, kk > 0);
+        }
+        mma_commit(&bars[bAcc]);
+        if (!mbar_wait(&bars[bPReady], c & 1, abort_flag, status, kTagP)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kM / 16; ++kk) {
+          const uint32_t offa = (kk >> 2) * kTile + (kk & 3) * 32;
+          mma_bf16_ss(tmem + kColY, smem_desc_sw128(sbase + K::OFF_P + offa, 16, 1024),
+                      smem_desc_sw128(cX + kk * 2048, kTile, 1024), iY, kk > 0);
+        }
+        mma_commit(&bars[bYFull]);
+        mma_commit(&bars[bEmpty0 + s]);
+      }
+      // every MMA this thread issued must be complete before TMEM is released
+      mma_commit(&bars[bDone]);
+      mbar_wait(&bars[bDone], 0, abort_flag, status, kTagDrain, 400000000LL);
+    }
+  } else if (tid < kEpi0) {
+    prep_role<N, R>(smem, a, nchunks, b, hh, Ah, bars, abort_flag, status, phi);
+  } else {
+    epi_role<N, R>(smem, a, nchunks, b, hh, Ah, bars, abort_flag, status, tmem);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [batch, L, H, R, inner] bf16 tensor, box = {64, R, 1, Q, 1}, 128-byte swizzle,
+// zero fill past the end of the sequence.
+bool make_map(CUtensorMap* m, const void* base, int inner, const ScanArgs& a, int Q) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[5] = {(cuuint64_t)inner, (cuuint64_t)a.R, (cuuint64_t)a.nheads, (cuuint64_t)a.seqlen,
+                              (cuuint64_t)a.batch};
+  const cuuint64_t e = 2;
+  const cuuint64_t strides[4] = {e * inner, e * inner * a.R, e * inner * a.R * a.nheads,
+                                 e * inner * a.R * a.nheads * a.seqlen};
+  const cuuint32_t box[5] = {64, (cuuint32_t)a.R, 1, (cuuint32_t)Q, 1};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int N, int R>
+int launch_nr(const ScanArgs& a, cudaStream_t s) {
+  using K = Cfg<N, R>;
+  CUtensorMap tmB, tmC, tmX;
+  if (!make_map(&tmB, a.B, N, a, K::Q) || !make_map(&tmC, a.C, N, a, K::Q) || !make_map(&tmX, a.x, kP, a, K::Q))
+    return MAMBA3_ERR_CUDA;
+  TcParams prm;
+  prm.a = a;
+  prm.nchunks = (a.seqlen + K::Q - 1) / K::Q;
+  auto kern = scan_tc_kernel<N, R>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess)
+    return MAMBA3_ERR_CUDA;
+  kern<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmC, tmX, prm);
+  return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
+}
+
+}  // namespace
+
+int tc_scan_supported(const ScanArgs& a) {
+  if (a.dtype != MAMBA3_BF16 || a.P != kP || a.seqlen < 1) return MAMBA3_ERR_UNSUPPORTED;
+  if (a.N != 64 && a.N != 128) return MAMBA3_ERR_UNSUPPORTED;
+  if (a.R != 1 && a.R != 2 && a.R != 4) return MAMBA3_ERR_UNSUPPORTED;
+  if (a.Q != 0 && a.Q != kM / a.R) return MAMBA3_ERR_UNSUPPORTED;
+  return MAMBA3_OK;
+}
+
+int launch_scan_tc(const ScanArgs& a, cudaStream_t s) {
+  if (a.N == 128) {
+    if (a.R == 1) return launch_nr<128, 1>(a, s);
+    if (a.R == 2) return launch_nr<128, 2>(a, s);
+    if (a.R == 4) return launch_nr<128, 4>(a, s);
+  } else {
+    if (a.R == 1) return launch_nr<64, 1>(a, s);
+    if (a.R == 2) return launch_nr<64, 2>(a, s);
+    if (a.R == 4) return launch_nr<64, 4>(a, s);
+  }
+  return MAMBA3_ERR_UNSUPPORTED;
+}
+
 }  // namespace m3

@@ -189,3 +189,16 @@ def test_decode_single_step_vs_oracle_step(R):
     yr, fr = oracle.decode_step(ref0, *(f[n] for n in NAMES), f["A"], f["D"])
     assert rel_err(y.cpu().double().numpy(), yr) < 1e-4
     check_state(st, fr, 1e-4)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_chunk_size_invariance(dtype):
+    """The chunk length is a blocking choice only: chunks of 1, 8, 32, 64 tokens (SIMT path)
+    and the tensor-core default (128 rows) all match the oracle."""
+    b, L, H, P, N, R = 1, 300, 2, 64, 128, 1
+    inp = small_inputs(b, L, H, P, N, R, dtype, seed=900)
+    yr, fr = oracle_scan(inp)
+    for chunk in (1, 8, 32, 64, 0):
+        y, fin = gpu_scan(inp, chunk=chunk)
+        assert rel_err(y.float().cpu().double().numpy(), yr) < TOL[dtype], chunk
+        check_state(fin, fr, TOL[dtype])
