@@ -1,0 +1,61 @@
+"""Run a few prefills (and optionally decode steps) of one workload, for profilers.
+
+    python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --batch 2 --reps 3
+    python -m linear_recurrent_scan_b200.profile_case --workload siso_decode_b128 --decode --reps 3
+
+Inputs are seeded synthetic tensors on cuda:0.  Prints the CUDA-event time
+of each call; under a profiler those times are not benchmark numbers.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+import linear_recurrent_scan_b200 as m3
+from linear_recurrent_scan_b200 import workloads as wl
+
+NAMES = ("x", "B", "C", "theta", "dt", "lam")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="siso_prefill_b8_l2048", choices=sorted(wl.CONFIGS))
+    ap.add_argument("--batch", type=int, default=0, help="override the batch size (0 = workload's)")
+    ap.add_argument("--seqlen", type=int, default=0, help="override the sequence length (0 = workload's)")
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--decode", action="store_true", help="time decode steps instead of the prefill")
+    args = ap.parse_args()
+    w = wl.CONFIGS[args.workload]
+    if args.batch:
+        w = w.with_(batch=args.batch)
+    if args.seqlen:
+        w = w.with_(seqlen=args.seqlen)
+    dev = torch.device("cuda", 0)
+    m3.load_library()
+    st = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
+    if args.decode:
+        pre = wl.make_inputs(w.with_(seqlen=max(1, w.prefill_tokens)), device=dev)
+        m3.mamba3_scan_fwd(*(pre[n] for n in NAMES), pre["A"], pre["D"], final_state=st)
+        steps = wl.decode_inputs(w, args.reps, device=dev)
+        for i in range(args.reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            m3.mamba3_decode_step(st, *(steps[n][i] for n in NAMES), pre["A"], pre["D"])
+            e1.record()
+            torch.cuda.synchronize()
+            print(f"decode step {i}: {e0.elapsed_time(e1) * 1000:.1f} us")
+        return
+    inp = wl.make_inputs(w, device=dev)
+    y = torch.empty_like(inp["x"])
+    for i in range(args.reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        m3.mamba3_scan_fwd(*(inp[n] for n in NAMES), inp["A"], inp["D"], y=y, final_state=st)
+        e1.record()
+        torch.cuda.synchronize()
+        print(f"prefill {w.name} b{w.batch} L{w.seqlen} rep {i}: {e0.elapsed_time(e1):.3f} ms")
+
+
+if __name__ == "__main__":
+    main()
