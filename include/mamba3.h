@@ -129,6 +129,43 @@ MAMBA3_API int mamba3_decode_step(const mamba3_dims* dims, const mamba3_state* s
  * MAMBA3_ERR_CUDA / MAMBA3_ERR_INVALID. */
 MAMBA3_API int mamba3_device_status(const void* workspace, void* stream);
 
+/*
+ * Bytes of library-owned device scratch behind mamba3_scan_fwd_noalloc
+ * (a file-scope device array; every GPU that loads the library holds it
+ * until the process exits).
+ */
+#define MAMBA3_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/*
+ * mamba3_scan_fwd without a workspace argument.  The pages on the method have
+ * no counterpart for this entry point; it exists for callers that cannot call
+ * cudaMalloc themselves: code embedded in a host framework that owns all device
+ * memory through its own pool (an allocation outside the pool can fail against
+ * the pool's reservation), latency-critical serving loops (cudaMalloc/cudaFree
+ * may synchronise the device and stall other streams), and runtimes that fix
+ * their memory budget at start-up.
+ *
+ * Arguments, layouts and results are those of mamba3_scan_fwd; the scratch is
+ * MAMBA3_NOALLOC_SCRATCH_BYTES of library-owned device memory instead of a
+ * caller workspace.  Nothing is allocated and nothing is freed.
+ *  - The first call on a device (with that device current) looks the scratch's
+ *    device address up once (cudaGetSymbolAddress); make that first call
+ *    before any stream capture on that device.
+ *  - Problems that need more scratch than MAMBA3_NOALLOC_SCRATCH_BYTES
+ *    (mamba3_scan_workspace_bytes) are rejected with MAMBA3_ERR_WORKSPACE
+ *    before anything is enqueued.
+ *  - Every call on a device shares the same scratch and it keeps the last
+ *    call's contents; the parts that must start at zero (the device status
+ *    word) are cleared by each call on its stream.  Calls that overlap on the
+ *    GPU (different streams without ordering between them) race on it.
+ *  - The device status word stays in the library's scratch: use
+ *    mamba3_scan_fwd with a caller workspace when mamba3_device_status is needed.
+ */
+MAMBA3_API int mamba3_scan_fwd_noalloc(const mamba3_dims* dims, const void* x, const void* B, const void* C,
+                                       const void* theta, const void* dt, const void* lam, const float* A,
+                                       const float* D, const mamba3_state* init, void* y,
+                                       const mamba3_state* final_state, void* stream);
+
 /* Static, human-readable text for a status code. */
 MAMBA3_API const char* mamba3_status_string(int status);
 

@@ -204,12 +204,38 @@ def mamba3_decode_step(state: State, x, B, C, theta, dt, lam, A, D=None, y: Opti
     return y
 
 
+def mamba3_scan_fwd_noalloc(x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = None,
+                            y: Optional[torch.Tensor] = None, final_state: Optional[State] = None,
+                            chunk: int = 0, stream=None):
+    """The prefill with the library's own scratch instead of a workspace tensor,
+    for callers that cannot allocate device memory (see mamba3.h).  Passing no
+    ``y`` makes this wrapper allocate one with torch; pass ``y`` to allocate nothing."""
+    lib = load_library()
+    f = lib.mamba3_scan_fwd_noalloc
+    f.argtypes = [ctypes.POINTER(Dims), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(_CState),
+                  ctypes.c_void_p, ctypes.POINTER(_CState), ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    _check_inputs(x, B, C, theta, dt, lam, A, D, decode=False)
+    dims = make_dims(x, B, chunk)
+    if y is None:
+        y = torch.empty_like(x)
+    ci = init._c() if init is not None else None
+    cf = final_state._c() if final_state is not None else None
+    rc = f(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam), _ptr(A), _ptr(D),
+           ctypes.byref(ci) if ci is not None else None, _ptr(y), ctypes.byref(cf) if cf is not None else None,
+           _stream(stream))
+    _check(rc, "mamba3_scan_fwd_noalloc")
+    return y
+
+
 def mamba3_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(load_library().mamba3_device_status(_ptr(workspace), _stream(stream)))
 
 
 __all__ = [
     "Dims", "State", "Mamba3Error", "load_library", "make_dims",
-    "mamba3_scan_workspace_bytes", "mamba3_scan_fwd", "mamba3_decode_step", "mamba3_device_status",
+    "mamba3_scan_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc", "mamba3_decode_step",
+    "mamba3_device_status",
     "mamba3_status_string",
 ]
