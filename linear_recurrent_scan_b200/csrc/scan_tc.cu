@@ -14,24 +14,27 @@
 //   S      = C~ B~^T                                         (M x M, K = N)
 //   P[m,j] = S[m,j] * { e^{cum_tm - cum_tj} w_tj  if t_j < t_m
 //                       lam_tm dt_tm               if t_j = t_m   (all rank pairs)
-//                       0                          if t_j > t_m }
-//   Y      = P X  +  diag(e^{cum_t}) C~ hbar_in  +  D X          (M x P)
-//   hbar_out = e^{cum_end} hbar_in + (diag(e^{cum_end - cum_t} w_t) B~)^T X
-// Every exponent is a difference of chunk-local sums, so nothing overflows.
+//                       0                          if t_j > t_m }  + D [m = j]
+//   Y      = P X  +  diag(e^{cum_t}) C~ hbar_in                   (M x P)
+//   hbar_out = e^{cum_end} hbar_in + B~^T diag(e^{cum_end - cum_t} w_t) X
+// Every exponent is a difference of chunk-local sums (<= 0), so nothing
+// overflows.  The skip term D x rides on the diagonal of P.
 //
-// Design (one CTA per (batch, head), marching over the chunks; the state stays
-// on chip in fp32 registers of the epilogue warps):
-//   warp 0      TMA producer: B, C, X tiles of chunk c into a 2-stage ring
-//               (128-byte swizzle, the layout the MMA descriptors read).
-//   warp 1      TMEM allocator and single-thread MMA issuer.
-//   warps 2..5  "prep": decay scalars, accumulated angles (wrapped), RoPE of
-//               B and C in place in shared memory, then B~ scaled in place by
-//               e^{cum_end - cum_t} w_t for the state MMA.
-//   warps 6..9  "epilogue" (one TMEM lane per thread): mask S into P (bf16,
-//               shared memory), the state update hbar (fp32 registers) and its
-//               bf16 copy for the next chunk's inter-chunk MMA, and y.
-// MMAs per chunk: S = C~ B~^T; Yi = C~ hbar_in; Hacc = B~s^T X; Y = P X.
-// TMEM columns: S [0,128), Y [128,192), Yi x2 [192,320), Hacc x2 [320,448).
+// Design: one CTA per (batch, head) marches over its chunks; the state stays on
+// chip, in fp32 registers of the epilogue warps.  18 warps:
+//   warp 0       TMA producer: B, C, X tiles of chunk c into a 2-stage ring
+//                (128-byte swizzle, the layout the MMA descriptors read).
+//   warp 1       TMEM allocator and single-thread MMA issuer.
+//   warps 2..9   prep: decay scalars and the rank-1 decay factors of the mask,
+//                X_w = diag(e^{cum_end - cum_t} w_t) X, accumulated angles
+//                (wrapped) and RoPE of B and C in place, 16 bytes per access.
+//                Prep runs up to two chunks ahead of the MMAs.
+//   warps 10..17 epilogue, two warps per TMEM lane quadrant (column halves):
+//                S -> P (bf16, back into TMEM), hbar update and its bf16 copy
+//                for the next chunk's inter-chunk MMA, y = Y + e^{cum} Yi.
+// MMAs per chunk: S = C~ B~^T; Yi = C~ hbar_in; Hacc = B~^T X_w (smem operands);
+// Y = P X (P from TMEM).  TMEM columns: S [0,128), P [128,192) (bf16 pairs),
+// Y [192,256), Yi [256,320), Hacc [320,384).
 // Every wait is bounded: on expiry the CTA raises an abort flag, reports
 // MAMBA3_ERR_TIMEOUT in the device status word, drains and returns.
 #include <cuda.h>
@@ -49,28 +52,32 @@ constexpr int kP = 64;          // head dim handled by this kernel
 constexpr int kM = 128;         // rows per chunk (MMA M)
 constexpr int kTile = 16384;    // one 128-row x 128-byte swizzled tile
 constexpr int kStages = 2;
-constexpr int kThreads = 320;   // 10 warps
+constexpr int kThreads = 576;   // 18 warps
 constexpr int kPrep0 = 64;      // first prep thread
-constexpr int kEpi0 = 192;      // first epilogue thread
+constexpr int kNPrep = 256;
+constexpr int kEpi0 = kPrep0 + kNPrep;
+constexpr int kNEpi = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColY = 128, kColYi = 192, kColH = 320;
+constexpr uint32_t kColS = 0, kColP = 128, kColY = 192, kColYi = 256, kColH = 320;
 
-enum Tag { kTagEmpty = 1, kTagFull, kTagPrep1, kTagPrep2, kTagSFull, kTagSFree, kTagAcc, kTagHb, kTagP, kTagY, kTagDrain };
+enum Tag { kTagEmpty = 1, kTagFull, kTagPrep1, kTagSFull, kTagAcc, kTagEpiDone, kTagP, kTagY, kTagDrain };
 
 template <int N, int R>
 struct Cfg {
   static constexpr int Q = kM / R;     // tokens per chunk
   static constexpr int NKB = N / 64;   // 64-wide blocks of the state dimension
   static constexpr int K2 = N / 2;     // rotation pairs
-  static constexpr int NPART = 128 / K2;
-  static constexpr int TP = Q / NPART; // tokens per prep thread in the angle scan
-  static constexpr int STAGE_BYTES = (2 * NKB + 1) * kTile;
-  static constexpr int OFF_B = 0, OFF_C = NKB * kTile, OFF_X = 2 * NKB * kTile;
-  static constexpr int OFF_P = kStages * STAGE_BYTES;  // masked scores, 2 tiles (K = 128)
-  static constexpr int OFF_H = OFF_P + 2 * kTile;      // hbar bf16, N rows x 128 bytes
+  static constexpr int NG = K2 / 4;    // groups of 4 pairs (16 bytes of a row)
+  static constexpr int NPART = kNPrep / NG;  // token parts of the angle scan
+  static constexpr int TPP = (Q + NPART - 1) / NPART;  // tokens per part (last part may be short)
+  static constexpr int STAGE_BYTES = (2 * NKB + 2) * kTile;  // B, C, X, X_w
+  static constexpr int TMA_BYTES = (2 * NKB + 1) * kTile;    // B, C, X
+  static constexpr int OFF_B = 0, OFF_C = NKB * kTile, OFF_X = 2 * NKB * kTile, OFF_XW = (2 * NKB + 1) * kTile;
+  static constexpr int OFF_H = kStages * STAGE_BYTES;  // hbar bf16, N rows x 128 bytes
   static constexpr int OFF_SC = OFF_H + N * 128;       // scalars
-  // per stage scalar arrays (float, Q each): c2 (log2 cum), w, gam, ws (state scale), dt
-  static constexpr int SC_PER_STAGE = 5 * Q;
+  // per stage (floats): c2[Q] (log2 of the chunk-local decay), gam[Q], wv[Q],
+  // wsc[Q] (X_w row scale), dt[Q], colf[192] (rank-1 column factors of the mask)
+  static constexpr int SC_PER_STAGE = 5 * Q + 192;
   static constexpr int OFF_PART = OFF_SC + kStages * SC_PER_STAGE * 4;  // angle partials [NPART][K2]
   static constexpr int OFF_PHI = OFF_PART + NPART * K2 * 4;            // running base angle [K2]
   static constexpr int OFF_WARP = OFF_PHI + K2 * 4;                     // scan scratch [8]
@@ -79,12 +86,12 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
   static constexpr int SMEM = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;       // slack for 1024-byte alignment
-  static_assert(TP >= 1 && TP * NPART == Q, "angle partition");
+  static_assert(NG * NPART == kNPrep, "angle partition");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
 // barrier slots
-enum Bar { bFull0 = 0, bFull1, bEmpty0, bEmpty1, bPrep1, bPrep2, bSFull, bSFree, bAcc, bHb, bPReady, bYFull, bDone };
+enum Bar { bFull0 = 0, bFull1, bEmpty0, bEmpty1, bPrep0, bPrep1, bSFull, bAcc, bEpiDone, bPReady, bYFull, bDone };
 
 struct TcParams {
   ScanArgs a;
@@ -103,47 +110,45 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
-  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
-  return __bfloat1622float2(v);
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
-// named barrier for the 128 prep threads (id 1)
-__device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-
-// named barrier over the 128 prep threads that also ORs a predicate across them,
+// named barrier over the 256 prep threads (id 1) that also ORs a predicate,
 // so that every prep thread takes the same abort decision
 __device__ __forceinline__ bool prep_sync_any(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.or.pred p, 1, 128, q;\n\t"
+      "bar.red.or.pred p, 1, 256, q;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)v)
       : "memory");
   return r != 0;
 }
+__device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // ------------------------------------------------------------------ prep warps
-// Decay scalars, accumulated angles, RoPE of B and C in place, then B~ scaled
-// in place for the state MMA.  Thread pt in [0,128).
+// Thread pt in [0,256).  Per chunk: decay scalars (thread = token), the rank-1
+// column factors of the mask, X_w, the angle scan (thread = group of 4 pairs x
+// token part) and RoPE of B and C in place, 16 bytes per shared-memory access.
 template <int N, int R>
 __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh, float Ah,
-                                          uint64_t* bars, volatile int* abort_flag, DeviceStatus* status,
-                                          float* phi) {
+                                          uint64_t* bars, volatile int* abort_flag, DeviceStatus* status) {
   using K = Cfg<N, R>;
-  constexpr int Q = K::Q, K2 = K::K2, TP = K::TP;
+  constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, TPP = K::TPP;
   const int pt = threadIdx.x - kPrep0;
   const int L = a.seqlen;
   const __nv_bfloat16* DT = static_cast<const __nv_bfloat16*>(a.dt);
   const __nv_bfloat16* LM = static_cast<const __nv_bfloat16*>(a.lam);
   const __nv_bfloat16* TH = static_cast<const __nv_bfloat16*>(a.theta);
   float* part_sum = reinterpret_cast<float*>(smem + K::OFF_PART);
+  float* phi = reinterpret_cast<float*>(smem + K::OFF_PHI);
   float* warp_tot = reinterpret_cast<float*>(smem + K::OFF_WARP);
   const size_t unit = (size_t)b * a.nheads + hh;
-  const int pk = pt % K2, part = pt / K2;
+  const int g = pt % NG, part = pt / NG;  // 4-pair group (one 16-byte chunk of a row), token part
+  const int kb = g / 8, c8 = g % 8;       // 64-element block and 16-byte chunk of the group
 
   if (pt < K2) phi[pt] = a.angle0 ? a.angle0[unit * K2 + pt] : 0.f;
   prep_sync();
@@ -152,10 +157,11 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
     const int s = c & 1, u = c >> 1;
     const int t0 = c * Q;
     float* sc = reinterpret_cast<float*>(smem + K::OFF_SC) + s * K::SC_PER_STAGE;
-    float *c2 = sc, *wv = sc + Q, *gm = sc + 2 * Q, *wsc = sc + 3 * Q, *dts = sc + 4 * Q;
+    float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *wsc = sc + 3 * Q, *dts = sc + 4 * Q, *colf = sc + 5 * Q;
     uint8_t* st = smem + s * K::STAGE_BYTES;
+    const bool last_chunk = (c == nchunks - 1);
 
-    // ---- decay scalars (thread = token) ----
+    // ---- global loads first: dt, lam of this token and the next; theta of this thread's part ----
     float dt = 0.f, lm = 1.f, dtn = 0.f, lmn = 1.f;
     if (pt < Q) {
       const int tg = t0 + pt;
@@ -170,6 +176,13 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
         lmn = __bfloat162float(LM[i]);
       }
     }
+    uint2 thv[TPP];
+#pragma unroll
+    for (int i = 0; i < TPP; ++i) {
+      const int tg = t0 + part * TPP + i;
+      thv[i] = (tg < L) ? *reinterpret_cast<const uint2*>(TH + tok_index(a, b, tg, hh) * K2 + 4 * g)
+                        : make_uint2(0u, 0u);
+    }
     // inclusive scan of dt*A*log2(e) over the chunk's tokens
     float v = (pt < Q) ? dt * Ah * kLog2e : 0.f;
 #pragma unroll
@@ -179,7 +192,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
     }
     mbar_wait(&bars[bFull0 + s], u & 1, abort_flag, status, kTagFull);
     if ((pt & 31) == 31) warp_tot[pt >> 5] = v;
-    if (prep_sync_any(*abort_flag != 0)) return;  // one decision for all 128 prep threads
+    if (prep_sync_any(*abort_flag != 0)) return;  // one decision for all prep threads
     for (int w = 0; w < (pt >> 5); ++w) v += warp_tot[w];
     if (pt < Q) {
       const float gam = lm * dt;
@@ -191,254 +204,289 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
     prep_sync();
     const float c2end = c2[Q - 1];
     if (pt < Q) wsc[pt] = wv[pt] * ex2(c2end - c2[pt]);
-
-    // ---- accumulated angles: thread = (pair pk, token part) ----
-    float inc[TP];
-    float loc = 0.f;
-#pragma unroll
-    for (int i = 0; i < TP; ++i) {
-      const int t = part * TP + i, tg = t0 + t;
-      const float th = (tg < L) ? __bfloat162float(TH[tok_index(a, b, tg, hh) * K2 + pk]) : 0.f;
-      inc[i] = dts[t] * th;
-      loc += inc[i];
+    if (pt < 192) {  // column factors e^{cum_ref - cum_tj} w_tj of the off-diagonal mask blocks
+      const int qq = pt < 32 ? 1 : (pt < 96 ? 2 : 3);
+      const int j = pt - (qq == 1 ? 0 : (qq == 2 ? 32 : 96));
+      const int tj = j / R, tref = (32 * qq) / R;
+      colf[pt] = ex2(c2[tref] - c2[tj]) * wv[tj];
     }
-    part_sum[part * K2 + pk] = loc;
-    const float base = phi[pk];
-    prep_sync();
-    float run = base;
-    for (int p2 = 0; p2 < part; ++p2) run += part_sum[p2 * K2 + pk];
-    // rotate pair pk of every row of this part's tokens by -angle
-    const int kb = (2 * pk) / 64;
-    const int e = (2 * pk) % 64;  // element inside the 64-wide block
-    const int cidx = e >> 3, within = (e & 7) * 2;
-    const bool last_chunk = (c == nchunks - 1);
+
+    // ---- angle increments of this thread's 4 pairs and tokens ----
+    float loc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < TP; ++i) {
-      run += inc[i];
-      const int t = part * TP + i;
-      float sn, cs;
-      __sincosf(wrap_angle(run), &sn, &cs);
+    for (int i = 0; i < TPP; ++i) {
+      const float d = dts[part * TPP + i];
+      const float2 t01 = unpack_bf16(thv[i].x), t23 = unpack_bf16(thv[i].y);
+      loc[0] += d * t01.x;
+      loc[1] += d * t01.y;
+      loc[2] += d * t23.x;
+      loc[3] += d * t23.y;
+    }
+    *reinterpret_cast<float4*>(part_sum + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
+    const float4 base = *reinterpret_cast<const float4*>(phi + 4 * g);
+    prep_sync();
+
+    // ---- X_w = diag(e^{cum_end - cum_t} w_t) X (B operand of the state MMA) ----
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = pt + kNPrep * i;
+      const int row = idx >> 3, cc = idx & 7;
+      const float f = wsc[row / R];
+      const uint4 q = *reinterpret_cast<const uint4*>(st + K::OFF_X + swz(row, cc));
+      const float2 f0 = unpack_bf16(q.x), f1 = unpack_bf16(q.y), f2 = unpack_bf16(q.z), f3 = unpack_bf16(q.w);
+      uint4 o;
+      o.x = pack_bf16(f * f0.x, f * f0.y);
+      o.y = pack_bf16(f * f1.x, f * f1.y);
+      o.z = pack_bf16(f * f2.x, f * f2.y);
+      o.w = pack_bf16(f * f3.x, f * f3.y);
+      *reinterpret_cast<uint4*>(st + K::OFF_XW + swz(row, cc)) = o;
+    }
+
+    // ---- accumulated angle at the start of this part, then RoPE of every row ----
+    float run[4] = {base.x, base.y, base.z, base.w};
+    for (int p2 = 0; p2 < part; ++p2) {
+      const float4 ps = *reinterpret_cast<const float4*>(part_sum + p2 * K2 + 4 * g);
+      run[0] += ps.x;
+      run[1] += ps.y;
+      run[2] += ps.z;
+      run[3] += ps.w;
+    }
+#pragma unroll
+    for (int i = 0; i < TPP; ++i) {
+      const int t = part * TPP + i;
+      float sn[4], cs[4];
+      {  // same products as in the partial sums above, so the running sum ends at the part total
+        const float d = dts[t];
+        const float2 t01 = unpack_bf16(thv[i].x), t23 = unpack_bf16(thv[i].y);
+        run[0] += d * t01.x;
+        run[1] += d * t01.y;
+        run[2] += d * t23.x;
+        run[3] += d * t23.y;
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) __sincosf(wrap_angle(run[k]), &sn[k], &cs[k]);
+      const bool export_row = last_chunk && (t0 + t == L - 1) && a.bprev_out != nullptr;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         const int row = t * R + r;
-        const uint32_t off = kb * kTile + swz(row, cidx) + within;
-        uint32_t* pb = reinterpret_cast<uint32_t*>(st + K::OFF_B + off);
-        uint32_t* pc = reinterpret_cast<uint32_t*>(st + K::OFF_C + off);
-        const float2 bv = unpack_bf16(*pb), cv = unpack_bf16(*pc);
-        const float b0 = cs * bv.x + sn * bv.y, b1 = -sn * bv.x + cs * bv.y;
-        *pb = pack_bf16(b0, b1);
-        *pc = pack_bf16(cs * cv.x + sn * cv.y, -sn * cv.x + cs * cv.y);
-        if (last_chunk && t0 + t == L - 1 && a.bprev_out) {
-          a.bprev_out[(unit * R + r) * N + 2 * pk] = b0;
-          a.bprev_out[(unit * R + r) * N + 2 * pk + 1] = b1;
+        const uint32_t off = kb * kTile + swz(row, c8);
+        uint4* pb = reinterpret_cast<uint4*>(st + K::OFF_B + off);
+        uint4* pc = reinterpret_cast<uint4*>(st + K::OFF_C + off);
+        const uint4 bq = *pb, cq = *pc;
+        const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w};
+        const uint32_t cw[4] = {cq.x, cq.y, cq.z, cq.w};
+        uint32_t bo[4], co[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 bv = unpack_bf16(bw[k]), cv = unpack_bf16(cw[k]);
+          const float b0 = cs[k] * bv.x + sn[k] * bv.y, b1 = cs[k] * bv.y - sn[k] * bv.x;
+          bo[k] = pack_bf16(b0, b1);
+          co[k] = pack_bf16(cs[k] * cv.x + sn[k] * cv.y, cs[k] * cv.y - sn[k] * cv.x);
+          if (export_row) {
+            a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k] = b0;
+            a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k + 1] = b1;
+          }
         }
+        *pb = make_uint4(bo[0], bo[1], bo[2], bo[3]);
+        *pc = make_uint4(co[0], co[1], co[2], co[3]);
       }
     }
     fence_proxy_async_smem();
-    mbar_arrive(&bars[bPrep1]);
-    if (part == 0) {
-      float tot = base;
-      for (int p2 = 0; p2 < K::NPART; ++p2) tot += part_sum[p2 * K2 + pk];
-      phi[pk] = wrap_angle(tot);
+    mbar_arrive(&bars[bPrep0 + s]);
+
+    if (part == 0) {  // carry the wrapped angle to the next chunk (every part has read phi)
+      float tot[4] = {base.x, base.y, base.z, base.w};
+      for (int p2 = 0; p2 < K::NPART; ++p2) {
+        const float4 ps = *reinterpret_cast<const float4*>(part_sum + p2 * K2 + 4 * g);
+        tot[0] += ps.x;
+        tot[1] += ps.y;
+        tot[2] += ps.z;
+        tot[3] += ps.w;
+      }
+      *reinterpret_cast<float4*>(phi + 4 * g) =
+          make_float4(wrap_angle(tot[0]), wrap_angle(tot[1]), wrap_angle(tot[2]), wrap_angle(tot[3]));
+      if (last_chunk && a.angle_out)
+        for (int k = 0; k < 4; ++k) a.angle_out[unit * K2 + 4 * g + k] = wrap_angle(tot[k]);
     }
     if (last_chunk && a.xprev_out && L > 0) {
       const __nv_bfloat16* xl = static_cast<const __nv_bfloat16*>(a.x) + tok_index(a, b, L - 1, hh) * R * kP;
-      for (int i = pt; i < R * kP; i += 128) a.xprev_out[unit * R * kP + i] = __bfloat162float(xl[i]);
+      for (int i = pt; i < R * kP; i += kNPrep) a.xprev_out[unit * R * kP + i] = __bfloat162float(xl[i]);
     }
-
-    // ---- B~ scaled in place by e^{cum_end - cum_t} w_t once S has read it ----
-    mbar_wait(&bars[bSFull], c & 1, abort_flag, status, kTagSFull);
-    if (prep_sync_any(*abort_flag != 0)) return;
-    {
-      const int row = pt;
-      const float f = wsc[row / R];
-#pragma unroll
-      for (int kb2 = 0; kb2 < K::NKB; ++kb2) {
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          uint4* p = reinterpret_cast<uint4*>(st + K::OFF_B + kb2 * kTile + swz(row, c8));
-          uint4 q = *p;
-          float2 f0 = unpack_bf16(q.x), f1 = unpack_bf16(q.y), f2 = unpack_bf16(q.z), f3 = unpack_bf16(q.w);
-          q.x = pack_bf16(f * f0.x, f * f0.y);
-          q.y = pack_bf16(f * f1.x, f * f1.y);
-          q.z = pack_bf16(f * f2.x, f * f2.y);
-          q.w = pack_bf16(f * f3.x, f * f3.y);
-          *p = q;
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(&bars[bPrep2]);
   }
-  if (pt < K2 && a.angle_out) a.angle_out[unit * K2 + pt] = phi[pt];
+}
+
+// bf16 copy of this thread's 32 state columns into the swizzled hbar tile
+__device__ __forceinline__ void store_hbar_bf16(const float (&hb)[32], uint8_t* Hs, int n, int ch) {
+  if (n < 0) return;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint4 q;
+    q.x = pack_bf16(hb[8 * q4 + 0], hb[8 * q4 + 1]);
+    q.y = pack_bf16(hb[8 * q4 + 2], hb[8 * q4 + 3]);
+    q.z = pack_bf16(hb[8 * q4 + 4], hb[8 * q4 + 5]);
+    q.w = pack_bf16(hb[8 * q4 + 6], hb[8 * q4 + 7]);
+    *reinterpret_cast<uint4*>(Hs + swz(n, 4 * ch + q4)) = q;
+  }
 }
 
 // ------------------------------------------------------------------ epilogue warps
-// One TMEM lane per thread: row m = 32 (warp % 4) + lane of S, Y, Yi; state
-// row n of Hacc / hbar (for N = 64 the M = 64 accumulator uses lanes 0..15 of
-// each 32-lane quadrant).
+// Two warps per TMEM lane quadrant: thread = (row m = 32 quad + lane, column
+// half ch).  Row m of S, P, Y, Yi; state row n of Hacc / hbar (for N = 64 the
+// M = 64 accumulator uses lanes 0..15 of each 32-lane quadrant).
 template <int N, int R>
-__device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh, float Ah,
+__device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh,
                                          uint64_t* bars, volatile int* abort_flag, DeviceStatus* status,
                                          uint32_t tmem) {
   using K = Cfg<N, R>;
   constexpr int Q = K::Q;
+  const int et = threadIdx.x - kEpi0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;
-  const int m = quad * 32 + lane;        // chunk row of S, Y, Yi, P
+  const int ch = et >> 7;                // column half
+  const int m = quad * 32 + lane;        // chunk row of S, P, Y, Yi
   const int tm = m / R, rm = m % R;      // token and rank of row m
   const int n = (N == 128) ? m : (lane < 16 ? quad * 16 + lane : -1);  // state row of hbar
   const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
   const int L = a.seqlen;
   const size_t unit = (size_t)b * a.nheads + hh;
   const float Dh = a.D ? a.D[hh] : 0.f;
-  uint8_t* Pt = smem + K::OFF_P;
+  const int tref = (32 * quad) / R;      // first token of this quadrant's rows
+  const int colf_off = quad == 1 ? 0 : (quad == 2 ? 32 : 96);
   uint8_t* Hs = smem + K::OFF_H;
 
-  // ---- initial carried state hbar_0 = h_0 + (1 - lam_1) dt_1 B~_0^T x_0 ----
-  float hb[kP];
+  // ---- initial carried state hbar_0 = h_0 + (1 - lam_1) dt_1 B~_0^T x_0 (columns of this half) ----
+  float hb[32];
 #pragma unroll
-  for (int p = 0; p < kP; ++p) hb[p] = 0.f;
-  if (n >= 0 && a.h0 != nullptr && L > 0) {
+  for (int p = 0; p < 32; ++p) hb[p] = 0.f;
+  if (n >= 0 && a.h0 != nullptr) {
     const size_t i0 = tok_index(a, b, 0, hh);
     const float mu1 = (1.f - __bfloat162float(static_cast<const __nv_bfloat16*>(a.lam)[i0])) *
                       __bfloat162float(static_cast<const __nv_bfloat16*>(a.dt)[i0]);
-    const float* h0 = a.h0 + (unit * N + n) * kP;
+    const float* h0 = a.h0 + (unit * N + n) * kP + 32 * ch;
 #pragma unroll
-    for (int p = 0; p < kP; ++p) hb[p] = h0[p];
+    for (int p = 0; p < 32; ++p) hb[p] = h0[p];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const float bp = mu1 * a.bprev0[(unit * R + r) * N + n];
-      const float* xp = a.xprev0 + (unit * R + r) * kP;
+      const float* xp = a.xprev0 + (unit * R + r) * kP + 32 * ch;
 #pragma unroll
-      for (int p = 0; p < kP; ++p) hb[p] += bp * xp[p];
+      for (int p = 0; p < 32; ++p) hb[p] += bp * xp[p];
     }
   }
-  auto store_hbar_bf16 = [&]() {
-    if (n >= 0) {
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        uint4 q;
-        q.x = pack_bf16(hb[8 * c8 + 0], hb[8 * c8 + 1]);
-        q.y = pack_bf16(hb[8 * c8 + 2], hb[8 * c8 + 3]);
-        q.z = pack_bf16(hb[8 * c8 + 4], hb[8 * c8 + 5]);
-        q.w = pack_bf16(hb[8 * c8 + 6], hb[8 * c8 + 7]);
-        *reinterpret_cast<uint4*>(Hs + swz(n, c8)) = q;
-      }
-    }
-  };
-  store_hbar_bf16();
+  store_hbar_bf16(hb, Hs, n, ch);
   fence_proxy_async_smem();
-  mbar_arrive(&bars[bHb]);
+  mbar_arrive(&bars[bEpiDone]);
 
   for (int c = 0; c < nchunks; ++c) {
-    const int s = c & 1;
+    const int s = c & 1, u = c >> 1;
     const int t0 = c * Q;
     const float* sc = reinterpret_cast<const float*>(smem + K::OFF_SC) + s * K::SC_PER_STAGE;
-    const float *c2 = sc, *wv = sc + Q, *gm = sc + 2 * Q;
+    const float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *colf = sc + 5 * Q + colf_off;
 
-    // ---- mask S into P ----
-    mbar_wait(&bars[bPrep1], c & 1, abort_flag, status, kTagPrep1);
+    // ---- S -> P (bf16, into TMEM) ----
+    mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1);
     mbar_wait(&bars[bSFull], c & 1, abort_flag, status, kTagSFull);
     if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
     tc_fence_after();
+    // every scalar this chunk needs is read now: prep may refill this stage's
+    // scalars once P has been consumed
     const float my_c2 = c2[tm];
     const float my_gam = gm[tm];
     const float my_e = ex2(my_c2);
     const float e_end = ex2(c2[Q - 1]);
+    const float rowf = ex2(my_c2 - c2[tref]);
+#pragma unroll 1
+    for (int k = 0; k < 4; ++k) {
+      const int cb = 2 * ch + (k >> 1);  // 32-column block of S
+      const int j0 = 32 * cb + 16 * (k & 1);  // first of this piece's 16 columns
+      uint32_t pk[8];
+      if (cb > quad) {  // warp-uniform: every column is a later token
 #pragma unroll
-    for (int blk = 0; blk < 4; ++blk) {
-      float sv[32];
-      if (blk <= quad) {  // warp-uniform: columns past the warp's last token are all zero
-        tmem_ld32(tmem + lane_base + kColS + 32 * blk, sv);
-        tmem_ld_wait();
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int tj = (32 * blk + jj) / R;
-          float kf;
-          if (tj < tm)
-            kf = ex2(my_c2 - c2[tj]) * wv[tj];
-          else if (tj == tm)
-            kf = my_gam;
-          else
-            kf = 0.f;
-          sv[jj] *= kf;
-        }
+        for (int i = 0; i < 8; ++i) pk[i] = 0u;
       } else {
+        float sv[16];
+        tmem_ld16(tmem + lane_base + kColS + j0, sv);
+        tmem_ld_wait();
+        if (cb < quad) {  // every column is an earlier token: rank-1 decay factors
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) sv[jj] = 0.f;
-      }
-      // columns 32*blk .. +31 live in k-block blk/2, 16-byte chunks 4*(blk&1) .. +3
+          for (int j4 = 0; j4 < 4; ++j4) {
+            const float4 cf = *reinterpret_cast<const float4*>(colf + j0 + 4 * j4);
+            sv[4 * j4 + 0] *= cf.x * rowf;
+            sv[4 * j4 + 1] *= cf.y * rowf;
+            sv[4 * j4 + 2] *= cf.z * rowf;
+            sv[4 * j4 + 3] *= cf.w * rowf;
+          }
+        } else {  // diagonal block: causal mask, trapezoid weights, D on the diagonal
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint4 q;
-        q.x = pack_bf16(sv[8 * q4 + 0], sv[8 * q4 + 1]);
-        q.y = pack_bf16(sv[8 * q4 + 2], sv[8 * q4 + 3]);
-        q.z = pack_bf16(sv[8 * q4 + 4], sv[8 * q4 + 5]);
-        q.w = pack_bf16(sv[8 * q4 + 6], sv[8 * q4 + 7]);
-        *reinterpret_cast<uint4*>(Pt + (blk >> 1) * kTile + swz(m, 4 * (blk & 1) + q4)) = q;
+          for (int jj = 0; jj < 16; ++jj) {
+            const int j = j0 + jj;
+            const int tj = j / R;
+            float kf = 0.f;
+            if (tj < tm) kf = ex2(my_c2 - c2[tj]) * wv[tj];
+            else if (tj == tm) kf = my_gam;
+            sv[jj] = sv[jj] * kf + (j == m ? Dh : 0.f);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(sv[2 * i], sv[2 * i + 1]);
       }
+      tmem_st8(tmem + lane_base + kColP + j0 / 2, pk);
     }
+    tmem_st_wait();
     tc_fence_before();
-    mbar_arrive(&bars[bSFree]);
-    fence_proxy_async_smem();
     mbar_arrive(&bars[bPReady]);
 
-    // ---- state update hbar = e^{cum_end} hbar + Hacc ----
+    // ---- state update hbar = e^{cum_end} hbar + Hacc (this half's 32 columns) ----
     mbar_wait(&bars[bAcc], c & 1, abort_flag, status, kTagAcc);
     if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
     tc_fence_after();
-    {
-      float acc[32];
-      const uint32_t cH = kColH + (c & 1) * 64;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tmem + lane_base + cH + 32 * half, acc);
-        tmem_ld_wait();
+    for (int half = 0; half < 2; ++half) {
+      float acc[16];
+      tmem_ld16(tmem + lane_base + kColH + 32 * ch + 16 * half, acc);
+      tmem_ld_wait();
 #pragma unroll
-        for (int p = 0; p < 32; ++p) hb[32 * half + p] = e_end * hb[32 * half + p] + acc[p];
-      }
+      for (int p = 0; p < 16; ++p) hb[16 * half + p] = e_end * hb[16 * half + p] + acc[p];
     }
-    store_hbar_bf16();
+    store_hbar_bf16(hb, Hs, n, ch);
     if (c == nchunks - 1 && a.h_out != nullptr && n >= 0) {
-      float* ho = a.h_out + (unit * N + n) * kP;
+      float* ho = a.h_out + (unit * N + n) * kP + 32 * ch;
 #pragma unroll
-      for (int p = 0; p < kP; p += 4) *reinterpret_cast<float4*>(ho + p) = make_float4(hb[p], hb[p + 1], hb[p + 2], hb[p + 3]);
+      for (int p = 0; p < 32; p += 4)
+        *reinterpret_cast<float4*>(ho + p) = make_float4(hb[p], hb[p + 1], hb[p + 2], hb[p + 3]);
     }
-    fence_proxy_async_smem();
-    mbar_arrive(&bars[bHb]);
 
-    // ---- y = Y + e^{cum_t} Yi + D x ----
+    // ---- y = Y + e^{cum_t} Yi ----
     mbar_wait(&bars[bYFull], c & 1, abort_flag, status, kTagY);
     if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
     tc_fence_after();
-    const int tg = t0 + tm;
-    const size_t row = tok_index(a, b, tg < L ? tg : 0, hh) * R + rm;
-    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.x) + row * kP);
-    uint4* yr = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) + row * kP);
-    const uint32_t cYi = kColYi + (c & 1) * 64;
+    {
+      const int tg = t0 + tm;
+      uint4* yr = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) +
+                                           (tok_index(a, b, tg < L ? tg : 0, hh) * R + rm) * kP + 32 * ch);
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        float yv[16], yi[16];
+        tmem_ld16(tmem + lane_base + kColY + 32 * ch + 16 * half, yv);
+        tmem_ld16(tmem + lane_base + kColYi + 32 * ch + 16 * half, yi);
+        tmem_ld_wait();
+        if (tg < L) {
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      float yv[32], yi[32];
-      tmem_ld32(tmem + lane_base + kColY + 32 * half, yv);
-      tmem_ld32(tmem + lane_base + cYi + 32 * half, yi);
-      tmem_ld_wait();
-      if (tg < L) {
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint4 xq = xr[4 * half + q4];
-          const float2 x0 = unpack_bf16(xq.x), x1 = unpack_bf16(xq.y), x2 = unpack_bf16(xq.z), x3 = unpack_bf16(xq.w);
-          const int o = 8 * q4;
-          uint4 q;
-          q.x = pack_bf16(yv[o + 0] + my_e * yi[o + 0] + Dh * x0.x, yv[o + 1] + my_e * yi[o + 1] + Dh * x0.y);
-          q.y = pack_bf16(yv[o + 2] + my_e * yi[o + 2] + Dh * x1.x, yv[o + 3] + my_e * yi[o + 3] + Dh * x1.y);
-          q.z = pack_bf16(yv[o + 4] + my_e * yi[o + 4] + Dh * x2.x, yv[o + 5] + my_e * yi[o + 5] + Dh * x2.y);
-          q.w = pack_bf16(yv[o + 6] + my_e * yi[o + 6] + Dh * x3.x, yv[o + 7] + my_e * yi[o + 7] + Dh * x3.y);
-          yr[4 * half + q4] = q;
+          for (int q2 = 0; q2 < 2; ++q2) {
+            const int o = 8 * q2;
+            uint4 q;
+            q.x = pack_bf16(yv[o + 0] + my_e * yi[o + 0], yv[o + 1] + my_e * yi[o + 1]);
+            q.y = pack_bf16(yv[o + 2] + my_e * yi[o + 2], yv[o + 3] + my_e * yi[o + 3]);
+            q.z = pack_bf16(yv[o + 4] + my_e * yi[o + 4], yv[o + 5] + my_e * yi[o + 5]);
+            q.w = pack_bf16(yv[o + 6] + my_e * yi[o + 6], yv[o + 7] + my_e * yi[o + 7]);
+            yr[2 * half + q2] = q;
+          }
         }
       }
     }
     tc_fence_before();
+    fence_proxy_async_smem();  // hbar (bf16) is read by the next chunk's MMA
+    mbar_arrive(&bars[bEpiDone]);
   }
 }
 
@@ -454,27 +502,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nchunks = prm.nchunks;
   const int unit = blockIdx.x;
   const int b = unit / a.nheads, hh = unit % a.nheads;
-  const int L = a.seqlen;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + K::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::OFF_MISC + 4);
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.workspace);
-  float* phi = reinterpret_cast<float*>(smem + K::OFF_PHI);
-  const float Ah = a.A[hh];
 
   if (tid == 0) {
     mbar_init(&bars[bFull0], 1);
     mbar_init(&bars[bFull1], 1);
     mbar_init(&bars[bEmpty0], 1);
     mbar_init(&bars[bEmpty1], 1);
-    mbar_init(&bars[bPrep1], 128);
-    mbar_init(&bars[bPrep2], 128);
+    mbar_init(&bars[bPrep0], kNPrep);
+    mbar_init(&bars[bPrep1], kNPrep);
     mbar_init(&bars[bSFull], 1);
-    mbar_init(&bars[bSFree], 128);
     mbar_init(&bars[bAcc], 1);
-    mbar_init(&bars[bHb], 128);
-    mbar_init(&bars[bPReady], 128);
+    mbar_init(&bars[bEpiDone], kNEpi);
+    mbar_init(&bars[bPReady], kNEpi);
     mbar_init(&bars[bYFull], 1);
     mbar_init(&bars[bDone], 1);
     *abort_flag = 0;
@@ -500,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = c & 1, u = c >> 1;
         if (!mbar_wait(&bars[bEmpty0 + s], (u & 1) ^ 1, abort_flag, status, kTagEmpty)) break;
         uint8_t* st = smem + s * K::STAGE_BYTES;
-        mbar_arrive_expect_tx(&bars[bFull0 + s], K::STAGE_BYTES);
+        mbar_arrive_expect_tx(&bars[bFull0 + s], K::TMA_BYTES);
         const int t0 = c * Q;
 #pragma unroll
         for (int kb = 0; kb < K::NKB; ++kb) {
@@ -517,17 +561,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t iS = idesc_bf16(kM, kM, 0, 0);     // S = C~ B~^T
-      const uint32_t iYi = idesc_bf16(kM, kP, 0, 1);    // Yi = C~ hbar
-      const uint32_t iH = idesc_bf16(N, kP, 1, 1);      // Hacc = B~s^T X
-      const uint32_t iY = idesc_bf16(kM, kP, 0, 1);     // Y = P X
+      const uint32_t iS = idesc_bf16(kM, kM, 0, 0);     // S = C~ B~^T        (both K-major)
+      const uint32_t iYi = idesc_bf16(kM, kP, 0, 1);    // Yi = C~ hbar       (B MN-major)
+      const uint32_t iH = idesc_bf16(N, kP, 1, 1);      // Hacc = B~^T X_w    (both MN-major)
+      const uint32_t iY = idesc_bf16(kM, kP, 0, 1);     // Y = P X            (A in TMEM)
       const uint32_t sbase = smem_u32(smem);
       for (int c = 0; c < nchunks; ++c) {
-        const int s = c & 1;
+        const int s = c & 1, u = c >> 1;
         const uint32_t st = sbase + s * K::STAGE_BYTES;
-        const uint32_t cB = st + K::OFF_B, cC = st + K::OFF_C, cX = st + K::OFF_X;
-        if (!mbar_wait(&bars[bPrep1], c & 1, abort_flag, status, kTagPrep1)) break;
-        if (c > 0 && !mbar_wait(&bars[bSFree], (c - 1) & 1, abort_flag, status, kTagSFree)) break;
+        const uint32_t cB = st + K::OFF_B, cC = st + K::OFF_C, cX = st + K::OFF_X, cXw = st + K::OFF_XW;
+        if (!mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < N / 16; ++kk) {
@@ -536,29 +579,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                       kk > 0);
         }
         mma_commit(&bars[bSFull]);
-        if (!mbar_wait(&bars[bPrep2], c & 1, abort_flag, status, kTagPrep2)) break;
-        if (!mbar_wait(&bars[bHb], c & 1, abort_flag, status, kTagHb)) break;
+        if (!mbar_wait(&bars[bEpiDone], c & 1, abort_flag, status, kTagEpiDone)) break;
         tc_fence_after();
-        const uint32_t cYi = kColYi + (c & 1) * 64, cH = kColH + (c & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < N / 16; ++kk) {
           const uint32_t offa = (kk >> 2) * kTile + (kk & 3) * 32;
-          mma_bf16_ss(tmem + cYi, smem_desc_sw128(cC + offa, 16, 1024),
+          mma_bf16_ss(tmem + kColYi, smem_desc_sw128(cC + offa, 16, 1024),
                       smem_desc_sw128(sbase + K::OFF_H + kk * 2048, N * 128, 1024), iYi, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < kM / 16; ++kk) {
-          mma_bf16_ss(tmem + cH, smem_desc_sw128(cB + kk * 2048, kTile, 1024),
-                      smem_desc_sw128(cX + kk * 2048, kTile, 1024), iH, kk > 0);
+          mma_bf16_ss(tmem + kColH, smem_desc_sw128(cB + kk * 2048, kTile, 1024),
+                      smem_desc_sw128(cXw + kk * 2048, kTile, 1024), iH, kk > 0);
         }
         mma_commit(&bars[bAcc]);
         if (!mbar_wait(&bars[bPReady], c & 1, abort_flag, status, kTagP)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kM / 16; ++kk) {
-          const uint32_t offa = (kk >> 2) * kTile + (kk & 3) * 32;
-          mma_bf16_ss(tmem + kColY, smem_desc_sw128(sbase + K::OFF_P + offa, 16, 1024),
-                      smem_desc_sw128(cX + kk * 2048, kTile, 1024), iY, kk > 0);
+          mma_bf16_ts(tmem + kColY, tmem + kColP + 8 * kk, smem_desc_sw128(cX + kk * 2048, kTile, 1024), iY,
+                      kk > 0);
         }
         mma_commit(&bars[bYFull]);
         mma_commit(&bars[bEmpty0 + s]);
@@ -568,9 +608,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bars[bDone], 0, abort_flag, status, kTagDrain, 400000000LL);
     }
   } else if (tid < kEpi0) {
-    prep_role<N, R>(smem, a, nchunks, b, hh, Ah, bars, abort_flag, status, phi);
+    prep_role<N, R>(smem, a, nchunks, b, hh, a.A[hh], bars, abort_flag, status);
   } else {
-    epi_role<N, R>(smem, a, nchunks, b, hh, Ah, bars, abort_flag, status, tmem);
+    epi_role<N, R>(smem, a, nchunks, b, hh, bars, abort_flag, status, tmem);
   }
 
   tc_fence_before();
