@@ -60,7 +60,7 @@ constexpr int kNEpi = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColP = 128, kColY = 192, kColYi = 256, kColH = 320;
 
-enum Tag { kTagEmpty = 1, kTagFull, kTagPrep1, kTagSFull, kTagAcc, kTagEpiDone, kTagP, kTagY, kTagDrain };
+enum Tag { kTagEmpty = 1, kTagFull, kTagPrep1, kTagSFull, kTagAcc, kTagEpiDone, kTagP, kTagY, kTagDrain, kTagTh };
 
 template <int N, int R>
 struct Cfg {
@@ -69,15 +69,19 @@ struct Cfg {
   static constexpr int K2 = N / 2;     // rotation pairs
   static constexpr int NG = K2 / 4;    // groups of 4 pairs (16 bytes of a row)
   static constexpr int NPART = kNPrep / NG;  // token parts of the angle scan
-  static constexpr int TPP = (Q + NPART - 1) / NPART;  // tokens per part (last part may be short)
-  static constexpr int STAGE_BYTES = (2 * NKB + 2) * kTile;  // B, C, X, X_w
-  static constexpr int TMA_BYTES = (2 * NKB + 1) * kTile;    // B, C, X
-  static constexpr int OFF_B = 0, OFF_C = NKB * kTile, OFF_X = 2 * NKB * kTile, OFF_XW = (2 * NKB + 1) * kTile;
-  static constexpr int OFF_H = kStages * STAGE_BYTES;  // hbar bf16, N rows x 128 bytes
+  static constexpr int TPP = Q / NPART;  // tokens per part
+  static constexpr int TB = (R == 1 && TPP % 2 == 0) ? 2 : 1;  // tokens per rotation batch
+  static constexpr int STAGE_BYTES = (2 * NKB + 1) * kTile;  // B, C, X
+  static constexpr int TMA_BYTES = STAGE_BYTES;
+  static constexpr int OFF_B = 0, OFF_C = NKB * kTile, OFF_X = 2 * NKB * kTile;
+  static constexpr int OFF_XW = kStages * STAGE_BYTES;   // X_w (single buffer)
+  static constexpr int OFF_TH = OFF_XW + kTile;          // theta tile [Q][N/2] bf16 (single buffer)
+  static constexpr int TH_BYTES = Q * K2 * 2;
+  static constexpr int OFF_H = OFF_TH + ((TH_BYTES + 1023) & ~1023);  // hbar bf16, N rows x 128 bytes
   static constexpr int OFF_SC = OFF_H + N * 128;       // scalars
   // per stage (floats): c2[Q] (log2 of the chunk-local decay), gam[Q], wv[Q],
-  // wsc[Q] (X_w row scale), dt[Q], colf[192] (rank-1 column factors of the mask)
-  static constexpr int SC_PER_STAGE = 5 * Q + 192;
+  // wsc[Q] (X_w row scale), colf[192] (rank-1 column factors of the mask)
+  static constexpr int SC_PER_STAGE = 4 * Q + 192;
   static constexpr int OFF_PART = OFF_SC + kStages * SC_PER_STAGE * 4;  // angle partials [NPART][K2]
   static constexpr int OFF_PHI = OFF_PART + NPART * K2 * 4;            // running base angle [K2]
   static constexpr int OFF_WARP = OFF_PHI + K2 * 4;                     // scan scratch [8]
@@ -86,12 +90,15 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
   static constexpr int SMEM = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;       // slack for 1024-byte alignment
-  static_assert(NG * NPART == kNPrep, "angle partition");
+  static_assert(NG * NPART == kNPrep && TPP * NPART == Q, "angle partition");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
 // barrier slots
-enum Bar { bFull0 = 0, bFull1, bEmpty0, bEmpty1, bPrep0, bPrep1, bSFull, bAcc, bEpiDone, bPReady, bYFull, bDone };
+enum Bar {
+  bFull0 = 0, bFull1, bEmpty0, bEmpty1, bPrep0, bPrep1, bSFull, bAcc, bEpiDone, bPReady, bYFull, bDone,
+  bThFull, bThFree
+};
 
 struct TcParams {
   ScanArgs a;
@@ -130,78 +137,163 @@ __device__ __forceinline__ bool prep_sync_any(bool v) {
 __device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // ------------------------------------------------------------------ prep warps
-// Thread pt in [0,256).  Per chunk: decay scalars (thread = token), the rank-1
-// column factors of the mask, X_w, the angle scan (thread = group of 4 pairs x
-// token part) and RoPE of B and C in place, 16 bytes per shared-memory access.
+// Thread pt in [0,256).  Per chunk: decay scalars (thread = token), accumulated
+// angles (thread = group g of 4 pairs x token part) and RoPE of B and C in
+// place (16 bytes per shared-memory access, 2 rows in flight), the rank-1
+// column factors of the mask and X_w.  dt and lam are prefetched one chunk
+// ahead into registers; theta arrives by TMA.
 template <int N, int R>
 __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh, float Ah,
                                           uint64_t* bars, volatile int* abort_flag, DeviceStatus* status) {
   using K = Cfg<N, R>;
-  constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, TPP = K::TPP;
+  constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, TPP = K::TPP, TB = K::TB, NPART = K::NPART;
   const int pt = threadIdx.x - kPrep0;
-  const int L = a.seqlen;
-  const __nv_bfloat16* DT = static_cast<const __nv_bfloat16*>(a.dt);
-  const __nv_bfloat16* LM = static_cast<const __nv_bfloat16*>(a.lam);
-  const __nv_bfloat16* TH = static_cast<const __nv_bfloat16*>(a.theta);
+  const int L = a.seqlen, H = a.nheads;
   float* part_sum = reinterpret_cast<float*>(smem + K::OFF_PART);
   float* phi = reinterpret_cast<float*>(smem + K::OFF_PHI);
   float* warp_tot = reinterpret_cast<float*>(smem + K::OFF_WARP);
-  const size_t unit = (size_t)b * a.nheads + hh;
+  const uint8_t* th_tile = smem + K::OFF_TH;
+  const size_t unit = (size_t)b * H + hh;
   const int g = pt % NG, part = pt / NG;  // 4-pair group (one 16-byte chunk of a row), token part
   const int kb = g / 8, c8 = g % 8;       // 64-element block and 16-byte chunk of the group
+  // dt, lam of this (batch, head): element t at [t * H]
+  const __nv_bfloat16* DTu = static_cast<const __nv_bfloat16*>(a.dt) + (size_t)b * L * H + hh;
+  const __nv_bfloat16* LMu = static_cast<const __nv_bfloat16*>(a.lam) + (size_t)b * L * H + hh;
 
   if (pt < K2) phi[pt] = a.angle0 ? a.angle0[unit * K2 + pt] : 0.f;
+
+  // prefetched per chunk: (scan threads) dt, lam of token pt and of the next
+  // token; (angle threads) dt of this part's tokens
+  float s_dt, s_lm, s_dtn, s_lmn, p_dt[TPP];
+  auto load_scalars = [&](int cc, float& o_dt, float& o_lm, float& o_dtn, float& o_lmn, float (&o_pdt)[TPP]) {
+    const int tc0 = cc * Q;
+    const int tg = tc0 + pt;
+    const bool ok = pt < Q && cc < nchunks;
+    o_dt = (ok && tg < L) ? __bfloat162float(DTu[(size_t)tg * H]) : 0.f;
+    o_lm = (ok && tg < L) ? __bfloat162float(LMu[(size_t)tg * H]) : 1.f;
+    o_dtn = (ok && tg + 1 < L) ? __bfloat162float(DTu[(size_t)(tg + 1) * H]) : 0.f;
+    o_lmn = (ok && tg + 1 < L) ? __bfloat162float(LMu[(size_t)(tg + 1) * H]) : 1.f;
+#pragma unroll
+    for (int i = 0; i < TPP; ++i) {
+      const int tp = tc0 + part * TPP + i;
+      o_pdt[i] = (cc < nchunks && tp < L) ? __bfloat162float(DTu[(size_t)tp * H]) : 0.f;
+    }
+  };
+  load_scalars(0, s_dt, s_lm, s_dtn, s_lmn, p_dt);
   prep_sync();
 
   for (int c = 0; c < nchunks; ++c) {
     const int s = c & 1, u = c >> 1;
     const int t0 = c * Q;
     float* sc = reinterpret_cast<float*>(smem + K::OFF_SC) + s * K::SC_PER_STAGE;
-    float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *wsc = sc + 3 * Q, *dts = sc + 4 * Q, *colf = sc + 5 * Q;
+    float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *wsc = sc + 3 * Q, *colf = sc + 4 * Q;
     uint8_t* st = smem + s * K::STAGE_BYTES;
     const bool last_chunk = (c == nchunks - 1);
 
-    // ---- global loads first: dt, lam of this token and the next; theta of this thread's part ----
-    float dt = 0.f, lm = 1.f, dtn = 0.f, lmn = 1.f;
-    if (pt < Q) {
-      const int tg = t0 + pt;
-      if (tg < L) {
-        const size_t i = tok_index(a, b, tg, hh);
-        dt = __bfloat162float(DT[i]);
-        lm = __bfloat162float(LM[i]);
-      }
-      if (tg + 1 < L) {
-        const size_t i = tok_index(a, b, tg + 1, hh);
-        dtn = __bfloat162float(DT[i]);
-        lmn = __bfloat162float(LM[i]);
-      }
-    }
-    uint2 thv[TPP];
-#pragma unroll
-    for (int i = 0; i < TPP; ++i) {
-      const int tg = t0 + part * TPP + i;
-      thv[i] = (tg < L) ? *reinterpret_cast<const uint2*>(TH + tok_index(a, b, tg, hh) * K2 + 4 * g)
-                        : make_uint2(0u, 0u);
-    }
-    // inclusive scan of dt*A*log2(e) over the chunk's tokens
-    float v = (pt < Q) ? dt * Ah * kLog2e : 0.f;
+    // ---- phase A (no shared state): in-warp scan of dt*A*log2(e); theta of this part ----
+    float v = (pt < Q) ? s_dt * Ah * kLog2e : 0.f;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const float n = __shfl_up_sync(0xffffffffu, v, o);
       if ((pt & 31) >= o) v += n;
     }
-    mbar_wait(&bars[bFull0 + s], u & 1, abort_flag, status, kTagFull);
     if ((pt & 31) == 31) warp_tot[pt >> 5] = v;
-    if (prep_sync_any(*abort_flag != 0)) return;  // one decision for all prep threads
+    mbar_wait(&bars[bThFull], c & 1, abort_flag, status, kTagTh);
+    uint2 thv[TPP];
+    float loc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < TPP; ++i) {
+      thv[i] = *reinterpret_cast<const uint2*>(th_tile + ((part * TPP + i) * K2 + 4 * g) * 2);
+      const float2 t01 = unpack_bf16(thv[i].x), t23 = unpack_bf16(thv[i].y);
+      loc[0] += p_dt[i] * t01.x;
+      loc[1] += p_dt[i] * t01.y;
+      loc[2] += p_dt[i] * t23.x;
+      loc[3] += p_dt[i] * t23.y;
+    }
+    mbar_arrive(&bars[bThFree]);  // the theta tile may be refilled
+    *reinterpret_cast<float4*>(part_sum + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
+    const float4 base = *reinterpret_cast<const float4*>(phi + 4 * g);
+    mbar_wait(&bars[bFull0 + s], u & 1, abort_flag, status, kTagFull);
+    if (prep_sync_any(*abort_flag != 0)) return;  // barrier 1: one decision for all prep threads
+
+    // ---- phase B: scalars, prefix of the angle, RoPE ----
     for (int w = 0; w < (pt >> 5); ++w) v += warp_tot[w];
     if (pt < Q) {
-      const float gam = lm * dt;
+      const float gam = s_lm * s_dt;
       c2[pt] = v;
       gm[pt] = gam;
-      wv[pt] = gam + (1.f - lmn) * dtn;
-      dts[pt] = dt;
+      wv[pt] = gam + (1.f - s_lmn) * s_dtn;
     }
-    prep_sync();
+    float run[4] = {base.x, base.y, base.z, base.w};
+#pragma unroll
+    for (int p2 = 0; p2 < NPART - 1; ++p2) {
+      if (p2 < part) {
+        const float4 ps = *reinterpret_cast<const float4*>(part_sum + p2 * K2 + 4 * g);
+        run[0] += ps.x;
+        run[1] += ps.y;
+        run[2] += ps.z;
+        run[3] += ps.w;
+      }
+    }
+    float pdt_cur[TPP];
+#pragma unroll
+    for (int i = 0; i < TPP; ++i) pdt_cur[i] = p_dt[i];
+    // next chunk's scalars, in flight during the rotation
+    load_scalars(c + 1, s_dt, s_lm, s_dtn, s_lmn, p_dt);
+#pragma unroll
+    for (int i0 = 0; i0 < TPP; i0 += TB) {
+      float sn[TB][4], cs[TB][4];
+#pragma unroll
+      for (int j = 0; j < TB; ++j) {
+        const float2 t01 = unpack_bf16(thv[i0 + j].x), t23 = unpack_bf16(thv[i0 + j].y);
+        const float d = pdt_cur[i0 + j];
+        run[0] += d * t01.x;
+        run[1] += d * t01.y;
+        run[2] += d * t23.x;
+        run[3] += d * t23.y;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) __sincosf(wrap_angle(run[k]), &sn[j][k], &cs[j][k]);
+      }
+      uint4 bq[TB * R], cq[TB * R];
+#pragma unroll
+      for (int j = 0; j < TB * R; ++j) {  // every load of the batch before any store
+        const uint32_t off = kb * kTile + swz((part * TPP + i0) * R + j, c8);
+        bq[j] = *reinterpret_cast<const uint4*>(st + K::OFF_B + off);
+        cq[j] = *reinterpret_cast<const uint4*>(st + K::OFF_C + off);
+      }
+#pragma unroll
+      for (int j = 0; j < TB * R; ++j) {
+        const int jt = j / R, r = j % R;
+        const int t = part * TPP + i0 + jt;
+        const bool export_row = last_chunk && (t0 + t == L - 1) && a.bprev_out != nullptr;
+        const uint32_t bw[4] = {bq[j].x, bq[j].y, bq[j].z, bq[j].w};
+        const uint32_t cw[4] = {cq[j].x, cq[j].y, cq[j].z, cq[j].w};
+        uint32_t bo[4], co[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 bv = unpack_bf16(bw[k]), cv = unpack_bf16(cw[k]);
+          const float b0 = cs[jt][k] * bv.x + sn[jt][k] * bv.y, b1 = cs[jt][k] * bv.y - sn[jt][k] * bv.x;
+          bo[k] = pack_bf16(b0, b1);
+          co[k] = pack_bf16(cs[jt][k] * cv.x + sn[jt][k] * cv.y, cs[jt][k] * cv.y - sn[jt][k] * cv.x);
+          if (export_row) {
+            a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k] = b0;
+            a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k + 1] = b1;
+          }
+        }
+        const uint32_t off = kb * kTile + swz(t * R + r, c8);
+        *reinterpret_cast<uint4*>(st + K::OFF_B + off) = make_uint4(bo[0], bo[1], bo[2], bo[3]);
+        *reinterpret_cast<uint4*>(st + K::OFF_C + off) = make_uint4(co[0], co[1], co[2], co[3]);
+      }
+    }
+    if (part == NPART - 1) {  // the last part's running angle is the chunk's end angle
+      *reinterpret_cast<float4*>(phi + 4 * g) =
+          make_float4(wrap_angle(run[0]), wrap_angle(run[1]), wrap_angle(run[2]), wrap_angle(run[3]));
+      if (last_chunk && a.angle_out)
+        for (int k = 0; k < 4; ++k) a.angle_out[unit * K2 + 4 * g + k] = wrap_angle(run[k]);
+    }
+    prep_sync();  // barrier 2: scalars complete, every part has read phi
+
+    // ---- phase C: mask factors, X_w (after the previous state MMA has read it) ----
     const float c2end = c2[Q - 1];
     if (pt < Q) wsc[pt] = wv[pt] * ex2(c2end - c2[pt]);
     if (pt < 192) {  // column factors e^{cum_ref - cum_tj} w_tj of the off-diagonal mask blocks
@@ -210,106 +302,36 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       const int tj = j / R, tref = (32 * qq) / R;
       colf[pt] = ex2(c2[tref] - c2[tj]) * wv[tj];
     }
-
-    // ---- angle increments of this thread's 4 pairs and tokens ----
-    float loc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (c > 0) mbar_wait(&bars[bAcc], (c - 1) & 1, abort_flag, status, kTagAcc);
+    if (prep_sync_any(*abort_flag != 0)) return;  // barrier 3: wsc visible, X_w free
+    {
+      uint4 xq[4];
 #pragma unroll
-    for (int i = 0; i < TPP; ++i) {
-      const float d = dts[part * TPP + i];
-      const float2 t01 = unpack_bf16(thv[i].x), t23 = unpack_bf16(thv[i].y);
-      loc[0] += d * t01.x;
-      loc[1] += d * t01.y;
-      loc[2] += d * t23.x;
-      loc[3] += d * t23.y;
-    }
-    *reinterpret_cast<float4*>(part_sum + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
-    const float4 base = *reinterpret_cast<const float4*>(phi + 4 * g);
-    prep_sync();
-
-    // ---- X_w = diag(e^{cum_end - cum_t} w_t) X (B operand of the state MMA) ----
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int idx = pt + kNPrep * i;
-      const int row = idx >> 3, cc = idx & 7;
-      const float f = wsc[row / R];
-      const uint4 q = *reinterpret_cast<const uint4*>(st + K::OFF_X + swz(row, cc));
-      const float2 f0 = unpack_bf16(q.x), f1 = unpack_bf16(q.y), f2 = unpack_bf16(q.z), f3 = unpack_bf16(q.w);
-      uint4 o;
-      o.x = pack_bf16(f * f0.x, f * f0.y);
-      o.y = pack_bf16(f * f1.x, f * f1.y);
-      o.z = pack_bf16(f * f2.x, f * f2.y);
-      o.w = pack_bf16(f * f3.x, f * f3.y);
-      *reinterpret_cast<uint4*>(st + K::OFF_XW + swz(row, cc)) = o;
-    }
-
-    // ---- accumulated angle at the start of this part, then RoPE of every row ----
-    float run[4] = {base.x, base.y, base.z, base.w};
-    for (int p2 = 0; p2 < part; ++p2) {
-      const float4 ps = *reinterpret_cast<const float4*>(part_sum + p2 * K2 + 4 * g);
-      run[0] += ps.x;
-      run[1] += ps.y;
-      run[2] += ps.z;
-      run[3] += ps.w;
-    }
-#pragma unroll
-    for (int i = 0; i < TPP; ++i) {
-      const int t = part * TPP + i;
-      float sn[4], cs[4];
-      {  // same products as in the partial sums above, so the running sum ends at the part total
-        const float d = dts[t];
-        const float2 t01 = unpack_bf16(thv[i].x), t23 = unpack_bf16(thv[i].y);
-        run[0] += d * t01.x;
-        run[1] += d * t01.y;
-        run[2] += d * t23.x;
-        run[3] += d * t23.y;
+      for (int i = 0; i < 4; ++i) {
+        const int idx = pt + kNPrep * i;
+        xq[i] = *reinterpret_cast<const uint4*>(st + K::OFF_X + swz(idx >> 3, idx & 7));
       }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) __sincosf(wrap_angle(run[k]), &sn[k], &cs[k]);
-      const bool export_row = last_chunk && (t0 + t == L - 1) && a.bprev_out != nullptr;
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int row = t * R + r;
-        const uint32_t off = kb * kTile + swz(row, c8);
-        uint4* pb = reinterpret_cast<uint4*>(st + K::OFF_B + off);
-        uint4* pc = reinterpret_cast<uint4*>(st + K::OFF_C + off);
-        const uint4 bq = *pb, cq = *pc;
-        const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w};
-        const uint32_t cw[4] = {cq.x, cq.y, cq.z, cq.w};
-        uint32_t bo[4], co[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 bv = unpack_bf16(bw[k]), cv = unpack_bf16(cw[k]);
-          const float b0 = cs[k] * bv.x + sn[k] * bv.y, b1 = cs[k] * bv.y - sn[k] * bv.x;
-          bo[k] = pack_bf16(b0, b1);
-          co[k] = pack_bf16(cs[k] * cv.x + sn[k] * cv.y, cs[k] * cv.y - sn[k] * cv.x);
-          if (export_row) {
-            a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k] = b0;
-            a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k + 1] = b1;
-          }
-        }
-        *pb = make_uint4(bo[0], bo[1], bo[2], bo[3]);
-        *pc = make_uint4(co[0], co[1], co[2], co[3]);
+      for (int i = 0; i < 4; ++i) {
+        const int idx = pt + kNPrep * i;
+        const int row = idx >> 3, cc = idx & 7;
+        const float f = wsc[row / R];
+        const float2 f0 = unpack_bf16(xq[i].x), f1 = unpack_bf16(xq[i].y), f2 = unpack_bf16(xq[i].z),
+                     f3 = unpack_bf16(xq[i].w);
+        uint4 o;
+        o.x = pack_bf16(f * f0.x, f * f0.y);
+        o.y = pack_bf16(f * f1.x, f * f1.y);
+        o.z = pack_bf16(f * f2.x, f * f2.y);
+        o.w = pack_bf16(f * f3.x, f * f3.y);
+        *reinterpret_cast<uint4*>(smem + K::OFF_XW + swz(row, cc)) = o;
       }
     }
     fence_proxy_async_smem();
     mbar_arrive(&bars[bPrep0 + s]);
 
-    if (part == 0) {  // carry the wrapped angle to the next chunk (every part has read phi)
-      float tot[4] = {base.x, base.y, base.z, base.w};
-      for (int p2 = 0; p2 < K::NPART; ++p2) {
-        const float4 ps = *reinterpret_cast<const float4*>(part_sum + p2 * K2 + 4 * g);
-        tot[0] += ps.x;
-        tot[1] += ps.y;
-        tot[2] += ps.z;
-        tot[3] += ps.w;
-      }
-      *reinterpret_cast<float4*>(phi + 4 * g) =
-          make_float4(wrap_angle(tot[0]), wrap_angle(tot[1]), wrap_angle(tot[2]), wrap_angle(tot[3]));
-      if (last_chunk && a.angle_out)
-        for (int k = 0; k < 4; ++k) a.angle_out[unit * K2 + 4 * g + k] = wrap_angle(tot[k]);
-    }
     if (last_chunk && a.xprev_out && L > 0) {
-      const __nv_bfloat16* xl = static_cast<const __nv_bfloat16*>(a.x) + tok_index(a, b, L - 1, hh) * R * kP;
+      const __nv_bfloat16* xl =
+          static_cast<const __nv_bfloat16*>(a.x) + tok_index(a, b, L - 1, hh) * R * kP;
       for (int i = pt; i < R * kP; i += kNPrep) a.xprev_out[unit * R * kP + i] = __bfloat162float(xl[i]);
     }
   }
@@ -381,7 +403,7 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     const int s = c & 1, u = c >> 1;
     const int t0 = c * Q;
     const float* sc = reinterpret_cast<const float*>(smem + K::OFF_SC) + s * K::SC_PER_STAGE;
-    const float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *colf = sc + 5 * Q + colf_off;
+    const float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *colf = sc + 4 * Q + colf_off;
 
     // ---- S -> P (bf16, into TMEM) ----
     mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1);
@@ -493,7 +515,8 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
 template <int N, int R>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
-                   const __grid_constant__ CUtensorMap tmX, const TcParams prm) {
+                   const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
+                   const TcParams prm) {
   using K = Cfg<N, R>;
   constexpr int Q = K::Q;
   extern __shared__ uint8_t smem_raw[];
@@ -521,11 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[bPReady], kNEpi);
     mbar_init(&bars[bYFull], 1);
     mbar_init(&bars[bDone], 1);
+    mbar_init(&bars[bThFull], 1);
+    mbar_init(&bars[bThFree], kNPrep);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmC);
     prefetch_tmap(&tmX);
+    prefetch_tmap(&tmT);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -539,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int issued = 0;
+      int issued = 0, th_issued = 0;
       for (int c = 0; c < nchunks; ++c) {
         const int s = c & 1, u = c >> 1;
         if (!mbar_wait(&bars[bEmpty0 + s], (u & 1) ^ 1, abort_flag, status, kTagEmpty)) break;
@@ -553,10 +579,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tma_load_5d(st + K::OFF_X, &tmX, &bars[bFull0 + s], 0, 0, hh, t0, b);
         issued = c + 1;
+        // theta of chunk c into the single theta tile once prep has read chunk c-1's
+        if (c > 0 && !mbar_wait(&bars[bThFree], (c - 1) & 1, abort_flag, status, kTagTh)) break;
+        mbar_arrive_expect_tx(&bars[bThFull], K::TH_BYTES);
+        tma_load_4d(smem + K::OFF_TH, &tmT, &bars[bThFull], 0, hh, t0, b);
+        th_issued = c + 1;
       }
       // drain: never leave this CTA with bulk copies still landing in its smem
       for (int c = issued - 2; c < issued; ++c)
         if (c >= 0) mbar_wait(&bars[bFull0 + (c & 1)], (c >> 1) & 1, abort_flag, status, kTagDrain, 400000000LL);
+      if (th_issued > 0) mbar_wait(&bars[bThFull], (th_issued - 1) & 1, abort_flag, status, kTagDrain, 400000000LL);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -569,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < nchunks; ++c) {
         const int s = c & 1, u = c >> 1;
         const uint32_t st = sbase + s * K::STAGE_BYTES;
-        const uint32_t cB = st + K::OFF_B, cC = st + K::OFF_C, cX = st + K::OFF_X, cXw = st + K::OFF_XW;
+        const uint32_t cB = st + K::OFF_B, cC = st + K::OFF_C, cX = st + K::OFF_X, cXw = sbase + K::OFF_XW;
         if (!mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1)) break;
         tc_fence_after();
 #pragma unroll
@@ -655,11 +687,26 @@ bool make_map(CUtensorMap* m, const void* base, int inner, const ScanArgs& a, in
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// theta [batch, L, H, N/2] bf16, box = {N/2, 1, Q, 1}, no swizzle, zero fill past the end.
+bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int K2 = a.N / 2;
+  const cuuint64_t dims[4] = {(cuuint64_t)K2, (cuuint64_t)a.nheads, (cuuint64_t)a.seqlen, (cuuint64_t)a.batch};
+  const cuuint64_t strides[3] = {2ull * K2, 2ull * K2 * a.nheads, 2ull * K2 * a.nheads * a.seqlen};
+  const cuuint32_t box[4] = {(cuuint32_t)K2, 1, (cuuint32_t)Q, 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(a.theta), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int N, int R>
 int launch_nr(const ScanArgs& a, cudaStream_t s) {
   using K = Cfg<N, R>;
-  CUtensorMap tmB, tmC, tmX;
-  if (!make_map(&tmB, a.B, N, a, K::Q) || !make_map(&tmC, a.C, N, a, K::Q) || !make_map(&tmX, a.x, kP, a, K::Q))
+  CUtensorMap tmB, tmC, tmX, tmT;
+  if (!make_map(&tmB, a.B, N, a, K::Q) || !make_map(&tmC, a.C, N, a, K::Q) || !make_map(&tmX, a.x, kP, a, K::Q) ||
+      !make_theta_map(&tmT, a, K::Q))
     return MAMBA3_ERR_CUDA;
   TcParams prm;
   prm.a = a;
@@ -667,7 +714,7 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
   auto kern = scan_tc_kernel<N, R>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
-  kern<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmC, tmX, prm);
+  kern<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmC, tmX, tmT, prm);
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 
