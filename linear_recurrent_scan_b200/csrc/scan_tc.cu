@@ -520,7 +520,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   using K = Cfg<N, R>;
   constexpr int Q = K::Q;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // align to 1024 bytes by offsetting the __shared__ pointer itself, so that the
+  // compiler keeps every access below in the shared state space
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const ScanArgs& a = prm.a;
   const int nchunks = prm.nchunks;
   const int unit = blockIdx.x;
