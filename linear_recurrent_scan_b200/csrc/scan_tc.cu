@@ -235,6 +235,10 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
         run[3] += ps.w;
       }
     }
+    // wrap once at the start of the part; inside the part the angle grows by
+    // TPP increments only, which __sincosf takes without a further wrap
+#pragma unroll
+    for (int k = 0; k < 4; ++k) run[k] = wrap_angle(run[k]);
     float pdt_cur[TPP];
 #pragma unroll
     for (int i = 0; i < TPP; ++i) pdt_cur[i] = p_dt[i];
@@ -252,7 +256,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
         run[2] += d * t23.x;
         run[3] += d * t23.y;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) __sincosf(wrap_angle(run[k]), &sn[j][k], &cs[j][k]);
+        for (int k = 0; k < 4; ++k) __sincosf(run[k], &sn[j][k], &cs[j][k]);
       }
       uint4 bq[TB * R], cq[TB * R];
 #pragma unroll
