@@ -19,6 +19,7 @@
 // reduced over the G row groups through shared memory.
 #include "common.cuh"
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace m3 {
 namespace {
@@ -175,6 +176,218 @@ int launch_r(const DecodeArgs& a, cudaStream_t s) {
   return MAMBA3_ERR_UNSUPPORTED;
 }
 
+
+// ------------------------------------------------------------------ streaming version
+// Persistent CTAs stream (batch, head) units: while unit i is computed in
+// shared memory, the TMA engine brings unit i+1 (its N x P state slab and the
+// small per-unit inputs) into the other stage of a 2-stage ring, and a bulk
+// store writes unit i-1's new state back.  HBM traffic therefore does not wait
+// on the SIMT work.  Used for P = 64, N in {64, 128}.
+constexpr int kSThreads = 256;
+constexpr int kSP = 64;
+
+template <typename T, int N, int R>
+struct DStage {  // byte offsets inside one stage; every region is a multiple of 16 bytes
+  static constexpr int H = 0;                                   // state      N x P f32
+  static constexpr int BP = H + N * kSP * 4;                    // b_prev     R x N f32
+  static constexpr int XP = BP + R * N * 4;                     // x_prev     R x P f32
+  static constexpr int ANG = XP + R * kSP * 4;                  // angle      N/2 f32
+  static constexpr int B = ANG + (N / 2) * 4;                   // B          R x N T
+  static constexpr int C = B + R * N * (int)sizeof(T);          // C          R x N T
+  static constexpr int X = C + R * N * (int)sizeof(T);          // x          R x P T
+  static constexpr int TH = X + R * kSP * (int)sizeof(T);       // theta      N/2 T
+  static constexpr int LOADED = TH + (N / 2) * (int)sizeof(T);  // bytes brought by the bulk loads
+  static constexpr int BYTES = (LOADED + 127) & ~127;
+  // shared by both stages: rotated B, C (f32), readout partial sums per warp
+  static constexpr int SB = 2 * BYTES;
+  static constexpr int SC = SB + R * N * 4;
+  static constexpr int RED = SC + R * N * 4;
+  static constexpr int BAR = RED + (kSThreads / 32) * R * kSP * 4;
+  static constexpr int TOTAL = BAR + 64;
+};
+
+template <typename T, int N, int R>
+__global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) {
+  using S = DStage<T, N, R>;
+  constexpr int K2 = N / 2, ROWS = N / 16;
+  extern __shared__ __align__(128) uint8_t dsm[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(dsm + S::BAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + S::BAR + 16);
+  float* sB = reinterpret_cast<float*>(dsm + S::SB);
+  float* sC = reinterpret_cast<float*>(dsm + S::SC);
+  float* red = reinterpret_cast<float*>(dsm + S::RED);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int p4 = tid & 15, ty = tid >> 4;
+  const int units = a.batch * a.nheads;
+
+  if (tid == 0) {
+    ptx::mbar_init(&bars[0], 1);
+    ptx::mbar_init(&bars[1], 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  auto issue_loads = [&](int u, int stage) {
+    uint8_t* st = dsm + stage * S::BYTES;
+    uint64_t* bar = &bars[stage];
+    ptx::mbar_arrive_expect_tx(bar, S::LOADED);
+    ptx::bulk_load(st + S::H, a.h + (size_t)u * N * kSP, N * kSP * 4, bar);
+    ptx::bulk_load(st + S::BP, a.bprev + (size_t)u * R * N, R * N * 4, bar);
+    ptx::bulk_load(st + S::XP, a.xprev + (size_t)u * R * kSP, R * kSP * 4, bar);
+    ptx::bulk_load(st + S::ANG, a.angle + (size_t)u * K2, K2 * 4, bar);
+    ptx::bulk_load(st + S::B, static_cast<const T*>(a.B) + (size_t)u * R * N, R * N * sizeof(T), bar);
+    ptx::bulk_load(st + S::C, static_cast<const T*>(a.C) + (size_t)u * R * N, R * N * sizeof(T), bar);
+    ptx::bulk_load(st + S::X, static_cast<const T*>(a.x) + (size_t)u * R * kSP, R * kSP * sizeof(T), bar);
+    ptx::bulk_load(st + S::TH, static_cast<const T*>(a.theta) + (size_t)u * K2, K2 * sizeof(T), bar);
+  };
+
+  int it = 0;
+  int u = blockIdx.x;
+  if (tid == 0 && u < units) issue_loads(u, 0);
+  for (; u < units; u += gridDim.x, ++it) {
+    const int s = it & 1;
+    uint8_t* st = dsm + s * S::BYTES;
+    const int un = u + gridDim.x;
+    if (tid == 0 && un < units) {
+      ptx::bulk_wait_read<0>();  // the other stage's previous state store has read its source
+      issue_loads(un, s ^ 1);
+    }
+    const int hh = u % a.nheads;
+    const float dt = ld1(static_cast<const T*>(a.dt) + u);
+    const float lam = ld1(static_cast<const T*>(a.lam) + u);
+    const float alpha = expf(dt * a.A[hh]);
+    const float beta = (1.f - lam) * dt * alpha, gamma = lam * dt;
+    const float Dh = a.D ? a.D[hh] : 0.f;
+    ptx::mbar_wait(&bars[s], (it >> 1) & 1, abort_flag, nullptr, 0);
+    if (__syncthreads_or(*abort_flag != 0)) break;
+
+    // ---- rotation of B and C by the updated angle; the carry for the next step ----
+    const float* ang = reinterpret_cast<const float*>(st + S::ANG);
+    const T* Bs = reinterpret_cast<const T*>(st + S::B);
+    const T* Cs = reinterpret_cast<const T*>(st + S::C);
+    const T* Xs = reinterpret_cast<const T*>(st + S::X);
+    const T* THs = reinterpret_cast<const T*>(st + S::TH);
+    for (int i = tid; i < R * K2; i += kSThreads) {
+      const int r = i / K2, k = i % K2;
+      const float phi = wrap_angle(ang[k] + dt * ld1(THs + k));
+      float sn, cs;
+      sincosf(phi, &sn, &cs);
+      const float b0 = ld1(Bs + r * N + 2 * k), b1 = ld1(Bs + r * N + 2 * k + 1);
+      const float c0 = ld1(Cs + r * N + 2 * k), c1 = ld1(Cs + r * N + 2 * k + 1);
+      const float rb0 = cs * b0 + sn * b1, rb1 = -sn * b0 + cs * b1;
+      sB[r * N + 2 * k] = rb0;
+      sB[r * N + 2 * k + 1] = rb1;
+      sC[r * N + 2 * k] = cs * c0 + sn * c1;
+      sC[r * N + 2 * k + 1] = -sn * c0 + cs * c1;
+      *reinterpret_cast<float2*>(a.bprev + ((size_t)u * R + r) * N + 2 * k) = make_float2(rb0, rb1);
+      if (r == 0) a.angle[(size_t)u * K2 + k] = phi;
+    }
+    for (int i = tid; i < R * kSP; i += kSThreads) a.xprev[(size_t)u * R * kSP + i] = ld1(Xs + i);
+    __syncthreads();
+
+    // ---- state update in shared memory and readout partial sums ----
+    const float* bp = reinterpret_cast<const float*>(st + S::BP);
+    const float* xp = reinterpret_cast<const float*>(st + S::XP);
+    float* hs = reinterpret_cast<float*>(st + S::H);
+    float4 xr[R], xpr[R], yacc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      xr[r] = ld4(Xs + r * kSP + 4 * p4);
+      xpr[r] = *reinterpret_cast<const float4*>(xp + r * kSP + 4 * p4);
+      yacc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < ROWS; ++j) {
+      const int n = ty + 16 * j;
+      float4* hp = reinterpret_cast<float4*>(hs + n * kSP + 4 * p4);
+      const float4 hv = *hp;
+      float4 hn = make_float4(alpha * hv.x, alpha * hv.y, alpha * hv.z, alpha * hv.w);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float cb = beta * bp[r * N + n], cc = gamma * sB[r * N + n];
+        hn.x += cb * xpr[r].x + cc * xr[r].x;
+        hn.y += cb * xpr[r].y + cc * xr[r].y;
+        hn.z += cb * xpr[r].z + cc * xr[r].z;
+        hn.w += cb * xpr[r].w + cc * xr[r].w;
+      }
+      *hp = hn;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float cr = sC[r * N + n];
+        yacc[r].x += cr * hn.x;
+        yacc[r].y += cr * hn.y;
+        yacc[r].z += cr * hn.z;
+        yacc[r].w += cr * hn.w;
+      }
+    }
+    ptx::fence_proxy_async_smem();  // the new state is read by the bulk store
+#pragma unroll
+    for (int r = 0; r < R; ++r) {  // the two row groups of this warp
+      yacc[r].x += __shfl_xor_sync(0xffffffffu, yacc[r].x, 16);
+      yacc[r].y += __shfl_xor_sync(0xffffffffu, yacc[r].y, 16);
+      yacc[r].z += __shfl_xor_sync(0xffffffffu, yacc[r].z, 16);
+      yacc[r].w += __shfl_xor_sync(0xffffffffu, yacc[r].w, 16);
+      if (lane < 16) *reinterpret_cast<float4*>(red + (warp * R + r) * kSP + 4 * p4) = yacc[r];
+    }
+    __syncthreads();
+    if (tid == 0) {
+      ptx::bulk_store(a.h + (size_t)u * N * kSP, hs, N * kSP * 4);
+      ptx::bulk_commit();
+    }
+    T* yu = static_cast<T*>(a.y) + (size_t)u * R * kSP;
+    for (int i = tid; i < R * kSP; i += kSThreads) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kSThreads / 32; ++w) acc += red[w * R * kSP + i];
+      st1(yu + i, acc + Dh * ld1(Xs + i));
+    }
+    __syncthreads();  // stage s and the partial sums may be reused
+  }
+  if (tid == 0) ptx::bulk_wait_all();
+}
+
+template <typename T, int N, int R>
+int launch_stream_t(const DecodeArgs& a, cudaStream_t s) {
+  using S = DStage<T, N, R>;
+  auto k = decode_stream_kernel<T, N, R>;
+  static int blocks_per_sm = 0, sms = 0;
+  if (blocks_per_sm == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, k, kSThreads, S::TOTAL) != cudaSuccess ||
+        blocks_per_sm < 1)
+      return MAMBA3_ERR_CUDA;
+  }
+  const int units = a.batch * a.nheads;
+  const int grid = units < blocks_per_sm * sms ? units : blocks_per_sm * sms;
+  k<<<grid, kSThreads, S::TOTAL, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
+}
+
+bool stream_ok(const DecodeArgs& a) {
+  if (a.P != kSP || (a.N != 64 && a.N != 128) || !(a.R == 1 || a.R == 2 || a.R == 4)) return false;
+  const uintptr_t all = reinterpret_cast<uintptr_t>(a.h) | reinterpret_cast<uintptr_t>(a.bprev) |
+                        reinterpret_cast<uintptr_t>(a.xprev) | reinterpret_cast<uintptr_t>(a.angle) |
+                        reinterpret_cast<uintptr_t>(a.B) | reinterpret_cast<uintptr_t>(a.C) |
+                        reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.theta);
+  return (all & 15u) == 0;
+}
+
+template <typename T>
+int launch_stream(const DecodeArgs& a, cudaStream_t s) {
+  if (a.N == 128) {
+    if (a.R == 1) return launch_stream_t<T, 128, 1>(a, s);
+    if (a.R == 2) return launch_stream_t<T, 128, 2>(a, s);
+    return launch_stream_t<T, 128, 4>(a, s);
+  }
+  if (a.R == 1) return launch_stream_t<T, 64, 1>(a, s);
+  if (a.R == 2) return launch_stream_t<T, 64, 2>(a, s);
+  return launch_stream_t<T, 64, 4>(a, s);
+}
+
 }  // namespace
 
 int decode_supported(const DecodeArgs& a) {
@@ -188,6 +401,7 @@ int decode_supported(const DecodeArgs& a) {
 
 int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   if (a.batch * a.nheads == 0) return MAMBA3_OK;
+  if (stream_ok(a)) return a.dtype == MAMBA3_F32 ? launch_stream<float>(a, s) : launch_stream<__nv_bfloat16>(a, s);
   return a.dtype == MAMBA3_F32 ? launch_r<float>(a, s) : launch_r<__nv_bfloat16>(a, s);
 }
 
