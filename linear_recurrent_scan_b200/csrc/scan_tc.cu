@@ -210,8 +210,13 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       loc[2] += p_dt[i] * t23.x;
       loc[3] += p_dt[i] * t23.y;
     }
-    mbar_arrive(&bars[bThFree]);  // the theta tile may be refilled
     *reinterpret_cast<float4*>(part_sum + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
+    // Release the theta tile only after a store that consumes every loaded
+    // theta value: the arrive does not wait for shared-memory loads still in
+    // flight, and the refill is an async-proxy write that is not ordered
+    // after them, so arriving straight after the loads lets a slow part read
+    // the next chunk's theta.
+    mbar_arrive(&bars[bThFree]);
     const float4 base = *reinterpret_cast<const float4*>(phi + 4 * g);
     mbar_wait(&bars[bFull0 + s], u & 1, abort_flag, status, kTagFull);
     if (prep_sync_any(*abort_flag != 0)) return;  // barrier 1: one decision for all prep threads

@@ -60,6 +60,28 @@ def test_bf16_shapes(shape):
     check_state(fin, fr, TOL[torch.bfloat16])
 
 
+@pytest.mark.parametrize("shape", [(2, 200, 148, 64, 128, 2), (5, 200, 40, 64, 128, 2), (2, 300, 100, 64, 128, 1)])
+def test_repeated_launches_are_identical_and_match(shape):
+    """Many units in flight, launched repeatedly: every launch must match the
+    oracle and reproduce the first launch bit for bit (a race between a shared
+    tile's refill and its last readers shows up as a rare per-launch error)."""
+    b, L, H, P, N, R = shape
+    inp = small_inputs(b, L, H, P, N, R, torch.bfloat16, seed=1000 + L)
+    yr, fr = oracle_scan(inp)
+    first = None
+    for rep in range(8):
+        y, fin = gpu_scan(inp)
+        if first is None:
+            e = rel_err(y.float().cpu().double().numpy(), yr)
+            assert e < TOL[torch.bfloat16], e
+            check_state(fin, fr, TOL[torch.bfloat16])
+            first = (y.clone(), fin.h.clone(), fin.angle.clone())
+        else:
+            assert torch.equal(y, first[0]), f"launch {rep}: y differs from the first launch"
+            assert torch.equal(fin.h, first[1]), f"launch {rep}: h differs from the first launch"
+            assert torch.equal(fin.angle, first[2]), f"launch {rep}: angle differs from the first launch"
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_init_state_and_in_place_continuation(dtype):
     """Split prefill with the exported state == one prefill; final_state may alias init."""
