@@ -227,6 +227,13 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
     ptx::fence_mbar_init();
   }
   __syncthreads();
+  // Launched with programmatic stream serialization: let the next step's grid
+  // be scheduled now (its CTAs take SM slots as ours exit and run their
+  // prologue), then wait until the previous grid in the stream has completed
+  // and its writes are visible.  Every global access below follows the wait,
+  // so the ordering is that of a plain stream launch.
+  ptx::grid_launch_dependents();
+  ptx::grid_dependency_wait();
 
   auto issue_loads = [&](int u, int stage) {
     uint8_t* st = dsm + stage * S::BYTES;
@@ -363,7 +370,17 @@ int launch_stream_t(const DecodeArgs& a, cudaStream_t s) {
   }
   const int units = a.batch * a.nheads;
   const int grid = units < blocks_per_sm * sms ? units : blocks_per_sm * sms;
-  k<<<grid, kSThreads, S::TOTAL, s>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kSThreads);
+  cfg.dynamicSmemBytes = S::TOTAL;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k, a) != cudaSuccess) return MAMBA3_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 

@@ -38,6 +38,7 @@
 // Every wait is bounded: on expiry the CTA raises an abort flag, reports
 // MAMBA3_ERR_TIMEOUT in the device status word, drains and returns.
 #include <cuda.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -88,7 +89,13 @@ struct Cfg {
   static constexpr int OFF_BAR = (OFF_WARP + 32 + 7) & ~7;
   static constexpr int NBAR = 16;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
-  static constexpr int SMEM = OFF_MISC + 16;
+  // dt and lam of tokens [t0, t0 + Q] for the 8 heads of this head's 16-byte
+  // group (TMA tiles [Q + 1][8] bf16, single buffer, refilled with theta)
+  static constexpr int DL_BYTES = (Q + 1) * 16;
+  static constexpr int DL_PAD = (DL_BYTES + 127) & ~127;
+  static constexpr int OFF_DL = (OFF_MISC + 16 + 127) & ~127;
+  static constexpr int OFF_SINK = OFF_DL + 2 * DL_PAD;  // [Q] floats: consumes the tile reads
+  static constexpr int SMEM = OFF_SINK + Q * 4;
   static constexpr int SMEM_ALLOC = SMEM + 1024;       // slack for 1024-byte alignment
   static_assert(NG * NPART == kNPrep && TPP * NPART == Q, "angle partition");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -103,6 +110,7 @@ enum Bar {
 struct TcParams {
   ScanArgs a;
   int nchunks;
+  int dl_tma;  // dt and lam arrive by TMA with theta (else: global loads one chunk ahead)
 };
 
 __device__ __forceinline__ size_t tok_index(const ScanArgs& a, int b, int t, int h) {
@@ -143,8 +151,8 @@ __device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 256;" ::
 // column factors of the mask and X_w.  dt and lam are prefetched one chunk
 // ahead into registers; theta arrives by TMA.
 template <int N, int R>
-__device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh, float Ah,
-                                          uint64_t* bars, volatile int* abort_flag, DeviceStatus* status) {
+__device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int dl_tma, int b, int hh,
+                                          float Ah, uint64_t* bars, volatile int* abort_flag, DeviceStatus* status) {
   using K = Cfg<N, R>;
   constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, TPP = K::TPP, TB = K::TB, NPART = K::NPART;
   const int pt = threadIdx.x - kPrep0;
@@ -179,7 +187,17 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       o_pdt[i] = (cc < nchunks && tp < L) ? __bfloat162float(DTu[(size_t)tp * H]) : 0.f;
     }
   };
-  load_scalars(0, s_dt, s_lm, s_dtn, s_lmn, p_dt);
+  if (dl_tma) {
+    s_dt = s_dtn = 0.f;
+    s_lm = s_lmn = 1.f;
+#pragma unroll
+    for (int i = 0; i < TPP; ++i) p_dt[i] = 0.f;
+  } else {
+    load_scalars(0, s_dt, s_lm, s_dtn, s_lmn, p_dt);
+  }
+  const __nv_bfloat16* dts = reinterpret_cast<const __nv_bfloat16*>(smem + K::OFF_DL) + (hh & 7);
+  const __nv_bfloat16* lms = reinterpret_cast<const __nv_bfloat16*>(smem + K::OFF_DL + K::DL_PAD) + (hh & 7);
+  float* sink = reinterpret_cast<float*>(smem + K::OFF_SINK);
   prep_sync();
 
   for (int c = 0; c < nchunks; ++c) {
@@ -191,6 +209,17 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
     const bool last_chunk = (c == nchunks - 1);
 
     // ---- phase A (no shared state): in-warp scan of dt*A*log2(e); theta of this part ----
+    mbar_wait(&bars[bThFull], c & 1, abort_flag, status, kTagTh);
+    if (dl_tma) {  // this chunk's dt and lam from the tile (rows past the sequence read 0)
+      if (pt < Q) {
+        s_dt = __bfloat162float(dts[pt * 8]);
+        s_lm = __bfloat162float(lms[pt * 8]);
+        s_dtn = __bfloat162float(dts[(pt + 1) * 8]);
+        s_lmn = __bfloat162float(lms[(pt + 1) * 8]);
+      }
+#pragma unroll
+      for (int i = 0; i < TPP; ++i) p_dt[i] = __bfloat162float(dts[(part * TPP + i) * 8]);
+    }
     float v = (pt < Q) ? s_dt * Ah * kLog2e : 0.f;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -198,7 +227,6 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       if ((pt & 31) >= o) v += n;
     }
     if ((pt & 31) == 31) warp_tot[pt >> 5] = v;
-    mbar_wait(&bars[bThFull], c & 1, abort_flag, status, kTagTh);
     uint2 thv[TPP];
     float loc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -211,11 +239,12 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       loc[3] += p_dt[i] * t23.y;
     }
     *reinterpret_cast<float4*>(part_sum + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
-    // Release the theta tile only after a store that consumes every loaded
-    // theta value: the arrive does not wait for shared-memory loads still in
-    // flight, and the refill is an async-proxy write that is not ordered
-    // after them, so arriving straight after the loads lets a slow part read
-    // the next chunk's theta.
+    if (dl_tma && pt < Q) sink[pt] = (s_dt + s_lm) + (s_dtn + s_lmn);
+    // Release the theta (and dt, lam) tiles only after stores that consume
+    // every value loaded from them: the arrive does not wait for shared-memory
+    // loads still in flight, and the refill is an async-proxy write that is not
+    // ordered after them, so arriving straight after the loads lets a slow
+    // thread read the next chunk's values.
     mbar_arrive(&bars[bThFree]);
     const float4 base = *reinterpret_cast<const float4*>(phi + 4 * g);
     mbar_wait(&bars[bFull0 + s], u & 1, abort_flag, status, kTagFull);
@@ -247,8 +276,8 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
     float pdt_cur[TPP];
 #pragma unroll
     for (int i = 0; i < TPP; ++i) pdt_cur[i] = p_dt[i];
-    // next chunk's scalars, in flight during the rotation
-    load_scalars(c + 1, s_dt, s_lm, s_dtn, s_lmn, p_dt);
+    // next chunk's scalars, in flight during the rotation (unless they come by TMA)
+    if (!dl_tma) load_scalars(c + 1, s_dt, s_lm, s_dtn, s_lmn, p_dt);
 #pragma unroll
     for (int i0 = 0; i0 < TPP; i0 += TB) {
       float sn[TB][4], cs[TB][4];
@@ -525,6 +554,7 @@ template <int N, int R>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
+                   const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmL,
                    const TcParams prm) {
   using K = Cfg<N, R>;
   constexpr int Q = K::Q;
@@ -564,6 +594,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmC);
     prefetch_tmap(&tmX);
     prefetch_tmap(&tmT);
+    if (prm.dl_tma) {
+      prefetch_tmap(&tmD);
+      prefetch_tmap(&tmL);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -593,8 +627,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = c + 1;
         // theta of chunk c into the single theta tile once prep has read chunk c-1's
         if (c > 0 && !mbar_wait(&bars[bThFree], (c - 1) & 1, abort_flag, status, kTagTh)) break;
-        mbar_arrive_expect_tx(&bars[bThFull], K::TH_BYTES);
+        mbar_arrive_expect_tx(&bars[bThFull], K::TH_BYTES + (prm.dl_tma ? 2u * K::DL_BYTES : 0u));
         tma_load_4d(smem + K::OFF_TH, &tmT, &bars[bThFull], 0, hh, t0, b);
+        if (prm.dl_tma) {
+          tma_load_3d(smem + K::OFF_DL, &tmD, &bars[bThFull], hh & ~7, t0, b);
+          tma_load_3d(smem + K::OFF_DL + K::DL_PAD, &tmL, &bars[bThFull], hh & ~7, t0, b);
+        }
         th_issued = c + 1;
       }
       // drain: never leave this CTA with bulk copies still landing in its smem
@@ -652,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bars[bDone], 0, abort_flag, status, kTagDrain, 400000000LL);
     }
   } else if (tid < kEpi0) {
-    prep_role<N, R>(smem, a, nchunks, b, hh, a.A[hh], bars, abort_flag, status);
+    prep_role<N, R>(smem, a, nchunks, prm.dl_tma, b, hh, a.A[hh], bars, abort_flag, status);
   } else {
     epi_role<N, R>(smem, a, nchunks, b, hh, bars, abort_flag, status, tmem);
   }
@@ -699,6 +737,21 @@ bool make_map(CUtensorMap* m, const void* base, int inner, const ScanArgs& a, in
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// dt or lam [batch, L, H] bf16, box = {8, Q + 1, 1}: the 8 heads of a 16-byte
+// group over the chunk's tokens and the next one, zero fill past the end.
+// Needs H a multiple of 8 (16-byte row stride) and a 16-byte aligned base.
+bool make_dl_map(CUtensorMap* m, const void* base, const ScanArgs& a, int Q) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || a.nheads % 8 != 0 || (reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)a.nheads, (cuuint64_t)a.seqlen, (cuuint64_t)a.batch};
+  const cuuint64_t strides[2] = {2ull * a.nheads, 2ull * a.nheads * a.seqlen};
+  const cuuint32_t box[3] = {8, (cuuint32_t)(Q + 1), 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // theta [batch, L, H, N/2] bf16, box = {N/2, 1, Q, 1}, no swizzle, zero fill past the end.
 bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q) {
   EncodeTiledFn enc = encode_fn();
@@ -723,10 +776,14 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
   TcParams prm;
   prm.a = a;
   prm.nchunks = (a.seqlen + K::Q - 1) / K::Q;
+  CUtensorMap tmD, tmL;
+  memset(&tmD, 0, sizeof(tmD));
+  memset(&tmL, 0, sizeof(tmL));
+  prm.dl_tma = make_dl_map(&tmD, a.dt, a, K::Q) && make_dl_map(&tmL, a.lam, a, K::Q);
   auto kern = scan_tc_kernel<N, R>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
-  kern<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmC, tmX, tmT, prm);
+  kern<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmC, tmX, tmT, tmD, tmL, prm);
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 

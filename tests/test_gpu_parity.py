@@ -49,6 +49,8 @@ def test_ragged_lengths_fp32(L, R):
 @pytest.mark.parametrize("shape", [
     (2, 200, 3, 64, 128, 1), (1, 300, 2, 64, 128, 4), (2, 150, 2, 64, 64, 4), (1, 97, 2, 64, 128, 2),
     (1, 130, 2, 32, 64, 1), (1, 70, 3, 16, 32, 8),
+    # heads a multiple of 8: dt and lam are staged by TMA (ragged tails included)
+    (2, 333, 8, 64, 128, 2), (1, 200, 16, 64, 64, 4), (1, 129, 8, 64, 128, 1), (1, 31, 8, 64, 128, 4),
 ])
 def test_bf16_shapes(shape):
     b, L, H, P, N, R = shape
