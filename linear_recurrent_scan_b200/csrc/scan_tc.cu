@@ -23,7 +23,9 @@
 // Design: one CTA per (batch, head) marches over its chunks; the state stays on
 // chip, in fp32 registers of the epilogue warps.  18 warps:
 //   warp 0       TMA producer: B, C, X tiles of chunk c into a 2-stage ring
-//                (128-byte swizzle, the layout the MMA descriptors read).
+//                (128-byte swizzle, the layout the MMA descriptors read); B and C
+//                of a stage are refilled once the state MMAs have read them, X
+//                once the Y MMA has; theta (+ dt, lam) into single tiles.
 //   warp 1       TMEM allocator and single-thread MMA issuer.
 //   warps 2..9   prep: decay scalars and the rank-1 decay factors of the mask,
 //                X_w = diag(e^{cum_end - cum_t} w_t) X, accumulated angles
@@ -103,8 +105,8 @@ struct Cfg {
 
 // barrier slots
 enum Bar {
-  bFull0 = 0, bFull1, bEmpty0, bEmpty1, bPrep0, bPrep1, bSFull, bAcc, bEpiDone, bPReady, bYFull, bDone,
-  bThFull, bThFree
+  bFull0 = 0, bFull1, bEmptyBC0, bEmptyBC1, bPrep0, bPrep1, bSFull, bAcc, bEpiDone, bPReady, bYFull, bDone,
+  bThFull, bThFree, bEmptyX0, bEmptyX1
 };
 
 struct TcParams {
@@ -576,8 +578,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(&bars[bFull0], 1);
     mbar_init(&bars[bFull1], 1);
-    mbar_init(&bars[bEmpty0], 1);
-    mbar_init(&bars[bEmpty1], 1);
+    mbar_init(&bars[bEmptyBC0], 1);
+    mbar_init(&bars[bEmptyBC1], 1);
+    mbar_init(&bars[bEmptyX0], 1);
+    mbar_init(&bars[bEmptyX1], 1);
     mbar_init(&bars[bPrep0], kNPrep);
     mbar_init(&bars[bPrep1], kNPrep);
     mbar_init(&bars[bSFull], 1);
@@ -611,34 +615,65 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int issued = 0, th_issued = 0;
-      for (int c = 0; c < nchunks; ++c) {
-        const int s = c & 1, u = c >> 1;
-        if (!mbar_wait(&bars[bEmpty0 + s], (u & 1) ^ 1, abort_flag, status, kTagEmpty)) break;
-        uint8_t* st = smem + s * K::STAGE_BYTES;
-        mbar_arrive_expect_tx(&bars[bFull0 + s], K::TMA_BYTES);
-        const int t0 = c * Q;
+      // Three refill streams, each issued as soon as its buffer is free:
+      //   B and C of chunk cb into stage cb % 2 once the state MMAs of chunk cb - 2 have read them,
+      //   x of chunk cx once the Y MMA of chunk cx - 2 has read it,
+      //   theta (+ dt, lam) of chunk ct once prep has read chunk ct - 1's.
+      // One thread polls the three conditions (non-blocking), so no stream waits behind another.
+      int cb = 0, cx = 0, ct = 0;
+      long long t_last = clock64();
+      const uint32_t th_bytes = K::TH_BYTES + (prm.dl_tma ? 2u * K::DL_BYTES : 0u);
+      while (cx < nchunks || ct < nchunks) {
+        bool progress = false;
+        if (cb < nchunks && mbar_test(&bars[bEmptyBC0 + (cb & 1)], ((cb >> 1) & 1) ^ 1)) {
+          const int s = cb & 1, t0 = cb * Q;
+          uint8_t* st = smem + s * K::STAGE_BYTES;
+          mbar_arrive_expect_tx(&bars[bFull0 + s], K::TMA_BYTES);  // B, C and x of chunk cb
 #pragma unroll
-        for (int kb = 0; kb < K::NKB; ++kb) {
-          tma_load_5d(st + K::OFF_B + kb * kTile, &tmB, &bars[bFull0 + s], kb * 64, 0, hh, t0, b);
-          tma_load_5d(st + K::OFF_C + kb * kTile, &tmC, &bars[bFull0 + s], kb * 64, 0, hh, t0, b);
+          for (int kb = 0; kb < K::NKB; ++kb) {
+            tma_load_5d(st + K::OFF_B + kb * kTile, &tmB, &bars[bFull0 + s], kb * 64, 0, hh, t0, b);
+            tma_load_5d(st + K::OFF_C + kb * kTile, &tmC, &bars[bFull0 + s], kb * 64, 0, hh, t0, b);
+          }
+          ++cb;
+          progress = true;
         }
-        tma_load_5d(st + K::OFF_X, &tmX, &bars[bFull0 + s], 0, 0, hh, t0, b);
-        issued = c + 1;
-        // theta of chunk c into the single theta tile once prep has read chunk c-1's
-        if (c > 0 && !mbar_wait(&bars[bThFree], (c - 1) & 1, abort_flag, status, kTagTh)) break;
-        mbar_arrive_expect_tx(&bars[bThFull], K::TH_BYTES + (prm.dl_tma ? 2u * K::DL_BYTES : 0u));
-        tma_load_4d(smem + K::OFF_TH, &tmT, &bars[bThFull], 0, hh, t0, b);
-        if (prm.dl_tma) {
-          tma_load_3d(smem + K::OFF_DL, &tmD, &bars[bThFull], hh & ~7, t0, b);
-          tma_load_3d(smem + K::OFF_DL + K::DL_PAD, &tmL, &bars[bThFull], hh & ~7, t0, b);
+        if (cx < cb && mbar_test(&bars[bEmptyX0 + (cx & 1)], ((cx >> 1) & 1) ^ 1)) {
+          const int s = cx & 1;
+          tma_load_5d(smem + s * K::STAGE_BYTES + K::OFF_X, &tmX, &bars[bFull0 + s], 0, 0, hh, cx * Q, b);
+          ++cx;
+          progress = true;
         }
-        th_issued = c + 1;
+        if (ct < nchunks && (ct == 0 || mbar_test(&bars[bThFree], (ct - 1) & 1))) {
+          const int t0 = ct * Q;
+          mbar_arrive_expect_tx(&bars[bThFull], th_bytes);
+          tma_load_4d(smem + K::OFF_TH, &tmT, &bars[bThFull], 0, hh, t0, b);
+          if (prm.dl_tma) {
+            tma_load_3d(smem + K::OFF_DL, &tmD, &bars[bThFull], hh & ~7, t0, b);
+            tma_load_3d(smem + K::OFF_DL + K::DL_PAD, &tmL, &bars[bThFull], hh & ~7, t0, b);
+          }
+          ++ct;
+          progress = true;
+        }
+        if (progress) {
+          t_last = clock64();
+        } else {
+          if (*abort_flag) break;
+          if (clock64() - t_last > 4000000000LL) {
+            *abort_flag = 1;
+            report_timeout(status, kTagEmpty);
+            break;
+          }
+          __nanosleep(32);
+        }
       }
-      // drain: never leave this CTA with bulk copies still landing in its smem
-      for (int c = issued - 2; c < issued; ++c)
+      // drain: never leave this CTA with bulk copies still landing in its smem.  A
+      // stage whose x load was never issued (abort) gets it now, so that its
+      // full barrier can complete.
+      for (; cx < cb; ++cx)
+        tma_load_5d(smem + (cx & 1) * K::STAGE_BYTES + K::OFF_X, &tmX, &bars[bFull0 + (cx & 1)], 0, 0, hh, cx * Q, b);
+      for (int c = cb - 2; c < cb; ++c)
         if (c >= 0) mbar_wait(&bars[bFull0 + (c & 1)], (c >> 1) & 1, abort_flag, status, kTagDrain, 400000000LL);
-      if (th_issued > 0) mbar_wait(&bars[bThFull], (th_issued - 1) & 1, abort_flag, status, kTagDrain, 400000000LL);
+      if (ct > 0) mbar_wait(&bars[bThFull], (ct - 1) & 1, abort_flag, status, kTagDrain, 400000000LL);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -675,6 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       smem_desc_sw128(cXw + kk * 2048, kTile, 1024), iH, kk > 0);
         }
         mma_commit(&bars[bAcc]);
+        mma_commit(&bars[bEmptyBC0 + s]);  // B~, C~ of this stage are no longer read
         if (!mbar_wait(&bars[bPReady], c & 1, abort_flag, status, kTagP)) break;
         tc_fence_after();
 #pragma unroll
@@ -683,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       kk > 0);
         }
         mma_commit(&bars[bYFull]);
-        mma_commit(&bars[bEmpty0 + s]);
+        mma_commit(&bars[bEmptyX0 + s]);    // x of this stage is no longer read
       }
       // every MMA this thread issued must be complete before TMEM is released
       mma_commit(&bars[bDone]);
