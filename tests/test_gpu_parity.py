@@ -101,6 +101,23 @@ def test_init_state_and_in_place_continuation(dtype):
     check_state(st, fr, TOL[dtype])
 
 
+@pytest.mark.parametrize("shape", [(2, 150, 100, 64, 64, 2), (3, 97, 64, 64, 128, 1)])
+def test_random_init_state_many_units_bf16(shape):
+    """More (batch, head) units than SMs, each starting from its own random
+    state: every CTA initialises the carried state and angle per unit."""
+    b, L, H, P, N, R = shape
+    inp = small_inputs(b, L, H, P, N, R, torch.bfloat16, seed=320 + L)
+    g = torch.Generator().manual_seed(7)
+    st = m3.State(*(torch.randn(*s, generator=g).cuda() for s in
+                    ((b, H, N, P), (b, H, R, N), (b, H, R, P))), torch.rand(b, H, N // 2, generator=g).cuda() * 6 - 3)
+    ref_init = to_state_np(st)
+    y, fin = gpu_scan(inp, init=st)
+    yr, fr = oracle_scan(inp, init=ref_init)
+    e = rel_err(y.float().cpu().double().numpy(), yr)
+    assert e < TOL[torch.bfloat16], e
+    check_state(fin, fr, TOL[torch.bfloat16])
+
+
 def test_random_init_state_fp32():
     b, L, H, P, N, R = 1, 100, 2, 16, 16, 2
     inp = small_inputs(b, L, H, P, N, R, torch.float32, seed=310)
