@@ -31,7 +31,40 @@ from linear_recurrent_scan_b200 import workloads as wl  # noqa: E402
 
 PREFILL = wl.CONFIGS["siso_prefill_b8_l2048"]
 DECODE = [wl.CONFIGS["siso_decode_b128"], wl.CONFIGS["mimo4_decode_b128"]]
+# further prefill shapes of the benchmark table (reported beside the headline)
+PREFILL_MORE = [wl.CONFIGS["mimo4_prefill_b4_l8192"], wl.CONFIGS["mimo4_long_b1_l65536"]]
+# batch-1 decode after the 65536-token MIMO prefill: latency-bound (2.5 MB per step)
+DECODE_LONG = wl.CONFIGS["mimo4_long_b1_l65536"].with_(prefill_tokens=65536)
 FALLBACK_HBM_GBS = 6650.0
+
+# DRAM bytes (read + write) per launch from ncu captures of the kernels as they
+# stand: (kernel source files, sha256 of their concatenation, bytes per launch,
+# capture).  A kernel whose sources no longer hash to the recorded value gets
+# traffic null, since its counters are out of date.
+TRAFFIC = {
+    "prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"), None, None, None),
+    "siso_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), None, None, None),
+    "mimo4_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), None, None, None),
+}
+
+
+def sources_sha(files) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "linear_recurrent_scan_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def traffic(key):
+    files, sha, nbytes, _ = TRAFFIC[key]
+    if sha is None or nbytes is None:
+        return None
+    try:
+        return nbytes if sources_sha(files) == sha else None
+    except OSError:
+        return None
 
 
 def esize(dt):
@@ -237,6 +270,35 @@ def run_prefill(m3, args, world, rank, clk):
                 tokens=w.batch * w.seqlen, bytes=prefill_bytes(w))
 
 
+def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup):
+    """Median per-launch time (ms) of one prefill launch of workload `w`, inputs
+    resident on the device (larger than L2), final state exported."""
+    dev = torch.device("cuda")
+    inp = wl.make_inputs(w, seed=wl.BASE_SEED + rank, device=dev)
+    ins = [inp[n] for n in NAMES]
+    y = torch.empty_like(inp["x"])
+    fin = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
+    dims = m3.make_dims(inp["x"], inp["B"])
+    ws = torch.zeros(max(256, m3.mamba3_scan_workspace_bytes(dims)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        m3.mamba3_scan_fwd(*ins, inp["A"], inp["D"], y=y, final_state=fin, workspace=ws, stream=stream)
+    times = []
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        m3.mamba3_scan_fwd(*ins, inp["A"], inp["D"], y=y, final_state=fin, workspace=ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    status = m3.mamba3_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status after {w.name}: {m3.mamba3_status_string(status)}")
+    del inp, ins, y, fin, ws
+    torch.cuda.empty_cache()
+    return statistics.median(times)
+
+
 def run_decode(m3, w: wl.Workload, world, rank, steps):
     """Seed the state with a 512-token prefill, then time `steps` decode steps
     captured in one CUDA graph (per-step inputs pre-generated, larger than L2)."""
@@ -294,11 +356,25 @@ def ours(args):
         gbs = decode_bytes(w) / (us * 1e-6) / 1e9
         dec[w.name] = {"us_per_step": round(us, 2), "steps": w.decode_steps, "batch": w.batch, "rank": w.rank,
                        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                                    "frac": round(gbs / peak, 4), "traffic": None,
+                                    "frac": round(gbs / peak, 4), "traffic": traffic(w.name),
                                     "bytes_per_step": decode_bytes(w)}}
+    us = run_decode(m3, DECODE_LONG, world, rank, DECODE_LONG.decode_steps)
+    dec["mimo4_long_decode_b1"] = {"us_per_step": round(us, 2), "steps": DECODE_LONG.decode_steps, "batch": 1,
+                                   "rank": DECODE_LONG.rank, "dstate": DECODE_LONG.dstate,
+                                   "state_from_prefill_tokens": DECODE_LONG.prefill_tokens,
+                                   "roofline": None, "note": "latency-bound: %d bytes per step" % decode_bytes(DECODE_LONG)}
+    more = {}
+    for w in PREFILL_MORE:
+        ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=max(5, min(args.steps, 20)), warmup=3), world)
+        by = prefill_bytes(w)
+        gbs = by / (ms * 1e-3) / 1e9
+        more[w.name] = {"ms_per_launch": round(ms, 4), "mtokens_s": round(w.batch * w.seqlen / (ms * 1e-3) / 1e6, 3),
+                        "batch": w.batch, "seqlen": w.seqlen, "rank": w.rank, "dstate": w.dstate,
+                        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                                     "frac": round(gbs / peak, 4), "bytes_per_launch": by}}
     clk.stop()
     clocks = clk.summary()
-    clocks["window"] = "prefill timed steps through the decode graph replays"
+    clocks["window"] = "headline prefill timed steps through the decode replays and the further prefill shapes"
     e2e_value = tokens_all / (r["e2e_ms"] * 1e-3) / 1e6
     out = {
         "metric": "prefill Mtokens/s (SISO, batch 8, seqlen 2048) and decode step us at batch 128",
@@ -318,8 +394,9 @@ def ours(args):
                    "rank": PREFILL.rank, "state_dtype": "fp32", "parallelism": f"batch-sharded x{world} (weak)",
                    "l2": "inputs (%.0f MB) larger than L2 (126 MB); no flush" % (r["bytes"] / 1e6)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                     "frac": round(achieved / peak, 4), "traffic": traffic("prefill"), "peak_kind": peak_kind,
                      "bytes_per_launch": r["bytes"], "launch_ms": round(r["launch_ms"], 4)},
+        "prefill_more": more,
         "decode": dec,
         "e2e": {"value": round(e2e_value, 3), "unit": "Mtokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},

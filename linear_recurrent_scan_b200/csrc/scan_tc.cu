@@ -33,10 +33,13 @@
 //                Prep runs up to two chunks ahead of the MMAs.
 //   warps 10..17 epilogue, two warps per TMEM lane quadrant (column halves):
 //                S -> P (bf16, back into TMEM), hbar update and its bf16 copy
-//                for the next chunk's inter-chunk MMA, y = Y + e^{cum} Yi.
+//                for the next chunk's inter-chunk MMA, y = Y + e^{cum} Yi
+//                (with R = 1 for the previous chunk, so that the Y MMA's
+//                latency is off the epilogue's path).
 // MMAs per chunk: S = C~ B~^T; Yi = C~ hbar_in; Hacc = B~^T X_w (smem operands);
 // Y = P X (P from TMEM).  TMEM columns: S [0,128), P [128,192) (bf16 pairs),
-// Y [192,256), Yi [256,320), Hacc [320,384).
+// Y [192,256), Yi [256,320), Hacc [320,384); with R = 1 a second Y, Yi buffer at
+// [384,448), [448,512) (y written one chunk late).
 // Every wait is bounded: on expiry the CTA raises an abort flag, reports
 // MAMBA3_ERR_TIMEOUT in the device status word, drains and returns.
 #include <cuda.h>
@@ -61,7 +64,9 @@ constexpr int kNPrep = 256;
 constexpr int kEpi0 = kPrep0 + kNPrep;
 constexpr int kNEpi = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColP = 128, kColY = 192, kColYi = 256, kColH = 320;
+// With R = 1, Y and Yi are double-buffered (chunk c at + (c % 2) * kColYBuf) and
+// the epilogue writes y of chunk c while the MMAs of chunk c + 1 run.
+constexpr uint32_t kColS = 0, kColP = 128, kColY = 192, kColYi = 256, kColH = 320, kColYBuf = 192;
 
 enum Tag { kTagEmpty = 1, kTagFull, kTagPrep1, kTagSFull, kTagAcc, kTagEpiDone, kTagP, kTagY, kTagDrain, kTagTh };
 
@@ -74,6 +79,9 @@ struct Cfg {
   static constexpr int NPART = kNPrep / NG;  // token parts of the angle scan
   static constexpr int TPP = Q / NPART;  // tokens per part
   static constexpr int TB = (R == 1 && TPP % 2 == 0) ? 2 : 1;  // tokens per rotation batch
+  // y one chunk late (double-buffered Y, Yi): shortens the epilogue's chain;
+  // measured faster for R = 1 only
+  static constexpr bool DEFER_Y = (R == 1);
   static constexpr int STAGE_BYTES = (2 * NKB + 1) * kTile;  // B, C, X
   static constexpr int TMA_BYTES = STAGE_BYTES;
   static constexpr int OFF_B = 0, OFF_C = NKB * kTile, OFF_X = 2 * NKB * kTile;
@@ -391,6 +399,34 @@ __device__ __forceinline__ void store_hbar_bf16(const float (&hb)[32], uint8_t* 
   }
 }
 
+// y rows of one chunk from its Y and Yi accumulators: y = Y + e^{cum_t} Yi
+// (this thread's 32 columns of row m); rows past the sequence are not stored
+__device__ __forceinline__ void store_y(const ScanArgs& a, uint32_t tY, uint32_t tYi, float e, int b, int hh, int tg,
+                                        int rm, int R, int ch) {
+  uint4* yr = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) +
+                                       (tok_index(a, b, tg < a.seqlen ? tg : 0, hh) * R + rm) * kP + 32 * ch);
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    float yv[16], yi[16];
+    __syncwarp();
+    tmem_ld16(tY + 32 * ch + 16 * half, yv);
+    tmem_ld16(tYi + 32 * ch + 16 * half, yi);
+    tmem_ld_wait();
+    if (tg < a.seqlen) {
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int o = 8 * q2;
+        uint4 q;
+        q.x = pack_bf16(yv[o + 0] + e * yi[o + 0], yv[o + 1] + e * yi[o + 1]);
+        q.y = pack_bf16(yv[o + 2] + e * yi[o + 2], yv[o + 3] + e * yi[o + 3]);
+        q.z = pack_bf16(yv[o + 4] + e * yi[o + 4], yv[o + 5] + e * yi[o + 5]);
+        q.w = pack_bf16(yv[o + 6] + e * yi[o + 6], yv[o + 7] + e * yi[o + 7]);
+        yr[2 * half + q2] = q;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ epilogue warps
 // Two warps per TMEM lane quadrant: thread = (row m = 32 quad + lane, column
 // half ch).  Row m of S, P, Y, Yi; state row n of Hacc / hbar (for N = 64 the
@@ -439,6 +475,7 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
   fence_proxy_async_smem();
   mbar_arrive(&bars[bEpiDone]);
 
+  float e_prev = 0.f;  // (deferred y) e^{cum} of row m in the previous chunk
   for (int c = 0; c < nchunks; ++c) {
     const int s = c & 1, u = c >> 1;
     const int t0 = c * Q;
@@ -519,10 +556,15 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     }
 
     // ---- y = Y + e^{cum_t} Yi ----
-    mbar_wait(&bars[bYFull], c & 1, abort_flag, status, kTagY);
-    if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
-    tc_fence_after();
-    {
+    if constexpr (K::DEFER_Y) {  // the previous chunk's (its Y MMA completed before this chunk's S)
+      if (c > 0)
+        store_y(a, tmem + lane_base + kColY + ((c - 1) & 1) * kColYBuf,
+                tmem + lane_base + kColYi + ((c - 1) & 1) * kColYBuf, e_prev, b, hh, t0 - Q + tm, rm, R, ch);
+      e_prev = my_e;
+    } else {
+      mbar_wait(&bars[bYFull], c & 1, abort_flag, status, kTagY);
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
+      tc_fence_after();
       const int tg = t0 + tm;
       uint4* yr = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) +
                                            (tok_index(a, b, tg < L ? tg : 0, hh) * R + rm) * kP + 32 * ch);
@@ -549,6 +591,15 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     tc_fence_before();
     fence_proxy_async_smem();  // hbar (bf16) is read by the next chunk's MMA
     mbar_arrive(&bars[bEpiDone]);
+  }
+  if constexpr (K::DEFER_Y) {  // y of the last chunk (the Y barrier is committed for it alone)
+    mbar_wait(&bars[bYFull], 0, abort_flag, status, kTagY);
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
+    tc_fence_after();
+    const int cl = nchunks - 1;
+    store_y(a, tmem + lane_base + kColY + (cl & 1) * kColYBuf, tmem + lane_base + kColYi + (cl & 1) * kColYBuf, e_prev,
+            b, hh, cl * Q + tm, rm, R, ch);
+    tc_fence_before();
   }
 }
 
@@ -687,6 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = c & 1, u = c >> 1;
         const uint32_t st = sbase + s * K::STAGE_BYTES;
         const uint32_t cB = st + K::OFF_B, cC = st + K::OFF_C, cX = st + K::OFF_X, cXw = sbase + K::OFF_XW;
+        const uint32_t ybuf = K::DEFER_Y ? (c & 1) * kColYBuf : 0u;  // Y, Yi buffer of this chunk
         if (!mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1)) break;
         tc_fence_after();
 #pragma unroll
@@ -701,7 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < N / 16; ++kk) {
           const uint32_t offa = (kk >> 2) * kTile + (kk & 3) * 32;
-          mma_bf16_ss(tmem + kColYi, smem_desc_sw128(cC + offa, 16, 1024),
+          mma_bf16_ss(tmem + kColYi + ybuf, smem_desc_sw128(cC + offa, 16, 1024),
                       smem_desc_sw128(sbase + K::OFF_H + kk * 2048, N * 128, 1024), iYi, kk > 0);
         }
 #pragma unroll
@@ -715,10 +767,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kM / 16; ++kk) {
-          mma_bf16_ts(tmem + kColY, tmem + kColP + 8 * kk, smem_desc_sw128(cX + kk * 2048, kTile, 1024), iY,
+          mma_bf16_ts(tmem + kColY + ybuf, tmem + kColP + 8 * kk, smem_desc_sw128(cX + kk * 2048, kTile, 1024), iY,
                       kk > 0);
         }
-        mma_commit(&bars[bYFull]);
+        // (deferred y: Y of chunk c is complete once S of chunk c + 1 is, since a
+        // commit covers every earlier MMA; only the last chunk's Y gets the barrier)
+        if (!K::DEFER_Y || c == nchunks - 1) mma_commit(&bars[bYFull]);
         mma_commit(&bars[bEmptyX0 + s]);    // x of this stage is no longer read
       }
       // every MMA this thread issued must be complete before TMEM is released
