@@ -42,9 +42,15 @@ FALLBACK_HBM_GBS = 6650.0
 # capture).  A kernel whose sources no longer hash to the recorded value gets
 # traffic null, since its counters are out of date.
 TRAFFIC = {
-    "prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"), None, None, None),
-    "siso_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), None, None, None),
-    "mimo4_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), None, None, None),
+    "prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"),
+                "cab7ade096cf20b585c2edafd11f8c802cbee49440e69063f1f9c8ac5a5e7de7", 811488256 + 136867584,
+                "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "siso_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
+                         "ac70b819247a216ebf772caf5eae8b70b922c205d4f263759cc72849df1f75dd", 283208192 + 218755840,
+                         "profiles/decode_stream_b128_traffic_and_counters.txt"),
+    "mimo4_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
+                          "ac70b819247a216ebf772caf5eae8b70b922c205d4f263759cc72849df1f75dd", 317780736 + 239914496,
+                          "profiles/decode_stream_b128_traffic_and_counters.txt"),
 }
 
 
