@@ -75,6 +75,8 @@ def _bind(lib):
         f = getattr(lib, name)
         f.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_IO), ctypes.c_int]
         f.restype = ctypes.c_int
+    lib.m3o_bc_norm.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.c_double, _P]
+    lib.m3o_bc_norm.restype = ctypes.c_int
     return lib
 
 
@@ -195,3 +197,22 @@ def decode_step(state: State, x, B, C, theta, dt, lam, A, D=None, nthreads=None)
 
 
 __all__ = ["build", "State", "scan_complex", "scan_rope", "scan_quadratic", "decode_step"]
+
+
+def bc_norm(z, w=None, bias=None, eps: float = 1e-6) -> np.ndarray:
+    """RMS normalisation of raw B or C projections over the state dimension N,
+    then a per-(head, rank) weight and bias: z [..., L, H, R, N] (leading batch
+    dims flattened), w, bias [H, R, N] or None.  Source: "Mamba-3: 2x smaller
+    state ..." (MarkTechPost, Korean translation), section 2 (B/C norm and
+    head-specific bias)."""
+    z = _f64(z)
+    *lead, H, R, N = z.shape
+    rows = int(np.prod(lead)) if lead else 1
+    dims = _Dims(1, rows, H, 0, N, R)
+    w = _f64(w) if w is not None else None
+    bias = _f64(bias) if bias is not None else None
+    for a in (w, bias):
+        assert a is None or a.shape == (H, R, N), "weight and bias must be [H, R, N]"
+    out = np.empty_like(z)
+    _load().m3o_bc_norm(ctypes.byref(dims), _ptr(z), _ptr(w), _ptr(bias), float(eps), _ptr(out))
+    return out

@@ -30,7 +30,10 @@
  *   m3o_scan_quadratic  -- the L x L masked-kernel ("quadratic") form, brute
  *                          force, for tiny inputs.
  * plus m3o_decode_step, which is one token of m3o_scan_complex continued
- * from a state.
+ * from a state, and m3o_bc_norm, the RMS normalisation of raw B or C
+ * projections over the state dimension with a per-(head, rank) weight and bias
+ * (same page, section 2: "BC norm" and head-specific B/C bias), which the
+ * recurrence then consumes.
  *
  * Layouts (row-major, contiguous; b = batch, L = seqlen, H = heads):
  *   x      [b, L, H, R, P]     B, C  [b, L, H, R, N]     theta [b, L, H, N/2]
@@ -393,4 +396,29 @@ int m3o_scan_quadratic(const m3o_dims* d, const m3o_io* io, int nthreads) {
 int m3o_decode_step(const m3o_dims* d, const m3o_io* io, int nthreads) {
   if (!d || d->seqlen != 1) return -1;
   return run_units(d, io, unit_complex, nthreads, NULL, 0);
+}
+
+/* ------------------------------------------------------------------------- */
+/* B/C normalisation: for every row (b, t, h, r) of a raw projection Z
+ * [b, L, H, R, N],
+ *     out[n] = Z[n] / sqrt(mean_n' Z[n']^2 + eps) * w[h, r, n] + bias[h, r, n],
+ * with w = 1 when NULL and bias = 0 when NULL.  Same page, section 2 (RMS norm
+ * of B and C, head-specific bias); the placement of eps inside the square root
+ * and of the bias after the weight is the standard RMS-norm form. */
+int m3o_bc_norm(const m3o_dims* d, const double* z, const double* w, const double* bias, double eps, double* out) {
+  const int N = d->dstate, R = d->rank, H = d->nheads;
+  const size_t rows = (size_t)d->batch * d->seqlen * H * R;
+  for (size_t row = 0; row < rows; ++row) {
+    const int r = (int)(row % R), h = (int)((row / R) % H);
+    const double* zr = z + row * N;
+    double ms = 0.0;
+    for (int n = 0; n < N; ++n) ms += zr[n] * zr[n];
+    ms /= N;
+    const double inv = 1.0 / sqrt(ms + eps);
+    for (int n = 0; n < N; ++n) {
+      const size_t p = ((size_t)h * R + r) * N + n;
+      out[row * N + n] = zr[n] * inv * (w ? w[p] : 1.0) + (bias ? bias[p] : 0.0);
+    }
+  }
+  return 0;
 }

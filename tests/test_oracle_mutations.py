@@ -26,6 +26,9 @@ MUTATIONS = {
     "rope_sign": ("*o1 = -sin(phi) * v0 + cos(phi) * v1;", "*o1 = sin(phi) * v0 + cos(phi) * v1;"),
     "quadratic_weight_next": ("(1.0 - io->lam[in]) * io->dt[in]", "(1.0 - io->lam[is]) * io->dt[is]"),
     "mimo_rank_drop": ("for (int r = 0; r < R; ++r)\n          s += (Bt", "for (int r = 0; r < 1; ++r)\n          s += (Bt"),
+    "bcnorm_sum_not_mean": ("    ms /= N;\n", "\n"),
+    "bcnorm_eps_outside_sqrt": ("1.0 / sqrt(ms + eps)", "1.0 / (sqrt(ms) + eps)"),
+    "bcnorm_bias_index_swapped": ("const size_t p = ((size_t)h * R + r) * N + n;", "const size_t p = ((size_t)r * H + h) * N + n;"),
 }
 
 PIN_FUNCS = [
@@ -38,6 +41,10 @@ PIN_FUNCS = [
     lambda: [pins.test_complex_equals_rope(r) for r in (1, 3)],
     lambda: [pins.test_quadratic_equals_recurrence(r) for r in (1, 2)],
     pins.test_mimo_is_superposition_of_siso,
+    pins.test_bc_norm_constant_row_closed_form,
+    pins.test_bc_norm_unit_rms_per_row,
+    pins.test_bc_norm_scale_invariant_and_odd,
+    pins.test_bc_norm_weight_and_bias_per_head_and_rank,
 ]
 
 

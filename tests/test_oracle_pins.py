@@ -373,3 +373,52 @@ def test_units_subset_matches_full():
         bb, hh = divmod(u, 3)
         assert np.array_equal(ys[bb, :, hh], y[bb, :, hh])
         assert np.array_equal(fs.h[bb, hh], f.h[bb, hh])
+
+
+# ---------------------------------------------------------------- B/C normalisation
+# "Mamba-3: 2x smaller state ..." (MarkTechPost, Korean translation), section 2:
+# RMS norm of B and C over the state dimension, then a head-specific weight and bias.
+
+def test_bc_norm_constant_row_closed_form():
+    """A constant row c * 1_N gives c / sqrt(c^2 + eps) exactly: pins the mean (not
+    the sum) over N and eps inside the square root (eps dominates here)."""
+    N, c, eps = 16, 1e-3, 1e-4
+    z = np.full((1, 1, 1, 1, N), c)
+    out = oracle.bc_norm(z, eps=eps)
+    assert np.allclose(out, c / np.sqrt(c * c + eps), rtol=1e-14, atol=0)
+    assert abs(out[0, 0, 0, 0, 0] - 0.0995037190209989) < 1e-15
+
+
+def test_bc_norm_unit_rms_per_row():
+    """With eps = 0, unit weight and no bias every (b, t, h, r) row has RMS 1 over
+    N, whatever the scale of the rows (pins the axis of the norm)."""
+    rng = np.random.default_rng(91)
+    z = rng.normal(size=(2, 5, 3, 2, 8)) * rng.uniform(0.01, 100.0, size=(2, 5, 3, 2, 1))
+    out = oracle.bc_norm(z, eps=0.0)
+    assert np.allclose(np.sqrt((out ** 2).mean(-1)), 1.0, rtol=1e-13)
+
+
+def test_bc_norm_scale_invariant_and_odd():
+    rng = np.random.default_rng(92)
+    z = rng.normal(size=(1, 4, 2, 3, 8))
+    base = oracle.bc_norm(z, eps=0.0)
+    assert np.allclose(oracle.bc_norm(7.5 * z, eps=0.0), base, rtol=1e-13)
+    assert np.allclose(oracle.bc_norm(-z, eps=0.0), -base, rtol=1e-13)
+
+
+def test_bc_norm_weight_and_bias_per_head_and_rank():
+    """Weight and bias index (head, rank, n): with H != R and distinct values per
+    (h, r), a transposed or shared operand moves the rows' means away from the
+    bias and their scale away from the weight."""
+    rng = np.random.default_rng(93)
+    H, R, N = 3, 2, 8
+    z = rng.normal(size=(2, 6, H, R, N))
+    w = rng.uniform(0.5, 2.0, size=(H, R, N))
+    bias = rng.normal(size=(H, R, N)) * 3
+    out = oracle.bc_norm(z, w, bias, eps=0.0)
+    unit = oracle.bc_norm(z, eps=0.0)
+    assert np.allclose((out - bias) / w, unit, rtol=1e-12, atol=1e-12)
+    for h in range(H):
+        for r in range(R):
+            rows = (out[:, :, h, r, :] - bias[h, r]) / w[h, r]
+            assert np.allclose(np.sqrt((rows ** 2).mean(-1)), 1.0, rtol=1e-12)
