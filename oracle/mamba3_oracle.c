@@ -402,7 +402,8 @@ int m3o_decode_step(const m3o_dims* d, const m3o_io* io, int nthreads) {
 /* B/C normalisation: for every row (b, t, h, r) of a raw projection Z
  * [b, L, H, R, N],
  *     out[n] = Z[n] / sqrt(mean_n' Z[n']^2 + eps) * w[h, r, n] + bias[h, r, n],
- * with w = 1 when NULL and bias = 0 when NULL.  Same page, section 2 (RMS norm
+ * with w = 1 when NULL and bias = 0 when NULL (an all-zero row with eps = 0
+ * gives bias: 0/0 is read as 0).  Same page, section 2 (RMS norm
  * of B and C, head-specific bias); the placement of eps inside the square root
  * and of the bias after the weight is the standard RMS-norm form. */
 int m3o_bc_norm(const m3o_dims* d, const double* z, const double* w, const double* bias, double eps, double* out) {
@@ -414,7 +415,8 @@ int m3o_bc_norm(const m3o_dims* d, const double* z, const double* w, const doubl
     double ms = 0.0;
     for (int n = 0; n < N; ++n) ms += zr[n] * zr[n];
     ms /= N;
-    const double inv = 1.0 / sqrt(ms + eps);
+    /* an all-zero row with eps = 0 is 0/0; it normalises to 0 (then the bias) */
+    const double inv = (ms + eps > 0.0) ? 1.0 / sqrt(ms + eps) : 0.0;
     for (int n = 0; n < N; ++n) {
       const size_t p = ((size_t)h * R + r) * N + n;
       out[row * N + n] = zr[n] * inv * (w ? w[p] : 1.0) + (bias ? bias[p] : 0.0);

@@ -422,3 +422,12 @@ def test_bc_norm_weight_and_bias_per_head_and_rank():
         for r in range(R):
             rows = (out[:, :, h, r, :] - bias[h, r]) / w[h, r]
             assert np.allclose(np.sqrt((rows ** 2).mean(-1)), 1.0, rtol=1e-12)
+
+
+def test_bc_norm_zero_row_gives_bias():
+    """Reading: an all-zero row with eps = 0 (0/0) normalises to 0, leaving the bias."""
+    H, R, N = 2, 1, 8
+    z = np.zeros((1, 1, H, R, N))
+    bias = np.arange(H * R * N, dtype=np.float64).reshape(H, R, N)
+    out = oracle.bc_norm(z, None, bias, eps=0.0)
+    assert np.array_equal(out[0, 0], bias)
