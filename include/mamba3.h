@@ -124,6 +124,45 @@ MAMBA3_API int mamba3_decode_step(const mamba3_dims* dims, const mamba3_state* s
                        const void* B, const void* C, const void* theta, const void* dt,
                        const void* lam, const float* A, const float* D, void* y, void* stream);
 
+/*
+ * Fused B/C normalisation ahead of the recurrence ("Mamba-3: 2x smaller state
+ * ..." (MarkTechPost, Korean translation), section 2: RMS norm of B and C and a
+ * head-specific bias).  For every (b, t, h, r) row of the raw projections,
+ *     B[n] = B_raw[n] / sqrt(mean_n B_raw^2 + eps) * w_B[h,r,n] + bias_B[h,r,n]
+ * (C likewise), computed in float32 from the raw inputs and then rotated as in
+ * mamba3_scan_fwd.  w_B, w_C, bias_B, bias_C: device float32 [H, R, N],
+ * contiguous, 4-byte aligned, each nullable (weight 1, bias 0); eps >= 0.
+ */
+typedef struct {
+  const float *w_B, *w_C, *bias_B, *bias_C;
+  float eps;
+} mamba3_bc_norm;
+
+/*
+ * mamba3_scan_fwd with raw B and C projections (layouts as B and C there) and
+ * the normalisation `norm` (not nullable) fused in front of the rotation.  The
+ * exported state (b_prev) holds the normalised, rotated B, so a continuation
+ * may use either entry point.  Supported: bf16 inputs, P = 64, N in {64, 128},
+ * R in {1, 2, 4} (the tensor-core path); other shapes return
+ * MAMBA3_ERR_UNSUPPORTED before anything is enqueued.
+ */
+MAMBA3_API int mamba3_scan_fwd_bcnorm(const mamba3_dims* dims, const void* x, const void* B_raw,
+                                      const void* C_raw, const void* theta, const void* dt, const void* lam,
+                                      const float* A, const float* D, const mamba3_bc_norm* norm,
+                                      const mamba3_state* init, void* y, const mamba3_state* final_state,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mamba3_decode_step with raw B and C of the token and the normalisation
+ * `norm` (not nullable) fused in front of the rotation.  Supported: P = 64,
+ * N in {64, 128}, R in {1, 2, 4}, 16-byte aligned state and input pointers;
+ * other cases return MAMBA3_ERR_UNSUPPORTED.
+ */
+MAMBA3_API int mamba3_decode_step_bcnorm(const mamba3_dims* dims, const mamba3_state* state, const void* x,
+                                         const void* B_raw, const void* C_raw, const void* theta, const void* dt,
+                                         const void* lam, const float* A, const float* D,
+                                         const mamba3_bc_norm* norm, void* y, void* stream);
+
 /* Synchronises `stream`, then returns the device status word that the last
  * mamba3_scan_fwd on `workspace` left (MAMBA3_OK or MAMBA3_ERR_TIMEOUT), or
  * MAMBA3_ERR_CUDA / MAMBA3_ERR_INVALID. */

@@ -10,6 +10,7 @@ Entry points (same names as the C ABI):
   mamba3_scan_workspace_bytes(dims)
   mamba3_scan_fwd(x, B, C, theta, dt, lam, A, D=None, init=None, ...)
   mamba3_decode_step(state, x, B, C, theta, dt, lam, A, D=None, ...)
+  mamba3_scan_fwd_bcnorm / mamba3_decode_step_bcnorm (raw B, C + BCNorm)
   mamba3_device_status(workspace)
   mamba3_status_string(code)
 """
@@ -56,6 +57,11 @@ class _CState(ctypes.Structure):
                 ("angle", ctypes.c_void_p)]
 
 
+class _CNorm(ctypes.Structure):
+    _fields_ = [("w_B", ctypes.c_void_p), ("w_C", ctypes.c_void_p), ("bias_B", ctypes.c_void_p),
+                ("bias_C", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
 _lib = None
 
 
@@ -82,6 +88,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba3_status_string.restype = ctypes.c_char_p
     lib.mamba3_version.argtypes = []
     lib.mamba3_version.restype = i
+    lib.mamba3_scan_fwd_bcnorm.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(_CNorm),
+                                           ctypes.POINTER(_CState), vp, ctypes.POINTER(_CState), vp, sz, vp]
+    lib.mamba3_scan_fwd_bcnorm.restype = i
+    lib.mamba3_decode_step_bcnorm.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(_CState), vp, vp, vp, vp, vp, vp,
+                                              vp, vp, ctypes.POINTER(_CNorm), vp, vp]
+    lib.mamba3_decode_step_bcnorm.restype = i
     _lib = lib
     return lib
 
@@ -229,13 +241,76 @@ def mamba3_scan_fwd_noalloc(x, B, C, theta, dt, lam, A, D=None, init: Optional[S
     return y
 
 
+@dataclass
+class BCNorm:
+    """Fused B/C normalisation (see mamba3.h): float32 device tensors [H, R, N]
+    or None (weight 1, bias 0), and eps."""
+    w_B: Optional[torch.Tensor] = None
+    w_C: Optional[torch.Tensor] = None
+    bias_B: Optional[torch.Tensor] = None
+    bias_C: Optional[torch.Tensor] = None
+    eps: float = 1e-6
+
+    def _c(self, H, R, N) -> _CNorm:
+        for name in ("w_B", "w_C", "bias_B", "bias_C"):
+            t = getattr(self, name)
+            if t is not None and (t.dtype != torch.float32 or t.shape != (H, R, N) or not t.is_contiguous()):
+                raise ValueError(f"{name} must be a contiguous float32 tensor of shape [H, R, N]")
+        return _CNorm(_ptr(self.w_B), _ptr(self.w_C), _ptr(self.bias_B), _ptr(self.bias_C), float(self.eps))
+
+
+def mamba3_scan_fwd_bcnorm(x, B_raw, C_raw, theta, dt, lam, A, D=None, norm: Optional[BCNorm] = None,
+                           init: Optional[State] = None, y: Optional[torch.Tensor] = None,
+                           final_state: Optional[State] = None, workspace: Optional[torch.Tensor] = None,
+                           chunk: int = 0, stream=None):
+    """mamba3_scan_fwd on raw B, C projections with the B/C normalisation fused in."""
+    lib = load_library()
+    _check_inputs(x, B_raw, C_raw, theta, dt, lam, A, D, decode=False)
+    norm = norm if norm is not None else BCNorm()
+    dims = make_dims(x, B_raw, chunk)
+    cn = norm._c(x.shape[2], x.shape[3], B_raw.shape[-1])
+    if y is None:
+        y = torch.empty_like(x)
+    if workspace is None:
+        workspace = torch.empty(mamba3_scan_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
+    ci = init._c() if init is not None else None
+    cf = final_state._c() if final_state is not None else None
+    rc = lib.mamba3_scan_fwd_bcnorm(ctypes.byref(dims), _ptr(x), _ptr(B_raw), _ptr(C_raw), _ptr(theta), _ptr(dt),
+                                    _ptr(lam), _ptr(A), _ptr(D), ctypes.byref(cn),
+                                    ctypes.byref(ci) if ci is not None else None, _ptr(y),
+                                    ctypes.byref(cf) if cf is not None else None, _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mamba3_scan_fwd_bcnorm")
+    return y
+
+
+def mamba3_decode_step_bcnorm(state: State, x, B_raw, C_raw, theta, dt, lam, A, D=None,
+                              norm: Optional[BCNorm] = None, y: Optional[torch.Tensor] = None, stream=None):
+    """mamba3_decode_step on the raw B, C projections of the token with the B/C
+    normalisation fused in."""
+    lib = load_library()
+    _check_inputs(x, B_raw, C_raw, theta, dt, lam, A, D, decode=True)
+    norm = norm if norm is not None else BCNorm()
+    dims = make_dims(x, B_raw, decode=True)
+    cn = norm._c(x.shape[1], x.shape[2], B_raw.shape[-1])
+    if y is None:
+        y = torch.empty_like(x)
+    cs = state._c()
+    rc = lib.mamba3_decode_step_bcnorm(ctypes.byref(dims), ctypes.byref(cs), _ptr(x), _ptr(B_raw), _ptr(C_raw),
+                                       _ptr(theta), _ptr(dt), _ptr(lam), _ptr(A), _ptr(D), ctypes.byref(cn), _ptr(y),
+                                       _stream(stream))
+    _check(rc, "mamba3_decode_step_bcnorm")
+    return y
+
+
 def mamba3_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(load_library().mamba3_device_status(_ptr(workspace), _stream(stream)))
 
 
 __all__ = [
-    "Dims", "State", "Mamba3Error", "load_library", "make_dims",
+    "Dims", "State", "BCNorm", "Mamba3Error", "load_library", "make_dims",
     "mamba3_scan_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc", "mamba3_decode_step",
+    "mamba3_scan_fwd_bcnorm", "mamba3_decode_step_bcnorm",
     "mamba3_device_status",
     "mamba3_status_string",
 ]

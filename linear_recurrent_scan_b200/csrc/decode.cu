@@ -206,7 +206,7 @@ struct DStage {  // byte offsets inside one stage; every region is a multiple of
   static constexpr int TOTAL = BAR + 64;
 };
 
-template <typename T, int N, int R>
+template <typename T, int N, int R, bool BCN>
 __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) {
   using S = DStage<T, N, R>;
   constexpr int K2 = N / 2, ROWS = N / 16;
@@ -268,6 +268,22 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
     const float Dh = a.D ? a.D[hh] : 0.f;
     ptx::mbar_wait(&bars[s], (it >> 1) & 1, abort_flag, nullptr, 0);
     if (__syncthreads_or(*abort_flag != 0)) break;
+    float* rinv = reinterpret_cast<float*>(dsm + S::BAR + 32);  // fused norm: 1/RMS of B rows, then C rows
+    if constexpr (BCN) {  // warp w < 2R: raw row w % R of B (w < R) or of C
+      if (warp < 2 * R) {
+        const T* row = reinterpret_cast<const T*>(st + (warp < R ? S::B : S::C)) + (warp % R) * N;
+        float ss = 0.f;
+        for (int n = lane; n < N; n += 32) {
+          const float v = ld1(row + n);
+          ss += v * v;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float v = ss * (1.f / N) + a.neps;
+        if (lane == 0) rinv[warp] = v > 0.f ? rsqrtf(v) : 0.f;  // all-zero row, eps = 0: 0, not 0/0
+      }
+      __syncthreads();
+    }
 
     // ---- rotation of B and C by the updated angle; the carry for the next step ----
     const float* ang = reinterpret_cast<const float*>(st + S::ANG);
@@ -280,8 +296,16 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
       const float phi = wrap_angle(ang[k] + dt * ld1(THs + k));
       float sn, cs;
       sincosf(phi, &sn, &cs);
-      const float b0 = ld1(Bs + r * N + 2 * k), b1 = ld1(Bs + r * N + 2 * k + 1);
-      const float c0 = ld1(Cs + r * N + 2 * k), c1 = ld1(Cs + r * N + 2 * k + 1);
+      float b0 = ld1(Bs + r * N + 2 * k), b1 = ld1(Bs + r * N + 2 * k + 1);
+      float c0 = ld1(Cs + r * N + 2 * k), c1 = ld1(Cs + r * N + 2 * k + 1);
+      if constexpr (BCN) {  // normalised row times the head's weight, plus its bias
+        const size_t q = ((size_t)hh * R + r) * N + 2 * k;
+        const float ib = rinv[r], ic = rinv[R + r];
+        b0 = b0 * ib * (a.nw_B ? a.nw_B[q] : 1.f) + (a.nb_B ? a.nb_B[q] : 0.f);
+        b1 = b1 * ib * (a.nw_B ? a.nw_B[q + 1] : 1.f) + (a.nb_B ? a.nb_B[q + 1] : 0.f);
+        c0 = c0 * ic * (a.nw_C ? a.nw_C[q] : 1.f) + (a.nb_C ? a.nb_C[q] : 0.f);
+        c1 = c1 * ic * (a.nw_C ? a.nw_C[q + 1] : 1.f) + (a.nb_C ? a.nb_C[q + 1] : 0.f);
+      }
       const float rb0 = cs * b0 + sn * b1, rb1 = -sn * b0 + cs * b1;
       sB[r * N + 2 * k] = rb0;
       sB[r * N + 2 * k + 1] = rb1;
@@ -354,10 +378,10 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
   if (tid == 0) ptx::bulk_wait_all();
 }
 
-template <typename T, int N, int R>
-int launch_stream_t(const DecodeArgs& a, cudaStream_t s) {
+template <typename T, int N, int R, bool BCN>
+int launch_stream_k(const DecodeArgs& a, cudaStream_t s) {
   using S = DStage<T, N, R>;
-  auto k = decode_stream_kernel<T, N, R>;
+  auto k = decode_stream_kernel<T, N, R, BCN>;
   static int blocks_per_sm = 0, sms = 0;
   if (blocks_per_sm == 0) {
     int dev = 0;
@@ -384,6 +408,11 @@ int launch_stream_t(const DecodeArgs& a, cudaStream_t s) {
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 
+template <typename T, int N, int R>
+int launch_stream_t(const DecodeArgs& a, cudaStream_t s) {
+  return a.bcnorm ? launch_stream_k<T, N, R, true>(a, s) : launch_stream_k<T, N, R, false>(a, s);
+}
+
 bool stream_ok(const DecodeArgs& a) {
   if (a.P != kSP || (a.N != 64 && a.N != 128) || !(a.R == 1 || a.R == 2 || a.R == 4)) return false;
   const uintptr_t all = reinterpret_cast<uintptr_t>(a.h) | reinterpret_cast<uintptr_t>(a.bprev) |
@@ -408,6 +437,7 @@ int launch_stream(const DecodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 int decode_supported(const DecodeArgs& a) {
+  if (a.bcnorm && !stream_ok(a)) return MAMBA3_ERR_UNSUPPORTED;  // the fused norm lives in the streaming kernel
   if (a.P % 4 != 0 || a.P / 4 > kThreads || kThreads % (a.P / 4) != 0) return MAMBA3_ERR_UNSUPPORTED;
   const int G = kThreads / (a.P / 4);
   if (a.N > kMaxRows * G) return MAMBA3_ERR_UNSUPPORTED;

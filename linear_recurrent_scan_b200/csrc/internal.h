@@ -18,6 +18,10 @@ struct ScanArgs {
   float *h_out, *bprev_out, *xprev_out, *angle_out;  // all null = no export
   void* workspace;  // device status word at offset 0
   size_t workspace_bytes;
+  // fused B/C normalisation (bcnorm != 0): B and C are the raw projections
+  int bcnorm;
+  const float *nw_B, *nw_C, *nb_B, *nb_C;  // [H, R, N], each nullable
+  float neps;
 };
 
 struct DecodeArgs {
@@ -27,6 +31,9 @@ struct DecodeArgs {
   const void *x, *B, *C, *theta, *dt, *lam;
   const float *A, *D;
   void* y;
+  int bcnorm;  // as in ScanArgs
+  const float *nw_B, *nw_C, *nb_B, *nb_C;
+  float neps;
 };
 
 // Each launcher returns MAMBA3_OK, MAMBA3_ERR_UNSUPPORTED (shape not compiled)

@@ -47,6 +47,18 @@ int check_inputs(const void* x, const void* B, const void* C, const void* theta,
   return MAMBA3_OK;
 }
 
+bool norm_ok(const mamba3_bc_norm* n) {
+  if (!n || !(n->eps >= 0.f)) return false;
+  return aligned4(n->w_B) && aligned4(n->w_C) && aligned4(n->bias_B) && aligned4(n->bias_C);
+}
+
+template <typename Args>
+void set_norm(Args& a, const mamba3_bc_norm* n) {
+  a.bcnorm = 1;
+  a.nw_B = n->w_B; a.nw_C = n->w_C; a.nb_B = n->bias_B; a.nb_C = n->bias_C;
+  a.neps = n->eps;
+}
+
 }  // namespace
 
 extern "C" {
@@ -108,6 +120,58 @@ int mamba3_scan_fwd(const mamba3_dims* d, const void* x, const void* B, const vo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
   return use_tc ? m3::launch_scan_tc(a, s) : m3::launch_scan_simt(a, s);
+}
+
+int mamba3_scan_fwd_bcnorm(const mamba3_dims* d, const void* x, const void* B_raw, const void* C_raw,
+                           const void* theta, const void* dt, const void* lam, const float* A, const float* D,
+                           const mamba3_bc_norm* norm, const mamba3_state* init, void* y,
+                           const mamba3_state* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(d, true);
+  if (rc) return rc;
+  if (!norm_ok(norm)) return MAMBA3_ERR_INVALID;
+  if (d->seqlen == 0)  // nothing to normalise: the state passes through
+    return mamba3_scan_fwd(d, x, B_raw, C_raw, theta, dt, lam, A, D, init, y, final_state, workspace,
+                           workspace_bytes, stream);
+  if ((rc = check_inputs(x, B_raw, C_raw, theta, dt, lam, A, D, y))) return rc;
+  if ((rc = check_state(init)) || (rc = check_state(final_state))) return rc;
+  if (!workspace || !aligned16(workspace)) return MAMBA3_ERR_WORKSPACE;
+  if (workspace_bytes < mamba3_scan_workspace_bytes(d)) return MAMBA3_ERR_WORKSPACE;
+  m3::ScanArgs a;
+  memset(&a, 0, sizeof(a));
+  a.batch = d->batch; a.seqlen = d->seqlen; a.nheads = d->nheads; a.P = d->headdim; a.N = d->dstate;
+  a.R = d->rank; a.Q = d->chunk; a.dtype = d->in_dtype;
+  a.x = x; a.B = B_raw; a.C = C_raw; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.D = D;
+  if (init) { a.h0 = init->h; a.bprev0 = init->b_prev; a.xprev0 = init->x_prev; a.angle0 = init->angle; }
+  a.y = y;
+  if (final_state) {
+    a.h_out = final_state->h; a.bprev_out = final_state->b_prev;
+    a.xprev_out = final_state->x_prev; a.angle_out = final_state->angle;
+  }
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
+  set_norm(a, norm);
+  if (m3::tc_scan_supported(a) != MAMBA3_OK) return MAMBA3_ERR_UNSUPPORTED;  // the fused form is tensor-core only
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  return m3::launch_scan_tc(a, s);
+}
+
+int mamba3_decode_step_bcnorm(const mamba3_dims* d, const mamba3_state* state, const void* x, const void* B_raw,
+                              const void* C_raw, const void* theta, const void* dt, const void* lam, const float* A,
+                              const float* D, const mamba3_bc_norm* norm, void* y, void* stream) {
+  int rc = check_dims(d, false);
+  if (rc) return rc;
+  if (!state || !norm_ok(norm)) return MAMBA3_ERR_INVALID;
+  if ((rc = check_state(state))) return rc;
+  if ((rc = check_inputs(x, B_raw, C_raw, theta, dt, lam, A, D, y))) return rc;
+  m3::DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.batch = d->batch; a.nheads = d->nheads; a.P = d->headdim; a.N = d->dstate; a.R = d->rank; a.dtype = d->in_dtype;
+  a.h = state->h; a.bprev = state->b_prev; a.xprev = state->x_prev; a.angle = state->angle;
+  a.x = x; a.B = B_raw; a.C = C_raw; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.D = D; a.y = y;
+  set_norm(a, norm);
+  if ((rc = m3::decode_supported(a))) return rc;
+  return m3::launch_decode(a, static_cast<cudaStream_t>(stream));
 }
 
 int mamba3_decode_step(const mamba3_dims* d, const mamba3_state* state, const void* x, const void* B,

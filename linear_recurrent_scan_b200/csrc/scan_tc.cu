@@ -105,7 +105,9 @@ struct Cfg {
   static constexpr int DL_PAD = (DL_BYTES + 127) & ~127;
   static constexpr int OFF_DL = (OFF_MISC + 16 + 127) & ~127;
   static constexpr int OFF_SINK = OFF_DL + 2 * DL_PAD;  // [Q] floats: consumes the tile reads
-  static constexpr int SMEM = OFF_SINK + Q * 4;
+  // fused B/C normalisation: w_B, bias_B, w_C, bias_C of this head, [R][N] floats each
+  static constexpr int OFF_NRM = (OFF_SINK + Q * 4 + 15) & ~15;
+  static constexpr int SMEM = OFF_NRM + 4 * R * N * 4;
   static constexpr int SMEM_ALLOC = SMEM + 1024;       // slack for 1024-byte alignment
   static_assert(NG * NPART == kNPrep && TPP * NPART == Q, "angle partition");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -160,7 +162,7 @@ __device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 256;" ::
 // place (16 bytes per shared-memory access, 2 rows in flight), the rank-1
 // column factors of the mask and X_w.  dt and lam are prefetched one chunk
 // ahead into registers; theta arrives by TMA.
-template <int N, int R>
+template <int N, int R, bool BCN>
 __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int dl_tma, int b, int hh,
                                           float Ah, uint64_t* bars, volatile int* abort_flag, DeviceStatus* status) {
   using K = Cfg<N, R>;
@@ -208,6 +210,17 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
   const __nv_bfloat16* dts = reinterpret_cast<const __nv_bfloat16*>(smem + K::OFF_DL) + (hh & 7);
   const __nv_bfloat16* lms = reinterpret_cast<const __nv_bfloat16*>(smem + K::OFF_DL + K::DL_PAD) + (hh & 7);
   float* sink = reinterpret_cast<float*>(smem + K::OFF_SINK);
+  const float* nrm = reinterpret_cast<const float*>(smem + K::OFF_NRM);
+  if constexpr (BCN) {  // this head's normalisation weights and biases, [4][R][N]
+    float* nw = reinterpret_cast<float*>(smem + K::OFF_NRM);
+    const size_t base = (size_t)hh * R * N;
+    for (int i = pt; i < R * N; i += kNPrep) {
+      nw[i] = a.nw_B ? a.nw_B[base + i] : 1.f;
+      nw[R * N + i] = a.nb_B ? a.nb_B[base + i] : 0.f;
+      nw[2 * R * N + i] = a.nw_C ? a.nw_C[base + i] : 1.f;
+      nw[3 * R * N + i] = a.nb_C ? a.nb_C[base + i] : 0.f;
+    }
+  }
   prep_sync();
 
   for (int c = 0; c < nchunks; ++c) {
@@ -317,15 +330,56 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
         const uint32_t bw[4] = {bq[j].x, bq[j].y, bq[j].z, bq[j].w};
         const uint32_t cw[4] = {cq[j].x, cq[j].y, cq[j].z, cq[j].w};
         uint32_t bo[4], co[4];
+        if constexpr (BCN) {
+          // raw row (t, r): RMS over N (its NG groups sit in NG consecutive
+          // lanes), weight and bias, then the rotation
+          float bv[8], cv[8], ssb = 0.f, ssc = 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 bv = unpack_bf16(bw[k]), cv = unpack_bf16(cw[k]);
-          const float b0 = cs[jt][k] * bv.x + sn[jt][k] * bv.y, b1 = cs[jt][k] * bv.y - sn[jt][k] * bv.x;
-          bo[k] = pack_bf16(b0, b1);
-          co[k] = pack_bf16(cs[jt][k] * cv.x + sn[jt][k] * cv.y, cs[jt][k] * cv.y - sn[jt][k] * cv.x);
-          if (export_row) {
-            a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k] = b0;
-            a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k + 1] = b1;
+          for (int k = 0; k < 4; ++k) {
+            const float2 b2 = unpack_bf16(bw[k]), c2v = unpack_bf16(cw[k]);
+            bv[2 * k] = b2.x; bv[2 * k + 1] = b2.y;
+            cv[2 * k] = c2v.x; cv[2 * k + 1] = c2v.y;
+            ssb += b2.x * b2.x + b2.y * b2.y;
+            ssc += c2v.x * c2v.x + c2v.y * c2v.y;
+          }
+#pragma unroll
+          for (int o = 1; o < NG; o <<= 1) {
+            ssb += __shfl_xor_sync(0xffffffffu, ssb, o);
+            ssc += __shfl_xor_sync(0xffffffffu, ssc, o);
+          }
+          // an all-zero row with eps = 0 (e.g. the padding past the sequence end)
+          // normalises to 0 instead of 0/0
+          const float vb = ssb * (1.f / N) + a.neps, vc = ssc * (1.f / N) + a.neps;
+          const float ib = vb > 0.f ? rsqrtf(vb) : 0.f, ic = vc > 0.f ? rsqrtf(vc) : 0.f;
+          const float* wB = nrm + r * N + 8 * g;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            bv[e] = bv[e] * ib * wB[e] + wB[R * N + e];
+            cv[e] = cv[e] * ic * wB[2 * R * N + e] + wB[3 * R * N + e];
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float b0 = cs[jt][k] * bv[2 * k] + sn[jt][k] * bv[2 * k + 1];
+            const float b1 = cs[jt][k] * bv[2 * k + 1] - sn[jt][k] * bv[2 * k];
+            bo[k] = pack_bf16(b0, b1);
+            co[k] = pack_bf16(cs[jt][k] * cv[2 * k] + sn[jt][k] * cv[2 * k + 1],
+                              cs[jt][k] * cv[2 * k + 1] - sn[jt][k] * cv[2 * k]);
+            if (export_row) {
+              a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k] = b0;
+              a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k + 1] = b1;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 bv = unpack_bf16(bw[k]), cv = unpack_bf16(cw[k]);
+            const float b0 = cs[jt][k] * bv.x + sn[jt][k] * bv.y, b1 = cs[jt][k] * bv.y - sn[jt][k] * bv.x;
+            bo[k] = pack_bf16(b0, b1);
+            co[k] = pack_bf16(cs[jt][k] * cv.x + sn[jt][k] * cv.y, cs[jt][k] * cv.y - sn[jt][k] * cv.x);
+            if (export_row) {
+              a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k] = b0;
+              a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k + 1] = b1;
+            }
           }
         }
         const uint32_t off = kb * kTile + swz(t * R + r, c8);
@@ -603,7 +657,7 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
   }
 }
 
-template <int N, int R>
+template <int N, int R, bool BCN>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
@@ -780,7 +834,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bars[bDone], 0, abort_flag, status, kTagDrain, 400000000LL);
     }
   } else if (tid < kEpi0) {
-    prep_role<N, R>(smem, a, nchunks, prm.dl_tma, b, hh, a.A[hh], bars, abort_flag, status);
+    prep_role<N, R, BCN>(smem, a, nchunks, prm.dl_tma, b, hh, a.A[hh], bars, abort_flag, status);
   } else {
     epi_role<N, R>(smem, a, nchunks, b, hh, bars, abort_flag, status, tmem);
   }
@@ -870,7 +924,7 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
   memset(&tmD, 0, sizeof(tmD));
   memset(&tmL, 0, sizeof(tmL));
   prm.dl_tma = make_dl_map(&tmD, a.dt, a, K::Q) && make_dl_map(&tmL, a.lam, a, K::Q);
-  auto kern = scan_tc_kernel<N, R>;
+  auto kern = a.bcnorm ? scan_tc_kernel<N, R, true> : scan_tc_kernel<N, R, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
   kern<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmC, tmX, tmT, tmD, tmL, prm);

@@ -148,6 +148,27 @@ def decode_inputs(w: Workload, steps: int, seed: int = BASE_SEED + 1, device="cp
     return {k: v.transpose(0, 1).contiguous() for k, v in d.items()}
 
 
+def raw_bc_inputs(inp: Dict[str, torch.Tensor], seed: int = BASE_SEED + 2) -> Dict[str, torch.Tensor]:
+    """Raw (not yet normalised) B and C projections with the shapes, dtype and
+    device of inp["B"], inp["C"]: N(0, 1) rows times a per-row scale drawn
+    log-uniform in [0.1, 10]; and the B/C norm parameters of the heads, float32
+    [H, R, N]: weights U(0.5, 1.5), biases N(0, 0.1^2)."""
+    B = inp["B"]
+    dev = B.device
+    *lead, H, R, N = B.shape
+    g = _gen(dev, seed)
+    out = {}
+    for name in ("B_raw", "C_raw"):
+        z = torch.randn(B.shape, generator=g, device=dev, dtype=torch.float32)
+        scale = torch.exp(torch.empty(*lead, H, R, 1, device=dev).uniform_(math.log(0.1), math.log(10.0), generator=g))
+        out[name] = (z * scale).to(B.dtype).contiguous()
+    for name in ("w_B", "w_C"):
+        out[name] = torch.empty(H, R, N, device=dev).uniform_(0.5, 1.5, generator=g)
+    for name in ("bias_B", "bias_C"):
+        out[name] = torch.randn(H, R, N, generator=g, device=dev) * 0.1
+    return out
+
+
 def to_f64(d: Dict[str, torch.Tensor]):
     """Widen every tensor to a float64 numpy array (exact for bf16/fp32)."""
     return {k: v.detach().to("cpu", torch.float64).numpy() for k, v in d.items()}

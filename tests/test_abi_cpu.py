@@ -159,3 +159,29 @@ def test_python_binding_validates_shapes(lib):
     A = torch.zeros(2)
     with pytest.raises(ValueError):
         m3.mamba3_scan_fwd(x, B, B, th, dt, dt, A)
+
+
+def scan_bcn(lib, d, norm, ptrs=None):
+    p = dict(x=FAKE, B=FAKE, C=FAKE, theta=FAKE, dt=FAKE, lam=FAKE, A=FAKE, D=None, y=FAKE)
+    p.update(ptrs or {})
+    return lib.mamba3_scan_fwd_bcnorm(ctypes.byref(d), p["x"], p["B"], p["C"], p["theta"], p["dt"], p["lam"],
+                                      p["A"], p["D"], ctypes.byref(norm) if norm is not None else None, None, p["y"],
+                                      None, FAKE, 1 << 20, None)
+
+
+def decode_bcn(lib, d, norm):
+    cs = m3._CState(FAKE, FAKE, FAKE, FAKE)
+    return lib.mamba3_decode_step_bcnorm(ctypes.byref(d), ctypes.byref(cs), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                         FAKE, None, ctypes.byref(norm) if norm is not None else None, FAKE, None)
+
+
+def test_bcnorm_entry_points_validate_on_host(lib):
+    ok = m3._CNorm(None, None, None, None, 1e-6)
+    assert scan_bcn(lib, dims(), None) == m3.MAMBA3_ERR_INVALID                         # norm is required
+    assert scan_bcn(lib, dims(), m3._CNorm(None, None, None, None, -1.0)) == m3.MAMBA3_ERR_INVALID
+    assert scan_bcn(lib, dims(), m3._CNorm(FAKE + 2, None, None, None, 1e-6)) == m3.MAMBA3_ERR_INVALID
+    assert scan_bcn(lib, dims(), ok, {"B": None}) == m3.MAMBA3_ERR_INVALID
+    # the fused form runs on the tensor-core path only (bf16, P = 64, N in {64, 128})
+    assert scan_bcn(lib, dims(in_dtype=m3.MAMBA3_F32), ok) == m3.MAMBA3_ERR_UNSUPPORTED
+    assert decode_bcn(lib, dims(), None) == m3.MAMBA3_ERR_INVALID
+    assert decode_bcn(lib, dims(headdim=32), ok) == m3.MAMBA3_ERR_UNSUPPORTED            # streaming kernel: P = 64
