@@ -43,13 +43,13 @@ FALLBACK_HBM_GBS = 6650.0
 # traffic null, since its counters are out of date.
 TRAFFIC = {
     "prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"),
-                "cab7ade096cf20b585c2edafd11f8c802cbee49440e69063f1f9c8ac5a5e7de7", 811488256 + 136867584,
+                "659087eb7f4d6efea1eb120319c5416d33015294b3cb0218d382ba67740923a4", 811429120 + 136969984,
                 "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     "siso_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                         "ac70b819247a216ebf772caf5eae8b70b922c205d4f263759cc72849df1f75dd", 283208192 + 218755840,
+                         "923a0a98013ff1e6d7f8375e370d839f543d8639e3709532d541eff2459467d6", 283177472 + 219342848,
                          "profiles/decode_stream_b128_traffic_and_counters.txt"),
     "mimo4_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                          "ac70b819247a216ebf772caf5eae8b70b922c205d4f263759cc72849df1f75dd", 317780736 + 239914496,
+                          "923a0a98013ff1e6d7f8375e370d839f543d8639e3709532d541eff2459467d6", 317801728 + 240049920,
                           "profiles/decode_stream_b128_traffic_and_counters.txt"),
 }
 
@@ -276,24 +276,38 @@ def run_prefill(m3, args, world, rank, clk):
                 tokens=w.batch * w.seqlen, bytes=prefill_bytes(w))
 
 
-def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup):
+def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False):
     """Median per-launch time (ms) of one prefill launch of workload `w`, inputs
-    resident on the device (larger than L2), final state exported."""
+    resident on the device (larger than L2), final state exported.  With
+    fused_norm the launch takes raw B, C and normalises them in the kernel."""
     dev = torch.device("cuda")
     inp = wl.make_inputs(w, seed=wl.BASE_SEED + rank, device=dev)
+    norm = None
+    if fused_norm:
+        raw = wl.raw_bc_inputs(inp, seed=wl.BASE_SEED + 2 + rank)
+        inp["B"], inp["C"] = raw["B_raw"], raw["C_raw"]
+        norm = m3.BCNorm(raw["w_B"], raw["w_C"], raw["bias_B"], raw["bias_C"], 1e-6)
     ins = [inp[n] for n in NAMES]
     y = torch.empty_like(inp["x"])
     fin = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
     dims = m3.make_dims(inp["x"], inp["B"])
     ws = torch.zeros(max(256, m3.mamba3_scan_workspace_bytes(dims)), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+
+    def launch():
+        if fused_norm:
+            m3.mamba3_scan_fwd_bcnorm(*ins, inp["A"], inp["D"], norm=norm, y=y, final_state=fin, workspace=ws,
+                                      stream=stream)
+        else:
+            m3.mamba3_scan_fwd(*ins, inp["A"], inp["D"], y=y, final_state=fin, workspace=ws, stream=stream)
+
     for _ in range(warmup):
-        m3.mamba3_scan_fwd(*ins, inp["A"], inp["D"], y=y, final_state=fin, workspace=ws, stream=stream)
+        launch()
     times = []
     for _ in range(steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        m3.mamba3_scan_fwd(*ins, inp["A"], inp["D"], y=y, final_state=fin, workspace=ws, stream=stream)
+        launch()
         e1.record(stream)
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1))
@@ -305,9 +319,10 @@ def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup):
     return statistics.median(times)
 
 
-def run_decode(m3, w: wl.Workload, world, rank, steps):
+def run_decode(m3, w: wl.Workload, world, rank, steps, fused_norm=False):
     """Seed the state with a 512-token prefill, then time `steps` decode steps
-    captured in one CUDA graph (per-step inputs pre-generated, larger than L2)."""
+    captured in one CUDA graph (per-step inputs pre-generated, larger than L2).
+    With fused_norm each step takes raw B, C and normalises them in the kernel."""
     dev = torch.device("cuda")
     pre = wl.make_inputs(w.with_(seqlen=w.prefill_tokens), seed=wl.BASE_SEED + rank, device=dev)
     st = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
@@ -315,17 +330,27 @@ def run_decode(m3, w: wl.Workload, world, rank, steps):
     A, D = pre["A"], pre["D"]
     del pre
     steps_in = wl.decode_inputs(w, steps, seed=wl.BASE_SEED + 1 + rank, device=dev)
+    norm = None
+    if fused_norm:
+        raw = wl.raw_bc_inputs(steps_in, seed=wl.BASE_SEED + 3 + rank)
+        steps_in["B"], steps_in["C"] = raw["B_raw"], raw["C_raw"]
+        norm = m3.BCNorm(raw["w_B"], raw["w_C"], raw["bias_B"], raw["bias_C"], 1e-6)
+    step_fn = ((lambda st_, i_, y_: m3.mamba3_decode_step_bcnorm(st_, *(steps_in[n][i_] for n in NAMES), A, D,
+                                                                 norm=norm, y=y_, stream=s))
+               if fused_norm else
+               (lambda st_, i_, y_: m3.mamba3_decode_step(st_, *(steps_in[n][i_] for n in NAMES), A, D, y=y_,
+                                                          stream=s)))
     ys = torch.empty((steps,) + steps_in["x"].shape[1:], dtype=w.dtype, device=dev)
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     saved = st.clone()
     with torch.cuda.stream(s):
         for i in range(3):  # warm-up outside the graph
-            m3.mamba3_decode_step(st, *(steps_in[n][i] for n in NAMES), A, D, y=ys[i], stream=s)
+            step_fn(st, i, ys[i])
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
             for i in range(steps):
-                m3.mamba3_decode_step(st, *(steps_in[n][i] for n in NAMES), A, D, y=ys[i], stream=s)
+                step_fn(st, i, ys[i])
     torch.cuda.synchronize()
     times = []
     for rep in range(3):
@@ -369,6 +394,18 @@ def ours(args):
                                    "rank": DECODE_LONG.rank, "dstate": DECODE_LONG.dstate,
                                    "state_from_prefill_tokens": DECODE_LONG.prefill_tokens,
                                    "roofline": None, "note": "latency-bound: %d bytes per step" % decode_bytes(DECODE_LONG)}
+    # the fused B/C norm variant of the headline prefill and of the SISO decode step
+    ms = max_over_ranks(run_prefill_plain(m3, PREFILL, rank, steps=max(5, min(args.steps, 20)), warmup=3,
+                                          fused_norm=True), world)
+    gbs = prefill_bytes(PREFILL) / (ms * 1e-3) / 1e9
+    fused = {"prefill_" + PREFILL.name: {"ms_per_launch": round(ms, 4), "roofline": {
+        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
+        "bytes_per_launch": prefill_bytes(PREFILL)}}}
+    us = run_decode(m3, DECODE[0], world, rank, DECODE[0].decode_steps, fused_norm=True)
+    gbs = decode_bytes(DECODE[0]) / (us * 1e-6) / 1e9
+    fused["decode_" + DECODE[0].name] = {"us_per_step": round(us, 2), "roofline": {
+        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
+        "bytes_per_step": decode_bytes(DECODE[0])}}
     more = {}
     for w in PREFILL_MORE:
         ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=max(5, min(args.steps, 20)), warmup=3), world)
@@ -403,6 +440,7 @@ def ours(args):
                      "frac": round(achieved / peak, 4), "traffic": traffic("prefill"), "peak_kind": peak_kind,
                      "bytes_per_launch": r["bytes"], "launch_ms": round(r["launch_ms"], 4)},
         "prefill_more": more,
+        "fused_bc_norm": fused,
         "decode": dec,
         "e2e": {"value": round(e2e_value, 3), "unit": "Mtokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
