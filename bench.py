@@ -46,10 +46,10 @@ TRAFFIC = {
                 "659087eb7f4d6efea1eb120319c5416d33015294b3cb0218d382ba67740923a4", 811429120 + 136969984,
                 "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     "siso_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                         "923a0a98013ff1e6d7f8375e370d839f543d8639e3709532d541eff2459467d6", 283177472 + 219342848,
+                         "80cdf686cd24e1026aee9bce7e53a1796ca03d6a41fbc32c95d37ddc31e190e4", 283177472 + 219342848,
                          "profiles/decode_stream_b128_traffic_and_counters.txt"),
     "mimo4_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                          "923a0a98013ff1e6d7f8375e370d839f543d8639e3709532d541eff2459467d6", 317801728 + 240049920,
+                          "80cdf686cd24e1026aee9bce7e53a1796ca03d6a41fbc32c95d37ddc31e190e4", 317801728 + 240049920,
                           "profiles/decode_stream_b128_traffic_and_counters.txt"),
 }
 

@@ -11,7 +11,13 @@
 // ops per byte for standard SSM decoding), so the kernel is organised around
 // streaming the N x P fp32 state exactly once with 16-byte loads and stores.
 //
-// Work split: one CTA of 128 threads per (b, h).  A thread owns four
+// Two kernels.  decode_stream_kernel (second half of this file) is the main
+// path for P = 64, N in {64, 128}, R in {1, 2, 4}: persistent CTAs stream the
+// (b, h) units through a 2-stage shared-memory ring filled and drained by bulk
+// copies, and can fuse the B/C RMS norm.  decode_kernel below covers every
+// other supported shape (and unaligned pointers).
+//
+// decode_kernel work split: one CTA of 128 threads per (b, h).  A thread owns four
 // consecutive columns p..p+3 of h and the rows n = ty, ty + G, ... (G = 128 /
 // (P/4) row groups); it issues all of its state loads before any arithmetic
 // so that up to 16 independent 16-byte loads are in flight per thread.  The
