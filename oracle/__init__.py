@@ -58,6 +58,7 @@ class _IO(ctypes.Structure):
             "x", "B", "C", "theta", "dt", "lam", "A", "D",
             "h0", "bprev0", "xprev0", "angle0",
             "y", "h_out", "bprev_out", "xprev_out", "angle_out",
+            "A_t",
         )
     ]
 
@@ -123,7 +124,8 @@ def _prepare(x, B, C, theta, dt, lam, A, D):
     N = B.shape[-1]
     assert B.shape == (b, L, H, R, N) and C.shape == B.shape, "B/C must be [b,L,H,R,N]"
     assert theta.shape == (b, L, H, N // 2), "theta must be [b,L,H,N/2]"
-    assert dt.shape == (b, L, H) and lam.shape == (b, L, H) and A.shape == (H,)
+    assert dt.shape == (b, L, H) and lam.shape == (b, L, H)
+    assert A.shape == (H,) or A.shape == (b, L, H), "A must be [H] (per head) or [b,L,H] (per token)"
     dims = _Dims(b, L, H, P, N, R)
     return dims, (x, B, C, theta, dt, lam, A, D)
 
@@ -137,9 +139,13 @@ def _run(fn_name, x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = No
     N = B.shape[-1]
     y = np.zeros_like(x)
     fin = State.zeros(b, H, P, N, R) if want_state else None
-    keep = [x, B, C, theta, dt, lam, A, D, y]
+    A_t = None
+    if A.ndim == 3:  # time-varying decay: A_t [b, L, H] replaces the per-head A
+        A_t, A = A, np.zeros(H)
+    keep = [x, B, C, theta, dt, lam, A, A_t, D, y]
     io = _IO()
     io.x, io.B, io.C, io.theta, io.dt, io.lam, io.A, io.D = map(_ptr, (x, B, C, theta, dt, lam, A, D))
+    io.A_t = _ptr(A_t)
     if init is not None:
         ih, ib, ix, ia = (_f64(init.h), _f64(init.b_prev), _f64(init.x_prev), _f64(init.angle))
         keep += [ih, ib, ix, ia]
@@ -166,6 +172,7 @@ def _run(fn_name, x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = No
 
 def scan_complex(x, B, C, theta, dt, lam, A, D=None, init=None, nthreads=None, units=None):
     """The definition: explicit complex-diagonal state, sequential in t.
+    A is [H] (one decay rate per head) or [b, L, H] (time-varying, one per token).
 
     Returns (y [b,L,H,R,P], final State).  ``units`` optionally restricts the
     work to a list of flattened (b*H + h) indices (others stay zero).
@@ -188,15 +195,17 @@ def decode_step(state: State, x, B, C, theta, dt, lam, A, D=None, nthreads=None)
     """One token continued from ``state``.
 
     Per-token inputs are shaped without the L axis: x [b,H,R,P], B/C [b,H,R,N],
-    theta [b,H,N/2], dt/lam [b,H].  Returns (y [b,H,R,P], new State).
+    theta [b,H,N/2], dt/lam [b,H]; A is [H] or, time-varying, [b,H].
+    Returns (y [b,H,R,P], new State).
     """
     add = lambda a: _f64(a)[:, None]
-    y, fin = _run("m3o_decode_step", add(x), add(B), add(C), add(theta), add(dt), add(lam), A, D,
-                  state, True, nthreads)
+    A = _f64(A)
+    y, fin = _run("m3o_decode_step", add(x), add(B), add(C), add(theta), add(dt), add(lam),
+                  add(A) if A.ndim == 2 else A, D, state, True, nthreads)
     return y[:, 0], fin
 
 
-__all__ = ["build", "State", "scan_complex", "scan_rope", "scan_quadratic", "decode_step"]
+__all__ = ["build", "State", "scan_complex", "scan_rope", "scan_quadratic", "decode_step", "bc_norm"]
 
 
 def bc_norm(z, w=None, bias=None, eps: float = 1e-6) -> np.ndarray:

@@ -58,7 +58,12 @@ typedef struct {
   const double *h0, *bprev0, *xprev0, *angle0;          /* all NULL = zero state */
   double *y;                                            /* may be NULL */
   double *h_out, *bprev_out, *xprev_out, *angle_out;    /* all NULL = no export */
+  const double* A_t; /* NULL, or a time-varying decay [b, L, H] that replaces A[h] token by token */
 } m3o_io;
+
+/* The decay rate of token t: A_t[b, t, h] when given (section 1.1 writes the
+ * discretisation with a per-step A_t), else the per-head A[h]. */
+static double decay_rate(const m3o_io* io, size_t it, int h) { return io->A_t ? io->A_t[it] : io->A[h]; }
 
 /* ------------------------------------------------------------------------- */
 /* index helpers                                                               */
@@ -75,7 +80,6 @@ static size_t ix_state(const m3o_dims* d, int b, int h) {
 /* ------------------------------------------------------------------------- */
 static void unit_complex(const m3o_dims* d, const m3o_io* io, int b, int h) {
   const int L = d->seqlen, P = d->headdim, N = d->dstate, R = d->rank, K = N / 2;
-  const double A = io->A[h];
   const double Dh = io->D ? io->D[h] : 0.0;
   double complex* Hs = calloc((size_t)K * P, sizeof(double complex));  /* state H */
   double complex* u_prev = calloc((size_t)K * P, sizeof(double complex));
@@ -111,8 +115,9 @@ static void unit_complex(const m3o_dims* d, const m3o_io* io, int b, int h) {
     const double* Bt = io->B + it * R * N;
     const double* Ct = io->C + it * R * N;
     const double* th = io->theta + it * K;
+    const double At = decay_rate(io, it, h);
     for (int k = 0; k < K; ++k) {
-      a[k] = cexp(dt * (A + I * th[k]));
+      a[k] = cexp(dt * (At + I * th[k]));
       Phi[k] += dt * th[k];
     }
     /* u_t = sum_r b_{t,r} x_{t,r}^T with b complexified by adjacent pairs */
@@ -185,7 +190,6 @@ static void rot_neg(double phi, double v0, double v1, double* o0, double* o1) {
 
 static void unit_rope(const m3o_dims* d, const m3o_io* io, int b, int h) {
   const int L = d->seqlen, P = d->headdim, N = d->dstate, R = d->rank, K = N / 2;
-  const double A = io->A[h];
   const double Dh = io->D ? io->D[h] : 0.0;
   double* hs = calloc((size_t)N * P, sizeof(double));
   double* u_prev = calloc((size_t)N * P, sizeof(double));
@@ -218,7 +222,7 @@ static void unit_rope(const m3o_dims* d, const m3o_io* io, int b, int h) {
         rot_neg(Phi[k], Bt[2 * k], Bt[2 * k + 1], &Br[r * N + 2 * k], &Br[r * N + 2 * k + 1]);
         rot_neg(Phi[k], Ct[2 * k], Ct[2 * k + 1], &Cr[r * N + 2 * k], &Cr[r * N + 2 * k + 1]);
       }
-    const double alpha = exp(dt * A);
+    const double alpha = exp(dt * decay_rate(io, it, h));
     const double beta = (1.0 - lam) * dt * alpha;
     const double gamma = lam * dt;
     for (int n = 0; n < N; ++n)
@@ -266,7 +270,6 @@ static void unit_rope(const m3o_dims* d, const m3o_io* io, int b, int h) {
  */
 static void unit_quadratic(const m3o_dims* d, const m3o_io* io, int b, int h) {
   const int L = d->seqlen, P = d->headdim, N = d->dstate, R = d->rank, K = N / 2;
-  const double A = io->A[h];
   const double Dh = io->D ? io->D[h] : 0.0;
   const size_t us = ix_state(d, b, h);
   double* Br = calloc((size_t)L * R * N + 1, sizeof(double));
@@ -289,7 +292,7 @@ static void unit_quadratic(const m3o_dims* d, const m3o_io* io, int b, int h) {
         rot_neg(Phi[k], Bt[2 * k], Bt[2 * k + 1], &Br[(t * R + r) * N + 2 * k], &Br[(t * R + r) * N + 2 * k + 1]);
         rot_neg(Phi[k], Ct[2 * k], Ct[2 * k + 1], &Cr[(t * R + r) * N + 2 * k], &Cr[(t * R + r) * N + 2 * k + 1]);
       }
-    c += io->dt[it] * A;
+    c += io->dt[it] * decay_rate(io, it, h);
     cum[t] = c;
   }
   for (int t = 0; t < L; ++t)

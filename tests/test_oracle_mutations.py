@@ -20,12 +20,13 @@ MUTATIONS = {
     "drop_lag_term": ("(1.0 - lam) * dt * a[k] * u_prev[k * P + p]", "0.0 * u_prev[k * P + p]"),
     "lag_without_pole": ("(1.0 - lam) * dt * a[k] * u_prev[k * P + p]", "(1.0 - lam) * dt * u_prev[k * P + p]"),
     "lag_weight_lam": ("(1.0 - lam) * dt * a[k] * u_prev[k * P + p]", "lam * dt * a[k] * u_prev[k * P + p]"),
-    "rotation_sign": ("cexp(dt * (A + I * th[k]))", "cexp(dt * (A - I * th[k]))"),
+    "rotation_sign": ("cexp(dt * (At + I * th[k]))", "cexp(dt * (At - I * th[k]))"),
     "readout_no_conj": ("creal(conj(c) * Hs[k * P + p])", "creal(c * Hs[k * P + p])"),
     "pair_swap": ("(Bt[r * N + 2 * k] + I * Bt[r * N + 2 * k + 1])", "(Bt[r * N + 2 * k + 1] + I * Bt[r * N + 2 * k])"),
     "rope_sign": ("*o1 = -sin(phi) * v0 + cos(phi) * v1;", "*o1 = sin(phi) * v0 + cos(phi) * v1;"),
     "quadratic_weight_next": ("(1.0 - io->lam[in]) * io->dt[in]", "(1.0 - io->lam[is]) * io->dt[is]"),
     "mimo_rank_drop": ("for (int r = 0; r < R; ++r)\n          s += (Bt", "for (int r = 0; r < 1; ++r)\n          s += (Bt"),
+    "decay_ignores_A_t": ("return io->A_t ? io->A_t[it] : io->A[h];", "return io->A[h];"),
     "bcnorm_sum_not_mean": ("    ms /= N;\n", "\n"),
     "bcnorm_eps_outside_sqrt": ("1.0 / sqrt(ms + eps)", "1.0 / (sqrt(ms) + eps)"),
     "bcnorm_bias_index_swapped": ("const size_t p = ((size_t)h * R + r) * N + n;", "const size_t p = ((size_t)r * H + h) * N + n;"),
@@ -41,6 +42,8 @@ PIN_FUNCS = [
     lambda: [pins.test_complex_equals_rope(r) for r in (1, 3)],
     lambda: [pins.test_quadratic_equals_recurrence(r) for r in (1, 2)],
     pins.test_mimo_is_superposition_of_siso,
+    lambda: [pins.test_time_varying_decay_impulse_closed_form(f) for f in ("scan_complex", "scan_rope",
+                                                                           "scan_quadratic")],
     pins.test_bc_norm_constant_row_closed_form,
     pins.test_bc_norm_unit_rms_per_row,
     pins.test_bc_norm_scale_invariant_and_odd,

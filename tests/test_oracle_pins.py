@@ -431,3 +431,75 @@ def test_bc_norm_zero_row_gives_bias():
     bias = np.arange(H * R * N, dtype=np.float64).reshape(H, R, N)
     out = oracle.bc_norm(z, None, bias, eps=0.0)
     assert np.array_equal(out[0, 0], bias)
+
+
+# ---------------------------------------------------------------- time-varying decay A_t
+# "Mamba-3: 2x smaller state ..." (MarkTechPost, Korean translation), section 1.1
+# writes the discretisation with a per-step A_t: each step's pole is exp(dt_t A_t).
+
+@pytest.mark.parametrize("fn", ["scan_complex", "scan_rope", "scan_quadratic"])
+def test_time_varying_decay_impulse_closed_form(fn):
+    """Single impulse at t0 with a per-token A_t: the pole product runs over the
+    per-token rates, H_t = prod_{q=t0+1..t} exp(dt_q (A_q + i theta_q)) * w_hat * u."""
+    rng = np.random.default_rng(111)
+    L, N, P, R, t0 = 15, 6, 3, 2, 4
+    inp = rand_inputs(1, L, 1, P, N, R, rng)
+    inp["x"][:] = 0
+    inp["x"][0, t0] = rng.standard_normal((1, R, P))
+    inp["D"][:] = 0.0
+    At = -rng.uniform(0.1, 3.0, (1, L, 1))
+    inp["A"] = At
+    y = getattr(oracle, fn)(**inp)
+    y = y[0] if isinstance(y, tuple) else y
+    dt, lam, th = inp["dt"][0, :, 0], inp["lam"][0, :, 0], inp["theta"][0, :, 0]
+    a_t = At[0, :, 0]
+    Bc = inp["B"][0, :, 0, :, 0::2] + 1j * inp["B"][0, :, 0, :, 1::2]
+    Cc = inp["C"][0, :, 0, :, 0::2] + 1j * inp["C"][0, :, 0, :, 1::2]
+    u = np.einsum("rk,rp->kp", Bc[t0], inp["x"][0, t0, 0])
+    ref = np.zeros((L, R, P))
+    w_hat = lam[t0] * dt[t0] + (1 - lam[t0 + 1]) * dt[t0 + 1]
+    for t in range(t0, L):
+        if t == t0:
+            Ht = lam[t0] * dt[t0] * u
+        else:
+            logp = np.sum(dt[t0 + 1:t + 1, None] * (a_t[t0 + 1:t + 1, None] + 1j * th[t0 + 1:t + 1]), axis=0)
+            Ht = np.exp(logp)[:, None] * w_hat * u
+        ref[t] = np.real(np.einsum("rk,kp->rp", np.conj(Cc[t]), Ht))
+    assert rel_err(y[0, :, 0], ref) < 1e-12
+
+
+def test_time_varying_decay_constant_in_time_is_per_head():
+    """A_t[b, t, h] = A[h] for every token reproduces the per-head recurrence."""
+    rng = np.random.default_rng(112)
+    inp = rand_inputs(2, 19, 3, 4, 6, 2, rng)
+    y, f = oracle.scan_complex(**inp)
+    tv = dict(inp, A=np.broadcast_to(inp["A"], inp["dt"].shape).copy())
+    y2, f2 = oracle.scan_complex(**tv)
+    assert rel_err(y2, y) < 1e-14 and rel_err(f2.h, f.h) < 1e-14
+
+
+@pytest.mark.parametrize("R", [1, 3])
+def test_time_varying_decay_forms_agree(R):
+    """Complex == RoPE == quadratic with a per-token decay (the chunk algebra of the
+    quadratic form multiplies per-token poles)."""
+    rng = np.random.default_rng(113 + R)
+    inp = rand_inputs(1, 21, 2, 3, 6, R, rng)
+    inp["A"] = -rng.uniform(0.05, 2.5, inp["dt"].shape)
+    yc, _ = oracle.scan_complex(**inp)
+    yr, _ = oracle.scan_rope(**inp)
+    yq = oracle.scan_quadratic(**inp)
+    assert rel_err(yr, yc) < 1e-12 and rel_err(yq, yc) < 1e-12
+
+
+def test_time_varying_decay_prefill_then_decode():
+    rng = np.random.default_rng(114)
+    b, L, H, P, N, R, k = 2, 12, 2, 3, 4, 2, 8
+    inp = rand_inputs(b, L, H, P, N, R, rng)
+    inp["A"] = -rng.uniform(0.05, 2.5, (b, L, H))
+    y_all, f_all = oracle.scan_complex(**inp)
+    _, st = oracle.scan_complex(**slice_t(inp, 0, k))
+    for t in range(k, L):
+        step = {n: inp[n][:, t] for n in ("x", "B", "C", "theta", "dt", "lam", "A")}
+        yt, st = oracle.decode_step(st, **step, D=inp["D"])
+        assert rel_err(yt, y_all[:, t]) < 1e-12
+    assert rel_err(st.h, f_all.h) < 1e-12
