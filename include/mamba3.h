@@ -163,6 +163,24 @@ MAMBA3_API int mamba3_decode_step_bcnorm(const mamba3_dims* dims, const mamba3_s
                                          const void* lam, const float* A, const float* D,
                                          const mamba3_bc_norm* norm, void* y, void* stream);
 
+/*
+ * Time-varying decay ("Mamba-3: 2x smaller state ..." (MarkTechPost, Korean
+ * translation), section 1.1 writes the discretisation with a per-step A_t):
+ * mamba3_scan_fwd / mamba3_decode_step with the per-head A replaced by a rate
+ * per token and head, A_t, so that alpha_t = exp(dt_t A_t) and
+ * beta_t = (1 - lam_t) dt_t alpha_t.  A_t has the dtype of x and the layout of
+ * dt: [b, L, H] for the prefill, [b, H] for the decode step; not nullable.
+ * Every other argument, layout and result is that of the plain entry point.
+ */
+MAMBA3_API int mamba3_scan_fwd_at(const mamba3_dims* dims, const void* x, const void* B, const void* C,
+                                  const void* theta, const void* dt, const void* lam, const void* A_t,
+                                  const float* D, const mamba3_state* init, void* y,
+                                  const mamba3_state* final_state, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+MAMBA3_API int mamba3_decode_step_at(const mamba3_dims* dims, const mamba3_state* state, const void* x,
+                                     const void* B, const void* C, const void* theta, const void* dt,
+                                     const void* lam, const void* A_t, const float* D, void* y, void* stream);
+
 /* Synchronises `stream`, then returns the device status word that the last
  * mamba3_scan_fwd on `workspace` left (MAMBA3_OK or MAMBA3_ERR_TIMEOUT), or
  * MAMBA3_ERR_CUDA / MAMBA3_ERR_INVALID. */

@@ -11,6 +11,7 @@ Entry points (same names as the C ABI):
   mamba3_scan_fwd(x, B, C, theta, dt, lam, A, D=None, init=None, ...)
   mamba3_decode_step(state, x, B, C, theta, dt, lam, A, D=None, ...)
   mamba3_scan_fwd_bcnorm / mamba3_decode_step_bcnorm (raw B, C + BCNorm)
+  mamba3_scan_fwd_at / mamba3_decode_step_at (time-varying decay A_t)
   mamba3_device_status(workspace)
   mamba3_status_string(code)
 """
@@ -94,6 +95,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba3_decode_step_bcnorm.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(_CState), vp, vp, vp, vp, vp, vp,
                                               vp, vp, ctypes.POINTER(_CNorm), vp, vp]
     lib.mamba3_decode_step_bcnorm.restype = i
+    lib.mamba3_scan_fwd_at.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, vp, vp, vp, vp,
+                                       ctypes.POINTER(_CState), vp, ctypes.POINTER(_CState), vp, sz, vp]
+    lib.mamba3_scan_fwd_at.restype = i
+    lib.mamba3_decode_step_at.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(_CState), vp, vp, vp, vp, vp, vp,
+                                          vp, vp, vp, vp]
+    lib.mamba3_decode_step_at.restype = i
     _lib = lib
     return lib
 
@@ -303,6 +310,50 @@ def mamba3_decode_step_bcnorm(state: State, x, B_raw, C_raw, theta, dt, lam, A, 
     return y
 
 
+def _check_at(A_t, dt, x):
+    if A_t.shape != dt.shape or A_t.dtype != x.dtype or not A_t.is_contiguous() or A_t.device != x.device:
+        raise ValueError("A_t must be a contiguous tensor shaped like dt, with the dtype and device of x")
+
+
+def mamba3_scan_fwd_at(x, B, C, theta, dt, lam, A_t, D=None, init: Optional[State] = None,
+                       y: Optional[torch.Tensor] = None, final_state: Optional[State] = None,
+                       workspace: Optional[torch.Tensor] = None, chunk: int = 0, stream=None):
+    """mamba3_scan_fwd with a time-varying decay A_t [b, L, H] (dtype of x) in
+    place of the per-head A."""
+    lib = load_library()
+    _check_inputs(x, B, C, theta, dt, lam, None, D, decode=False)
+    _check_at(A_t, dt, x)
+    dims = make_dims(x, B, chunk)
+    if y is None:
+        y = torch.empty_like(x)
+    if workspace is None:
+        workspace = torch.empty(mamba3_scan_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
+    ci = init._c() if init is not None else None
+    cf = final_state._c() if final_state is not None else None
+    rc = lib.mamba3_scan_fwd_at(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam),
+                                _ptr(A_t), _ptr(D), ctypes.byref(ci) if ci is not None else None, _ptr(y),
+                                ctypes.byref(cf) if cf is not None else None, _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mamba3_scan_fwd_at")
+    return y
+
+
+def mamba3_decode_step_at(state: State, x, B, C, theta, dt, lam, A_t, D=None, y: Optional[torch.Tensor] = None,
+                          stream=None):
+    """mamba3_decode_step with the token's decay rate A_t [b, H] (dtype of x)."""
+    lib = load_library()
+    _check_inputs(x, B, C, theta, dt, lam, None, D, decode=True)
+    _check_at(A_t, dt, x)
+    dims = make_dims(x, B, decode=True)
+    if y is None:
+        y = torch.empty_like(x)
+    cs = state._c()
+    rc = lib.mamba3_decode_step_at(ctypes.byref(dims), ctypes.byref(cs), _ptr(x), _ptr(B), _ptr(C), _ptr(theta),
+                                   _ptr(dt), _ptr(lam), _ptr(A_t), _ptr(D), _ptr(y), _stream(stream))
+    _check(rc, "mamba3_decode_step_at")
+    return y
+
+
 def mamba3_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(load_library().mamba3_device_status(_ptr(workspace), _stream(stream)))
 
@@ -310,7 +361,7 @@ def mamba3_device_status(workspace: torch.Tensor, stream=None) -> int:
 __all__ = [
     "Dims", "State", "BCNorm", "Mamba3Error", "load_library", "make_dims",
     "mamba3_scan_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc", "mamba3_decode_step",
-    "mamba3_scan_fwd_bcnorm", "mamba3_decode_step_bcnorm",
+    "mamba3_scan_fwd_bcnorm", "mamba3_decode_step_bcnorm", "mamba3_scan_fwd_at", "mamba3_decode_step_at",
     "mamba3_device_status",
     "mamba3_status_string",
 ]

@@ -71,7 +71,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
   const float dt = ld1(static_cast<const T*>(a.dt) + unit);
   if (tid == 0) {
     const float lam = ld1(static_cast<const T*>(a.lam) + unit);
-    const float alpha = expf(dt * a.A[h_idx]);
+    const float rate = a.A_t ? ld1(static_cast<const T*>(a.A_t) + unit) : a.A[h_idx];  // A_t [b, H] or A [H]
+    const float alpha = expf(dt * rate);
     sCoef[0] = alpha;
     sCoef[1] = (1.f - lam) * dt * alpha;
     sCoef[2] = lam * dt;
@@ -269,7 +270,8 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
     const int hh = u % a.nheads;
     const float dt = ld1(static_cast<const T*>(a.dt) + u);
     const float lam = ld1(static_cast<const T*>(a.lam) + u);
-    const float alpha = expf(dt * a.A[hh]);
+    const float rate = a.A_t ? ld1(static_cast<const T*>(a.A_t) + u) : a.A[hh];  // A_t [b, H] or A [H]
+    const float alpha = expf(dt * rate);
     const float beta = (1.f - lam) * dt * alpha, gamma = lam * dt;
     const float Dh = a.D ? a.D[hh] : 0.f;
     ptx::mbar_wait(&bars[s], (it >> 1) & 1, abort_flag, nullptr, 0);

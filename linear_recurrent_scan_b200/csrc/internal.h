@@ -12,7 +12,8 @@ struct ScanArgs {
   int batch, seqlen, nheads, P, N, R, Q;
   mamba3_dtype dtype;
   const void *x, *B, *C, *theta, *dt, *lam;
-  const float *A, *D;
+  const float *A, *D;  // A null when A_t is given
+  const void* A_t;     // time-varying decay [b, L, H] (dtype of x), or null: A[h] per head
   const float *h0, *bprev0, *xprev0, *angle0;  // all null = zero state
   void* y;
   float *h_out, *bprev_out, *xprev_out, *angle_out;  // all null = no export
@@ -29,7 +30,8 @@ struct DecodeArgs {
   mamba3_dtype dtype;
   float *h, *bprev, *xprev, *angle;
   const void *x, *B, *C, *theta, *dt, *lam;
-  const float *A, *D;
+  const float *A, *D;  // A null when A_t is given
+  const void* A_t;     // time-varying decay of the token [b, H] (dtype of x), or null
   void* y;
   int bcnorm;  // as in ScanArgs
   const float *nw_B, *nw_C, *nb_B, *nb_C;

@@ -82,14 +82,20 @@ size_t mamba3_scan_workspace_bytes(const mamba3_dims* d) {
   return kStatusBytes;
 }
 
-int mamba3_scan_fwd(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
-                    const void* dt, const void* lam, const float* A, const float* D,
-                    const mamba3_state* init, void* y, const mamba3_state* final_state, void* workspace,
-                    size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// The prefill behind mamba3_scan_fwd (A per head) and mamba3_scan_fwd_at (A_t
+// per token; A null).
+int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                  const void* dt, const void* lam, const float* A, const void* A_t, const float* D,
+                  const mamba3_state* init, void* y, const mamba3_state* final_state, void* workspace,
+                  size_t workspace_bytes, void* stream) {
   int rc = check_dims(d, true);
   if (rc) return rc;
-  if (d->seqlen > 0 && (rc = check_inputs(x, B, C, theta, dt, lam, A, D, y))) return rc;
-  if (d->seqlen == 0 && !A) return MAMBA3_ERR_INVALID;
+  const float* A_chk = A ? A : static_cast<const float*>(A_t);  // the rate array that must be present
+  if (d->seqlen > 0 && (rc = check_inputs(x, B, C, theta, dt, lam, A_chk, D, y))) return rc;
+  if (d->seqlen == 0 && !A_chk) return MAMBA3_ERR_INVALID;
   if ((rc = check_state(init)) || (rc = check_state(final_state))) return rc;
   if (!workspace || !aligned16(workspace)) return MAMBA3_ERR_WORKSPACE;
   if (workspace_bytes < mamba3_scan_workspace_bytes(d)) return MAMBA3_ERR_WORKSPACE;
@@ -104,7 +110,7 @@ int mamba3_scan_fwd(const mamba3_dims* d, const void* x, const void* B, const vo
   a.R = d->rank;
   a.Q = d->chunk;
   a.dtype = d->in_dtype;
-  a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.D = D;
+  a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.A_t = A_t; a.D = D;
   if (init) { a.h0 = init->h; a.bprev0 = init->b_prev; a.xprev0 = init->x_prev; a.angle0 = init->angle; }
   a.y = y;
   if (final_state) {
@@ -120,6 +126,57 @@ int mamba3_scan_fwd(const mamba3_dims* d, const void* x, const void* B, const vo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
   return use_tc ? m3::launch_scan_tc(a, s) : m3::launch_scan_simt(a, s);
+}
+
+// The decode step behind mamba3_decode_step and mamba3_decode_step_at.
+int decode_impl(const mamba3_dims* d, const mamba3_state* state, const void* x, const void* B, const void* C,
+                const void* theta, const void* dt, const void* lam, const float* A, const void* A_t,
+                const float* D, void* y, void* stream) {
+  int rc = check_dims(d, false);
+  if (rc) return rc;
+  if (!state) return MAMBA3_ERR_INVALID;
+  if ((rc = check_state(state))) return rc;
+  const float* A_chk = A ? A : static_cast<const float*>(A_t);
+  if ((rc = check_inputs(x, B, C, theta, dt, lam, A_chk, D, y))) return rc;
+  m3::DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.batch = d->batch;
+  a.nheads = d->nheads;
+  a.P = d->headdim;
+  a.N = d->dstate;
+  a.R = d->rank;
+  a.dtype = d->in_dtype;
+  a.h = state->h; a.bprev = state->b_prev; a.xprev = state->x_prev; a.angle = state->angle;
+  a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.A_t = A_t; a.D = D; a.y = y;
+  if ((rc = m3::decode_supported(a))) return rc;
+  return m3::launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+extern "C" {
+
+int mamba3_scan_fwd(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                    const void* dt, const void* lam, const float* A, const float* D,
+                    const mamba3_state* init, void* y, const mamba3_state* final_state, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  return scan_fwd_impl(d, x, B, C, theta, dt, lam, A, nullptr, D, init, y, final_state, workspace, workspace_bytes,
+                       stream);
+}
+
+int mamba3_scan_fwd_at(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                       const void* dt, const void* lam, const void* A_t, const float* D, const mamba3_state* init,
+                       void* y, const mamba3_state* final_state, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (!A_t) return MAMBA3_ERR_INVALID;
+  return scan_fwd_impl(d, x, B, C, theta, dt, lam, nullptr, A_t, D, init, y, final_state, workspace,
+                       workspace_bytes, stream);
+}
+
+int mamba3_decode_step_at(const mamba3_dims* d, const mamba3_state* state, const void* x, const void* B,
+                          const void* C, const void* theta, const void* dt, const void* lam, const void* A_t,
+                          const float* D, void* y, void* stream) {
+  if (!A_t) return MAMBA3_ERR_INVALID;
+  return decode_impl(d, state, x, B, C, theta, dt, lam, nullptr, A_t, D, y, stream);
 }
 
 int mamba3_scan_fwd_bcnorm(const mamba3_dims* d, const void* x, const void* B_raw, const void* C_raw,
@@ -177,23 +234,7 @@ int mamba3_decode_step_bcnorm(const mamba3_dims* d, const mamba3_state* state, c
 int mamba3_decode_step(const mamba3_dims* d, const mamba3_state* state, const void* x, const void* B,
                        const void* C, const void* theta, const void* dt, const void* lam, const float* A,
                        const float* D, void* y, void* stream) {
-  int rc = check_dims(d, false);
-  if (rc) return rc;
-  if (!state) return MAMBA3_ERR_INVALID;
-  if ((rc = check_state(state))) return rc;
-  if ((rc = check_inputs(x, B, C, theta, dt, lam, A, D, y))) return rc;
-  m3::DecodeArgs a;
-  memset(&a, 0, sizeof(a));
-  a.batch = d->batch;
-  a.nheads = d->nheads;
-  a.P = d->headdim;
-  a.N = d->dstate;
-  a.R = d->rank;
-  a.dtype = d->in_dtype;
-  a.h = state->h; a.bprev = state->b_prev; a.xprev = state->x_prev; a.angle = state->angle;
-  a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.D = D; a.y = y;
-  if ((rc = m3::decode_supported(a))) return rc;
-  return m3::launch_decode(a, static_cast<cudaStream_t>(stream));
+  return decode_impl(d, state, x, B, C, theta, dt, lam, A, nullptr, D, y, stream);
 }
 
 int mamba3_device_status(const void* workspace, void* stream) {

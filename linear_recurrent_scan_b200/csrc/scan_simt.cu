@@ -77,7 +77,8 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(ScanArgs a, SimtLay
   float* phi = sm + lay.off_phi;
   __shared__ float s_lam[kMaxRows + 1];
 
-  const float Ah = a.A[hh];
+  const float Ah = a.A ? a.A[hh] : 0.f;
+  const T* AT = static_cast<const T*>(a.A_t);  // time-varying decay [b, L, H], or null
   const float Dh = a.D ? a.D[hh] : 0.f;
   const T* X = static_cast<const T*>(a.x);
   const T* Bg = static_cast<const T*>(a.B);
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(ScanArgs a, SimtLay
     if (tid == 0) {
       float c = 0.f;
       for (int i = 0; i < q; ++i) {
-        c += sdt[i] * Ah;
+        c += sdt[i] * (AT ? ld1(AT + tok(t0 + i)) : Ah);
         cum[i] = c;
         gam[i] = s_lam[i] * sdt[i];
         w[i] = gam[i] + (1.f - s_lam[i + 1]) * sdt[i + 1];

@@ -40,6 +40,8 @@
 // Y = P X (P from TMEM).  TMEM columns: S [0,128), P [128,192) (bf16 pairs),
 // Y [192,256), Yi [256,320), Hacc [320,384); with R = 1 a second Y, Yi buffer at
 // [384,448), [448,512) (y written one chunk late).
+// Variants (template V): the plain recurrence; the fused B/C RMS norm in front of
+// the rotation; a time-varying decay A_t per token in place of A per head.
 // Every wait is bounded: on expiry the CTA raises an abort flag, reports
 // MAMBA3_ERR_TIMEOUT in the device status word, drains and returns.
 #include <cuda.h>
@@ -105,9 +107,13 @@ struct Cfg {
   static constexpr int DL_PAD = (DL_BYTES + 127) & ~127;
   static constexpr int OFF_DL = (OFF_MISC + 16 + 127) & ~127;
   static constexpr int OFF_SINK = OFF_DL + 2 * DL_PAD;  // [Q] floats: consumes the tile reads
-  // fused B/C normalisation: w_B, bias_B, w_C, bias_C of this head, [R][N] floats each
-  static constexpr int OFF_NRM = (OFF_SINK + Q * 4 + 15) & ~15;
-  static constexpr int SMEM = OFF_NRM + 4 * R * N * 4;
+  // fused B/C normalisation: w_B, bias_B, w_C, bias_C of this head, [R][N] floats
+  // each; or, with a time-varying decay by TMA (the two are never combined), the
+  // A_t tile [Q][8] bf16 (refilled with theta)
+  static constexpr int OFF_NRM = (OFF_SINK + Q * 4 + 127) & ~127;
+  static constexpr int AT_BYTES = Q * 16;
+  static constexpr int NRM_BYTES = 4 * R * N * 4 > AT_BYTES ? 4 * R * N * 4 : AT_BYTES;
+  static constexpr int SMEM = OFF_NRM + NRM_BYTES;
   static constexpr int SMEM_ALLOC = SMEM + 1024;       // slack for 1024-byte alignment
   static_assert(NG * NPART == kNPrep && TPP * NPART == Q, "angle partition");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -123,6 +129,7 @@ struct TcParams {
   ScanArgs a;
   int nchunks;
   int dl_tma;  // dt and lam arrive by TMA with theta (else: global loads one chunk ahead)
+  int at_tma;  // a time-varying decay A_t arrives by TMA with theta (needs dl_tma)
 };
 
 __device__ __forceinline__ size_t tok_index(const ScanArgs& a, int b, int t, int h) {
@@ -162,9 +169,13 @@ __device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 256;" ::
 // place (16 bytes per shared-memory access, 2 rows in flight), the rank-1
 // column factors of the mask and X_w.  dt and lam are prefetched one chunk
 // ahead into registers; theta arrives by TMA.
-template <int N, int R, bool BCN>
+// kernel variants: the plain recurrence, the fused B/C norm, the time-varying decay A_t
+enum Variant { kPlain = 0, kBCNorm = 1, kTimeA = 2 };
+
+template <int N, int R, int V>
 __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int dl_tma, int b, int hh,
                                           float Ah, uint64_t* bars, volatile int* abort_flag, DeviceStatus* status) {
+  constexpr bool BCN = V == kBCNorm, TVA = V == kTimeA;
   using K = Cfg<N, R>;
   constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, TPP = K::TPP, TB = K::TB, NPART = K::NPART;
   const int pt = threadIdx.x - kPrep0;
@@ -176,19 +187,26 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
   const size_t unit = (size_t)b * H + hh;
   const int g = pt % NG, part = pt / NG;  // 4-pair group (one 16-byte chunk of a row), token part
   const int kb = g / 8, c8 = g % 8;       // 64-element block and 16-byte chunk of the group
-  // dt, lam of this (batch, head): element t at [t * H]
+  // dt, lam (and A_t) of this (batch, head): element t at [t * H]
   const __nv_bfloat16* DTu = static_cast<const __nv_bfloat16*>(a.dt) + (size_t)b * L * H + hh;
   const __nv_bfloat16* LMu = static_cast<const __nv_bfloat16*>(a.lam) + (size_t)b * L * H + hh;
+
 
   if (pt < K2) phi[pt] = a.angle0 ? a.angle0[unit * K2 + pt] : 0.f;
 
   // prefetched per chunk: (scan threads) dt, lam of token pt and of the next
-  // token; (angle threads) dt of this part's tokens
-  float s_dt, s_lm, s_dtn, s_lmn, p_dt[TPP];
-  auto load_scalars = [&](int cc, float& o_dt, float& o_lm, float& o_dtn, float& o_lmn, float (&o_pdt)[TPP]) {
+  // token, and its decay rate (A_t, else A); (angle threads) dt of this part's tokens
+  float s_dt, s_lm, s_dtn, s_lmn, s_at, p_dt[TPP];
+  auto load_scalars = [&](int cc, float& o_dt, float& o_lm, float& o_dtn, float& o_lmn, float& o_at,
+                          float (&o_pdt)[TPP]) {
     const int tc0 = cc * Q;
     const int tg = tc0 + pt;
     const bool ok = pt < Q && cc < nchunks;
+    o_at = Ah;
+    if constexpr (TVA) {  // A_t sits at the same offset as dt
+      const __nv_bfloat16* ATu = static_cast<const __nv_bfloat16*>(a.A_t) + (DTu - static_cast<const __nv_bfloat16*>(a.dt));
+      o_at = (ok && tg < L) ? __bfloat162float(ATu[(size_t)tg * H]) : 0.f;
+    }
     o_dt = (ok && tg < L) ? __bfloat162float(DTu[(size_t)tg * H]) : 0.f;
     o_lm = (ok && tg < L) ? __bfloat162float(LMu[(size_t)tg * H]) : 1.f;
     o_dtn = (ok && tg + 1 < L) ? __bfloat162float(DTu[(size_t)(tg + 1) * H]) : 0.f;
@@ -202,11 +220,13 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
   if (dl_tma) {
     s_dt = s_dtn = 0.f;
     s_lm = s_lmn = 1.f;
+    s_at = Ah;
 #pragma unroll
     for (int i = 0; i < TPP; ++i) p_dt[i] = 0.f;
   } else {
-    load_scalars(0, s_dt, s_lm, s_dtn, s_lmn, p_dt);
+    load_scalars(0, s_dt, s_lm, s_dtn, s_lmn, s_at, p_dt);
   }
+  const __nv_bfloat16* ats = reinterpret_cast<const __nv_bfloat16*>(smem + K::OFF_NRM) + (hh & 7);
   const __nv_bfloat16* dts = reinterpret_cast<const __nv_bfloat16*>(smem + K::OFF_DL) + (hh & 7);
   const __nv_bfloat16* lms = reinterpret_cast<const __nv_bfloat16*>(smem + K::OFF_DL + K::DL_PAD) + (hh & 7);
   float* sink = reinterpret_cast<float*>(smem + K::OFF_SINK);
@@ -239,11 +259,12 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
         s_lm = __bfloat162float(lms[pt * 8]);
         s_dtn = __bfloat162float(dts[(pt + 1) * 8]);
         s_lmn = __bfloat162float(lms[(pt + 1) * 8]);
+        if constexpr (TVA) s_at = __bfloat162float(ats[pt * 8]);
       }
 #pragma unroll
       for (int i = 0; i < TPP; ++i) p_dt[i] = __bfloat162float(dts[(part * TPP + i) * 8]);
     }
-    float v = (pt < Q) ? s_dt * Ah * kLog2e : 0.f;
+    float v = (pt < Q) ? s_dt * (TVA ? s_at : Ah) * kLog2e : 0.f;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const float n = __shfl_up_sync(0xffffffffu, v, o);
@@ -262,7 +283,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       loc[3] += p_dt[i] * t23.y;
     }
     *reinterpret_cast<float4*>(part_sum + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
-    if (dl_tma && pt < Q) sink[pt] = (s_dt + s_lm) + (s_dtn + s_lmn);
+    if (dl_tma && pt < Q) sink[pt] = (s_dt + s_lm) + (s_dtn + s_lmn) + (TVA ? s_at : 0.f);
     // Release the theta (and dt, lam) tiles only after stores that consume
     // every value loaded from them: the arrive does not wait for shared-memory
     // loads still in flight, and the refill is an async-proxy write that is not
@@ -300,7 +321,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
 #pragma unroll
     for (int i = 0; i < TPP; ++i) pdt_cur[i] = p_dt[i];
     // next chunk's scalars, in flight during the rotation (unless they come by TMA)
-    if (!dl_tma) load_scalars(c + 1, s_dt, s_lm, s_dtn, s_lmn, p_dt);
+    if (!dl_tma) load_scalars(c + 1, s_dt, s_lm, s_dtn, s_lmn, s_at, p_dt);
 #pragma unroll
     for (int i0 = 0; i0 < TPP; i0 += TB) {
       float sn[TB][4], cs[TB][4];
@@ -657,12 +678,12 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
   }
 }
 
-template <int N, int R, bool BCN>
+template <int N, int R, int V>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
                    const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmL,
-                   const TcParams prm) {
+                   const __grid_constant__ CUtensorMap tmA, const TcParams prm) {
   using K = Cfg<N, R>;
   constexpr int Q = K::Q;
   extern __shared__ uint8_t smem_raw[];
@@ -707,6 +728,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmD);
       prefetch_tmap(&tmL);
     }
+    if (prm.at_tma) prefetch_tmap(&tmA);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -727,7 +749,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // One thread polls the three conditions (non-blocking), so no stream waits behind another.
       int cb = 0, cx = 0, ct = 0;
       long long t_last = clock64();
-      const uint32_t th_bytes = K::TH_BYTES + (prm.dl_tma ? 2u * K::DL_BYTES : 0u);
+      const uint32_t th_bytes =
+          K::TH_BYTES + (prm.dl_tma ? 2u * K::DL_BYTES : 0u) + (prm.at_tma ? (uint32_t)K::AT_BYTES : 0u);
       while (cx < nchunks || ct < nchunks) {
         bool progress = false;
         if (cb < nchunks && mbar_test(&bars[bEmptyBC0 + (cb & 1)], ((cb >> 1) & 1) ^ 1)) {
@@ -756,6 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(smem + K::OFF_DL, &tmD, &bars[bThFull], hh & ~7, t0, b);
             tma_load_3d(smem + K::OFF_DL + K::DL_PAD, &tmL, &bars[bThFull], hh & ~7, t0, b);
           }
+          if (prm.at_tma) tma_load_3d(smem + K::OFF_NRM, &tmA, &bars[bThFull], hh & ~7, t0, b);
           ++ct;
           progress = true;
         }
@@ -834,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bars[bDone], 0, abort_flag, status, kTagDrain, 400000000LL);
     }
   } else if (tid < kEpi0) {
-    prep_role<N, R, BCN>(smem, a, nchunks, prm.dl_tma, b, hh, a.A[hh], bars, abort_flag, status);
+    prep_role<N, R, V>(smem, a, nchunks, prm.dl_tma, b, hh, a.A ? a.A[hh] : 0.f, bars, abort_flag, status);
   } else {
     epi_role<N, R>(smem, a, nchunks, b, hh, bars, abort_flag, status, tmem);
   }
@@ -884,12 +908,12 @@ bool make_map(CUtensorMap* m, const void* base, int inner, const ScanArgs& a, in
 // dt or lam [batch, L, H] bf16, box = {8, Q + 1, 1}: the 8 heads of a 16-byte
 // group over the chunk's tokens and the next one, zero fill past the end.
 // Needs H a multiple of 8 (16-byte row stride) and a 16-byte aligned base.
-bool make_dl_map(CUtensorMap* m, const void* base, const ScanArgs& a, int Q) {
+bool make_dl_map(CUtensorMap* m, const void* base, const ScanArgs& a, int rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc || a.nheads % 8 != 0 || (reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)a.nheads, (cuuint64_t)a.seqlen, (cuuint64_t)a.batch};
   const cuuint64_t strides[2] = {2ull * a.nheads, 2ull * a.nheads * a.seqlen};
-  const cuuint32_t box[3] = {8, (cuuint32_t)(Q + 1), 1};
+  const cuuint32_t box[3] = {8, (cuuint32_t)rows, 1};
   const cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -920,14 +944,20 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
   TcParams prm;
   prm.a = a;
   prm.nchunks = (a.seqlen + K::Q - 1) / K::Q;
-  CUtensorMap tmD, tmL;
+  CUtensorMap tmD, tmL, tmA;
   memset(&tmD, 0, sizeof(tmD));
   memset(&tmL, 0, sizeof(tmL));
-  prm.dl_tma = make_dl_map(&tmD, a.dt, a, K::Q) && make_dl_map(&tmL, a.lam, a, K::Q);
-  auto kern = a.bcnorm ? scan_tc_kernel<N, R, true> : scan_tc_kernel<N, R, false>;
+  memset(&tmA, 0, sizeof(tmA));
+  prm.dl_tma = make_dl_map(&tmD, a.dt, a, K::Q + 1) && make_dl_map(&tmL, a.lam, a, K::Q + 1);
+  prm.at_tma = 0;
+  if (a.A_t) {  // the A_t tile shares the region of the B/C norm table; all three tiles or none
+    prm.at_tma = prm.dl_tma && !a.bcnorm && make_dl_map(&tmA, a.A_t, a, K::Q);
+    if (!prm.at_tma) prm.dl_tma = 0;
+  }
+  auto kern = a.bcnorm ? scan_tc_kernel<N, R, kBCNorm> : (a.A_t ? scan_tc_kernel<N, R, kTimeA> : scan_tc_kernel<N, R, kPlain>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
-  kern<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmC, tmX, tmT, tmD, tmL, prm);
+  kern<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmC, tmX, tmT, tmD, tmL, tmA, prm);
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 

@@ -169,6 +169,14 @@ def raw_bc_inputs(inp: Dict[str, torch.Tensor], seed: int = BASE_SEED + 2) -> Di
     return out
 
 
+def decay_rates(like: torch.Tensor, seed: int = BASE_SEED + 4) -> torch.Tensor:
+    """A time-varying decay rate per token and head, shaped, typed and placed like
+    `like` (dt): A_t = -exp(U(log 0.5, log 16))."""
+    g = _gen(like.device, seed)
+    u = torch.empty(like.shape, device=like.device).uniform_(math.log(0.5), math.log(16.0), generator=g)
+    return (-torch.exp(u)).to(like.dtype).contiguous()
+
+
 def to_f64(d: Dict[str, torch.Tensor]):
     """Widen every tensor to a float64 numpy array (exact for bf16/fp32)."""
     return {k: v.detach().to("cpu", torch.float64).numpy() for k, v in d.items()}

@@ -185,3 +185,17 @@ def test_bcnorm_entry_points_validate_on_host(lib):
     assert scan_bcn(lib, dims(in_dtype=m3.MAMBA3_F32), ok) == m3.MAMBA3_ERR_UNSUPPORTED
     assert decode_bcn(lib, dims(), None) == m3.MAMBA3_ERR_INVALID
     assert decode_bcn(lib, dims(headdim=32), ok) == m3.MAMBA3_ERR_UNSUPPORTED            # streaming kernel: P = 64
+
+
+def test_time_varying_decay_entry_points_validate_on_host(lib):
+    p = dict(x=FAKE, B=FAKE, C=FAKE, theta=FAKE, dt=FAKE, lam=FAKE, y=FAKE)
+    rc = lib.mamba3_scan_fwd_at(ctypes.byref(dims()), p["x"], p["B"], p["C"], p["theta"], p["dt"], p["lam"], None,
+                                None, None, p["y"], None, FAKE, 1 << 20, None)
+    assert rc == m3.MAMBA3_ERR_INVALID                                   # A_t is required
+    rc = lib.mamba3_scan_fwd_at(ctypes.byref(dims()), p["x"], p["B"], p["C"], p["theta"], p["dt"], p["lam"], FAKE + 2,
+                                None, None, p["y"], None, FAKE, 1 << 20, None)
+    assert rc == m3.MAMBA3_ERR_INVALID                                   # misaligned A_t
+    cs = m3._CState(FAKE, FAKE, FAKE, FAKE)
+    rc = lib.mamba3_decode_step_at(ctypes.byref(dims()), ctypes.byref(cs), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                   None, FAKE, None)
+    assert rc == m3.MAMBA3_ERR_INVALID
