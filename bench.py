@@ -43,13 +43,13 @@ FALLBACK_HBM_GBS = 6650.0
 # traffic null, since its counters are out of date.
 TRAFFIC = {
     "prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"),
-                "659087eb7f4d6efea1eb120319c5416d33015294b3cb0218d382ba67740923a4", 811429120 + 136969984,
+                "a613588c5d8a7a7ed3a8d0443bf6b4317e11f1585fe3846bc45bf7fd32acb056", 811438592 + 137308416,
                 "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     "siso_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                         "80cdf686cd24e1026aee9bce7e53a1796ca03d6a41fbc32c95d37ddc31e190e4", 283177472 + 219342848,
+                         "eea54a57c8c5a78d7ea5371966f93b0c2696c767db27ec84c749b918dc4d9c7c", 283173120 + 219014656,
                          "profiles/decode_stream_b128_traffic_and_counters.txt"),
     "mimo4_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                          "80cdf686cd24e1026aee9bce7e53a1796ca03d6a41fbc32c95d37ddc31e190e4", 317801728 + 240049920,
+                          "eea54a57c8c5a78d7ea5371966f93b0c2696c767db27ec84c749b918dc4d9c7c", 317781504 + 240473600,
                           "profiles/decode_stream_b128_traffic_and_counters.txt"),
 }
 
@@ -276,10 +276,11 @@ def run_prefill(m3, args, world, rank, clk):
                 tokens=w.batch * w.seqlen, bytes=prefill_bytes(w))
 
 
-def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False):
+def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False, time_varying_a=False):
     """Median per-launch time (ms) of one prefill launch of workload `w`, inputs
     resident on the device (larger than L2), final state exported.  With
-    fused_norm the launch takes raw B, C and normalises them in the kernel."""
+    fused_norm the launch takes raw B, C and normalises them in the kernel; with
+    time_varying_a it takes a decay rate per token (A_t) instead of A per head."""
     dev = torch.device("cuda")
     inp = wl.make_inputs(w, seed=wl.BASE_SEED + rank, device=dev)
     norm = None
@@ -287,6 +288,7 @@ def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False)
         raw = wl.raw_bc_inputs(inp, seed=wl.BASE_SEED + 2 + rank)
         inp["B"], inp["C"] = raw["B_raw"], raw["C_raw"]
         norm = m3.BCNorm(raw["w_B"], raw["w_C"], raw["bias_B"], raw["bias_C"], 1e-6)
+    A_t = wl.decay_rates(inp["dt"], seed=wl.BASE_SEED + 4 + rank) if time_varying_a else None
     ins = [inp[n] for n in NAMES]
     y = torch.empty_like(inp["x"])
     fin = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
@@ -295,7 +297,9 @@ def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False)
     stream = torch.cuda.current_stream()
 
     def launch():
-        if fused_norm:
+        if time_varying_a:
+            m3.mamba3_scan_fwd_at(*ins, A_t, inp["D"], y=y, final_state=fin, workspace=ws, stream=stream)
+        elif fused_norm:
             m3.mamba3_scan_fwd_bcnorm(*ins, inp["A"], inp["D"], norm=norm, y=y, final_state=fin, workspace=ws,
                                       stream=stream)
         else:
@@ -319,7 +323,7 @@ def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False)
     return statistics.median(times)
 
 
-def run_decode(m3, w: wl.Workload, world, rank, steps, fused_norm=False):
+def run_decode(m3, w: wl.Workload, world, rank, steps, fused_norm=False, time_varying_a=False):
     """Seed the state with a 512-token prefill, then time `steps` decode steps
     captured in one CUDA graph (per-step inputs pre-generated, larger than L2).
     With fused_norm each step takes raw B, C and normalises them in the kernel."""
@@ -335,11 +339,16 @@ def run_decode(m3, w: wl.Workload, world, rank, steps, fused_norm=False):
         raw = wl.raw_bc_inputs(steps_in, seed=wl.BASE_SEED + 3 + rank)
         steps_in["B"], steps_in["C"] = raw["B_raw"], raw["C_raw"]
         norm = m3.BCNorm(raw["w_B"], raw["w_C"], raw["bias_B"], raw["bias_C"], 1e-6)
-    step_fn = ((lambda st_, i_, y_: m3.mamba3_decode_step_bcnorm(st_, *(steps_in[n][i_] for n in NAMES), A, D,
-                                                                 norm=norm, y=y_, stream=s))
-               if fused_norm else
-               (lambda st_, i_, y_: m3.mamba3_decode_step(st_, *(steps_in[n][i_] for n in NAMES), A, D, y=y_,
-                                                          stream=s)))
+    A_t = wl.decay_rates(steps_in["dt"], seed=wl.BASE_SEED + 5 + rank) if time_varying_a else None
+    if time_varying_a:
+        step_fn = lambda st_, i_, y_: m3.mamba3_decode_step_at(st_, *(steps_in[n][i_] for n in NAMES), A_t[i_], D,
+                                                               y=y_, stream=s)
+    elif fused_norm:
+        step_fn = lambda st_, i_, y_: m3.mamba3_decode_step_bcnorm(st_, *(steps_in[n][i_] for n in NAMES), A, D,
+                                                                   norm=norm, y=y_, stream=s)
+    else:
+        step_fn = lambda st_, i_, y_: m3.mamba3_decode_step(st_, *(steps_in[n][i_] for n in NAMES), A, D, y=y_,
+                                                            stream=s)
     ys = torch.empty((steps,) + steps_in["x"].shape[1:], dtype=w.dtype, device=dev)
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -406,6 +415,20 @@ def ours(args):
     fused["decode_" + DECODE[0].name] = {"us_per_step": round(us, 2), "roofline": {
         "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
         "bytes_per_step": decode_bytes(DECODE[0])}}
+    # the time-varying decay variant (A_t per token: 2 more bytes per token-head)
+    ms = max_over_ranks(run_prefill_plain(m3, PREFILL, rank, steps=max(5, min(args.steps, 20)), warmup=3,
+                                          time_varying_a=True), world)
+    by = prefill_bytes(PREFILL) + 2 * PREFILL.token_heads
+    gbs = by / (ms * 1e-3) / 1e9
+    tva = {"prefill_" + PREFILL.name: {"ms_per_launch": round(ms, 4), "roofline": {
+        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
+        "bytes_per_launch": by}}}
+    us = run_decode(m3, DECODE[0], world, rank, DECODE[0].decode_steps, time_varying_a=True)
+    by = decode_bytes(DECODE[0]) + 2 * DECODE[0].batch * DECODE[0].nheads
+    gbs = by / (us * 1e-6) / 1e9
+    tva["decode_" + DECODE[0].name] = {"us_per_step": round(us, 2), "roofline": {
+        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
+        "bytes_per_step": by}}
     more = {}
     for w in PREFILL_MORE:
         ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=max(5, min(args.steps, 20)), warmup=3), world)
@@ -441,6 +464,7 @@ def ours(args):
                      "bytes_per_launch": r["bytes"], "launch_ms": round(r["launch_ms"], 4)},
         "prefill_more": more,
         "fused_bc_norm": fused,
+        "time_varying_decay": tva,
         "decode": dec,
         "e2e": {"value": round(e2e_value, 3), "unit": "Mtokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
