@@ -45,7 +45,7 @@ def build(force: bool = False) -> str:
 
 
 class _Dims(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int) for n in ("batch", "seqlen", "nheads", "headdim", "dstate", "rank")]
+    _fields_ = [(n, ctypes.c_int) for n in ("batch", "seqlen", "nheads", "headdim", "dstate", "rank", "ngroups")]
 
 
 _P = ctypes.POINTER(ctypes.c_double)
@@ -122,11 +122,13 @@ def _prepare(x, B, C, theta, dt, lam, A, D):
     D = _f64(D) if D is not None else None
     b, L, H, R, P = x.shape
     N = B.shape[-1]
-    assert B.shape == (b, L, H, R, N) and C.shape == B.shape, "B/C must be [b,L,H,R,N]"
+    G = B.shape[2]
+    assert B.shape == (b, L, G, R, N) and C.shape == B.shape and H % G == 0, \
+        "B/C must be [b,L,H,R,N] or, grouped, [b,L,G,R,N] with H a multiple of G"
     assert theta.shape == (b, L, H, N // 2), "theta must be [b,L,H,N/2]"
     assert dt.shape == (b, L, H) and lam.shape == (b, L, H)
     assert A.shape == (H,) or A.shape == (b, L, H), "A must be [H] (per head) or [b,L,H] (per token)"
-    dims = _Dims(b, L, H, P, N, R)
+    dims = _Dims(b, L, H, P, N, R, 0 if G == H else G)
     return dims, (x, B, C, theta, dt, lam, A, D)
 
 
@@ -173,6 +175,8 @@ def _run(fn_name, x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = No
 def scan_complex(x, B, C, theta, dt, lam, A, D=None, init=None, nthreads=None, units=None):
     """The definition: explicit complex-diagonal state, sequential in t.
     A is [H] (one decay rate per head) or [b, L, H] (time-varying, one per token).
+    B, C are [b, L, H, R, N] or, shared by groups of heads, [b, L, G, R, N]
+    (head h reads group h // (H // G)).
 
     Returns (y [b,L,H,R,P], final State).  ``units`` optionally restricts the
     work to a list of flattened (b*H + h) indices (others stay zero).
@@ -217,7 +221,7 @@ def bc_norm(z, w=None, bias=None, eps: float = 1e-6) -> np.ndarray:
     z = _f64(z)
     *lead, H, R, N = z.shape
     rows = int(np.prod(lead)) if lead else 1
-    dims = _Dims(1, rows, H, 0, N, R)
+    dims = _Dims(1, rows, H, 0, N, R, 0)
     w = _f64(w) if w is not None else None
     bias = _f64(bias) if bias is not None else None
     for a in (w, bias):

@@ -38,6 +38,11 @@
  * Layouts (row-major, contiguous; b = batch, L = seqlen, H = heads):
  *   x      [b, L, H, R, P]     B, C  [b, L, H, R, N]     theta [b, L, H, N/2]
  *   dt,lam [b, L, H]           A, D  [H]                 y     [b, L, H, R, P]
+ * Optional: A_t [b, L, H] (a decay rate per token, replacing A), and grouped
+ * B, C [b, L, G, R, N] with ngroups G dividing H, head h reading group
+ * h / (H / G) (the Mamba line's shared B/C; not on the pages, whose heads each
+ * have their own: a grouped input equals the per-head one with every group's
+ * rows repeated over its heads).
  * State (the real frame rotated by -Phi, as the CUDA library stores it):
  *   h [b,H,N,P]  (row 2k = Re, row 2k+1 = Im of e^{-i Phi} H)
  *   b_prev [b,H,R,N] (B of the last token, rotated by -Phi of that token)
@@ -51,6 +56,7 @@
 
 typedef struct {
   int batch, seqlen, nheads, headdim, dstate, rank;
+  int ngroups; /* 0: B, C per head; else B, C [b, L, ngroups, R, N] shared by nheads / ngroups heads */
 } m3o_dims;
 
 typedef struct {
@@ -70,6 +76,12 @@ static double decay_rate(const m3o_io* io, size_t it, int h) { return io->A_t ? 
 /* ------------------------------------------------------------------------- */
 static size_t ix_tok(const m3o_dims* d, int b, int t, int h) {
   return ((size_t)b * d->seqlen + t) * d->nheads + h;
+}
+/* row (b, t, group of head h) of B and C: heads h = g * (H / G) ... (g + 1) * (H / G) - 1
+ * share group g (the Mamba line's grouped B/C; the pages use one per head) */
+static size_t ix_bc(const m3o_dims* d, int b, int t, int h) {
+  if (d->ngroups <= 0) return ix_tok(d, b, t, h);
+  return ((size_t)b * d->seqlen + t) * d->ngroups + h / (d->nheads / d->ngroups);
 }
 static size_t ix_state(const m3o_dims* d, int b, int h) {
   return (size_t)b * d->nheads + h;
@@ -112,8 +124,8 @@ static void unit_complex(const m3o_dims* d, const m3o_io* io, int b, int h) {
     const size_t it = ix_tok(d, b, t, h);
     const double dt = io->dt[it], lam = io->lam[it];
     const double* x = io->x + it * R * P;
-    const double* Bt = io->B + it * R * N;
-    const double* Ct = io->C + it * R * N;
+    const double* Bt = io->B + ix_bc(d, b, t, h) * R * N;
+    const double* Ct = io->C + ix_bc(d, b, t, h) * R * N;
     const double* th = io->theta + it * K;
     const double At = decay_rate(io, it, h);
     for (int k = 0; k < K; ++k) {
@@ -161,10 +173,10 @@ static void unit_complex(const m3o_dims* d, const m3o_io* io, int b, int h) {
     for (int k = 0; k < K; ++k) io->angle_out[us * K + k] = Phi[k];
   if (io->bprev_out && io->xprev_out) {
     if (L > 0) {
-      const size_t il = ix_tok(d, b, L - 1, h);
+      const size_t il = ix_tok(d, b, L - 1, h), ilb = ix_bc(d, b, L - 1, h);
       for (int r = 0; r < R; ++r) {
         for (int k = 0; k < K; ++k) {
-          double complex bt = io->B[il * R * N + r * N + 2 * k] + I * io->B[il * R * N + r * N + 2 * k + 1];
+          double complex bt = io->B[ilb * R * N + r * N + 2 * k] + I * io->B[ilb * R * N + r * N + 2 * k + 1];
           double complex g = cexp(-I * Phi[k]) * bt;
           io->bprev_out[(us * R + r) * N + 2 * k] = creal(g);
           io->bprev_out[(us * R + r) * N + 2 * k + 1] = cimag(g);
@@ -217,8 +229,8 @@ static void unit_rope(const m3o_dims* d, const m3o_io* io, int b, int h) {
     for (int k = 0; k < K; ++k) Phi[k] += dt * io->theta[it * K + k];
     for (int r = 0; r < R; ++r)
       for (int k = 0; k < K; ++k) {
-        const double* Bt = io->B + it * R * N + r * N;
-        const double* Ct = io->C + it * R * N + r * N;
+        const double* Bt = io->B + ix_bc(d, b, t, h) * R * N + r * N;
+        const double* Ct = io->C + ix_bc(d, b, t, h) * R * N + r * N;
         rot_neg(Phi[k], Bt[2 * k], Bt[2 * k + 1], &Br[r * N + 2 * k], &Br[r * N + 2 * k + 1]);
         rot_neg(Phi[k], Ct[2 * k], Ct[2 * k + 1], &Cr[r * N + 2 * k], &Cr[r * N + 2 * k + 1]);
       }
@@ -287,8 +299,8 @@ static void unit_quadratic(const m3o_dims* d, const m3o_io* io, int b, int h) {
     for (int k = 0; k < K; ++k) Phi[k] += io->dt[it] * io->theta[it * K + k];
     for (int r = 0; r < R; ++r)
       for (int k = 0; k < K; ++k) {
-        const double* Bt = io->B + it * R * N + r * N;
-        const double* Ct = io->C + it * R * N + r * N;
+        const double* Bt = io->B + ix_bc(d, b, t, h) * R * N + r * N;
+        const double* Ct = io->C + ix_bc(d, b, t, h) * R * N + r * N;
         rot_neg(Phi[k], Bt[2 * k], Bt[2 * k + 1], &Br[(t * R + r) * N + 2 * k], &Br[(t * R + r) * N + 2 * k + 1]);
         rot_neg(Phi[k], Ct[2 * k], Ct[2 * k + 1], &Cr[(t * R + r) * N + 2 * k], &Cr[(t * R + r) * N + 2 * k + 1]);
       }

@@ -29,6 +29,7 @@ MUTATIONS = {
     "decay_ignores_A_t": ("return io->A_t ? io->A_t[it] : io->A[h];", "return io->A[h];"),
     "bcnorm_sum_not_mean": ("    ms /= N;\n", "\n"),
     "bcnorm_eps_outside_sqrt": ("1.0 / sqrt(ms + eps)", "1.0 / (sqrt(ms) + eps)"),
+    "bc_group_interleaved": ("h / (d->nheads / d->ngroups)", "h % d->ngroups"),
     "bcnorm_bias_index_swapped": ("const size_t p = ((size_t)h * R + r) * N + n;", "const size_t p = ((size_t)r * H + h) * N + n;"),
 }
 
@@ -48,6 +49,7 @@ PIN_FUNCS = [
     pins.test_bc_norm_unit_rms_per_row,
     pins.test_bc_norm_scale_invariant_and_odd,
     pins.test_bc_norm_weight_and_bias_per_head_and_rank,
+    lambda: [pins.test_grouped_bc_equals_per_head_broadcast("scan_complex", G, R) for G, R in ((2, 2), (3, 1))],
 ]
 
 

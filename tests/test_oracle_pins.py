@@ -503,3 +503,43 @@ def test_time_varying_decay_prefill_then_decode():
         yt, st = oracle.decode_step(st, **step, D=inp["D"])
         assert rel_err(yt, y_all[:, t]) < 1e-12
     assert rel_err(st.h, f_all.h) < 1e-12
+
+
+# ---------------------------------------------------------------- grouped B/C
+# The pages give every head its own B and C.  The Mamba line also shares one B and
+# C among a group of consecutive heads (ngroups G, head h reads group h // (H // G));
+# the reading here: a grouped input is exactly the per-head input with each group's
+# rows repeated over its heads.
+
+@pytest.mark.parametrize("fn", ["scan_complex", "scan_rope", "scan_quadratic"])
+@pytest.mark.parametrize("G,R", [(1, 1), (2, 2), (3, 1)])
+def test_grouped_bc_equals_per_head_broadcast(fn, G, R):
+    rng = np.random.default_rng(120 + 7 * G + R)
+    b, L, H, P, N = 2, 17, 6, 3, 6
+    inp = rand_inputs(b, L, H, P, N, R, rng)
+    grp = dict(inp, B=rng.standard_normal((b, L, G, R, N)), C=rng.standard_normal((b, L, G, R, N)))
+    rep = dict(inp, B=np.repeat(grp["B"], H // G, axis=2), C=np.repeat(grp["C"], H // G, axis=2))
+    out_g = getattr(oracle, fn)(**grp)
+    out_r = getattr(oracle, fn)(**rep)
+    if isinstance(out_g, tuple):
+        (yg, fg), (yr, fr) = out_g, out_r
+        for n in ("h", "b_prev", "x_prev", "angle"):
+            assert np.array_equal(getattr(fg, n), getattr(fr, n)), n
+    else:
+        yg, yr = out_g, out_r
+    assert np.array_equal(yg, yr)
+
+
+def test_grouped_bc_prefill_then_decode():
+    rng = np.random.default_rng(131)
+    b, L, H, P, N, R, G, k = 2, 12, 4, 3, 4, 2, 2, 7
+    inp = rand_inputs(b, L, H, P, N, R, rng)
+    inp["B"] = rng.standard_normal((b, L, G, R, N))
+    inp["C"] = rng.standard_normal((b, L, G, R, N))
+    y_all, f_all = oracle.scan_complex(**inp)
+    _, st = oracle.scan_complex(**slice_t(inp, 0, k))
+    for t in range(k, L):
+        step = {n: inp[n][:, t] for n in ("x", "B", "C", "theta", "dt", "lam")}
+        yt, st = oracle.decode_step(st, **step, A=inp["A"], D=inp["D"])
+        assert rel_err(yt, y_all[:, t]) < 1e-12
+    assert rel_err(st.h, f_all.h) < 1e-12
