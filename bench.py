@@ -43,14 +43,18 @@ FALLBACK_HBM_GBS = 6650.0
 # traffic null, since its counters are out of date.
 TRAFFIC = {
     "prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"),
-                "a613588c5d8a7a7ed3a8d0443bf6b4317e11f1585fe3846bc45bf7fd32acb056", 811438592 + 137308416,
+                "d553b6c25b666d8f4a80634013f03686f468b3f560dcd4cc96708923e1c92176", 811524352 + 136936960,
                 "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     "siso_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                         "eea54a57c8c5a78d7ea5371966f93b0c2696c767db27ec84c749b918dc4d9c7c", 283173120 + 219014656,
+                         "7ccbdf6b735872e61661a0e4d8ad33ec2f120e42692c1cc6ce802987011c2987", 283237376 + 220529664,
                          "profiles/decode_stream_b128_traffic_and_counters.txt"),
     "mimo4_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                          "eea54a57c8c5a78d7ea5371966f93b0c2696c767db27ec84c749b918dc4d9c7c", 317781504 + 240473600,
+                          "7ccbdf6b735872e61661a0e4d8ad33ec2f120e42692c1cc6ce802987011c2987", 317788672 + 239549184,
                           "profiles/decode_stream_b128_traffic_and_counters.txt"),
+    "grouped_prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"), "d553b6c25b666d8f4a80634013f03686f468b3f560dcd4cc96708923e1c92176", 284591616 + 113454080,
+                        "profiles/grouped_bc_prefill_decode_traffic.txt"),
+    "grouped_decode": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), "7ccbdf6b735872e61661a0e4d8ad33ec2f120e42692c1cc6ce802987011c2987", 279056128 + 219058176,
+                       "profiles/grouped_bc_prefill_decode_traffic.txt"),
 }
 
 
@@ -77,25 +81,28 @@ def esize(dt):
     return torch.tensor([], dtype=dt).element_size()
 
 
-def prefill_bytes(w: wl.Workload, export_state=True) -> int:
+def prefill_bytes(w: wl.Workload, export_state=True, groups=0) -> int:
     """Algorithmic bytes of one prefill: every input read once, y written once,
-    the final state written once (A, D included)."""
+    the final state written once (A, D included).  groups > 0: B and C hold
+    `groups` rows per token instead of one per head."""
     s = esize(w.dtype)
     th = w.token_heads
-    per_th = s * (2 * w.rank * w.headdim + 2 * w.rank * w.dstate + w.dstate // 2 + 2)
+    per_th = s * (2 * w.rank * w.headdim + w.dstate // 2 + 2)
+    bc = s * 2 * w.rank * w.dstate * w.batch * w.seqlen * (groups or w.nheads)
     units = w.batch * w.nheads
     state = 4 * units * (w.dstate * w.headdim + w.rank * w.dstate + w.rank * w.headdim + w.dstate // 2)
-    return th * per_th + (state if export_state else 0) + 8 * w.nheads
+    return th * per_th + bc + (state if export_state else 0) + 8 * w.nheads
 
 
-def decode_bytes(w: wl.Workload) -> int:
+def decode_bytes(w: wl.Workload, groups=0) -> int:
     """Algorithmic bytes of one decode step: the fp32 state read and written once,
-    the per-token inputs read once, y written once."""
+    the per-token inputs read once, y written once (groups as in prefill_bytes)."""
     s = esize(w.dtype)
     units = w.batch * w.nheads
     state = 4 * (w.dstate * w.headdim + w.rank * w.dstate + w.rank * w.headdim + w.dstate // 2)
-    io = s * (2 * w.rank * w.headdim + 2 * w.rank * w.dstate + w.dstate // 2 + 2)
-    return units * (2 * state + io) + 8 * w.nheads
+    io = s * (2 * w.rank * w.headdim + w.dstate // 2 + 2)
+    bc = s * 2 * w.rank * w.dstate * w.batch * (groups or w.nheads)
+    return units * (2 * state + io) + bc + 8 * w.nheads
 
 
 def measured_peaks():
@@ -276,13 +283,16 @@ def run_prefill(m3, args, world, rank, clk):
                 tokens=w.batch * w.seqlen, bytes=prefill_bytes(w))
 
 
-def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False, time_varying_a=False):
+def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False, time_varying_a=False, groups=0):
     """Median per-launch time (ms) of one prefill launch of workload `w`, inputs
     resident on the device (larger than L2), final state exported.  With
     fused_norm the launch takes raw B, C and normalises them in the kernel; with
-    time_varying_a it takes a decay rate per token (A_t) instead of A per head."""
+    time_varying_a it takes a decay rate per token (A_t) instead of A per head;
+    with groups > 0, B and C are shared by groups of nheads / groups heads."""
     dev = torch.device("cuda")
     inp = wl.make_inputs(w, seed=wl.BASE_SEED + rank, device=dev)
+    if groups:
+        inp.update(wl.grouped_bc(inp, groups, seed=wl.BASE_SEED + 6 + rank))
     norm = None
     if fused_norm:
         raw = wl.raw_bc_inputs(inp, seed=wl.BASE_SEED + 2 + rank)
@@ -323,10 +333,11 @@ def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False,
     return statistics.median(times)
 
 
-def run_decode(m3, w: wl.Workload, world, rank, steps, fused_norm=False, time_varying_a=False):
+def run_decode(m3, w: wl.Workload, world, rank, steps, fused_norm=False, time_varying_a=False, groups=0):
     """Seed the state with a 512-token prefill, then time `steps` decode steps
     captured in one CUDA graph (per-step inputs pre-generated, larger than L2).
-    With fused_norm each step takes raw B, C and normalises them in the kernel."""
+    With fused_norm each step takes raw B, C and normalises them in the kernel;
+    with groups > 0 each step's B and C are shared by groups of heads."""
     dev = torch.device("cuda")
     pre = wl.make_inputs(w.with_(seqlen=w.prefill_tokens), seed=wl.BASE_SEED + rank, device=dev)
     st = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
@@ -334,6 +345,8 @@ def run_decode(m3, w: wl.Workload, world, rank, steps, fused_norm=False, time_va
     A, D = pre["A"], pre["D"]
     del pre
     steps_in = wl.decode_inputs(w, steps, seed=wl.BASE_SEED + 1 + rank, device=dev)
+    if groups:
+        steps_in.update(wl.grouped_bc(steps_in, groups, seed=wl.BASE_SEED + 7 + rank))
     norm = None
     if fused_norm:
         raw = wl.raw_bc_inputs(steps_in, seed=wl.BASE_SEED + 3 + rank)
@@ -429,6 +442,20 @@ def ours(args):
     tva["decode_" + DECODE[0].name] = {"us_per_step": round(us, 2), "roofline": {
         "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
         "bytes_per_step": by}}
+    # grouped B/C: one B and C row per token shared by all heads (ngroups 1)
+    ms = max_over_ranks(run_prefill_plain(m3, PREFILL, rank, steps=max(5, min(args.steps, 20)), warmup=3,
+                                          groups=1), world)
+    by = prefill_bytes(PREFILL, groups=1)
+    gbs = by / (ms * 1e-3) / 1e9
+    grp = {"prefill_" + PREFILL.name: {"ngroups": 1, "ms_per_launch": round(ms, 4), "roofline": {
+        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
+        "traffic": traffic("grouped_prefill"), "bytes_per_launch": by}}}
+    us = run_decode(m3, DECODE[0], world, rank, DECODE[0].decode_steps, groups=1)
+    by = decode_bytes(DECODE[0], groups=1)
+    gbs = by / (us * 1e-6) / 1e9
+    grp["decode_" + DECODE[0].name] = {"ngroups": 1, "us_per_step": round(us, 2), "roofline": {
+        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
+        "traffic": traffic("grouped_decode"), "bytes_per_step": by}}
     more = {}
     for w in PREFILL_MORE:
         ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=max(5, min(args.steps, 20)), warmup=3), world)
@@ -465,6 +492,7 @@ def ours(args):
         "prefill_more": more,
         "fused_bc_norm": fused,
         "time_varying_decay": tva,
+        "grouped_bc": grp,
         "decode": dec,
         "e2e": {"value": round(e2e_value, 3), "unit": "Mtokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},

@@ -27,7 +27,11 @@
  *    default stream).
  *  - Layouts are dense row-major with the last index fastest:
  *      x, y      [batch, seqlen, nheads, rank, headdim]      (in_dtype)
- *      B, C      [batch, seqlen, nheads, rank, dstate]       (in_dtype)
+ *      B, C      [batch, seqlen, G, rank, dstate]            (in_dtype)
+ *                G = dims->ngroups (nheads when 0): the pages give each head
+ *                its own B and C; sharing them among G groups of consecutive
+ *                heads is the Mamba line's grouped form (head h reads row
+ *                h / (nheads / G)).
  *      theta     [batch, seqlen, nheads, dstate/2]           (in_dtype)
  *      dt, lam   [batch, seqlen, nheads]                     (in_dtype)
  *      A, D      [nheads]                                    (float32)
@@ -72,6 +76,9 @@ typedef struct {
   int rank;     /* R: 1 (SISO) or 2, 4, 8 (MIMO) */
   int chunk;    /* Q tokens per chunk for the prefill; 0 = library default */
   mamba3_dtype in_dtype; /* dtype of x, B, C, theta, dt, lam and y */
+  int ngroups;  /* G rows of B and C per token: 0 = one per head (G = nheads);
+                 * otherwise G divides nheads and heads g*(H/G) .. (g+1)*(H/G)-1
+                 * share row g.  Added in ABI 2.00. */
 } mamba3_dims;
 
 /*

@@ -45,11 +45,14 @@ class Mamba3Error(RuntimeError):
         super().__init__(f"{where}: {mamba3_status_string(code)} (status {code})")
 
 
+ABI_MAJOR = 2
+
+
 class Dims(ctypes.Structure):
     _fields_ = [
         ("batch", ctypes.c_int), ("seqlen", ctypes.c_int), ("nheads", ctypes.c_int),
         ("headdim", ctypes.c_int), ("dstate", ctypes.c_int), ("rank", ctypes.c_int),
-        ("chunk", ctypes.c_int), ("in_dtype", ctypes.c_int),
+        ("chunk", ctypes.c_int), ("in_dtype", ctypes.c_int), ("ngroups", ctypes.c_int),
     ]
 
 
@@ -89,6 +92,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba3_status_string.restype = ctypes.c_char_p
     lib.mamba3_version.argtypes = []
     lib.mamba3_version.restype = i
+    if lib.mamba3_version() // 100 != ABI_MAJOR:  # Dims must match the library's mamba3_dims
+        raise ImportError(f"{path} has ABI {lib.mamba3_version()}, this binding needs {ABI_MAJOR}.xx: rebuild it")
     lib.mamba3_scan_fwd_bcnorm.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(_CNorm),
                                            ctypes.POINTER(_CState), vp, ctypes.POINTER(_CState), vp, sz, vp]
     lib.mamba3_scan_fwd_bcnorm.restype = i
@@ -155,7 +160,7 @@ def make_dims(x: torch.Tensor, B: torch.Tensor, chunk: int = 0, decode: bool = F
         b, L, H, R, P = x.shape
     if x.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {x.dtype}")
-    return Dims(b, L, H, P, B.shape[-1], R, chunk, _DTYPES[x.dtype])
+    return Dims(b, L, H, P, B.shape[-1], R, chunk, _DTYPES[x.dtype], B.shape[-3])
 
 
 def mamba3_status_string(code: int) -> str:
@@ -175,11 +180,13 @@ def _check_inputs(x, B, C, theta, dt, lam, A, D, decode):
             raise ValueError(f"{name} must have the dtype of x ({x.dtype})")
         if t.device != x.device:
             raise ValueError(f"{name} must be on the device of x")
-    if B.shape != C.shape or B.shape[:-1] != lead + (x.shape[-2],):
-        raise ValueError("B and C must be [..., R, N] with the leading shape of x")
+    H = x.shape[-3]
+    if (B.shape != C.shape or B.dim() != x.dim() or B.shape[:-3] != x.shape[:-3] or B.shape[-2] != x.shape[-2]
+            or H % B.shape[-3] != 0):
+        raise ValueError("B and C must be [..., G, R, N] with the leading shape of x and G dividing H "
+                         "(G = H: one row per head)")
     if theta.shape != lead + (B.shape[-1] // 2,) or dt.shape != lead or lam.shape != lead:
         raise ValueError("theta must be [..., N/2] and dt, lam [...] with the leading shape of x")
-    H = x.shape[-3]
     for name, t in (("A", A), ("D", D)):
         if t is not None and (t.dtype != torch.float32 or t.shape != (H,) or not t.is_contiguous()):
             raise ValueError(f"{name} must be a contiguous float32 tensor of shape [H]")
@@ -188,8 +195,9 @@ def _check_inputs(x, B, C, theta, dt, lam, A, D, decode):
 def mamba3_scan_fwd(x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = None,
                     y: Optional[torch.Tensor] = None, final_state: Optional[State] = None,
                     workspace: Optional[torch.Tensor] = None, chunk: int = 0, stream=None):
-    """Chunked prefill. Shapes: x [b,L,H,R,P], B/C [b,L,H,R,N], theta [b,L,H,N/2],
-    dt/lam [b,L,H], A/D [H] fp32. Returns y (allocated if not given)."""
+    """Chunked prefill. Shapes: x [b,L,H,R,P], B/C [b,L,H,R,N] (or [b,L,G,R,N],
+    shared by groups of H/G consecutive heads), theta [b,L,H,N/2], dt/lam [b,L,H],
+    A/D [H] fp32. Returns y (allocated if not given)."""
     lib = load_library()
     _check_inputs(x, B, C, theta, dt, lam, A, D, decode=False)
     dims = make_dims(x, B, chunk)
@@ -209,8 +217,8 @@ def mamba3_scan_fwd(x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = 
 
 def mamba3_decode_step(state: State, x, B, C, theta, dt, lam, A, D=None, y: Optional[torch.Tensor] = None,
                        stream=None):
-    """One decode step in place on ``state``. Shapes: x [b,H,R,P], B/C [b,H,R,N],
-    theta [b,H,N/2], dt/lam [b,H]. Returns y [b,H,R,P]."""
+    """One decode step in place on ``state``. Shapes: x [b,H,R,P], B/C [b,H,R,N]
+    (or [b,G,R,N]), theta [b,H,N/2], dt/lam [b,H]. Returns y [b,H,R,P]."""
     lib = load_library()
     _check_inputs(x, B, C, theta, dt, lam, A, D, decode=True)
     dims = make_dims(x, B, decode=True)

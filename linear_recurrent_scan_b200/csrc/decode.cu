@@ -30,6 +30,12 @@
 namespace m3 {
 namespace {
 
+// Row of B and C that unit (b, h) = (u / H, u % H) reads: u itself with one row
+// per head; b * G + h / (H / G) when G groups of heads share B and C.
+__device__ __forceinline__ size_t bc_row(const DecodeArgs& a, int u) {
+  return (size_t)(u / a.nheads) * a.ngroups + (u % a.nheads) / (a.nheads / a.ngroups);
+}
+
 constexpr int kThreads = 128;
 constexpr int kMaxRows = 16;  // rows of h per thread (N <= kMaxRows * G)
 
@@ -65,8 +71,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
 
   // 2. per-token scalars, angles and rotated B, C into shared memory
   const T* xu = static_cast<const T*>(a.x) + (size_t)unit * R * P;
-  const T* Bu = static_cast<const T*>(a.B) + (size_t)unit * R * N;
-  const T* Cu = static_cast<const T*>(a.C) + (size_t)unit * R * N;
+  const T* Bu = static_cast<const T*>(a.B) + bc_row(a, unit) * R * N;
+  const T* Cu = static_cast<const T*>(a.C) + bc_row(a, unit) * R * N;
   const T* thu = static_cast<const T*>(a.theta) + (size_t)unit * K;
   const float dt = ld1(static_cast<const T*>(a.dt) + unit);
   if (tid == 0) {
@@ -250,8 +256,8 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
     ptx::bulk_load(st + S::BP, a.bprev + (size_t)u * R * N, R * N * 4, bar);
     ptx::bulk_load(st + S::XP, a.xprev + (size_t)u * R * kSP, R * kSP * 4, bar);
     ptx::bulk_load(st + S::ANG, a.angle + (size_t)u * K2, K2 * 4, bar);
-    ptx::bulk_load(st + S::B, static_cast<const T*>(a.B) + (size_t)u * R * N, R * N * sizeof(T), bar);
-    ptx::bulk_load(st + S::C, static_cast<const T*>(a.C) + (size_t)u * R * N, R * N * sizeof(T), bar);
+    ptx::bulk_load(st + S::B, static_cast<const T*>(a.B) + bc_row(a, u) * R * N, R * N * sizeof(T), bar);
+    ptx::bulk_load(st + S::C, static_cast<const T*>(a.C) + bc_row(a, u) * R * N, R * N * sizeof(T), bar);
     ptx::bulk_load(st + S::X, static_cast<const T*>(a.x) + (size_t)u * R * kSP, R * kSP * sizeof(T), bar);
     ptx::bulk_load(st + S::TH, static_cast<const T*>(a.theta) + (size_t)u * K2, K2 * sizeof(T), bar);
   };
@@ -445,6 +451,7 @@ int launch_stream(const DecodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 int decode_supported(const DecodeArgs& a) {
+  if (a.ngroups < 1 || a.nheads % a.ngroups != 0) return MAMBA3_ERR_INVALID;  // B, C rows per token
   if (a.bcnorm && !stream_ok(a)) return MAMBA3_ERR_UNSUPPORTED;  // the fused norm lives in the streaming kernel
   if (a.P % 4 != 0 || a.P / 4 > kThreads || kThreads % (a.P / 4) != 0) return MAMBA3_ERR_UNSUPPORTED;
   const int G = kThreads / (a.P / 4);

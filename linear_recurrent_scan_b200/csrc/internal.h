@@ -10,6 +10,7 @@ namespace m3 {
 
 struct ScanArgs {
   int batch, seqlen, nheads, P, N, R, Q;
+  int ngroups;  // B, C rows per (batch, token): nheads, or G dividing it (head h reads row h / (nheads / G))
   mamba3_dtype dtype;
   const void *x, *B, *C, *theta, *dt, *lam;
   const float *A, *D;  // A null when A_t is given
@@ -27,6 +28,7 @@ struct ScanArgs {
 
 struct DecodeArgs {
   int batch, nheads, P, N, R;
+  int ngroups;  // as in ScanArgs
   mamba3_dtype dtype;
   float *h, *bprev, *xprev, *angle;
   const void *x, *B, *C, *theta, *dt, *lam;

@@ -22,6 +22,7 @@ int check_dims(const mamba3_dims* d, bool need_seqlen) {
   if (!(d->rank == 1 || d->rank == 2 || d->rank == 4 || d->rank == 8)) return MAMBA3_ERR_INVALID;
   if (d->in_dtype != MAMBA3_F32 && d->in_dtype != MAMBA3_BF16) return MAMBA3_ERR_INVALID;
   if (need_seqlen && d->chunk < 0) return MAMBA3_ERR_INVALID;
+  if (d->ngroups < 0 || (d->ngroups > 0 && d->nheads % d->ngroups != 0)) return MAMBA3_ERR_INVALID;
   // every flattened index must fit comfortably in 64 bits and the grid in 31
   const double tokens = (double)d->batch * (need_seqlen ? (d->seqlen > 0 ? d->seqlen : 1) : 1) * d->nheads;
   const double row = (double)d->rank * (d->dstate > d->headdim ? d->dstate : d->headdim);
@@ -29,6 +30,9 @@ int check_dims(const mamba3_dims* d, bool need_seqlen) {
   if (d->dstate > 1024 || d->headdim > 1024) return MAMBA3_ERR_UNSUPPORTED;
   return MAMBA3_OK;
 }
+
+// B, C rows per (batch, token): 0 in the dims means one per head.
+int bc_groups(const mamba3_dims* d) { return d->ngroups > 0 ? d->ngroups : d->nheads; }
 
 int check_state(const mamba3_state* s) {
   if (!s) return MAMBA3_OK;
@@ -63,7 +67,7 @@ void set_norm(Args& a, const mamba3_bc_norm* n) {
 
 extern "C" {
 
-int mamba3_version(void) { return 100; }
+int mamba3_version(void) { return 200; }
 
 const char* mamba3_status_string(int status) {
   switch (status) {
@@ -85,12 +89,12 @@ size_t mamba3_scan_workspace_bytes(const mamba3_dims* d) {
 }  // extern "C"
 
 namespace {
-// The prefill behind mamba3_scan_fwd (A per head) and mamba3_scan_fwd_at (A_t
-// per token; A null).
+// The prefill behind mamba3_scan_fwd (A per head), mamba3_scan_fwd_at (A_t per
+// token; A null) and mamba3_scan_fwd_bcnorm (norm non-null, already checked).
 int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
                   const void* dt, const void* lam, const float* A, const void* A_t, const float* D,
-                  const mamba3_state* init, void* y, const mamba3_state* final_state, void* workspace,
-                  size_t workspace_bytes, void* stream) {
+                  const mamba3_bc_norm* norm, const mamba3_state* init, void* y,
+                  const mamba3_state* final_state, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_dims(d, true);
   if (rc) return rc;
   const float* A_chk = A ? A : static_cast<const float*>(A_t);  // the rate array that must be present
@@ -109,6 +113,7 @@ int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
   a.N = d->dstate;
   a.R = d->rank;
   a.Q = d->chunk;
+  a.ngroups = bc_groups(d);
   a.dtype = d->in_dtype;
   a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.A_t = A_t; a.D = D;
   if (init) { a.h0 = init->h; a.bprev0 = init->b_prev; a.xprev0 = init->x_prev; a.angle0 = init->angle; }
@@ -119,8 +124,10 @@ int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
   }
   a.workspace = workspace;
   a.workspace_bytes = workspace_bytes;
+  if (norm && d->seqlen > 0) set_norm(a, norm);  // with no tokens there is nothing to normalise
 
   const bool use_tc = m3::tc_scan_supported(a) == MAMBA3_OK;
+  if (!use_tc && a.bcnorm) return MAMBA3_ERR_UNSUPPORTED;  // the fused form is tensor-core only
   if (!use_tc && (rc = m3::simt_scan_supported(a))) return rc;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -128,10 +135,11 @@ int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
   return use_tc ? m3::launch_scan_tc(a, s) : m3::launch_scan_simt(a, s);
 }
 
-// The decode step behind mamba3_decode_step and mamba3_decode_step_at.
+// The decode step behind mamba3_decode_step, mamba3_decode_step_at and
+// mamba3_decode_step_bcnorm (norm non-null, already checked).
 int decode_impl(const mamba3_dims* d, const mamba3_state* state, const void* x, const void* B, const void* C,
                 const void* theta, const void* dt, const void* lam, const float* A, const void* A_t,
-                const float* D, void* y, void* stream) {
+                const float* D, const mamba3_bc_norm* norm, void* y, void* stream) {
   int rc = check_dims(d, false);
   if (rc) return rc;
   if (!state) return MAMBA3_ERR_INVALID;
@@ -145,9 +153,11 @@ int decode_impl(const mamba3_dims* d, const mamba3_state* state, const void* x, 
   a.P = d->headdim;
   a.N = d->dstate;
   a.R = d->rank;
+  a.ngroups = bc_groups(d);
   a.dtype = d->in_dtype;
   a.h = state->h; a.bprev = state->b_prev; a.xprev = state->x_prev; a.angle = state->angle;
   a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.A_t = A_t; a.D = D; a.y = y;
+  if (norm) set_norm(a, norm);
   if ((rc = m3::decode_supported(a))) return rc;
   return m3::launch_decode(a, static_cast<cudaStream_t>(stream));
 }
@@ -159,8 +169,8 @@ int mamba3_scan_fwd(const mamba3_dims* d, const void* x, const void* B, const vo
                     const void* dt, const void* lam, const float* A, const float* D,
                     const mamba3_state* init, void* y, const mamba3_state* final_state, void* workspace,
                     size_t workspace_bytes, void* stream) {
-  return scan_fwd_impl(d, x, B, C, theta, dt, lam, A, nullptr, D, init, y, final_state, workspace, workspace_bytes,
-                       stream);
+  return scan_fwd_impl(d, x, B, C, theta, dt, lam, A, nullptr, D, nullptr, init, y, final_state, workspace,
+                       workspace_bytes, stream);
 }
 
 int mamba3_scan_fwd_at(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
@@ -168,7 +178,7 @@ int mamba3_scan_fwd_at(const mamba3_dims* d, const void* x, const void* B, const
                        void* y, const mamba3_state* final_state, void* workspace, size_t workspace_bytes,
                        void* stream) {
   if (!A_t) return MAMBA3_ERR_INVALID;
-  return scan_fwd_impl(d, x, B, C, theta, dt, lam, nullptr, A_t, D, init, y, final_state, workspace,
+  return scan_fwd_impl(d, x, B, C, theta, dt, lam, nullptr, A_t, D, nullptr, init, y, final_state, workspace,
                        workspace_bytes, stream);
 }
 
@@ -176,65 +186,29 @@ int mamba3_decode_step_at(const mamba3_dims* d, const mamba3_state* state, const
                           const void* C, const void* theta, const void* dt, const void* lam, const void* A_t,
                           const float* D, void* y, void* stream) {
   if (!A_t) return MAMBA3_ERR_INVALID;
-  return decode_impl(d, state, x, B, C, theta, dt, lam, nullptr, A_t, D, y, stream);
+  return decode_impl(d, state, x, B, C, theta, dt, lam, nullptr, A_t, D, nullptr, y, stream);
 }
 
 int mamba3_scan_fwd_bcnorm(const mamba3_dims* d, const void* x, const void* B_raw, const void* C_raw,
                            const void* theta, const void* dt, const void* lam, const float* A, const float* D,
                            const mamba3_bc_norm* norm, const mamba3_state* init, void* y,
                            const mamba3_state* final_state, void* workspace, size_t workspace_bytes, void* stream) {
-  int rc = check_dims(d, true);
-  if (rc) return rc;
   if (!norm_ok(norm)) return MAMBA3_ERR_INVALID;
-  if (d->seqlen == 0)  // nothing to normalise: the state passes through
-    return mamba3_scan_fwd(d, x, B_raw, C_raw, theta, dt, lam, A, D, init, y, final_state, workspace,
-                           workspace_bytes, stream);
-  if ((rc = check_inputs(x, B_raw, C_raw, theta, dt, lam, A, D, y))) return rc;
-  if ((rc = check_state(init)) || (rc = check_state(final_state))) return rc;
-  if (!workspace || !aligned16(workspace)) return MAMBA3_ERR_WORKSPACE;
-  if (workspace_bytes < mamba3_scan_workspace_bytes(d)) return MAMBA3_ERR_WORKSPACE;
-  m3::ScanArgs a;
-  memset(&a, 0, sizeof(a));
-  a.batch = d->batch; a.seqlen = d->seqlen; a.nheads = d->nheads; a.P = d->headdim; a.N = d->dstate;
-  a.R = d->rank; a.Q = d->chunk; a.dtype = d->in_dtype;
-  a.x = x; a.B = B_raw; a.C = C_raw; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.D = D;
-  if (init) { a.h0 = init->h; a.bprev0 = init->b_prev; a.xprev0 = init->x_prev; a.angle0 = init->angle; }
-  a.y = y;
-  if (final_state) {
-    a.h_out = final_state->h; a.bprev_out = final_state->b_prev;
-    a.xprev_out = final_state->x_prev; a.angle_out = final_state->angle;
-  }
-  a.workspace = workspace;
-  a.workspace_bytes = workspace_bytes;
-  set_norm(a, norm);
-  if (m3::tc_scan_supported(a) != MAMBA3_OK) return MAMBA3_ERR_UNSUPPORTED;  // the fused form is tensor-core only
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
-  return m3::launch_scan_tc(a, s);
+  return scan_fwd_impl(d, x, B_raw, C_raw, theta, dt, lam, A, nullptr, D, norm, init, y, final_state, workspace,
+                       workspace_bytes, stream);
 }
 
 int mamba3_decode_step_bcnorm(const mamba3_dims* d, const mamba3_state* state, const void* x, const void* B_raw,
                               const void* C_raw, const void* theta, const void* dt, const void* lam, const float* A,
                               const float* D, const mamba3_bc_norm* norm, void* y, void* stream) {
-  int rc = check_dims(d, false);
-  if (rc) return rc;
-  if (!state || !norm_ok(norm)) return MAMBA3_ERR_INVALID;
-  if ((rc = check_state(state))) return rc;
-  if ((rc = check_inputs(x, B_raw, C_raw, theta, dt, lam, A, D, y))) return rc;
-  m3::DecodeArgs a;
-  memset(&a, 0, sizeof(a));
-  a.batch = d->batch; a.nheads = d->nheads; a.P = d->headdim; a.N = d->dstate; a.R = d->rank; a.dtype = d->in_dtype;
-  a.h = state->h; a.bprev = state->b_prev; a.xprev = state->x_prev; a.angle = state->angle;
-  a.x = x; a.B = B_raw; a.C = C_raw; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.D = D; a.y = y;
-  set_norm(a, norm);
-  if ((rc = m3::decode_supported(a))) return rc;
-  return m3::launch_decode(a, static_cast<cudaStream_t>(stream));
+  if (!norm_ok(norm)) return MAMBA3_ERR_INVALID;
+  return decode_impl(d, state, x, B_raw, C_raw, theta, dt, lam, A, nullptr, D, norm, y, stream);
 }
 
 int mamba3_decode_step(const mamba3_dims* d, const mamba3_state* state, const void* x, const void* B,
                        const void* C, const void* theta, const void* dt, const void* lam, const float* A,
                        const float* D, void* y, void* stream) {
-  return decode_impl(d, state, x, B, C, theta, dt, lam, A, nullptr, D, y, stream);
+  return decode_impl(d, state, x, B, C, theta, dt, lam, A, nullptr, D, nullptr, y, stream);
 }
 
 int mamba3_device_status(const void* workspace, void* stream) {

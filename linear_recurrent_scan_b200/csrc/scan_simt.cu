@@ -89,6 +89,8 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(ScanArgs a, SimtLay
   T* Y = static_cast<T*>(a.y);
   const size_t us = (size_t)unit;
   auto tok = [&](int t) { return ((size_t)b * L + t) * a.nheads + hh; };
+  const int gh = hh / (a.nheads / a.ngroups);  // B, C row of this head
+  auto tok_bc = [&](int t) { return ((size_t)b * L + t) * a.ngroups + gh; };
 
   // ---- initial state: hbar_0 = h_0 + (1 - lam_1) dt_1 B~_0^T x_0 ----
   const bool has_init = a.h0 != nullptr;
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(ScanArgs a, SimtLay
     // ---- raw B, C, x rows ----
     for (int i = tid; i < M * N; i += kThreads) {
       const int m = i / N, n = i % N;
-      const size_t g = tok(t0 + m / R) * R * N + (size_t)(m % R) * N + n;
+      const size_t g = tok_bc(t0 + m / R) * R * N + (size_t)(m % R) * N + n;
       sB[i] = ld1(Bg + g);
       sC[i] = ld1(Cg + g);
     }
@@ -223,6 +225,7 @@ int default_q(const ScanArgs& a) { return a.Q > 0 ? a.Q : kMaxRows / a.R; }
 }  // namespace
 
 int simt_scan_supported(const ScanArgs& a) {
+  if (a.ngroups < 1 || a.nheads % a.ngroups != 0) return MAMBA3_ERR_INVALID;  // B, C rows per token
   const int Q = default_q(a);
   if (Q < 1 || Q * a.R > kMaxRows) return MAMBA3_ERR_UNSUPPORTED;
   if (simt_layout(a.P, a.N, a.R, Q).total > 220 * 1024) return MAMBA3_ERR_UNSUPPORTED;

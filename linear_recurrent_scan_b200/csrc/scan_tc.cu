@@ -748,6 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       //   theta (+ dt, lam) of chunk ct once prep has read chunk ct - 1's.
       // One thread polls the three conditions (non-blocking), so no stream waits behind another.
       int cb = 0, cx = 0, ct = 0;
+      const int gh = hh / (prm.a.nheads / prm.a.ngroups);  // the B/C row this head reads
       long long t_last = clock64();
       const uint32_t th_bytes =
           K::TH_BYTES + (prm.dl_tma ? 2u * K::DL_BYTES : 0u) + (prm.at_tma ? (uint32_t)K::AT_BYTES : 0u);
@@ -759,8 +760,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&bars[bFull0 + s], K::TMA_BYTES);  // B, C and x of chunk cb
 #pragma unroll
           for (int kb = 0; kb < K::NKB; ++kb) {
-            tma_load_5d(st + K::OFF_B + kb * kTile, &tmB, &bars[bFull0 + s], kb * 64, 0, hh, t0, b);
-            tma_load_5d(st + K::OFF_C + kb * kTile, &tmC, &bars[bFull0 + s], kb * 64, 0, hh, t0, b);
+            tma_load_5d(st + K::OFF_B + kb * kTile, &tmB, &bars[bFull0 + s], kb * 64, 0, gh, t0, b);
+            tma_load_5d(st + K::OFF_C + kb * kTile, &tmC, &bars[bFull0 + s], kb * 64, 0, gh, t0, b);
           }
           ++cb;
           progress = true;
@@ -890,14 +891,14 @@ EncodeTiledFn encode_fn() {
 
 // [batch, L, H, R, inner] bf16 tensor, box = {64, R, 1, Q, 1}, 128-byte swizzle,
 // zero fill past the end of the sequence.
-bool make_map(CUtensorMap* m, const void* base, int inner, const ScanArgs& a, int Q) {
+bool make_map(CUtensorMap* m, const void* base, int inner, int heads, const ScanArgs& a, int Q) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const cuuint64_t dims[5] = {(cuuint64_t)inner, (cuuint64_t)a.R, (cuuint64_t)a.nheads, (cuuint64_t)a.seqlen,
+  const cuuint64_t dims[5] = {(cuuint64_t)inner, (cuuint64_t)a.R, (cuuint64_t)heads, (cuuint64_t)a.seqlen,
                               (cuuint64_t)a.batch};
   const cuuint64_t e = 2;
-  const cuuint64_t strides[4] = {e * inner, e * inner * a.R, e * inner * a.R * a.nheads,
-                                 e * inner * a.R * a.nheads * a.seqlen};
+  const cuuint64_t strides[4] = {e * inner, e * inner * a.R, e * inner * a.R * heads,
+                                 e * inner * a.R * heads * a.seqlen};
   const cuuint32_t box[5] = {64, (cuuint32_t)a.R, 1, (cuuint32_t)Q, 1};
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
@@ -938,7 +939,8 @@ template <int N, int R>
 int launch_nr(const ScanArgs& a, cudaStream_t s) {
   using K = Cfg<N, R>;
   CUtensorMap tmB, tmC, tmX, tmT;
-  if (!make_map(&tmB, a.B, N, a, K::Q) || !make_map(&tmC, a.C, N, a, K::Q) || !make_map(&tmX, a.x, kP, a, K::Q) ||
+  if (!make_map(&tmB, a.B, N, a.ngroups, a, K::Q) || !make_map(&tmC, a.C, N, a.ngroups, a, K::Q) ||
+      !make_map(&tmX, a.x, kP, a.nheads, a, K::Q) ||
       !make_theta_map(&tmT, a, K::Q))
     return MAMBA3_ERR_CUDA;
   TcParams prm;
@@ -964,6 +966,7 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
 }  // namespace
 
 int tc_scan_supported(const ScanArgs& a) {
+  if (a.ngroups < 1 || a.nheads % a.ngroups != 0) return MAMBA3_ERR_INVALID;  // B, C rows per token
   if (a.dtype != MAMBA3_BF16 || a.P != kP || a.seqlen < 1) return MAMBA3_ERR_UNSUPPORTED;
   if (a.N != 64 && a.N != 128) return MAMBA3_ERR_UNSUPPORTED;
   if (a.R != 1 && a.R != 2 && a.R != 4) return MAMBA3_ERR_UNSUPPORTED;

@@ -2,6 +2,7 @@
 
     python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --batch 2 --reps 3
     python -m linear_recurrent_scan_b200.profile_case --workload siso_decode_b128 --decode --reps 3
+    python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --groups 1 --reps 3
 
 Inputs are seeded synthetic tensors on cuda:0.  Prints the CUDA-event time
 of each call; under a profiler those times are not benchmark numbers.
@@ -25,6 +26,7 @@ def main():
     ap.add_argument("--seqlen", type=int, default=0, help="override the sequence length (0 = workload's)")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--decode", action="store_true", help="time decode steps instead of the prefill")
+    ap.add_argument("--groups", type=int, default=0, help="B, C shared by this many groups of heads (0 = per head)")
     args = ap.parse_args()
     w = wl.CONFIGS[args.workload]
     if args.batch:
@@ -38,6 +40,8 @@ def main():
         pre = wl.make_inputs(w.with_(seqlen=max(1, w.prefill_tokens)), device=dev)
         m3.mamba3_scan_fwd(*(pre[n] for n in NAMES), pre["A"], pre["D"], final_state=st)
         steps = wl.decode_inputs(w, args.reps, device=dev)
+        if args.groups:
+            steps.update(wl.grouped_bc(steps, args.groups))
         for i in range(args.reps):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
@@ -47,6 +51,8 @@ def main():
             print(f"decode step {i}: {e0.elapsed_time(e1) * 1000:.1f} us")
         return
     inp = wl.make_inputs(w, device=dev)
+    if args.groups:
+        inp.update(wl.grouped_bc(inp, args.groups))
     y = torch.empty_like(inp["x"])
     for i in range(args.reps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

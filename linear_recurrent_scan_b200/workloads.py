@@ -12,7 +12,8 @@ projections that feed the layer):
 * x ~ N(0, 1)
 * B, C ~ N(0, 1), RMS-normalised over N per (b, t, h, r) (eps 1e-6, unit
   weight; the "BC norm" of the Mamba-3 block) plus a head-specific
-  channel-wise bias [H, R, N] ~ N(0, 0.1^2)
+  channel-wise bias [H, R, N] ~ N(0, 0.1^2); grouped B, C (shared by several
+  heads) the same without the bias
 * dt = clamp(softplus(z + b_h), 1e-3, 0.1), z ~ N(0, 1), with
   b_h = softplus^-1(dt0_h) and dt0_h log-uniform in [1e-3, 0.1]
 * A_h = -exp(U(0, log 16))  (one real scalar per head, in [-16, -1])
@@ -167,6 +168,19 @@ def raw_bc_inputs(inp: Dict[str, torch.Tensor], seed: int = BASE_SEED + 2) -> Di
     for name in ("bias_B", "bias_C"):
         out[name] = torch.randn(H, R, N, generator=g, device=dev) * 0.1
     return out
+
+
+def grouped_bc(inp: Dict[str, torch.Tensor], ngroups: int, seed: int = BASE_SEED + 5) -> Dict[str, torch.Tensor]:
+    """B and C shared by ``ngroups`` groups of heads: [..., G, R, N] in place of
+    inp["B"], inp["C"] [..., H, R, N] (dtype and device kept), drawn like the
+    per-head rows but without the head-specific bias, which a row shared by
+    several heads cannot carry."""
+    B = inp["B"]
+    *lead, H, R, N = B.shape
+    assert H % ngroups == 0
+    g = _gen(B.device, seed)
+    shape = (*lead, ngroups, R, N)
+    return {name: _bc(shape, 0.0, g, B.device).to(B.dtype).contiguous() for name in ("B", "C")}
 
 
 def decay_rates(like: torch.Tensor, seed: int = BASE_SEED + 4) -> torch.Tensor:

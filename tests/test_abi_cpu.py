@@ -60,7 +60,7 @@ def test_status_strings(lib):
     for c in (-1, -2, -3, -4, -5):
         assert m3.mamba3_status_string(c) != "unknown status"
     assert m3.mamba3_status_string(17) == "unknown status"
-    assert lib.mamba3_version() >= 100
+    assert lib.mamba3_version() // 100 == m3.ABI_MAJOR == 2
 
 
 def dims(**kw):
@@ -72,6 +72,7 @@ def dims(**kw):
 @pytest.mark.parametrize("bad", [
     dict(batch=0), dict(nheads=0), dict(headdim=6), dict(headdim=0), dict(dstate=15), dict(dstate=0),
     dict(rank=3), dict(rank=0), dict(in_dtype=7), dict(seqlen=-1), dict(chunk=-2),
+    dict(ngroups=-1), dict(ngroups=2), dict(ngroups=6),
 ])
 def test_workspace_bytes_rejects_bad_dims(lib, bad):
     assert lib.mamba3_scan_workspace_bytes(ctypes.byref(dims(**bad))) == 0
@@ -184,6 +185,8 @@ def test_bcnorm_entry_points_validate_on_host(lib):
     # the fused form runs on the tensor-core path only (bf16, P = 64, N in {64, 128})
     assert scan_bcn(lib, dims(in_dtype=m3.MAMBA3_F32), ok) == m3.MAMBA3_ERR_UNSUPPORTED
     assert decode_bcn(lib, dims(), None) == m3.MAMBA3_ERR_INVALID
+    assert scan_bcn(lib, dims(ngroups=2), ok) == m3.MAMBA3_ERR_INVALID                 # 2 groups, 3 heads
+    assert decode_bcn(lib, dims(ngroups=2), ok) == m3.MAMBA3_ERR_INVALID
     assert decode_bcn(lib, dims(headdim=32), ok) == m3.MAMBA3_ERR_UNSUPPORTED            # streaming kernel: P = 64
 
 
@@ -199,3 +202,29 @@ def test_time_varying_decay_entry_points_validate_on_host(lib):
     rc = lib.mamba3_decode_step_at(ctypes.byref(dims()), ctypes.byref(cs), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
                                    None, FAKE, None)
     assert rc == m3.MAMBA3_ERR_INVALID
+
+
+def test_grouped_bc_dims(lib):
+    """ngroups: 0 (one B/C row per head) or a divisor of nheads; the valid forms
+    pass the host checks and, with no GPU, fail in CUDA."""
+    for g in (0, 1, 3):
+        assert lib.mamba3_scan_workspace_bytes(ctypes.byref(dims(ngroups=g))) >= 256
+        assert scan(lib, dims(ngroups=g)) == m3.MAMBA3_ERR_CUDA
+        assert decode(lib, dims(ngroups=g)) == m3.MAMBA3_ERR_CUDA
+    assert scan(lib, dims(ngroups=2)) == m3.MAMBA3_ERR_INVALID
+    assert decode(lib, dims(ngroups=2)) == m3.MAMBA3_ERR_INVALID
+
+
+def test_python_binding_infers_groups(lib):
+    x = torch.zeros(1, 4, 6, 1, 8, dtype=torch.bfloat16)
+    th = torch.zeros(1, 4, 6, 8, dtype=torch.bfloat16)
+    dt = torch.zeros(1, 4, 6, dtype=torch.bfloat16)
+    for G in (1, 2, 3, 6):
+        B = torch.zeros(1, 4, G, 1, 16, dtype=torch.bfloat16)
+        assert m3.make_dims(x, B).ngroups == G
+    with pytest.raises(ValueError):  # 4 groups do not divide 6 heads
+        m3.mamba3_scan_fwd(x, *(2 * [torch.zeros(1, 4, 4, 1, 16, dtype=torch.bfloat16)]), th, dt, dt,
+                           torch.zeros(6))
+    with pytest.raises(ValueError):  # grouped B with a per-head C
+        m3.mamba3_scan_fwd(x, torch.zeros(1, 4, 2, 1, 16, dtype=torch.bfloat16),
+                           torch.zeros(1, 4, 6, 1, 16, dtype=torch.bfloat16), th, dt, dt, torch.zeros(6))
