@@ -60,6 +60,17 @@ class _IO(ctypes.Structure):
             "y", "h_out", "bprev_out", "xprev_out", "angle_out",
             "A_t",
         )
+    ] + [("grad", ctypes.c_void_p)]
+
+
+class _Grad(ctypes.Structure):
+    _fields_ = [
+        (n, _P)
+        for n in (
+            "dy", "dh_out", "dbprev_out", "dxprev_out", "dangle_out",
+            "dx", "dB", "dC", "dtheta", "ddt", "dlam", "dA", "dD",
+            "dh0", "dbprev0", "dxprev0", "dangle0",
+        )
     ]
 
 
@@ -76,6 +87,8 @@ def _bind(lib):
         f = getattr(lib, name)
         f.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_IO), ctypes.c_int]
         f.restype = ctypes.c_int
+    lib.m3o_scan_rope_bwd.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_IO), ctypes.c_int]
+    lib.m3o_scan_rope_bwd.restype = ctypes.c_int
     lib.m3o_bc_norm.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.c_double, _P]
     lib.m3o_bc_norm.restype = ctypes.c_int
     return lib
@@ -209,7 +222,65 @@ def decode_step(state: State, x, B, C, theta, dt, lam, A, D=None, nthreads=None)
     return y[:, 0], fin
 
 
-__all__ = ["build", "State", "scan_complex", "scan_rope", "scan_quadratic", "decode_step", "bc_norm"]
+def scan_bwd(x, B, C, theta, dt, lam, A, D, dy, init: Optional[State] = None,
+             d_final: Optional[State] = None, nthreads=None) -> dict:
+    """Gradients of the prefill (y and, with ``d_final``, the exported state) by
+    reverse-mode differentiation of the RoPE form, token by token (the pages give
+    no gradient formulas; the oracle's C source states the steps).
+
+    dy is shaped like x; ``d_final`` holds the gradients of the exported state.
+    Returns a dict: dx, dB, dC (shaped like x, B, C; grouped B, C get their
+    heads' sums), dtheta, ddt, dlam (like theta, dt, lam), dA (like A: [H]
+    summed over batch and tokens, or [b, L, H]), dD ([H]), and dh0, dbprev0,
+    dxprev0, dangle0 (the initial state's, zero-state inputs included)."""
+    dims, arrs = _prepare(x, B, C, theta, dt, lam, A, D)
+    x, B, C, theta, dt, lam, A, D = arrs
+    b, L, H, R, P = x.shape
+    N = B.shape[-1]
+    G = B.shape[2]
+    dy = _f64(dy)
+    assert dy.shape == x.shape, "dy must be shaped like x"
+    A_t = None
+    if A.ndim == 3:
+        A_t, A = A, np.zeros(H)
+    out = {
+        "dx": np.zeros_like(x), "dB": np.zeros((b, L, H, R, N)), "dC": np.zeros((b, L, H, R, N)),
+        "dtheta": np.zeros_like(theta), "ddt": np.zeros_like(dt), "dlam": np.zeros_like(lam),
+        "dA": np.zeros((b, L, H)) if A_t is not None else np.zeros((b, H)), "dD": np.zeros((b, H)),
+    }
+    st0 = State.zeros(b, H, P, N, R)
+    out.update(dh0=st0.h.copy(), dbprev0=st0.b_prev.copy(), dxprev0=st0.x_prev.copy(), dangle0=st0.angle.copy())
+    keep = [x, B, C, theta, dt, lam, A, A_t, D, dy]
+    io = _IO()
+    io.x, io.B, io.C, io.theta, io.dt, io.lam, io.A, io.D = map(_ptr, (x, B, C, theta, dt, lam, A, D))
+    io.A_t = _ptr(A_t)
+    if init is not None:
+        ih, ib, ix, ia = (_f64(init.h), _f64(init.b_prev), _f64(init.x_prev), _f64(init.angle))
+        keep += [ih, ib, ix, ia]
+        io.h0, io.bprev0, io.xprev0, io.angle0 = map(_ptr, (ih, ib, ix, ia))
+    gr = _Grad()
+    gr.dy = _ptr(dy)
+    if d_final is not None:
+        fh, fb, fx, fa = (_f64(d_final.h), _f64(d_final.b_prev), _f64(d_final.x_prev), _f64(d_final.angle))
+        keep += [fh, fb, fx, fa]
+        gr.dh_out, gr.dbprev_out, gr.dxprev_out, gr.dangle_out = map(_ptr, (fh, fb, fx, fa))
+    for n in ("dx", "dB", "dC", "dtheta", "ddt", "dlam", "dA", "dD", "dh0", "dbprev0", "dxprev0", "dangle0"):
+        setattr(gr, n, _ptr(out[n]))
+    io.grad = ctypes.cast(ctypes.pointer(gr), ctypes.c_void_p)
+    nt = nthreads if nthreads is not None else (os.cpu_count() or 1)
+    rc = _load().m3o_scan_rope_bwd(ctypes.byref(dims), ctypes.byref(io), nt)
+    if rc != 0:
+        raise ValueError(f"m3o_scan_rope_bwd rejected its arguments (rc={rc})")
+    if G != H:  # a shared row's gradient is the sum over the heads that read it
+        out["dB"] = out["dB"].reshape(b, L, G, H // G, R, N).sum(axis=3)
+        out["dC"] = out["dC"].reshape(b, L, G, H // G, R, N).sum(axis=3)
+    if A_t is None:
+        out["dA"] = out["dA"].sum(axis=0)
+    out["dD"] = out["dD"].sum(axis=0)
+    return out
+
+
+__all__ = ["build", "State", "scan_complex", "scan_rope", "scan_quadratic", "decode_step", "bc_norm", "scan_bwd"]
 
 
 def bc_norm(z, w=None, bias=None, eps: float = 1e-6) -> np.ndarray:

@@ -30,7 +30,9 @@
  *   m3o_scan_quadratic  -- the L x L masked-kernel ("quadratic") form, brute
  *                          force, for tiny inputs.
  * plus m3o_decode_step, which is one token of m3o_scan_complex continued
- * from a state, and m3o_bc_norm, the RMS normalisation of raw B or C
+ * from a state; m3o_scan_rope_bwd, the gradients of the prefill by reverse-mode
+ * differentiation of the RoPE form (the pages give no gradient formulas; it is
+ * pinned against finite differences of m3o_scan_complex); and m3o_bc_norm, the RMS normalisation of raw B or C
  * projections over the state dimension with a per-(head, rank) weight and bias
  * (same page, section 2: "BC norm" and head-specific B/C bias), which the
  * recurrence then consumes.
@@ -65,6 +67,7 @@ typedef struct {
   double *y;                                            /* may be NULL */
   double *h_out, *bprev_out, *xprev_out, *angle_out;    /* all NULL = no export */
   const double* A_t; /* NULL, or a time-varying decay [b, L, H] that replaces A[h] token by token */
+  const struct m3o_grad* grad; /* the backward pass's gradients (m3o_scan_rope_bwd only) */
 } m3o_io;
 
 /* The decay rate of token t: A_t[b, t, h] when given (section 1.1 writes the
@@ -267,6 +270,237 @@ static void unit_rope(const m3o_dims* d, const m3o_io* io, int b, int h) {
 }
 
 /* ------------------------------------------------------------------------- */
+/* backward: reverse-mode gradient of the RoPE-form recurrence                 */
+/* ------------------------------------------------------------------------- */
+/*
+ * The pages give no gradient formulas; this is the chain rule applied to
+ * unit_rope's steps, token by token from the last to the first, with the
+ * forward states h_t kept from a first pass (gh = dL/dh_t, gu = dL/du_t):
+ *   y_t = C~_t^T h_t + D x_t      gh_t += C~_t dy_t,  dC~_t[r] = h_t dy_t[r],  dD += <dy_t, x_t>
+ *   h_t = alpha_t h_{t-1} + beta_t u_{t-1} + gamma_t u_t
+ *                                 d alpha_t = <gh_t, h_{t-1}>, d beta_t = <gh_t, u_{t-1}>,
+ *                                 d gamma_t = <gh_t, u_t>, gu_t += gamma_t gh_t,
+ *                                 gu_{t-1} += beta_t gh_t, gh_{t-1} = alpha_t gh_t
+ *   u_t = sum_r B~_t[r] x_t[r]^T  dB~_t[r] = gu_t x_t[r],  dx_t[r] += gu_t^T B~_t[r]
+ *   alpha = exp(dt a), beta = (1 - lam) dt alpha, gamma = lam dt    (into dt, lam, a)
+ *   (B~0, B~1) = rot(-Phi)(B0, B1) dB = rot(+Phi) dB~,  dPhi += dB~0 B~1 - dB~1 B~0  (B and C)
+ *   Phi_t = Phi_{t-1} + dt_t theta_t
+ *                                 S_t = d angle_out + sum_{s >= t} dPhi_s,
+ *                                 dtheta_t = dt_t S_t,  ddt_t += <theta_t, S_t>
+ * The exported state (h_{L-1}, B~_{L-1}, x_{L-1}, Phi_{L-1}) adds its gradients
+ * at t = L - 1; those of the initial state (h_0, B~_0, x_0, Phi_0) come out after
+ * t = 0.  dB and dC are written per head (a caller with grouped B, C sums them
+ * over each group); dA and dD per (batch, head), or dA per token with A_t.
+ */
+typedef struct m3o_grad {
+  const double* dy;                                              /* [b, L, H, R, P] */
+  const double *dh_out, *dbprev_out, *dxprev_out, *dangle_out;   /* each NULL = zero */
+  double* dx;                                                    /* [b, L, H, R, P] */
+  double *dB, *dC;                                               /* per head [b, L, H, R, N] */
+  double *dtheta, *ddt, *dlam;                                   /* [b, L, H, N/2], [b, L, H], [b, L, H] */
+  double *dA, *dD;                                               /* [b, H] ([b, L, H] for dA with A_t) */
+  double *dh0, *dbprev0, *dxprev0, *dangle0;                     /* each NULL = not wanted */
+} m3o_grad;
+
+/* u = sum_r Bt[r] x[r]^T */
+static void outer_sum(int N, int P, int R, const double* Bt, const double* x, double* u) {
+  for (int n = 0; n < N; ++n)
+    for (int p = 0; p < P; ++p) {
+      double s = 0;
+      for (int r = 0; r < R; ++r) s += Bt[r * N + n] * x[r * P + p];
+      u[n * P + p] = s;
+    }
+}
+
+static double dot(const double* a, const double* b, size_t n) {
+  double s = 0;
+  for (size_t i = 0; i < n; ++i) s += a[i] * b[i];
+  return s;
+}
+
+static void unit_rope_bwd(const m3o_dims* d, const m3o_io* io, int b, int h) {
+  const m3o_grad* g = io->grad;
+  const int L = d->seqlen, P = d->headdim, N = d->dstate, R = d->rank, K = N / 2;
+  const size_t NP = (size_t)N * P;
+  const double Dh = io->D ? io->D[h] : 0.0;
+  const size_t us = ix_state(d, b, h);
+  double* Hs = calloc((size_t)(L + 1) * NP, sizeof(double)); /* Hs[t + 1] = h_t, Hs[0] = h_{-1} */
+  double* Bt = calloc((size_t)(L > 0 ? L : 1) * R * N, sizeof(double));
+  double* Ct = calloc((size_t)(L > 0 ? L : 1) * R * N, sizeof(double));
+  double* Ph = calloc((size_t)(L > 0 ? L : 1) * K, sizeof(double));
+  double* Phi = calloc((size_t)K, sizeof(double));
+  double* u0 = calloc(NP, sizeof(double)); /* u_{-1} = B~_0^T x_0 of the initial state */
+  double* u_prev = calloc(NP, sizeof(double));
+  double* u_cur = calloc(NP, sizeof(double));
+
+  /* ---- forward: unit_rope's steps, keeping h_t, B~_t, C~_t, Phi_t ---- */
+  if (io->angle0)
+    for (int k = 0; k < K; ++k) Phi[k] = io->angle0[us * K + k];
+  if (io->h0) memcpy(Hs, io->h0 + us * NP, sizeof(double) * NP);
+  if (io->bprev0 && io->xprev0) outer_sum(N, P, R, io->bprev0 + us * R * N, io->xprev0 + us * R * P, u0);
+  memcpy(u_prev, u0, sizeof(double) * NP);
+  for (int t = 0; t < L; ++t) {
+    const size_t it = ix_tok(d, b, t, h), ib = ix_bc(d, b, t, h);
+    const double dt = io->dt[it], lam = io->lam[it];
+    for (int k = 0; k < K; ++k) {
+      Phi[k] += dt * io->theta[it * K + k];
+      Ph[(size_t)t * K + k] = Phi[k];
+    }
+    for (int r = 0; r < R; ++r)
+      for (int k = 0; k < K; ++k) {
+        const double* Bv = io->B + ib * R * N + r * N;
+        const double* Cv = io->C + ib * R * N + r * N;
+        double* bo = Bt + ((size_t)t * R + r) * N;
+        double* co = Ct + ((size_t)t * R + r) * N;
+        rot_neg(Phi[k], Bv[2 * k], Bv[2 * k + 1], &bo[2 * k], &bo[2 * k + 1]);
+        rot_neg(Phi[k], Cv[2 * k], Cv[2 * k + 1], &co[2 * k], &co[2 * k + 1]);
+      }
+    const double alpha = exp(dt * decay_rate(io, it, h));
+    const double beta = (1.0 - lam) * dt * alpha, gamma = lam * dt;
+    outer_sum(N, P, R, Bt + (size_t)t * R * N, io->x + it * R * P, u_cur);
+    const double* hp = Hs + (size_t)t * NP;
+    double* hn = Hs + (size_t)(t + 1) * NP;
+    for (size_t i = 0; i < NP; ++i) hn[i] = alpha * hp[i] + beta * u_prev[i] + gamma * u_cur[i];
+    double* tmp = u_prev;
+    u_prev = u_cur;
+    u_cur = tmp;
+  }
+
+  /* ---- backward ---- */
+  double* gh = calloc(NP, sizeof(double));
+  double* gu = calloc(NP, sizeof(double));   /* dL/du_t, collecting beta_{t+1} gh_{t+1} first */
+  double* gup = calloc(NP, sizeof(double));  /* dL/du_{t-1} */
+  double* S = calloc((size_t)K, sizeof(double));
+  double* dBt = calloc((size_t)R * N, sizeof(double));
+  double* dCt = calloc((size_t)R * N, sizeof(double));
+  double* dPhi = calloc((size_t)K, sizeof(double));
+  if (g->dh_out) memcpy(gh, g->dh_out + us * NP, sizeof(double) * NP);
+  if (g->dangle_out)
+    for (int k = 0; k < K; ++k) S[k] = g->dangle_out[us * K + k];
+  double dA_unit = 0.0, dD_unit = 0.0;
+  for (int t = L - 1; t >= 0; --t) {
+    const size_t it = ix_tok(d, b, t, h);
+    const double* x = io->x + it * R * P;
+    const double* dy = g->dy + it * R * P;
+    double* dx = g->dx + it * R * P;
+    const double* Bv = Bt + (size_t)t * R * N;
+    const double* Cv = Ct + (size_t)t * R * N;
+    const double* h_t = Hs + (size_t)(t + 1) * NP;
+    const double* h_p = Hs + (size_t)t * NP;
+    const double dt = io->dt[it], lam = io->lam[it], a = decay_rate(io, it, h);
+    const double alpha = exp(dt * a), beta = (1.0 - lam) * dt * alpha, gamma = lam * dt;
+    /* u_t and u_{t-1} again (cheaper to recompute than to keep) */
+    outer_sum(N, P, R, Bv, x, u_cur);
+    if (t > 0)
+      outer_sum(N, P, R, Bt + (size_t)(t - 1) * R * N, io->x + ix_tok(d, b, t - 1, h) * R * P, u_prev);
+    else
+      memcpy(u_prev, u0, sizeof(double) * NP);
+    /* readout */
+    for (int n = 0; n < N; ++n)
+      for (int p = 0; p < P; ++p) {
+        double s = 0;
+        for (int r = 0; r < R; ++r) s += Cv[r * N + n] * dy[r * P + p];
+        gh[n * P + p] += s;
+      }
+    for (int r = 0; r < R; ++r)
+      for (int n = 0; n < N; ++n) {
+        double s = 0;
+        for (int p = 0; p < P; ++p) s += h_t[n * P + p] * dy[r * P + p];
+        dCt[r * N + n] = s;
+      }
+    for (int i = 0; i < R * P; ++i) {
+      dx[i] = Dh * dy[i];
+      dD_unit += dy[i] * x[i];
+    }
+    /* three-term update */
+    const double d_alpha = dot(gh, h_p, NP), d_beta = dot(gh, u_prev, NP), d_gamma = dot(gh, u_cur, NP);
+    for (size_t i = 0; i < NP; ++i) {
+      gu[i] += gamma * gh[i];
+      gup[i] = beta * gh[i];
+    }
+    /* u_t = sum_r B~_t[r] x_t[r]^T */
+    for (int r = 0; r < R; ++r) {
+      for (int n = 0; n < N; ++n) {
+        double s = 0;
+        for (int p = 0; p < P; ++p) s += gu[n * P + p] * x[r * P + p];
+        dBt[r * N + n] = s;
+      }
+      for (int p = 0; p < P; ++p) {
+        double s = 0;
+        for (int n = 0; n < N; ++n) s += gu[n * P + p] * Bv[r * N + n];
+        dx[r * P + p] += s;
+      }
+    }
+    if (t == L - 1) { /* the exported B~_{L-1} and x_{L-1} */
+      if (g->dbprev_out)
+        for (int i = 0; i < R * N; ++i) dBt[i] += g->dbprev_out[us * R * N + i];
+      if (g->dxprev_out)
+        for (int i = 0; i < R * P; ++i) dx[i] += g->dxprev_out[us * R * P + i];
+    }
+    /* scalars: alpha = exp(dt a), beta = (1 - lam) dt alpha, gamma = lam dt */
+    const double d_alpha_all = d_alpha + d_beta * (1.0 - lam) * dt;
+    double ddt = d_alpha_all * alpha * a + d_beta * (1.0 - lam) * alpha + d_gamma * lam;
+    g->dlam[it] = -d_beta * dt * alpha + d_gamma * dt;
+    const double da = d_alpha_all * alpha * dt;
+    if (io->A_t)
+      g->dA[it] = da;
+    else
+      dA_unit += da;
+    /* rotation back, and the angle's share */
+    for (int k = 0; k < K; ++k) dPhi[k] = 0.0;
+    for (int r = 0; r < R; ++r)
+      for (int k = 0; k < K; ++k) {
+        const double ph = Ph[(size_t)t * K + k], c = cos(ph), sn = sin(ph);
+        const double* db = dBt + r * N + 2 * k;
+        const double* dc = dCt + r * N + 2 * k;
+        const double* bt = Bv + r * N + 2 * k;
+        const double* ct = Cv + r * N + 2 * k;
+        double* oB = g->dB + it * R * N + r * N + 2 * k;
+        double* oC = g->dC + it * R * N + r * N + 2 * k;
+        oB[0] = c * db[0] - sn * db[1];
+        oB[1] = sn * db[0] + c * db[1];
+        oC[0] = c * dc[0] - sn * dc[1];
+        oC[1] = sn * dc[0] + c * dc[1];
+        dPhi[k] += db[0] * bt[1] - db[1] * bt[0] + dc[0] * ct[1] - dc[1] * ct[0];
+      }
+    for (int k = 0; k < K; ++k) {
+      S[k] += dPhi[k];
+      g->dtheta[it * K + k] = dt * S[k];
+      ddt += io->theta[it * K + k] * S[k];
+    }
+    g->ddt[it] = ddt;
+    for (size_t i = 0; i < NP; ++i) gh[i] *= alpha;
+    double* tmp = gu;
+    gu = gup;
+    gup = tmp;
+  }
+  /* initial state: h_{-1} = h_0, u_{-1} = B~_0^T x_0, Phi_{-1} = Phi_0 */
+  if (g->dh0) memcpy(g->dh0 + us * NP, gh, sizeof(double) * NP);
+  if (g->dbprev0 && g->dxprev0) {
+    const double* b0 = io->bprev0 ? io->bprev0 + us * R * N : NULL;
+    const double* x0 = io->xprev0 ? io->xprev0 + us * R * P : NULL;
+    for (int r = 0; r < R; ++r) {
+      for (int n = 0; n < N; ++n) {
+        double s = 0;
+        for (int p = 0; p < P; ++p) s += gu[n * P + p] * (x0 ? x0[r * P + p] : 0.0);
+        g->dbprev0[(us * R + r) * N + n] = s;
+      }
+      for (int p = 0; p < P; ++p) {
+        double s = 0;
+        for (int n = 0; n < N; ++n) s += gu[n * P + p] * (b0 ? b0[r * N + n] : 0.0);
+        g->dxprev0[(us * R + r) * P + p] = s;
+      }
+    }
+  }
+  if (g->dangle0)
+    for (int k = 0; k < K; ++k) g->dangle0[us * K + k] = S[k];
+  if (!io->A_t) g->dA[us] = dA_unit;
+  g->dD[us] = dD_unit;
+  free(Hs); free(Bt); free(Ct); free(Ph); free(Phi); free(u0); free(u_prev); free(u_cur);
+  free(gh); free(gu); free(gup); free(S); free(dBt); free(dCt); free(dPhi);
+}
+
+/* ------------------------------------------------------------------------- */
 /* quadratic (materialised L x L kernel) form                                  */
 /* ------------------------------------------------------------------------- */
 /*
@@ -401,6 +635,13 @@ int m3o_scan_complex(const m3o_dims* d, const m3o_io* io, int nthreads, const in
 }
 int m3o_scan_rope(const m3o_dims* d, const m3o_io* io, int nthreads, const int* units, int nunits) {
   return run_units(d, io, unit_rope, nthreads, units, nunits);
+}
+/* Gradients of the prefill (see unit_rope_bwd); io->grad must be set. */
+int m3o_scan_rope_bwd(const m3o_dims* d, const m3o_io* io, int nthreads) {
+  if (!io || !io->grad || !io->grad->dy || !io->grad->dx || !io->grad->dB || !io->grad->dC ||
+      !io->grad->dtheta || !io->grad->ddt || !io->grad->dlam || !io->grad->dA || !io->grad->dD)
+    return -1;
+  return run_units(d, io, unit_rope_bwd, nthreads, NULL, 0);
 }
 int m3o_scan_quadratic(const m3o_dims* d, const m3o_io* io, int nthreads) {
   if (!io || !io->y) return -1;

@@ -12,6 +12,7 @@ import subprocess
 import pytest
 
 import oracle
+from tests import test_oracle_bwd_pins as bwd_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "mamba3_oracle.c")
@@ -30,6 +31,13 @@ MUTATIONS = {
     "bcnorm_sum_not_mean": ("    ms /= N;\n", "\n"),
     "bcnorm_eps_outside_sqrt": ("1.0 / sqrt(ms + eps)", "1.0 / (sqrt(ms) + eps)"),
     "bc_group_interleaved": ("h / (d->nheads / d->ngroups)", "h % d->ngroups"),
+    "bwd_angle_sign_of_C": ("+ dc[0] * ct[1] - dc[1] * ct[0];", "- dc[0] * ct[1] + dc[1] * ct[0];"),
+    "bwd_rotate_back_wrong_way": ("oB[0] = c * db[0] - sn * db[1];", "oB[0] = c * db[0] + sn * db[1];"),
+    "bwd_no_lagged_adjoint": ("gup[i] = beta * gh[i];", "gup[i] = 0.0;"),
+    "bwd_beta_not_through_alpha": ("const double d_alpha_all = d_alpha + d_beta * (1.0 - lam) * dt;",
+                                   "const double d_alpha_all = d_alpha;"),
+    "bwd_theta_without_dt": ("g->dtheta[it * K + k] = dt * S[k];", "g->dtheta[it * K + k] = S[k];"),
+    "bwd_adjoint_not_decayed": ("for (size_t i = 0; i < NP; ++i) gh[i] *= alpha;", ""),
     "bcnorm_bias_index_swapped": ("const size_t p = ((size_t)h * R + r) * N + n;", "const size_t p = ((size_t)r * H + h) * N + n;"),
 }
 
@@ -50,6 +58,10 @@ PIN_FUNCS = [
     pins.test_bc_norm_scale_invariant_and_odd,
     pins.test_bc_norm_weight_and_bias_per_head_and_rank,
     lambda: [pins.test_grouped_bc_equals_per_head_broadcast("scan_complex", G, R) for G, R in ((2, 2), (3, 1))],
+    lambda: bwd_pins.test_backward_matches_finite_differences_of_the_definition({}),
+    lambda: bwd_pins.test_backward_matches_finite_differences_of_the_definition(dict(R=1, L=11, H=3, N=6, P=2)),
+    bwd_pins.test_backward_linear_in_x_and_state,
+    bwd_pins.test_backward_linear_in_C_and_D,
 ]
 
 
