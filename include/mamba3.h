@@ -188,6 +188,38 @@ MAMBA3_API int mamba3_decode_step_at(const mamba3_dims* dims, const mamba3_state
                                      const void* B, const void* C, const void* theta, const void* dt,
                                      const void* lam, const void* A_t, const float* D, void* y, void* stream);
 
+/*
+ * Backward pass of mamba3_scan_fwd: the gradients of a loss L given dL/dy and,
+ * optionally, dL/d(exported state).  The pages give no gradient formulas; these
+ * are the chain rule applied to the recurrence above (section 1.1), its
+ * rotation (section 1.2) and the rank-R products (section 1.3), in reverse
+ * order over the sequence.
+ *   x .. D, init  as for mamba3_scan_fwd (A per head; B, C one row per head:
+ *                 dims->ngroups 0 or nheads; dims->chunk is ignored).
+ *   dy            layout and dtype of y.
+ *   d_final       nullable: float32 gradients of the four exported state fields
+ *                 (all non-null when given).
+ *   dx, dB, dC, dtheta, ddt, dlam
+ *                 outputs, the layouts and dtype of x, B, C, theta, dt, lam.
+ *   dA, dD        outputs, float32 [nheads], summed over batch and tokens;
+ *                 overwritten (zeroed on `stream`, then accumulated).  dD nullable.
+ *   d_init        nullable: float32 gradients of the four initial-state fields
+ *                 (with init NULL, those of a zero initial state).
+ *   workspace     at least mamba3_scan_bwd_workspace_bytes(dims): the state at
+ *                 every chunk start, kept between the forward and the reverse
+ *                 sweep (batch * nheads * ceil(seqlen / Q) * (N P + N/2) floats,
+ *                 Q = 32 / rank), after the 256-byte status word.
+ * Computed in float32 whatever in_dtype is.  Returns MAMBA3_ERR_UNSUPPORTED for
+ * grouped B/C, and for N, P whose per-chunk tiles exceed shared memory.
+ */
+MAMBA3_API size_t mamba3_scan_bwd_workspace_bytes(const mamba3_dims* dims);
+MAMBA3_API int mamba3_scan_bwd(const mamba3_dims* dims, const void* x, const void* B, const void* C,
+                               const void* theta, const void* dt, const void* lam, const float* A,
+                               const float* D, const mamba3_state* init, const void* dy,
+                               const mamba3_state* d_final, void* dx, void* dB, void* dC, void* dtheta,
+                               void* ddt, void* dlam, float* dA, float* dD, const mamba3_state* d_init,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then returns the device status word that the last
  * mamba3_scan_fwd on `workspace` left (MAMBA3_OK or MAMBA3_ERR_TIMEOUT), or
  * MAMBA3_ERR_CUDA / MAMBA3_ERR_INVALID. */

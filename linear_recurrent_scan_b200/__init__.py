@@ -106,6 +106,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba3_decode_step_at.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(_CState), vp, vp, vp, vp, vp, vp,
                                           vp, vp, vp, vp]
     lib.mamba3_decode_step_at.restype = i
+    lib.mamba3_scan_bwd_workspace_bytes.argtypes = [ctypes.POINTER(Dims)]
+    lib.mamba3_scan_bwd_workspace_bytes.restype = sz
+    lib.mamba3_scan_bwd.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(_CState), vp,
+                                    ctypes.POINTER(_CState), vp, vp, vp, vp, vp, vp, vp, vp,
+                                    ctypes.POINTER(_CState), vp, sz, vp]
+    lib.mamba3_scan_bwd.restype = i
     _lib = lib
     return lib
 
@@ -362,6 +368,49 @@ def mamba3_decode_step_at(state: State, x, B, C, theta, dt, lam, A_t, D=None, y:
     return y
 
 
+def mamba3_scan_bwd_workspace_bytes(dims: Dims) -> int:
+    return int(load_library().mamba3_scan_bwd_workspace_bytes(ctypes.byref(dims)))
+
+
+def mamba3_scan_bwd(x, B, C, theta, dt, lam, A, D, dy, init: Optional[State] = None,
+                    d_final: Optional[State] = None, grads: Optional[dict] = None,
+                    workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Gradients of mamba3_scan_fwd (see mamba3.h) given dy (shaped like y) and,
+    optionally, the gradients of the exported state.  Returns a dict: dx, dB,
+    dC, dtheta, ddt, dlam (shaped and typed like the inputs), dA, dD (fp32
+    [H]) and d_init (a State: the initial state's gradients).  ``grads`` may
+    hold preallocated outputs under those names."""
+    lib = load_library()
+    _check_inputs(x, B, C, theta, dt, lam, A, D, decode=False)
+    if dy.shape != x.shape or dy.dtype != x.dtype or not dy.is_contiguous() or dy.device != x.device:
+        raise ValueError("dy must be a contiguous tensor shaped and typed like x")
+    dims = make_dims(x, B)
+    b, L, H, R, P = x.shape
+    N = B.shape[-1]
+    out = dict(grads or {})
+    for name, like in (("dx", x), ("dB", B), ("dC", C), ("dtheta", theta), ("ddt", dt), ("dlam", lam)):
+        if name not in out:
+            out[name] = torch.empty_like(like)
+    for name in ("dA", "dD"):
+        if name not in out:
+            out[name] = torch.empty(H, dtype=torch.float32, device=x.device)
+    if "d_init" not in out:
+        out["d_init"] = State.zeros(b, H, P, N, R, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(mamba3_scan_bwd_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
+    ci = init._c() if init is not None else None
+    cf = d_final._c() if d_final is not None else None
+    cd = out["d_init"]._c()
+    rc = lib.mamba3_scan_bwd(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam),
+                             _ptr(A), _ptr(D), ctypes.byref(ci) if ci is not None else None, _ptr(dy),
+                             ctypes.byref(cf) if cf is not None else None, _ptr(out["dx"]), _ptr(out["dB"]),
+                             _ptr(out["dC"]), _ptr(out["dtheta"]), _ptr(out["ddt"]), _ptr(out["dlam"]),
+                             _ptr(out["dA"]), _ptr(out["dD"]), ctypes.byref(cd), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mamba3_scan_bwd")
+    return out
+
+
 def mamba3_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(load_library().mamba3_device_status(_ptr(workspace), _stream(stream)))
 
@@ -370,6 +419,6 @@ __all__ = [
     "Dims", "State", "BCNorm", "Mamba3Error", "load_library", "make_dims",
     "mamba3_scan_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc", "mamba3_decode_step",
     "mamba3_scan_fwd_bcnorm", "mamba3_decode_step_bcnorm", "mamba3_scan_fwd_at", "mamba3_decode_step_at",
-    "mamba3_device_status",
+    "mamba3_scan_bwd_workspace_bytes", "mamba3_scan_bwd", "mamba3_device_status",
     "mamba3_status_string",
 ]

@@ -40,6 +40,22 @@ struct DecodeArgs {
   float neps;
 };
 
+// Backward of the prefill: the forward's arguments in `f` (its y and final
+// state unused), the output gradient and the gradients to produce.
+struct BwdArgs {
+  ScanArgs f;
+  const void* dy;                                                // layout of y
+  const float *dh_out, *dbprev_out, *dxprev_out, *dangle_out;    // all null = no exported-state gradient
+  void *dx, *dB, *dC, *dtheta, *ddt, *dlam;                      // layouts and dtype of the inputs
+  float *dA, *dD;                                                // [H], zeroed by the launcher; dD nullable
+  float *dh0, *dbprev0, *dxprev0, *dangle0;                      // all null = not wanted
+  float* ckpt;  // [units][chunks][N*P + N/2]: hbar and Phi at every chunk start
+};
+
+size_t bwd_checkpoint_bytes(const ScanArgs& a);
+int bwd_supported(const ScanArgs& a);
+int launch_scan_bwd(const BwdArgs& g, cudaStream_t s);
+
 // Each launcher returns MAMBA3_OK, MAMBA3_ERR_UNSUPPORTED (shape not compiled)
 // or MAMBA3_ERR_CUDA (launch failure).
 int decode_supported(const DecodeArgs& a);

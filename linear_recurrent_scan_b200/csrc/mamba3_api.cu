@@ -89,6 +89,25 @@ size_t mamba3_scan_workspace_bytes(const mamba3_dims* d) {
 }  // extern "C"
 
 namespace {
+// The forward arguments common to the prefill and its backward pass.
+m3::ScanArgs scan_args(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                       const void* dt, const void* lam, const float* A, const float* D, const mamba3_state* init) {
+  m3::ScanArgs a;
+  memset(&a, 0, sizeof(a));
+  a.batch = d->batch;
+  a.seqlen = d->seqlen;
+  a.nheads = d->nheads;
+  a.P = d->headdim;
+  a.N = d->dstate;
+  a.R = d->rank;
+  a.Q = d->chunk;
+  a.ngroups = bc_groups(d);
+  a.dtype = d->in_dtype;
+  a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.D = D;
+  if (init) { a.h0 = init->h; a.bprev0 = init->b_prev; a.xprev0 = init->x_prev; a.angle0 = init->angle; }
+  return a;
+}
+
 // The prefill behind mamba3_scan_fwd (A per head), mamba3_scan_fwd_at (A_t per
 // token; A null) and mamba3_scan_fwd_bcnorm (norm non-null, already checked).
 int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
@@ -104,19 +123,8 @@ int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
   if (!workspace || !aligned16(workspace)) return MAMBA3_ERR_WORKSPACE;
   if (workspace_bytes < mamba3_scan_workspace_bytes(d)) return MAMBA3_ERR_WORKSPACE;
 
-  m3::ScanArgs a;
-  memset(&a, 0, sizeof(a));
-  a.batch = d->batch;
-  a.seqlen = d->seqlen;
-  a.nheads = d->nheads;
-  a.P = d->headdim;
-  a.N = d->dstate;
-  a.R = d->rank;
-  a.Q = d->chunk;
-  a.ngroups = bc_groups(d);
-  a.dtype = d->in_dtype;
-  a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.A_t = A_t; a.D = D;
-  if (init) { a.h0 = init->h; a.bprev0 = init->b_prev; a.xprev0 = init->x_prev; a.angle0 = init->angle; }
+  m3::ScanArgs a = scan_args(d, x, B, C, theta, dt, lam, A, D, init);
+  a.A_t = A_t;
   a.y = y;
   if (final_state) {
     a.h_out = final_state->h; a.bprev_out = final_state->b_prev;
@@ -218,6 +226,45 @@ int mamba3_device_status(const void* workspace, void* stream) {
   m3::DeviceStatus st;
   if (cudaMemcpy(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return MAMBA3_ERR_CUDA;
   return st.code;
+}
+
+size_t mamba3_scan_bwd_workspace_bytes(const mamba3_dims* d) {
+  if (check_dims(d, true) != MAMBA3_OK) return 0;
+  const m3::ScanArgs a = scan_args(d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return kStatusBytes + m3::bwd_checkpoint_bytes(a);
+}
+
+int mamba3_scan_bwd(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                    const void* dt, const void* lam, const float* A, const float* D, const mamba3_state* init,
+                    const void* dy, const mamba3_state* d_final, void* dx, void* dB, void* dC, void* dtheta,
+                    void* ddt, void* dlam, float* dA, float* dD, const mamba3_state* d_init, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  int rc = check_dims(d, true);
+  if (rc) return rc;
+  if (!A || !dA || !aligned4(dA) || (dD && !aligned4(dD))) return MAMBA3_ERR_INVALID;
+  if (d->seqlen > 0) {
+    if ((rc = check_inputs(x, B, C, theta, dt, lam, A, D, dy))) return rc;
+    if ((rc = check_inputs(dx, dB, dC, dtheta, ddt, dlam, A, D, dy))) return rc;  // the gradients' layouts
+  }
+  if ((rc = check_state(init)) || (rc = check_state(d_final)) || (rc = check_state(d_init))) return rc;
+  if (!workspace || !aligned16(workspace)) return MAMBA3_ERR_WORKSPACE;
+  if (workspace_bytes < mamba3_scan_bwd_workspace_bytes(d)) return MAMBA3_ERR_WORKSPACE;
+  m3::BwdArgs g;
+  memset(&g, 0, sizeof(g));
+  g.f = scan_args(d, x, B, C, theta, dt, lam, A, D, init);
+  g.f.workspace = workspace;
+  g.f.workspace_bytes = workspace_bytes;
+  if ((rc = m3::bwd_supported(g.f))) return rc;
+  g.dy = dy;
+  if (d_final) {
+    g.dh_out = d_final->h; g.dbprev_out = d_final->b_prev; g.dxprev_out = d_final->x_prev; g.dangle_out = d_final->angle;
+  }
+  g.dx = dx; g.dB = dB; g.dC = dC; g.dtheta = dtheta; g.ddt = ddt; g.dlam = dlam; g.dA = dA; g.dD = dD;
+  if (d_init) { g.dh0 = d_init->h; g.dbprev0 = d_init->b_prev; g.dxprev0 = d_init->x_prev; g.dangle0 = d_init->angle; }
+  g.ckpt = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  return m3::launch_scan_bwd(g, s);
 }
 
 }  // extern "C"

@@ -3,6 +3,7 @@
     python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --batch 2 --reps 3
     python -m linear_recurrent_scan_b200.profile_case --workload siso_decode_b128 --decode --reps 3
     python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --groups 1 --reps 3
+    python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --backward --reps 3
 
 Inputs are seeded synthetic tensors on cuda:0.  Prints the CUDA-event time
 of each call; under a profiler those times are not benchmark numbers.
@@ -27,6 +28,7 @@ def main():
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--decode", action="store_true", help="time decode steps instead of the prefill")
     ap.add_argument("--groups", type=int, default=0, help="B, C shared by this many groups of heads (0 = per head)")
+    ap.add_argument("--backward", action="store_true", help="time the prefill's backward pass")
     args = ap.parse_args()
     w = wl.CONFIGS[args.workload]
     if args.batch:
@@ -54,6 +56,21 @@ def main():
     if args.groups:
         inp.update(wl.grouped_bc(inp, args.groups))
     y = torch.empty_like(inp["x"])
+    if args.backward:
+        g = torch.Generator(device=dev)
+        g.manual_seed(wl.BASE_SEED + 9)
+        dy = torch.randn(inp["x"].shape, generator=g, device=dev).to(inp["x"].dtype)
+        dims = m3.make_dims(inp["x"], inp["B"])
+        ws = torch.empty(m3.mamba3_scan_bwd_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+        grads = None
+        for i in range(args.reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            grads = m3.mamba3_scan_bwd(*(inp[n] for n in NAMES), inp["A"], inp["D"], dy, grads=grads, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            print(f"backward {w.name} b{w.batch} L{w.seqlen} rep {i}: {e0.elapsed_time(e1):.3f} ms")
+        return
     for i in range(args.reps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()

@@ -204,15 +204,20 @@ def test_time_varying_decay_entry_points_validate_on_host(lib):
     assert rc == m3.MAMBA3_ERR_INVALID
 
 
-def test_grouped_bc_dims(lib):
-    """ngroups: 0 (one B/C row per head) or a divisor of nheads; the valid forms
-    pass the host checks and, with no GPU, fail in CUDA."""
+def test_grouped_bc_dims_rejected(lib):
+    """ngroups must be 0 (one B/C row per head) or a divisor of nheads."""
     for g in (0, 1, 3):
         assert lib.mamba3_scan_workspace_bytes(ctypes.byref(dims(ngroups=g))) >= 256
-        assert scan(lib, dims(ngroups=g)) == m3.MAMBA3_ERR_CUDA
-        assert decode(lib, dims(ngroups=g)) == m3.MAMBA3_ERR_CUDA
     assert scan(lib, dims(ngroups=2)) == m3.MAMBA3_ERR_INVALID
     assert decode(lib, dims(ngroups=2)) == m3.MAMBA3_ERR_INVALID
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_grouped_bc_dims_accepted(lib):
+    """The valid group counts pass the host checks and, with no GPU, fail in CUDA."""
+    for g in (0, 1, 3):
+        assert scan(lib, dims(ngroups=g)) == m3.MAMBA3_ERR_CUDA
+        assert decode(lib, dims(ngroups=g)) == m3.MAMBA3_ERR_CUDA
 
 
 def test_python_binding_infers_groups(lib):
@@ -228,3 +233,35 @@ def test_python_binding_infers_groups(lib):
     with pytest.raises(ValueError):  # grouped B with a per-head C
         m3.mamba3_scan_fwd(x, torch.zeros(1, 4, 2, 1, 16, dtype=torch.bfloat16),
                            torch.zeros(1, 4, 6, 1, 16, dtype=torch.bfloat16), th, dt, dt, torch.zeros(6))
+
+
+def bwd(lib, d, ptrs=None, ws=FAKE, ws_bytes=1 << 40):
+    p = dict(x=FAKE, B=FAKE, C=FAKE, theta=FAKE, dt=FAKE, lam=FAKE, A=FAKE, D=None, dy=FAKE, dx=FAKE, dB=FAKE,
+             dC=FAKE, dtheta=FAKE, ddt=FAKE, dlam=FAKE, dA=FAKE, dD=None)
+    p.update(ptrs or {})
+    return lib.mamba3_scan_bwd(ctypes.byref(d), p["x"], p["B"], p["C"], p["theta"], p["dt"], p["lam"], p["A"],
+                               p["D"], None, p["dy"], None, p["dx"], p["dB"], p["dC"], p["dtheta"], p["ddt"],
+                               p["dlam"], p["dA"], p["dD"], None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("name", ["x", "B", "dy", "dx", "dB", "dC", "dtheta", "ddt", "dlam", "dA", "A"])
+def test_backward_rejects_null_pointer(lib, name):
+    assert bwd(lib, dims(), {name: None}) == m3.MAMBA3_ERR_INVALID
+
+
+def test_backward_host_validation(lib):
+    d = dims()
+    need = lib.mamba3_scan_bwd_workspace_bytes(ctypes.byref(d))
+    # 2 x 3 units, 64 tokens in chunks of 32: the state (16 x 16) and angle (8) at each chunk start
+    assert need == 256 + 2 * 3 * 2 * (16 * 16 + 8) * 4
+    assert bwd(lib, d, ws_bytes=need - 1) == m3.MAMBA3_ERR_WORKSPACE
+    assert bwd(lib, d, ws=FAKE + 8) == m3.MAMBA3_ERR_WORKSPACE
+    assert bwd(lib, d, {"dB": FAKE + 4}) == m3.MAMBA3_ERR_INVALID
+    assert bwd(lib, dims(ngroups=1)) == m3.MAMBA3_ERR_UNSUPPORTED  # grouped B/C: not in this pass
+    assert bwd(lib, dims(dstate=256, headdim=128)) == m3.MAMBA3_ERR_UNSUPPORTED  # tiles beyond shared memory
+    assert lib.mamba3_scan_bwd_workspace_bytes(ctypes.byref(dims(rank=3))) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_backward_valid_call_without_device_is_a_cuda_error(lib):
+    assert bwd(lib, dims()) == m3.MAMBA3_ERR_CUDA
