@@ -105,6 +105,15 @@ def decode_bytes(w: wl.Workload, groups=0) -> int:
     return units * (2 * state + io) + bc + 8 * w.nheads
 
 
+def backward_bytes(w: wl.Workload) -> int:
+    """Algorithmic bytes of one backward pass: the forward's inputs and dy read
+    once, the gradients of x, B, C, theta, dt, lam written once, A, D and their
+    gradients (zero initial state, no exported-state gradient)."""
+    s = esize(w.dtype)
+    per_th = s * (w.rank * w.headdim + 2 * w.rank * w.dstate + w.dstate // 2 + 2)  # x, B, C, theta, dt, lam
+    return w.token_heads * (2 * per_th + s * w.rank * w.headdim) + 16 * w.nheads
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -333,6 +342,34 @@ def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False,
     return statistics.median(times)
 
 
+def run_backward(m3, w: wl.Workload, rank, steps, warmup):
+    """Median per-launch time (ms) of the prefill's backward pass on workload w
+    (dy drawn N(0, 1); inputs and outputs resident on the device)."""
+    dev = torch.device("cuda")
+    inp = wl.make_inputs(w, seed=wl.BASE_SEED + rank, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.BASE_SEED + 8 + rank)
+    dy = torch.randn(inp["x"].shape, generator=g, device=dev).to(w.dtype)
+    ins = [inp[n] for n in NAMES]
+    dims = m3.make_dims(inp["x"], inp["B"])
+    ws = torch.zeros(m3.mamba3_scan_bwd_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    grads = m3.mamba3_scan_bwd(*ins, inp["A"], inp["D"], dy, workspace=ws, stream=stream)
+    for _ in range(warmup):
+        m3.mamba3_scan_bwd(*ins, inp["A"], inp["D"], dy, grads=grads, workspace=ws, stream=stream)
+    times = []
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        m3.mamba3_scan_bwd(*ins, inp["A"], inp["D"], dy, grads=grads, workspace=ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    del inp, ins, dy, grads, ws
+    torch.cuda.empty_cache()
+    return statistics.median(times)
+
+
 def run_decode(m3, w: wl.Workload, world, rank, steps, fused_norm=False, time_varying_a=False, groups=0):
     """Seed the state with a 512-token prefill, then time `steps` decode steps
     captured in one CUDA graph (per-step inputs pre-generated, larger than L2).
@@ -456,6 +493,14 @@ def ours(args):
     grp["decode_" + DECODE[0].name] = {"ngroups": 1, "us_per_step": round(us, 2), "roofline": {
         "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
         "traffic": traffic("grouped_decode"), "bytes_per_step": by}}
+    # the backward pass of the headline prefill (dy given; zero initial state)
+    ms = max_over_ranks(run_backward(m3, PREFILL, rank, steps=3, warmup=1), world)
+    by = backward_bytes(PREFILL)
+    gbs = by / (ms * 1e-3) / 1e9
+    bwd = {"prefill_" + PREFILL.name: {"ms_per_launch": round(ms, 3), "kernel": "scan_bwd_kernel (SIMT, fp32)",
+                                       "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                                                    "unit": "GB/s", "frac": round(gbs / peak, 5),
+                                                    "bytes_per_launch": by}}}
     more = {}
     for w in PREFILL_MORE:
         ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=max(5, min(args.steps, 20)), warmup=3), world)
@@ -493,6 +538,7 @@ def ours(args):
         "fused_bc_norm": fused,
         "time_varying_decay": tva,
         "grouped_bc": grp,
+        "backward": bwd,
         "decode": dec,
         "e2e": {"value": round(e2e_value, 3), "unit": "Mtokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},

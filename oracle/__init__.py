@@ -90,6 +90,8 @@ def _bind(lib):
     lib.m3o_scan_rope_bwd.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_IO), ctypes.c_int]
     lib.m3o_scan_rope_bwd.restype = ctypes.c_int
     lib.m3o_bc_norm.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.c_double, _P]
+    lib.m3o_gated_norm.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int, _P, _P, _P, ctypes.c_double, _P]
+    lib.m3o_gated_norm.restype = ctypes.c_int
     lib.m3o_bc_norm.restype = ctypes.c_int
     return lib
 
@@ -280,7 +282,29 @@ def scan_bwd(x, B, C, theta, dt, lam, A, D, dy, init: Optional[State] = None,
     return out
 
 
-__all__ = ["build", "State", "scan_complex", "scan_rope", "scan_quadratic", "decode_step", "bc_norm", "scan_bwd"]
+def gated_norm(y, z, w=None, groups: Optional[int] = None, eps: float = 1e-6) -> np.ndarray:
+    """Pre-gate grouped RMS norm and gate of the layer output: y, z [..., H, R, P]
+    (leading axes flattened to tokens), w [H, R, P] or None, ``groups`` norm
+    groups of H / groups consecutive heads (default H: one per head).  Source:
+    "Mamba-3: 2x smaller state ..." (MarkTechPost, Korean translation), section 2
+    (grouped RMS norm ahead of the gate); the gate is silu(z)."""
+    y, z = _f64(y), _f64(z)
+    assert y.shape == z.shape, "y and z must have the same shape"
+    *lead, H, R, P = y.shape
+    groups = H if groups is None else groups
+    rows = int(np.prod(lead)) if lead else 1
+    dims = _Dims(1, rows, H, P, 0, R, 0)
+    w = _f64(w) if w is not None else None
+    assert w is None or w.shape == (H, R, P), "w must be [H, R, P]"
+    out = np.empty_like(y)
+    rc = _load().m3o_gated_norm(ctypes.byref(dims), int(groups), _ptr(y), _ptr(z), _ptr(w), float(eps), _ptr(out))
+    if rc != 0:
+        raise ValueError("groups must divide the number of heads")
+    return out
+
+
+__all__ = ["build", "State", "scan_complex", "scan_rope", "scan_quadratic", "decode_step", "bc_norm", "scan_bwd",
+           "gated_norm"]
 
 
 def bc_norm(z, w=None, bias=None, eps: float = 1e-6) -> np.ndarray:

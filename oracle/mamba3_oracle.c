@@ -680,3 +680,38 @@ int m3o_bc_norm(const m3o_dims* d, const double* z, const double* w, const doubl
   }
   return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Output side: pre-gate grouped RMS norm and the gate                         */
+/* ------------------------------------------------------------------------- */
+/*
+ * Same page, section 2: hybrids add a grouped RMS norm in front of the output
+ * gate.  For every token (b, t) and norm group g of H / G consecutive heads,
+ * over the group's channels c = (h, r, p):
+ *     out[c] = y[c] / sqrt(mean_c y[c]^2 + eps) * w[h, r, p] * silu(z[c]),
+ * silu(z) = z / (1 + e^{-z}) (the gate of the Mamba line; the pages do not name
+ * it).  y, z, out [b, L, H, R, P]; w [H, R, P] or NULL (weight 1).  An all-zero
+ * group with eps = 0 gives 0.
+ */
+int m3o_gated_norm(const m3o_dims* d, int groups, const double* y, const double* z, const double* w, double eps,
+                   double* out) {
+  const int H = d->nheads, R = d->rank, P = d->headdim;
+  if (groups <= 0 || H % groups != 0) return -1;
+  const size_t hpg = (size_t)(H / groups), gsize = hpg * R * P;
+  const size_t rows = (size_t)d->batch * d->seqlen * groups; /* (b, t, g) in order */
+  for (size_t row = 0; row < rows; ++row) {
+    const size_t g = row % groups;
+    const double* yr = y + row * gsize;
+    double ms = 0.0;
+    for (size_t c = 0; c < gsize; ++c) ms += yr[c] * yr[c];
+    ms /= (double)gsize;
+    const double inv = (ms + eps) > 0.0 ? 1.0 / sqrt(ms + eps) : 0.0;
+    for (size_t c = 0; c < gsize; ++c) {
+      const size_t h = g * hpg + c / ((size_t)R * P), rp = c % ((size_t)R * P);
+      const double wt = w ? w[h * R * P + rp] : 1.0;
+      const double zv = z[row * gsize + c];
+      out[row * gsize + c] = yr[c] * inv * wt * (zv / (1.0 + exp(-zv)));
+    }
+  }
+  return 0;
+}

@@ -38,6 +38,12 @@ MUTATIONS = {
                                    "const double d_alpha_all = d_alpha;"),
     "bwd_theta_without_dt": ("g->dtheta[it * K + k] = dt * S[k];", "g->dtheta[it * K + k] = S[k];"),
     "bwd_adjoint_not_decayed": ("for (size_t i = 0; i < NP; ++i) gh[i] *= alpha;", ""),
+    "gate_before_norm": ("out[row * gsize + c] = yr[c] * inv * wt * (zv / (1.0 + exp(-zv)));",
+                         "out[row * gsize + c] = yr[c] * wt * (zv / (1.0 + exp(-zv)));"),
+    "gate_sigmoid_only": ("(zv / (1.0 + exp(-zv)))", "(1.0 / (1.0 + exp(-zv)))"),
+    "gated_norm_sum_not_mean": ("ms /= (double)gsize;", "ms /= 1.0;"),
+    "gated_norm_interleaved_groups": ("const size_t h = g * hpg + c / ((size_t)R * P)",
+                                      "const size_t h = g + groups * (c / ((size_t)R * P))"),
     "bcnorm_bias_index_swapped": ("const size_t p = ((size_t)h * R + r) * N + n;", "const size_t p = ((size_t)r * H + h) * N + n;"),
 }
 
@@ -61,6 +67,11 @@ PIN_FUNCS = [
     lambda: bwd_pins.test_backward_matches_finite_differences_of_the_definition({}),
     lambda: bwd_pins.test_backward_matches_finite_differences_of_the_definition(dict(R=1, L=11, H=3, N=6, P=2)),
     bwd_pins.test_backward_linear_in_x_and_state,
+    pins.test_gate_is_silu_at_exact_points,
+    pins.test_gate_odd_part_is_the_identity,
+    lambda: [pins.test_normalised_group_has_unit_rms(g) for g in (1, 2, 6)],
+    pins.test_gated_norm_scale_invariant_and_group_local,
+    pins.test_gated_norm_weight_per_head_rank_channel_and_eps,
     bwd_pins.test_backward_linear_in_C_and_D,
 ]
 

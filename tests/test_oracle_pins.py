@@ -543,3 +543,71 @@ def test_grouped_bc_prefill_then_decode():
         yt, st = oracle.decode_step(st, **step, A=inp["A"], D=inp["D"])
         assert rel_err(yt, y_all[:, t]) < 1e-12
     assert rel_err(st.h, f_all.h) < 1e-12
+
+
+# ---------------------------------------------------------------- output side
+# "Mamba-3: 2x smaller state ..." (MarkTechPost, Korean translation), section 2:
+# a grouped RMS norm ahead of the output gate.  Pins: silu's exact values and its
+# odd part, unit RMS of the normalised group, scale invariance, group locality,
+# and the weight placed per (head, rank, channel).
+
+def _gn_case(rng, b=2, L=5, H=6, R=2, P=4):
+    return rng.standard_normal((b, L, H, R, P)), rng.standard_normal((b, L, H, R, P))
+
+
+def test_gate_is_silu_at_exact_points():
+    """z = 0 closes the gate; z = +-1 give +-1 / (1 + e^{-+1}) times the norm."""
+    rng = np.random.default_rng(141)
+    y, _ = _gn_case(rng)
+    n1 = oracle.gated_norm(y, np.ones_like(y), eps=0.0)
+    assert np.array_equal(oracle.gated_norm(y, np.zeros_like(y)), np.zeros_like(y))
+    nm1 = oracle.gated_norm(y, -np.ones_like(y), eps=0.0)
+    # silu(1) = 0.7310585786300049, silu(-1) = -0.2689414213699951
+    assert np.allclose(nm1 / n1, -0.2689414213699951 / 0.7310585786300049, rtol=1e-13)
+
+
+def test_gate_odd_part_is_the_identity():
+    """silu(z) - silu(-z) = z, so out(z) - out(-z) = norm(y) w z exactly (no sigmoid)."""
+    rng = np.random.default_rng(142)
+    y, z = _gn_case(rng)
+    w = rng.uniform(0.5, 1.5, (6, 2, 4))
+    d = oracle.gated_norm(y, z, w, groups=3) - oracle.gated_norm(y, -z, w, groups=3)
+    ones = oracle.gated_norm(y, np.ones_like(z), w, groups=3) - oracle.gated_norm(y, -np.ones_like(z), w, groups=3)
+    assert np.allclose(d, ones * z, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("groups", [1, 2, 6])
+def test_normalised_group_has_unit_rms(groups):
+    """With the gate's odd part (out(z) - out(-z) = norm(y) z) at z = 1 and w = 1,
+    every group of H / groups heads has unit RMS over its (h, r, p) channels."""
+    rng = np.random.default_rng(143 + groups)
+    y, _ = _gn_case(rng)
+    one = np.ones_like(y)
+    nrm = oracle.gated_norm(y, one, groups=groups, eps=0.0) - oracle.gated_norm(y, -one, groups=groups, eps=0.0)
+    g = nrm.reshape(2, 5, groups, -1)
+    assert np.allclose(np.sqrt((g ** 2).mean(axis=-1)), 1.0, rtol=1e-13)
+
+
+def test_gated_norm_scale_invariant_and_group_local():
+    rng = np.random.default_rng(145)
+    y, z = _gn_case(rng)
+    out = oracle.gated_norm(y, z, groups=3, eps=0.0)
+    assert np.allclose(oracle.gated_norm(7.5 * y, z, groups=3, eps=0.0), out, rtol=1e-13)
+    y2 = y.copy()
+    y2[:, :, 2:4] *= rng.uniform(0.1, 10.0, y2[:, :, 2:4].shape)  # heads 2, 3 = group 1 of 3
+    out2 = oracle.gated_norm(y2, z, groups=3, eps=0.0)
+    assert np.array_equal(out2[:, :, :2], out[:, :, :2]) and np.array_equal(out2[:, :, 4:], out[:, :, 4:])
+    assert not np.allclose(out2[:, :, 2:4], out[:, :, 2:4])
+
+
+def test_gated_norm_weight_per_head_rank_channel_and_eps():
+    rng = np.random.default_rng(146)
+    y, z = _gn_case(rng)
+    w = rng.uniform(0.5, 1.5, (6, 2, 4))
+    assert np.allclose(oracle.gated_norm(y, z, w, groups=2), oracle.gated_norm(y, z, groups=2) * w, rtol=1e-14)
+    # a constant group c: mean square c^2, so out = c / sqrt(c^2 + eps) silu(z)
+    c, eps = 0.01, 1e-3
+    yc = np.full_like(y, c)
+    one = np.ones_like(y)
+    nrm = oracle.gated_norm(yc, one, eps=eps) - oracle.gated_norm(yc, -one, eps=eps)
+    assert np.allclose(nrm, c / np.sqrt(c * c + eps), rtol=1e-13)
