@@ -370,6 +370,33 @@ def run_backward(m3, w: wl.Workload, rank, steps, warmup):
     return statistics.median(times)
 
 
+def run_gated_norm(m3, w: wl.Workload, rank, groups, steps, warmup):
+    """Median per-launch time (ms) of the output side (grouped RMS norm + gate) on
+    a prefill output of workload w: y, z drawn N(0, 1), weights U(0.5, 1.5)."""
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.BASE_SEED + 10 + rank)
+    shape = (w.batch, w.seqlen, w.nheads, w.rank, w.headdim)
+    y = torch.randn(shape, generator=g, device=dev).to(w.dtype)
+    z = torch.randn(shape, generator=g, device=dev).to(w.dtype)
+    wt = torch.rand((w.nheads, w.rank, w.headdim), generator=g, device=dev) + 0.5
+    out = torch.empty_like(y)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        m3.mamba3_gated_norm(y, z, wt, groups=groups, out=out, stream=stream)
+    times = []
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        m3.mamba3_gated_norm(y, z, wt, groups=groups, out=out, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    del y, z, out
+    torch.cuda.empty_cache()
+    return statistics.median(times)
+
+
 def run_decode(m3, w: wl.Workload, world, rank, steps, fused_norm=False, time_varying_a=False, groups=0):
     """Seed the state with a 512-token prefill, then time `steps` decode steps
     captured in one CUDA graph (per-step inputs pre-generated, larger than L2).
@@ -501,6 +528,17 @@ def ours(args):
                                        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
                                                     "unit": "GB/s", "frac": round(gbs / peak, 5),
                                                     "bytes_per_launch": by}}}
+    # the output side on the headline prefill's y: grouped RMS norm + gate
+    gated = {}
+    for ng in (PREFILL.nheads, 8):
+        ms = max_over_ranks(run_gated_norm(m3, PREFILL, rank, ng, steps=max(5, min(args.steps, 20)), warmup=3), world)
+        by = 3 * esize(PREFILL.dtype) * PREFILL.token_heads * PREFILL.rank * PREFILL.headdim + 4 * PREFILL.nheads * \
+            PREFILL.rank * PREFILL.headdim
+        gbs = by / (ms * 1e-3) / 1e9
+        gated["prefill_%s_groups%d" % (PREFILL.name, ng)] = {
+            "ms_per_launch": round(ms, 4), "norm_groups": ng,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs / peak, 4), "bytes_per_launch": by}}
     more = {}
     for w in PREFILL_MORE:
         ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=max(5, min(args.steps, 20)), warmup=3), world)
@@ -539,6 +577,7 @@ def ours(args):
         "time_varying_decay": tva,
         "grouped_bc": grp,
         "backward": bwd,
+        "gated_norm": gated,
         "decode": dec,
         "e2e": {"value": round(e2e_value, 3), "unit": "Mtokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},

@@ -220,6 +220,26 @@ MAMBA3_API int mamba3_scan_bwd(const mamba3_dims* dims, const void* x, const voi
                                void* ddt, void* dlam, float* dA, float* dD, const mamba3_state* d_init,
                                void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Output side of the layer: the pre-gate grouped RMS norm and the gate
+ * ("Mamba-3: 2x smaller state ..." (MarkTechPost, Korean translation),
+ * section 2: a grouped RMS norm ahead of the output gate in hybrids).  Per token
+ * and norm group g of nheads / groups consecutive heads, over the group's
+ * channels c = (h, r, p):
+ *     out[c] = y[c] / sqrt(mean_c y[c]^2 + eps) * w[h, r, p] * silu(z[c]),
+ * silu(z) = z / (1 + e^{-z}) (the pages do not name the gate's nonlinearity;
+ * this is the Mamba line's).  An all-zero group with eps = 0 gives 0.
+ *   dims   batch, seqlen (1 for one decode step's output), nheads, headdim, rank,
+ *          in_dtype; dstate, chunk and ngroups are ignored.
+ *   y, z, out  [batch, seqlen, nheads, rank, headdim] in_dtype, 16-byte aligned;
+ *          out may alias y.
+ *   w      float32 [nheads, rank, headdim], 4-byte aligned, or NULL (weight 1).
+ *   groups divides nheads (nheads: one group per head); eps >= 0.
+ * HBM-bound: y and z read once, out written once; computed in float32.
+ */
+MAMBA3_API int mamba3_gated_norm(const mamba3_dims* dims, int groups, const void* y, const void* z, const float* w,
+                                 float eps, void* out, void* stream);
+
 /* Synchronises `stream`, then returns the device status word that the last
  * mamba3_scan_fwd on `workspace` left (MAMBA3_OK or MAMBA3_ERR_TIMEOUT), or
  * MAMBA3_ERR_CUDA / MAMBA3_ERR_INVALID. */

@@ -112,6 +112,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                     ctypes.POINTER(_CState), vp, vp, vp, vp, vp, vp, vp, vp,
                                     ctypes.POINTER(_CState), vp, sz, vp]
     lib.mamba3_scan_bwd.restype = i
+    lib.mamba3_gated_norm.argtypes = [ctypes.POINTER(Dims), i, vp, vp, vp, ctypes.c_float, vp, vp]
+    lib.mamba3_gated_norm.restype = i
     _lib = lib
     return lib
 
@@ -411,6 +413,36 @@ def mamba3_scan_bwd(x, B, C, theta, dt, lam, A, D, dy, init: Optional[State] = N
     return out
 
 
+def mamba3_gated_norm(y, z, w=None, groups: Optional[int] = None, eps: float = 1e-6,
+                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Pre-gate grouped RMS norm and gate of the layer output (see mamba3.h):
+    y, z [..., H, R, P] (same shape, dtype, device; contiguous), w fp32
+    [H, R, P] or None, ``groups`` norm groups of H / groups consecutive heads
+    (default H).  Returns out (allocated if not given; may be y)."""
+    lib = load_library()
+    if y.shape != z.shape or y.dtype != z.dtype or y.device != z.device or y.dim() < 3:
+        raise ValueError("y and z must have the same shape [..., H, R, P], dtype and device")
+    for name, t in (("y", y), ("z", z)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if y.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {y.dtype}")
+    H, R, P = y.shape[-3:]
+    if w is not None and (w.dtype != torch.float32 or w.shape != (H, R, P) or not w.is_contiguous()):
+        raise ValueError("w must be a contiguous float32 tensor of shape [H, R, P]")
+    groups = H if groups is None else groups
+    if out is None:
+        out = torch.empty_like(y)
+    elif out.shape != y.shape or out.dtype != y.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor shaped and typed like y")
+    tokens = y.numel() // (H * R * P) if H * R * P else 0
+    dims = Dims(1, tokens, H, P, 0, R, 0, _DTYPES[y.dtype], 0)
+    rc = lib.mamba3_gated_norm(ctypes.byref(dims), int(groups), _ptr(y), _ptr(z), _ptr(w), float(eps), _ptr(out),
+                               _stream(stream))
+    _check(rc, "mamba3_gated_norm")
+    return out
+
+
 def mamba3_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(load_library().mamba3_device_status(_ptr(workspace), _stream(stream)))
 
@@ -419,6 +451,6 @@ __all__ = [
     "Dims", "State", "BCNorm", "Mamba3Error", "load_library", "make_dims",
     "mamba3_scan_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc", "mamba3_decode_step",
     "mamba3_scan_fwd_bcnorm", "mamba3_decode_step_bcnorm", "mamba3_scan_fwd_at", "mamba3_decode_step_at",
-    "mamba3_scan_bwd_workspace_bytes", "mamba3_scan_bwd", "mamba3_device_status",
+    "mamba3_scan_bwd_workspace_bytes", "mamba3_scan_bwd", "mamba3_gated_norm", "mamba3_device_status",
     "mamba3_status_string",
 ]

@@ -52,6 +52,19 @@ struct BwdArgs {
   float* ckpt;  // [units][chunks][N*P + N/2]: hbar and Phi at every chunk start
 };
 
+// Pre-gate grouped RMS norm and gate of the layer output: rows = tokens x groups
+// contiguous groups of group_size values each.
+struct GatedNormArgs {
+  long long rows;
+  int groups, group_size;
+  mamba3_dtype dtype;
+  const void *y, *z;
+  const float* w;  // [groups * group_size] (= [H, R, P]) or null
+  float eps;
+  void* out;
+};
+int launch_gated_norm(const GatedNormArgs& a, cudaStream_t s);
+
 size_t bwd_checkpoint_bytes(const ScanArgs& a);
 int bwd_supported(const ScanArgs& a);
 int launch_scan_bwd(const BwdArgs& g, cudaStream_t s);

@@ -267,4 +267,24 @@ int mamba3_scan_bwd(const mamba3_dims* d, const void* x, const void* B, const vo
   return m3::launch_scan_bwd(g, s);
 }
 
+int mamba3_gated_norm(const mamba3_dims* d, int groups, const void* y, const void* z, const float* w, float eps,
+                      void* out, void* stream) {
+  if (!d || d->batch < 1 || d->seqlen < 0 || d->nheads < 1 || d->headdim < 1 || d->rank < 1) return MAMBA3_ERR_INVALID;
+  if (d->in_dtype != MAMBA3_F32 && d->in_dtype != MAMBA3_BF16) return MAMBA3_ERR_INVALID;
+  if (groups < 1 || d->nheads % groups != 0 || !(eps >= 0.f)) return MAMBA3_ERR_INVALID;
+  const double total = (double)d->batch * d->seqlen * d->nheads * d->rank * d->headdim;
+  if (total > 9.0e15 || (double)d->nheads / groups * d->rank * d->headdim > 2.0e9) return MAMBA3_ERR_INVALID;
+  m3::GatedNormArgs a;
+  a.rows = (long long)d->batch * d->seqlen * groups;
+  a.groups = groups;
+  a.group_size = d->nheads / groups * d->rank * d->headdim;
+  a.dtype = d->in_dtype;
+  a.y = y; a.z = z; a.w = w; a.eps = eps; a.out = out;
+  if (a.rows > 0) {
+    if (!y || !z || !out || !aligned16(y) || !aligned16(z) || !aligned16(out)) return MAMBA3_ERR_INVALID;
+    if (w && !aligned4(w)) return MAMBA3_ERR_INVALID;
+  }
+  return m3::launch_gated_norm(a, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

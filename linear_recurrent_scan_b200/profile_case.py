@@ -4,6 +4,7 @@
     python -m linear_recurrent_scan_b200.profile_case --workload siso_decode_b128 --decode --reps 3
     python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --groups 1 --reps 3
     python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --backward --reps 3
+    python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --gated-norm 64 --reps 3
 
 Inputs are seeded synthetic tensors on cuda:0.  Prints the CUDA-event time
 of each call; under a profiler those times are not benchmark numbers.
@@ -29,6 +30,8 @@ def main():
     ap.add_argument("--decode", action="store_true", help="time decode steps instead of the prefill")
     ap.add_argument("--groups", type=int, default=0, help="B, C shared by this many groups of heads (0 = per head)")
     ap.add_argument("--backward", action="store_true", help="time the prefill's backward pass")
+    ap.add_argument("--gated-norm", type=int, default=0, metavar="G",
+                    help="time the output side (grouped RMS norm + gate, G norm groups) on a prefill-sized y")
     args = ap.parse_args()
     w = wl.CONFIGS[args.workload]
     if args.batch:
@@ -51,6 +54,22 @@ def main():
             e1.record()
             torch.cuda.synchronize()
             print(f"decode step {i}: {e0.elapsed_time(e1) * 1000:.1f} us")
+        return
+    if args.gated_norm:
+        g = torch.Generator(device=dev)
+        g.manual_seed(wl.BASE_SEED + 10)
+        shape = (w.batch, w.seqlen, w.nheads, w.rank, w.headdim)
+        y = torch.randn(shape, generator=g, device=dev).to(w.dtype)
+        z = torch.randn(shape, generator=g, device=dev).to(w.dtype)
+        wt = torch.rand((w.nheads, w.rank, w.headdim), generator=g, device=dev) + 0.5
+        out = torch.empty_like(y)
+        for i in range(args.reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            m3.mamba3_gated_norm(y, z, wt, groups=args.gated_norm, out=out)
+            e1.record()
+            torch.cuda.synchronize()
+            print(f"gated norm {w.name} groups {args.gated_norm} rep {i}: {e0.elapsed_time(e1) * 1000:.1f} us")
         return
     inp = wl.make_inputs(w, device=dev)
     if args.groups:

@@ -265,3 +265,23 @@ def test_backward_host_validation(lib):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_backward_valid_call_without_device_is_a_cuda_error(lib):
     assert bwd(lib, dims()) == m3.MAMBA3_ERR_CUDA
+
+
+def gnorm(lib, d, groups, y=FAKE, z=FAKE, w=None, eps=1e-6, out=FAKE):
+    return lib.mamba3_gated_norm(ctypes.byref(d), groups, y, z, w, eps, out, None)
+
+
+def test_gated_norm_host_validation(lib):
+    d = dims(nheads=4)
+    assert gnorm(lib, d, 3) == m3.MAMBA3_ERR_INVALID          # 3 groups, 4 heads
+    assert gnorm(lib, d, 0) == m3.MAMBA3_ERR_INVALID
+    assert gnorm(lib, d, 2, eps=-1.0) == m3.MAMBA3_ERR_INVALID
+    assert gnorm(lib, d, 2, y=None) == m3.MAMBA3_ERR_INVALID
+    assert gnorm(lib, d, 2, out=FAKE + 8) == m3.MAMBA3_ERR_INVALID
+    assert gnorm(lib, d, 2, w=FAKE + 2) == m3.MAMBA3_ERR_INVALID
+    assert gnorm(lib, dims(nheads=4, seqlen=0), 2, y=None, z=None, out=None) == m3.MAMBA3_OK  # nothing to do
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_gated_norm_valid_call_without_device_is_a_cuda_error(lib):
+    assert gnorm(lib, dims(nheads=4), 2) == m3.MAMBA3_ERR_CUDA
