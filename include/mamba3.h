@@ -233,7 +233,7 @@ MAMBA3_API int mamba3_scan_bwd(const mamba3_dims* dims, const void* x, const voi
  *          in_dtype; dstate, chunk and ngroups are ignored.
  *   y, z, out  [batch, seqlen, nheads, rank, headdim] in_dtype, 16-byte aligned;
  *          out may alias y.
- *   w      float32 [nheads, rank, headdim], 4-byte aligned, or NULL (weight 1).
+ *   w      float32 [nheads, rank, headdim], 16-byte aligned, or NULL (weight 1).
  *   groups divides nheads (nheads: one group per head); eps >= 0.
  * HBM-bound: y and z read once, out written once; computed in float32.
  */

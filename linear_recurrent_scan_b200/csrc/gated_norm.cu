@@ -62,6 +62,24 @@ struct Vec<float> {
 // quotient is 0, the limit of silu
 __device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.f + __expf(-z)); }
 
+// n weights (n a multiple of 4) from a 16-byte aligned address, or 1 without weights
+template <int n>
+__device__ __forceinline__ void load_w(const float* w, float* out) {
+  if (!w) {
+#pragma unroll
+    for (int e = 0; e < n; ++e) out[e] = 1.f;
+    return;
+  }
+#pragma unroll
+  for (int q = 0; q < n / 4; ++q) {
+    const float4 t = reinterpret_cast<const float4*>(w)[q];
+    out[4 * q] = t.x;
+    out[4 * q + 1] = t.y;
+    out[4 * q + 2] = t.z;
+    out[4 * q + 3] = t.w;
+  }
+}
+
 // group of a row (rows are (token, group) in order), in 32 bits when the count fits
 __device__ __forceinline__ int group_of(long long row, const GatedNormArgs& a) {
   return a.rows <= 0xffffffffLL ? (int)((unsigned)row % (unsigned)a.groups) : (int)(row % a.groups);
@@ -121,12 +139,12 @@ __global__ void __launch_bounds__(kTeamThreads) gated_norm_team_kernel(GatedNorm
         const float* w = a.w ? a.w + (size_t)group_of(row, a) * S : nullptr;
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
-          float y[V::N], z[V::N], o[V::N];
+          float y[V::N], z[V::N], wt[V::N], o[V::N];
           V::unpack(yv[u][v], y);
           V::unpack(zv[u][v], z);
-          const int c0 = (v * TEAM + member) * V::N;
+          load_w<V::N>(w ? w + (v * TEAM + member) * V::N : nullptr, wt);
 #pragma unroll
-          for (int e = 0; e < V::N; ++e) o[e] = y[e] * inv * (w ? w[c0 + e] : 1.f) * silu(z[e]);
+          for (int e = 0; e < V::N; ++e) o[e] = y[e] * inv * wt[e] * silu(z[e]);
           O[row * (TEAM * NV) + v * TEAM + member] = V::pack(o);
         }
       }
@@ -176,11 +194,12 @@ __global__ void __launch_bounds__(kRowThreads) gated_norm_row_kernel(GatedNormAr
     const float inv = s_inv;
     for (int v = tid; v < nv; v += nt) {
       if (VEC) {
-        float y[V::N], z[V::N], o[V::N];
+        float y[V::N], z[V::N], wt[V::N], o[V::N];
         V::unpack(reinterpret_cast<const typename V::U*>(yr)[v], y);
         V::unpack(reinterpret_cast<const typename V::U*>(zr)[v], z);
+        load_w<V::N>(w ? w + v * V::N : nullptr, wt);
 #pragma unroll
-        for (int e = 0; e < V::N; ++e) o[e] = y[e] * inv * (w ? w[v * V::N + e] : 1.f) * silu(z[e]);
+        for (int e = 0; e < V::N; ++e) o[e] = y[e] * inv * wt[e] * silu(z[e]);
         reinterpret_cast<typename V::U*>(orow)[v] = V::pack(o);
       } else {
         st1(orow + v, ld1(yr + v) * inv * (w ? w[v] : 1.f) * silu(ld1(zr + v)));

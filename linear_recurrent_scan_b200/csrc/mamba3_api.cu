@@ -282,7 +282,7 @@ int mamba3_gated_norm(const mamba3_dims* d, int groups, const void* y, const voi
   a.y = y; a.z = z; a.w = w; a.eps = eps; a.out = out;
   if (a.rows > 0) {
     if (!y || !z || !out || !aligned16(y) || !aligned16(z) || !aligned16(out)) return MAMBA3_ERR_INVALID;
-    if (w && !aligned4(w)) return MAMBA3_ERR_INVALID;
+    if (w && !aligned16(w)) return MAMBA3_ERR_INVALID;
   }
   return m3::launch_gated_norm(a, static_cast<cudaStream_t>(stream));
 }

@@ -85,12 +85,16 @@ __device__ __forceinline__ void block_add(float v, float* dst) {
   if ((threadIdx.x & 31) == 0) atomicAdd(dst, v);
 }
 
-template <typename T>
+// NT, PT, RT: N, P, R fixed at compile time (inner loops unrolled), or 0 to take
+// them from the arguments.
+template <typename T, int NT, int PT, int RT>
 __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLayout lay) {
   extern __shared__ float sm[];
   __shared__ int s_pend_t;  // first token of the chunk processed last, its lagged-weight share pending
+  __shared__ float s_erow[kRows];  // e^{cum} of each row's token
   const ScanArgs& a = g.f;
-  const int P = a.P, N = a.N, R = a.R, Q = lay.Q, L = a.seqlen, K = N / 2, NP = N * P;
+  const int P = PT ? PT : a.P, N = NT ? NT : a.N, R = RT ? RT : a.R;
+  const int Q = RT ? kRows / RT : lay.Q, L = a.seqlen, K = N / 2, NP = N * P;
   const int PS = P + 1, NS = N + 1;  // padded row strides (hbar, G, X, dY; B~, C~)
   const int unit = blockIdx.x;
   const int b = unit / a.nheads, hh = unit % a.nheads;
@@ -253,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     for (int i = tid; i < NP; i += kThreads) {
       const int n = i / P, p = i % P;
       float acc = ecend * hb[n * PS + p];
+#pragma unroll 8
       for (int j = 0; j < M; ++j) acc += sB[j * NS + n] * sX[j * PS + p];
       hb[n * PS + p] = acc;
     }
@@ -288,12 +293,15 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     const float ecend = expf(s_cum[q - 1]);
 
     // (1) row pairs (token of j <= token of m): S = K o P1, W = K o P2, P1 o P2
+    for (int m = tid; m < M; m += kThreads) s_erow[m] = s_ecum[m / R];
     for (int i = tid; i < M * M; i += kThreads) {
       const int m = i / M, j = i % M, tm = m / R, tj = j / R;
       float vs = 0.f, vw = 0.f, vq = 0.f;
       if (tj <= tm) {
         float p1 = 0.f, p2 = 0.f;
+#pragma unroll 8
         for (int n = 0; n < N; ++n) p1 += sC[m * NS + n] * sB[j * NS + n];
+#pragma unroll 8
         for (int p = 0; p < P; ++p) p2 += sdY[m * PS + p] * sX[j * PS + p];
         const float kern = (tj == tm) ? s_gam[tm] : expf(s_cum[tm] - s_cum[tj]) * s_w[tj];
         vs = kern * p1;
@@ -320,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     for (int i = tid; i < M * P; i += kThreads) {
       const int m = i / P, p = i % P, t = m / R, r = m % R;
       float yi = 0.f, bg = 0.f;
+#pragma unroll 8
       for (int n = 0; n < N; ++n) {
         yi += sC[m * NS + n] * hb[n * PS + p];
         bg += sB[m * NS + n] * G[n * PS + p];
@@ -345,6 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     for (int i = tid; i < M * N; i += kThreads) {
       const int m = i / N, n = i % N, t = m / R, r = m % R;
       float dc = 0.f, db = 0.f;
+#pragma unroll 8
       for (int p = 0; p < P; ++p) {
         dc += sdY[m * PS + p] * hb[n * PS + p];
         db += sX[m * PS + p] * G[n * PS + p];
@@ -363,7 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     for (int i = tid; i < NP; i += kThreads) {
       const int n = i / P, p = i % P;
       float acc = ecend * G[n * PS + p];
-      for (int m = 0; m < M; ++m) acc += s_ecum[m / R] * sC[m * NS + n] * sdY[m * PS + p];
+#pragma unroll 8
+      for (int m = 0; m < M; ++m) acc += s_erow[m] * sC[m * NS + n] * sdY[m * PS + p];
       G[n * PS + p] = acc;
     }
     // rotation back (dB = rot(+Phi) dB~) and the angle's share, from the chunk's last token
@@ -509,17 +520,22 @@ int launch_scan_bwd(const BwdArgs& g, cudaStream_t s) {
   const int units = a.batch * a.nheads;
   if (units == 0) return MAMBA3_OK;
   const BwdLayout lay = bwd_layout(a.P, a.N, a.R);
-  if (a.dtype == MAMBA3_F32) {
-    auto k = scan_bwd_kernel<float>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total) != cudaSuccess)
-      return MAMBA3_ERR_CUDA;
-    k<<<units, kThreads, lay.total, s>>>(g, lay);
+  using KFn = void (*)(BwdArgs, BwdLayout);
+  KFn k = nullptr;
+  if (a.dtype == MAMBA3_BF16 && a.P == 64 && (a.N == 64 || a.N == 128) && (a.R == 1 || a.R == 2 || a.R == 4)) {
+    using B16 = __nv_bfloat16;
+    if (a.N == 128)
+      k = a.R == 1 ? scan_bwd_kernel<B16, 128, 64, 1> : (a.R == 2 ? scan_bwd_kernel<B16, 128, 64, 2>
+                                                                  : scan_bwd_kernel<B16, 128, 64, 4>);
+    else
+      k = a.R == 1 ? scan_bwd_kernel<B16, 64, 64, 1> : (a.R == 2 ? scan_bwd_kernel<B16, 64, 64, 2>
+                                                                 : scan_bwd_kernel<B16, 64, 64, 4>);
   } else {
-    auto k = scan_bwd_kernel<__nv_bfloat16>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total) != cudaSuccess)
-      return MAMBA3_ERR_CUDA;
-    k<<<units, kThreads, lay.total, s>>>(g, lay);
+    k = a.dtype == MAMBA3_F32 ? scan_bwd_kernel<float, 0, 0, 0> : scan_bwd_kernel<__nv_bfloat16, 0, 0, 0>;
   }
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total) != cudaSuccess)
+    return MAMBA3_ERR_CUDA;
+  k<<<units, kThreads, lay.total, s>>>(g, lay);
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 

@@ -278,7 +278,7 @@ def test_gated_norm_host_validation(lib):
     assert gnorm(lib, d, 2, eps=-1.0) == m3.MAMBA3_ERR_INVALID
     assert gnorm(lib, d, 2, y=None) == m3.MAMBA3_ERR_INVALID
     assert gnorm(lib, d, 2, out=FAKE + 8) == m3.MAMBA3_ERR_INVALID
-    assert gnorm(lib, d, 2, w=FAKE + 2) == m3.MAMBA3_ERR_INVALID
+    assert gnorm(lib, d, 2, w=FAKE + 4) == m3.MAMBA3_ERR_INVALID  # w: 16-byte aligned
     assert gnorm(lib, dims(nheads=4, seqlen=0), 2, y=None, z=None, out=None) == m3.MAMBA3_OK  # nothing to do
 
 
