@@ -41,8 +41,8 @@ constexpr int kNScal = 14;  // per-token scalar arrays of the backward chunk
 
 struct BwdLayout {
   int M, Q;
-  size_t off_hb, off_G, off_B, off_C, off_dB, off_dC, off_X, off_dY, off_S, off_W, off_Q, off_phi, off_T, off_sc,
-      off_ang, off_misc, total;
+  size_t off_hb, off_G, off_B, off_C, off_dB, off_dC, off_X, off_dY, off_S, off_W, off_Q, off_phi, off_th, off_T,
+      off_sc, off_ang, off_misc, total;
 };
 
 BwdLayout bwd_layout(int P, int N, int R) {
@@ -70,6 +70,7 @@ BwdLayout bwd_layout(int P, int N, int R) {
   l.off_W = take((size_t)l.M * l.M);
   l.off_Q = take((size_t)l.M * l.M);
   l.off_phi = take((size_t)l.Q * K);
+  l.off_th = take((size_t)l.Q * K);
   l.off_T = take((size_t)l.Q * l.Q);
   l.off_sc = take((size_t)kNScal * (l.Q + 1));
   l.off_ang = take((size_t)2 * K);
@@ -111,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
   float* sW = sm + lay.off_W;      // [M][M] K o (dY X^T)
   float* sQ = sm + lay.off_Q;      // [M][M] (C~ B~^T) o (dY X^T)
   float* phit = sm + lay.off_phi;  // [Q][K] angle of each token of the chunk
+  float* sth = sm + lay.off_th;    // [Q][K] theta of the chunk's tokens
   float* sT = sm + lay.off_T;      // [Q][Q] e^{cum_t - cum_j} Z(t, j) for t > j
   const int QS = Q + 1;
   float* sc = sm + lay.off_sc;
@@ -179,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
       sX[m * PS + p] = ld1(X + gi);
       if (backward) sdY[m * PS + p] = ld1(DY + gi);
     }
+    for (int i = tid; i < q * K; i += kThreads) sth[i] = ld1(TH + tok(t0 + i / K) * K + i % K);
   };
   // decay scan of the chunk (one thread): cum, gamma, w, e^{cum}, e^{cum_end - cum}
   auto decay_scalars = [&](int q) {
@@ -201,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     for (int k = tid; k < K; k += kThreads) {
       float local = 0.f;
       for (int i = 0; i < q; ++i) {
-        local += s_dt[i] * ld1(TH + tok(t0 + i) * K + k);
+        local += s_dt[i] * sth[i * K + k];
         const float ph = phi[k] + local;
         phit[i * K + k] = ph;
         float sn, cs;
@@ -399,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
         Sk += dphi;
         const size_t ti = tok(t0 + i) * K + k;
         st1(dTHg + ti, s_dt[i] * Sk);
-        atomicAdd(&s_dth[i], ld1(TH + ti) * Sk);
+        atomicAdd(&s_dth[i], sth[i * K + k] * Sk);
       }
       Sang[k] = Sk;
     }
