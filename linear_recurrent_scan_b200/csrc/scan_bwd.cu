@@ -226,6 +226,45 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     }
   };
 
+  // St[n][p] = scale St[n][p] + sum_{j < M} f_j A[j][n] Bm[j][p]  (f = 1 when f_row is null).
+  // With N, P fixed at compile time a thread keeps N/16 rows x 2 columns in registers.
+  auto state_update = [&](float* St, const float* A, const float* Bm, const float* f_row, float scale, int M) {
+    if constexpr (NT != 0 && PT == 64 && kThreads == 512) {
+      constexpr int NR = NT / 16;
+      const int n0 = tid >> 5, p0 = tid & 31;
+      float acc[NR][2];
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        acc[i][0] = scale * St[(n0 + 16 * i) * PS + p0];
+        acc[i][1] = scale * St[(n0 + 16 * i) * PS + p0 + 32];
+      }
+#pragma unroll 4
+      for (int j = 0; j < M; ++j) {
+        const float f = f_row ? f_row[j] : 1.f;
+        const float d0 = f * Bm[j * PS + p0], d1 = f * Bm[j * PS + p0 + 32];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          const float c = A[j * NS + n0 + 16 * i];
+          acc[i][0] += c * d0;
+          acc[i][1] += c * d1;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        St[(n0 + 16 * i) * PS + p0] = acc[i][0];
+        St[(n0 + 16 * i) * PS + p0 + 32] = acc[i][1];
+      }
+    } else {
+      for (int i = tid; i < NP; i += kThreads) {
+        const int n = i / P, p = i % P;
+        float acc = scale * St[n * PS + p];
+#pragma unroll 8
+        for (int j = 0; j < M; ++j) acc += (f_row ? f_row[j] : 1.f) * A[j * NS + n] * Bm[j * PS + p];
+        St[n * PS + p] = acc;
+      }
+    }
+  };
+
   // ---------------- pass 1: hbar and Phi at every chunk start ----------------
   const float mu1 = (1.f - ld1(LM + tok(0))) * ld1(DT + tok(0));  // weight of the initial lagged term
   for (int i = tid; i < NP; i += kThreads) {
@@ -256,14 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
       sX[m * PS + p] *= s_eend[m / R] * s_w[m / R];
     }
     __syncthreads();
-    const float ecend = expf(s_cum[q - 1]);
-    for (int i = tid; i < NP; i += kThreads) {
-      const int n = i / P, p = i % P;
-      float acc = ecend * hb[n * PS + p];
-#pragma unroll 8
-      for (int j = 0; j < M; ++j) acc += sB[j * NS + n] * sX[j * PS + p];
-      hb[n * PS + p] = acc;
-    }
+    state_update(hb, sB, sX, nullptr, expf(s_cum[q - 1]), M);
     __syncthreads();
   }
 
@@ -328,14 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
       sT[t * Q + j] = (j < t) ? expf(s_cum[t] - s_cum[j]) * z : 0.f;
     }
     // (3) dX, and per token the paths hbar_in -> y_t and u_j -> hbar_out
-    for (int i = tid; i < M * P; i += kThreads) {
-      const int m = i / P, p = i % P, t = m / R, r = m % R;
-      float yi = 0.f, bg = 0.f;
-#pragma unroll 8
-      for (int n = 0; n < N; ++n) {
-        yi += sC[m * NS + n] * hb[n * PS + p];
-        bg += sB[m * NS + n] * G[n * PS + p];
-      }
+    // (yi = (C~ hbar_in)[m][p] and bg = (B~ G)[m][p] come in from the loops below)
+    auto dx_out = [&](int m, int p, float yi, float bg) {
+      const int t = m / R, r = m % R;
       float sdy = 0.f;
       for (int j = t * R; j < M; ++j) sdy += sS[j * M + m] * sdY[j * PS + p];
       const float dy = sdY[m * PS + p], xv = sX[m * PS + p];
@@ -345,6 +372,41 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
       atomicAdd(&s_zin[t], s_ecum[t] * dy * yi);
       atomicAdd(&s_zue[t], s_eend[t] * xv * bg);
       dD_acc += dy * xv;
+    };
+    if constexpr (NT != 0 && PT == 64 && kThreads == 512) {
+      const int m0 = tid >> 5, p0 = tid & 31;  // rows m0, m0 + 16; columns p0, p0 + 32
+      float yi[2][2] = {}, bg[2][2] = {};
+#pragma unroll 4
+      for (int n = 0; n < NT; ++n) {
+        const float c0 = sC[m0 * NS + n], c1 = sC[(m0 + 16) * NS + n];
+        const float b0 = sB[m0 * NS + n], b1 = sB[(m0 + 16) * NS + n];
+        const float h0 = hb[n * PS + p0], h1 = hb[n * PS + p0 + 32];
+        const float g0 = G[n * PS + p0], g1 = G[n * PS + p0 + 32];
+        yi[0][0] += c0 * h0;
+        yi[0][1] += c0 * h1;
+        yi[1][0] += c1 * h0;
+        yi[1][1] += c1 * h1;
+        bg[0][0] += b0 * g0;
+        bg[0][1] += b0 * g1;
+        bg[1][0] += b1 * g0;
+        bg[1][1] += b1 * g1;
+      }
+#pragma unroll
+      for (int a2 = 0; a2 < 2; ++a2)
+#pragma unroll
+        for (int b2 = 0; b2 < 2; ++b2)
+          if (m0 + 16 * a2 < M) dx_out(m0 + 16 * a2, p0 + 32 * b2, yi[a2][b2], bg[a2][b2]);
+    } else {
+      for (int i = tid; i < M * P; i += kThreads) {
+        const int m = i / P, p = i % P;
+        float yi = 0.f, bg = 0.f;
+#pragma unroll 8
+        for (int n = 0; n < N; ++n) {
+          yi += sC[m * NS + n] * hb[n * PS + p];
+          bg += sB[m * NS + n] * G[n * PS + p];
+        }
+        dx_out(m, p, yi, bg);
+      }
     }
     {
       float part = 0.f;
@@ -354,6 +416,60 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     __syncthreads();
 
     // (4) dC~ = diag(e^cum) dY hbar_in^T + W B~,  dB~ = diag(w e^{cum_end - cum}) X G^T + W^T C~
+    if constexpr (NT != 0 && PT == 64 && kThreads == 512) {
+      constexpr int NC = NT / 32;
+      const int m0 = tid >> 5, n0 = tid & 31;  // rows m0, m0 + 16; columns n0 + 32 c
+      float dc[2][NC] = {}, db[2][NC] = {};
+#pragma unroll 4
+      for (int p = 0; p < PT; ++p) {
+        const float y0 = sdY[m0 * PS + p], y1 = sdY[(m0 + 16) * PS + p];
+        const float x0 = sX[m0 * PS + p], x1 = sX[(m0 + 16) * PS + p];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          const float h = hb[(n0 + 32 * c) * PS + p], gg = G[(n0 + 32 * c) * PS + p];
+          dc[0][c] += y0 * h;
+          dc[1][c] += y1 * h;
+          db[0][c] += x0 * gg;
+          db[1][c] += x1 * gg;
+        }
+      }
+#pragma unroll
+      for (int a2 = 0; a2 < 2; ++a2) {
+        const int t = (m0 + 16 * a2) / R;  // rows past M are computed but never stored
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          dc[a2][c] *= s_ecum[t];
+          db[a2][c] *= s_w[t] * s_eend[t];
+        }
+      }
+      // W is zero outside the causal triangle, so j runs over every row
+#pragma unroll 4
+      for (int j = 0; j < M; ++j) {
+        const float wa0 = sW[m0 * M + j], wa1 = sW[(m0 + 16) * M + j];
+        const float wb0 = sW[j * M + m0], wb1 = sW[j * M + m0 + 16];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          const float bj = sB[j * NS + n0 + 32 * c], cj = sC[j * NS + n0 + 32 * c];
+          dc[0][c] += wa0 * bj;
+          dc[1][c] += wa1 * bj;
+          db[0][c] += wb0 * cj;
+          db[1][c] += wb1 * cj;
+        }
+      }
+#pragma unroll
+      for (int a2 = 0; a2 < 2; ++a2) {
+        const int m = m0 + 16 * a2, t = m / R, r = m % R;
+        if (m < M)
+#pragma unroll
+          for (int c = 0; c < NC; ++c) {
+            const int n = n0 + 32 * c;
+            float dbv = db[a2][c];
+            if (t0 + t == L - 1 && g.dbprev_out) dbv += g.dbprev_out[(us * R + r) * N + n];
+            dBt[m * N + n] = dbv;
+            dCt[m * N + n] = dc[a2][c];
+          }
+      }
+    } else
     for (int i = tid; i < M * N; i += kThreads) {
       const int m = i / N, n = i % N, t = m / R, r = m % R;
       float dc = 0.f, db = 0.f;
@@ -373,13 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     __syncthreads();
 
     // (5) dL/dhbar_in = e^{cum_end} G + C~^T diag(e^cum) dY (in place)
-    for (int i = tid; i < NP; i += kThreads) {
-      const int n = i / P, p = i % P;
-      float acc = ecend * G[n * PS + p];
-#pragma unroll 8
-      for (int m = 0; m < M; ++m) acc += s_erow[m] * sC[m * NS + n] * sdY[m * PS + p];
-      G[n * PS + p] = acc;
-    }
+    state_update(G, sC, sdY, s_erow, ecend, M);
     // rotation back (dB = rot(+Phi) dB~) and the angle's share, from the chunk's last token
     for (int k = tid; k < K; k += kThreads) {
       float Sk = Sang[k];
