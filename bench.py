@@ -55,6 +55,10 @@ TRAFFIC = {
                         "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "grouped_decode": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), "7ccbdf6b735872e61661a0e4d8ad33ec2f120e42692c1cc6ce802987011c2987", 279056128 + 219058176,
                        "profiles/grouped_bc_prefill_decode_traffic.txt"),
+    "backward": (("scan_bwd.cu", "common.cuh"), "6422b8e559b99e07fbcfd9e284d4def475a0227dc70fb805a8181346dcad0f77", 2411331328 + 1887158016,
+                 "profiles/scan_bwd_siso_b8_l2048_traffic_and_counters.txt"),
+    "gated_norm_per_head": (("gated_norm.cu", "common.cuh"), "eb90ad7d72a2607cc062684461d599cc86e5eea7058c9d970afd24eac530e380", 268479232 + 103046400,
+                            "profiles/gated_norm_b8_l2048_traffic_and_counters.txt"),
 }
 
 
@@ -527,7 +531,7 @@ def ours(args):
     bwd = {"prefill_" + PREFILL.name: {"ms_per_launch": round(ms, 3), "kernel": "scan_bwd_kernel (SIMT, fp32)",
                                        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
                                                     "unit": "GB/s", "frac": round(gbs / peak, 5),
-                                                    "bytes_per_launch": by}}}
+                                                    "traffic": traffic("backward"), "bytes_per_launch": by}}}
     # the output side on the headline prefill's y: grouped RMS norm + gate
     gated = {}
     for ng in (PREFILL.nheads, 8):
@@ -538,7 +542,8 @@ def ours(args):
         gated["prefill_%s_groups%d" % (PREFILL.name, ng)] = {
             "ms_per_launch": round(ms, 4), "norm_groups": ng,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(gbs / peak, 4), "bytes_per_launch": by}}
+                         "frac": round(gbs / peak, 4), "bytes_per_launch": by,
+                         "traffic": traffic("gated_norm_per_head") if ng == PREFILL.nheads else None}}
     more = {}
     for w in PREFILL_MORE:
         ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=max(5, min(args.steps, 20)), warmup=3), world)
