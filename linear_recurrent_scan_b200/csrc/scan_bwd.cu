@@ -79,6 +79,12 @@ BwdLayout bwd_layout(int P, int N, int R) {
   return l;
 }
 
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 // Block-wide sum of one float per thread, added to *dst (shared memory).
 __device__ __forceinline__ void block_add(float v, float* dst) {
 #pragma unroll
@@ -183,19 +189,24 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     }
     for (int i = tid; i < q * K; i += kThreads) sth[i] = ld1(TH + tok(t0 + i / K) * K + i % K);
   };
-  // decay scan of the chunk (one thread): cum, gamma, w, e^{cum}, e^{cum_end - cum}
+  // decay scan of the chunk (warp 0, one lane per token, q <= 32): cum, gamma, w,
+  // e^{cum}, e^{cum_end - cum}
   auto decay_scalars = [&](int q) {
-    if (tid == 0) {
-      float c = 0.f;
-      for (int i = 0; i < q; ++i) {
-        c += s_dt[i] * Ah;
+    if (tid < 32) {
+      const int i = tid;
+      float c = i < q ? s_dt[i] * Ah : 0.f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, c, o);
+        if (i >= o) c += v;
+      }
+      const float cend = __shfl_sync(0xffffffffu, c, q - 1);
+      if (i < q) {
         s_cum[i] = c;
         s_gam[i] = s_lam[i] * s_dt[i];
         s_w[i] = s_gam[i] + (1.f - s_lam[i + 1]) * s_dt[i + 1];
-      }
-      for (int i = 0; i < q; ++i) {
-        s_ecum[i] = expf(s_cum[i]);
-        s_eend[i] = expf(c - s_cum[i]);
+        s_ecum[i] = expf(c);
+        s_eend[i] = expf(cend - c);
       }
     }
   };
@@ -361,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     }
     // (3) dX, and per token the paths hbar_in -> y_t and u_j -> hbar_out
     // (yi = (C~ hbar_in)[m][p] and bg = (B~ G)[m][p] come in from the loops below)
-    auto dx_out = [&](int m, int p, float yi, float bg) {
+    auto dx_out = [&](int m, int p, float yi, float bg, float& zin_c, float& zue_c) {
       const int t = m / R, r = m % R;
       float sdy = 0.f;
       for (int j = t * R; j < M; ++j) sdy += sS[j * M + m] * sdY[j * PS + p];
@@ -369,8 +380,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
       float dxv = s_w[t] * s_eend[t] * bg + sdy + Dh * dy;
       if (t0 + t == L - 1 && g.dxprev_out) dxv += g.dxprev_out[(us * R + r) * P + p];
       st1(dXg + tok(t0 + t) * R * P + (size_t)r * P + p, dxv);
-      atomicAdd(&s_zin[t], s_ecum[t] * dy * yi);
-      atomicAdd(&s_zue[t], s_eend[t] * xv * bg);
+      zin_c = s_ecum[t] * dy * yi;
+      zue_c = s_eend[t] * xv * bg;
       dD_acc += dy * xv;
     };
     if constexpr (NT != 0 && PT == 64 && kThreads == 512) {
@@ -391,11 +402,26 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
         bg[1][0] += b1 * g0;
         bg[1][1] += b1 * g1;
       }
+      // a warp holds one row (one token): sum its lanes before the shared atomics
 #pragma unroll
-      for (int a2 = 0; a2 < 2; ++a2)
+      for (int a2 = 0; a2 < 2; ++a2) {
+        const int m = m0 + 16 * a2;
+        float zi = 0.f, zu = 0.f;
+        if (m < M)
 #pragma unroll
-        for (int b2 = 0; b2 < 2; ++b2)
-          if (m0 + 16 * a2 < M) dx_out(m0 + 16 * a2, p0 + 32 * b2, yi[a2][b2], bg[a2][b2]);
+          for (int b2 = 0; b2 < 2; ++b2) {
+            float ci, cu;
+            dx_out(m, p0 + 32 * b2, yi[a2][b2], bg[a2][b2], ci, cu);
+            zi += ci;
+            zu += cu;
+          }
+        zi = warp_sum(zi);
+        zu = warp_sum(zu);
+        if (p0 == 0 && m < M) {
+          atomicAdd(&s_zin[m / R], zi);
+          atomicAdd(&s_zue[m / R], zu);
+        }
+      }
     } else {
       for (int i = tid; i < M * P; i += kThreads) {
         const int m = i / P, p = i % P;
@@ -405,7 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
           yi += sC[m * NS + n] * hb[n * PS + p];
           bg += sB[m * NS + n] * G[n * PS + p];
         }
-        dx_out(m, p, yi, bg);
+        float ci, cu;
+        dx_out(m, p, yi, bg, ci, cu);
+        atomicAdd(&s_zin[m / R], ci);
+        atomicAdd(&s_zue[m / R], cu);
       }
     }
     {
@@ -512,7 +541,12 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
         Sk += dphi;
         const size_t ti = tok(t0 + i) * K + k;
         st1(dTHg + ti, s_dt[i] * Sk);
-        atomicAdd(&s_dth[i], sth[i * K + k] * Sk);
+        if constexpr (NT != 0) {  // K a multiple of 32: whole warps walk the tokens together
+          const float v = warp_sum(sth[i * K + k] * Sk);
+          if ((tid & 31) == 0) atomicAdd(&s_dth[i], v);
+        } else {
+          atomicAdd(&s_dth[i], sth[i * K + k] * Sk);
+        }
       }
       Sang[k] = Sk;
     }
