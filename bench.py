@@ -55,7 +55,7 @@ TRAFFIC = {
                         "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "grouped_decode": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), "7ccbdf6b735872e61661a0e4d8ad33ec2f120e42692c1cc6ce802987011c2987", 279056128 + 219058176,
                        "profiles/grouped_bc_prefill_decode_traffic.txt"),
-    "backward": (("scan_bwd.cu", "common.cuh"), "6422b8e559b99e07fbcfd9e284d4def475a0227dc70fb805a8181346dcad0f77", 2411331328 + 1887158016,
+    "backward": (("scan_bwd.cu", "common.cuh"), "cfca736f5dd9e50ceaf7e528b3eed4f8a06f38efcfde4246e604a60514bcf42f", 2366348288 + 1885662208,
                  "profiles/scan_bwd_siso_b8_l2048_traffic_and_counters.txt"),
     "gated_norm_per_head": (("gated_norm.cu", "common.cuh"), "eb90ad7d72a2607cc062684461d599cc86e5eea7058c9d970afd24eac530e380", 268479232 + 103046400,
                             "profiles/gated_norm_b8_l2048_traffic_and_counters.txt"),
