@@ -211,6 +211,8 @@ MAMBA3_API int mamba3_decode_step_at(const mamba3_dims* dims, const mamba3_state
  *                 Q = 32 / rank), after the 256-byte status word.
  * Computed in float32 whatever in_dtype is.  Returns MAMBA3_ERR_UNSUPPORTED for
  * grouped B/C, and for N, P whose per-chunk tiles exceed shared memory.
+ * mamba3_scan_bwd_at is the same for mamba3_scan_fwd_at: A_t [b, L, H] (dtype of x)
+ * in place of A, and dA_t (layout and dtype of A_t, not nullable) in place of dA.
  */
 MAMBA3_API size_t mamba3_scan_bwd_workspace_bytes(const mamba3_dims* dims);
 MAMBA3_API int mamba3_scan_bwd(const mamba3_dims* dims, const void* x, const void* B, const void* C,
@@ -219,6 +221,12 @@ MAMBA3_API int mamba3_scan_bwd(const mamba3_dims* dims, const void* x, const voi
                                const mamba3_state* d_final, void* dx, void* dB, void* dC, void* dtheta,
                                void* ddt, void* dlam, float* dA, float* dD, const mamba3_state* d_init,
                                void* workspace, size_t workspace_bytes, void* stream);
+MAMBA3_API int mamba3_scan_bwd_at(const mamba3_dims* dims, const void* x, const void* B, const void* C,
+                                  const void* theta, const void* dt, const void* lam, const void* A_t,
+                                  const float* D, const mamba3_state* init, const void* dy,
+                                  const mamba3_state* d_final, void* dx, void* dB, void* dC, void* dtheta,
+                                  void* ddt, void* dlam, void* dA_t, float* dD, const mamba3_state* d_init,
+                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Output side of the layer: the pre-gate grouped RMS norm and the gate

@@ -112,6 +112,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                     ctypes.POINTER(_CState), vp, vp, vp, vp, vp, vp, vp, vp,
                                     ctypes.POINTER(_CState), vp, sz, vp]
     lib.mamba3_scan_bwd.restype = i
+    lib.mamba3_scan_bwd_at.argtypes = lib.mamba3_scan_bwd.argtypes
+    lib.mamba3_scan_bwd_at.restype = i
     lib.mamba3_gated_norm.argtypes = [ctypes.POINTER(Dims), i, vp, vp, vp, ctypes.c_float, vp, vp]
     lib.mamba3_gated_norm.restype = i
     _lib = lib
@@ -382,8 +384,22 @@ def mamba3_scan_bwd(x, B, C, theta, dt, lam, A, D, dy, init: Optional[State] = N
     dC, dtheta, ddt, dlam (shaped and typed like the inputs), dA, dD (fp32
     [H]) and d_init (a State: the initial state's gradients).  ``grads`` may
     hold preallocated outputs under those names."""
+    return _scan_bwd(x, B, C, theta, dt, lam, A, None, D, dy, init, d_final, grads, workspace, stream)
+
+
+def mamba3_scan_bwd_at(x, B, C, theta, dt, lam, A_t, D, dy, init: Optional[State] = None,
+                       d_final: Optional[State] = None, grads: Optional[dict] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """mamba3_scan_bwd for mamba3_scan_fwd_at: A_t [b, L, H] (dtype of x); the
+    dict holds dA_t (shaped and typed like A_t) in place of dA."""
+    return _scan_bwd(x, B, C, theta, dt, lam, None, A_t, D, dy, init, d_final, grads, workspace, stream)
+
+
+def _scan_bwd(x, B, C, theta, dt, lam, A, A_t, D, dy, init, d_final, grads, workspace, stream) -> dict:
     lib = load_library()
     _check_inputs(x, B, C, theta, dt, lam, A, D, decode=False)
+    if A_t is not None:
+        _check_at(A_t, dt, x)
     if dy.shape != x.shape or dy.dtype != x.dtype or not dy.is_contiguous() or dy.device != x.device:
         raise ValueError("dy must be a contiguous tensor shaped and typed like x")
     dims = make_dims(x, B)
@@ -393,9 +409,12 @@ def mamba3_scan_bwd(x, B, C, theta, dt, lam, A, D, dy, init: Optional[State] = N
     for name, like in (("dx", x), ("dB", B), ("dC", C), ("dtheta", theta), ("ddt", dt), ("dlam", lam)):
         if name not in out:
             out[name] = torch.empty_like(like)
-    for name in ("dA", "dD"):
-        if name not in out:
-            out[name] = torch.empty(H, dtype=torch.float32, device=x.device)
+    rate_grad = "dA" if A_t is None else "dA_t"
+    if rate_grad not in out:
+        out[rate_grad] = (torch.empty(H, dtype=torch.float32, device=x.device) if A_t is None
+                          else torch.empty_like(A_t))
+    if "dD" not in out:
+        out["dD"] = torch.empty(H, dtype=torch.float32, device=x.device)
     if "d_init" not in out:
         out["d_init"] = State.zeros(b, H, P, N, R, device=x.device)
     if workspace is None:
@@ -403,13 +422,14 @@ def mamba3_scan_bwd(x, B, C, theta, dt, lam, A, D, dy, init: Optional[State] = N
     ci = init._c() if init is not None else None
     cf = d_final._c() if d_final is not None else None
     cd = out["d_init"]._c()
-    rc = lib.mamba3_scan_bwd(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam),
-                             _ptr(A), _ptr(D), ctypes.byref(ci) if ci is not None else None, _ptr(dy),
-                             ctypes.byref(cf) if cf is not None else None, _ptr(out["dx"]), _ptr(out["dB"]),
-                             _ptr(out["dC"]), _ptr(out["dtheta"]), _ptr(out["ddt"]), _ptr(out["dlam"]),
-                             _ptr(out["dA"]), _ptr(out["dD"]), ctypes.byref(cd), _ptr(workspace),
-                             workspace.numel() * workspace.element_size(), _stream(stream))
-    _check(rc, "mamba3_scan_bwd")
+    fn = lib.mamba3_scan_bwd if A_t is None else lib.mamba3_scan_bwd_at
+    rc = fn(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam),
+            _ptr(A if A_t is None else A_t), _ptr(D), ctypes.byref(ci) if ci is not None else None, _ptr(dy),
+            ctypes.byref(cf) if cf is not None else None, _ptr(out["dx"]), _ptr(out["dB"]),
+            _ptr(out["dC"]), _ptr(out["dtheta"]), _ptr(out["ddt"]), _ptr(out["dlam"]),
+            _ptr(out[rate_grad]), _ptr(out["dD"]), ctypes.byref(cd), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mamba3_scan_bwd" if A_t is None else "mamba3_scan_bwd_at")
     return out
 
 
@@ -451,6 +471,7 @@ __all__ = [
     "Dims", "State", "BCNorm", "Mamba3Error", "load_library", "make_dims",
     "mamba3_scan_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc", "mamba3_decode_step",
     "mamba3_scan_fwd_bcnorm", "mamba3_decode_step_bcnorm", "mamba3_scan_fwd_at", "mamba3_decode_step_at",
-    "mamba3_scan_bwd_workspace_bytes", "mamba3_scan_bwd", "mamba3_gated_norm", "mamba3_device_status",
+    "mamba3_scan_bwd_workspace_bytes", "mamba3_scan_bwd", "mamba3_scan_bwd_at", "mamba3_gated_norm",
+    "mamba3_device_status",
     "mamba3_status_string",
 ]

@@ -48,6 +48,7 @@ struct BwdArgs {
   const float *dh_out, *dbprev_out, *dxprev_out, *dangle_out;    // all null = no exported-state gradient
   void *dx, *dB, *dC, *dtheta, *ddt, *dlam;                      // layouts and dtype of the inputs
   float *dA, *dD;                                                // [H], zeroed by the launcher; dD nullable
+  void* dA_t;  // with f.A_t: the decay-rate gradient per token (layout of dt, dtype of x); dA null
   float *dh0, *dbprev0, *dxprev0, *dangle0;                      // all null = not wanted
   float* ckpt;  // [units][chunks][N*P + N/2]: hbar and Phi at every chunk start
 };

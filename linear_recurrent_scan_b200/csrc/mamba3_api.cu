@@ -228,6 +228,52 @@ int mamba3_device_status(const void* workspace, void* stream) {
   return st.code;
 }
 
+}  // extern "C"
+
+namespace {
+// The backward pass behind mamba3_scan_bwd (A per head, dA) and mamba3_scan_bwd_at
+// (A_t per token, dA_t); the rate and its gradient were checked by the caller.
+int scan_bwd_impl(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                  const void* dt, const void* lam, const float* A, const void* A_t, const float* D,
+                  const mamba3_state* init, const void* dy, const mamba3_state* d_final, void* dx, void* dB,
+                  void* dC, void* dtheta, void* ddt, void* dlam, float* dA, void* dA_t, float* dD,
+                  const mamba3_state* d_init, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(d, true);
+  if (rc) return rc;
+  if (dD && !aligned4(dD)) return MAMBA3_ERR_INVALID;
+  const float* rate = A ? A : static_cast<const float*>(A_t);  // the rate array that must be present
+  if (d->seqlen > 0) {
+    if ((rc = check_inputs(x, B, C, theta, dt, lam, rate, D, dy))) return rc;
+    if ((rc = check_inputs(dx, dB, dC, dtheta, ddt, dlam, rate, D, dy))) return rc;  // the gradients' layouts
+  }
+  if ((rc = check_state(init)) || (rc = check_state(d_final)) || (rc = check_state(d_init))) return rc;
+  if (!workspace || !aligned16(workspace)) return MAMBA3_ERR_WORKSPACE;
+  if (workspace_bytes < kStatusBytes + m3::bwd_checkpoint_bytes(scan_args(d, nullptr, nullptr, nullptr, nullptr,
+                                                                           nullptr, nullptr, nullptr, nullptr,
+                                                                           nullptr)))
+    return MAMBA3_ERR_WORKSPACE;
+  m3::BwdArgs g;
+  memset(&g, 0, sizeof(g));
+  g.f = scan_args(d, x, B, C, theta, dt, lam, A, D, init);
+  g.f.A_t = A_t;
+  g.f.workspace = workspace;
+  g.f.workspace_bytes = workspace_bytes;
+  if ((rc = m3::bwd_supported(g.f))) return rc;
+  g.dy = dy;
+  if (d_final) {
+    g.dh_out = d_final->h; g.dbprev_out = d_final->b_prev; g.dxprev_out = d_final->x_prev; g.dangle_out = d_final->angle;
+  }
+  g.dx = dx; g.dB = dB; g.dC = dC; g.dtheta = dtheta; g.ddt = ddt; g.dlam = dlam; g.dA = dA; g.dA_t = dA_t; g.dD = dD;
+  if (d_init) { g.dh0 = d_init->h; g.dbprev0 = d_init->b_prev; g.dxprev0 = d_init->x_prev; g.dangle0 = d_init->angle; }
+  g.ckpt = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  return m3::launch_scan_bwd(g, s);
+}
+}  // namespace
+
+extern "C" {
+
 size_t mamba3_scan_bwd_workspace_bytes(const mamba3_dims* d) {
   if (check_dims(d, true) != MAMBA3_OK) return 0;
   const m3::ScanArgs a = scan_args(d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
@@ -239,32 +285,19 @@ int mamba3_scan_bwd(const mamba3_dims* d, const void* x, const void* B, const vo
                     const void* dy, const mamba3_state* d_final, void* dx, void* dB, void* dC, void* dtheta,
                     void* ddt, void* dlam, float* dA, float* dD, const mamba3_state* d_init, void* workspace,
                     size_t workspace_bytes, void* stream) {
-  int rc = check_dims(d, true);
-  if (rc) return rc;
-  if (!A || !dA || !aligned4(dA) || (dD && !aligned4(dD))) return MAMBA3_ERR_INVALID;
-  if (d->seqlen > 0) {
-    if ((rc = check_inputs(x, B, C, theta, dt, lam, A, D, dy))) return rc;
-    if ((rc = check_inputs(dx, dB, dC, dtheta, ddt, dlam, A, D, dy))) return rc;  // the gradients' layouts
-  }
-  if ((rc = check_state(init)) || (rc = check_state(d_final)) || (rc = check_state(d_init))) return rc;
-  if (!workspace || !aligned16(workspace)) return MAMBA3_ERR_WORKSPACE;
-  if (workspace_bytes < mamba3_scan_bwd_workspace_bytes(d)) return MAMBA3_ERR_WORKSPACE;
-  m3::BwdArgs g;
-  memset(&g, 0, sizeof(g));
-  g.f = scan_args(d, x, B, C, theta, dt, lam, A, D, init);
-  g.f.workspace = workspace;
-  g.f.workspace_bytes = workspace_bytes;
-  if ((rc = m3::bwd_supported(g.f))) return rc;
-  g.dy = dy;
-  if (d_final) {
-    g.dh_out = d_final->h; g.dbprev_out = d_final->b_prev; g.dxprev_out = d_final->x_prev; g.dangle_out = d_final->angle;
-  }
-  g.dx = dx; g.dB = dB; g.dC = dC; g.dtheta = dtheta; g.ddt = ddt; g.dlam = dlam; g.dA = dA; g.dD = dD;
-  if (d_init) { g.dh0 = d_init->h; g.dbprev0 = d_init->b_prev; g.dxprev0 = d_init->x_prev; g.dangle0 = d_init->angle; }
-  g.ckpt = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
-  return m3::launch_scan_bwd(g, s);
+  if (!A || !dA || !aligned4(dA)) return MAMBA3_ERR_INVALID;
+  return scan_bwd_impl(d, x, B, C, theta, dt, lam, A, nullptr, D, init, dy, d_final, dx, dB, dC, dtheta, ddt, dlam,
+                       dA, nullptr, dD, d_init, workspace, workspace_bytes, stream);
+}
+
+int mamba3_scan_bwd_at(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                       const void* dt, const void* lam, const void* A_t, const float* D, const mamba3_state* init,
+                       const void* dy, const mamba3_state* d_final, void* dx, void* dB, void* dC, void* dtheta,
+                       void* ddt, void* dlam, void* dA_t, float* dD, const mamba3_state* d_init, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (!A_t || !dA_t || !aligned4(A_t) || !aligned4(dA_t)) return MAMBA3_ERR_INVALID;
+  return scan_bwd_impl(d, x, B, C, theta, dt, lam, nullptr, A_t, D, init, dy, d_final, dx, dB, dC, dtheta, ddt, dlam,
+                       nullptr, dA_t, dD, d_init, workspace, workspace_bytes, stream);
 }
 
 int mamba3_gated_norm(const mamba3_dims* d, int groups, const void* y, const void* z, const float* w, float eps,

@@ -37,7 +37,7 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kRows = 32;  // M = Q * R rows per chunk
-constexpr int kNScal = 14;  // per-token scalar arrays of the backward chunk
+constexpr int kNScal = 15;  // per-token scalar arrays of the backward chunk
 
 struct BwdLayout {
   int M, Q;
@@ -126,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
   float *s_zin = sc + 5 * QS, *s_zue = sc + 6 * QS, *s_dg = sc + 7 * QS, *s_cZu = sc + 8 * QS;
   float *s_cT = sc + 9 * QS, *s_rT = sc + 10 * QS, *s_dth = sc + 11 * QS, *s_ecum = sc + 12 * QS;
   float* s_eend = sc + 13 * QS;
+  float* s_at = sc + 14 * QS;  // decay rate of each token (A_t, or A of the head)
   float* phi = sm + lay.off_ang;  // [K] running angle (pass 1) or angle at the chunk start (pass 2)
   float* Sang = phi + K;          // [K] dL/dPhi summed from the end
   float* misc = sm + lay.off_misc;  // [0] <hbar_in, G>, [1] dD, [2] initial lagged share, [3..4] pending ddt, dlam
@@ -143,7 +144,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
   T* dTHg = static_cast<T*>(g.dtheta);
   T* dDTg = static_cast<T*>(g.ddt);
   T* dLMg = static_cast<T*>(g.dlam);
-  const float Ah = a.A[hh];
+  const T* AT = static_cast<const T*>(a.A_t);  // time-varying decay [b, L, H], or null
+  T* dATg = static_cast<T*>(g.dA_t);
+  const float Ah = AT ? 0.f : a.A[hh];
   const float Dh = a.D ? a.D[hh] : 0.f;
   const size_t us = (size_t)unit;
   auto tok = [&](int t) { return ((size_t)b * L + t) * a.nheads + hh; };
@@ -188,13 +191,14 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
       if (backward) sdY[m * PS + p] = ld1(DY + gi);
     }
     for (int i = tid; i < q * K; i += kThreads) sth[i] = ld1(TH + tok(t0 + i / K) * K + i % K);
+    for (int i = tid; i < q; i += kThreads) s_at[i] = AT ? ld1(AT + tok(t0 + i)) : Ah;
   };
   // decay scan of the chunk (warp 0, one lane per token, q <= 32): cum, gamma, w,
   // e^{cum}, e^{cum_end - cum}
   auto decay_scalars = [&](int q) {
     if (tid < 32) {
       const int i = tid;
-      float c = i < q ? s_dt[i] * Ah : 0.f;
+      float c = i < q ? s_dt[i] * s_at[i] : 0.f;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float v = __shfl_up_sync(0xffffffffu, c, o);
@@ -571,9 +575,12 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
         const float da = c0 + suf_zin + pre + F;
         const float dw = s_zue[i] + s_cZu[i];
         const float dgt = s_dg[i] + dw;  // gamma_i enters K(i, i) and w_i
-        float ddt = da * Ah + dgt * s_lam[i] + s_dth[i];
+        float ddt = da * s_at[i] + dgt * s_lam[i] + s_dth[i];
         float dlm = dgt * s_dt[i];
-        dA_acc += da * s_dt[i];
+        if (AT)
+          st1(dATg + tok(t0 + i), da * s_dt[i]);
+        else
+          dA_acc += da * s_dt[i];
         if (i > 0) {  // token i's lagged weight (1 - lam_i) dt_i sits in w_{i-1}
           ddt += dw_prev * (1.f - s_lam[i]);
           dlm -= dw_prev * s_dt[i];
@@ -620,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     const float dmu = misc[2];
     st1(dDTg + tok(0), misc[3] + dmu * (1.f - s_lam[0]));
     st1(dLMg + tok(0), misc[4] - dmu * s_dt[0]);
-    atomicAdd(g.dA + hh, dA_acc);
+    if (!AT) atomicAdd(g.dA + hh, dA_acc);
     if (g.dD) atomicAdd(g.dD + hh, misc[1]);
   }
   if (g.dh0) {
@@ -653,8 +660,8 @@ size_t bwd_checkpoint_bytes(const ScanArgs& a) {
 
 int bwd_supported(const ScanArgs& a) {
   if (a.ngroups < 1 || a.nheads % a.ngroups != 0) return MAMBA3_ERR_INVALID;
-  // this pass covers one B, C row per head and A per head
-  if (a.ngroups != a.nheads || a.A_t || a.bcnorm || !a.A) return MAMBA3_ERR_UNSUPPORTED;
+  // this pass covers one B, C row per head, and A per head or A_t per token
+  if (a.ngroups != a.nheads || a.bcnorm || (!a.A && !a.A_t)) return MAMBA3_ERR_UNSUPPORTED;
   if (a.R > kRows) return MAMBA3_ERR_UNSUPPORTED;
   if (bwd_layout(a.P, a.N, a.R).total > 220 * 1024) return MAMBA3_ERR_UNSUPPORTED;
   return MAMBA3_OK;
@@ -662,7 +669,7 @@ int bwd_supported(const ScanArgs& a) {
 
 int launch_scan_bwd(const BwdArgs& g, cudaStream_t s) {
   const ScanArgs& a = g.f;
-  if (cudaMemsetAsync(g.dA, 0, sizeof(float) * a.nheads, s) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  if (g.dA && cudaMemsetAsync(g.dA, 0, sizeof(float) * a.nheads, s) != cudaSuccess) return MAMBA3_ERR_CUDA;
   if (g.dD && cudaMemsetAsync(g.dD, 0, sizeof(float) * a.nheads, s) != cudaSuccess) return MAMBA3_ERR_CUDA;
   const int units = a.batch * a.nheads;
   if (units == 0) return MAMBA3_OK;

@@ -285,3 +285,22 @@ def test_gated_norm_host_validation(lib):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_gated_norm_valid_call_without_device_is_a_cuda_error(lib):
     assert gnorm(lib, dims(nheads=4), 2) == m3.MAMBA3_ERR_CUDA
+
+
+def bwd_at(lib, d, ptrs=None):
+    p = dict(A_t=FAKE, dA_t=FAKE)
+    p.update(ptrs or {})
+    return lib.mamba3_scan_bwd_at(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, p["A_t"], None, None, FAKE,
+                                  None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, p["dA_t"], None, None, FAKE, 1 << 40, None)
+
+
+def test_backward_time_varying_decay_host_validation(lib):
+    assert bwd_at(lib, dims(), {"A_t": None}) == m3.MAMBA3_ERR_INVALID
+    assert bwd_at(lib, dims(), {"dA_t": None}) == m3.MAMBA3_ERR_INVALID
+    assert bwd_at(lib, dims(), {"A_t": FAKE + 2}) == m3.MAMBA3_ERR_INVALID
+    assert bwd_at(lib, dims(ngroups=1)) == m3.MAMBA3_ERR_UNSUPPORTED
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_backward_time_varying_decay_valid_call_without_device(lib):
+    assert bwd_at(lib, dims()) == m3.MAMBA3_ERR_CUDA

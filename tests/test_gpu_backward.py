@@ -147,3 +147,26 @@ def test_backward_full_size_sampled_units():
         for n in ("dx", "dB", "dC", "dtheta", "ddt", "dlam"):
             e = rel_err(np64(gr[n][bb:bb + 1, :, hh:hh + 1]), ref[n])
             assert e < TOL[torch.bfloat16], (n, bb, hh, e)
+
+
+@pytest.mark.parametrize("shape,dtype", [
+    ((2, 100, 3, 16, 16, 1), torch.float32),
+    ((2, 45, 2, 16, 32, 4), torch.float32),
+    ((1, 130, 4, 64, 128, 1), torch.bfloat16),
+    ((1, 70, 4, 64, 128, 4), torch.bfloat16),
+])
+def test_backward_time_varying_decay_matches_oracle(shape, dtype):
+    """mamba3_scan_bwd_at: a decay rate per token; its gradient dA_t is per token."""
+    b, L, H, P, N, R = shape
+    inp = small_inputs(b, L, H, P, N, R, dtype, seed=3300 + L + R)
+    A_t = wl.decay_rates(inp["dt"], seed=3400 + L)
+    dy = dy_like(inp["x"], 3500 + L)
+    init, d_final = rand_state(b, H, P, N, R, 3600 + L), rand_state(b, H, P, N, R, 3700 + L)
+    gr = m3.mamba3_scan_bwd_at(*(inp[n] for n in NAMES), A_t, inp["D"], dy, init=init, d_final=d_final)
+    torch.cuda.synchronize()
+    f = wl.to_f64({k: inp[k] for k in (*NAMES, "D")})
+    f["A"] = np64(A_t)
+    st = lambda s: oracle.State(*(np64(getattr(s, n)) for n, _ in STATE))
+    ref = oracle.scan_bwd(**f, dy=np64(dy), init=st(init), d_final=st(d_final))
+    gr["dA"] = gr["dA_t"]
+    check(gr, ref, TOL[dtype])
