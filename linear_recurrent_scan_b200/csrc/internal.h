@@ -51,6 +51,8 @@ struct BwdArgs {
   void* dA_t;  // with f.A_t: the decay-rate gradient per token (layout of dt, dtype of x); dA null
   float *dh0, *dbprev0, *dxprev0, *dangle0;                      // all null = not wanted
   float* ckpt;  // [units][chunks][N*P + N/2]: hbar and Phi at every chunk start
+  float *dBh, *dCh;  // grouped B, C: per-head fp32 gradients [b, L, H, R, N], summed into dB, dC
+                     // over each group's heads afterwards; null with one row per head
 };
 
 // Pre-gate grouped RMS norm and gate of the layer output: rows = tokens x groups
@@ -67,6 +69,7 @@ struct GatedNormArgs {
 int launch_gated_norm(const GatedNormArgs& a, cudaStream_t s);
 
 size_t bwd_checkpoint_bytes(const ScanArgs& a);
+size_t bwd_group_bytes(const ScanArgs& a);  // per-head B, C gradients when B, C are grouped
 int bwd_supported(const ScanArgs& a);
 int launch_scan_bwd(const BwdArgs& g, cudaStream_t s);
 

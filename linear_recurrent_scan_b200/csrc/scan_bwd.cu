@@ -150,6 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
   const float Dh = a.D ? a.D[hh] : 0.f;
   const size_t us = (size_t)unit;
   auto tok = [&](int t) { return ((size_t)b * L + t) * a.nheads + hh; };
+  const int gh = hh / (a.nheads / a.ngroups);  // B, C row of this head
+  auto tok_bc = [&](int t) { return ((size_t)b * L + t) * a.ngroups + gh; };
   const bool has_init = a.h0 != nullptr;
 
   if (L == 0) {  // the exported state is the initial state: its gradients pass through
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
     const int M = q * R;
     for (int i = tid; i < M * N; i += kThreads) {
       const int m = i / N, n = i % N;
-      const size_t gi = tok(t0 + m / R) * R * N + (size_t)(m % R) * N + n;
+      const size_t gi = tok_bc(t0 + m / R) * R * N + (size_t)(m % R) * N + n;
       sB[m * NS + n] = ld1(Bg + gi);
       if (backward) sC[m * NS + n] = ld1(Cg + gi);
     }
@@ -537,10 +539,17 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
           dphi += db0 * sB[m * NS + 2 * k + 1] - db1 * sB[m * NS + 2 * k] + dc0 * sC[m * NS + 2 * k + 1] -
                   dc1 * sC[m * NS + 2 * k];
           const size_t gi = tok(t0 + i) * R * N + (size_t)r * N + 2 * k;
-          st1(dBg + gi, cs * db0 - sn * db1);
-          st1(dBg + gi + 1, sn * db0 + cs * db1);
-          st1(dCg + gi, cs * dc0 - sn * dc1);
-          st1(dCg + gi + 1, sn * dc0 + cs * dc1);
+          if (g.dBh) {  // grouped: this head's share, summed over the group afterwards
+            g.dBh[gi] = cs * db0 - sn * db1;
+            g.dBh[gi + 1] = sn * db0 + cs * db1;
+            g.dCh[gi] = cs * dc0 - sn * dc1;
+            g.dCh[gi + 1] = sn * dc0 + cs * dc1;
+          } else {
+            st1(dBg + gi, cs * db0 - sn * db1);
+            st1(dBg + gi + 1, sn * db0 + cs * db1);
+            st1(dCg + gi, cs * dc0 - sn * dc1);
+            st1(dCg + gi + 1, sn * dc0 + cs * dc1);
+          }
         }
         Sk += dphi;
         const size_t ti = tok(t0 + i) * K + k;
@@ -650,7 +659,32 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
   }
 }
 
+// dB[b, t, g] = sum of dBh[b, t, h] over the heads h of group g (and dC likewise)
+template <typename T>
+__global__ void __launch_bounds__(256) bc_group_sum_kernel(const float* dBh, const float* dCh, T* dB, T* dC,
+                                                           long long total, int groups, int hpg, int rn) {
+  for (long long e = (long long)blockIdx.x * 256 + threadIdx.x; e < total; e += (long long)gridDim.x * 256) {
+    const long long row = e / rn;  // (b, t, g)
+    const int c = (int)(e % rn);
+    const long long bt = row / groups;
+    const int grp = (int)(row % groups);
+    const size_t base = ((size_t)bt * groups * hpg + (size_t)grp * hpg) * rn + c;
+    float sb = 0.f, sc = 0.f;
+    for (int j = 0; j < hpg; ++j) {
+      sb += dBh[base + (size_t)j * rn];
+      sc += dCh[base + (size_t)j * rn];
+    }
+    st1(dB + e, sb);
+    st1(dC + e, sc);
+  }
+}
+
 }  // namespace
+
+size_t bwd_group_bytes(const ScanArgs& a) {
+  if (a.ngroups >= a.nheads) return 0;
+  return 2 * (size_t)a.batch * a.seqlen * a.nheads * a.R * a.N * sizeof(float);
+}
 
 size_t bwd_checkpoint_bytes(const ScanArgs& a) {
   const BwdLayout l = bwd_layout(a.P, a.N, a.R);
@@ -660,8 +694,8 @@ size_t bwd_checkpoint_bytes(const ScanArgs& a) {
 
 int bwd_supported(const ScanArgs& a) {
   if (a.ngroups < 1 || a.nheads % a.ngroups != 0) return MAMBA3_ERR_INVALID;
-  // this pass covers one B, C row per head, and A per head or A_t per token
-  if (a.ngroups != a.nheads || a.bcnorm || (!a.A && !a.A_t)) return MAMBA3_ERR_UNSUPPORTED;
+  // A per head or A_t per token; B, C per head or grouped; no fused norm
+  if (a.bcnorm || (!a.A && !a.A_t)) return MAMBA3_ERR_UNSUPPORTED;
   if (a.R > kRows) return MAMBA3_ERR_UNSUPPORTED;
   if (bwd_layout(a.P, a.N, a.R).total > 220 * 1024) return MAMBA3_ERR_UNSUPPORTED;
   return MAMBA3_OK;
@@ -690,6 +724,22 @@ int launch_scan_bwd(const BwdArgs& g, cudaStream_t s) {
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
   k<<<units, kThreads, lay.total, s>>>(g, lay);
+  if (cudaGetLastError() != cudaSuccess) return MAMBA3_ERR_CUDA;
+  if (g.dBh) {
+    const long long total = (long long)a.batch * a.seqlen * a.ngroups * a.R * a.N;
+    if (total > 0) {
+      long long blocks = (total + 255) / 256;
+      if (blocks > 148 * 16) blocks = 148 * 16;
+      const int hpg = a.nheads / a.ngroups, rn = a.R * a.N;
+      if (a.dtype == MAMBA3_F32)
+        bc_group_sum_kernel<float><<<(int)blocks, 256, 0, s>>>(g.dBh, g.dCh, static_cast<float*>(g.dB),
+                                                               static_cast<float*>(g.dC), total, a.ngroups, hpg, rn);
+      else
+        bc_group_sum_kernel<__nv_bfloat16><<<(int)blocks, 256, 0, s>>>(
+            g.dBh, g.dCh, static_cast<__nv_bfloat16*>(g.dB), static_cast<__nv_bfloat16*>(g.dC), total, a.ngroups,
+            hpg, rn);
+    }
+  }
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 

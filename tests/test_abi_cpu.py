@@ -257,7 +257,10 @@ def test_backward_host_validation(lib):
     assert bwd(lib, d, ws_bytes=need - 1) == m3.MAMBA3_ERR_WORKSPACE
     assert bwd(lib, d, ws=FAKE + 8) == m3.MAMBA3_ERR_WORKSPACE
     assert bwd(lib, d, {"dB": FAKE + 4}) == m3.MAMBA3_ERR_INVALID
-    assert bwd(lib, dims(ngroups=1)) == m3.MAMBA3_ERR_UNSUPPORTED  # grouped B/C: not in this pass
+    # grouped B/C: the per-head B, C gradients (2 x b L H R N fp32) come on top of the checkpoints
+    dg = dims(ngroups=1)
+    assert lib.mamba3_scan_bwd_workspace_bytes(ctypes.byref(dg)) == need + 2 * 2 * 64 * 3 * 1 * 16 * 4
+    assert bwd(lib, dg, ws_bytes=need) == m3.MAMBA3_ERR_WORKSPACE
     assert bwd(lib, dims(dstate=256, headdim=128)) == m3.MAMBA3_ERR_UNSUPPORTED  # tiles beyond shared memory
     assert lib.mamba3_scan_bwd_workspace_bytes(ctypes.byref(dims(rank=3))) == 0
 
@@ -265,6 +268,7 @@ def test_backward_host_validation(lib):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_backward_valid_call_without_device_is_a_cuda_error(lib):
     assert bwd(lib, dims()) == m3.MAMBA3_ERR_CUDA
+    assert bwd(lib, dims(ngroups=1)) == m3.MAMBA3_ERR_CUDA  # grouped B/C
 
 
 def gnorm(lib, d, groups, y=FAKE, z=FAKE, w=None, eps=1e-6, out=FAKE):
@@ -298,7 +302,6 @@ def test_backward_time_varying_decay_host_validation(lib):
     assert bwd_at(lib, dims(), {"A_t": None}) == m3.MAMBA3_ERR_INVALID
     assert bwd_at(lib, dims(), {"dA_t": None}) == m3.MAMBA3_ERR_INVALID
     assert bwd_at(lib, dims(), {"A_t": FAKE + 2}) == m3.MAMBA3_ERR_INVALID
-    assert bwd_at(lib, dims(ngroups=1)) == m3.MAMBA3_ERR_UNSUPPORTED
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")

@@ -170,3 +170,22 @@ def test_backward_time_varying_decay_matches_oracle(shape, dtype):
     ref = oracle.scan_bwd(**f, dy=np64(dy), init=st(init), d_final=st(d_final))
     gr["dA"] = gr["dA_t"]
     check(gr, ref, TOL[dtype])
+
+
+@pytest.mark.parametrize("shape,G,dtype", [
+    ((2, 100, 6, 16, 16, 1), 2, torch.float32),
+    ((2, 45, 4, 16, 32, 4), 1, torch.float32),
+    ((1, 130, 8, 64, 128, 1), 2, torch.bfloat16),
+    ((1, 70, 8, 64, 128, 4), 4, torch.bfloat16),
+])
+def test_backward_grouped_bc_matches_oracle(shape, G, dtype):
+    """B, C shared by groups of H / G heads: dB, dC are the sums of the group's
+    heads' gradients (the oracle sums its per-head ones the same way)."""
+    b, L, H, P, N, R = shape
+    inp = small_inputs(b, L, H, P, N, R, dtype, seed=3800 + L + G)
+    inp.update(wl.grouped_bc(inp, G, seed=3900 + L))
+    dy = dy_like(inp["x"], 4000 + L)
+    init, d_final = rand_state(b, H, P, N, R, 4100 + L), rand_state(b, H, P, N, R, 4200 + L)
+    gr, ref = run_both(inp, dy, init, d_final)
+    assert gr["dB"].shape == inp["B"].shape
+    check(gr, ref, TOL[dtype])
