@@ -194,8 +194,9 @@ MAMBA3_API int mamba3_decode_step_at(const mamba3_dims* dims, const mamba3_state
  * are the chain rule applied to the recurrence above (section 1.1), its
  * rotation (section 1.2) and the rank-R products (section 1.3), in reverse
  * order over the sequence.
- *   x .. D, init  as for mamba3_scan_fwd (A per head; B, C one row per head:
- *                 dims->ngroups 0 or nheads; dims->chunk is ignored).
+ *   x .. D, init  as for mamba3_scan_fwd (A per head; B, C per head or grouped
+ *                 by dims->ngroups, dB, dC then summed over each group's heads;
+ *                 dims->chunk is ignored).
  *   dy            layout and dtype of y.
  *   d_final       nullable: float32 gradients of the four exported state fields
  *                 (all non-null when given).
@@ -208,9 +209,10 @@ MAMBA3_API int mamba3_decode_step_at(const mamba3_dims* dims, const mamba3_state
  *   workspace     at least mamba3_scan_bwd_workspace_bytes(dims): the state at
  *                 every chunk start, kept between the forward and the reverse
  *                 sweep (batch * nheads * ceil(seqlen / Q) * (N P + N/2) floats,
- *                 Q = 32 / rank), after the 256-byte status word.
+ *                 Q = 32 / rank), after the 256-byte status word; with grouped
+ *                 B/C also 2 * batch * seqlen * nheads * rank * dstate floats.
  * Computed in float32 whatever in_dtype is.  Returns MAMBA3_ERR_UNSUPPORTED for
- * grouped B/C, and for N, P whose per-chunk tiles exceed shared memory.
+ * N, P whose per-chunk tiles exceed shared memory.
  * mamba3_scan_bwd_at is the same for mamba3_scan_fwd_at: A_t [b, L, H] (dtype of x)
  * in place of A, and dA_t (layout and dtype of A_t, not nullable) in place of dA.
  */
