@@ -35,7 +35,8 @@
  * pinned against finite differences of m3o_scan_complex); and m3o_bc_norm, the RMS normalisation of raw B or C
  * projections over the state dimension with a per-(head, rank) weight and bias
  * (same page, section 2: "BC norm" and head-specific B/C bias), which the
- * recurrence then consumes.
+ * recurrence then consumes; and m3o_gated_norm, the output side (grouped RMS
+ * norm ahead of the silu gate, same page, section 2).
  *
  * Layouts (row-major, contiguous; b = batch, L = seqlen, H = heads):
  *   x      [b, L, H, R, P]     B, C  [b, L, H, R, N]     theta [b, L, H, N/2]
