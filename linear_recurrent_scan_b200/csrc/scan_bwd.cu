@@ -504,22 +504,23 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
             dCt[m * N + n] = dc[a2][c];
           }
       }
-    } else
-    for (int i = tid; i < M * N; i += kThreads) {
-      const int m = i / N, n = i % N, t = m / R, r = m % R;
-      float dc = 0.f, db = 0.f;
+    } else {
+      for (int i = tid; i < M * N; i += kThreads) {
+        const int m = i / N, n = i % N, t = m / R, r = m % R;
+        float dc = 0.f, db = 0.f;
 #pragma unroll 8
-      for (int p = 0; p < P; ++p) {
-        dc += sdY[m * PS + p] * hb[n * PS + p];
-        db += sX[m * PS + p] * G[n * PS + p];
+        for (int p = 0; p < P; ++p) {
+          dc += sdY[m * PS + p] * hb[n * PS + p];
+          db += sX[m * PS + p] * G[n * PS + p];
+        }
+        dc *= s_ecum[t];
+        db *= s_w[t] * s_eend[t];
+        for (int j = 0; j < (t + 1) * R; ++j) dc += sW[m * M + j] * sB[j * NS + n];
+        for (int j = t * R; j < M; ++j) db += sW[j * M + m] * sC[j * NS + n];
+        if (t0 + t == L - 1 && g.dbprev_out) db += g.dbprev_out[(us * R + r) * N + n];
+        dBt[i] = db;
+        dCt[i] = dc;
       }
-      dc *= s_ecum[t];
-      db *= s_w[t] * s_eend[t];
-      for (int j = 0; j < (t + 1) * R; ++j) dc += sW[m * M + j] * sB[j * NS + n];
-      for (int j = t * R; j < M; ++j) db += sW[j * M + m] * sC[j * NS + n];
-      if (t0 + t == L - 1 && g.dbprev_out) db += g.dbprev_out[(us * R + r) * N + n];
-      dBt[i] = db;
-      dCt[i] = dc;
     }
     __syncthreads();
 
