@@ -37,3 +37,15 @@ def sum_over_ranks(value: float, device=None) -> float:
     t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def all_reduce_sum_(tensors) -> None:
+    """In-place sum over ranks of parameter gradients (the backward pass's dA and
+    dD, which sum over the batch): the one exchange that data-parallel training adds.
+    A no-op on a single rank.  Every rank must pass the same tensors in the same order."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return
+    for t in tensors:
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
