@@ -36,6 +36,7 @@ PREFILL_MORE = [wl.CONFIGS["mimo4_prefill_b4_l8192"], wl.CONFIGS["mimo4_long_b1_
 # batch-1 decode after the 65536-token MIMO prefill: latency-bound (2.5 MB per step)
 DECODE_LONG = wl.CONFIGS["mimo4_long_b1_l65536"].with_(prefill_tokens=65536)
 FALLBACK_HBM_GBS = 6650.0
+BACKWARD_KERNEL = "scan_bwd_kernel (SIMT, fp32)"
 
 # DRAM bytes (read + write) per launch from ncu captures of the kernels as they
 # stand: (kernel source files, sha256 of their concatenation, bytes per launch,
@@ -188,6 +189,35 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["unsampled"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def rl(nbytes: int, ms: float, peak: float, traffic_bytes=None) -> dict:
+    """Compact roofline of one side measurement: GB/s achieved on the algorithmic
+    bytes and its fraction of the HBM peak of the headline line."""
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    d = {"bytes": nbytes, "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+    if traffic_bytes is not None:
+        d["traffic"] = traffic_bytes
+    return d
+
+
+def bench_config(world: int) -> dict:
+    """The workload of the headline line (the same dict in both arms)."""
+    w = PREFILL
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads, "headdim": w.headdim,
+            "dstate": w.dstate, "rank": w.rank, "state_dtype": "fp32", "parallelism": f"batch-sharded x{world} (weak)",
+            "l2": "inputs (%.0f MB) larger than L2 (126 MB); no flush" % (prefill_bytes(w) / 1e6)}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 # --------------------------------------------------------------------------- ranks
@@ -474,88 +504,52 @@ def ours(args):
     dec = {}
     for w in DECODE:
         us = run_decode(m3, w, world, rank, w.decode_steps)
-        gbs = decode_bytes(w) / (us * 1e-6) / 1e9
         dec[w.name] = {"us_per_step": round(us, 2), "steps": w.decode_steps, "batch": w.batch, "rank": w.rank,
-                       "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                                    "frac": round(gbs / peak, 4), "traffic": traffic(w.name),
-                                    "bytes_per_step": decode_bytes(w)}}
+                       **rl(decode_bytes(w), us * 1e-3, peak, traffic(w.name))}
     us = run_decode(m3, DECODE_LONG, world, rank, DECODE_LONG.decode_steps)
     dec["mimo4_long_decode_b1"] = {"us_per_step": round(us, 2), "steps": DECODE_LONG.decode_steps, "batch": 1,
                                    "rank": DECODE_LONG.rank, "dstate": DECODE_LONG.dstate,
-                                   "state_from_prefill_tokens": DECODE_LONG.prefill_tokens,
-                                   "roofline": None, "note": "latency-bound: %d bytes per step" % decode_bytes(DECODE_LONG)}
+                                   "note": "after a %d-token prefill; latency-bound: %d bytes per step" % (
+                                       DECODE_LONG.prefill_tokens, decode_bytes(DECODE_LONG))}
+    side_steps = max(5, min(args.steps, 20))
     # the fused B/C norm variant of the headline prefill and of the SISO decode step
-    ms = max_over_ranks(run_prefill_plain(m3, PREFILL, rank, steps=max(5, min(args.steps, 20)), warmup=3,
-                                          fused_norm=True), world)
-    gbs = prefill_bytes(PREFILL) / (ms * 1e-3) / 1e9
-    fused = {"prefill_" + PREFILL.name: {"ms_per_launch": round(ms, 4), "roofline": {
-        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
-        "bytes_per_launch": prefill_bytes(PREFILL)}}}
+    ms = max_over_ranks(run_prefill_plain(m3, PREFILL, rank, steps=side_steps, warmup=3, fused_norm=True), world)
+    fused = {"prefill": {"ms": round(ms, 4), **rl(prefill_bytes(PREFILL), ms, peak)}}
     us = run_decode(m3, DECODE[0], world, rank, DECODE[0].decode_steps, fused_norm=True)
-    gbs = decode_bytes(DECODE[0]) / (us * 1e-6) / 1e9
-    fused["decode_" + DECODE[0].name] = {"us_per_step": round(us, 2), "roofline": {
-        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
-        "bytes_per_step": decode_bytes(DECODE[0])}}
+    fused["decode_siso_b128"] = {"us": round(us, 2), **rl(decode_bytes(DECODE[0]), us * 1e-3, peak)}
     # the time-varying decay variant (A_t per token: 2 more bytes per token-head)
-    ms = max_over_ranks(run_prefill_plain(m3, PREFILL, rank, steps=max(5, min(args.steps, 20)), warmup=3,
-                                          time_varying_a=True), world)
-    by = prefill_bytes(PREFILL) + 2 * PREFILL.token_heads
-    gbs = by / (ms * 1e-3) / 1e9
-    tva = {"prefill_" + PREFILL.name: {"ms_per_launch": round(ms, 4), "roofline": {
-        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
-        "bytes_per_launch": by}}}
+    ms = max_over_ranks(run_prefill_plain(m3, PREFILL, rank, steps=side_steps, warmup=3, time_varying_a=True), world)
+    tva = {"prefill": {"ms": round(ms, 4), **rl(prefill_bytes(PREFILL) + 2 * PREFILL.token_heads, ms, peak)}}
     us = run_decode(m3, DECODE[0], world, rank, DECODE[0].decode_steps, time_varying_a=True)
-    by = decode_bytes(DECODE[0]) + 2 * DECODE[0].batch * DECODE[0].nheads
-    gbs = by / (us * 1e-6) / 1e9
-    tva["decode_" + DECODE[0].name] = {"us_per_step": round(us, 2), "roofline": {
-        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
-        "bytes_per_step": by}}
+    tva["decode_siso_b128"] = {"us": round(us, 2), **rl(decode_bytes(DECODE[0]) + 2 * DECODE[0].batch *
+                                                        DECODE[0].nheads, us * 1e-3, peak)}
     # grouped B/C: one B and C row per token shared by all heads (ngroups 1)
-    ms = max_over_ranks(run_prefill_plain(m3, PREFILL, rank, steps=max(5, min(args.steps, 20)), warmup=3,
-                                          groups=1), world)
-    by = prefill_bytes(PREFILL, groups=1)
-    gbs = by / (ms * 1e-3) / 1e9
-    grp = {"prefill_" + PREFILL.name: {"ngroups": 1, "ms_per_launch": round(ms, 4), "roofline": {
-        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
-        "traffic": traffic("grouped_prefill"), "bytes_per_launch": by}}}
+    ms = max_over_ranks(run_prefill_plain(m3, PREFILL, rank, steps=side_steps, warmup=3, groups=1), world)
+    grp = {"prefill": {"ngroups": 1, "ms": round(ms, 4),
+                       **rl(prefill_bytes(PREFILL, groups=1), ms, peak, traffic("grouped_prefill"))}}
     us = run_decode(m3, DECODE[0], world, rank, DECODE[0].decode_steps, groups=1)
-    by = decode_bytes(DECODE[0], groups=1)
-    gbs = by / (us * 1e-6) / 1e9
-    grp["decode_" + DECODE[0].name] = {"ngroups": 1, "us_per_step": round(us, 2), "roofline": {
-        "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
-        "traffic": traffic("grouped_decode"), "bytes_per_step": by}}
+    grp["decode_siso_b128"] = {"ngroups": 1, "us": round(us, 2),
+                               **rl(decode_bytes(DECODE[0], groups=1), us * 1e-3, peak, traffic("grouped_decode"))}
     # the backward pass of the headline prefill (dy given; zero initial state)
     ms = max_over_ranks(run_backward(m3, PREFILL, rank, steps=3, warmup=1), world)
-    by = backward_bytes(PREFILL)
-    gbs = by / (ms * 1e-3) / 1e9
-    bwd = {"prefill_" + PREFILL.name: {"ms_per_launch": round(ms, 3), "kernel": "scan_bwd_kernel (SIMT, fp32)",
-                                       "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
-                                                    "unit": "GB/s", "frac": round(gbs / peak, 5),
-                                                    "traffic": traffic("backward"), "bytes_per_launch": by}}}
+    bwd = {"prefill_" + PREFILL.name: {"ms": round(ms, 3), "kernel": BACKWARD_KERNEL,
+                                       **rl(backward_bytes(PREFILL), ms, peak, traffic("backward"))}}
     # the output side on the headline prefill's y: grouped RMS norm + gate
     gated = {}
     for ng in (PREFILL.nheads, 8):
-        ms = max_over_ranks(run_gated_norm(m3, PREFILL, rank, ng, steps=max(5, min(args.steps, 20)), warmup=3), world)
+        ms = max_over_ranks(run_gated_norm(m3, PREFILL, rank, ng, steps=side_steps, warmup=3), world)
         by = 3 * esize(PREFILL.dtype) * PREFILL.token_heads * PREFILL.rank * PREFILL.headdim + 4 * PREFILL.nheads * \
             PREFILL.rank * PREFILL.headdim
-        gbs = by / (ms * 1e-3) / 1e9
-        gated["prefill_%s_groups%d" % (PREFILL.name, ng)] = {
-            "ms_per_launch": round(ms, 4), "norm_groups": ng,
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(gbs / peak, 4), "bytes_per_launch": by,
-                         "traffic": traffic("gated_norm_per_head") if ng == PREFILL.nheads else None}}
+        gated["groups%d" % ng] = {"ms": round(ms, 4), **rl(by, ms, peak, traffic("gated_norm_per_head")
+                                                         if ng == PREFILL.nheads else None)}
     more = {}
     for w in PREFILL_MORE:
-        ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=max(5, min(args.steps, 20)), warmup=3), world)
-        by = prefill_bytes(w)
-        gbs = by / (ms * 1e-3) / 1e9
-        more[w.name] = {"ms_per_launch": round(ms, 4), "mtokens_s": round(w.batch * w.seqlen / (ms * 1e-3) / 1e6, 3),
-                        "batch": w.batch, "seqlen": w.seqlen, "rank": w.rank, "dstate": w.dstate,
-                        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                                     "frac": round(gbs / peak, 4), "bytes_per_launch": by}}
+        ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=side_steps, warmup=3), world)
+        more[w.name] = {"ms": round(ms, 4), "mtokens_s": round(w.batch * w.seqlen / (ms * 1e-3) / 1e6, 3),
+                        **rl(prefill_bytes(w), ms, peak)}
     clk.stop()
     clocks = clk.summary()
-    clocks["window"] = "headline prefill timed steps through the decode replays and the further prefill shapes"
+    clocks["window"] = "headline prefill timed steps through the last side measurement"
     e2e_value = tokens_all / (r["e2e_ms"] * 1e-3) / 1e6
     out = {
         "metric": "prefill Mtokens/s (SISO, batch 8, seqlen 2048) and decode step us at batch 128",
@@ -570,24 +564,23 @@ def ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; distributions of the layer inputs, no dataset or weights)",
-        "config": {"workload": PREFILL.name, "batch": PREFILL.batch, "seqlen": PREFILL.seqlen,
-                   "nheads": PREFILL.nheads, "headdim": PREFILL.headdim, "dstate": PREFILL.dstate,
-                   "rank": PREFILL.rank, "state_dtype": "fp32", "parallelism": f"batch-sharded x{world} (weak)",
-                   "l2": "inputs (%.0f MB) larger than L2 (126 MB); no flush" % (r["bytes"] / 1e6)},
+        "config": bench_config(world),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic("prefill"), "peak_kind": peak_kind,
                      "bytes_per_launch": r["bytes"], "launch_ms": round(r["launch_ms"], 4)},
-        "prefill_more": more,
-        "fused_bc_norm": fused,
-        "time_varying_decay": tva,
-        "grouped_bc": grp,
-        "backward": bwd,
-        "gated_norm": gated,
-        "decode": dec,
         "e2e": {"value": round(e2e_value, 3), "unit": "Mtokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": args.steps,
+        "nccl_world_size": world,
         "clocks": clocks,
+        "side_units": "ms / us per launch or step; gbs and frac against the same HBM peak as roofline",
+        "fused_bc_norm": fused,
+        "time_varying_decay": tva,
+        "grouped_bc": grp,
+        "gated_norm": gated,
+        "backward": bwd,
+        "decode": dec,
+        "prefill_more": more,
     }
     if rank == 0:
         cpu = cpu_baseline(args)
@@ -600,21 +593,37 @@ def ours(args):
 
 
 # --------------------------------------------------------------------------- oracle arms
+def host_threads() -> int:
+    """Host threads this process may use: its CPU affinity, capped by a cgroup
+    CPU quota when one is set (a container's os.cpu_count() reports the host)."""
+    n = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    try:
+        with open("/sys/fs/cgroup/cpu.max") as f:
+            q, per = f.read().split()[:2]
+        if q != "max":
+            n = min(n, max(1, int(math.ceil(int(q) / int(per)))))
+    except (OSError, ValueError):
+        pass
+    return max(1, n)
+
+
 class OracleSample:
-    """The fp64 oracle (as it stands, all host cores) on whole (batch, head)
-    units of the prefill workload, sized by a one-unit calibration."""
+    """The fp64 oracle (as it stands, on the host threads available) on whole
+    (batch, head) units of the prefill workload, sized by a calibration round of
+    one unit per thread run in parallel."""
 
     def __init__(self, target_s: float):
         import oracle
         self.oracle = oracle
         w = PREFILL
-        self.threads = os.cpu_count() or 1
-        one_in = wl.to_f64({k: v for k, v in wl.make_inputs(w.with_(batch=1), device="cpu").items()})
+        self.threads = min(host_threads(), w.batch * w.nheads)
+        cal_batch = -(-self.threads // w.nheads)
+        cal = wl.to_f64(wl.make_inputs(w.with_(batch=cal_batch), device="cpu"))
         t = time.perf_counter()
-        oracle.scan_complex(**one_in, units=[0], nthreads=1)
-        one = time.perf_counter() - t
-        units = int(target_s * self.threads / max(one, 1e-3))
-        self.units = max(1, min(units, w.batch * w.nheads))
+        oracle.scan_complex(**cal, units=list(range(self.threads)), nthreads=self.threads)
+        per_round = time.perf_counter() - t
+        rounds = max(1, int(target_s / max(per_round, 1e-3)))
+        self.units = max(1, min(self.threads * rounds, w.batch * w.nheads))
         batch = -(-self.units // w.nheads)
         self.f = wl.to_f64(wl.make_inputs(w.with_(batch=batch), device="cpu"))
 
@@ -636,7 +645,7 @@ def cpu_baseline(args):
         mtok, sec = o.run()
     except Exception as e:  # the baseline is a report, never a reason to lose the line
         return {"error": str(e)[:200]}
-    return {"value": round(mtok, 6), "unit": "Mtokens/s", "cores": o.cores, "kind": "oracle",
+    return {"value": round(mtok, 6), "unit": "Mtokens/s", "cores": o.cores, "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"{o.units} of {PREFILL.batch * PREFILL.nheads} (batch, head) units of the prefill workload, "
                       f"all {PREFILL.seqlen} tokens each, {sec:.1f} s"}
 
@@ -670,10 +679,9 @@ def reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded)",
-        "config": {"workload": PREFILL.name, "batch": PREFILL.batch, "seqlen": PREFILL.seqlen,
-                   "nheads": PREFILL.nheads, "headdim": PREFILL.headdim, "dstate": PREFILL.dstate,
-                   "rank": PREFILL.rank},
+        "config": bench_config(world),
         "cpu_baseline": {"value": round(value, 6), "unit": "Mtokens/s", "cores": threads, "kind": "oracle",
+                         "cpu_model": cpu_model(),
                          "sample": f"each step: {units} (batch, head) units x {PREFILL.seqlen} tokens on host cores"},
         "e2e": {"value": round(value, 6), "unit": "Mtokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -689,6 +697,18 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    world_env = os.environ.get("WORLD_SIZE")
+    if args.impl == "ours" and args.gpus > 1 and world_env is None:
+        # one process per GPU: relaunch this script under torchrun with --gpus ranks
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+        sys.exit(subprocess.call(cmd))
+    if args.impl == "ours" and world_env is not None and int(world_env) != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world_env}: launch one rank per GPU")
     if args.impl == "reference":
         reference(args)
     else:

@@ -256,6 +256,35 @@ MAMBA3_API int mamba3_gated_norm(const mamba3_dims* dims, int groups, const void
 MAMBA3_API int mamba3_device_status(const void* workspace, void* stream);
 
 /*
+ * Device status of the decode step.  The decode entry points take no
+ * workspace, so their status word is a library-owned one per device: a decode
+ * kernel whose bounded wait for its own state copies gives up records
+ * MAMBA3_ERR_TIMEOUT there (and lets the copies already issued land before it
+ * exits).  The word is sticky: this call synchronises `stream`, returns the
+ * code recorded on the current device since the last call (MAMBA3_OK if none)
+ * and clears it.  Shared by every decode call on the device.
+ */
+MAMBA3_API int mamba3_decode_status(void* stream);
+
+/*
+ * Bound of every on-device wait (the prefill's pipeline barriers, the decode
+ * step's copy barriers, the backward pass's), in SM clock cycles; default
+ * 4e9 (about 2 s).  A wait that reaches it ends its kernel with
+ * MAMBA3_ERR_TIMEOUT in the status word; the kernel first lets every copy and
+ * tensor-core operation it issued complete, so the context stays usable.
+ * Process-wide, read at each launch; cycles >= 1000, else MAMBA3_ERR_INVALID.
+ */
+MAMBA3_API int mamba3_set_wait_limit(long long cycles);
+
+/*
+ * For testing the timeout path only: while `on` is non-zero, the prefill's
+ * producer and the decode step issue none of their input copies, so every
+ * kernel launched meanwhile ends with MAMBA3_ERR_TIMEOUT after the wait limit
+ * (its outputs are then undefined).  Process-wide; off by default.
+ */
+MAMBA3_API int mamba3_test_withhold_loads(int on);
+
+/*
  * Bytes of library-owned device scratch behind mamba3_scan_fwd_noalloc
  * (a file-scope device array; every GPU that loads the library holds it
  * until the process exits).
@@ -276,7 +305,9 @@ MAMBA3_API int mamba3_device_status(const void* workspace, void* stream);
  * caller workspace.  Nothing is allocated and nothing is freed.
  *  - The first call on a device (with that device current) looks the scratch's
  *    device address up once (cudaGetSymbolAddress); make that first call
- *    before any stream capture on that device.
+ *    before any stream capture on that device.  The address is kept for the
+ *    life of the process: it assumes the device's primary context is never
+ *    torn down (no cudaDeviceReset between calls).
  *  - Problems that need more scratch than MAMBA3_NOALLOC_SCRATCH_BYTES
  *    (mamba3_scan_workspace_bytes) are rejected with MAMBA3_ERR_WORKSPACE
  *    before anything is enqueued.

@@ -12,7 +12,8 @@ Entry points (same names as the C ABI):
   mamba3_decode_step(state, x, B, C, theta, dt, lam, A, D=None, ...)
   mamba3_scan_fwd_bcnorm / mamba3_decode_step_bcnorm (raw B, C + BCNorm)
   mamba3_scan_fwd_at / mamba3_decode_step_at (time-varying decay A_t)
-  mamba3_device_status(workspace)
+  mamba3_device_status(workspace), mamba3_decode_status()
+  mamba3_set_wait_limit(cycles), mamba3_test_withhold_loads(on)
   mamba3_status_string(code)
 """
 from __future__ import annotations
@@ -116,6 +117,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba3_scan_bwd_at.restype = i
     lib.mamba3_gated_norm.argtypes = [ctypes.POINTER(Dims), i, vp, vp, vp, ctypes.c_float, vp, vp]
     lib.mamba3_gated_norm.restype = i
+    lib.mamba3_decode_status.argtypes = [vp]
+    lib.mamba3_decode_status.restype = i
+    lib.mamba3_set_wait_limit.argtypes = [ctypes.c_longlong]
+    lib.mamba3_set_wait_limit.restype = i
+    lib.mamba3_test_withhold_loads.argtypes = [i]
+    lib.mamba3_test_withhold_loads.restype = i
     _lib = lib
     return lib
 
@@ -467,11 +474,28 @@ def mamba3_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(load_library().mamba3_device_status(_ptr(workspace), _stream(stream)))
 
 
+def mamba3_decode_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the decode step's status word on
+    the current device (MAMBA3_OK, or MAMBA3_ERR_TIMEOUT since the last call)."""
+    return int(load_library().mamba3_decode_status(_stream(stream)))
+
+
+def mamba3_set_wait_limit(cycles: int) -> None:
+    """Bound of every on-device wait in SM cycles (default 4e9, about 2 s)."""
+    _check(load_library().mamba3_set_wait_limit(int(cycles)), "mamba3_set_wait_limit")
+
+
+def mamba3_test_withhold_loads(on: bool) -> None:
+    """Testing the timeout path only: kernels launched while on issue no input
+    copies, so their waits give up with MAMBA3_ERR_TIMEOUT."""
+    _check(load_library().mamba3_test_withhold_loads(1 if on else 0), "mamba3_test_withhold_loads")
+
+
 __all__ = [
     "Dims", "State", "BCNorm", "Mamba3Error", "load_library", "make_dims",
     "mamba3_scan_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc", "mamba3_decode_step",
     "mamba3_scan_fwd_bcnorm", "mamba3_decode_step_bcnorm", "mamba3_scan_fwd_at", "mamba3_decode_step_at",
     "mamba3_scan_bwd_workspace_bytes", "mamba3_scan_bwd", "mamba3_scan_bwd_at", "mamba3_gated_norm",
-    "mamba3_device_status",
+    "mamba3_device_status", "mamba3_decode_status", "mamba3_set_wait_limit", "mamba3_test_withhold_loads",
     "mamba3_status_string",
 ]

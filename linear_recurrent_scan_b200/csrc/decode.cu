@@ -39,6 +39,11 @@ __device__ __forceinline__ size_t bc_row(const DecodeArgs& a, int u) {
 constexpr int kThreads = 128;
 constexpr int kMaxRows = 16;  // rows of h per thread (N <= kMaxRows * G)
 
+// Status word of the decode step, one per device (the decode entry points take
+// no workspace).  A timed-out wait records MAMBA3_ERR_TIMEOUT here; it stays set
+// until mamba3_decode_status reads and clears it.
+__device__ DeviceStatus g_decode_status;
+
 template <typename T, int R>
 __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
   const int P = a.P, N = a.N, K = N / 2;
@@ -248,7 +253,11 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
   ptx::grid_launch_dependents();
   ptx::grid_dependency_wait();
 
-  auto issue_loads = [&](int u, int stage) {
+  // stage -> 1 + iteration whose loads were issued into it and not yet waited for
+  int inflight[2] = {0, 0};
+  auto issue_loads = [&](int u, int stage, int iter) {
+    if (a.test_withhold) return;  // testing the timeout path only: the wait below must give up
+    inflight[stage] = iter + 1;
     uint8_t* st = dsm + stage * S::BYTES;
     uint64_t* bar = &bars[stage];
     ptx::mbar_arrive_expect_tx(bar, S::LOADED);
@@ -264,14 +273,14 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
 
   int it = 0;
   int u = blockIdx.x;
-  if (tid == 0 && u < units) issue_loads(u, 0);
+  if (tid == 0 && u < units) issue_loads(u, 0, 0);
   for (; u < units; u += gridDim.x, ++it) {
     const int s = it & 1;
     uint8_t* st = dsm + s * S::BYTES;
     const int un = u + gridDim.x;
     if (tid == 0 && un < units) {
       ptx::bulk_wait_read<0>();  // the other stage's previous state store has read its source
-      issue_loads(un, s ^ 1);
+      issue_loads(un, s ^ 1, it + 1);
     }
     const int hh = u % a.nheads;
     const float dt = ld1(static_cast<const T*>(a.dt) + u);
@@ -280,8 +289,9 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
     const float alpha = expf(dt * rate);
     const float beta = (1.f - lam) * dt * alpha, gamma = lam * dt;
     const float Dh = a.D ? a.D[hh] : 0.f;
-    ptx::mbar_wait(&bars[s], (it >> 1) & 1, abort_flag, nullptr, 0);
+    ptx::mbar_wait(&bars[s], (it >> 1) & 1, abort_flag, &g_decode_status, 1, a.wait_limit);
     if (__syncthreads_or(*abort_flag != 0)) break;
+    if (tid == 0) inflight[s] = 0;
     float* rinv = reinterpret_cast<float*>(dsm + S::BAR + 32);  // fused norm: 1/RMS of B rows, then C rows
     if constexpr (BCN) {  // warp w < 2R: raw row w % R of B (w < R) or of C
       if (warp < 2 * R) {
@@ -389,7 +399,13 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
     }
     __syncthreads();  // stage s and the partial sums may be reused
   }
-  if (tid == 0) ptx::bulk_wait_all();
+  if (tid == 0) {
+    // after an abort: the loads already issued land before the CTA exits
+    for (int st2 = 0; st2 < 2; ++st2)
+      if (inflight[st2] && !ptx::mbar_wait_drain(&bars[st2], ((inflight[st2] - 1) >> 1) & 1))
+        report_timeout(&g_decode_status, 2);
+    ptx::bulk_wait_all();
+  }
 }
 
 template <typename T, int N, int R, bool BCN>
@@ -449,6 +465,14 @@ int launch_stream(const DecodeArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+int decode_status_read_and_clear(int* code) {
+  DeviceStatus st, zero = {0, 0, 0, 0};
+  if (cudaMemcpyFromSymbol(&st, g_decode_status, sizeof(st)) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  if (st.code != 0 && cudaMemcpyToSymbol(g_decode_status, &zero, sizeof(zero)) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  *code = st.code;
+  return MAMBA3_OK;
+}
 
 int decode_supported(const DecodeArgs& a) {
   if (a.ngroups < 1 || a.nheads % a.ngroups != 0) return MAMBA3_ERR_INVALID;  // B, C rows per token

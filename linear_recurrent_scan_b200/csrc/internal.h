@@ -24,6 +24,9 @@ struct ScanArgs {
   int bcnorm;
   const float *nw_B, *nw_C, *nb_B, *nb_C;  // [H, R, N], each nullable
   float neps;
+  // bounded device waits: give up after about this many SM cycles (mamba3_set_wait_limit)
+  long long wait_limit;
+  int test_withhold;  // testing the timeout path only: issue no input loads
 };
 
 struct DecodeArgs {
@@ -38,6 +41,8 @@ struct DecodeArgs {
   int bcnorm;  // as in ScanArgs
   const float *nw_B, *nw_C, *nb_B, *nb_C;
   float neps;
+  long long wait_limit;  // as in ScanArgs
+  int test_withhold;
 };
 
 // Backward of the prefill: the forward's arguments in `f` (its y and final
@@ -80,6 +85,9 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s);
 
 int simt_scan_supported(const ScanArgs& a);
 int launch_scan_simt(const ScanArgs& a, cudaStream_t s);
+
+// Device status word of the decode step (one per device, sticky until read).
+int decode_status_read_and_clear(int* code);
 
 int tc_scan_supported(const ScanArgs& a);
 int launch_scan_tc(const ScanArgs& a, cudaStream_t s);

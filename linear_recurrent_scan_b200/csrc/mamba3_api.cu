@@ -11,6 +11,12 @@ namespace {
 
 constexpr size_t kStatusBytes = 256;
 
+// Process-wide settings of the bounded device waits (mamba3_set_wait_limit,
+// mamba3_test_withhold_loads), read at every launch.
+constexpr long long kDefaultWaitLimit = 4000000000LL;  // SM cycles, about 2 s at 1.9 GHz
+volatile long long g_wait_limit = kDefaultWaitLimit;
+volatile int g_test_withhold = 0;
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
@@ -105,6 +111,8 @@ m3::ScanArgs scan_args(const mamba3_dims* d, const void* x, const void* B, const
   a.dtype = d->in_dtype;
   a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.D = D;
   if (init) { a.h0 = init->h; a.bprev0 = init->b_prev; a.xprev0 = init->x_prev; a.angle0 = init->angle; }
+  a.wait_limit = g_wait_limit;
+  a.test_withhold = g_test_withhold;
   return a;
 }
 
@@ -166,6 +174,8 @@ int decode_impl(const mamba3_dims* d, const mamba3_state* state, const void* x, 
   a.h = state->h; a.bprev = state->b_prev; a.xprev = state->x_prev; a.angle = state->angle;
   a.x = x; a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.lam = lam; a.A = A; a.A_t = A_t; a.D = D; a.y = y;
   if (norm) set_norm(a, norm);
+  a.wait_limit = g_wait_limit;
+  a.test_withhold = g_test_withhold;
   if ((rc = m3::decode_supported(a))) return rc;
   return m3::launch_decode(a, static_cast<cudaStream_t>(stream));
 }
@@ -217,6 +227,24 @@ int mamba3_decode_step(const mamba3_dims* d, const mamba3_state* state, const vo
                        const void* C, const void* theta, const void* dt, const void* lam, const float* A,
                        const float* D, void* y, void* stream) {
   return decode_impl(d, state, x, B, C, theta, dt, lam, A, nullptr, D, nullptr, y, stream);
+}
+
+int mamba3_decode_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  int code = 0;
+  const int rc = m3::decode_status_read_and_clear(&code);
+  return rc != MAMBA3_OK ? rc : code;
+}
+
+int mamba3_set_wait_limit(long long cycles) {
+  if (cycles < 1000) return MAMBA3_ERR_INVALID;
+  g_wait_limit = cycles;
+  return MAMBA3_OK;
+}
+
+int mamba3_test_withhold_loads(int on) {
+  g_test_withhold = on ? 1 : 0;
+  return MAMBA3_OK;
 }
 
 int mamba3_device_status(const void* workspace, void* stream) {

@@ -252,7 +252,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
     const bool last_chunk = (c == nchunks - 1);
 
     // ---- phase A (no shared state): in-warp scan of dt*A*log2(e); theta of this part ----
-    mbar_wait(&bars[bThFull], c & 1, abort_flag, status, kTagTh);
+    mbar_wait(&bars[bThFull], c & 1, abort_flag, status, kTagTh, a.wait_limit);
     if (dl_tma) {  // this chunk's dt and lam from the tile (rows past the sequence read 0)
       if (pt < Q) {
         s_dt = __bfloat162float(dts[pt * 8]);
@@ -291,7 +291,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
     // thread read the next chunk's values.
     mbar_arrive(&bars[bThFree]);
     const float4 base = *reinterpret_cast<const float4*>(phi + 4 * g);
-    mbar_wait(&bars[bFull0 + s], u & 1, abort_flag, status, kTagFull);
+    mbar_wait(&bars[bFull0 + s], u & 1, abort_flag, status, kTagFull, a.wait_limit);
     if (prep_sync_any(*abort_flag != 0)) return;  // barrier 1: one decision for all prep threads
 
     // ---- phase B: scalars, prefix of the angle, RoPE ----
@@ -425,7 +425,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       const int tj = j / R, tref = (32 * qq) / R;
       colf[pt] = ex2(c2[tref] - c2[tj]) * wv[tj];
     }
-    if (c > 0) mbar_wait(&bars[bAcc], (c - 1) & 1, abort_flag, status, kTagAcc);
+    if (c > 0) mbar_wait(&bars[bAcc], (c - 1) & 1, abort_flag, status, kTagAcc, a.wait_limit);
     if (prep_sync_any(*abort_flag != 0)) return;  // barrier 3: wsc visible, X_w free
     {
       uint4 xq[4];
@@ -558,8 +558,8 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     const float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *colf = sc + 4 * Q + colf_off;
 
     // ---- S -> P (bf16, into TMEM) ----
-    mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1);
-    mbar_wait(&bars[bSFull], c & 1, abort_flag, status, kTagSFull);
+    mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1, a.wait_limit);
+    mbar_wait(&bars[bSFull], c & 1, abort_flag, status, kTagSFull, a.wait_limit);
     if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
     tc_fence_after();
     // every scalar this chunk needs is read now: prep may refill this stage's
@@ -611,7 +611,7 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     mbar_arrive(&bars[bPReady]);
 
     // ---- state update hbar = e^{cum_end} hbar + Hacc (this half's 32 columns) ----
-    mbar_wait(&bars[bAcc], c & 1, abort_flag, status, kTagAcc);
+    mbar_wait(&bars[bAcc], c & 1, abort_flag, status, kTagAcc, a.wait_limit);
     if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
     tc_fence_after();
 #pragma unroll
@@ -637,7 +637,7 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
                 tmem + lane_base + kColYi + ((c - 1) & 1) * kColYBuf, e_prev, b, hh, t0 - Q + tm, rm, R, ch);
       e_prev = my_e;
     } else {
-      mbar_wait(&bars[bYFull], c & 1, abort_flag, status, kTagY);
+      mbar_wait(&bars[bYFull], c & 1, abort_flag, status, kTagY, a.wait_limit);
       if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
       tc_fence_after();
       const int tg = t0 + tm;
@@ -668,7 +668,7 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     mbar_arrive(&bars[bEpiDone]);
   }
   if constexpr (K::DEFER_Y) {  // y of the last chunk (the Y barrier is committed for it alone)
-    mbar_wait(&bars[bYFull], 0, abort_flag, status, kTagY);
+    mbar_wait(&bars[bYFull], 0, abort_flag, status, kTagY, a.wait_limit);
     if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
     tc_fence_after();
     const int cl = nchunks - 1;
@@ -752,7 +752,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long t_last = clock64();
       const uint32_t th_bytes =
           K::TH_BYTES + (prm.dl_tma ? 2u * K::DL_BYTES : 0u) + (prm.at_tma ? (uint32_t)K::AT_BYTES : 0u);
-      while (cx < nchunks || ct < nchunks) {
+      // (test_withhold: issue nothing, so that every wait on a load must time out)
+      while (!a.test_withhold && (cx < nchunks || ct < nchunks)) {
         bool progress = false;
         if (cb < nchunks && mbar_test(&bars[bEmptyBC0 + (cb & 1)], ((cb >> 1) & 1) ^ 1)) {
           const int s = cb & 1, t0 = cb * Q;
@@ -788,7 +789,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           t_last = clock64();
         } else {
           if (*abort_flag) break;
-          if (clock64() - t_last > 4000000000LL) {
+          if (clock64() - t_last > a.wait_limit) {
             *abort_flag = 1;
             report_timeout(status, kTagEmpty);
             break;
@@ -802,8 +803,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (; cx < cb; ++cx)
         tma_load_5d(smem + (cx & 1) * K::STAGE_BYTES + K::OFF_X, &tmX, &bars[bFull0 + (cx & 1)], 0, 0, hh, cx * Q, b);
       for (int c = cb - 2; c < cb; ++c)
-        if (c >= 0) mbar_wait(&bars[bFull0 + (c & 1)], (c >> 1) & 1, abort_flag, status, kTagDrain, 400000000LL);
-      if (ct > 0) mbar_wait(&bars[bThFull], (ct - 1) & 1, abort_flag, status, kTagDrain, 400000000LL);
+        if (c >= 0 && !mbar_wait_drain(&bars[bFull0 + (c & 1)], (c >> 1) & 1)) report_timeout(status, kTagDrain);
+      if (ct > 0 && !mbar_wait_drain(&bars[bThFull], (ct - 1) & 1)) report_timeout(status, kTagDrain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -818,7 +819,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t st = sbase + s * K::STAGE_BYTES;
         const uint32_t cB = st + K::OFF_B, cC = st + K::OFF_C, cX = st + K::OFF_X, cXw = sbase + K::OFF_XW;
         const uint32_t ybuf = K::DEFER_Y ? (c & 1) * kColYBuf : 0u;  // Y, Yi buffer of this chunk
-        if (!mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1)) break;
+        if (!mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1, a.wait_limit)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < N / 16; ++kk) {
@@ -827,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       kk > 0);
         }
         mma_commit(&bars[bSFull]);
-        if (!mbar_wait(&bars[bEpiDone], c & 1, abort_flag, status, kTagEpiDone)) break;
+        if (!mbar_wait(&bars[bEpiDone], c & 1, abort_flag, status, kTagEpiDone, a.wait_limit)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < N / 16; ++kk) {
@@ -842,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bars[bAcc]);
         mma_commit(&bars[bEmptyBC0 + s]);  // B~, C~ of this stage are no longer read
-        if (!mbar_wait(&bars[bPReady], c & 1, abort_flag, status, kTagP)) break;
+        if (!mbar_wait(&bars[bPReady], c & 1, abort_flag, status, kTagP, a.wait_limit)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kM / 16; ++kk) {
@@ -856,7 +857,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every MMA this thread issued must be complete before TMEM is released
       mma_commit(&bars[bDone]);
-      mbar_wait(&bars[bDone], 0, abort_flag, status, kTagDrain, 400000000LL);
+      if (!mbar_wait_drain(&bars[bDone], 0)) report_timeout(status, kTagDrain);
     }
   } else if (tid < kEpi0) {
     prep_role<N, R, V>(smem, a, nchunks, prm.dl_tma, b, hh, a.A ? a.A[hh] : 0.f, bars, abort_flag, status);

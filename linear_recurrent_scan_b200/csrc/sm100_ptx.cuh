@@ -86,6 +86,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait that ignores the abort flag, for the abort path itself: copies
+// and MMAs that were already issued must land before the CTA frees TMEM or
+// exits, whatever the other roles decided.  Returns false after ~`limit` cycles.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, long long limit = 400000000LL) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (clock64() - t0 > limit) return false;
+  }
+}
+
 // ---------------------------------------------------------------- programmatic dependent launch
 // Allow the grid launched after this one in the stream (with programmatic
 // stream serialization) to be scheduled before this grid completes.

@@ -1,10 +1,11 @@
-"""Run a few prefills (and optionally decode steps) of one workload, for profilers.
+"""Benchmark tool beside bench.py: run a few prefills (or decode steps, backward
+passes, output-side norms) of one workload, for profilers.
 
-    python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --batch 2 --reps 3
-    python -m linear_recurrent_scan_b200.profile_case --workload siso_decode_b128 --decode --reps 3
-    python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --groups 1 --reps 3
-    python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --backward --reps 3
-    python -m linear_recurrent_scan_b200.profile_case --workload siso_prefill_b8_l2048 --gated-norm 64 --reps 3
+    python profile_case.py --workload siso_prefill_b8_l2048 --batch 2 --reps 3
+    python profile_case.py --workload siso_decode_b128 --decode --reps 3
+    python profile_case.py --workload siso_prefill_b8_l2048 --groups 1 --reps 3
+    python profile_case.py --workload siso_prefill_b8_l2048 --backward --reps 3
+    python profile_case.py --workload siso_prefill_b8_l2048 --gated-norm 64 --reps 3
 
 Inputs are seeded synthetic tensors on cuda:0.  Prints the CUDA-event time
 of each call; under a profiler those times are not benchmark numbers.

@@ -189,3 +189,27 @@ def test_backward_grouped_bc_matches_oracle(shape, G, dtype):
     gr, ref = run_both(inp, dy, init, d_final)
     assert gr["dB"].shape == inp["B"].shape
     check(gr, ref, TOL[dtype])
+
+
+@pytest.mark.parametrize("shape,G,dtype", [
+    ((2, 45, 4, 16, 32, 4), 2, torch.float32),
+    ((1, 130, 8, 64, 128, 1), 2, torch.bfloat16),
+])
+def test_backward_time_varying_decay_grouped_bc_matches_oracle(shape, G, dtype):
+    """mamba3_scan_bwd_at with B, C shared by groups of heads: dB, dC summed over
+    each group's heads and dA_t per token, against the oracle with A as [b, L, H]."""
+    b, L, H, P, N, R = shape
+    inp = small_inputs(b, L, H, P, N, R, dtype, seed=4300 + L + G)
+    inp.update(wl.grouped_bc(inp, G, seed=4400 + L))
+    A_t = wl.decay_rates(inp["dt"], seed=4500 + L)
+    dy = dy_like(inp["x"], 4600 + L)
+    init, d_final = rand_state(b, H, P, N, R, 4700 + L), rand_state(b, H, P, N, R, 4800 + L)
+    gr = m3.mamba3_scan_bwd_at(*(inp[n] for n in NAMES), A_t, inp["D"], dy, init=init, d_final=d_final)
+    torch.cuda.synchronize()
+    f = wl.to_f64({k: inp[k] for k in (*NAMES, "D")})
+    f["A"] = np64(A_t)
+    st = lambda s: oracle.State(*(np64(getattr(s, n)) for n, _ in STATE))
+    ref = oracle.scan_bwd(**f, dy=np64(dy), init=st(init), d_final=st(d_final))
+    gr["dA"] = gr["dA_t"]
+    assert gr["dB"].shape == inp["B"].shape
+    check(gr, ref, TOL[dtype])
