@@ -1,6 +1,7 @@
 // Internal launcher interface between the C ABI (mamba3_api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -56,8 +57,9 @@ struct BwdArgs {
   void* dA_t;  // with f.A_t: the decay-rate gradient per token (layout of dt, dtype of x); dA null
   float *dh0, *dbprev0, *dxprev0, *dangle0;                      // all null = not wanted
   float* ckpt;  // [units][chunks][N*P + N/2]: hbar and Phi at every chunk start
-  float *dBh, *dCh;  // grouped B, C: per-head fp32 gradients [b, L, H, R, N], summed into dB, dC
-                     // over each group's heads afterwards; null with one row per head
+  float *dBh, *dCh;  // grouped B, C: fp32 scratch for their gradients (SIMT path: per head
+                     // [b, L, H, R, N], summed afterwards; tensor-core path: the group sums
+                     // [b, L, G, R, N] themselves); null with one row per head
 };
 
 // Pre-gate grouped RMS norm and gate of the layer output: rows = tokens x groups
@@ -77,6 +79,12 @@ size_t bwd_checkpoint_bytes(const ScanArgs& a);
 size_t bwd_group_bytes(const ScanArgs& a);  // per-head B, C gradients when B, C are grouped
 int bwd_supported(const ScanArgs& a);
 int launch_scan_bwd(const BwdArgs& g, cudaStream_t s);
+// The tensor-core backward (scan_bwd_tc.cu): bf16, P = 64, N in {64, 128}, R in
+// {1, 2, 4}, seqlen >= 1.  Its workspace after the status word: the state
+// checkpoints, then (grouped B/C) the fp32 group sums of dB and dC.
+int bwd_tc_supported(const ScanArgs& a);
+size_t bwd_tc_workspace_bytes(const ScanArgs& a);
+int launch_scan_bwd_tc(BwdArgs g, cudaStream_t s);
 
 // Each launcher returns MAMBA3_OK, MAMBA3_ERR_UNSUPPORTED (shape not compiled)
 // or MAMBA3_ERR_CUDA (launch failure).
@@ -88,6 +96,14 @@ int launch_scan_simt(const ScanArgs& a, cudaStream_t s);
 
 // Device status word of the decode step (one per device, sticky until read).
 int decode_status_read_and_clear(int* code);
+
+// TMA tensor maps over the prefill's inputs (scan_tc.cu): a [batch, L, heads, R,
+// inner] bf16 tensor with box {64, R, 1, Q, 1} and 128-byte swizzle; dt or lam
+// [batch, L, H] with box {8, rows, 1}; theta [batch, L, H, N/2] with box
+// {N/2, 1, Q, 1}.  Each returns false when the driver rejects the map.
+bool make_map(CUtensorMap* m, const void* base, int inner, int heads, const ScanArgs& a, int Q);
+bool make_dl_map(CUtensorMap* m, const void* base, const ScanArgs& a, int rows);
+bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q);
 
 int tc_scan_supported(const ScanArgs& a);
 int launch_scan_tc(const ScanArgs& a, cudaStream_t s);

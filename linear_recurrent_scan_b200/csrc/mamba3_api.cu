@@ -276,10 +276,12 @@ int scan_bwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
   }
   if ((rc = check_state(init)) || (rc = check_state(d_final)) || (rc = check_state(d_init))) return rc;
   if (!workspace || !aligned16(workspace)) return MAMBA3_ERR_WORKSPACE;
-  const m3::ScanArgs sizes = scan_args(d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                       nullptr);
+  m3::ScanArgs sizes = scan_args(d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                 nullptr);
+  const bool use_tc = m3::bwd_tc_supported(sizes) == MAMBA3_OK;
   const size_t ckpt_bytes = m3::bwd_checkpoint_bytes(sizes);
-  if (workspace_bytes < kStatusBytes + ckpt_bytes + m3::bwd_group_bytes(sizes)) return MAMBA3_ERR_WORKSPACE;
+  const size_t need = use_tc ? m3::bwd_tc_workspace_bytes(sizes) : ckpt_bytes + m3::bwd_group_bytes(sizes);
+  if (workspace_bytes < kStatusBytes + need) return MAMBA3_ERR_WORKSPACE;
   m3::BwdArgs g;
   memset(&g, 0, sizeof(g));
   g.f = scan_args(d, x, B, C, theta, dt, lam, A, D, init);
@@ -294,11 +296,15 @@ int scan_bwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
   g.dx = dx; g.dB = dB; g.dC = dC; g.dtheta = dtheta; g.ddt = ddt; g.dlam = dlam; g.dA = dA; g.dA_t = dA_t; g.dD = dD;
   if (d_init) { g.dh0 = d_init->h; g.dbprev0 = d_init->b_prev; g.dxprev0 = d_init->x_prev; g.dangle0 = d_init->angle; }
   g.ckpt = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_tc) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
+    return m3::launch_scan_bwd_tc(g, s);
+  }
   if (m3::bwd_group_bytes(sizes)) {
     g.dBh = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes + ckpt_bytes);
     g.dCh = g.dBh + (size_t)d->batch * d->seqlen * d->nheads * d->rank * d->dstate;
   }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
   return m3::launch_scan_bwd(g, s);
 }
@@ -309,6 +315,7 @@ extern "C" {
 size_t mamba3_scan_bwd_workspace_bytes(const mamba3_dims* d) {
   if (check_dims(d, true) != MAMBA3_OK) return 0;
   const m3::ScanArgs a = scan_args(d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  if (m3::bwd_tc_supported(a) == MAMBA3_OK) return kStatusBytes + m3::bwd_tc_workspace_bytes(a);
   return kStatusBytes + m3::bwd_checkpoint_bytes(a) + m3::bwd_group_bytes(a);
 }
 

@@ -52,6 +52,71 @@
 #include "sm100_ptx.cuh"
 
 namespace m3 {
+
+// ------------------------------------------------------------------ TMA tensor maps (shared with the backward pass)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [batch, L, H, R, inner] bf16 tensor, box = {64, R, 1, Q, 1}, 128-byte swizzle,
+// zero fill past the end of the sequence.
+bool make_map(CUtensorMap* m, const void* base, int inner, int heads, const ScanArgs& a, int Q) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[5] = {(cuuint64_t)inner, (cuuint64_t)a.R, (cuuint64_t)heads, (cuuint64_t)a.seqlen,
+                              (cuuint64_t)a.batch};
+  const cuuint64_t e = 2;
+  const cuuint64_t strides[4] = {e * inner, e * inner * a.R, e * inner * a.R * heads,
+                                 e * inner * a.R * heads * a.seqlen};
+  const cuuint32_t box[5] = {64, (cuuint32_t)a.R, 1, (cuuint32_t)Q, 1};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// dt or lam [batch, L, H] bf16, box = {8, Q + 1, 1}: the 8 heads of a 16-byte
+// group over the chunk's tokens and the next one, zero fill past the end.
+// Needs H a multiple of 8 (16-byte row stride) and a 16-byte aligned base.
+bool make_dl_map(CUtensorMap* m, const void* base, const ScanArgs& a, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || a.nheads % 8 != 0 || (reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)a.nheads, (cuuint64_t)a.seqlen, (cuuint64_t)a.batch};
+  const cuuint64_t strides[2] = {2ull * a.nheads, 2ull * a.nheads * a.seqlen};
+  const cuuint32_t box[3] = {8, (cuuint32_t)rows, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// theta [batch, L, H, N/2] bf16, box = {N/2, 1, Q, 1}, no swizzle, zero fill past the end.
+bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int K2 = a.N / 2;
+  const cuuint64_t dims[4] = {(cuuint64_t)K2, (cuuint64_t)a.nheads, (cuuint64_t)a.seqlen, (cuuint64_t)a.batch};
+  const cuuint64_t strides[3] = {2ull * K2, 2ull * K2 * a.nheads, 2ull * K2 * a.nheads * a.seqlen};
+  const cuuint32_t box[4] = {(cuuint32_t)K2, 1, (cuuint32_t)Q, 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(a.theta), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+
 namespace {
 
 using namespace ptx;
@@ -874,68 +939,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// [batch, L, H, R, inner] bf16 tensor, box = {64, R, 1, Q, 1}, 128-byte swizzle,
-// zero fill past the end of the sequence.
-bool make_map(CUtensorMap* m, const void* base, int inner, int heads, const ScanArgs& a, int Q) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[5] = {(cuuint64_t)inner, (cuuint64_t)a.R, (cuuint64_t)heads, (cuuint64_t)a.seqlen,
-                              (cuuint64_t)a.batch};
-  const cuuint64_t e = 2;
-  const cuuint64_t strides[4] = {e * inner, e * inner * a.R, e * inner * a.R * heads,
-                                 e * inner * a.R * heads * a.seqlen};
-  const cuuint32_t box[5] = {64, (cuuint32_t)a.R, 1, (cuuint32_t)Q, 1};
-  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// dt or lam [batch, L, H] bf16, box = {8, Q + 1, 1}: the 8 heads of a 16-byte
-// group over the chunk's tokens and the next one, zero fill past the end.
-// Needs H a multiple of 8 (16-byte row stride) and a 16-byte aligned base.
-bool make_dl_map(CUtensorMap* m, const void* base, const ScanArgs& a, int rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc || a.nheads % 8 != 0 || (reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)a.nheads, (cuuint64_t)a.seqlen, (cuuint64_t)a.batch};
-  const cuuint64_t strides[2] = {2ull * a.nheads, 2ull * a.nheads * a.seqlen};
-  const cuuint32_t box[3] = {8, (cuuint32_t)rows, 1};
-  const cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// theta [batch, L, H, N/2] bf16, box = {N/2, 1, Q, 1}, no swizzle, zero fill past the end.
-bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const int K2 = a.N / 2;
-  const cuuint64_t dims[4] = {(cuuint64_t)K2, (cuuint64_t)a.nheads, (cuuint64_t)a.seqlen, (cuuint64_t)a.batch};
-  const cuuint64_t strides[3] = {2ull * K2, 2ull * K2 * a.nheads, 2ull * K2 * a.nheads * a.seqlen};
-  const cuuint32_t box[4] = {(cuuint32_t)K2, 1, (cuuint32_t)Q, 1};
-  const cuuint32_t es[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(a.theta), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int N, int R>
 int launch_nr(const ScanArgs& a, cudaStream_t s) {
   using K = Cfg<N, R>;
