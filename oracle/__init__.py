@@ -93,6 +93,10 @@ def _bind(lib):
     lib.m3o_gated_norm.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int, _P, _P, _P, ctypes.c_double, _P]
     lib.m3o_gated_norm.restype = ctypes.c_int
     lib.m3o_bc_norm.restype = ctypes.c_int
+    for name in ("m3o_mimo_up", "m3o_mimo_down"):
+        f = getattr(lib, name)
+        f.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P]
+        f.restype = ctypes.c_int
     return lib
 
 
@@ -303,8 +307,37 @@ def gated_norm(y, z, w=None, groups: Optional[int] = None, eps: float = 1e-6) ->
     return out
 
 
+def mimo_up(u, Wx, rank: int) -> np.ndarray:
+    """MIMO input projection (rank R) per head: u [..., H, P], Wx [H, R P, P]
+    -> x [..., H, R, P] with x[.., h, r, p] = sum_q Wx[h, r P + p, q] u[.., h, q].
+    Source: "Mamba-3: 2x smaller state ..." (MarkTechPost, Korean translation),
+    section 1.3 (x_t is P x R); one dense matrix per head is this build's reading."""
+    u, Wx = _f64(u), _f64(Wx)
+    *lead, H, P = u.shape
+    assert Wx.shape == (H, rank * P, P), "Wx must be [H, R P, P]"
+    rows = int(np.prod(lead)) if lead else 1
+    dims = _Dims(1, rows, H, P, 0, rank, 0)
+    x = np.empty((*lead, H, rank, P))
+    _load().m3o_mimo_up(ctypes.byref(dims), _ptr(u), _ptr(Wx), _ptr(x))
+    return x
+
+
+def mimo_down(y, Wy) -> np.ndarray:
+    """MIMO output projection per head: y [..., H, R, P], Wy [H, P, R P] -> o
+    [..., H, P] with o[.., h, p] = sum_{r, q} Wy[h, p, r P + q] y[.., h, r, q]
+    (same page and reading as mimo_up)."""
+    y, Wy = _f64(y), _f64(Wy)
+    *lead, H, R, P = y.shape
+    assert Wy.shape == (H, P, R * P), "Wy must be [H, P, R P]"
+    rows = int(np.prod(lead)) if lead else 1
+    dims = _Dims(1, rows, H, P, 0, R, 0)
+    o = np.empty((*lead, H, P))
+    _load().m3o_mimo_down(ctypes.byref(dims), _ptr(y), _ptr(Wy), _ptr(o))
+    return o
+
+
 __all__ = ["build", "State", "scan_complex", "scan_rope", "scan_quadratic", "decode_step", "bc_norm", "scan_bwd",
-           "gated_norm"]
+           "gated_norm", "mimo_up", "mimo_down"]
 
 
 def bc_norm(z, w=None, bias=None, eps: float = 1e-6) -> np.ndarray:

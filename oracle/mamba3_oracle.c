@@ -716,3 +716,51 @@ int m3o_gated_norm(const m3o_dims* d, int groups, const double* y, const double*
   }
   return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* MIMO rank-R projections around the recurrence.
+ *
+ * Same page, section 1.3: MIMO raises the rank of the input and output
+ * projections to R, so that x_t is P x R (and B_t N x R) and the state update
+ * becomes a matrix product.  The page prints no weights; the plainest reading
+ * taken here is one dense matrix per head on each side of the recurrence:
+ *   up:    x[b,t,h,r,p] = sum_q Wx[h, r P + p, q] u[b,t,h,q]
+ *          u [b, L, H, P],  Wx [H, R P, P],  x [b, L, H, R, P]
+ *   down:  o[b,t,h,p]   = sum_r sum_q Wy[h, p, r P + q] y[b,t,h,r,q]
+ *          y [b, L, H, R, P],  Wy [H, P, R P],  o [b, L, H, P]
+ * (R = 1 with identity weights leaves u and y unchanged: SISO.)  Plain loops,
+ * fp64; d->dstate is ignored.
+ */
+int m3o_mimo_up(const m3o_dims* d, const double* u, const double* Wx, double* x) {
+  const int H = d->nheads, R = d->rank, P = d->headdim;
+  const size_t tokens = (size_t)d->batch * d->seqlen;
+  for (size_t t = 0; t < tokens; ++t)
+    for (int h = 0; h < H; ++h) {
+      const double* ut = u + (t * H + h) * P;
+      const double* W = Wx + (size_t)h * R * P * P;
+      double* xt = x + (t * H + h) * (size_t)R * P;
+      for (int rp = 0; rp < R * P; ++rp) {
+        double acc = 0.0;
+        for (int q = 0; q < P; ++q) acc += W[(size_t)rp * P + q] * ut[q];
+        xt[rp] = acc;
+      }
+    }
+  return 0;
+}
+
+int m3o_mimo_down(const m3o_dims* d, const double* y, const double* Wy, double* o) {
+  const int H = d->nheads, R = d->rank, P = d->headdim;
+  const size_t tokens = (size_t)d->batch * d->seqlen;
+  for (size_t t = 0; t < tokens; ++t)
+    for (int h = 0; h < H; ++h) {
+      const double* yt = y + (t * H + h) * (size_t)R * P;
+      const double* W = Wy + (size_t)h * P * R * P;
+      double* ot = o + (t * H + h) * P;
+      for (int p = 0; p < P; ++p) {
+        double acc = 0.0;
+        for (int rq = 0; rq < R * P; ++rq) acc += W[(size_t)p * R * P + rq] * yt[rq];
+        ot[p] = acc;
+      }
+    }
+  return 0;
+}

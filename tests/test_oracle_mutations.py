@@ -13,6 +13,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_bwd_pins as bwd_pins
+from tests import test_oracle_mimo_proj_pins as proj_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "mamba3_oracle.c")
@@ -44,6 +45,8 @@ MUTATIONS = {
     "gated_norm_sum_not_mean": ("ms /= (double)gsize;", "ms /= 1.0;"),
     "gated_norm_interleaved_groups": ("const size_t h = g * hpg + c / ((size_t)R * P)",
                                       "const size_t h = g + groups * (c / ((size_t)R * P))"),
+    "mimo_up_weight_transposed": ("acc += W[(size_t)rp * P + q] * ut[q];", "acc += W[(size_t)q * P + rp % P] * ut[q];"),
+    "mimo_down_rank_stride": ("acc += W[(size_t)p * R * P + rq] * yt[rq];", "acc += W[(size_t)p * R * P + rq % P] * yt[rq];"),
     "bcnorm_bias_index_swapped": ("const size_t p = ((size_t)h * R + r) * N + n;", "const size_t p = ((size_t)r * H + h) * N + n;"),
 }
 
@@ -73,6 +76,8 @@ PIN_FUNCS = [
     pins.test_gated_norm_scale_invariant_and_group_local,
     pins.test_gated_norm_weight_per_head_rank_channel_and_eps,
     bwd_pins.test_backward_linear_in_C_and_D,
+    lambda: [proj_pins.test_up_and_down_equal_library_matrix_products(r) for r in (1, 4)],
+    proj_pins.test_rank_one_weights_closed_form,
 ]
 
 
