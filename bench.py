@@ -404,6 +404,53 @@ def run_backward(m3, w: wl.Workload, rank, steps, warmup):
     return statistics.median(times)
 
 
+def run_mimo_proj(m3, w: wl.Workload, rank, steps, warmup):
+    """Median per-launch times (ms) of the MIMO rank-R projections on workload w:
+    up (u [b, L, H, P] -> x [b, L, H, R, P]) and down with the fused RMS norm and
+    silu gate (y [b, L, H, R, P], z -> out [b, L, H, P]); bf16, weights per head."""
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.BASE_SEED + 12 + rank)
+    H, R, P = w.nheads, w.rank, w.headdim
+    u = torch.randn((w.batch, w.seqlen, H, P), generator=g, device=dev).to(w.dtype)
+    Wx = (torch.randn((H, R * P, P), generator=g, device=dev) * P ** -0.5).to(w.dtype)
+    Wy = (torch.randn((H, P, R * P), generator=g, device=dev) * (R * P) ** -0.5).to(w.dtype)
+    z = torch.randn((w.batch, w.seqlen, H, P), generator=g, device=dev).to(w.dtype)
+    wt = torch.rand((H, P), generator=g, device=dev) + 0.5
+    x = torch.empty((w.batch, w.seqlen, H, R, P), dtype=w.dtype, device=dev)
+    o = torch.empty_like(u)
+    stream = torch.cuda.current_stream()
+    res = {}
+    for name, fn in (("up", lambda: m3.mamba3_mimo_up(u, Wx, out=x, stream=stream)),
+                     ("down_gated", lambda: m3.mamba3_mimo_down(x, Wy, z=z, w=wt, out=o, stream=stream))):
+        for _ in range(warmup):
+            fn()
+        times = []
+        for _ in range(steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        res[name] = statistics.median(times)
+    status = m3.mamba3_library_status()
+    if status != 0:
+        raise RuntimeError(f"library status after the projections: {m3.mamba3_status_string(status)}")
+    del u, Wx, Wy, z, wt, x, o
+    torch.cuda.empty_cache()
+    return res
+
+
+def mimo_proj_bytes(w: wl.Workload) -> dict:
+    """Algorithmic bytes of the two projections: inputs read once, outputs written
+    once, the per-head weights once (and the gate z and norm weight for down)."""
+    s = esize(w.dtype)
+    th, H, R, P = w.token_heads, w.nheads, w.rank, w.headdim
+    wts = s * H * R * P * P
+    return {"up": th * s * (P + R * P) + wts, "down_gated": th * s * (R * P + 2 * P) + wts + 4 * H * P}
+
+
 def run_gated_norm(m3, w: wl.Workload, rank, groups, steps, warmup):
     """Median per-launch time (ms) of the output side (grouped RMS norm + gate) on
     a prefill output of workload w: y, z drawn N(0, 1), weights U(0.5, 1.5)."""
@@ -542,6 +589,13 @@ def ours(args):
             PREFILL.rank * PREFILL.headdim
         gated["groups%d" % ng] = {"ms": round(ms, 4), **rl(by, ms, peak, traffic("gated_norm_per_head")
                                                          if ng == PREFILL.nheads else None)}
+    # the MIMO rank-R projections around the recurrence (R 4 prefill shape)
+    pw = PREFILL_MORE[0]
+    pt = run_mimo_proj(m3, pw, rank, steps=side_steps, warmup=3)
+    pb = mimo_proj_bytes(pw)
+    proj = {k: {"ms": round(max_over_ranks(v, world), 4), **rl(pb[k], max_over_ranks(v, world), peak)}
+            for k, v in pt.items()}
+    proj["workload"] = pw.name
     more = {}
     for w in PREFILL_MORE:
         ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=side_steps, warmup=3), world)
@@ -578,6 +632,7 @@ def ours(args):
         "time_varying_decay": tva,
         "grouped_bc": grp,
         "gated_norm": gated,
+        "mimo_proj": proj,
         "backward": bwd,
         "decode": dec,
         "prefill_more": more,

@@ -250,21 +250,71 @@ MAMBA3_API int mamba3_scan_bwd_at(const mamba3_dims* dims, const void* x, const 
 MAMBA3_API int mamba3_gated_norm(const mamba3_dims* dims, int groups, const void* y, const void* z, const float* w,
                                  float eps, void* out, void* stream);
 
+/*
+ * Workspace with which mamba3_scan_fwd (and its _at variant) runs a long
+ * sequence over few (batch, head) units in segments: with fewer units than the
+ * GPU has SMs, the sequence is cut into S segments (S divides seqlen, at least
+ * 1024 tokens each), every segment's end state from a zero state is computed,
+ * the segment states are chained in order (a decay, a rotation by the entering
+ * angle and the sum, exact up to rounding), and the prefill runs on the b S
+ * segments at once.  The constant-size state and the angle summed over time
+ * steps ("Mamba-3 paper review" (no1joon.github.io), Table 7 discussion;
+ * "Mamba-3: 2x smaller state ..." (MarkTechPost, Korean translation), section
+ * 1.2) make the split exact.  Returns the status word's 256 bytes plus
+ * 2 b S H (N P + R N + R P + N/2) floats, or 256 when `dims` do not qualify
+ * (bf16, P = 64, N in {64, 128}, R in {1, 2, 4}, seqlen >= 2048, b H < 148);
+ * 0 for invalid dims.  Any workspace of at least mamba3_scan_workspace_bytes
+ * is accepted: a smaller one than this runs the sequence unsegmented.
+ */
+MAMBA3_API size_t mamba3_scan_segmented_workspace_bytes(const mamba3_dims* dims);
+
+/*
+ * For testing the segmented prefill on small problems only: while S >= 2, the
+ * prefill (and mamba3_scan_segmented_workspace_bytes) uses S segments whenever S
+ * divides seqlen and the shape has the segmented path, whatever the sequence
+ * length and unit count; 0 restores the library's own choice.  Process-wide.
+ */
+MAMBA3_API int mamba3_test_set_segments(int S);
+
 /* Synchronises `stream`, then returns the device status word that the last
  * mamba3_scan_fwd on `workspace` left (MAMBA3_OK or MAMBA3_ERR_TIMEOUT), or
  * MAMBA3_ERR_CUDA / MAMBA3_ERR_INVALID. */
 MAMBA3_API int mamba3_device_status(const void* workspace, void* stream);
 
 /*
- * Device status of the decode step.  The decode entry points take no
- * workspace, so their status word is a library-owned one per device: a decode
- * kernel whose bounded wait for its own state copies gives up records
- * MAMBA3_ERR_TIMEOUT there (and lets the copies already issued land before it
- * exits).  The word is sticky: this call synchronises `stream`, returns the
- * code recorded on the current device since the last call (MAMBA3_OK if none)
- * and clears it.  Shared by every decode call on the device.
+ * MIMO rank-R projections around the recurrence ("Mamba-3: 2x smaller state
+ * ..." (MarkTechPost, Korean translation), section 1.3: MIMO raises the rank of
+ * the input and output projections so that x_t is P x R).  The page prints no
+ * weights; the reading here is one dense matrix per head on each side:
+ *   up:   x[t, h, r, p] = sum_q Wx[h, r P + p, q] u[t, h, q]
+ *   down: o[t, h, p]    = sum_{r, q} Wy[h, p, r P + q] y[t, h, r, q]
+ * over every (batch, token) pair t.  With z non-null the down projection is
+ * followed by the output side of section 2 for norm groups of one head:
+ *   out = o / sqrt(mean_p o^2 + eps) * w[h, p] * silu(z[t, h, p])
+ * (w nullable: weight 1; an all-zero row with eps = 0 gives 0).
+ *   dims   batch, seqlen, nheads, headdim (P), rank (R), in_dtype; dstate,
+ *          chunk and ngroups are ignored.
+ *   u [b, L, H, P]; Wx [H, R P, P]; x [b, L, H, R, P]        (bf16)
+ *   y [b, L, H, R, P]; Wy [H, P, R P]; z, out [b, L, H, P]   (bf16); w float32 [H, P]
+ * Supported: bf16, P = 64, R in {1, 2, 4} (tcgen05 products per 128-token tile,
+ * fp32 accumulation); other valid shapes return MAMBA3_ERR_UNSUPPORTED.  Every
+ * pointer 16-byte aligned (w: 4).  Asynchronous on `stream`; no workspace (a
+ * timed-out wait is reported by mamba3_library_status).
  */
-MAMBA3_API int mamba3_decode_status(void* stream);
+MAMBA3_API int mamba3_mimo_up(const mamba3_dims* dims, const void* u, const void* Wx, void* x, void* stream);
+MAMBA3_API int mamba3_mimo_down(const mamba3_dims* dims, const void* y, const void* Wy, const void* z,
+                                const float* w, float eps, void* out, void* stream);
+
+/*
+ * Device status of the entry points that take no workspace (the decode steps
+ * and the MIMO projections): their status words are library-owned, one per
+ * device.  A kernel whose bounded wait for its own copies gives up records
+ * MAMBA3_ERR_TIMEOUT there (and lets what it issued land before it exits).
+ * The words are sticky: this call synchronises `stream`, returns the first code
+ * recorded on the current device since the last call (MAMBA3_OK if none) and
+ * clears them.  Shared by every such call on the device.
+ */
+MAMBA3_API int mamba3_library_status(void* stream);
 
 /*
  * Bound of every on-device wait (the prefill's pipeline barriers, the decode

@@ -12,7 +12,8 @@ Entry points (same names as the C ABI):
   mamba3_decode_step(state, x, B, C, theta, dt, lam, A, D=None, ...)
   mamba3_scan_fwd_bcnorm / mamba3_decode_step_bcnorm (raw B, C + BCNorm)
   mamba3_scan_fwd_at / mamba3_decode_step_at (time-varying decay A_t)
-  mamba3_device_status(workspace), mamba3_decode_status()
+  mamba3_mimo_up / mamba3_mimo_down (MIMO rank-R projections, optional fused gate)
+  mamba3_device_status(workspace), mamba3_library_status()
   mamba3_set_wait_limit(cycles), mamba3_test_withhold_loads(on)
   mamba3_status_string(code)
 """
@@ -117,8 +118,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba3_scan_bwd_at.restype = i
     lib.mamba3_gated_norm.argtypes = [ctypes.POINTER(Dims), i, vp, vp, vp, ctypes.c_float, vp, vp]
     lib.mamba3_gated_norm.restype = i
-    lib.mamba3_decode_status.argtypes = [vp]
-    lib.mamba3_decode_status.restype = i
+    lib.mamba3_scan_segmented_workspace_bytes.argtypes = [ctypes.POINTER(Dims)]
+    lib.mamba3_scan_segmented_workspace_bytes.restype = sz
+    lib.mamba3_test_set_segments.argtypes = [i]
+    lib.mamba3_test_set_segments.restype = i
+    lib.mamba3_library_status.argtypes = [vp]
+    lib.mamba3_library_status.restype = i
+    lib.mamba3_mimo_up.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp]
+    lib.mamba3_mimo_up.restype = i
+    lib.mamba3_mimo_down.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, ctypes.c_float, vp, vp]
+    lib.mamba3_mimo_down.restype = i
     lib.mamba3_set_wait_limit.argtypes = [ctypes.c_longlong]
     lib.mamba3_set_wait_limit.restype = i
     lib.mamba3_test_withhold_loads.argtypes = [i]
@@ -188,6 +197,12 @@ def mamba3_scan_workspace_bytes(dims: Dims) -> int:
     return int(load_library().mamba3_scan_workspace_bytes(ctypes.byref(dims)))
 
 
+def mamba3_scan_segmented_workspace_bytes(dims: Dims) -> int:
+    """Workspace with which a long sequence over few (batch, head) units runs in
+    segments (mamba3_scan_workspace_bytes when the dims do not qualify)."""
+    return int(load_library().mamba3_scan_segmented_workspace_bytes(ctypes.byref(dims)))
+
+
 def _check_inputs(x, B, C, theta, dt, lam, A, D, decode):
     lead = x.shape[:-2]
     for name, t in (("x", x), ("B", B), ("C", C), ("theta", theta), ("dt", dt), ("lam", lam)):
@@ -221,7 +236,7 @@ def mamba3_scan_fwd(x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = 
     if y is None:
         y = torch.empty_like(x)
     if workspace is None:
-        workspace = torch.empty(mamba3_scan_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
+        workspace = torch.empty(mamba3_scan_segmented_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
     ci = init._c() if init is not None else None
     cf = final_state._c() if final_state is not None else None
     rc = lib.mamba3_scan_fwd(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam),
@@ -304,7 +319,7 @@ def mamba3_scan_fwd_bcnorm(x, B_raw, C_raw, theta, dt, lam, A, D=None, norm: Opt
     if y is None:
         y = torch.empty_like(x)
     if workspace is None:
-        workspace = torch.empty(mamba3_scan_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
+        workspace = torch.empty(mamba3_scan_segmented_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
     ci = init._c() if init is not None else None
     cf = final_state._c() if final_state is not None else None
     rc = lib.mamba3_scan_fwd_bcnorm(ctypes.byref(dims), _ptr(x), _ptr(B_raw), _ptr(C_raw), _ptr(theta), _ptr(dt),
@@ -352,7 +367,7 @@ def mamba3_scan_fwd_at(x, B, C, theta, dt, lam, A_t, D=None, init: Optional[Stat
     if y is None:
         y = torch.empty_like(x)
     if workspace is None:
-        workspace = torch.empty(mamba3_scan_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
+        workspace = torch.empty(mamba3_scan_segmented_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
     ci = init._c() if init is not None else None
     cf = final_state._c() if final_state is not None else None
     rc = lib.mamba3_scan_fwd_at(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam),
@@ -474,15 +489,64 @@ def mamba3_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(load_library().mamba3_device_status(_ptr(workspace), _stream(stream)))
 
 
-def mamba3_decode_status(stream=None) -> int:
-    """Synchronise the stream; return and clear the decode step's status word on
-    the current device (MAMBA3_OK, or MAMBA3_ERR_TIMEOUT since the last call)."""
-    return int(load_library().mamba3_decode_status(_stream(stream)))
+def mamba3_library_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the status words of the calls
+    without a workspace (decode steps, MIMO projections) on the current device."""
+    return int(load_library().mamba3_library_status(_stream(stream)))
+
+
+def mamba3_mimo_up(u, Wx, out=None, stream=None):
+    """MIMO input projection per head: u [..., H, P] bf16, Wx [H, R P, P] bf16 ->
+    x [..., H, R, P] bf16 (allocated if not given)."""
+    lib = load_library()
+    *lead, H, P = u.shape
+    if Wx.dim() != 3 or Wx.shape[0] != H or Wx.shape[2] != P or Wx.shape[1] % P:
+        raise ValueError("Wx must be [H, R P, P]")
+    R = Wx.shape[1] // P
+    for name, t in (("u", u), ("Wx", Wx)):
+        if not t.is_contiguous() or t.dtype not in _DTYPES:
+            raise ValueError(f"{name} must be a contiguous float32 or bfloat16 tensor")
+    if out is None:
+        out = torch.empty((*lead, H, R, P), dtype=u.dtype, device=u.device)
+    tokens = u.numel() // (H * P) if H * P else 0
+    dims = Dims(1, tokens, H, P, 0, R, 0, _DTYPES[u.dtype], 0)
+    _check(lib.mamba3_mimo_up(ctypes.byref(dims), _ptr(u), _ptr(Wx), _ptr(out), _stream(stream)), "mamba3_mimo_up")
+    return out
+
+
+def mamba3_mimo_down(y, Wy, z=None, w=None, eps: float = 1e-6, out=None, stream=None):
+    """MIMO output projection per head: y [..., H, R, P] bf16, Wy [H, P, R P] bf16
+    -> [..., H, P] bf16; with the gate z [..., H, P] the RMS norm over P (weight w
+    [H, P] float32 or None) and silu(z) follow in the same kernel."""
+    lib = load_library()
+    *lead, H, R, P = y.shape
+    if tuple(Wy.shape) != (H, P, R * P):
+        raise ValueError("Wy must be [H, P, R P]")
+    for name, t in (("y", y), ("Wy", Wy)):
+        if not t.is_contiguous() or t.dtype not in _DTYPES:
+            raise ValueError(f"{name} must be a contiguous float32 or bfloat16 tensor")
+    if z is not None and (tuple(z.shape) != (*lead, H, P) or not z.is_contiguous() or z.dtype != y.dtype):
+        raise ValueError("z must be contiguous [..., H, P] in the dtype of y")
+    if w is not None and (w.dtype != torch.float32 or tuple(w.shape) != (H, P) or not w.is_contiguous()):
+        raise ValueError("w must be a contiguous float32 tensor [H, P]")
+    if out is None:
+        out = torch.empty((*lead, H, P), dtype=y.dtype, device=y.device)
+    tokens = y.numel() // (H * R * P) if H * R * P else 0
+    dims = Dims(1, tokens, H, P, 0, R, 0, _DTYPES[y.dtype], 0)
+    _check(lib.mamba3_mimo_down(ctypes.byref(dims), _ptr(y), _ptr(Wy), _ptr(z), _ptr(w), float(eps), _ptr(out),
+                                _stream(stream)), "mamba3_mimo_down")
+    return out
 
 
 def mamba3_set_wait_limit(cycles: int) -> None:
     """Bound of every on-device wait in SM cycles (default 4e9, about 2 s)."""
     _check(load_library().mamba3_set_wait_limit(int(cycles)), "mamba3_set_wait_limit")
+
+
+def mamba3_test_set_segments(S: int) -> None:
+    """Testing the segmented prefill only: S >= 2 segments whenever S divides the
+    sequence length; 0 restores the library's choice."""
+    _check(load_library().mamba3_test_set_segments(int(S)), "mamba3_test_set_segments")
 
 
 def mamba3_test_withhold_loads(on: bool) -> None:
@@ -493,9 +557,9 @@ def mamba3_test_withhold_loads(on: bool) -> None:
 
 __all__ = [
     "Dims", "State", "BCNorm", "Mamba3Error", "load_library", "make_dims",
-    "mamba3_scan_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc", "mamba3_decode_step",
+    "mamba3_scan_workspace_bytes", "mamba3_scan_segmented_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc", "mamba3_decode_step",
     "mamba3_scan_fwd_bcnorm", "mamba3_decode_step_bcnorm", "mamba3_scan_fwd_at", "mamba3_decode_step_at",
     "mamba3_scan_bwd_workspace_bytes", "mamba3_scan_bwd", "mamba3_scan_bwd_at", "mamba3_gated_norm",
-    "mamba3_device_status", "mamba3_decode_status", "mamba3_set_wait_limit", "mamba3_test_withhold_loads",
+    "mamba3_device_status", "mamba3_library_status", "mamba3_mimo_up", "mamba3_mimo_down", "mamba3_set_wait_limit", "mamba3_test_withhold_loads", "mamba3_test_set_segments",
     "mamba3_status_string",
 ]

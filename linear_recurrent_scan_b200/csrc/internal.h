@@ -94,16 +94,49 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s);
 int simt_scan_supported(const ScanArgs& a);
 int launch_scan_simt(const ScanArgs& a, cudaStream_t s);
 
-// Device status word of the decode step (one per device, sticky until read).
+// Device status words of the entry points without a workspace (one per device
+// and kernel file, sticky until read): the decode step and the MIMO projections.
 int decode_status_read_and_clear(int* code);
+int proj_status_read_and_clear(int* code);
+
+// MIMO rank-R projections (mimo_proj.cu): up u [T, H, P] -> x [T, H, R, P] with
+// Wx [H, R P, P]; down y [T, H, R, P] -> out [T, H, P] with Wy [H, P, R P], then
+// (z non-null) the RMS norm over P with weight w [H, P] (nullable) and the silu
+// gate.  bf16, P = 64, R in {1, 2, 4}.
+struct ProjArgs {
+  long long tokens;
+  int nheads, R, up;
+  const void *in, *weight;
+  void* out;
+  const void* z;
+  const float* w;
+  float eps;
+  long long wait_limit;
+  int test_withhold;
+};
+int launch_mimo_proj(const ProjArgs& a, cudaStream_t s);
 
 // TMA tensor maps over the prefill's inputs (scan_tc.cu): a [batch, L, heads, R,
 // inner] bf16 tensor with box {64, R, 1, Q, 1} and 128-byte swizzle; dt or lam
 // [batch, L, H] with box {8, rows, 1}; theta [batch, L, H, N/2] with box
 // {N/2, 1, Q, 1}.  Each returns false when the driver rejects the map.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn();  // cuTensorMapEncodeTiled from the driver, or null
 bool make_map(CUtensorMap* m, const void* base, int inner, int heads, const ScanArgs& a, int Q);
 bool make_dl_map(CUtensorMap* m, const void* base, const ScanArgs& a, int rows);
 bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q);
+
+// Long sequences with few (batch, head) units (scan_seg.cu): segments per unit
+// (0 = run unsegmented), the workspace they need after the status word, and the
+// segmented prefill; launch_state_export (scan_bwd_tc.cu) gives every
+// sequence's end state from a zero state, the segments' aggregates.
+constexpr int kSMs = 148;
+int seg_count(const ScanArgs& a, int sms);
+size_t seg_workspace_bytes(const ScanArgs& a, int S);
+int launch_scan_segmented(const ScanArgs& a, int S, cudaStream_t s);
+int launch_state_export(const ScanArgs& a, cudaStream_t s);
 
 int tc_scan_supported(const ScanArgs& a);
 int launch_scan_tc(const ScanArgs& a, cudaStream_t s);

@@ -16,6 +16,7 @@ constexpr size_t kStatusBytes = 256;
 constexpr long long kDefaultWaitLimit = 4000000000LL;  // SM cycles, about 2 s at 1.9 GHz
 volatile long long g_wait_limit = kDefaultWaitLimit;
 volatile int g_test_withhold = 0;
+volatile int g_test_segments = 0;  // mamba3_test_set_segments: 0 = the library's choice
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -60,6 +61,16 @@ int check_inputs(const void* x, const void* B, const void* C, const void* theta,
 bool norm_ok(const mamba3_bc_norm* n) {
   if (!n || !(n->eps >= 0.f)) return false;
   return aligned4(n->w_B) && aligned4(n->w_C) && aligned4(n->bias_B) && aligned4(n->bias_C);
+}
+
+// mamba3_test_set_segments: S when it divides seqlen and the shape has the
+// segmented path, else 0
+int forced_segments(const m3::ScanArgs& a) {
+  const int S = g_test_segments;
+  if (S < 2 || a.seqlen % S != 0 || m3::tc_scan_supported(a) != MAMBA3_OK || m3::bwd_tc_supported(a) != MAMBA3_OK ||
+      a.bcnorm)
+    return 0;
+  return S;
 }
 
 template <typename Args>
@@ -148,6 +159,11 @@ int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
+  if (use_tc) {  // a long sequence over few units runs in segments when the workspace allows it
+    const int S = g_test_segments ? forced_segments(a) : m3::seg_count(a, m3::kSMs);
+    if (S > 0 && workspace_bytes >= kStatusBytes + m3::seg_workspace_bytes(a, S))
+      return m3::launch_scan_segmented(a, S, s);
+  }
   return use_tc ? m3::launch_scan_tc(a, s) : m3::launch_scan_simt(a, s);
 }
 
@@ -229,11 +245,50 @@ int mamba3_decode_step(const mamba3_dims* d, const mamba3_state* state, const vo
   return decode_impl(d, state, x, B, C, theta, dt, lam, A, nullptr, D, nullptr, y, stream);
 }
 
-int mamba3_decode_status(void* stream) {
+int mamba3_library_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MAMBA3_ERR_CUDA;
-  int code = 0;
-  const int rc = m3::decode_status_read_and_clear(&code);
-  return rc != MAMBA3_OK ? rc : code;
+  int dec = 0, proj = 0;
+  int rc = m3::decode_status_read_and_clear(&dec);
+  if (rc == MAMBA3_OK) rc = m3::proj_status_read_and_clear(&proj);
+  if (rc != MAMBA3_OK) return rc;
+  return dec != 0 ? dec : proj;
+}
+
+namespace {
+int mimo_proj_impl(const mamba3_dims* d, int up, const void* in, const void* weight, const void* z, const float* w,
+                   float eps, void* out, void* stream) {
+  if (!d || d->batch < 1 || d->seqlen < 0 || d->nheads < 1) return MAMBA3_ERR_INVALID;
+  if (!(d->rank == 1 || d->rank == 2 || d->rank == 4 || d->rank == 8)) return MAMBA3_ERR_INVALID;
+  if (d->in_dtype != MAMBA3_F32 && d->in_dtype != MAMBA3_BF16) return MAMBA3_ERR_INVALID;
+  if (!(eps >= 0.f)) return MAMBA3_ERR_INVALID;
+  const double tokens = (double)d->batch * d->seqlen;
+  if (tokens * d->nheads * d->rank * d->headdim > 9.0e15 || tokens > 2.0e9) return MAMBA3_ERR_INVALID;
+  if (d->in_dtype != MAMBA3_BF16 || d->headdim != 64 || d->rank == 8) return MAMBA3_ERR_UNSUPPORTED;
+  if (tokens > 0) {
+    if (!in || !weight || !out || !aligned16(in) || !aligned16(weight) || !aligned16(out)) return MAMBA3_ERR_INVALID;
+    if (z && !aligned16(z)) return MAMBA3_ERR_INVALID;
+    if (w && !aligned4(w)) return MAMBA3_ERR_INVALID;
+  }
+  m3::ProjArgs a;
+  memset(&a, 0, sizeof(a));
+  a.tokens = (long long)d->batch * d->seqlen;
+  a.nheads = d->nheads;
+  a.R = d->rank;
+  a.up = up;
+  a.in = in; a.weight = weight; a.out = out; a.z = z; a.w = w; a.eps = eps;
+  a.wait_limit = g_wait_limit;
+  a.test_withhold = g_test_withhold;
+  return m3::launch_mimo_proj(a, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+int mamba3_mimo_up(const mamba3_dims* d, const void* u, const void* Wx, void* x, void* stream) {
+  return mimo_proj_impl(d, 1, u, Wx, nullptr, nullptr, 0.f, x, stream);
+}
+
+int mamba3_mimo_down(const mamba3_dims* d, const void* y, const void* Wy, const void* z, const float* w, float eps,
+                     void* out, void* stream) {
+  return mimo_proj_impl(d, 0, y, Wy, z, w, eps, out, stream);
 }
 
 int mamba3_set_wait_limit(long long cycles) {
@@ -244,6 +299,19 @@ int mamba3_set_wait_limit(long long cycles) {
 
 int mamba3_test_withhold_loads(int on) {
   g_test_withhold = on ? 1 : 0;
+  return MAMBA3_OK;
+}
+
+size_t mamba3_scan_segmented_workspace_bytes(const mamba3_dims* d) {
+  if (check_dims(d, true) != MAMBA3_OK) return 0;
+  m3::ScanArgs a = scan_args(d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  const int S = g_test_segments ? forced_segments(a) : m3::seg_count(a, m3::kSMs);
+  return kStatusBytes + m3::seg_workspace_bytes(a, S);
+}
+
+int mamba3_test_set_segments(int S) {
+  if (S < 0) return MAMBA3_ERR_INVALID;
+  g_test_segments = S;
   return MAMBA3_OK;
 }
 

@@ -1,0 +1,223 @@
+// Long single sequences with few (batch, head) units: the prefill split into S
+// segments per unit, so that S times as many CTAs share the GPU.
+//
+// The state is constant in size and the cost linear in the sequence length
+// ("Mamba-3 paper review" (no1joon.github.io), Table 7 discussion), and the
+// rotation angles are sums over time steps ("Mamba-3: 2x smaller state ..."
+// (MarkTechPost, Korean translation), section 1.2), so a segment's effect on
+// the state is a decay, a rotation and an additive term:
+//   1. launch_state_export: every segment's end state from a zero state and a
+//      zero angle (h_loc, the rotated B and the x of its last token, its angle
+//      sum Phi_loc), on the sequence viewed as batch b S of length L / S;
+//   2. seg_combine_kernel: per unit, in segment order, the state entering
+//      segment s + 1 from the one entering segment s (frame rotated by -Phi_in):
+//        h     = e^{sum_seg dt A} (h_in + (1 - lam_f) dt_f sum_r b_in[r] x_in[r]^T)
+//                + rot(-Phi_in) h_loc
+//        b_prev = rot(-Phi_in) b_loc,  x_prev = x_loc,  Phi = wrap(Phi_in + Phi_loc)
+//      (f = the segment's first token; rot acts on the (2k, 2k+1) pairs of the
+//      state dimension), written as the initial states of the segments and, for
+//      the last one, as the exported final state;
+//   3. the tensor-core prefill on the b S segments from those initial states.
+// Passes 1 and 3 both read B, x, theta, dt, lam: the price of the parallelism.
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace m3 {
+namespace {
+
+constexpr int kThreads = 256;
+
+struct SegParams {
+  ScanArgs a;        // the unsegmented problem (its init and final state, inputs)
+  int S, Ls;         // segments per unit and their length
+  const float *loc_h, *loc_b, *loc_x, *loc_ang;  // [b S, H, ...] segment aggregates
+  float *in_h, *in_b, *in_x, *in_ang;            // [b S, H, ...] initial state of every segment
+};
+
+template <typename T>
+__device__ __forceinline__ float ldv(const void* p, size_t i) {
+  return ld1(static_cast<const T*>(p) + i);
+}
+
+// One CTA per unit (b, h); the running state lives in shared memory.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) seg_combine_kernel(const SegParams sp) {
+  extern __shared__ float sm[];
+  const ScanArgs& a = sp.a;
+  const int N = a.N, P = a.P, R = a.R, K2 = N / 2, NP = N * P;
+  const int H = a.nheads, L = a.seqlen, S = sp.S, Ls = sp.Ls;
+  const int unit = blockIdx.x, b = unit / H, hh = unit % H;
+  const int tid = threadIdx.x;
+  float* h = sm;               // [N][P]
+  float* bp = h + NP;          // [R][N]
+  float* xp = bp + R * N;      // [R][P]
+  float* ang = xp + R * P;     // [K2]
+  float* red = ang + K2;       // [S] decay sums, then scratch
+  __shared__ float warp_part[kThreads / 32];
+  const size_t us = (size_t)unit;
+
+  // the sum of dt * A over every segment (a block reduction per segment)
+  for (int s = 0; s < S; ++s) {
+    float v = 0.f;
+    for (int t = s * Ls + tid; t < (s + 1) * Ls; t += kThreads) {
+      const size_t i = ((size_t)b * L + t) * H + hh;
+      const float rate = a.A_t ? ldv<T>(a.A_t, i) : a.A[hh];
+      v += ldv<T>(a.dt, i) * rate;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((tid & 31) == 0) warp_part[tid >> 5] = v;
+    __syncthreads();
+    if (tid == 0) {
+      float tot = 0.f;
+      for (int w = 0; w < kThreads / 32; ++w) tot += warp_part[w];
+      red[s] = tot;
+    }
+    __syncthreads();
+  }
+  // the state entering segment 0: the caller's initial state, or zero
+  for (int i = tid; i < NP; i += kThreads) h[i] = a.h0 ? a.h0[us * NP + i] : 0.f;
+  for (int i = tid; i < R * N; i += kThreads) bp[i] = a.bprev0 ? a.bprev0[us * R * N + i] : 0.f;
+  for (int i = tid; i < R * P; i += kThreads) xp[i] = a.xprev0 ? a.xprev0[us * R * P + i] : 0.f;
+  for (int i = tid; i < K2; i += kThreads) ang[i] = a.angle0 ? a.angle0[us * K2 + i] : 0.f;
+  __syncthreads();
+
+  for (int s = 0; s < S; ++s) {
+    const size_t su = ((size_t)b * S + s) * H + hh;  // the segment's unit in the b S x H view
+    // the initial state of segment s
+    for (int i = tid; i < NP; i += kThreads) sp.in_h[su * NP + i] = h[i];
+    for (int i = tid; i < R * N; i += kThreads) sp.in_b[su * R * N + i] = bp[i];
+    for (int i = tid; i < R * P; i += kThreads) sp.in_x[su * R * P + i] = xp[i];
+    for (int i = tid; i < K2; i += kThreads) sp.in_ang[su * K2 + i] = ang[i];
+    // the state leaving it
+    const size_t f = ((size_t)b * L + (size_t)s * Ls) * H + hh;  // its first token
+    const float mu = (1.f - ldv<T>(a.lam, f)) * ldv<T>(a.dt, f);
+    const float decay = expf(red[s]);
+    const float* lh = sp.loc_h + su * NP;
+    for (int i = tid; i < NP / 2; i += kThreads) {  // one (pair k, column p) per step
+      const int k = i / P, p = i % P;
+      float sn, cs;
+      sincosf(ang[k], &sn, &cs);
+      float c0 = h[(2 * k) * P + p], c1 = h[(2 * k + 1) * P + p];
+      for (int r = 0; r < R; ++r) {
+        const float xr = mu * xp[r * P + p];
+        c0 += bp[r * N + 2 * k] * xr;
+        c1 += bp[r * N + 2 * k + 1] * xr;
+      }
+      const float l0 = lh[(2 * k) * P + p], l1 = lh[(2 * k + 1) * P + p];
+      h[(2 * k) * P + p] = decay * c0 + cs * l0 + sn * l1;
+      h[(2 * k + 1) * P + p] = decay * c1 + cs * l1 - sn * l0;
+    }
+    __syncthreads();  // every thread has read bp, xp, ang of the entering state
+    for (int i = tid; i < R * K2; i += kThreads) {
+      const int r = i / K2, k = i % K2;
+      float sn, cs;
+      sincosf(ang[k], &sn, &cs);
+      const float l0 = sp.loc_b[su * R * N + r * N + 2 * k], l1 = sp.loc_b[su * R * N + r * N + 2 * k + 1];
+      bp[r * N + 2 * k] = cs * l0 + sn * l1;
+      bp[r * N + 2 * k + 1] = cs * l1 - sn * l0;
+    }
+    for (int i = tid; i < R * P; i += kThreads) xp[i] = sp.loc_x[su * R * P + i];
+    __syncthreads();  // bp rotated with the entering angle before it moves on
+    for (int i = tid; i < K2; i += kThreads) ang[i] = wrap_angle(ang[i] + sp.loc_ang[su * K2 + i]);
+    __syncthreads();
+  }
+  if (a.h_out) {  // the state after the whole sequence
+    for (int i = tid; i < NP; i += kThreads) a.h_out[us * NP + i] = h[i];
+    for (int i = tid; i < R * N; i += kThreads) a.bprev_out[us * R * N + i] = bp[i];
+    for (int i = tid; i < R * P; i += kThreads) a.xprev_out[us * R * P + i] = xp[i];
+    for (int i = tid; i < K2; i += kThreads) a.angle_out[us * K2 + i] = ang[i];
+  }
+}
+
+// per (b S x H) unit: h, b_prev, x_prev, angle (floats)
+size_t seg_state_floats(const ScanArgs& a) {
+  return (size_t)a.N * a.P + (size_t)a.R * a.N + (size_t)a.R * a.P + (size_t)a.N / 2;
+}
+
+}  // namespace
+
+// Segments per unit for `a`, or 0 when the plain prefill is the better choice:
+// only the tensor-core shapes, long sequences (at least 1024 tokens per
+// segment) and fewer units than SMs; S divides L and is chosen so that the b S H
+// CTAs fill the SMs' waves as evenly as possible.
+int seg_count(const ScanArgs& a, int sms) {
+  if (tc_scan_supported(a) != MAMBA3_OK || bwd_tc_supported(a) != MAMBA3_OK || a.bcnorm) return 0;
+  const long long units = (long long)a.batch * a.nheads;
+  if (units >= sms || a.seqlen < 2048) return 0;
+  int best = 0;
+  double best_eff = 0.0;
+  for (int S = 2; S <= 64; S *= 2) {
+    if (a.seqlen % S != 0 || a.seqlen / S < 1024) break;
+    const long long ctas = units * S;
+    const double waves = (double)ctas / sms;
+    const double eff = waves / (double)((ctas + sms - 1) / sms);
+    if (ctas >= sms && eff > best_eff + 1e-9) {
+      best = S;
+      best_eff = eff;
+    }
+  }
+  return best;
+}
+
+size_t seg_workspace_bytes(const ScanArgs& a, int S) {
+  if (S <= 0) return 0;
+  return 2 * (size_t)a.batch * S * a.nheads * seg_state_floats(a) * sizeof(float);
+}
+
+// The prefill of `a` in S segments (workspace: the status word, then the segment
+// aggregates and the segments' initial states).
+int launch_scan_segmented(const ScanArgs& a, int S, cudaStream_t s) {
+  const size_t per = seg_state_floats(a);
+  const size_t units_s = (size_t)a.batch * S * a.nheads;
+  float* loc = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + 256);
+  float* ini = loc + units_s * per;
+  SegParams sp;
+  memset(&sp, 0, sizeof(sp));
+  sp.a = a;
+  sp.S = S;
+  sp.Ls = a.seqlen / S;
+  // [b S H] arrays of each field, one after the other
+  sp.loc_h = loc;
+  sp.loc_b = loc + units_s * a.N * a.P;
+  sp.loc_x = sp.loc_b + units_s * a.R * a.N;
+  sp.loc_ang = sp.loc_x + units_s * a.R * a.P;
+  sp.in_h = ini;
+  sp.in_b = ini + units_s * a.N * a.P;
+  sp.in_x = sp.in_b + units_s * a.R * a.N;
+  sp.in_ang = sp.in_x + units_s * a.R * a.P;
+
+  // 1. segment aggregates
+  ScanArgs a1 = a;
+  a1.batch = a.batch * S;
+  a1.seqlen = sp.Ls;
+  a1.h0 = a1.bprev0 = a1.xprev0 = a1.angle0 = nullptr;
+  a1.h_out = const_cast<float*>(sp.loc_h);
+  a1.bprev_out = const_cast<float*>(sp.loc_b);
+  a1.xprev_out = const_cast<float*>(sp.loc_x);
+  a1.angle_out = const_cast<float*>(sp.loc_ang);
+  a1.y = nullptr;
+  int rc = launch_state_export(a1, s);
+  if (rc != MAMBA3_OK) return rc;
+  // 2. the segments' initial states (and the final state)
+  const size_t smem = (per + S) * sizeof(float);
+  auto kc = a.dtype == MAMBA3_F32 ? seg_combine_kernel<float> : seg_combine_kernel<__nv_bfloat16>;
+  if (smem > 48 * 1024 && cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MAMBA3_ERR_CUDA;
+  kc<<<a.batch * a.nheads, kThreads, smem, s>>>(sp);
+  if (cudaGetLastError() != cudaSuccess) return MAMBA3_ERR_CUDA;
+  // 3. the prefill of every segment from its initial state
+  ScanArgs a3 = a;
+  a3.batch = a.batch * S;
+  a3.seqlen = sp.Ls;
+  a3.h0 = sp.in_h;
+  a3.bprev0 = sp.in_b;
+  a3.xprev0 = sp.in_x;
+  a3.angle0 = sp.in_ang;
+  a3.h_out = a3.bprev_out = a3.xprev_out = a3.angle_out = nullptr;
+  return launch_scan_tc(a3, s);
+}
+
+}  // namespace m3

@@ -307,3 +307,32 @@ def test_backward_time_varying_decay_host_validation(lib):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_backward_time_varying_decay_valid_call_without_device(lib):
     assert bwd_at(lib, dims()) == m3.MAMBA3_ERR_CUDA
+
+
+def proj_up(lib, d, u=FAKE, W=FAKE, x=FAKE):
+    return lib.mamba3_mimo_up(ctypes.byref(d), u, W, x, None)
+
+
+def proj_down(lib, d, y=FAKE, W=FAKE, z=None, w=None, eps=1e-6, out=FAKE):
+    return lib.mamba3_mimo_down(ctypes.byref(d), y, W, z, w, eps, out, None)
+
+
+def test_mimo_projection_host_validation(lib):
+    d = dims(rank=4, headdim=64)
+    assert proj_up(lib, d, u=None) == m3.MAMBA3_ERR_INVALID
+    assert proj_up(lib, d, x=FAKE + 8) == m3.MAMBA3_ERR_INVALID
+    assert proj_down(lib, d, W=None) == m3.MAMBA3_ERR_INVALID
+    assert proj_down(lib, d, z=FAKE + 8) == m3.MAMBA3_ERR_INVALID
+    assert proj_down(lib, d, w=FAKE + 2, z=FAKE) == m3.MAMBA3_ERR_INVALID
+    assert proj_down(lib, d, eps=-1.0) == m3.MAMBA3_ERR_INVALID
+    assert proj_up(lib, dims(rank=3, headdim=64)) == m3.MAMBA3_ERR_INVALID
+    assert proj_up(lib, dims(rank=4, headdim=32)) == m3.MAMBA3_ERR_UNSUPPORTED
+    assert proj_up(lib, dims(rank=8, headdim=64)) == m3.MAMBA3_ERR_UNSUPPORTED
+    assert proj_down(lib, dims(rank=4, headdim=64, in_dtype=m3.MAMBA3_F32)) == m3.MAMBA3_ERR_UNSUPPORTED
+    assert proj_up(lib, dims(rank=4, headdim=64, seqlen=0), u=None, W=None, x=None) == m3.MAMBA3_OK  # nothing to do
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_mimo_projection_valid_call_without_device_is_a_cuda_error(lib):
+    assert proj_up(lib, dims(rank=4, headdim=64)) == m3.MAMBA3_ERR_CUDA
+    assert proj_down(lib, dims(rank=2, headdim=64), z=FAKE, w=FAKE) == m3.MAMBA3_ERR_CUDA

@@ -43,3 +43,11 @@ def test_traffic_is_null_when_sources_change(monkeypatch):
     assert bench.traffic(key) is None
     monkeypatch.setitem(bench.TRAFFIC, key, (files, bench.sources_sha(files), nbytes, cite))
     assert bench.traffic(key) == nbytes
+
+
+def test_mimo_proj_bytes():
+    w = wl.CONFIGS["mimo4_prefill_b4_l8192"]
+    th = 4 * 8192 * 64
+    wts = 2 * 64 * 4 * 64 * 64
+    # up: u (128 B) read, x (512 B) written per token-head; down: y (512 B), z (128 B) read, out (128 B) written
+    assert bench.mimo_proj_bytes(w) == {"up": th * 640 + wts, "down_gated": th * 768 + wts + 4 * 64 * 64}

@@ -60,13 +60,13 @@ def test_decode_timeout_is_reported_and_context_survives():
     pre = small_inputs(b, 1, H, P, N, R, torch.bfloat16, seed=5200)
     st = m3.State.zeros(b, H, P, N, R, device="cuda")
     step = {n: pre[n][:, 0].contiguous() for n in NAMES}
-    assert m3.mamba3_decode_status() == m3.MAMBA3_OK
+    assert m3.mamba3_library_status() == m3.MAMBA3_OK
     _starved(lambda: m3.mamba3_decode_step(st, *(step[n] for n in NAMES), pre["A"], pre["D"]))
-    assert m3.mamba3_decode_status() == m3.MAMBA3_ERR_TIMEOUT
-    assert m3.mamba3_decode_status() == m3.MAMBA3_OK  # read and cleared
+    assert m3.mamba3_library_status() == m3.MAMBA3_ERR_TIMEOUT
+    assert m3.mamba3_library_status() == m3.MAMBA3_OK  # read and cleared
     # a normal step from a fresh zero state equals the one-token prefill
     st = m3.State.zeros(b, H, P, N, R, device="cuda")
     y = m3.mamba3_decode_step(st, *(step[n] for n in NAMES), pre["A"], pre["D"])
-    assert m3.mamba3_decode_status() == m3.MAMBA3_OK
+    assert m3.mamba3_library_status() == m3.MAMBA3_OK
     yr, _ = oracle_scan(pre)
     assert rel_err(y.float().cpu().double().numpy(), yr[:, 0]) < TOL[torch.bfloat16]
