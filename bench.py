@@ -36,7 +36,7 @@ PREFILL_MORE = [wl.CONFIGS["mimo4_prefill_b4_l8192"], wl.CONFIGS["mimo4_long_b1_
 # batch-1 decode after the 65536-token MIMO prefill: latency-bound (2.5 MB per step)
 DECODE_LONG = wl.CONFIGS["mimo4_long_b1_l65536"].with_(prefill_tokens=65536)
 FALLBACK_HBM_GBS = 6650.0
-BACKWARD_KERNEL = "scan_bwd_kernel (SIMT, fp32)"
+BACKWARD_KERNEL = "bwd_state_kernel + bwd_chunk_kernel (tcgen05, TMA)"
 
 # DRAM bytes (read + write) per launch from ncu captures of the kernels as they
 # stand: (kernel source files, sha256 of their concatenation, bytes per launch,
@@ -346,7 +346,8 @@ def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False,
     y = torch.empty_like(inp["x"])
     fin = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
     dims = m3.make_dims(inp["x"], inp["B"])
-    ws = torch.zeros(max(256, m3.mamba3_scan_workspace_bytes(dims)), dtype=torch.uint8, device=dev)
+    # the workspace size with which a long sequence over few units runs in segments
+    ws = torch.zeros(max(256, m3.mamba3_scan_segmented_workspace_bytes(dims)), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def launch():
@@ -599,8 +600,10 @@ def ours(args):
     more = {}
     for w in PREFILL_MORE:
         ms = max_over_ranks(run_prefill_plain(m3, w, rank, steps=side_steps, warmup=3), world)
+        dims = m3.Dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.rank, 0, m3.MAMBA3_BF16, 0)
+        segmented = m3.mamba3_scan_segmented_workspace_bytes(dims) > m3.mamba3_scan_workspace_bytes(dims)
         more[w.name] = {"ms": round(ms, 4), "mtokens_s": round(w.batch * w.seqlen / (ms * 1e-3) / 1e6, 3),
-                        **rl(prefill_bytes(w), ms, peak)}
+                        "segmented": segmented, **rl(prefill_bytes(w), ms, peak)}
     clk.stop()
     clocks = clk.summary()
     clocks["window"] = "headline prefill timed steps through the last side measurement"
