@@ -46,15 +46,17 @@ def run_both(inp, dy, init=None, d_final=None):
     return gr, ref
 
 
-def check(gr, ref, tol, with_state=True):
+def check(gr, ref, tol, with_state=True, dt=None):
     errs = {n: rel_err(np64(gr[n]), ref[n]) for n in GRADS}
     if with_state:
         for n, gn in STATE:
             errs[gn] = rel_err(np64(getattr(gr["d_init"], n)), ref[gn])
-        # from a zero state the initial angle's gradient vanishes (y sees only angle
-        # differences); measure it on the scale of the other angle gradients
+        # From a zero state the initial angle's gradient vanishes (y sees only angle
+        # differences), so measure it on the scale of the angle-gradient sums it is
+        # one of: S_t = dtheta_t / dt_t (dtheta carries the factor dt, dangle0 none).
         d = np.abs(np64(gr["d_init"].angle) - ref["dangle0"]).max()
-        errs["dangle0"] = float(d / max(np.abs(ref["dangle0"]).max(), np.abs(ref["dtheta"]).max()))
+        sums = np.abs(ref["dtheta"] / dt[..., None]).max() if dt is not None else np.abs(ref["dtheta"]).max()
+        errs["dangle0"] = float(d / max(np.abs(ref["dangle0"]).max(), sums))
     bad = {k: v for k, v in errs.items() if not v < tol}
     assert not bad, (bad, errs)
 
@@ -82,7 +84,7 @@ def test_backward_matches_oracle(shape, dtype, with_state):
     init = rand_state(b, H, P, N, R, 2400 + L) if with_state else None
     d_final = rand_state(b, H, P, N, R, 2500 + L) if with_state else None
     gr, ref = run_both(inp, dy, init, d_final)
-    check(gr, ref, TOL[dtype])
+    check(gr, ref, TOL[dtype], dt=np64(inp["dt"]))
 
 
 @pytest.mark.parametrize("L", [1, 2, 31, 32, 33])
