@@ -44,20 +44,23 @@ BACKWARD_KERNEL = "bwd_state_kernel + bwd_chunk_kernel (tcgen05, TMA)"
 # traffic null, since its counters are out of date.
 TRAFFIC = {
     "prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"),
-                "d553b6c25b666d8f4a80634013f03686f468b3f560dcd4cc96708923e1c92176", 811524352 + 136936960,
+                "8c7315685dc21c6b771e1d8a843e5fbc2fbd942e638f9df041ae26dd4adc3a9a", 811532288 + 137174784,
                 "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "mimo4_prefill_b4_l8192": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"),
+                               "8c7315685dc21c6b771e1d8a843e5fbc2fbd942e638f9df041ae26dd4adc3a9a",
+                               5648189440 + 1064534272, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     "siso_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                         "7ccbdf6b735872e61661a0e4d8ad33ec2f120e42692c1cc6ce802987011c2987", 283237376 + 220529664,
+                         "33d2df3c2627df690ecd8bd830abc94739f24a010222682500fc194bcbbee128", 283179520 + 219435264,
                          "profiles/decode_stream_b128_traffic_and_counters.txt"),
     "mimo4_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                          "7ccbdf6b735872e61661a0e4d8ad33ec2f120e42692c1cc6ce802987011c2987", 317788672 + 239549184,
+                          "33d2df3c2627df690ecd8bd830abc94739f24a010222682500fc194bcbbee128", 317792000 + 240657408,
                           "profiles/decode_stream_b128_traffic_and_counters.txt"),
-    "grouped_prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"), "d553b6c25b666d8f4a80634013f03686f468b3f560dcd4cc96708923e1c92176", 284591616 + 113454080,
+    "grouped_prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"), None, None,
                         "profiles/grouped_bc_prefill_decode_traffic.txt"),
-    "grouped_decode": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), "7ccbdf6b735872e61661a0e4d8ad33ec2f120e42692c1cc6ce802987011c2987", 279056128 + 219058176,
+    "grouped_decode": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), None, None,
                        "profiles/grouped_bc_prefill_decode_traffic.txt"),
-    "backward": (("scan_bwd.cu", "common.cuh"), "cfca736f5dd9e50ceaf7e528b3eed4f8a06f38efcfde4246e604a60514bcf42f", 2366348288 + 1885662208,
-                 "profiles/scan_bwd_siso_b8_l2048_traffic_and_counters.txt"),
+    "backward": (("scan_bwd_tc.cu", "sm100_ptx.cuh", "common.cuh"), None, None,
+                 "profiles/scan_bwd_tc_siso_b8_l2048_traffic_and_counters.txt"),
     "gated_norm_per_head": (("gated_norm.cu", "common.cuh"), "eb90ad7d72a2607cc062684461d599cc86e5eea7058c9d970afd24eac530e380", 268479232 + 103046400,
                             "profiles/gated_norm_b8_l2048_traffic_and_counters.txt"),
 }
@@ -603,7 +606,8 @@ def ours(args):
         dims = m3.Dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.rank, 0, m3.MAMBA3_BF16, 0)
         segmented = m3.mamba3_scan_segmented_workspace_bytes(dims) > m3.mamba3_scan_workspace_bytes(dims)
         more[w.name] = {"ms": round(ms, 4), "mtokens_s": round(w.batch * w.seqlen / (ms * 1e-3) / 1e6, 3),
-                        "segmented": segmented, **rl(prefill_bytes(w), ms, peak)}
+                        "segmented": segmented,
+                        **rl(prefill_bytes(w), ms, peak, traffic(w.name) if w.name in TRAFFIC else None)}
     clk.stop()
     clocks = clk.summary()
     clocks["window"] = "headline prefill timed steps through the last side measurement"

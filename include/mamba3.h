@@ -206,13 +206,22 @@ MAMBA3_API int mamba3_decode_step_at(const mamba3_dims* dims, const mamba3_state
  *                 overwritten (zeroed on `stream`, then accumulated).  dD nullable.
  *   d_init        nullable: float32 gradients of the four initial-state fields
  *                 (with init NULL, those of a zero initial state).
- *   workspace     at least mamba3_scan_bwd_workspace_bytes(dims): the state at
- *                 every chunk start, kept between the forward and the reverse
- *                 sweep (batch * nheads * ceil(seqlen / Q) * (N P + N/2) floats,
- *                 Q = 32 / rank), after the 256-byte status word; with grouped
- *                 B/C also 2 * batch * seqlen * nheads * rank * dstate floats.
- * Computed in float32 whatever in_dtype is.  Returns MAMBA3_ERR_UNSUPPORTED for
- * N, P whose per-chunk tiles exceed shared memory.
+ *   workspace     at least mamba3_scan_bwd_workspace_bytes(dims), after the
+ *                 256-byte status word: the state at every chunk start, kept
+ *                 between the forward state march and the reverse sweep.
+ *                 Tensor-core path (bf16, P = 64, N in {64, 128}, R in {1, 2, 4},
+ *                 seqlen >= 1): per (b, h) and 64-row chunk (Q = 64 / rank tokens)
+ *                 a bf16 N x P tile and N/2 float angles, i.e.
+ *                 batch * nheads * ceil(seqlen / Q) * (128 N + 2 N) bytes (SISO
+ *                 b8 L2048 H64 N128: 272 MB); with grouped B/C then the fp32 sums
+ *                 of dB and dC, 2 * batch * seqlen * ngroups * rank * dstate
+ *                 floats.  Other shapes (SIMT path): per (b, h) and chunk of
+ *                 Q = 32 / rank tokens, N P + N/2 floats; with grouped B/C
+ *                 2 * batch * seqlen * nheads * rank * dstate floats of per-head
+ *                 gradients.
+ * Products on the tensor cores take bf16 operands with float32 accumulation;
+ * everything else is float32.  Returns MAMBA3_ERR_UNSUPPORTED for N, P whose
+ * per-chunk tiles exceed shared memory.
  * mamba3_scan_bwd_at is the same for mamba3_scan_fwd_at: A_t [b, L, H] (dtype of x)
  * in place of A, and dA_t (layout and dtype of A_t, not nullable) in place of dA.
  */

@@ -28,6 +28,7 @@ struct ScanArgs {
   // bounded device waits: give up after about this many SM cycles (mamba3_set_wait_limit)
   long long wait_limit;
   int test_withhold;  // testing the timeout path only: issue no input loads
+  float* decay_out;   // segment aggregates: sum of dt * A over each sequence [b, H], or null
 };
 
 struct DecodeArgs {
@@ -137,6 +138,8 @@ int seg_count(const ScanArgs& a, int sms);
 size_t seg_workspace_bytes(const ScanArgs& a, int S);
 int launch_scan_segmented(const ScanArgs& a, int S, cudaStream_t s);
 int launch_state_export(const ScanArgs& a, cudaStream_t s);
+// The same end states as one streaming tensor-core reduction per sequence (seg_state.cu).
+int launch_seg_state(const ScanArgs& a, cudaStream_t s);
 
 int tc_scan_supported(const ScanArgs& a);
 int launch_scan_tc(const ScanArgs& a, cudaStream_t s);

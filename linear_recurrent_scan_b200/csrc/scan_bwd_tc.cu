@@ -455,8 +455,9 @@ struct CCfg : BCfg<N, R> {
   static constexpr int OFF_G = OFF_XW + kBlk;             // G (bf16 state tile)
   static constexpr int OFF_S = OFF_G + B::HB_BYTES;       // S, then W; later the angle gradients [Q][K2] f32
   static constexpr int OFF_W = OFF_S + kBlk;
-  static constexpr int OFF_PHT = OFF_W + kBlk;            // angle of every token [Q][K2] f32
-  static constexpr int OFF_SC = OFF_PHT + B::Q * B::K2 * 4;
+  static constexpr int QP = B::Q + 1;                     // odd row stride of the angle table
+  static constexpr int OFF_PHT = OFF_W + kBlk;            // angle of every token [K2][QP] f32
+  static constexpr int OFF_SC = OFF_PHT + B::K2 * QP * 4;
   static constexpr int PART_FLOATS = (NPA > NPART2 ? NPA : NPART2) * B::K2;
   static constexpr int OFF_PART = OFF_SC + kNScal * kScalStride * 4;
   static constexpr int OFF_SANG = OFF_PART + PART_FLOATS * 4;  // angle gradient from the end [K2]
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
                      const __grid_constant__ CUtensorMap tmT, const BwdArgs g, const uint8_t* ckpt, int nchunks) {
   using K = CCfg<N, R>;
   constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, NPA = K::NPA, TPP = K::TPP, NKB = K::NKB;
-  constexpr int NPART2 = K::NPART2, TPP2 = K::TPP2;
+  constexpr int NPART2 = K::NPART2, TPP2 = K::TPP2, QP = K::QP;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -499,8 +500,12 @@ __global__ void __launch_bounds__(kCThreads, 1)
   float* part_sum = reinterpret_cast<float*>(smem + K::OFF_PART);
   float* sang = reinterpret_cast<float*>(smem + K::OFF_SANG);
   float* red = reinterpret_cast<float*>(smem + K::OFF_RED);
-  float* pht = reinterpret_cast<float*>(smem + K::OFF_PHT);
+  float* pht = reinterpret_cast<float*>(smem + K::OFF_PHT);  // [K2][QP]: consecutive tokens, consecutive banks
   float* dphi_s = reinterpret_cast<float*>(smem + K::OFF_S);
+  // angle gradient of (token t, pair k): rows of K2, the pairs XOR-swizzled in groups of
+  // four by the row, so that the 16 rows a warp stores at once fall in different banks
+  // and a row read by 32 consecutive pairs stays conflict-free
+  auto dphi_at = [](int t, int k) { return t * K::K2 + (k ^ ((t & 7) << 2)); };
   const __nv_bfloat16* DT = static_cast<const __nv_bfloat16*>(a.dt);
   const __nv_bfloat16* LM = static_cast<const __nv_bfloat16*>(a.lam);
   const __nv_bfloat16* AT = static_cast<const __nv_bfloat16*>(a.A_t);
@@ -701,8 +706,8 @@ __global__ void __launch_bounds__(kCThreads, 1)
         const uint2 tv = *reinterpret_cast<const uint2*>(th + t * K2 + 4 * ag);
         const float2 t01 = unpack_bf16(tv.x), t23 = unpack_bf16(tv.y);
         run[0] += d * t01.x; run[1] += d * t01.y; run[2] += d * t23.x; run[3] += d * t23.y;
-        *reinterpret_cast<float4*>(pht + t * K2 + 4 * ag) =
-            make_float4(wrap_angle(run[0]), wrap_angle(run[1]), wrap_angle(run[2]), wrap_angle(run[3]));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) pht[(4 * ag + k) * QP + t] = wrap_angle(run[k]);
         float sn[4], cs[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) __sincosf(run[k], &sn[k], &cs[k]);
@@ -1004,7 +1009,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
           const float db0 = db[2 * i], db1 = db[2 * i + 1], dc0 = dc[2 * i], dc1 = dc[2 * i + 1];
           dph[i] = db0 * bt[2 * i + 1] - db1 * bt[2 * i] + dc0 * ct[2 * i + 1] - dc1 * ct[2 * i];
           float sn, cs;
-          __sincosf(pht[tm * K2 + nn / 2 + i], &sn, &cs);
+          __sincosf(pht[(nn / 2 + i) * QP + tm], &sn, &cs);
           ob[2 * i] = cs * db0 - sn * db1;
           ob[2 * i + 1] = sn * db0 + cs * db1;
           oc[2 * i] = cs * dc0 - sn * dc1;
@@ -1036,10 +1041,11 @@ __global__ void __launch_bounds__(kCThreads, 1)
         for (int o = 1; o < R; o <<= 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) dph[i] += __shfl_xor_sync(0xffffffffu, dph[i], o);
-        if (vrow && rm == 0) {
-          float4* dst = reinterpret_cast<float4*>(dphi_s + tm * K2 + nn / 2);
-          dst[0] = make_float4(dph[0], dph[1], dph[2], dph[3]);
-          dst[1] = make_float4(dph[4], dph[5], dph[6], dph[7]);
+        if (vrow && rm == 0) {  // row tm, pairs XOR-swizzled by the row (see dphi_at)
+          const int sw = (tm & 7) << 2;
+          *reinterpret_cast<float4*>(dphi_s + tm * K2 + ((nn / 2) ^ sw)) = make_float4(dph[0], dph[1], dph[2], dph[3]);
+          *reinterpret_cast<float4*>(dphi_s + tm * K2 + ((nn / 2 + 4) ^ sw)) =
+              make_float4(dph[4], dph[5], dph[6], dph[7]);
         }
       }
     }
@@ -1050,14 +1056,14 @@ __global__ void __launch_bounds__(kCThreads, 1)
       const int k = tid % K2, part = tid / K2;
       const int tb = part * TPP2, te = (tb + TPP2 < Q) ? tb + TPP2 : Q;
       float ps = 0.f;
-      for (int t = tb; t < te; ++t) ps += dphi_s[t * K2 + k];
+      for (int t = tb; t < te; ++t) ps += dphi_s[dphi_at(t, k)];
       part_sum[part * K2 + k] = ps;
       __syncthreads();
       float S = sang[k];
       for (int p2 = part + 1; p2 < NPART2; ++p2) S += part_sum[p2 * K2 + k];
       __syncthreads();  // every thread has read sang[k]
       for (int t = te - 1; t >= tb; --t) {
-        S += dphi_s[t * K2 + k];
+        S += dphi_s[dphi_at(t, k)];
         const float dtv = sc[sDt * kScalStride + t];
         const int tg = t0 + t;
         if (tg < L) dTHg[tok_index(a, b, tg, hh) * K2 + k] = __float2bfloat16_rn(dtv * S);

@@ -6,9 +6,10 @@
 // rotation angles are sums over time steps ("Mamba-3: 2x smaller state ..."
 // (MarkTechPost, Korean translation), section 1.2), so a segment's effect on
 // the state is a decay, a rotation and an additive term:
-//   1. launch_state_export: every segment's end state from a zero state and a
+//   1. launch_seg_state: every segment's end state from a zero state and a
 //      zero angle (h_loc, the rotated B and the x of its last token, its angle
-//      sum Phi_loc), on the sequence viewed as batch b S of length L / S;
+//      sum Phi_loc), on the sequence viewed as batch b S of length L / S, as one
+//      streaming tensor-core reduction per segment (seg_state.cu);
 //   2. seg_combine_kernel: per unit, in segment order, the state entering
 //      segment s + 1 from the one entering segment s (frame rotated by -Phi_in):
 //        h     = e^{sum_seg dt A} (h_in + (1 - lam_f) dt_f sum_r b_in[r] x_in[r]^T)
@@ -33,6 +34,7 @@ struct SegParams {
   ScanArgs a;        // the unsegmented problem (its init and final state, inputs)
   int S, Ls;         // segments per unit and their length
   const float *loc_h, *loc_b, *loc_x, *loc_ang;  // [b S, H, ...] segment aggregates
+  const float* loc_decay;                        // [b S, H] sum of dt * A over each segment
   float *in_h, *in_b, *in_x, *in_ang;            // [b S, H, ...] initial state of every segment
 };
 
@@ -54,29 +56,10 @@ __global__ void __launch_bounds__(kThreads) seg_combine_kernel(const SegParams s
   float* bp = h + NP;          // [R][N]
   float* xp = bp + R * N;      // [R][P]
   float* ang = xp + R * P;     // [K2]
-  float* red = ang + K2;       // [S] decay sums, then scratch
-  __shared__ float warp_part[kThreads / 32];
+  float* red = ang + K2;       // [S] decay sums
   const size_t us = (size_t)unit;
 
-  // the sum of dt * A over every segment (a block reduction per segment)
-  for (int s = 0; s < S; ++s) {
-    float v = 0.f;
-    for (int t = s * Ls + tid; t < (s + 1) * Ls; t += kThreads) {
-      const size_t i = ((size_t)b * L + t) * H + hh;
-      const float rate = a.A_t ? ldv<T>(a.A_t, i) : a.A[hh];
-      v += ldv<T>(a.dt, i) * rate;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if ((tid & 31) == 0) warp_part[tid >> 5] = v;
-    __syncthreads();
-    if (tid == 0) {
-      float tot = 0.f;
-      for (int w = 0; w < kThreads / 32; ++w) tot += warp_part[w];
-      red[s] = tot;
-    }
-    __syncthreads();
-  }
+  for (int i = tid; i < S; i += kThreads) red[i] = sp.loc_decay[((size_t)b * S + i) * H + hh];
   // the state entering segment 0: the caller's initial state, or zero
   for (int i = tid; i < NP; i += kThreads) h[i] = a.h0 ? a.h0[us * NP + i] : 0.f;
   for (int i = tid; i < R * N; i += kThreads) bp[i] = a.bprev0 ? a.bprev0[us * R * N + i] : 0.f;
@@ -96,19 +79,34 @@ __global__ void __launch_bounds__(kThreads) seg_combine_kernel(const SegParams s
     const float mu = (1.f - ldv<T>(a.lam, f)) * ldv<T>(a.dt, f);
     const float decay = expf(red[s]);
     const float* lh = sp.loc_h + su * NP;
-    for (int i = tid; i < NP / 2; i += kThreads) {  // one (pair k, column p) per step
-      const int k = i / P, p = i % P;
-      float sn, cs;
-      sincosf(ang[k], &sn, &cs);
-      float c0 = h[(2 * k) * P + p], c1 = h[(2 * k + 1) * P + p];
-      for (int r = 0; r < R; ++r) {
-        const float xr = mu * xp[r * P + p];
-        c0 += bp[r * N + 2 * k] * xr;
-        c1 += bp[r * N + 2 * k + 1] * xr;
+    constexpr int kMaxPer = 16;  // (pair, column) steps per thread: NP / 2 / 256 <= 16 (N <= 128, P = 64)
+    float l0v[kMaxPer], l1v[kMaxPer];
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {  // every load of the segment's state before any use
+      const int i = tid + j * kThreads;
+      if (i < NP / 2) {
+        const int k = i / P, p = i % P;
+        l0v[j] = lh[(2 * k) * P + p];
+        l1v[j] = lh[(2 * k + 1) * P + p];
       }
-      const float l0 = lh[(2 * k) * P + p], l1 = lh[(2 * k + 1) * P + p];
-      h[(2 * k) * P + p] = decay * c0 + cs * l0 + sn * l1;
-      h[(2 * k + 1) * P + p] = decay * c1 + cs * l1 - sn * l0;
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {  // one (pair k, column p) per step
+      const int i = tid + j * kThreads;
+      if (i < NP / 2) {
+        const int k = i / P, p = i % P;
+        float sn, cs;
+        sincosf(ang[k], &sn, &cs);
+        float c0 = h[(2 * k) * P + p], c1 = h[(2 * k + 1) * P + p];
+        for (int r = 0; r < R; ++r) {
+          const float xr = mu * xp[r * P + p];
+          c0 += bp[r * N + 2 * k] * xr;
+          c1 += bp[r * N + 2 * k + 1] * xr;
+        }
+        const float l0 = l0v[j], l1 = l1v[j];
+        h[(2 * k) * P + p] = decay * c0 + cs * l0 + sn * l1;
+        h[(2 * k + 1) * P + p] = decay * c1 + cs * l1 - sn * l0;
+      }
     }
     __syncthreads();  // every thread has read bp, xp, ang of the entering state
     for (int i = tid; i < R * K2; i += kThreads) {
@@ -164,7 +162,7 @@ int seg_count(const ScanArgs& a, int sms) {
 
 size_t seg_workspace_bytes(const ScanArgs& a, int S) {
   if (S <= 0) return 0;
-  return 2 * (size_t)a.batch * S * a.nheads * seg_state_floats(a) * sizeof(float);
+  return (2 * seg_state_floats(a) + 1) * (size_t)a.batch * S * a.nheads * sizeof(float);
 }
 
 // The prefill of `a` in S segments (workspace: the status word, then the segment
@@ -188,6 +186,8 @@ int launch_scan_segmented(const ScanArgs& a, int S, cudaStream_t s) {
   sp.in_b = ini + units_s * a.N * a.P;
   sp.in_x = sp.in_b + units_s * a.R * a.N;
   sp.in_ang = sp.in_x + units_s * a.R * a.P;
+  float* decay = ini + units_s * per;  // [b S, H]
+  sp.loc_decay = decay;
 
   // 1. segment aggregates
   ScanArgs a1 = a;
@@ -198,10 +198,12 @@ int launch_scan_segmented(const ScanArgs& a, int S, cudaStream_t s) {
   a1.bprev_out = const_cast<float*>(sp.loc_b);
   a1.xprev_out = const_cast<float*>(sp.loc_x);
   a1.angle_out = const_cast<float*>(sp.loc_ang);
+  a1.decay_out = decay;
   a1.y = nullptr;
-  int rc = launch_state_export(a1, s);
+  int rc = launch_seg_state(a1, s);
   if (rc != MAMBA3_OK) return rc;
   // 2. the segments' initial states (and the final state)
+  if (a.N * a.P / 2 > 16 * kThreads) return MAMBA3_ERR_UNSUPPORTED;  // the combine's register prefetch
   const size_t smem = (per + S) * sizeof(float);
   auto kc = a.dtype == MAMBA3_F32 ? seg_combine_kernel<float> : seg_combine_kernel<__nv_bfloat16>;
   if (smem > 48 * 1024 && cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)

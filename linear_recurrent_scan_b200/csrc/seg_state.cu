@@ -1,0 +1,407 @@
+// End state of every segment of a long sequence from a zero state and a zero
+// angle (the segment aggregates of the segmented prefill, scan_seg.cu), as one
+// streaming tensor-core reduction per segment (tcgen05 + TMA, bf16, sm_100a).
+//
+// In the frame rotated by -Phi the decay is real ("Mamba-3: 2x smaller state ..."
+// (MarkTechPost, Korean translation), sections 1.1-1.2), so the state after the
+// last token of a segment is one sum over its tokens,
+//   h_end = sum_s e^{cum_end - cum_s} w_s B~_s^T x_s        (cum inclusive, from the
+//                                                             segment start)
+// with the trapezoid weight w_s = lam_s dt_s + (1 - lam_{s+1}) dt_{s+1} (the last
+// token's next one lies outside the segment: w = gamma).  Every 128-row chunk adds
+// B~^T X_w (K = 128) to ONE TMEM accumulator, with X_w = diag(e^{cum_end - cum} w)
+// X weighted to the segment's end: no per-chunk epilogue, so the MMAs run behind
+// the chunk preparation (decay prefix, angles, RoPE of B in place, X_w) through a
+// 3-stage TMA ring (2 where shared memory is short).  cum_end - cum_s is the difference of two fp32 sums over the
+// segment (<= 1.6 per token here), a relative error near 1e-4 in the weight; a
+// weight that underflows belongs to a term below fp32 resolution.
+// 256 threads; at the end the accumulator becomes h (fp32), with the B of the
+// last token rotated by its angle (fp32), its x and the angle.
+#include <cuda.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace m3 {
+namespace {
+
+using namespace ptx;
+
+constexpr int kP = 64;
+constexpr int kM = 128;          // rows per chunk
+constexpr int kTile = 16384;     // 128 rows x 128 bytes, 128-byte swizzle
+constexpr int kThreads = 256;
+constexpr int kScal = 136;       // per-token scalar stride (>= Q + 1)
+
+enum Tag { kTagFull = 41, kTagMma, kTagDrain };
+
+__device__ __forceinline__ uint32_t swz(int row, int c) { return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4)); }
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+// NST stages of inputs: 3 where they fit, so that a stage is refilled two chunks
+// after its MMA was issued (no wait on the MMA just issued); else 2.
+template <int N, int R>
+struct GCfg {
+  static constexpr int Q = kM / R;
+  static constexpr int NKB = N / 64;
+  static constexpr int K2 = N / 2;
+  static constexpr int NG = K2 / 4;                     // 16-byte groups of a row
+  static constexpr int NPART = kThreads / NG;
+  static constexpr int NPA = NPART < Q ? NPART : Q;     // token parts of the angle scan
+  static constexpr int TPP = Q / NPA;
+  static constexpr int TH_BYTES = Q * K2 * 2;
+  static constexpr int OFF_B = 0;
+  static constexpr int OFF_X = NKB * kTile;
+  static constexpr int OFF_TH = OFF_X + kTile;
+  static constexpr int STAGE = OFF_TH + ((TH_BYTES + 1023) & ~1023);
+  static constexpr int NST = 3 * STAGE + 2 * kTile + 16384 <= 232448 - 1024 ? 3 : 2;
+  static constexpr int OFF_XW = NST * STAGE;            // two X_w buffers
+  static constexpr int OFF_SC = OFF_XW + 2 * kTile;     // dt, lam, rate, log2 prefix, f  [5][kScal]
+  static constexpr int OFF_PART = OFF_SC + 5 * kScal * 4;
+  static constexpr int OFF_PHI = OFF_PART + NPA * K2 * 4;
+  static constexpr int OFF_RED = OFF_PHI + K2 * 4;      // [8] warp sums, [8] scan carries
+  static constexpr int OFF_BAR = (OFF_RED + 64 + 7) & ~7;  // full[NST], mma[NST]
+  static constexpr int OFF_MISC = OFF_BAR + 64;
+  static constexpr int SMEM = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = SMEM + 1024;
+  static_assert(Q % NPA == 0, "parts");
+  static_assert(SMEM_ALLOC <= 232448, "shared memory");
+};
+
+template <int N, int R, bool TVA>
+__global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_constant__ CUtensorMap tmB,
+                                                             const __grid_constant__ CUtensorMap tmX,
+                                                             const __grid_constant__ CUtensorMap tmT,
+                                                             const ScanArgs a) {
+  using K = GCfg<N, R>;
+  constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, NPA = K::NPA, TPP = K::TPP, NST = K::NST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int unit = blockIdx.x, b = unit / a.nheads, hh = unit % a.nheads;
+  const int L = a.seqlen, H = a.nheads;
+  const int gh = hh / (a.nheads / a.ngroups);
+  const int nchunks = (L + Q - 1) / Q;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + K::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::OFF_MISC + 4);
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.workspace);
+  float* sdt = reinterpret_cast<float*>(smem + K::OFF_SC);
+  float* slm = sdt + kScal;
+  float* sat = slm + kScal;
+  float* sc2 = sat + kScal;   // inclusive log2 decay prefix from the segment start
+  float* sf = sc2 + kScal;    // X_w row weight of each token
+  float* part_sum = reinterpret_cast<float*>(smem + K::OFF_PART);
+  float* phi = reinterpret_cast<float*>(smem + K::OFF_PHI);
+  float* red = reinterpret_cast<float*>(smem + K::OFF_RED);
+  const __nv_bfloat16* DT = static_cast<const __nv_bfloat16*>(a.dt);
+  const __nv_bfloat16* LM = static_cast<const __nv_bfloat16*>(a.lam);
+  const __nv_bfloat16* AT = static_cast<const __nv_bfloat16*>(a.A_t);
+  const float Ah = TVA ? 0.f : a.A[hh];
+  auto tok = [&](int t) { return ((size_t)b * L + t) * H + hh; };
+
+  if (tid == 0) {
+    for (int i = 0; i < 2 * NST; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmT);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 64);
+    tmem_relinquish();
+  }
+  if (tid < K2) phi[tid] = 0.f;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto issue = [&](int c) {
+    const int s = c % NST;
+    uint8_t* st = smem + s * K::STAGE;
+    const int t0 = c * Q;
+    mbar_arrive_expect_tx(&bars[s], (uint32_t)(K::NKB * kTile + kTile + K::TH_BYTES));
+#pragma unroll
+    for (int kb = 0; kb < K::NKB; ++kb) tma_load_5d(st + K::OFF_B + kb * kTile, &tmB, &bars[s], kb * 64, 0, gh, t0, b);
+    tma_load_5d(st + K::OFF_X, &tmX, &bars[s], 0, 0, hh, t0, b);
+    tma_load_4d(st + K::OFF_TH, &tmT, &bars[s], 0, hh, t0, b);
+  };
+  int issued = 0;
+  if (tid == 0 && !a.test_withhold && nchunks > 0) {
+    issue(0);
+    issued = 1;
+  }
+
+  // the segment's total log2 decay (block reduction over its tokens)
+  float tot = 0.f;
+  for (int t = tid; t < L; t += kThreads) {
+    const size_t i = tok(t);
+    tot += __bfloat162float(DT[i]) * (TVA ? __bfloat162float(AT[i]) : Ah);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  if (lane == 0) red[warp] = tot;
+  __syncthreads();
+  float total = 0.f;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) total += red[w];
+  if (tid == 0 && a.decay_out) a.decay_out[unit] = total;
+  total *= kLog2e;
+
+  float r_dt = 0.f, r_lm = 1.f, r_at = Ah;  // token t0 + tid of the next chunk (tid <= Q)
+  auto load_scalars = [&](int c) {
+    const int t = c * Q + tid;
+    r_dt = 0.f; r_lm = 1.f; r_at = Ah;
+    if (tid <= Q && t < L) {
+      const size_t i = tok(t);
+      r_dt = __bfloat162float(DT[i]);
+      r_lm = __bfloat162float(LM[i]);
+      if constexpr (TVA) r_at = __bfloat162float(AT[i]);
+    }
+  };
+  load_scalars(0);
+  float carry = 0.f;  // (warp 0) log2 decay through the end of the previous chunk
+  const int g = tid % NG, part = tid / NG, kb = g / 8, c8 = g % 8;
+  int abort_c = -1;
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int s = c % NST;
+    uint8_t* st = smem + s * K::STAGE;
+    // load chunk c + 1 into the stage of chunk c + 1 - NST once that chunk's MMA has read
+    // it (with 3 stages an MMA issued two chunks ago; it also frees X_w buffer c % 2)
+    if (tid == 0) {
+      bool ok = true;
+      const int prev = c + 1 - NST;
+      if (prev >= 0)
+        ok = mbar_wait(&bars[NST + prev % NST], (prev / NST) & 1, abort_flag, status, kTagMma, a.wait_limit);
+      if (ok && c + 1 < nchunks && !a.test_withhold) {
+        fence_proxy_async_smem();
+        issue(c + 1);
+        issued = c + 2;
+      }
+    }
+    if (tid <= Q) {
+      sdt[tid] = r_dt;
+      slm[tid] = r_lm;
+      sat[tid] = r_at;
+    }
+    load_scalars(c + 1);
+    __syncthreads();
+    // decay prefix (warp 0: Q <= 128 tokens, four per lane) and the X_w weight of every token
+    if (warp == 0) {
+      float v[4], run = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * lane + e;
+        v[e] = i < Q ? sdt[i] * sat[i] * kLog2e : 0.f;
+        run += v[e];
+      }
+      float incl = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      float acc = carry + incl - run;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * lane + e;
+        acc += v[e];
+        if (i < Q) {
+          const float w = slm[i] * sdt[i] + (1.f - slm[i + 1]) * sdt[i + 1];
+          sc2[i] = acc;
+          sf[i] = w * ex2(total - acc);
+        }
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (!mbar_wait(&bars[s], (c / NST) & 1, abort_flag, status, kTagFull, a.wait_limit)) {}
+    if (__syncthreads_or(*abort_flag != 0)) {
+      abort_c = c;
+      break;
+    }
+    // angles: part sums of dt theta, prefix, RoPE of B in place
+    const __nv_bfloat16* th = reinterpret_cast<const __nv_bfloat16*>(st + K::OFF_TH);
+    float run[4] = {0.f, 0.f, 0.f, 0.f};
+    if (part < NPA) {
+      float loc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < TPP; ++i) {
+        const int t = part * TPP + i;
+        const float d = sdt[t];
+        const uint2 tv = *reinterpret_cast<const uint2*>(th + t * K2 + 4 * g);
+        const float2 t01 = unpack_bf16(tv.x), t23 = unpack_bf16(tv.y);
+        loc[0] += d * t01.x; loc[1] += d * t01.y; loc[2] += d * t23.x; loc[3] += d * t23.y;
+      }
+      *reinterpret_cast<float4*>(part_sum + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
+    }
+    __syncthreads();
+    if (part < NPA) {
+      const float4 base = *reinterpret_cast<const float4*>(phi + 4 * g);
+      run[0] = base.x; run[1] = base.y; run[2] = base.z; run[3] = base.w;
+      for (int p2 = 0; p2 < part; ++p2) {
+        const float4 ps = *reinterpret_cast<const float4*>(part_sum + p2 * K2 + 4 * g);
+        run[0] += ps.x; run[1] += ps.y; run[2] += ps.z; run[3] += ps.w;
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) run[k] = wrap_angle(run[k]);
+#pragma unroll
+      for (int i = 0; i < TPP; ++i) {
+        const int t = part * TPP + i;
+        const float d = sdt[t];
+        const uint2 tv = *reinterpret_cast<const uint2*>(th + t * K2 + 4 * g);
+        const float2 t01 = unpack_bf16(tv.x), t23 = unpack_bf16(tv.y);
+        run[0] += d * t01.x; run[1] += d * t01.y; run[2] += d * t23.x; run[3] += d * t23.y;
+        float sn[4], cs[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) __sincosf(run[k], &sn[k], &cs[k]);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          uint4* p = reinterpret_cast<uint4*>(st + K::OFF_B + kb * kTile + swz(t * R + r, c8));
+          const uint4 q = *p;
+          const uint32_t bw[4] = {q.x, q.y, q.z, q.w};
+          uint32_t bo[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 v = unpack_bf16(bw[k]);
+            bo[k] = pack_bf16(cs[k] * v.x + sn[k] * v.y, cs[k] * v.y - sn[k] * v.x);
+          }
+          *p = make_uint4(bo[0], bo[1], bo[2], bo[3]);
+        }
+      }
+    }
+    // X_w = diag(f) X into X_w buffer c % 2 (its last reader, the MMA of chunk c - 2,
+    // completed before thread 0 reached the barrier after this chunk's scalars)
+    uint8_t* xw = smem + K::OFF_XW + (c & 1) * kTile;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = tid + kThreads * i;
+      const int row = idx >> 3, cc = idx & 7;
+      const float f = sf[row / R];
+      const uint4 xq = *reinterpret_cast<const uint4*>(st + K::OFF_X + swz(row, cc));
+      const float2 f0 = unpack_bf16(xq.x), f1 = unpack_bf16(xq.y), f2 = unpack_bf16(xq.z), f3 = unpack_bf16(xq.w);
+      *reinterpret_cast<uint4*>(xw + swz(row, cc)) =
+          make_uint4(pack_bf16(f * f0.x, f * f0.y), pack_bf16(f * f1.x, f * f1.y), pack_bf16(f * f2.x, f * f2.y),
+                     pack_bf16(f * f3.x, f * f3.y));
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (part == NPA - 1) {  // the last part's running angle is the chunk's end angle
+      *reinterpret_cast<float4*>(phi + 4 * g) =
+          make_float4(wrap_angle(run[0]), wrap_angle(run[1]), wrap_angle(run[2]), wrap_angle(run[3]));
+    }
+    if (tid == 0) {  // Hacc += B~^T X_w  (N x 64, K = 128 rows)
+      tc_fence_after();
+      const uint32_t iH = idesc_bf16(N, kP, 1, 1);
+      const uint32_t cB = smem_u32(st + K::OFF_B), cX = smem_u32(xw);
+#pragma unroll
+      for (int kk = 0; kk < kM / 16; ++kk)
+        mma_bf16_ss(tmem, smem_desc_sw128(cB + kk * 2048, kTile, 1024), smem_desc_sw128(cX + kk * 2048, kTile, 1024),
+                    iH, (c > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&bars[NST + s]);
+    }
+    __syncthreads();  // phi, the scalars and the part sums may be rewritten
+  }
+
+  // chunks whose MMA was issued; a commit covers every earlier MMA of this thread
+  const int mma_issued = abort_c >= 0 ? abort_c : nchunks;
+  if (tid == 0) {
+    if (abort_c < 0 && nchunks > 0)
+      mbar_wait(&bars[NST + (nchunks - 1) % NST], ((nchunks - 1) / NST) & 1, abort_flag, status, kTagMma,
+                a.wait_limit);
+    if (*abort_flag) {
+      // let the copies and MMAs issued land before TMEM is freed and the CTA exits
+      for (int c2 = abort_c >= 0 ? abort_c : nchunks; c2 < issued; ++c2)
+        if (!mbar_wait_drain(&bars[c2 % NST], (c2 / NST) & 1)) report_timeout(status, kTagDrain);
+      if (mma_issued > 0 &&
+          !mbar_wait_drain(&bars[NST + (mma_issued - 1) % NST], ((mma_issued - 1) / NST) & 1))
+        report_timeout(status, kTagDrain);
+    }
+  }
+  if (__syncthreads_or(*abort_flag != 0)) {
+    // aborted: outputs undefined, the status word says so
+  } else if (L > 0) {
+    tc_fence_after();
+    // h_end from the accumulator: state row n, 32 columns per thread
+    const int quad = warp & 3, half = warp >> 2;
+    const int n = (N == 128) ? quad * 32 + lane : (lane < 16 ? quad * 16 + lane : -1);
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    float hv[32];
+    tmem_ld32(tmem + lane_base + 32 * half, hv);
+    tmem_ld_wait();
+    if (n >= 0) {
+      float* ho = a.h_out + ((size_t)unit * N + n) * kP + 32 * half;
+#pragma unroll
+      for (int p = 0; p < 32; p += 4) *reinterpret_cast<float4*>(ho + p) = make_float4(hv[p], hv[p + 1], hv[p + 2], hv[p + 3]);
+    }
+    const size_t il = tok(L - 1);
+    const size_t ib = ((size_t)b * L + (L - 1)) * a.ngroups + gh;
+    const __nv_bfloat16* Bl = static_cast<const __nv_bfloat16*>(a.B) + ib * R * N;
+    const __nv_bfloat16* Xl = static_cast<const __nv_bfloat16*>(a.x) + il * R * kP;
+    for (int i = tid; i < R * K2; i += kThreads) {  // B of the last token rotated by its angle, in fp32
+      const int r = i / K2, k = i % K2;
+      float sn, cs;
+      sincosf(phi[k], &sn, &cs);
+      const float b0 = __bfloat162float(Bl[r * N + 2 * k]), b1 = __bfloat162float(Bl[r * N + 2 * k + 1]);
+      a.bprev_out[((size_t)unit * R + r) * N + 2 * k] = cs * b0 + sn * b1;
+      a.bprev_out[((size_t)unit * R + r) * N + 2 * k + 1] = cs * b1 - sn * b0;
+    }
+    for (int i = tid; i < R * kP; i += kThreads) a.xprev_out[(size_t)unit * R * kP + i] = __bfloat162float(Xl[i]);
+    if (tid < K2) a.angle_out[(size_t)unit * K2 + tid] = phi[tid];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+template <int N, int R, bool TVA>
+int launch_nr(const ScanArgs& a, cudaStream_t s) {
+  using K = GCfg<N, R>;
+  constexpr int Q = K::Q;
+  CUtensorMap tmB, tmX, tmT;
+  if (!make_map(&tmB, a.B, N, a.ngroups, a, Q) || !make_map(&tmX, a.x, kP, a.nheads, a, Q) ||
+      !make_theta_map(&tmT, a, Q))
+    return MAMBA3_ERR_CUDA;
+  auto k = seg_state_kernel<N, R, TVA>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess)
+    return MAMBA3_ERR_CUDA;
+  k<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmX, tmT, a);
+  return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
+}
+
+template <int N, int R>
+int launch_r(const ScanArgs& a, cudaStream_t s) {
+  return a.A_t ? launch_nr<N, R, true>(a, s) : launch_nr<N, R, false>(a, s);
+}
+
+}  // namespace
+
+int launch_seg_state(const ScanArgs& a, cudaStream_t s) {
+  if (bwd_tc_supported(a) != MAMBA3_OK || a.h0 || a.angle0) return MAMBA3_ERR_UNSUPPORTED;
+  if (a.N == 128) {
+    if (a.R == 1) return launch_r<128, 1>(a, s);
+    if (a.R == 2) return launch_r<128, 2>(a, s);
+    if (a.R == 4) return launch_r<128, 4>(a, s);
+  } else {
+    if (a.R == 1) return launch_r<64, 1>(a, s);
+    if (a.R == 2) return launch_r<64, 2>(a, s);
+    if (a.R == 4) return launch_r<64, 4>(a, s);
+  }
+  return MAMBA3_ERR_UNSUPPORTED;
+}
+
+}  // namespace m3
