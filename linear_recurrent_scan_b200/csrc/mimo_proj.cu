@@ -13,9 +13,11 @@
 //   out = o / sqrt(mean_p o^2 + eps) * w[h, p] * silu(z[t, h, p]).
 // t runs over every (batch, token) pair.
 //
-// One CTA per (head, range of 128-token tiles).  Warp 4 (one lane) loads the
-// head's weight tile once, then streams the token tiles through a 2-stage TMA
-// ring and issues one MMA chain per tile into one of two TMEM accumulators;
+// Persistent CTAs (one or two per SM) each take an even share of the (head,
+// 128-token tile) work items in head order.  Warp 4 (one lane) loads each head's
+// weight tile into one of two buffers as the CTA's items reach that head, streams
+// the token tiles through a 2-stage TMA ring and issues one MMA chain per tile
+// into one of two TMEM accumulators;
 // warps 0..3 (one TMEM lane quadrant each, thread = token row) drain the other
 // accumulator: fp32 -> (norm, gate) -> bf16 -> 16-byte stores.  The work is
 // HBM-bound (about 50 FLOP per byte at R = 4, against a ridge near 250).
@@ -47,7 +49,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 struct ProjParams {
   long long tokens;  // batch * seqlen
-  int nheads, tiles, tiles_per_cta;
+  int nheads, tiles;  // tiles of 128 tokens per head; work item = head * tiles + tile
+  long long items;    // nheads * tiles, split evenly over the grid
   void* out;               // x [T, H, R, P] (up) or o [T, H, P] (down), bf16
   const void* z;           // down: gate [T, H, P] bf16, or null (no norm, no gate)
   const float* w;          // down with gate: norm weight [H, P] or null (1)
@@ -64,9 +67,9 @@ struct PCfg {
   static constexpr int NOUT = UP ? R * kP : kP;           // accumulator columns
   static constexpr int IN_BYTES = KB * kRows * 128;       // one token tile
   static constexpr int W_BYTES = UP ? R * kP * 128 : R * kP * 128;  // (R P rows x 128 B) or (64 rows x R blocks)
-  static constexpr int OFF_W = 0;
-  static constexpr int OFF_IN = OFF_W + W_BYTES;
-  static constexpr int OFF_BAR = OFF_IN + 2 * IN_BYTES;   // full[2], empty[2], accf[2], acce[2], wfull
+  static constexpr int OFF_W = 0;                         // two weight buffers (heads alternate)
+  static constexpr int OFF_IN = OFF_W + 2 * W_BYTES;
+  static constexpr int OFF_BAR = OFF_IN + 2 * IN_BYTES;   // full[2], empty[2], accf[2], acce[2], wfull[2]
   static constexpr int OFF_MISC = OFF_BAR + 128;
   static constexpr int SMEM = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
@@ -76,6 +79,21 @@ struct PCfg {
 };
 
 enum { bFull = 0, bEmpty = 2, bAccF = 4, bAccE = 6, bW = 8 };
+
+// The CTA's work items [i0, i1) of the flattened (head, tile) space; the heads
+// they span are its head segments k = 0, 1, ... (head = item / tiles), each using
+// weight buffer k % 2.
+struct ItemRange {
+  long long i0, i1;
+  int h0;
+};
+__device__ __forceinline__ ItemRange item_range(const ProjParams& p) {
+  ItemRange r;
+  r.i0 = p.items * blockIdx.x / gridDim.x;
+  r.i1 = p.items * (blockIdx.x + 1) / gridDim.x;
+  r.h0 = (int)(r.i0 / p.tiles);
+  return r;
+}
 
 template <int R, bool UP, bool GATE>
 __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_constant__ CUtensorMap tmIn,
@@ -89,10 +107,13 @@ __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_consta
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + K::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::OFF_MISC + 4);
-  const int ctas_per_head = (prm.tiles + prm.tiles_per_cta - 1) / prm.tiles_per_cta;
-  const int h = blockIdx.x / ctas_per_head;
-  const int tile0 = (blockIdx.x % ctas_per_head) * prm.tiles_per_cta;
-  const int ntile = min(prm.tiles_per_cta, prm.tiles - tile0);
+  // items whose MMA is known complete (the epilogue saw their accumulator full);
+  // monotone, so the producer can tell when a weight buffer is free
+  volatile int* mma_done = reinterpret_cast<volatile int*>(smem + K::OFF_MISC + 8);
+  const ItemRange rg = item_range(prm);
+  const int n = (int)(rg.i1 - rg.i0);  // items of this CTA
+  auto head_of = [&](int j) { return (int)((rg.i0 + j) / prm.tiles); };
+  auto tile_of = [&](int j) { return (int)((rg.i0 + j) % prm.tiles); };
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -100,9 +121,10 @@ __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_consta
       mbar_init(&bars[bEmpty + i], 1);
       mbar_init(&bars[bAccF + i], 1);
       mbar_init(&bars[bAccE + i], 128);
+      mbar_init(&bars[bW + i], 1);
     }
-    mbar_init(&bars[bW], 1);
     *abort_flag = 0;
+    *mma_done = 0;
     fence_mbar_init();
     prefetch_tmap(&tmIn);
     prefetch_tmap(&tmW);
@@ -118,56 +140,72 @@ __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_consta
 
   if (warp == 4) {
     if (lane == 0) {
-      // ---- producer and MMA issuer ----
-      int loaded = 0, done = 0;  // tiles whose loads were issued / whose MMAs were issued
-      int wload = 0;
-      if (!prm.test_withhold) {
-        mbar_arrive_expect_tx(&bars[bW], K::W_BYTES);
-        if (UP) {
-          tma_load_3d(smem + K::OFF_W, &tmW, &bars[bW], 0, 0, h);
-        } else {
-#pragma unroll
-          for (int kb = 0; kb < R; ++kb) tma_load_3d(smem + K::OFF_W + kb * kP * 128, &tmW, &bars[bW], kb * 64, 0, h);
-        }
-        wload = 1;
-      }
+      // ---- producer and MMA issuer: inputs through a 2-stage ring, the weights of
+      // head segment k into buffer k % 2 once segment k - 2's MMAs are complete ----
+      int loaded = 0, done = 0;        // items whose loads / MMAs were issued
+      int wseg = 0;                    // head segments whose weights were issued
+      int last_of_slot[2] = {-1, -1};  // last item whose MMA read each weight buffer
       const uint32_t idesc = idesc_bf16(kRows, K::NOUT, 0, 0);
       bool ok = true;
       long long t_last = clock64();
-      while (ok && done < ntile) {
+      while (ok && done < n) {
         bool progress = false;
-        // load tile `loaded` into stage loaded & 1 once its previous MMA has read it
-        if (!prm.test_withhold && loaded < ntile && loaded < done + 2 &&
+        // weights of the next head segment, once its buffer is free
+        const int seg_needed = head_of(loaded < n ? loaded : n - 1) - rg.h0;
+        if (!prm.test_withhold && wseg <= seg_needed && wseg <= head_of(n - 1) - rg.h0) {
+          const int slot = wseg & 1, prev = last_of_slot[slot];
+          // buffer free once segment wseg - 2's last MMA has completed
+          if (prev < *mma_done) {
+            const int h = rg.h0 + wseg;
+            uint8_t* wb = smem + K::OFF_W + slot * K::W_BYTES;
+            mbar_arrive_expect_tx(&bars[bW + slot], K::W_BYTES);
+            if (UP) {
+              tma_load_3d(wb, &tmW, &bars[bW + slot], 0, 0, h);
+            } else {
+#pragma unroll
+              for (int kb = 0; kb < R; ++kb) tma_load_3d(wb + kb * kP * 128, &tmW, &bars[bW + slot], kb * 64, 0, h);
+            }
+            ++wseg;
+            progress = true;
+          }
+        }
+        // inputs of item `loaded` into stage loaded & 1 once the MMA of item loaded - 2 has read it
+        if (!prm.test_withhold && loaded < n && loaded < done + 2 &&
             (loaded < 2 || mbar_test(&bars[bEmpty + (loaded & 1)], ((loaded >> 1) - 1) & 1))) {
           const int s = loaded & 1;
-          const long long row0 = (long long)(tile0 + loaded) * kRows;
+          const int row0 = tile_of(loaded) * kRows;
           mbar_arrive_expect_tx(&bars[bFull + s], K::IN_BYTES);
 #pragma unroll
           for (int kb = 0; kb < K::KB; ++kb)
-            tma_load_3d(smem + K::OFF_IN + s * K::IN_BYTES + kb * kRows * 128, &tmIn, &bars[bFull + s], kb * 64, h,
-                        (int)row0);
+            tma_load_3d(smem + K::OFF_IN + s * K::IN_BYTES + kb * kRows * 128, &tmIn, &bars[bFull + s], kb * 64,
+                        head_of(loaded), row0);
           ++loaded;
           progress = true;
         }
-        // MMA of tile `done` once its input landed and its accumulator is free
-        if (done < loaded && mbar_test(&bars[bFull + (done & 1)], (done >> 1) & 1) &&
-            (done < 2 || mbar_test(&bars[bAccE + (done & 1)], ((done >> 1) - 1) & 1)) &&
-            (done > 0 || mbar_test(&bars[bW], 0))) {
-          tc_fence_after();
-          const int s = done & 1;
-          const uint32_t cIn = smem_u32(smem + K::OFF_IN + s * K::IN_BYTES), cW = smem_u32(smem + K::OFF_W);
-          const uint32_t d = tmem + (uint32_t)(s * K::NOUT);
+        // MMA of item `done`: inputs landed, accumulator free, its head's weights loaded
+        if (done < loaded) {
+          const int seg = head_of(done) - rg.h0, slot = seg & 1;
+          if (seg < wseg && mbar_test(&bars[bFull + (done & 1)], (done >> 1) & 1) &&
+              (done < 2 || mbar_test(&bars[bAccE + (done & 1)], ((done >> 1) - 1) & 1)) &&
+              mbar_test(&bars[bW + slot], (seg >> 1) & 1)) {
+            tc_fence_after();
+            const int s = done & 1;
+            const uint32_t cIn = smem_u32(smem + K::OFF_IN + s * K::IN_BYTES);
+            const uint32_t cW = smem_u32(smem + K::OFF_W + slot * K::W_BYTES);
+            const uint32_t d = tmem + (uint32_t)(s * K::NOUT);
 #pragma unroll
-          for (int kk = 0; kk < K::KB * 4; ++kk) {
-            const uint32_t offa = (kk >> 2) * kRows * 128 + (kk & 3) * 32;
-            const uint32_t offb = (kk >> 2) * kP * 128 + (kk & 3) * 32;
-            mma_bf16_ss(d, smem_desc_sw128(cIn + offa, 16, 1024), smem_desc_sw128(cW + offb, 16, 1024), idesc,
-                        kk > 0);
+            for (int kk = 0; kk < K::KB * 4; ++kk) {
+              const uint32_t offa = (kk >> 2) * kRows * 128 + (kk & 3) * 32;
+              const uint32_t offb = (kk >> 2) * kP * 128 + (kk & 3) * 32;
+              mma_bf16_ss(d, smem_desc_sw128(cIn + offa, 16, 1024), smem_desc_sw128(cW + offb, 16, 1024), idesc,
+                          kk > 0);
+            }
+            mma_commit(&bars[bEmpty + s]);
+            mma_commit(&bars[bAccF + s]);
+            last_of_slot[slot] = done;
+            ++done;
+            progress = true;
           }
-          mma_commit(&bars[bEmpty + s]);
-          mma_commit(&bars[bAccF + s]);
-          ++done;
-          progress = true;
         }
         if (progress) {
           t_last = clock64();
@@ -181,7 +219,8 @@ __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_consta
         }
       }
       // let the copies and MMAs issued land before TMEM is freed and the CTA exits
-      if (wload && !mbar_wait_drain(&bars[bW], 0)) report_timeout(&g_proj_status, 32);
+      for (int k = (wseg >= 2 ? wseg - 2 : 0); k < wseg; ++k)
+        if (!mbar_wait_drain(&bars[bW + (k & 1)], (k >> 1) & 1)) report_timeout(&g_proj_status, 32);
       for (int i = done; i < loaded; ++i)
         if (!mbar_wait_drain(&bars[bFull + (i & 1)], (i >> 1) & 1)) report_timeout(&g_proj_status, 32);
       if (done > 0 && !mbar_wait_drain(&bars[bAccF + ((done - 1) & 1)], ((done - 1) >> 1) & 1))
@@ -191,11 +230,13 @@ __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_consta
     // ---- epilogue: warp w reads TMEM lanes 32 w .. 32 w + 31 (thread = token row) ----
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(prm.out);
-    for (int i = 0; i < ntile; ++i) {
+    for (int i = 0; i < n; ++i) {
       const int s = i & 1;
       if (!mbar_wait(&bars[bAccF + s], (i >> 1) & 1, abort_flag, &g_proj_status, 33, prm.wait_limit)) break;
       tc_fence_after();
-      const long long tok = (long long)(tile0 + i) * kRows + warp * 32 + lane;
+      if (tid == 0) *mma_done = i + 1;  // MMA i (and every earlier one) has completed
+      const int h = head_of(i);
+      const long long tok = (long long)tile_of(i) * kRows + warp * 32 + lane;
       const bool valid = tok < prm.tokens;
       const uint32_t tacc = tmem + lane_base + (uint32_t)(s * K::NOUT);
       if constexpr (UP) {
@@ -292,13 +333,12 @@ int launch_k(const ProjArgs& a, cudaStream_t s) {
   prm.tokens = T;
   prm.nheads = H;
   prm.tiles = (int)((T + kRows - 1) / kRows);
-  // about two CTAs' worth of tiles per SM in total, whole tiles per CTA
-  const long long total = (long long)prm.tiles * H;
-  long long per = (total + 2 * 148 - 1) / (2 * 148);
-  if (per < 1) per = 1;
-  if (per > prm.tiles) per = prm.tiles;
-  prm.tiles_per_cta = (int)per;
-  const int ctas_per_head = (prm.tiles + prm.tiles_per_cta - 1) / prm.tiles_per_cta;
+  prm.items = (long long)prm.tiles * H;
+  // persistent: one CTA per SM when the two accumulators take all 512 TMEM columns
+  // (the shared memory asked for keeps a second CTA off the SM), else two
+  const int per_sm = K::TMEM_COLS >= 512 ? 1 : 2;
+  const long long grid = prm.items < (long long)kSMs * per_sm ? prm.items : (long long)kSMs * per_sm;
+  const int smem = per_sm == 1 && K::SMEM_ALLOC < 120 * 1024 ? 120 * 1024 : K::SMEM_ALLOC;
   prm.out = a.out;
   prm.z = a.z;
   prm.w = a.w;
@@ -306,9 +346,9 @@ int launch_k(const ProjArgs& a, cudaStream_t s) {
   prm.wait_limit = a.wait_limit;
   prm.test_withhold = a.test_withhold;
   auto k = mimo_proj_kernel<R, UP, GATE>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess)
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
-  k<<<ctas_per_head * H, kThreads, K::SMEM_ALLOC, s>>>(tmIn, tmW, prm);
+  k<<<(int)grid, kThreads, smem, s>>>(tmIn, tmW, prm);
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 

@@ -33,7 +33,6 @@ constexpr int kP = 64;
 constexpr int kM = 128;          // rows per chunk
 constexpr int kTile = 16384;     // 128 rows x 128 bytes, 128-byte swizzle
 constexpr int kThreads = 256;
-constexpr int kScal = 136;       // per-token scalar stride (>= Q + 1)
 
 enum Tag { kTagFull = 41, kTagMma, kTagDrain };
 
@@ -54,9 +53,6 @@ struct GCfg {
   static constexpr int NKB = N / 64;
   static constexpr int K2 = N / 2;
   static constexpr int NG = K2 / 4;                     // 16-byte groups of a row
-  static constexpr int NPART = kThreads / NG;
-  static constexpr int NPA = NPART < Q ? NPART : Q;     // token parts of the angle scan
-  static constexpr int TPP = Q / NPA;
   static constexpr int TH_BYTES = Q * K2 * 2;
   static constexpr int OFF_B = 0;
   static constexpr int OFF_X = NKB * kTile;
@@ -64,15 +60,12 @@ struct GCfg {
   static constexpr int STAGE = OFF_TH + ((TH_BYTES + 1023) & ~1023);
   static constexpr int NST = 3 * STAGE + 2 * kTile + 16384 <= 232448 - 1024 ? 3 : 2;
   static constexpr int OFF_XW = NST * STAGE;            // two X_w buffers
-  static constexpr int OFF_SC = OFF_XW + 2 * kTile;     // dt, lam, rate, log2 prefix, f  [5][kScal]
-  static constexpr int OFF_PART = OFF_SC + 5 * kScal * 4;
-  static constexpr int OFF_PHI = OFF_PART + NPA * K2 * 4;
+  static constexpr int OFF_PHI = OFF_XW + 2 * kTile;    // final angle [K2]
   static constexpr int OFF_RED = OFF_PHI + K2 * 4;      // [8] warp sums, [8] scan carries
   static constexpr int OFF_BAR = (OFF_RED + 64 + 7) & ~7;  // full[NST], mma[NST]
   static constexpr int OFF_MISC = OFF_BAR + 64;
   static constexpr int SMEM = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
-  static_assert(Q % NPA == 0, "parts");
   static_assert(SMEM_ALLOC <= 232448, "shared memory");
 };
 
@@ -82,7 +75,7 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
                                                              const __grid_constant__ CUtensorMap tmT,
                                                              const ScanArgs a) {
   using K = GCfg<N, R>;
-  constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, NPA = K::NPA, TPP = K::TPP, NST = K::NST;
+  constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, NST = K::NST;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -95,12 +88,6 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + K::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::OFF_MISC + 4);
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.workspace);
-  float* sdt = reinterpret_cast<float*>(smem + K::OFF_SC);
-  float* slm = sdt + kScal;
-  float* sat = slm + kScal;
-  float* sc2 = sat + kScal;   // inclusive log2 decay prefix from the segment start
-  float* sf = sc2 + kScal;    // X_w row weight of each token
-  float* part_sum = reinterpret_cast<float*>(smem + K::OFF_PART);
   float* phi = reinterpret_cast<float*>(smem + K::OFF_PHI);
   float* red = reinterpret_cast<float*>(smem + K::OFF_RED);
   const __nv_bfloat16* DT = static_cast<const __nv_bfloat16*>(a.dt);
@@ -121,7 +108,6 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
     tmem_alloc(tmem_slot, 64);
     tmem_relinquish();
   }
-  if (tid < K2) phi[tid] = 0.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -159,20 +145,37 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
   if (tid == 0 && a.decay_out) a.decay_out[unit] = total;
   total *= kLog2e;
 
-  float r_dt = 0.f, r_lm = 1.f, r_at = Ah;  // token t0 + tid of the next chunk (tid <= Q)
+  // Warp w owns the 4-pair groups w GPW .. w GPW + GPW - 1 of every row; lane l owns the
+  // tokens l TPL .. l TPL + TPL - 1 of every chunk.  The decay prefix and the angle
+  // prefix are warp scans over the lanes, so a chunk needs one block barrier, before
+  // its MMA.  Every warp keeps the decay carry and its groups' running angles.
+  constexpr int TPL = Q / 32, GPW = NG / (kThreads / 32);
+  static_assert(TPL >= 1 && Q % 32 == 0 && GPW >= 1 && NG % (kThreads / 32) == 0, "lanes and warps");
+  float p_dt[TPL + 1], p_lm[TPL + 1], p_at[TPL];  // this lane's tokens of the next chunk (+ the one after)
   auto load_scalars = [&](int c) {
-    const int t = c * Q + tid;
-    r_dt = 0.f; r_lm = 1.f; r_at = Ah;
-    if (tid <= Q && t < L) {
-      const size_t i = tok(t);
-      r_dt = __bfloat162float(DT[i]);
-      r_lm = __bfloat162float(LM[i]);
-      if constexpr (TVA) r_at = __bfloat162float(AT[i]);
+#pragma unroll
+    for (int i = 0; i <= TPL; ++i) {
+      const int t = c * Q + lane * TPL + i;
+      p_dt[i] = 0.f;
+      p_lm[i] = 1.f;
+      if (i < TPL) p_at[i] = Ah;
+      if (t < L) {
+        const size_t ti = tok(t);
+        p_dt[i] = __bfloat162float(DT[ti]);
+        p_lm[i] = __bfloat162float(LM[ti]);
+        if constexpr (TVA) {
+          if (i < TPL) p_at[i] = __bfloat162float(AT[ti]);
+        }
+      }
     }
   };
   load_scalars(0);
-  float carry = 0.f;  // (warp 0) log2 decay through the end of the previous chunk
-  const int g = tid % NG, part = tid / NG, kb = g / 8, c8 = g % 8;
+  float carry = 0.f;       // log2 decay through the end of the previous chunk
+  float phw[GPW][4];       // running angle of this warp's pair groups
+#pragma unroll
+  for (int q = 0; q < GPW; ++q)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) phw[q][k] = 0.f;
   int abort_c = -1;
 
   for (int c = 0; c < nchunks; ++c) {
@@ -191,21 +194,22 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
         issued = c + 2;
       }
     }
-    if (tid <= Q) {
-      sdt[tid] = r_dt;
-      slm[tid] = r_lm;
-      sat[tid] = r_at;
+    float dt[TPL + 1], lm[TPL + 1], at[TPL];
+#pragma unroll
+    for (int i = 0; i <= TPL; ++i) {
+      dt[i] = p_dt[i];
+      lm[i] = p_lm[i];
+      if (i < TPL) at[i] = p_at[i];
     }
     load_scalars(c + 1);
-    __syncthreads();
-    // decay prefix (warp 0: Q <= 128 tokens, four per lane) and the X_w weight of every token
-    if (warp == 0) {
-      float v[4], run = 0.f;
+    // decay prefix over the chunk (lane-local, then a warp scan) and the X_w weight f
+    float f[TPL];
+    {
+      float v[TPL], run = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * lane + e;
-        v[e] = i < Q ? sdt[i] * sat[i] * kLog2e : 0.f;
-        run += v[e];
+      for (int i = 0; i < TPL; ++i) {
+        v[i] = dt[i] * at[i] * kLog2e;
+        run += v[i];
       }
       float incl = run;
 #pragma unroll
@@ -215,91 +219,93 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
       }
       float acc = carry + incl - run;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * lane + e;
-        acc += v[e];
-        if (i < Q) {
-          const float w = slm[i] * sdt[i] + (1.f - slm[i + 1]) * sdt[i + 1];
-          sc2[i] = acc;
-          sf[i] = w * ex2(total - acc);
-        }
+      for (int i = 0; i < TPL; ++i) {
+        acc += v[i];
+        const float w = lm[i] * dt[i] + (1.f - lm[i + 1]) * dt[i + 1];
+        f[i] = w * ex2(total - acc);
       }
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (!mbar_wait(&bars[s], (c / NST) & 1, abort_flag, status, kTagFull, a.wait_limit)) {}
-    if (__syncthreads_or(*abort_flag != 0)) {
-      abort_c = c;
-      break;
+    if (*abort_flag) {  // block-wide decision at the barrier below
     }
-    // angles: part sums of dt theta, prefix, RoPE of B in place
+    // angles of this warp's pair groups at this lane's tokens, RoPE of B in place
     const __nv_bfloat16* th = reinterpret_cast<const __nv_bfloat16*>(st + K::OFF_TH);
-    float run[4] = {0.f, 0.f, 0.f, 0.f};
-    if (part < NPA) {
-      float loc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < TPP; ++i) {
-        const int t = part * TPP + i;
-        const float d = sdt[t];
+    for (int q = 0; q < GPW; ++q) {
+      const int g = warp * GPW + q, kb = g / 8, c8 = g % 8;
+      float inc[TPL][4], tot4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < TPL; ++i) {
+        const int t = lane * TPL + i;
         const uint2 tv = *reinterpret_cast<const uint2*>(th + t * K2 + 4 * g);
         const float2 t01 = unpack_bf16(tv.x), t23 = unpack_bf16(tv.y);
-        loc[0] += d * t01.x; loc[1] += d * t01.y; loc[2] += d * t23.x; loc[3] += d * t23.y;
+        inc[i][0] = dt[i] * t01.x; inc[i][1] = dt[i] * t01.y; inc[i][2] = dt[i] * t23.x; inc[i][3] = dt[i] * t23.y;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) tot4[k] += inc[i][k];
       }
-      *reinterpret_cast<float4*>(part_sum + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
-    }
-    __syncthreads();
-    if (part < NPA) {
-      const float4 base = *reinterpret_cast<const float4*>(phi + 4 * g);
-      run[0] = base.x; run[1] = base.y; run[2] = base.z; run[3] = base.w;
-      for (int p2 = 0; p2 < part; ++p2) {
-        const float4 ps = *reinterpret_cast<const float4*>(part_sum + p2 * K2 + 4 * g);
-        run[0] += ps.x; run[1] += ps.y; run[2] += ps.z; run[3] += ps.w;
+      float ex[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float x = tot4[k];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float u = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += u;
+        }
+        ex[k] = wrap_angle(phw[q][k] + x - tot4[k]);  // angle before this lane's first token
+        phw[q][k] = wrap_angle(phw[q][k] + __shfl_sync(0xffffffffu, x, 31));
       }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) run[k] = wrap_angle(run[k]);
-#pragma unroll
-      for (int i = 0; i < TPP; ++i) {
-        const int t = part * TPP + i;
-        const float d = sdt[t];
-        const uint2 tv = *reinterpret_cast<const uint2*>(th + t * K2 + 4 * g);
-        const float2 t01 = unpack_bf16(tv.x), t23 = unpack_bf16(tv.y);
-        run[0] += d * t01.x; run[1] += d * t01.y; run[2] += d * t23.x; run[3] += d * t23.y;
+      for (int i = 0; i < TPL; ++i) {
+        const int t = lane * TPL + i;
         float sn[4], cs[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) __sincosf(run[k], &sn[k], &cs[k]);
+        for (int k = 0; k < 4; ++k) {
+          ex[k] += inc[i][k];
+          __sincosf(ex[k], &sn[k], &cs[k]);
+        }
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           uint4* p = reinterpret_cast<uint4*>(st + K::OFF_B + kb * kTile + swz(t * R + r, c8));
-          const uint4 q = *p;
-          const uint32_t bw[4] = {q.x, q.y, q.z, q.w};
+          const uint4 qv = *p;
+          const uint32_t bw[4] = {qv.x, qv.y, qv.z, qv.w};
           uint32_t bo[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const float2 v = unpack_bf16(bw[k]);
-            bo[k] = pack_bf16(cs[k] * v.x + sn[k] * v.y, cs[k] * v.y - sn[k] * v.x);
+            const float2 vv = unpack_bf16(bw[k]);
+            bo[k] = pack_bf16(cs[k] * vv.x + sn[k] * vv.y, cs[k] * vv.y - sn[k] * vv.x);
           }
           *p = make_uint4(bo[0], bo[1], bo[2], bo[3]);
         }
       }
     }
-    // X_w = diag(f) X into X_w buffer c % 2 (its last reader, the MMA of chunk c - 2,
-    // completed before thread 0 reached the barrier after this chunk's scalars)
+    // X_w = diag(f) X into X_w buffer c % 2, once its last reader, the MMA of chunk
+    // c - 2, has completed: warp w writes rows 16 w .. 16 w + 15; the weight of row m is
+    // token m / R's f, held by lane (m / R) / TPL
+    if (c >= 2) mbar_wait(&bars[NST + (c - 2) % NST], ((c - 2) / NST) & 1, abort_flag, status, kTagMma, a.wait_limit);
     uint8_t* xw = smem + K::OFF_XW + (c & 1) * kTile;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int idx = tid + kThreads * i;
-      const int row = idx >> 3, cc = idx & 7;
-      const float f = sf[row / R];
+      const int u = warp * 128 + lane + 32 * i;
+      const int row = u >> 3, cc = u & 7;
+      const int tk = row / R;
+      float fsel = 0.f;
+#pragma unroll
+      for (int j = 0; j < TPL; ++j) {
+        const float fj = __shfl_sync(0xffffffffu, f[j], tk / TPL);
+        if (tk % TPL == j) fsel = fj;
+      }
       const uint4 xq = *reinterpret_cast<const uint4*>(st + K::OFF_X + swz(row, cc));
       const float2 f0 = unpack_bf16(xq.x), f1 = unpack_bf16(xq.y), f2 = unpack_bf16(xq.z), f3 = unpack_bf16(xq.w);
       *reinterpret_cast<uint4*>(xw + swz(row, cc)) =
-          make_uint4(pack_bf16(f * f0.x, f * f0.y), pack_bf16(f * f1.x, f * f1.y), pack_bf16(f * f2.x, f * f2.y),
-                     pack_bf16(f * f3.x, f * f3.y));
+          make_uint4(pack_bf16(fsel * f0.x, fsel * f0.y), pack_bf16(fsel * f1.x, fsel * f1.y),
+                     pack_bf16(fsel * f2.x, fsel * f2.y), pack_bf16(fsel * f3.x, fsel * f3.y));
     }
     fence_proxy_async_smem();
-    __syncthreads();
-    if (part == NPA - 1) {  // the last part's running angle is the chunk's end angle
-      *reinterpret_cast<float4*>(phi + 4 * g) =
-          make_float4(wrap_angle(run[0]), wrap_angle(run[1]), wrap_angle(run[2]), wrap_angle(run[3]));
+    if (__syncthreads_or(*abort_flag != 0)) {
+      abort_c = c;
+      break;
     }
     if (tid == 0) {  // Hacc += B~^T X_w  (N x 64, K = 128 rows)
       tc_fence_after();
@@ -311,8 +317,15 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
                     iH, (c > 0 || kk > 0) ? 1u : 0u);
       mma_commit(&bars[NST + s]);
     }
-    __syncthreads();  // phi, the scalars and the part sums may be rewritten
   }
+  // the final angle of every pair, for the export and the last token's rotation
+  if (lane == 0) {
+#pragma unroll
+    for (int q = 0; q < GPW; ++q)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) phi[4 * (warp * GPW + q) + k] = phw[q][k];
+  }
+  __syncthreads();
 
   // chunks whose MMA was issued; a commit covers every earlier MMA of this thread
   const int mma_issued = abort_c >= 0 ? abort_c : nchunks;
