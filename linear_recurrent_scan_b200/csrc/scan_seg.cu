@@ -10,7 +10,8 @@
 //      zero angle (h_loc, the rotated B and the x of its last token, its angle
 //      sum Phi_loc), on the sequence viewed as batch b S of length L / S, as one
 //      streaming tensor-core reduction per segment (seg_state.cu);
-//   2. seg_combine_kernel: per unit, in segment order, the state entering
+//   2. seg_combine_kernel: per unit (four CTAs, a quarter of the rotation pairs
+//      each), in segment order, the state entering
 //      segment s + 1 from the one entering segment s (frame rotated by -Phi_in):
 //        h     = e^{sum_seg dt A} (h_in + (1 - lam_f) dt_f sum_r b_in[r] x_in[r]^T)
 //                + rot(-Phi_in) h_loc
@@ -43,48 +44,63 @@ __device__ __forceinline__ float ldv(const void* p, size_t i) {
   return ld1(static_cast<const T*>(p) + i);
 }
 
-// One CTA per unit (b, h); the running state lives in shared memory.
+// kSplit CTAs per unit (b, h), each owning a quarter of the rotation pairs k (the
+// rows 2k, 2k+1 of h and b_prev and the angles k): the update acts within pairs, so
+// the parts are independent.  Part 0 also carries x_prev.  The running state of
+// the part lives in shared memory.
+constexpr int kSplit = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) seg_combine_kernel(const SegParams sp) {
   extern __shared__ float sm[];
   const ScanArgs& a = sp.a;
   const int N = a.N, P = a.P, R = a.R, K2 = N / 2, NP = N * P;
   const int H = a.nheads, L = a.seqlen, S = sp.S, Ls = sp.Ls;
-  const int unit = blockIdx.x, b = unit / H, hh = unit % H;
+  const int unit = blockIdx.x / kSplit, part = blockIdx.x % kSplit;
+  const int b = unit / H, hh = unit % H;
+  const int KP = K2 / kSplit, k0 = part * KP;  // this part's pairs k0 .. k0 + KP - 1
   const int tid = threadIdx.x;
-  float* h = sm;               // [N][P]
-  float* bp = h + NP;          // [R][N]
-  float* xp = bp + R * N;      // [R][P]
-  float* ang = xp + R * P;     // [K2]
-  float* red = ang + K2;       // [S] decay sums
+  float* h = sm;               // [2 KP][P]: rows 2 k0 .. 2 (k0 + KP) - 1 of h
+  float* bp = h + 2 * KP * P;  // [R][2 KP]
+  float* xp = bp + R * 2 * KP; // [R][P]
+  float* ang = xp + R * P;     // [KP]
+  float* red = ang + KP;       // [S] decay sums
   const size_t us = (size_t)unit;
+  const int row0 = 2 * k0, rows = 2 * KP;
 
   for (int i = tid; i < S; i += kThreads) red[i] = sp.loc_decay[((size_t)b * S + i) * H + hh];
   // the state entering segment 0: the caller's initial state, or zero
-  for (int i = tid; i < NP; i += kThreads) h[i] = a.h0 ? a.h0[us * NP + i] : 0.f;
-  for (int i = tid; i < R * N; i += kThreads) bp[i] = a.bprev0 ? a.bprev0[us * R * N + i] : 0.f;
+  for (int i = tid; i < rows * P; i += kThreads) h[i] = a.h0 ? a.h0[us * NP + row0 * P + i] : 0.f;
+  for (int i = tid; i < R * rows; i += kThreads) {
+    const int r = i / rows, n = row0 + i % rows;
+    bp[i] = a.bprev0 ? a.bprev0[(us * R + r) * N + n] : 0.f;
+  }
   for (int i = tid; i < R * P; i += kThreads) xp[i] = a.xprev0 ? a.xprev0[us * R * P + i] : 0.f;
-  for (int i = tid; i < K2; i += kThreads) ang[i] = a.angle0 ? a.angle0[us * K2 + i] : 0.f;
+  for (int i = tid; i < KP; i += kThreads) ang[i] = a.angle0 ? a.angle0[us * K2 + k0 + i] : 0.f;
   __syncthreads();
 
   for (int s = 0; s < S; ++s) {
     const size_t su = ((size_t)b * S + s) * H + hh;  // the segment's unit in the b S x H view
-    // the initial state of segment s
-    for (int i = tid; i < NP; i += kThreads) sp.in_h[su * NP + i] = h[i];
-    for (int i = tid; i < R * N; i += kThreads) sp.in_b[su * R * N + i] = bp[i];
-    for (int i = tid; i < R * P; i += kThreads) sp.in_x[su * R * P + i] = xp[i];
-    for (int i = tid; i < K2; i += kThreads) sp.in_ang[su * K2 + i] = ang[i];
+    // the initial state of segment s (this part's rows)
+    for (int i = tid; i < rows * P; i += kThreads) sp.in_h[su * NP + row0 * P + i] = h[i];
+    for (int i = tid; i < R * rows; i += kThreads) {
+      const int r = i / rows, n = row0 + i % rows;
+      sp.in_b[(su * R + r) * N + n] = bp[i];
+    }
+    if (part == 0)
+      for (int i = tid; i < R * P; i += kThreads) sp.in_x[su * R * P + i] = xp[i];
+    for (int i = tid; i < KP; i += kThreads) sp.in_ang[su * K2 + k0 + i] = ang[i];
     // the state leaving it
     const size_t f = ((size_t)b * L + (size_t)s * Ls) * H + hh;  // its first token
     const float mu = (1.f - ldv<T>(a.lam, f)) * ldv<T>(a.dt, f);
     const float decay = expf(red[s]);
-    const float* lh = sp.loc_h + su * NP;
-    constexpr int kMaxPer = 16;  // (pair, column) steps per thread: NP / 2 / 256 <= 16 (N <= 128, P = 64)
+    const float* lh = sp.loc_h + su * NP + row0 * P;
+    constexpr int kMaxPer = 4;  // (pair, column) steps per thread: KP P / 256 <= 4 (N <= 128, P = 64)
     float l0v[kMaxPer], l1v[kMaxPer];
 #pragma unroll
     for (int j = 0; j < kMaxPer; ++j) {  // every load of the segment's state before any use
       const int i = tid + j * kThreads;
-      if (i < NP / 2) {
+      if (i < KP * P) {
         const int k = i / P, p = i % P;
         l0v[j] = lh[(2 * k) * P + p];
         l1v[j] = lh[(2 * k + 1) * P + p];
@@ -93,15 +109,15 @@ __global__ void __launch_bounds__(kThreads) seg_combine_kernel(const SegParams s
 #pragma unroll
     for (int j = 0; j < kMaxPer; ++j) {  // one (pair k, column p) per step
       const int i = tid + j * kThreads;
-      if (i < NP / 2) {
+      if (i < KP * P) {
         const int k = i / P, p = i % P;
         float sn, cs;
         sincosf(ang[k], &sn, &cs);
         float c0 = h[(2 * k) * P + p], c1 = h[(2 * k + 1) * P + p];
         for (int r = 0; r < R; ++r) {
           const float xr = mu * xp[r * P + p];
-          c0 += bp[r * N + 2 * k] * xr;
-          c1 += bp[r * N + 2 * k + 1] * xr;
+          c0 += bp[r * rows + 2 * k] * xr;
+          c1 += bp[r * rows + 2 * k + 1] * xr;
         }
         const float l0 = l0v[j], l1 = l1v[j];
         h[(2 * k) * P + p] = decay * c0 + cs * l0 + sn * l1;
@@ -109,24 +125,29 @@ __global__ void __launch_bounds__(kThreads) seg_combine_kernel(const SegParams s
       }
     }
     __syncthreads();  // every thread has read bp, xp, ang of the entering state
-    for (int i = tid; i < R * K2; i += kThreads) {
-      const int r = i / K2, k = i % K2;
+    for (int i = tid; i < R * KP; i += kThreads) {
+      const int r = i / KP, k = i % KP;
       float sn, cs;
       sincosf(ang[k], &sn, &cs);
-      const float l0 = sp.loc_b[su * R * N + r * N + 2 * k], l1 = sp.loc_b[su * R * N + r * N + 2 * k + 1];
-      bp[r * N + 2 * k] = cs * l0 + sn * l1;
-      bp[r * N + 2 * k + 1] = cs * l1 - sn * l0;
+      const float* lb = sp.loc_b + (su * R + r) * N + row0;
+      const float l0 = lb[2 * k], l1 = lb[2 * k + 1];
+      bp[r * rows + 2 * k] = cs * l0 + sn * l1;
+      bp[r * rows + 2 * k + 1] = cs * l1 - sn * l0;
     }
     for (int i = tid; i < R * P; i += kThreads) xp[i] = sp.loc_x[su * R * P + i];
     __syncthreads();  // bp rotated with the entering angle before it moves on
-    for (int i = tid; i < K2; i += kThreads) ang[i] = wrap_angle(ang[i] + sp.loc_ang[su * K2 + i]);
+    for (int i = tid; i < KP; i += kThreads) ang[i] = wrap_angle(ang[i] + sp.loc_ang[su * K2 + k0 + i]);
     __syncthreads();
   }
-  if (a.h_out) {  // the state after the whole sequence
-    for (int i = tid; i < NP; i += kThreads) a.h_out[us * NP + i] = h[i];
-    for (int i = tid; i < R * N; i += kThreads) a.bprev_out[us * R * N + i] = bp[i];
-    for (int i = tid; i < R * P; i += kThreads) a.xprev_out[us * R * P + i] = xp[i];
-    for (int i = tid; i < K2; i += kThreads) a.angle_out[us * K2 + i] = ang[i];
+  if (a.h_out) {  // the state after the whole sequence (this part's rows)
+    for (int i = tid; i < rows * P; i += kThreads) a.h_out[us * NP + row0 * P + i] = h[i];
+    for (int i = tid; i < R * rows; i += kThreads) {
+      const int r = i / rows, n = row0 + i % rows;
+      a.bprev_out[(us * R + r) * N + n] = bp[i];
+    }
+    if (part == 0)
+      for (int i = tid; i < R * P; i += kThreads) a.xprev_out[us * R * P + i] = xp[i];
+    for (int i = tid; i < KP; i += kThreads) a.angle_out[us * K2 + k0 + i] = ang[i];
   }
 }
 
@@ -203,12 +224,14 @@ int launch_scan_segmented(const ScanArgs& a, int S, cudaStream_t s) {
   int rc = launch_seg_state(a1, s);
   if (rc != MAMBA3_OK) return rc;
   // 2. the segments' initial states (and the final state)
-  if (a.N * a.P / 2 > 16 * kThreads) return MAMBA3_ERR_UNSUPPORTED;  // the combine's register prefetch
-  const size_t smem = (per + S) * sizeof(float);
+  // the combine's register prefetch and pair split: K2 a multiple of kSplit, K2 P / kSplit <= 4 x 256
+  if (a.N / 2 % kSplit != 0 || a.N / 2 / kSplit * a.P > 4 * kThreads) return MAMBA3_ERR_UNSUPPORTED;
+  const int kp = a.N / 2 / kSplit;
+  const size_t smem = ((size_t)2 * kp * a.P + (size_t)a.R * 2 * kp + (size_t)a.R * a.P + kp + S) * sizeof(float);
   auto kc = a.dtype == MAMBA3_F32 ? seg_combine_kernel<float> : seg_combine_kernel<__nv_bfloat16>;
   if (smem > 48 * 1024 && cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
-  kc<<<a.batch * a.nheads, kThreads, smem, s>>>(sp);
+  kc<<<a.batch * a.nheads * kSplit, kThreads, smem, s>>>(sp);
   if (cudaGetLastError() != cudaSuccess) return MAMBA3_ERR_CUDA;
   // 3. the prefill of every segment from its initial state
   ScanArgs a3 = a;

@@ -45,8 +45,9 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
-// NST stages of inputs: 3 where they fit, so that a stage is refilled two chunks
-// after its MMA was issued (no wait on the MMA just issued); else 2.
+// NST stages of inputs (up to 4, as many as fit); chunk c + D is loaded while chunk
+// c is prepared (D = NST - 2 with 4 stages, else 1), so a load has D chunks to land
+// and the stage it refills was last read by the MMA of chunk c + D - NST.
 template <int N, int R>
 struct GCfg {
   static constexpr int Q = kM / R;
@@ -58,7 +59,10 @@ struct GCfg {
   static constexpr int OFF_X = NKB * kTile;
   static constexpr int OFF_TH = OFF_X + kTile;
   static constexpr int STAGE = OFF_TH + ((TH_BYTES + 1023) & ~1023);
-  static constexpr int NST = 3 * STAGE + 2 * kTile + 16384 <= 232448 - 1024 ? 3 : 2;
+  static constexpr int NST = 4 * STAGE + 2 * kTile + 16384 <= 232448 - 1024
+                                 ? 4
+                                 : (3 * STAGE + 2 * kTile + 16384 <= 232448 - 1024 ? 3 : 2);
+  static constexpr int D = NST == 4 ? 2 : 1;  // prefetch distance in chunks
   static constexpr int OFF_XW = NST * STAGE;            // two X_w buffers
   static constexpr int OFF_PHI = OFF_XW + 2 * kTile;    // final angle [K2]
   static constexpr int OFF_RED = OFF_PHI + K2 * 4;      // [8] warp sums, [8] scan carries
@@ -75,7 +79,7 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
                                                              const __grid_constant__ CUtensorMap tmT,
                                                              const ScanArgs a) {
   using K = GCfg<N, R>;
-  constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, NST = K::NST;
+  constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, NST = K::NST, D = K::D;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -124,10 +128,8 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
     tma_load_4d(st + K::OFF_TH, &tmT, &bars[s], 0, hh, t0, b);
   };
   int issued = 0;
-  if (tid == 0 && !a.test_withhold && nchunks > 0) {
-    issue(0);
-    issued = 1;
-  }
+  if (tid == 0 && !a.test_withhold)
+    for (; issued < D && issued < nchunks; ++issued) issue(issued);
 
   // the segment's total log2 decay (block reduction over its tokens)
   float tot = 0.f;
@@ -181,17 +183,16 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
   for (int c = 0; c < nchunks; ++c) {
     const int s = c % NST;
     uint8_t* st = smem + s * K::STAGE;
-    // load chunk c + 1 into the stage of chunk c + 1 - NST once that chunk's MMA has read
-    // it (with 3 stages an MMA issued two chunks ago; it also frees X_w buffer c % 2)
+    // load chunk c + D into the stage of chunk c + D - NST once that chunk's MMA has read it
     if (tid == 0) {
       bool ok = true;
-      const int prev = c + 1 - NST;
+      const int prev = c + D - NST;
       if (prev >= 0)
         ok = mbar_wait(&bars[NST + prev % NST], (prev / NST) & 1, abort_flag, status, kTagMma, a.wait_limit);
-      if (ok && c + 1 < nchunks && !a.test_withhold) {
+      if (ok && c + D < nchunks && !a.test_withhold) {
         fence_proxy_async_smem();
-        issue(c + 1);
-        issued = c + 2;
+        issue(c + D);
+        issued = c + D + 1;
       }
     }
     float dt[TPL + 1], lm[TPL + 1], at[TPL];
