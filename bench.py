@@ -60,8 +60,8 @@ TRAFFIC = {
     "grouped_decode": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), None, None,
                        "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "backward": (("scan_bwd_tc.cu", "sm100_ptx.cuh", "common.cuh"),
-                 "102786ae686331920255c43fbf04e4b921fc2386f49a0bc6719d4b8521bbd60f",
-                 541828864 + 240547840 + 1219436032 + 783431168,
+                 "79638a3c4e6edd16f5c6e844ddb97329b8bc3671680078e2e467b90ccba7bda7",
+                 541843200 + 242738176 + 1218750208 + 788295680,
                  "profiles/scan_bwd_tc_siso_b8_l2048_traffic_and_counters.txt"),
     "gated_norm_per_head": (("gated_norm.cu", "common.cuh"), "eb90ad7d72a2607cc062684461d599cc86e5eea7058c9d970afd24eac530e380", 268479232 + 103046400,
                             "profiles/gated_norm_b8_l2048_traffic_and_counters.txt"),

@@ -72,6 +72,19 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
+// 16 TMEM lanes, two 8-column halves: threads 0..15 read lanes base .. base + 15 at
+// columns [col, col + 8), threads 16..31 the same lanes at [col + 8, col + 16) -- the
+// layout that lets every lane of a warp carry a row of an M = 64 accumulator (whose
+// rows sit in lanes 0..15 of each 32-lane quadrant)
+__device__ __forceinline__ void tmem_ld_16x2(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], 8;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // per-token scalar arrays in shared memory ([kNScal][kScalStride] floats)
 enum Scal {
   sDt = 0, sLam, sAt, sC2, sGam, sW, sE, sF, sZin, sZue, sDg, sCZu, sRT, sDth, sEend, sSpare
@@ -544,7 +557,9 @@ __global__ void __launch_bounds__(kCThreads, 1)
   // geometry: M = 64 accumulators (row m, valid on lanes 0..15), N x 64 (state row n)
   const int quad = warp & 3, sl = warp >> 2;
   const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-  const bool vrow = lane < 16;
+  // M = 64 accumulators through tmem_ld_16x2: every lane carries row m, half selects
+  // the 8-column half of the warp's 16-column slice
+  const int half = lane >> 4;
   const int m = 16 * quad + (lane & 15);
   const int tm = m / R, rm = m % R;
   const int n = (N == 128) ? quad * 32 + lane : (lane < 16 ? quad * 16 + lane : -1);
@@ -791,23 +806,24 @@ __global__ void __launch_bounds__(kCThreads, 1)
     }
     tc_fence_after();
 
-    // ---- epilogue A: S, W (bf16 tiles), token sums, BG scaled by f, G update ----
+    // ---- epilogue A: S, W (bf16 tiles), token sums, G update ----
     {
       const float* c2 = sc + sC2 * kScalStride;
       const float* wv = sc + sW * kScalStride;
       const float c2m = c2[tm], gam_m = sc[sGam * kScalStride + tm];
-      float p1[16], p2[16];
-      tmem_ld16(tmem + lane_base + K::kColP1 + p0, p1);
-      tmem_ld16(tmem + lane_base + K::kColP2 + p0, p2);
+      const int c0 = 16 * sl + 8 * half;  // this thread's 8 columns of P1, P2
+      float p1[8], p2[8];
+      tmem_ld_16x2(tmem + lane_base + K::kColP1 + 16 * sl, p1);
+      tmem_ld_16x2(tmem + lane_base + K::kColP2 + 16 * sl, p2);
       tmem_ld_wait();
-      float z_diag = 0.f, z_row = 0.f, colz[16];
-      uint32_t sp[8], wp[8];
+      float z_diag = 0.f, z_row = 0.f, colz[8];
+      uint32_t sp[4], wp[4];
 #pragma unroll
-      for (int jj = 0; jj < 16; jj += 2) {
+      for (int jj = 0; jj < 8; jj += 2) {
         float sv[2], wvv[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int j = p0 + jj + e, tj = j / R;
+          const int j = c0 + jj + e, tj = j / R;
           const float q = p1[jj + e] * p2[jj + e];
           float kf = 0.f, ez = 0.f;
           if (tj < tm) {
@@ -818,85 +834,73 @@ __global__ void __launch_bounds__(kCThreads, 1)
             kf = gam_m;
             z_diag += q;
           }
-          colz[jj + e] = vrow ? ez * q : 0.f;
+          colz[jj + e] = ez * q;
           sv[e] = kf * p1[jj + e] + (j == m ? Dh : 0.f);
           wvv[e] = kf * p2[jj + e];
-          if (j == m && vrow) dD_acc += p2[jj + e];
+          if (j == m) dD_acc += p2[jj + e];
         }
         sp[jj / 2] = pack_bf16(sv[0], sv[1]);
         wp[jj / 2] = pack_bf16(wvv[0], wvv[1]);
       }
-      if (vrow) {
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          *reinterpret_cast<uint4*>(smem + K::OFF_S + swz(m, p0 / 8 + h2)) =
-              make_uint4(sp[4 * h2], sp[4 * h2 + 1], sp[4 * h2 + 2], sp[4 * h2 + 3]);
-          *reinterpret_cast<uint4*>(smem + K::OFF_W + swz(m, p0 / 8 + h2)) =
-              make_uint4(wp[4 * h2], wp[4 * h2 + 1], wp[4 * h2 + 2], wp[4 * h2 + 3]);
-        }
+      *reinterpret_cast<uint4*>(smem + K::OFF_S + swz(m, c0 / 8)) = make_uint4(sp[0], sp[1], sp[2], sp[3]);
+      *reinterpret_cast<uint4*>(smem + K::OFF_W + swz(m, c0 / 8)) = make_uint4(wp[0], wp[1], wp[2], wp[3]);
+      // the two halves hold the same row
+      z_diag += __shfl_xor_sync(0xffffffffu, z_diag, 16);
+      z_row += __shfl_xor_sync(0xffffffffu, z_row, 16);
+      if (half == 0) {
         atomicAdd(&sc[sDg * kScalStride + tm], z_diag);
         atomicAdd(&sc[sRT * kScalStride + tm], z_row);
       }
-      // column sums over the 16 rows of this warp (lanes 16..31 carry zeros)
+      // column sums over the 16 rows of each half
       float mine = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
+      for (int jj = 0; jj < 8; ++jj) {
         float v = colz[jj];
         v += __shfl_xor_sync(0xffffffffu, v, 8);
         v += __shfl_xor_sync(0xffffffffu, v, 4);
         v += __shfl_xor_sync(0xffffffffu, v, 2);
         v += __shfl_xor_sync(0xffffffffu, v, 1);
-        if (lane == jj) mine = v;
+        if ((lane & 15) == jj) mine = v;
       }
-      if (vrow && mine != 0.f) atomicAdd(&sc[sCZu * kScalStride + (p0 + lane) / R], mine);
+      if ((lane & 15) < 8 && mine != 0.f) atomicAdd(&sc[sCZu * kScalStride + (c0 + (lane & 15)) / R], mine);
 
-      // zin: sum_n C~[m][n] dC~1[m][n] over this thread's N / 4 columns
+      // zin: sum_n C~[m][n] dC~1[m][n] over the warp's N / 4 columns (8 per thread and piece)
       {
-        constexpr int NC = N / 4;
-        const int n0 = NC * sl;
+        constexpr int NCW = N / 4;
         float zin = 0.f;
 #pragma unroll
-        for (int pc = 0; pc < NC / 16; ++pc) {
-          float dc[16];
-          tmem_ld16(tmem + lane_base + K::kColDC + n0 + 16 * pc, dc);
+        for (int pc = 0; pc < NCW / 16; ++pc) {
+          const int cb = NCW * sl + 16 * pc;
+          float dc[8];
+          tmem_ld_16x2(tmem + lane_base + K::kColDC + cb, dc);
           tmem_ld_wait();
-          const int nn = n0 + 16 * pc;
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const uint4 cq = *reinterpret_cast<const uint4*>(st + K::OFF_C + (nn / 64) * kBlk +
-                                                              swz(m, (nn % 64) / 8 + h2));
-            const uint32_t cw[4] = {cq.x, cq.y, cq.z, cq.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float2 cv = unpack_bf16(cw[k]);
-              zin += cv.x * dc[8 * h2 + 2 * k] + cv.y * dc[8 * h2 + 2 * k + 1];
-            }
-          }
-        }
-        if (vrow) atomicAdd(&sc[sZin * kScalStride + tm], zin);
-      }
-      // zue: e^{cum_end - cum} sum_p X[m][p] (B~ G)[m][p]; then B~ G scaled by f in place
-      {
-        float bg[16];
-        tmem_ld16(tmem + lane_base + K::kColDX + p0, bg);
-        tmem_ld_wait();
-        float zue = 0.f;
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const uint4 xq = *reinterpret_cast<const uint4*>(st + K::OFF_X + swz(m, p0 / 8 + h2));
-          const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+          const int nn = cb + 8 * half;
+          const uint4 cq = *reinterpret_cast<const uint4*>(st + K::OFF_C + (nn / 64) * kBlk + swz(m, (nn % 64) / 8));
+          const uint32_t cw[4] = {cq.x, cq.y, cq.z, cq.w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const float2 xv = unpack_bf16(xw[k]);
-            zue += xv.x * bg[8 * h2 + 2 * k] + xv.y * bg[8 * h2 + 2 * k + 1];
+            const float2 cv = unpack_bf16(cw[k]);
+            zin += cv.x * dc[2 * k] + cv.y * dc[2 * k + 1];
           }
         }
-        if (vrow) atomicAdd(&sc[sZue * kScalStride + tm], zue * sc[sEend * kScalStride + tm]);
-        const float f = sc[sF * kScalStride + tm];
-        uint32_t o[16];
+        zin += __shfl_xor_sync(0xffffffffu, zin, 16);
+        if (half == 0) atomicAdd(&sc[sZin * kScalStride + tm], zin);
+      }
+      // zue: e^{cum_end - cum} sum_p X[m][p] (B~ G)[m][p] (B~ G is scaled by f in epilogue B)
+      {
+        float bg[8];
+        tmem_ld_16x2(tmem + lane_base + K::kColDX + 16 * sl, bg);
+        tmem_ld_wait();
+        const uint4 xq = *reinterpret_cast<const uint4*>(st + K::OFF_X + swz(m, (16 * sl + 8 * half) / 8));
+        const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+        float zue = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(f * bg[i]);
-        tmem_st16(tmem + lane_base + K::kColDX + p0, o);
+        for (int k = 0; k < 4; ++k) {
+          const float2 xv = unpack_bf16(xw[k]);
+          zue += xv.x * bg[2 * k] + xv.y * bg[2 * k + 1];
+        }
+        zue += __shfl_xor_sync(0xffffffffu, zue, 16);
+        if (half == 0) atomicAdd(&sc[sZue * kScalStride + tm], zue * sc[sEend * kScalStride + tm]);
       }
       // G <- e^{cum_end} G + C~^T dY_e; <hbar_in, G_out> for the decay of every token
       {
@@ -925,7 +929,6 @@ __global__ void __launch_bounds__(kCThreads, 1)
         store_G();
       }
     }
-    tmem_st_wait();
     tc_fence_before();
     fence_proxy_async_smem();
     __syncthreads();
@@ -937,15 +940,15 @@ __global__ void __launch_bounds__(kCThreads, 1)
       const uint32_t cS = smem_u32(smem + K::OFF_S), cW = smem_u32(smem + K::OFF_W);
       const uint32_t iWB = idesc_bf16(kM, N, 0, 1);    // W B~      (A K-major, B MN-major)
       const uint32_t iWC = idesc_bf16(kM, N, 1, 1);    // W^T C~    (both MN-major)
-      const uint32_t iSY = idesc_bf16(kM, kP, 1, 1);   // S^T dY    (both MN-major)
+      const uint32_t iSY = idesc_bf16(kM, kP, 1, 1);   // S^T dY    (both MN-major; into P1's columns)
 #pragma unroll
       for (int kk = 0; kk < kM / 16; ++kk) {
         mma_bf16_ss(tmem + K::kColDC, smem_desc_sw128(cW + kk * 32, 16, 1024),
                     smem_desc_sw128(cB + kk * 2048, kBlk, 1024), iWB, 1u);
         mma_bf16_ss(tmem + K::kColDB, smem_desc_sw128(cW + kk * 2048, kBlk, 1024),
                     smem_desc_sw128(cC + kk * 2048, kBlk, 1024), iWC, 1u);
-        mma_bf16_ss(tmem + K::kColDX, smem_desc_sw128(cS + kk * 2048, kBlk, 1024),
-                    smem_desc_sw128(cY + kk * 2048, kBlk, 1024), iSY, 1u);
+        mma_bf16_ss(tmem + K::kColP1, smem_desc_sw128(cS + kk * 2048, kBlk, 1024),
+                    smem_desc_sw128(cY + kk * 2048, kBlk, 1024), iSY, kk > 0 ? 1u : 0u);
       }
       mma_commit(&bars[3]);
     }
@@ -956,56 +959,59 @@ __global__ void __launch_bounds__(kCThreads, 1)
     }
     tc_fence_after();
 
-    // ---- epilogue B: dX; dB~, dC~ rotated back by +Phi; the angle gradient per token ----
+    // ---- epilogue B: dX = f B~G + S^T dY; dB~, dC~ rotated back by +Phi; the angle gradient ----
     {
       const int t = t0 + tm;
-      const bool store = vrow && t < L;
+      const bool store = t < L;
       const bool last = (t == L - 1);
       {
-        float dx[16];
-        tmem_ld16(tmem + lane_base + K::kColDX + p0, dx);
+        float bg[8], sx[8];
+        tmem_ld_16x2(tmem + lane_base + K::kColDX + 16 * sl, bg);
+        tmem_ld_16x2(tmem + lane_base + K::kColP1 + 16 * sl, sx);
         tmem_ld_wait();
+        const float f = sc[sF * kScalStride + tm];
+        const int c0 = 16 * sl + 8 * half;
+        float dx[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dx[i] = f * bg[i] + sx[i];
         if (last && g.dxprev_out) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) dx[i] += g.dxprev_out[((size_t)unit * R + rm) * kP + p0 + i];
+          for (int i = 0; i < 8; ++i) dx[i] += g.dxprev_out[((size_t)unit * R + rm) * kP + c0 + i];
         }
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(dXg + (tok_index(a, b, t, hh) * R + rm) * kP + p0);
-          dst[0] = make_uint4(pack_bf16(dx[0], dx[1]), pack_bf16(dx[2], dx[3]), pack_bf16(dx[4], dx[5]),
-                              pack_bf16(dx[6], dx[7]));
-          dst[1] = make_uint4(pack_bf16(dx[8], dx[9]), pack_bf16(dx[10], dx[11]), pack_bf16(dx[12], dx[13]),
-                              pack_bf16(dx[14], dx[15]));
-        }
+        if (store)
+          *reinterpret_cast<uint4*>(dXg + (tok_index(a, b, t, hh) * R + rm) * kP + c0) =
+              make_uint4(pack_bf16(dx[0], dx[1]), pack_bf16(dx[2], dx[3]), pack_bf16(dx[4], dx[5]),
+                         pack_bf16(dx[6], dx[7]));
       }
-      constexpr int NC = N / 4;
+      constexpr int NCW = N / 4;
 #pragma unroll 1
-      for (int pc = 0; pc < NC / 16; ++pc) {
-        const int nn = NC * sl + 16 * pc;  // first of 16 state columns (8 pairs)
-        float dc[16], db[16];
-        tmem_ld16(tmem + lane_base + K::kColDC + nn, dc);
-        tmem_ld16(tmem + lane_base + K::kColDB + nn, db);
+      for (int pc = 0; pc < NCW / 16; ++pc) {
+        const int cb = NCW * sl + 16 * pc;
+        const int nn = cb + 8 * half;  // this thread's 8 state columns (4 pairs)
+        float dc[8], db[8];
+        tmem_ld_16x2(tmem + lane_base + K::kColDC + cb, dc);
+        tmem_ld_16x2(tmem + lane_base + K::kColDB + cb, db);
         tmem_ld_wait();
         if (last && g.dbprev_out) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) db[i] += g.dbprev_out[((size_t)unit * R + rm) * N + nn + i];
+          for (int i = 0; i < 8; ++i) db[i] += g.dbprev_out[((size_t)unit * R + rm) * N + nn + i];
         }
-        float bt[16], ct[16];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const uint32_t off = (nn / 64) * kBlk + swz(m, (nn % 64) / 8 + h2);
+        float bt[8], ct[8];
+        {
+          const uint32_t off = (nn / 64) * kBlk + swz(m, (nn % 64) / 8);
           const uint4 bq = *reinterpret_cast<const uint4*>(st + K::OFF_B + off);
           const uint4 cq = *reinterpret_cast<const uint4*>(st + K::OFF_C + off);
           const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w}, cw[4] = {cq.x, cq.y, cq.z, cq.w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const float2 bv = unpack_bf16(bw[k]), cv = unpack_bf16(cw[k]);
-            bt[8 * h2 + 2 * k] = bv.x; bt[8 * h2 + 2 * k + 1] = bv.y;
-            ct[8 * h2 + 2 * k] = cv.x; ct[8 * h2 + 2 * k + 1] = cv.y;
+            bt[2 * k] = bv.x; bt[2 * k + 1] = bv.y;
+            ct[2 * k] = cv.x; ct[2 * k + 1] = cv.y;
           }
         }
-        float dph[8], ob[16], oc[16];
+        float dph[4], ob[8], oc[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
           const float db0 = db[2 * i], db1 = db[2 * i + 1], dc0 = dc[2 * i], dc1 = dc[2 * i + 1];
           dph[i] = db0 * bt[2 * i + 1] - db1 * bt[2 * i] + dc0 * ct[2 * i + 1] - dc1 * ct[2 * i];
           float sn, cs;
@@ -1019,36 +1025,28 @@ __global__ void __launch_bounds__(kCThreads, 1)
           if constexpr (GRP) {  // shared rows: this head's share, summed over the group in fp32
             const size_t gi = ((((size_t)b * L + t) * a.ngroups + gh) * R + rm) * N + nn;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 8; ++i) {
               atomicAdd(g.dBh + gi + i, ob[i]);
               atomicAdd(g.dCh + gi + i, oc[i]);
             }
           } else {
             const size_t gi = (tok_index(a, b, t, hh) * R + rm) * N + nn;
-            uint4* pb = reinterpret_cast<uint4*>(dBg + gi);
-            uint4* pcq = reinterpret_cast<uint4*>(dCg + gi);
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              pb[h2] = make_uint4(pack_bf16(ob[8 * h2], ob[8 * h2 + 1]), pack_bf16(ob[8 * h2 + 2], ob[8 * h2 + 3]),
-                                  pack_bf16(ob[8 * h2 + 4], ob[8 * h2 + 5]), pack_bf16(ob[8 * h2 + 6], ob[8 * h2 + 7]));
-              pcq[h2] = make_uint4(pack_bf16(oc[8 * h2], oc[8 * h2 + 1]), pack_bf16(oc[8 * h2 + 2], oc[8 * h2 + 3]),
-                                   pack_bf16(oc[8 * h2 + 4], oc[8 * h2 + 5]), pack_bf16(oc[8 * h2 + 6], oc[8 * h2 + 7]));
-            }
+            *reinterpret_cast<uint4*>(dBg + gi) = make_uint4(pack_bf16(ob[0], ob[1]), pack_bf16(ob[2], ob[3]),
+                                                             pack_bf16(ob[4], ob[5]), pack_bf16(ob[6], ob[7]));
+            *reinterpret_cast<uint4*>(dCg + gi) = make_uint4(pack_bf16(oc[0], oc[1]), pack_bf16(oc[2], oc[3]),
+                                                             pack_bf16(oc[4], oc[5]), pack_bf16(oc[6], oc[7]));
           }
         }
-        // the angle gradient of the token: sum over its R rows (consecutive lanes)
+        // the angle gradient of the token: sum over its R rows (consecutive lanes of a half)
 #pragma unroll
         for (int o = 1; o < R; o <<= 1)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dph[i] += __shfl_xor_sync(0xffffffffu, dph[i], o);
-        if (vrow && rm == 0) {  // row tm, pairs XOR-swizzled by the row (see dphi_at)
-          const int sw = (tm & 7) << 2;
-          *reinterpret_cast<float4*>(dphi_s + tm * K2 + ((nn / 2) ^ sw)) = make_float4(dph[0], dph[1], dph[2], dph[3]);
-          *reinterpret_cast<float4*>(dphi_s + tm * K2 + ((nn / 2 + 4) ^ sw)) =
-              make_float4(dph[4], dph[5], dph[6], dph[7]);
-        }
+          for (int i = 0; i < 4; ++i) dph[i] += __shfl_xor_sync(0xffffffffu, dph[i], o);
+        if (rm == 0)  // row tm, pairs XOR-swizzled by the row (see dphi_at)
+          *reinterpret_cast<float4*>(dphi_s + dphi_at(tm, nn / 2)) = make_float4(dph[0], dph[1], dph[2], dph[3]);
       }
     }
+    tc_fence_before();  // P1, DC, DB, DX are rewritten by the next chunk's first batch
     __syncthreads();
 
     // ---- the angle gradient summed from the end: dtheta = dt S, and sum_k theta S per token ----
