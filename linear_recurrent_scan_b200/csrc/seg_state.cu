@@ -11,8 +11,10 @@
 // token's next one lies outside the segment: w = gamma).  Every 128-row chunk adds
 // B~^T X_w (K = 128) to ONE TMEM accumulator, with X_w = diag(e^{cum_end - cum} w)
 // X weighted to the segment's end: no per-chunk epilogue, so the MMAs run behind
-// the chunk preparation (decay prefix, angles, RoPE of B in place, X_w) through a
-// 3-stage TMA ring (2 where shared memory is short).  cum_end - cum_s is the difference of two fp32 sums over the
+// the chunk preparation (decay prefix, angles, RoPE of B in place, X_w written over
+// X in place) through a TMA ring of 3-5 stages; where three stages fit in half an
+// SM's shared memory, two CTAs share the SM and hide each other's waits.
+// cum_end - cum_s is the difference of two fp32 sums over the
 // segment (<= 1.6 per token here), a relative error near 1e-4 in the weight; a
 // weight that underflows belongs to a term below fp32 resolution.
 // 256 threads; at the end the accumulator becomes h (fp32), with the B of the
@@ -45,9 +47,10 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
-// NST stages of inputs (up to 4, as many as fit); chunk c + D is loaded while chunk
-// c is prepared (D = NST - 2 with 4 stages, else 1), so a load has D chunks to land
-// and the stage it refills was last read by the MMA of chunk c + D - NST.
+// NST stages of inputs; chunk c + NST - 1 is loaded in the middle of chunk c, into the
+// stage that the MMA of chunk c - 1 read.  Two CTAs per SM with three stages where
+// they fit in half of the SM's 228 KB (less 1 KB per CTA), else one CTA with as many
+// stages (up to 5) as fit.
 template <int N, int R>
 struct GCfg {
   static constexpr int Q = kM / R;
@@ -56,25 +59,25 @@ struct GCfg {
   static constexpr int NG = K2 / 4;                     // 16-byte groups of a row
   static constexpr int TH_BYTES = Q * K2 * 2;
   static constexpr int OFF_B = 0;
-  static constexpr int OFF_X = NKB * kTile;
+  static constexpr int OFF_X = NKB * kTile;             // X, then X_w in place
   static constexpr int OFF_TH = OFF_X + kTile;
   static constexpr int STAGE = OFF_TH + ((TH_BYTES + 1023) & ~1023);
-  static constexpr int NST = 4 * STAGE + 2 * kTile + 16384 <= 232448 - 1024
-                                 ? 4
-                                 : (3 * STAGE + 2 * kTile + 16384 <= 232448 - 1024 ? 3 : 2);
-  static constexpr int D = NST == 4 ? 2 : 1;  // prefetch distance in chunks
-  static constexpr int OFF_XW = NST * STAGE;            // two X_w buffers
-  static constexpr int OFF_PHI = OFF_XW + 2 * kTile;    // final angle [K2]
-  static constexpr int OFF_RED = OFF_PHI + K2 * 4;      // [8] warp sums, [8] scan carries
+  static constexpr int TAIL = 1024;                     // final angle, sums, barriers, misc
+  static constexpr int fit(int st) { return st * STAGE + TAIL + 1024; }
+  static constexpr int CPS = fit(3) <= 233472 / 2 - 1024 ? 2 : 1;  // CTAs per SM
+  static constexpr int NST = CPS == 2 ? 3 : (fit(5) <= 232448 ? 5 : (fit(4) <= 232448 ? 4 : (fit(3) <= 232448 ? 3 : 2)));
+  static constexpr int D = NST - 1;                     // chunks loaded ahead
+  static constexpr int OFF_PHI = NST * STAGE;           // final angle [K2]
+  static constexpr int OFF_RED = OFF_PHI + K2 * 4;      // [8] warp sums
   static constexpr int OFF_BAR = (OFF_RED + 64 + 7) & ~7;  // full[NST], mma[NST]
-  static constexpr int OFF_MISC = OFF_BAR + 64;
+  static constexpr int OFF_MISC = OFF_BAR + 2 * NST * 8;
   static constexpr int SMEM = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
-  static_assert(SMEM_ALLOC <= 232448, "shared memory");
+  static_assert(SMEM - OFF_PHI <= TAIL && SMEM_ALLOC <= 232448 && NST >= 2, "shared memory");
 };
 
 template <int N, int R, bool TVA>
-__global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_constant__ CUtensorMap tmB,
+__global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(const __grid_constant__ CUtensorMap tmB,
                                                              const __grid_constant__ CUtensorMap tmX,
                                                              const __grid_constant__ CUtensorMap tmT,
                                                              const ScanArgs a) {
@@ -183,18 +186,6 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
   for (int c = 0; c < nchunks; ++c) {
     const int s = c % NST;
     uint8_t* st = smem + s * K::STAGE;
-    // load chunk c + D into the stage of chunk c + D - NST once that chunk's MMA has read it
-    if (tid == 0) {
-      bool ok = true;
-      const int prev = c + D - NST;
-      if (prev >= 0)
-        ok = mbar_wait(&bars[NST + prev % NST], (prev / NST) & 1, abort_flag, status, kTagMma, a.wait_limit);
-      if (ok && c + D < nchunks && !a.test_withhold) {
-        fence_proxy_async_smem();
-        issue(c + D);
-        issued = c + D + 1;
-      }
-    }
     float dt[TPL + 1], lm[TPL + 1], at[TPL];
 #pragma unroll
     for (int i = 0; i <= TPL; ++i) {
@@ -281,11 +272,20 @@ __global__ void __launch_bounds__(kThreads) seg_state_kernel(const __grid_consta
         }
       }
     }
-    // X_w = diag(f) X into X_w buffer c % 2, once its last reader, the MMA of chunk
-    // c - 2, has completed: warp w writes rows 16 w .. 16 w + 15; the weight of row m is
-    // token m / R's f, held by lane (m / R) / TPL
-    if (c >= 2) mbar_wait(&bars[NST + (c - 2) % NST], ((c - 2) / NST) & 1, abort_flag, status, kTagMma, a.wait_limit);
-    uint8_t* xw = smem + K::OFF_XW + (c & 1) * kTile;
+    // load chunk c + D into the stage of chunk c - 1 once that chunk's MMA has read it
+    if (tid == 0 && c + D < nchunks && !a.test_withhold) {
+      const int prev = c + D - NST;
+      if (prev < 0 ||
+          mbar_wait(&bars[NST + prev % NST], (prev / NST) & 1, abort_flag, status, kTagMma, a.wait_limit)) {
+        fence_proxy_async_smem();
+        issue(c + D);
+        issued = c + D + 1;
+      }
+    }
+    // X_w = diag(f) X over X in place (each thread rewrites the 16-byte pieces it
+    // read): warp w writes rows 16 w .. 16 w + 15; the weight of row m is token m / R's
+    // f, held by lane (m / R) / TPL
+    uint8_t* xw = st + K::OFF_X;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int u = warp * 128 + lane + 32 * i;
@@ -391,7 +391,8 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
       !make_theta_map(&tmT, a, Q))
     return MAMBA3_ERR_CUDA;
   auto k = seg_state_kernel<N, R, TVA>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess)
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess ||
+      cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
   k<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmX, tmT, a);
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
