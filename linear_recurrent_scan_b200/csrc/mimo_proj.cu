@@ -15,12 +15,14 @@
 //
 // Persistent CTAs (one or two per SM) each take an even share of the (head,
 // 128-token tile) work items in head order.  Warp 4 (one lane) loads each head's
-// weight tile into one of two buffers as the CTA's items reach that head, streams
-// the token tiles through a 2-stage TMA ring and issues one MMA chain per tile
-// into one of two TMEM accumulators;
+// weight tile as the CTA's items reach that head (two buffers where they fit),
+// streams the token tiles (and, with the gate, the z tiles) through 2-stage TMA
+// rings and issues one MMA chain per tile into one of two TMEM accumulators;
 // warps 0..3 (one TMEM lane quadrant each, thread = token row) drain the other
-// accumulator: fp32 -> (norm, gate) -> bf16 -> 16-byte stores.  The work is
-// HBM-bound (about 50 FLOP per byte at R = 4, against a ridge near 250).
+// accumulator: fp32 -> (norm, gate) -> bf16 into a 128-byte-swizzled staging tile
+// per 64 output columns, which one thread writes out with a TMA store (rows past
+// the last token are clipped by the tensor map).  The work is HBM-bound (about 50
+// FLOP per byte at R = 4, against a ridge near 250).
 // Every wait is bounded; on expiry the CTA records MAMBA3_ERR_TIMEOUT in the
 // library's status word, lets what it issued land, frees TMEM and returns.
 #include <cuda.h>
@@ -51,9 +53,7 @@ struct ProjParams {
   long long tokens;  // batch * seqlen
   int nheads, tiles;  // tiles of 128 tokens per head; work item = head * tiles + tile
   long long items;    // nheads * tiles, split evenly over the grid
-  void* out;               // x [T, H, R, P] (up) or o [T, H, P] (down), bf16
-  const void* z;           // down: gate [T, H, P] bf16, or null (no norm, no gate)
-  const float* w;          // down with gate: norm weight [H, P] or null (1)
+  const float* w;          // down with the gate: norm weight [H, P] or null (1)
   float eps;
   long long wait_limit;
   int test_withhold;
@@ -61,15 +61,22 @@ struct ProjParams {
 
 // UP: A = u tile [128 x 64], B = Wx[h] [R P x 64]      -> D [128 x R P]
 // DOWN: A = y tile [128 x R P] (R P / 64 blocks), B = Wy[h] [64 x R P] -> D [128 x 64]
-template <int R, bool UP>
+template <int R, bool UP, bool GATE>
 struct PCfg {
   static constexpr int KB = UP ? 1 : R;                   // 64-wide K blocks
   static constexpr int NOUT = UP ? R * kP : kP;           // accumulator columns
+  static constexpr int NB = NOUT / 64;                    // 64-column output blocks
   static constexpr int IN_BYTES = KB * kRows * 128;       // one token tile
-  static constexpr int W_BYTES = UP ? R * kP * 128 : R * kP * 128;  // (R P rows x 128 B) or (64 rows x R blocks)
-  static constexpr int OFF_W = 0;                         // two weight buffers (heads alternate)
-  static constexpr int OFF_IN = OFF_W + 2 * W_BYTES;
-  static constexpr int OFF_BAR = OFF_IN + 2 * IN_BYTES;   // full[2], empty[2], accf[2], acce[2], wfull[2]
+  static constexpr int W_BYTES = R * kP * 128;            // (R P rows x 128 B) or (64 rows x R blocks)
+  static constexpr int Z_BYTES = GATE ? kRows * 128 : 0;  // one gate tile
+  static constexpr int OUT_BYTES = NB * kRows * 128;      // staging of one output tile
+  static constexpr int fit(int nwb) { return nwb * W_BYTES + 2 * IN_BYTES + 2 * Z_BYTES + OUT_BYTES + 256 + 1024; }
+  static constexpr int NWB = fit(2) <= 232448 ? 2 : 1;   // weight buffers (heads alternate)
+  static constexpr int OFF_W = 0;
+  static constexpr int OFF_IN = OFF_W + NWB * W_BYTES;
+  static constexpr int OFF_Z = OFF_IN + 2 * IN_BYTES;
+  static constexpr int OFF_OUT = OFF_Z + 2 * Z_BYTES;
+  static constexpr int OFF_BAR = OFF_OUT + OUT_BYTES;     // full, empty, accf, acce, w, zf, ze: [2] each
   static constexpr int OFF_MISC = OFF_BAR + 128;
   static constexpr int SMEM = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
@@ -78,11 +85,30 @@ struct PCfg {
   static_assert(NOUT <= 256, "one MMA per tile");
 };
 
-enum { bFull = 0, bEmpty = 2, bAccF = 4, bAccE = 6, bW = 8 };
+enum { bFull = 0, bEmpty = 2, bAccF = 4, bAccE = 6, bW = 8, bZF = 10, bZE = 12 };
+
+// named barrier over the 128 epilogue threads (id 1) that also ORs a predicate, so
+// that every epilogue thread takes the same decision
+__device__ __forceinline__ bool epi_sync_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// byte offset of 16-byte chunk `c` (0..7) of row `row` inside a 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t swz(int row, int c) { return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4)); }
 
 // The CTA's work items [i0, i1) of the flattened (head, tile) space; the heads
 // they span are its head segments k = 0, 1, ... (head = item / tiles), each using
-// weight buffer k % 2.
+// weight buffer k % NWB.
 struct ItemRange {
   long long i0, i1;
   int h0;
@@ -98,8 +124,11 @@ __device__ __forceinline__ ItemRange item_range(const ProjParams& p) {
 template <int R, bool UP, bool GATE>
 __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_constant__ CUtensorMap tmIn,
                                                              const __grid_constant__ CUtensorMap tmW,
+                                                             const __grid_constant__ CUtensorMap tmOut,
+                                                             const __grid_constant__ CUtensorMap tmZ,
                                                              const ProjParams prm) {
-  using K = PCfg<R, UP>;
+  using K = PCfg<R, UP, GATE>;
+  constexpr int NWB = K::NWB;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -122,12 +151,16 @@ __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_consta
       mbar_init(&bars[bAccF + i], 1);
       mbar_init(&bars[bAccE + i], 128);
       mbar_init(&bars[bW + i], 1);
+      mbar_init(&bars[bZF + i], 1);
+      mbar_init(&bars[bZE + i], 128);
     }
     *abort_flag = 0;
     *mma_done = 0;
     fence_mbar_init();
     prefetch_tmap(&tmIn);
     prefetch_tmap(&tmW);
+    prefetch_tmap(&tmOut);
+    if (GATE) prefetch_tmap(&tmZ);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, K::TMEM_COLS);
@@ -140,22 +173,29 @@ __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_consta
 
   if (warp == 4) {
     if (lane == 0) {
-      // ---- producer and MMA issuer: inputs through a 2-stage ring, the weights of
-      // head segment k into buffer k % 2 once segment k - 2's MMAs are complete ----
-      int loaded = 0, done = 0;        // items whose loads / MMAs were issued
-      int wseg = 0;                    // head segments whose weights were issued
-      int last_of_slot[2] = {-1, -1};  // last item whose MMA read each weight buffer
+      // ---- producer and MMA issuer: inputs (and gate tiles) through 2-stage rings,
+      // the weights of head segment k into buffer k % NWB once segment k - NWB's
+      // MMAs are complete ----
+      int loaded = 0, done = 0, zl = 0;  // items whose loads / MMAs / gate loads were issued
+      int wseg = 0;                      // head segments whose weights were issued
+      // the CTA's last item of head segment k
+      auto seg_last = [&](int k) {
+        const long long e = (long long)(rg.h0 + k + 1) * prm.tiles - rg.i0;
+        return (int)(e < n ? e : n) - 1;
+      };
       const uint32_t idesc = idesc_bf16(kRows, K::NOUT, 0, 0);
       bool ok = true;
       long long t_last = clock64();
-      while (ok && done < n) {
+      // (the gate tiles follow the epilogue, so they can still be due after the last MMA)
+      while (ok && (done < n || (GATE && zl < n))) {
         bool progress = false;
         // weights of the next head segment, once its buffer is free
         const int seg_needed = head_of(loaded < n ? loaded : n - 1) - rg.h0;
         if (!prm.test_withhold && wseg <= seg_needed && wseg <= head_of(n - 1) - rg.h0) {
-          const int slot = wseg & 1, prev = last_of_slot[slot];
-          // buffer free once segment wseg - 2's last MMA has completed
-          if (prev < *mma_done) {
+          const int slot = wseg % NWB;
+          // buffer free once the MMA of segment wseg - NWB's last item has completed
+          // (every item of that segment, not only those issued so far)
+          if (wseg < NWB || seg_last(wseg - NWB) < *mma_done) {
             const int h = rg.h0 + wseg;
             uint8_t* wb = smem + K::OFF_W + slot * K::W_BYTES;
             mbar_arrive_expect_tx(&bars[bW + slot], K::W_BYTES);
@@ -182,12 +222,21 @@ __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_consta
           ++loaded;
           progress = true;
         }
+        // gate tile of item `zl` into slot zl & 1 once the epilogue of item zl - 2 has read it
+        if (GATE && !prm.test_withhold && zl < n &&
+            (zl < 2 || mbar_test(&bars[bZE + (zl & 1)], ((zl >> 1) - 1) & 1))) {
+          const int s = zl & 1;
+          mbar_arrive_expect_tx(&bars[bZF + s], K::Z_BYTES);
+          tma_load_3d(smem + K::OFF_Z + s * K::Z_BYTES, &tmZ, &bars[bZF + s], 0, head_of(zl), tile_of(zl) * kRows);
+          ++zl;
+          progress = true;
+        }
         // MMA of item `done`: inputs landed, accumulator free, its head's weights loaded
         if (done < loaded) {
-          const int seg = head_of(done) - rg.h0, slot = seg & 1;
+          const int seg = head_of(done) - rg.h0, slot = seg % NWB;
           if (seg < wseg && mbar_test(&bars[bFull + (done & 1)], (done >> 1) & 1) &&
               (done < 2 || mbar_test(&bars[bAccE + (done & 1)], ((done >> 1) - 1) & 1)) &&
-              mbar_test(&bars[bW + slot], (seg >> 1) & 1)) {
+              mbar_test(&bars[bW + slot], (seg / NWB) & 1)) {
             tc_fence_after();
             const int s = done & 1;
             const uint32_t cIn = smem_u32(smem + K::OFF_IN + s * K::IN_BYTES);
@@ -202,7 +251,6 @@ __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_consta
             }
             mma_commit(&bars[bEmpty + s]);
             mma_commit(&bars[bAccF + s]);
-            last_of_slot[slot] = done;
             ++done;
             progress = true;
           }
@@ -219,78 +267,79 @@ __global__ void __launch_bounds__(kThreads) mimo_proj_kernel(const __grid_consta
         }
       }
       // let the copies and MMAs issued land before TMEM is freed and the CTA exits
-      for (int k = (wseg >= 2 ? wseg - 2 : 0); k < wseg; ++k)
-        if (!mbar_wait_drain(&bars[bW + (k & 1)], (k >> 1) & 1)) report_timeout(&g_proj_status, 32);
+      for (int k = (wseg >= NWB ? wseg - NWB : 0); k < wseg; ++k)
+        if (!mbar_wait_drain(&bars[bW + (k % NWB)], (k / NWB) & 1)) report_timeout(&g_proj_status, 32);
       for (int i = done; i < loaded; ++i)
         if (!mbar_wait_drain(&bars[bFull + (i & 1)], (i >> 1) & 1)) report_timeout(&g_proj_status, 32);
+      if (GATE)  // gate tiles not yet waited for by the epilogue (at most the last two)
+        for (int i = (zl >= 2 ? zl - 2 : 0); i < zl; ++i)
+          if (!mbar_wait_drain(&bars[bZF + (i & 1)], (i >> 1) & 1)) report_timeout(&g_proj_status, 32);
       if (done > 0 && !mbar_wait_drain(&bars[bAccF + ((done - 1) & 1)], ((done - 1) >> 1) & 1))
         report_timeout(&g_proj_status, 32);
     }
   } else {
-    // ---- epilogue: warp w reads TMEM lanes 32 w .. 32 w + 31 (thread = token row) ----
+    // ---- epilogue: warp w reads TMEM lanes 32 w .. 32 w + 31 (thread = token row m) ----
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(prm.out);
+    const int m = warp * 32 + lane;
     for (int i = 0; i < n; ++i) {
       const int s = i & 1;
-      if (!mbar_wait(&bars[bAccF + s], (i >> 1) & 1, abort_flag, &g_proj_status, 33, prm.wait_limit)) break;
+      bool ok = mbar_wait(&bars[bAccF + s], (i >> 1) & 1, abort_flag, &g_proj_status, 33, prm.wait_limit);
+      if (GATE && ok) ok = mbar_wait(&bars[bZF + s], (i >> 1) & 1, abort_flag, &g_proj_status, 34, prm.wait_limit);
+      if (epi_sync_any(!ok || *abort_flag != 0)) break;  // one decision for all epilogue threads
       tc_fence_after();
       if (tid == 0) *mma_done = i + 1;  // MMA i (and every earlier one) has completed
-      const int h = head_of(i);
-      const long long tok = (long long)tile_of(i) * kRows + warp * 32 + lane;
-      const bool valid = tok < prm.tokens;
+      const int h = head_of(i), row0 = tile_of(i) * kRows;
       const uint32_t tacc = tmem + lane_base + (uint32_t)(s * K::NOUT);
-      if constexpr (UP) {
-        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(valid ? tok : 0) * prm.nheads + h) * (R * kP));
 #pragma unroll 1
-        for (int c = 0; c < K::NOUT / 32; ++c) {
-          float v[32];
-          tmem_ld32(tacc + 32 * c, v);
-          tmem_ld_wait();
-          if (valid) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[4 * c + q] = make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                                          pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
-          }
-        }
-      } else {
+      for (int k = 0; k < K::NB; ++k) {
         float v[64];
-        tmem_ld32(tacc, v);
-        tmem_ld32(tacc + 32, v + 32);
+        tmem_ld32(tacc + 64 * k, v);
+        tmem_ld32(tacc + 64 * k + 32, v + 32);
         tmem_ld_wait();
-        if (GATE) {
+        if (k == K::NB - 1) {  // the accumulator is free for the MMA of item i + 2
+          tc_fence_before();
+          mbar_arrive(&bars[bAccE + s]);
+        }
+        if constexpr (GATE) {
           float ms = 0.f;
 #pragma unroll
           for (int p = 0; p < 64; ++p) ms += v[p] * v[p];
           const float var = ms * (1.f / kP) + prm.eps;
           const float inv = var > 0.f ? rsqrtf(var) : 0.f;  // an all-zero row with eps = 0 gives 0
-          const uint4* zr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(prm.z) +
-                                                          ((size_t)(valid ? tok : 0) * prm.nheads + h) * kP);
+          const uint8_t* zt = smem + K::OFF_Z + s * K::Z_BYTES;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const uint4 zq = valid ? zr[q] : make_uint4(0, 0, 0, 0);
+            const uint4 zq = *reinterpret_cast<const uint4*>(zt + swz(m, q));
             const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float z0 = __uint_as_float(zw[k] << 16), z1 = __uint_as_float(zw[k] & 0xffff0000u);
-              const int p = 8 * q + 2 * k;
+            for (int kk = 0; kk < 4; ++kk) {
+              const float z0 = __uint_as_float(zw[kk] << 16), z1 = __uint_as_float(zw[kk] & 0xffff0000u);
+              const int p = 8 * q + 2 * kk;
               const float w0 = prm.w ? prm.w[h * kP + p] : 1.f, w1 = prm.w ? prm.w[h * kP + p + 1] : 1.f;
               v[p] = v[p] * inv * w0 * __fdividef(z0, 1.f + __expf(-z0));
               v[p + 1] = v[p + 1] * inv * w1 * __fdividef(z1, 1.f + __expf(-z1));
             }
           }
+          mbar_arrive(&bars[bZE + s]);  // every value read from the gate tile is consumed above
         }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)tok * prm.nheads + h) * kP);
+        // staging block k is free once the store that last read it (item i - 1) has
+        uint8_t* stg = smem + K::OFF_OUT + k * kRows * 128;
+        if (tid == 0) bulk_wait_read<K::NB - 1>();
+        epi_sync();
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                                pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4*>(stg + swz(m, q)) =
+              make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                         pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+        fence_proxy_async_smem();
+        epi_sync();
+        if (tid == 0) {
+          tma_store_3d(&tmOut, stg, 64 * k, h, row0);
+          bulk_commit();
         }
       }
-      tc_fence_before();
-      mbar_arrive(&bars[bAccE + s]);
     }
+    if (tid == 0) bulk_wait_all();  // the stores have read the staging tiles and completed
   }
   tc_fence_before();
   __syncthreads();
@@ -315,17 +364,20 @@ bool map3(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d
 
 template <int R, bool UP, bool GATE>
 int launch_k(const ProjArgs& a, cudaStream_t s) {
-  using K = PCfg<R, UP>;
+  using K = PCfg<R, UP, GATE>;
   const long long T = a.tokens;
   const int H = a.nheads;
-  CUtensorMap tmIn, tmW;
+  CUtensorMap tmIn, tmW, tmOut, tmZ;
+  memset(&tmZ, 0, sizeof(tmZ));
   if (UP) {
-    // u [T, H, P]; Wx [H, R P, P]
-    if (!map3(&tmIn, a.in, kP, H, T, 1, kRows) || !map3(&tmW, a.weight, kP, R * kP, H, R * kP, 1))
+    // u [T, H, P]; Wx [H, R P, P]; x [T, H, R P]
+    if (!map3(&tmIn, a.in, kP, H, T, 1, kRows) || !map3(&tmW, a.weight, kP, R * kP, H, R * kP, 1) ||
+        !map3(&tmOut, a.out, R * kP, H, T, 1, kRows))
       return MAMBA3_ERR_CUDA;
   } else {
-    // y [T, H, R P]; Wy [H, P, R P]
-    if (!map3(&tmIn, a.in, R * kP, H, T, 1, kRows) || !map3(&tmW, a.weight, R * kP, kP, H, kP, 1))
+    // y [T, H, R P]; Wy [H, P, R P]; o [T, H, P] (and z [T, H, P])
+    if (!map3(&tmIn, a.in, R * kP, H, T, 1, kRows) || !map3(&tmW, a.weight, R * kP, kP, H, kP, 1) ||
+        !map3(&tmOut, a.out, kP, H, T, 1, kRows) || (GATE && !map3(&tmZ, a.z, kP, H, T, 1, kRows)))
       return MAMBA3_ERR_CUDA;
   }
   ProjParams prm;
@@ -334,21 +386,21 @@ int launch_k(const ProjArgs& a, cudaStream_t s) {
   prm.nheads = H;
   prm.tiles = (int)((T + kRows - 1) / kRows);
   prm.items = (long long)prm.tiles * H;
-  // persistent: one CTA per SM when the two accumulators take all 512 TMEM columns
-  // (the shared memory asked for keeps a second CTA off the SM), else two
-  const int per_sm = K::TMEM_COLS >= 512 ? 1 : 2;
+  // persistent: two CTAs per SM where both fit (TMEM and shared memory), else one;
+  // a CTA that takes all 512 TMEM columns asks for enough shared memory to keep a
+  // second one off the SM
+  const int per_sm = (K::TMEM_COLS <= 256 && K::SMEM_ALLOC <= 233472 / 2 - 1024) ? 2 : 1;
   const long long grid = prm.items < (long long)kSMs * per_sm ? prm.items : (long long)kSMs * per_sm;
-  const int smem = per_sm == 1 && K::SMEM_ALLOC < 120 * 1024 ? 120 * 1024 : K::SMEM_ALLOC;
-  prm.out = a.out;
-  prm.z = a.z;
+  const int smem = K::TMEM_COLS >= 512 && K::SMEM_ALLOC < 120 * 1024 ? 120 * 1024 : K::SMEM_ALLOC;
   prm.w = a.w;
   prm.eps = a.eps;
   prm.wait_limit = a.wait_limit;
   prm.test_withhold = a.test_withhold;
   auto k = mimo_proj_kernel<R, UP, GATE>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
-  k<<<(int)grid, kThreads, smem, s>>>(tmIn, tmW, prm);
+  k<<<(int)grid, kThreads, smem, s>>>(tmIn, tmW, tmOut, tmZ, prm);
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 

@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
   // prefix are warp scans over the lanes, so a chunk needs one block barrier, before
   // its MMA.  Every warp keeps the decay carry and its groups' running angles.
   constexpr int TPL = Q / 32, GPW = NG / (kThreads / 32);
-  static_assert(TPL >= 1 && Q % 32 == 0 && GPW >= 1 && NG % (kThreads / 32) == 0, "lanes and warps");
+  static_assert(TPL >= 1 && Q % 32 == 0 && TPL * R == 4 && GPW >= 1 && NG % (kThreads / 32) == 0, "lanes and warps");
   float p_dt[TPL + 1], p_lm[TPL + 1], p_at[TPL];  // this lane's tokens of the next chunk (+ the one after)
   auto load_scalars = [&](int c) {
 #pragma unroll
@@ -248,28 +248,47 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
         ex[k] = wrap_angle(phw[q][k] + x - tot4[k]);  // angle before this lane's first token
         phw[q][k] = wrap_angle(phw[q][k] + __shfl_sync(0xffffffffu, x, 31));
       }
+      float sn[TPL][4], cs[TPL][4];
 #pragma unroll
-      for (int i = 0; i < TPL; ++i) {
-        const int t = lane * TPL + i;
-        float sn[4], cs[4];
+      for (int i = 0; i < TPL; ++i)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           ex[k] += inc[i][k];
-          __sincosf(ex[k], &sn[k], &cs[k]);
+          __sincosf(ex[k], &sn[i][k], &cs[i][k]);
+        }
+      // The lane's rows are 4 lane .. 4 lane + 3 (TPL R = 4).  Taken in the same order
+      // by every lane, a warp's 32 accesses would fall on 2 of the 8 16-byte columns
+      // of the 128-byte swizzle (row & 7 in {j, j + 4}); starting each lane pair one
+      // row further spreads them over all 8.
+      const int rot = (lane >> 1) & 3;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int jl = (j + rot) & 3, it = jl / R;
+        float s4[4], c4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          s4[k] = sn[0][k];
+          c4[k] = cs[0][k];
         }
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          uint4* p = reinterpret_cast<uint4*>(st + K::OFF_B + kb * kTile + swz(t * R + r, c8));
-          const uint4 qv = *p;
-          const uint32_t bw[4] = {qv.x, qv.y, qv.z, qv.w};
-          uint32_t bo[4];
+        for (int ii = 1; ii < TPL; ++ii)
+          if (it == ii) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 vv = unpack_bf16(bw[k]);
-            bo[k] = pack_bf16(cs[k] * vv.x + sn[k] * vv.y, cs[k] * vv.y - sn[k] * vv.x);
+            for (int k = 0; k < 4; ++k) {
+              s4[k] = sn[ii][k];
+              c4[k] = cs[ii][k];
+            }
           }
-          *p = make_uint4(bo[0], bo[1], bo[2], bo[3]);
+        uint4* p = reinterpret_cast<uint4*>(st + K::OFF_B + kb * kTile + swz(lane * 4 + jl, c8));
+        const uint4 qv = *p;
+        const uint32_t bw[4] = {qv.x, qv.y, qv.z, qv.w};
+        uint32_t bo[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 vv = unpack_bf16(bw[k]);
+          bo[k] = pack_bf16(c4[k] * vv.x + s4[k] * vv.y, c4[k] * vv.y - s4[k] * vv.x);
         }
+        *p = make_uint4(bo[0], bo[1], bo[2], bo[3]);
       }
     }
     // load chunk c + D into the stage of chunk c - 1 once that chunk's MMA has read it

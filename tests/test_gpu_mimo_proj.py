@@ -113,6 +113,29 @@ def test_mimo_layer_up_scan_down_matches_oracle():
     assert rel_err(f64(o), ref) < TOLB
 
 
+@pytest.mark.parametrize("R", [2, 4])
+def test_head_switches_inside_persistent_ctas(R):
+    """512 (head, tile) items on at most 296 persistent CTAs: most CTAs take two or
+    more items and many cross a head boundary, so the weight buffers are reloaded
+    mid-range (the gated R = 4 down projection has a single weight buffer).  Every
+    output row is checked, and the library status stays clean."""
+    b, L, H, P = 1, 8192, 8, 64
+    u = randn((b, L, H, P), 6900 + R)
+    Wx, Wy = weights(H, R, P, 6910 + R)
+    z = randn((b, L, H, P), 6920 + R)
+    w = torch.rand(H, P, device="cuda") + 0.5
+    x = m3.mamba3_mimo_up(u, Wx)
+    o = m3.mamba3_mimo_down(x, Wy)
+    og = m3.mamba3_mimo_down(x, Wy, z=z, w=w)
+    torch.cuda.synchronize()
+    assert m3.mamba3_library_status() == m3.MAMBA3_OK
+    assert rel_err(f64(x), oracle.mimo_up(f64(u), f64(Wx), R)) < TOLB
+    ref = oracle.mimo_down(f64(x), f64(Wy))
+    assert rel_err(f64(o), ref) < TOLB
+    refg = oracle.gated_norm(ref[..., None, :], f64(z)[..., None, :], f64(w)[:, None, :])[..., 0, :]
+    assert rel_err(f64(og), refg) < TOLB
+
+
 def test_full_size_sampled_tokens():
     """MIMO R4 prefill size (b4 L8192 H64): sampled (token, head) rows against the oracle."""
     b, L, H, R, P = 4, 8192, 64, 4, 64
@@ -122,6 +145,7 @@ def test_full_size_sampled_tokens():
     z = randn((b, L, H, P), 6802)
     o = m3.mamba3_mimo_down(x, Wy, z=z)
     torch.cuda.synchronize()
+    assert m3.mamba3_library_status() == m3.MAMBA3_OK
     rows = [(0, 0), (1, 4095), (2, 8191), (3, 77)]
     for bb, t in rows:
         xs = oracle.mimo_up(f64(u[bb, t]), f64(Wx), R)
