@@ -127,7 +127,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 EncodeTiledFn encode_fn();  // cuTensorMapEncodeTiled from the driver, or null
 bool make_map(CUtensorMap* m, const void* base, int inner, int heads, const ScanArgs& a, int Q);
 bool make_dl_map(CUtensorMap* m, const void* base, const ScanArgs& a, int rows);
-bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q);
+bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q, bool swizzle = false);
 
 // Long sequences with few (batch, head) units (scan_seg.cu): segments per unit
 // (0 = run unsegmented), the workspace they need after the status word, and the
@@ -135,6 +135,8 @@ bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q);
 // sequence's end state from a zero state, the segments' aggregates.
 constexpr int kSMs = 148;
 int seg_count(const ScanArgs& a, int sms);
+// CTAs of the segment-state kernel that share an SM for these sizes (1 or 2)
+int seg_state_ctas_per_sm(const ScanArgs& a);
 size_t seg_workspace_bytes(const ScanArgs& a, int S);
 int launch_scan_segmented(const ScanArgs& a, int S, cudaStream_t s);
 int launch_state_export(const ScanArgs& a, cudaStream_t s);

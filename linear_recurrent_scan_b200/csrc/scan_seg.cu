@@ -79,8 +79,43 @@ __global__ void __launch_bounds__(kThreads) seg_combine_kernel(const SegParams s
   for (int i = tid; i < KP; i += kThreads) ang[i] = a.angle0 ? a.angle0[us * K2 + k0 + i] : 0.f;
   __syncthreads();
 
+  // Per thread: its (pair, column) steps of h, and (tid < R KP) one pair of b_prev,
+  // (tid < R P) one x_prev entry, (tid < KP) one angle.  Segment s + 1's aggregates
+  // are loaded while segment s is combined, so the chain waits on no global load.
+  constexpr int kMaxPer = 4;  // (pair, column) steps per thread: KP P / 256 <= 4 (N <= 128, P = 64)
+  struct Agg {
+    float h0[kMaxPer], h1[kMaxPer], b0, b1, x, ang, lam, dt;
+  };
+  auto fetch = [&](int s, Agg& g) {
+    if (s >= S) return;
+    const size_t su = ((size_t)b * S + s) * H + hh;
+    const float* lh = sp.loc_h + su * NP + row0 * P;
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {
+      const int i = tid + j * kThreads;
+      if (i < KP * P) {
+        const int k = i / P, p = i % P;
+        g.h0[j] = lh[(2 * k) * P + p];
+        g.h1[j] = lh[(2 * k + 1) * P + p];
+      }
+    }
+    if (tid < R * KP) {
+      const int r = tid / KP, k = tid % KP;
+      const float* lb = sp.loc_b + (su * R + r) * N + row0;
+      g.b0 = lb[2 * k];
+      g.b1 = lb[2 * k + 1];
+    }
+    if (tid < R * P) g.x = sp.loc_x[su * R * P + tid];
+    if (tid < KP) g.ang = sp.loc_ang[su * K2 + k0 + tid];
+    const size_t f = ((size_t)b * L + (size_t)s * Ls) * H + hh;  // the segment's first token
+    g.lam = ldv<T>(a.lam, f);
+    g.dt = ldv<T>(a.dt, f);
+  };
+  Agg cur, nxt;
+  fetch(0, cur);
   for (int s = 0; s < S; ++s) {
     const size_t su = ((size_t)b * S + s) * H + hh;  // the segment's unit in the b S x H view
+    fetch(s + 1, nxt);
     // the initial state of segment s (this part's rows)
     for (int i = tid; i < rows * P; i += kThreads) sp.in_h[su * NP + row0 * P + i] = h[i];
     for (int i = tid; i < R * rows; i += kThreads) {
@@ -90,22 +125,12 @@ __global__ void __launch_bounds__(kThreads) seg_combine_kernel(const SegParams s
     if (part == 0)
       for (int i = tid; i < R * P; i += kThreads) sp.in_x[su * R * P + i] = xp[i];
     for (int i = tid; i < KP; i += kThreads) sp.in_ang[su * K2 + k0 + i] = ang[i];
+    // the copy above reads h in another thread-to-element map than the update below
+    // writes it: every thread has to finish the copy first
+    __syncthreads();
     // the state leaving it
-    const size_t f = ((size_t)b * L + (size_t)s * Ls) * H + hh;  // its first token
-    const float mu = (1.f - ldv<T>(a.lam, f)) * ldv<T>(a.dt, f);
+    const float mu = (1.f - cur.lam) * cur.dt;
     const float decay = expf(red[s]);
-    const float* lh = sp.loc_h + su * NP + row0 * P;
-    constexpr int kMaxPer = 4;  // (pair, column) steps per thread: KP P / 256 <= 4 (N <= 128, P = 64)
-    float l0v[kMaxPer], l1v[kMaxPer];
-#pragma unroll
-    for (int j = 0; j < kMaxPer; ++j) {  // every load of the segment's state before any use
-      const int i = tid + j * kThreads;
-      if (i < KP * P) {
-        const int k = i / P, p = i % P;
-        l0v[j] = lh[(2 * k) * P + p];
-        l1v[j] = lh[(2 * k + 1) * P + p];
-      }
-    }
 #pragma unroll
     for (int j = 0; j < kMaxPer; ++j) {  // one (pair k, column p) per step
       const int i = tid + j * kThreads;
@@ -119,25 +144,24 @@ __global__ void __launch_bounds__(kThreads) seg_combine_kernel(const SegParams s
           c0 += bp[r * rows + 2 * k] * xr;
           c1 += bp[r * rows + 2 * k + 1] * xr;
         }
-        const float l0 = l0v[j], l1 = l1v[j];
+        const float l0 = cur.h0[j], l1 = cur.h1[j];
         h[(2 * k) * P + p] = decay * c0 + cs * l0 + sn * l1;
         h[(2 * k + 1) * P + p] = decay * c1 + cs * l1 - sn * l0;
       }
     }
     __syncthreads();  // every thread has read bp, xp, ang of the entering state
-    for (int i = tid; i < R * KP; i += kThreads) {
-      const int r = i / KP, k = i % KP;
+    if (tid < R * KP) {
+      const int r = tid / KP, k = tid % KP;
       float sn, cs;
       sincosf(ang[k], &sn, &cs);
-      const float* lb = sp.loc_b + (su * R + r) * N + row0;
-      const float l0 = lb[2 * k], l1 = lb[2 * k + 1];
-      bp[r * rows + 2 * k] = cs * l0 + sn * l1;
-      bp[r * rows + 2 * k + 1] = cs * l1 - sn * l0;
+      bp[r * rows + 2 * k] = cs * cur.b0 + sn * cur.b1;
+      bp[r * rows + 2 * k + 1] = cs * cur.b1 - sn * cur.b0;
     }
-    for (int i = tid; i < R * P; i += kThreads) xp[i] = sp.loc_x[su * R * P + i];
+    if (tid < R * P) xp[tid] = cur.x;
     __syncthreads();  // bp rotated with the entering angle before it moves on
-    for (int i = tid; i < KP; i += kThreads) ang[i] = wrap_angle(ang[i] + sp.loc_ang[su * K2 + k0 + i]);
+    if (tid < KP) ang[tid] = wrap_angle(ang[tid] + cur.ang);
     __syncthreads();
+    cur = nxt;
   }
   if (a.h_out) {  // the state after the whole sequence (this part's rows)
     for (int i = tid; i < rows * P; i += kThreads) a.h_out[us * NP + row0 * P + i] = h[i];
@@ -166,16 +190,22 @@ int seg_count(const ScanArgs& a, int sms) {
   if (tc_scan_supported(a) != MAMBA3_OK || bwd_tc_supported(a) != MAMBA3_OK || a.bcnorm) return 0;
   const long long units = (long long)a.batch * a.nheads;
   if (units >= sms || a.seqlen < 2048) return 0;
+  // Time model: the prefill runs one CTA per SM, the segment-state pass
+  // seg_state_ctas_per_sm; each CTA costs its tokens plus about two chunks of
+  // pipeline fill and drain, the state pass about half as much per token.
+  const double fill = 2.0 * (128 / a.R);
+  const long long slots2 = (long long)sms * seg_state_ctas_per_sm(a);
   int best = 0;
-  double best_eff = 0.0;
+  double best_cost = 0.0;
   for (int S = 2; S <= 64; S *= 2) {
     if (a.seqlen % S != 0 || a.seqlen / S < 1024) break;
     const long long ctas = units * S;
-    const double waves = (double)ctas / sms;
-    const double eff = waves / (double)((ctas + sms - 1) / sms);
-    if (ctas >= sms && eff > best_eff + 1e-9) {
+    if (ctas < sms) continue;
+    const double per = (double)(a.seqlen / S) + fill;
+    const double cost = (double)((ctas + sms - 1) / sms) * per + 0.5 * (double)((ctas + slots2 - 1) / slots2) * per;
+    if (best == 0 || cost < best_cost - 1e-9) {
       best = S;
-      best_eff = eff;
+      best_cost = cost;
     }
   }
   return best;

@@ -98,8 +98,10 @@ bool make_dl_map(CUtensorMap* m, const void* base, const ScanArgs& a, int rows) 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// theta [batch, L, H, N/2] bf16, box = {N/2, 1, Q, 1}, no swizzle, zero fill past the end.
-bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q) {
+// theta [batch, L, H, N/2] bf16, box = {N/2, 1, Q, 1}, zero fill past the end; no
+// swizzle, or (swizzle) the 64-byte (N = 64) or 128-byte (N = 128) pattern, which
+// moves 16-byte chunk c of row t to c ^ ((t >> 1) & 3) or c ^ (t & 7).
+bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q, bool swizzle) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const int K2 = a.N / 2;
@@ -107,8 +109,10 @@ bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q) {
   const cuuint64_t strides[3] = {2ull * K2, 2ull * K2 * a.nheads, 2ull * K2 * a.nheads * a.seqlen};
   const cuuint32_t box[4] = {(cuuint32_t)K2, 1, (cuuint32_t)Q, 1};
   const cuuint32_t es[4] = {1, 1, 1, 1};
+  const CUtensorMapSwizzle sw =
+      !swizzle ? CU_TENSOR_MAP_SWIZZLE_NONE : (K2 == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(a.theta), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

@@ -230,7 +230,11 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
 #pragma unroll
       for (int i = 0; i < TPL; ++i) {
         const int t = lane * TPL + i;
-        const uint2 tv = *reinterpret_cast<const uint2*>(th + t * K2 + 4 * g);
+        // 8 bytes at byte 8 g of row t, through the tile's 64- / 128-byte swizzle (a
+        // warp reads one column of the tile; unswizzled that is a 16-way bank conflict)
+        const int chunk = (g >> 1) ^ (K2 == 32 ? ((t >> 1) & 3) : (t & 7));
+        const uint2 tv = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(th) + t * (2 * K2) +
+                                                         chunk * 16 + (g & 1) * 8);
         const float2 t01 = unpack_bf16(tv.x), t23 = unpack_bf16(tv.y);
         inc[i][0] = dt[i] * t01.x; inc[i][1] = dt[i] * t01.y; inc[i][2] = dt[i] * t23.x; inc[i][3] = dt[i] * t23.y;
 #pragma unroll
@@ -407,7 +411,7 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
   constexpr int Q = K::Q;
   CUtensorMap tmB, tmX, tmT;
   if (!make_map(&tmB, a.B, N, a.ngroups, a, Q) || !make_map(&tmX, a.x, kP, a.nheads, a, Q) ||
-      !make_theta_map(&tmT, a, Q))
+      !make_theta_map(&tmT, a, Q, true))
     return MAMBA3_ERR_CUDA;
   auto k = seg_state_kernel<N, R, TVA>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess ||
@@ -423,6 +427,11 @@ int launch_r(const ScanArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+int seg_state_ctas_per_sm(const ScanArgs& a) {
+  if (a.N == 128) return a.R == 1 ? GCfg<128, 1>::CPS : (a.R == 2 ? GCfg<128, 2>::CPS : GCfg<128, 4>::CPS);
+  return a.R == 1 ? GCfg<64, 1>::CPS : (a.R == 2 ? GCfg<64, 2>::CPS : GCfg<64, 4>::CPS);
+}
 
 int launch_seg_state(const ScanArgs& a, cudaStream_t s) {
   if (bwd_tc_supported(a) != MAMBA3_OK || a.h0 || a.angle0) return MAMBA3_ERR_UNSUPPORTED;

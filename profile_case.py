@@ -6,6 +6,7 @@ passes, output-side norms) of one workload, for profilers.
     python profile_case.py --workload siso_prefill_b8_l2048 --groups 1 --reps 3
     python profile_case.py --workload siso_prefill_b8_l2048 --backward --reps 3
     python profile_case.py --workload siso_prefill_b8_l2048 --gated-norm 64 --reps 3
+    python profile_case.py --workload mimo4_prefill_b4_l8192 --mimo-proj --reps 3
 
 Inputs are seeded synthetic tensors on cuda:0.  Prints the CUDA-event time
 of each call; under a profiler those times are not benchmark numbers.
@@ -33,6 +34,8 @@ def main():
     ap.add_argument("--backward", action="store_true", help="time the prefill's backward pass")
     ap.add_argument("--gated-norm", type=int, default=0, metavar="G",
                     help="time the output side (grouped RMS norm + gate, G norm groups) on a prefill-sized y")
+    ap.add_argument("--mimo-proj", action="store_true",
+                    help="time the rank-R up projection and the gated down projection on the workload's tokens")
     args = ap.parse_args()
     w = wl.CONFIGS[args.workload]
     if args.batch:
@@ -71,6 +74,30 @@ def main():
             e1.record()
             torch.cuda.synchronize()
             print(f"gated norm {w.name} groups {args.gated_norm} rep {i}: {e0.elapsed_time(e1) * 1000:.1f} us")
+        return
+    if args.mimo_proj:
+        g = torch.Generator(device=dev)
+        g.manual_seed(wl.BASE_SEED + 11)
+        P, R, H = w.headdim, w.rank, w.nheads
+        u = torch.randn((w.batch, w.seqlen, H, P), generator=g, device=dev).to(w.dtype)
+        Wx = (torch.randn((H, R * P, P), generator=g, device=dev) * P ** -0.5).to(w.dtype)
+        Wy = (torch.randn((H, P, R * P), generator=g, device=dev) * (R * P) ** -0.5).to(w.dtype)
+        z = torch.randn((w.batch, w.seqlen, H, P), generator=g, device=dev).to(w.dtype)
+        wn = torch.rand((H, P), generator=g, device=dev) + 0.5
+        x = torch.empty((w.batch, w.seqlen, H, R, P), device=dev, dtype=w.dtype)
+        o = torch.empty_like(u)
+        for i in range(args.reps):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            ev[0].record()
+            m3.mamba3_mimo_up(u, Wx, out=x)
+            ev[1].record()
+            m3.mamba3_mimo_down(x, Wy, z=z, w=wn, out=o)
+            ev[2].record()
+            torch.cuda.synchronize()
+            print(f"mimo up {w.name} rep {i}: {ev[0].elapsed_time(ev[1]):.4f} ms; "
+                  f"down (gated) {ev[1].elapsed_time(ev[2]):.4f} ms")
+        if m3.mamba3_library_status() != m3.MAMBA3_OK:
+            raise RuntimeError("library status after the projections is not OK")
         return
     inp = wl.make_inputs(w, device=dev)
     if args.groups:

@@ -116,3 +116,24 @@ def test_library_segments_long_context_with_its_own_workspace_size():
     for n in ("h", "b_prev", "x_prev"):
         a, b = getattr(fins[0], n), getattr(fins[1], n)
         assert rel_err(a.cpu().double().numpy(), b.cpu().double().numpy()) < TOLB, n
+
+
+def test_segmented_long_context_repeats_bit_identically():
+    """The library's segmented prefill at the long-context shape, three times: the
+    outputs must be bit-identical (a race between the combine's state copy and its
+    update showed up as run-to-run differences in some segments' initial states)
+    and match the unsegmented prefill."""
+    w = wl.CONFIGS["mimo4_long_b1_l65536"]
+    inp = wl.make_inputs(w, seed=7500, device="cuda")
+    dims = m3.make_dims(inp["x"], inp["B"])
+    ws = torch.zeros(m3.mamba3_scan_segmented_workspace_bytes(dims), dtype=torch.uint8, device="cuda")
+    ys = []
+    for _ in range(3):
+        ys.append(m3.mamba3_scan_fwd(*(inp[n] for n in NAMES), inp["A"], inp["D"], workspace=ws))
+        assert m3.mamba3_device_status(ws) == m3.MAMBA3_OK
+    y1 = m3.mamba3_scan_fwd(*(inp[n] for n in NAMES), inp["A"], inp["D"],
+                            workspace=torch.zeros(m3.mamba3_scan_workspace_bytes(dims), dtype=torch.uint8,
+                                                  device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
+    assert rel_err(ys[0].float().cpu().double().numpy(), y1.float().cpu().double().numpy()) < TOLB
