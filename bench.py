@@ -43,26 +43,34 @@ BACKWARD_KERNEL = "bwd_state_kernel + bwd_chunk_kernel (tcgen05, TMA)"
 # capture).  A kernel whose sources no longer hash to the recorded value gets
 # traffic null, since its counters are out of date.
 TRAFFIC = {
-    "prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"),
-                "8c7315685dc21c6b771e1d8a843e5fbc2fbd942e638f9df041ae26dd4adc3a9a", 811532288 + 137174784,
+    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'),
+                "8b5271dec5927f08b1e7b62c915f7c4ae4f53d752e17d4080da424d906cfc38c", 811494912 + 137460224,
                 "profiles/scan_tc_prefill_traffic_and_counters.txt"),
-    "mimo4_prefill_b4_l8192": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"),
-                               "8c7315685dc21c6b771e1d8a843e5fbc2fbd942e638f9df041ae26dd4adc3a9a",
-                               5648189440 + 1064534272, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
-    "siso_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                         "33d2df3c2627df690ecd8bd830abc94739f24a010222682500fc194bcbbee128", 283179520 + 219435264,
+    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'),
+                               "8b5271dec5927f08b1e7b62c915f7c4ae4f53d752e17d4080da424d906cfc38c",
+                               5649451264 + 1064985344, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    # the segmented prefill: seg_state_kernel + seg_combine_kernel + scan_tc_kernel of one call
+    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'),
+                             "f55253583dcfacbf3aae2da1a90b4641de93cd57faebf270d296c6a4dac2fff1",
+                             4592843520 + 36670720 + 38104320 + 283904 + 6778004480 + 2125286400,
+                             "profiles/segmented_prefill_mimo4_b1_l65536.txt"),
+    "siso_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'),
+                         "9b747bdffa9f5294aa353dae0a96868654ddfff0f6555cfdc2f3fb571284da7a", 283192832 + 219687936,
                          "profiles/decode_stream_b128_traffic_and_counters.txt"),
-    "mimo4_decode_b128": (("decode.cu", "sm100_ptx.cuh", "common.cuh"),
-                          "33d2df3c2627df690ecd8bd830abc94739f24a010222682500fc194bcbbee128", 317792000 + 240657408,
+    "mimo4_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'),
+                          "9b747bdffa9f5294aa353dae0a96868654ddfff0f6555cfdc2f3fb571284da7a", 317791232 + 240960768,
                           "profiles/decode_stream_b128_traffic_and_counters.txt"),
-    "grouped_prefill": (("scan_tc.cu", "sm100_ptx.cuh", "common.cuh"), None, None,
+    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "8b5271dec5927f08b1e7b62c915f7c4ae4f53d752e17d4080da424d906cfc38c", 284427264 + 114855680,
                         "profiles/grouped_bc_prefill_decode_traffic.txt"),
-    "grouped_decode": (("decode.cu", "sm100_ptx.cuh", "common.cuh"), None, None,
+    "grouped_decode": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9b747bdffa9f5294aa353dae0a96868654ddfff0f6555cfdc2f3fb571284da7a", 279049472 + 219701760,
                        "profiles/grouped_bc_prefill_decode_traffic.txt"),
-    "backward": (("scan_bwd_tc.cu", "sm100_ptx.cuh", "common.cuh"),
-                 "79638a3c4e6edd16f5c6e844ddb97329b8bc3671680078e2e467b90ccba7bda7",
-                 541843200 + 242738176 + 1218750208 + 788295680,
+    "backward": (('scan_bwd_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "a0704efc34dfba0f08202d6146eada4887be9e739a7a24d2bc9260e29e642250",
+                 541863680 + 240075776 + 1218802432 + 788110336,
                  "profiles/scan_bwd_tc_siso_b8_l2048_traffic_and_counters.txt"),
+    "mimo_proj_up": (('mimo_proj.cu', 'sm100_ptx.cuh', 'common.cuh'), "f6bb83215f2fb4b7a8f54d96530b10ab09ad42203469e8fb3e2387e8df3209a2", 406607360 + 1016255488,
+                     "profiles/mimo_proj_b4_l8192_traffic.txt"),
+    "mimo_proj_down_gated": (('mimo_proj.cu', 'sm100_ptx.cuh', 'common.cuh'), "f6bb83215f2fb4b7a8f54d96530b10ab09ad42203469e8fb3e2387e8df3209a2", 1480614656 + 247203840,
+                             "profiles/mimo_proj_b4_l8192_traffic.txt"),
     "gated_norm_per_head": (("gated_norm.cu", "common.cuh"), "eb90ad7d72a2607cc062684461d599cc86e5eea7058c9d970afd24eac530e380", 268479232 + 103046400,
                             "profiles/gated_norm_b8_l2048_traffic_and_counters.txt"),
 }
@@ -599,7 +607,8 @@ def ours(args):
     pw = PREFILL_MORE[0]
     pt = run_mimo_proj(m3, pw, rank, steps=side_steps, warmup=3)
     pb = mimo_proj_bytes(pw)
-    proj = {k: {"ms": round(max_over_ranks(v, world), 4), **rl(pb[k], max_over_ranks(v, world), peak)}
+    proj = {k: {"ms": round(max_over_ranks(v, world), 4),
+                **rl(pb[k], max_over_ranks(v, world), peak, traffic("mimo_proj_" + k))}
             for k, v in pt.items()}
     proj["workload"] = pw.name
     more = {}

@@ -216,9 +216,9 @@ MAMBA3_API int mamba3_decode_step_at(const mamba3_dims* dims, const mamba3_state
  *                 b8 L2048 H64 N128: 272 MB); with grouped B/C then the fp32 sums
  *                 of dB and dC, 2 * batch * seqlen * ngroups * rank * dstate
  *                 floats.  Other shapes (SIMT path): per (b, h) and chunk of
- *                 Q = 32 / rank tokens, N P + N/2 floats; with grouped B/C
- *                 2 * batch * seqlen * nheads * rank * dstate floats of per-head
- *                 gradients.
+ *                 Q = 32 / rank tokens, N P + N/2 floats; with grouped B/C then
+ *                 the same fp32 group sums (2 * batch * seqlen * ngroups * rank *
+ *                 dstate floats; each head adds its share with atomics).
  * Products on the tensor cores take bf16 operands with float32 accumulation;
  * everything else is float32.  Returns MAMBA3_ERR_UNSUPPORTED for N, P whose
  * per-chunk tiles exceed shared memory.

@@ -131,16 +131,15 @@ bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q, bool swizzle = fal
 
 // Long sequences with few (batch, head) units (scan_seg.cu): segments per unit
 // (0 = run unsegmented), the workspace they need after the status word, and the
-// segmented prefill; launch_state_export (scan_bwd_tc.cu) gives every
-// sequence's end state from a zero state, the segments' aggregates.
+// segmented prefill.
 constexpr int kSMs = 148;
 int seg_count(const ScanArgs& a, int sms);
 // CTAs of the segment-state kernel that share an SM for these sizes (1 or 2)
 int seg_state_ctas_per_sm(const ScanArgs& a);
 size_t seg_workspace_bytes(const ScanArgs& a, int S);
 int launch_scan_segmented(const ScanArgs& a, int S, cudaStream_t s);
-int launch_state_export(const ScanArgs& a, cudaStream_t s);
-// The same end states as one streaming tensor-core reduction per sequence (seg_state.cu).
+// Every sequence's end state from a zero state and zero angle (the segments'
+// aggregates), one streaming tensor-core reduction per sequence (seg_state.cu).
 int launch_seg_state(const ScanArgs& a, cudaStream_t s);
 
 int tc_scan_supported(const ScanArgs& a);

@@ -371,7 +371,7 @@ int scan_bwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
   }
   if (m3::bwd_group_bytes(sizes)) {
     g.dBh = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes + ckpt_bytes);
-    g.dCh = g.dBh + (size_t)d->batch * d->seqlen * d->nheads * d->rank * d->dstate;
+    g.dCh = g.dBh + (size_t)d->batch * d->seqlen * bc_groups(d) * d->rank * d->dstate;
   }
   if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
   return m3::launch_scan_bwd(g, s);

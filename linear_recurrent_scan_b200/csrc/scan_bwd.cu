@@ -540,11 +540,12 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
           dphi += db0 * sB[m * NS + 2 * k + 1] - db1 * sB[m * NS + 2 * k] + dc0 * sC[m * NS + 2 * k + 1] -
                   dc1 * sC[m * NS + 2 * k];
           const size_t gi = tok(t0 + i) * R * N + (size_t)r * N + 2 * k;
-          if (g.dBh) {  // grouped: this head's share, summed over the group afterwards
-            g.dBh[gi] = cs * db0 - sn * db1;
-            g.dBh[gi + 1] = sn * db0 + cs * db1;
-            g.dCh[gi] = cs * dc0 - sn * dc1;
-            g.dCh[gi + 1] = sn * dc0 + cs * dc1;
+          if (g.dBh) {  // grouped: this head's share added to the group's fp32 sum
+            const size_t gg = tok_bc(t0 + i) * R * N + (size_t)r * N + 2 * k;
+            atomicAdd(g.dBh + gg, cs * db0 - sn * db1);
+            atomicAdd(g.dBh + gg + 1, sn * db0 + cs * db1);
+            atomicAdd(g.dCh + gg, cs * dc0 - sn * dc1);
+            atomicAdd(g.dCh + gg + 1, sn * dc0 + cs * dc1);
           } else {
             st1(dBg + gi, cs * db0 - sn * db1);
             st1(dBg + gi + 1, sn * db0 + cs * db1);
@@ -660,31 +661,22 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_kernel(BwdArgs g, BwdLay
   }
 }
 
-// dB[b, t, g] = sum of dBh[b, t, h] over the heads h of group g (and dC likewise)
+// dB, dC [b, t, g] in the input dtype from the groups' fp32 sums
 template <typename T>
-__global__ void __launch_bounds__(256) bc_group_sum_kernel(const float* dBh, const float* dCh, T* dB, T* dC,
-                                                           long long total, int groups, int hpg, int rn) {
+__global__ void __launch_bounds__(256) bc_group_convert_kernel(const float* dBs, const float* dCs, T* dB, T* dC,
+                                                               long long total) {
   for (long long e = (long long)blockIdx.x * 256 + threadIdx.x; e < total; e += (long long)gridDim.x * 256) {
-    const long long row = e / rn;  // (b, t, g)
-    const int c = (int)(e % rn);
-    const long long bt = row / groups;
-    const int grp = (int)(row % groups);
-    const size_t base = ((size_t)bt * groups * hpg + (size_t)grp * hpg) * rn + c;
-    float sb = 0.f, sc = 0.f;
-    for (int j = 0; j < hpg; ++j) {
-      sb += dBh[base + (size_t)j * rn];
-      sc += dCh[base + (size_t)j * rn];
-    }
-    st1(dB + e, sb);
-    st1(dC + e, sc);
+    st1(dB + e, dBs[e]);
+    st1(dC + e, dCs[e]);
   }
 }
 
 }  // namespace
 
+// grouped B, C: the fp32 sums of dB and dC over each group's heads, [b, L, G, R, N] each
 size_t bwd_group_bytes(const ScanArgs& a) {
   if (a.ngroups >= a.nheads) return 0;
-  return 2 * (size_t)a.batch * a.seqlen * a.nheads * a.R * a.N * sizeof(float);
+  return 2 * (size_t)a.batch * a.seqlen * a.ngroups * a.R * a.N * sizeof(float);
 }
 
 size_t bwd_checkpoint_bytes(const ScanArgs& a) {
@@ -724,22 +716,19 @@ int launch_scan_bwd(const BwdArgs& g, cudaStream_t s) {
   }
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
+  const long long total = (long long)a.batch * a.seqlen * a.ngroups * a.R * a.N;
+  if (g.dBh && cudaMemsetAsync(g.dBh, 0, bwd_group_bytes(a), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
   k<<<units, kThreads, lay.total, s>>>(g, lay);
   if (cudaGetLastError() != cudaSuccess) return MAMBA3_ERR_CUDA;
-  if (g.dBh) {
-    const long long total = (long long)a.batch * a.seqlen * a.ngroups * a.R * a.N;
-    if (total > 0) {
-      long long blocks = (total + 255) / 256;
-      if (blocks > 148 * 16) blocks = 148 * 16;
-      const int hpg = a.nheads / a.ngroups, rn = a.R * a.N;
-      if (a.dtype == MAMBA3_F32)
-        bc_group_sum_kernel<float><<<(int)blocks, 256, 0, s>>>(g.dBh, g.dCh, static_cast<float*>(g.dB),
-                                                               static_cast<float*>(g.dC), total, a.ngroups, hpg, rn);
-      else
-        bc_group_sum_kernel<__nv_bfloat16><<<(int)blocks, 256, 0, s>>>(
-            g.dBh, g.dCh, static_cast<__nv_bfloat16*>(g.dB), static_cast<__nv_bfloat16*>(g.dC), total, a.ngroups,
-            hpg, rn);
-    }
+  if (g.dBh && total > 0) {
+    long long blocks = (total + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (a.dtype == MAMBA3_F32)
+      bc_group_convert_kernel<float><<<(int)blocks, 256, 0, s>>>(g.dBh, g.dCh, static_cast<float*>(g.dB),
+                                                                 static_cast<float*>(g.dC), total);
+    else
+      bc_group_convert_kernel<__nv_bfloat16><<<(int)blocks, 256, 0, s>>>(
+          g.dBh, g.dCh, static_cast<__nv_bfloat16*>(g.dB), static_cast<__nv_bfloat16*>(g.dC), total);
   }
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }

@@ -140,10 +140,7 @@ struct SCfg : BCfg<N, R> {
   static_assert(SMEM_ALLOC <= 232448, "shared memory");
 };
 
-// EXP: instead of the checkpoints, export the state at the end of the sequence
-// (h, the rotated B of the last token, its x, the angle) to a.h_out, a.bprev_out,
-// a.xprev_out, a.angle_out: the segment aggregate of the long-sequence prefill.
-template <int N, int R, bool TVA, bool EXP>
+template <int N, int R, bool TVA>
 __global__ void __launch_bounds__(kSThreads) bwd_state_kernel(const __grid_constant__ CUtensorMap tmB,
                                                               const __grid_constant__ CUtensorMap tmX,
                                                               const __grid_constant__ CUtensorMap tmT,
@@ -260,7 +257,7 @@ __global__ void __launch_bounds__(kSThreads) bwd_state_kernel(const __grid_const
     load_scalars(c + 1);
     // checkpoint of the chunk start: the bf16 state tile image and the angle
     uint8_t* ck = ckpt + (ck_unit + c) * (size_t)K::HB_BYTES;
-    if (!EXP && n >= 0) {
+    if (n >= 0) {
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint4 q;
@@ -271,7 +268,7 @@ __global__ void __launch_bounds__(kSThreads) bwd_state_kernel(const __grid_const
         *reinterpret_cast<uint4*>(ck + swz(n, 4 * half + q4)) = q;
       }
     }
-    if (!EXP && tid < K2) {
+    if (tid < K2) {
       float* ckphi = reinterpret_cast<float*>(ckpt + (size_t)gridDim.x * nchunks * K::HB_BYTES) + (ck_unit + c) * K2;
       ckphi[tid] = phi[tid];
     }
@@ -399,28 +396,6 @@ __global__ void __launch_bounds__(kSThreads) bwd_state_kernel(const __grid_const
     }
     tc_fence_before();
     __syncthreads();  // stage s, X_w and the scalars may be reused
-  }
-  if (EXP && abort_c < 0 && L > 0) {
-    // the state after the last token (w of the last token is gamma: no next token)
-    if (n >= 0) {
-      float* ho = a.h_out + ((size_t)unit * N + n) * kP + 32 * half;
-#pragma unroll
-      for (int p = 0; p < 32; p += 4) *reinterpret_cast<float4*>(ho + p) = make_float4(hb[p], hb[p + 1], hb[p + 2], hb[p + 3]);
-    }
-    const size_t il = tok_index(a, b, L - 1, hh);
-    const size_t ib = ((size_t)b * L + (L - 1)) * a.ngroups + gh;
-    const __nv_bfloat16* Bl = static_cast<const __nv_bfloat16*>(a.B) + ib * R * N;
-    const __nv_bfloat16* Xl = static_cast<const __nv_bfloat16*>(a.x) + il * R * kP;
-    for (int i = tid; i < R * K2; i += kSThreads) {  // B of the last token rotated by its angle, in fp32
-      const int r = i / K2, k = i % K2;
-      float sn, cs;
-      sincosf(phi[k], &sn, &cs);
-      const float b0 = __bfloat162float(Bl[r * N + 2 * k]), b1 = __bfloat162float(Bl[r * N + 2 * k + 1]);
-      a.bprev_out[((size_t)unit * R + r) * N + 2 * k] = cs * b0 + sn * b1;
-      a.bprev_out[((size_t)unit * R + r) * N + 2 * k + 1] = cs * b1 - sn * b0;
-    }
-    for (int i = tid; i < R * kP; i += kSThreads) a.xprev_out[(size_t)unit * R * kP + i] = __bfloat162float(Xl[i]);
-    if (tid < K2) a.angle_out[(size_t)unit * K2 + tid] = phi[tid];
   }
   if (abort_c >= 0 && tid == 0) {
     // Let what was issued land before TMEM is freed and the CTA exits: the loads of
@@ -1243,7 +1218,7 @@ int launch_nr(const BwdArgs& g, cudaStream_t s) {
       !make_map(&tmX, a.x, kP, a.nheads, a, Q) || !make_map(&tmDY, g.dy, kP, a.nheads, a, Q) ||
       !make_theta_map(&tmT, a, Q))
     return MAMBA3_ERR_CUDA;
-  auto ks = bwd_state_kernel<N, R, TVA, false>;
+  auto ks = bwd_state_kernel<N, R, TVA>;
   auto kc = bwd_chunk_kernel<N, R, TVA, GRP>;
   if (cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, SK::SMEM_ALLOC) != cudaSuccess ||
       cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, CK::SMEM_ALLOC) != cudaSuccess)
@@ -1270,45 +1245,7 @@ int launch_r(const BwdArgs& g, cudaStream_t s) {
   return grp ? launch_nr<N, R, false, true>(g, s) : launch_nr<N, R, false, false>(g, s);
 }
 
-template <int N, int R, bool TVA>
-int launch_state_export_nr(const ScanArgs& a, cudaStream_t s) {
-  using SK = SCfg<N, R>;
-  constexpr int Q = BCfg<N, R>::Q;
-  const int nchunks = (a.seqlen + Q - 1) / Q;
-  CUtensorMap tmB, tmX, tmT;
-  if (!make_map(&tmB, a.B, N, a.ngroups, a, Q) || !make_map(&tmX, a.x, kP, a.nheads, a, Q) ||
-      !make_theta_map(&tmT, a, Q))
-    return MAMBA3_ERR_CUDA;
-  auto ks = bwd_state_kernel<N, R, TVA, true>;
-  if (cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, SK::SMEM_ALLOC) != cudaSuccess)
-    return MAMBA3_ERR_CUDA;
-  ks<<<a.batch * a.nheads, kSThreads, SK::SMEM_ALLOC, s>>>(tmB, tmX, tmT, a, nullptr, nchunks);
-  return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
-}
-
-template <int N, int R>
-int launch_state_export_r(const ScanArgs& a, cudaStream_t s) {
-  return a.A_t ? launch_state_export_nr<N, R, true>(a, s) : launch_state_export_nr<N, R, false>(a, s);
-}
-
 }  // namespace
-
-// The state at the end of every (batch, head) sequence of `a` from its own zero
-// state and zero angle (a.h0 .. a.angle0 null), written to a.h_out .. a.angle_out;
-// the same shapes as the tensor-core backward.
-int launch_state_export(const ScanArgs& a, cudaStream_t s) {
-  if (bwd_tc_supported(a) != MAMBA3_OK || a.h0 || a.angle0) return MAMBA3_ERR_UNSUPPORTED;
-  if (a.N == 128) {
-    if (a.R == 1) return launch_state_export_r<128, 1>(a, s);
-    if (a.R == 2) return launch_state_export_r<128, 2>(a, s);
-    if (a.R == 4) return launch_state_export_r<128, 4>(a, s);
-  } else {
-    if (a.R == 1) return launch_state_export_r<64, 1>(a, s);
-    if (a.R == 2) return launch_state_export_r<64, 2>(a, s);
-    if (a.R == 4) return launch_state_export_r<64, 4>(a, s);
-  }
-  return MAMBA3_ERR_UNSUPPORTED;
-}
 
 int bwd_tc_supported(const ScanArgs& a) {
   if (a.dtype != MAMBA3_BF16 || a.P != kP || a.seqlen < 1 || a.bcnorm) return MAMBA3_ERR_UNSUPPORTED;

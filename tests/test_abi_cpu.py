@@ -257,9 +257,9 @@ def test_backward_host_validation(lib):
     assert bwd(lib, d, ws_bytes=need - 1) == m3.MAMBA3_ERR_WORKSPACE
     assert bwd(lib, d, ws=FAKE + 8) == m3.MAMBA3_ERR_WORKSPACE
     assert bwd(lib, d, {"dB": FAKE + 4}) == m3.MAMBA3_ERR_INVALID
-    # grouped B/C: the per-head B, C gradients (2 x b L H R N fp32) come on top of the checkpoints
+    # grouped B/C: the groups' fp32 sums of dB, dC (2 x b L G R N, here G = 1) come on top of the checkpoints
     dg = dims(ngroups=1)
-    assert lib.mamba3_scan_bwd_workspace_bytes(ctypes.byref(dg)) == need + 2 * 2 * 64 * 3 * 1 * 16 * 4
+    assert lib.mamba3_scan_bwd_workspace_bytes(ctypes.byref(dg)) == need + 2 * 2 * 64 * 1 * 1 * 16 * 4
     assert bwd(lib, dg, ws_bytes=need) == m3.MAMBA3_ERR_WORKSPACE
     assert bwd(lib, dims(dstate=256, headdim=128)) == m3.MAMBA3_ERR_UNSUPPORTED  # tiles beyond shared memory
     assert lib.mamba3_scan_bwd_workspace_bytes(ctypes.byref(dims(rank=3))) == 0
