@@ -137,7 +137,10 @@ constexpr uint32_t kColS = 0, kColP = 128, kColY = 192, kColYi = 256, kColH = 32
 
 enum Tag { kTagEmpty = 1, kTagFull, kTagPrep1, kTagSFull, kTagAcc, kTagEpiDone, kTagP, kTagY, kTagDrain, kTagTh };
 
-template <int N, int R>
+// kernel variants: the plain recurrence, the fused B/C norm, the time-varying decay A_t
+enum Variant { kPlain = 0, kBCNorm = 1, kTimeA = 2 };
+
+template <int N, int R, int V>
 struct Cfg {
   static constexpr int Q = kM / R;     // tokens per chunk
   static constexpr int NKB = N / 64;   // 64-wide blocks of the state dimension
@@ -172,13 +175,19 @@ struct Cfg {
   static constexpr int DL_PAD = (DL_BYTES + 127) & ~127;
   static constexpr int OFF_DL = (OFF_MISC + 16 + 127) & ~127;
   static constexpr int OFF_SINK = OFF_DL + 2 * DL_PAD;  // [Q] floats: consumes the tile reads
-  // fused B/C normalisation: w_B, bias_B, w_C, bias_C of this head, [R][N] floats
-  // each; or, with a time-varying decay by TMA (the two are never combined), the
-  // A_t tile [Q][8] bf16 (refilled with theta)
+  // fused B/C normalisation (V = kBCNorm): w_B, bias_B, w_C, bias_C of this head,
+  // [R][N] floats each; time-varying decay by TMA (V = kTimeA): the A_t tile [Q][8]
+  // bf16 (refilled with theta); nothing for the plain variant
   static constexpr int OFF_NRM = (OFF_SINK + Q * 4 + 127) & ~127;
   static constexpr int AT_BYTES = Q * 16;
-  static constexpr int NRM_BYTES = 4 * R * N * 4 > AT_BYTES ? 4 * R * N * 4 : AT_BYTES;
-  static constexpr int SMEM = OFF_NRM + NRM_BYTES;
+  static constexpr int NRM_BYTES = V == kBCNorm ? 4 * R * N * 4 : (V == kTimeA ? AT_BYTES : 0);
+  // y staging where shared memory allows (N = 64; N = 128 with R = 4 except the
+  // fused norm): per epilogue warp one or two
+  // 32-row x 64-byte tiles (64-byte swizzle) that the warp writes out with a TMA store
+  static constexpr int OFF_Y = (OFF_NRM + NRM_BYTES + 1023) & ~1023;
+  static constexpr int Y_TILE = 32 * 64;
+  static constexpr int YBUF = OFF_Y + 16 * Y_TILE + 1024 <= 232448 ? 2 : (OFF_Y + 8 * Y_TILE + 1024 <= 232448 ? 1 : 0);
+  static constexpr int SMEM = YBUF ? OFF_Y + 8 * YBUF * Y_TILE : OFF_NRM + NRM_BYTES;
   static constexpr int SMEM_ALLOC = SMEM + 1024;       // slack for 1024-byte alignment
   static_assert(NG * NPART == kNPrep && TPP * NPART == Q, "angle partition");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -234,14 +243,11 @@ __device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 256;" ::
 // place (16 bytes per shared-memory access, 2 rows in flight), the rank-1
 // column factors of the mask and X_w.  dt and lam are prefetched one chunk
 // ahead into registers; theta arrives by TMA.
-// kernel variants: the plain recurrence, the fused B/C norm, the time-varying decay A_t
-enum Variant { kPlain = 0, kBCNorm = 1, kTimeA = 2 };
-
 template <int N, int R, int V>
 __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int dl_tma, int b, int hh,
                                           float Ah, uint64_t* bars, volatile int* abort_flag, DeviceStatus* status) {
   constexpr bool BCN = V == kBCNorm, TVA = V == kTimeA;
-  using K = Cfg<N, R>;
+  using K = Cfg<N, R, V>;
   constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, TPP = K::TPP, TB = K::TB, NPART = K::NPART;
   const int pt = threadIdx.x - kPrep0;
   const int L = a.seqlen, H = a.nheads;
@@ -567,15 +573,51 @@ __device__ __forceinline__ void store_y(const ScanArgs& a, uint32_t tY, uint32_t
   }
 }
 
+// The same rows through the warp's staging tile: lane l writes row l's 64 bytes (its
+// 32 columns) into the 64-byte-swizzled 32 x 64 B tile `stg` (16-byte chunk c of row l
+// at c ^ ((l >> 1) & 3), so a store instruction covers all 32 banks), then lane 0
+// writes the tile out with one TMA store of the warp's 32 rows (rows past the sequence
+// are clipped by the tensor map).  The tile is rewritten once the store that last
+// read it has (PENDING younger stores may still be in flight).
+template <int PENDING>
+__device__ __forceinline__ void store_y_tma(const CUtensorMap* tmY, uint8_t* stg, uint32_t tY, uint32_t tYi, float e,
+                                            int b, int hh, int t_first, int ch, int lane) {
+  if (lane == 0) bulk_wait_read<PENDING>();
+  __syncwarp();
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    float yv[16], yi[16];
+    tmem_ld16(tY + 32 * ch + 16 * half, yv);
+    tmem_ld16(tYi + 32 * ch + 16 * half, yi);
+    tmem_ld_wait();
+#pragma unroll
+    for (int q2 = 0; q2 < 2; ++q2) {
+      const int o = 8 * q2, c = 2 * half + q2;
+      uint4 q;
+      q.x = pack_bf16(yv[o + 0] + e * yi[o + 0], yv[o + 1] + e * yi[o + 1]);
+      q.y = pack_bf16(yv[o + 2] + e * yi[o + 2], yv[o + 3] + e * yi[o + 3]);
+      q.z = pack_bf16(yv[o + 4] + e * yi[o + 4], yv[o + 5] + e * yi[o + 5]);
+      q.w = pack_bf16(yv[o + 6] + e * yi[o + 6], yv[o + 7] + e * yi[o + 7]);
+      *reinterpret_cast<uint4*>(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) = q;
+    }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_5d(tmY, stg, 32 * ch, 0, hh, t_first, b);
+    bulk_commit();
+  }
+}
+
 // ------------------------------------------------------------------ epilogue warps
 // Two warps per TMEM lane quadrant: thread = (row m = 32 quad + lane, column
 // half ch).  Row m of S, P, Y, Yi; state row n of Hacc / hbar (for N = 64 the
 // M = 64 accumulator uses lanes 0..15 of each 32-lane quadrant).
-template <int N, int R>
+template <int N, int R, int V>
 __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh,
                                          uint64_t* bars, volatile int* abort_flag, DeviceStatus* status,
-                                         uint32_t tmem) {
-  using K = Cfg<N, R>;
+                                         uint32_t tmem, const CUtensorMap* tmY) {
+  using K = Cfg<N, R, V>;
   constexpr int Q = K::Q;
   const int et = threadIdx.x - kEpi0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -591,6 +633,9 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
   const int tref = (32 * quad) / R;      // first token of this quadrant's rows
   const int colf_off = quad == 1 ? 0 : (quad == 2 ? 32 : 96);
   uint8_t* Hs = smem + K::OFF_H;
+  // (YBUF > 0) this warp's y staging tiles; the first token of its 32 rows in a chunk
+  uint8_t* ystg = smem + K::OFF_Y + (et >> 5) * (K::YBUF > 0 ? K::YBUF : 1) * K::Y_TILE;
+  const int trow = (32 * quad) / R;
 
   // ---- initial carried state hbar_0 = h_0 + (1 - lam_1) dt_1 B~_0^T x_0 (columns of this half) ----
   float hb[32];
@@ -697,14 +742,25 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
 
     // ---- y = Y + e^{cum_t} Yi ----
     if constexpr (K::DEFER_Y) {  // the previous chunk's (its Y MMA completed before this chunk's S)
-      if (c > 0)
-        store_y(a, tmem + lane_base + kColY + ((c - 1) & 1) * kColYBuf,
-                tmem + lane_base + kColYi + ((c - 1) & 1) * kColYBuf, e_prev, b, hh, t0 - Q + tm, rm, R, ch);
+      if (c > 0) {
+        if constexpr (K::YBUF > 0)
+          store_y_tma<K::YBUF - 1>(tmY, ystg + ((c - 1) % K::YBUF) * K::Y_TILE,
+                                   tmem + lane_base + kColY + ((c - 1) & 1) * kColYBuf,
+                                   tmem + lane_base + kColYi + ((c - 1) & 1) * kColYBuf, e_prev, b, hh,
+                                   t0 - Q + trow, ch, lane);
+        else
+          store_y(a, tmem + lane_base + kColY + ((c - 1) & 1) * kColYBuf,
+                  tmem + lane_base + kColYi + ((c - 1) & 1) * kColYBuf, e_prev, b, hh, t0 - Q + tm, rm, R, ch);
+      }
       e_prev = my_e;
     } else {
       mbar_wait(&bars[bYFull], c & 1, abort_flag, status, kTagY, a.wait_limit);
       if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
       tc_fence_after();
+      if constexpr (K::YBUF > 0) {
+        store_y_tma<K::YBUF - 1>(tmY, ystg + (c % K::YBUF) * K::Y_TILE, tmem + lane_base + kColY,
+                                 tmem + lane_base + kColYi, my_e, b, hh, t0 + trow, ch, lane);
+      } else {
       const int tg = t0 + tm;
       uint4* yr = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) +
                                            (tok_index(a, b, tg < L ? tg : 0, hh) * R + rm) * kP + 32 * ch);
@@ -727,6 +783,7 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
           }
         }
       }
+      }
     }
     tc_fence_before();
     fence_proxy_async_smem();  // hbar (bf16) is read by the next chunk's MMA
@@ -737,8 +794,12 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
     tc_fence_after();
     const int cl = nchunks - 1;
-    store_y(a, tmem + lane_base + kColY + (cl & 1) * kColYBuf, tmem + lane_base + kColYi + (cl & 1) * kColYBuf, e_prev,
-            b, hh, cl * Q + tm, rm, R, ch);
+    if constexpr (K::YBUF > 0)
+      store_y_tma<K::YBUF - 1>(tmY, ystg + (cl % K::YBUF) * K::Y_TILE, tmem + lane_base + kColY + (cl & 1) * kColYBuf,
+                               tmem + lane_base + kColYi + (cl & 1) * kColYBuf, e_prev, b, hh, cl * Q + trow, ch, lane);
+    else
+      store_y(a, tmem + lane_base + kColY + (cl & 1) * kColYBuf, tmem + lane_base + kColYi + (cl & 1) * kColYBuf,
+              e_prev, b, hh, cl * Q + tm, rm, R, ch);
     tc_fence_before();
   }
 }
@@ -748,8 +809,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
                    const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmL,
-                   const __grid_constant__ CUtensorMap tmA, const TcParams prm) {
-  using K = Cfg<N, R>;
+                   const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmY,
+                   const TcParams prm) {
+  using K = Cfg<N, R, V>;
   constexpr int Q = K::Q;
   extern __shared__ uint8_t smem_raw[];
   // align to 1024 bytes by offsetting the __shared__ pointer itself, so that the
@@ -927,7 +989,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (tid < kEpi0) {
     prep_role<N, R, V>(smem, a, nchunks, prm.dl_tma, b, hh, a.A ? a.A[hh] : 0.f, bars, abort_flag, status);
   } else {
-    epi_role<N, R>(smem, a, nchunks, b, hh, bars, abort_flag, status, tmem);
+    epi_role<N, R, V>(smem, a, nchunks, b, hh, bars, abort_flag, status, tmem, &tmY);
+    // the y stores issued by this warp have read their staging tiles (and completed)
+    if (K::YBUF > 0 && (tid & 31) == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -939,9 +1003,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host side
+// y [batch, L, H, R, 64] bf16 for the epilogue warps' stores: box = {32, R, 1, 32 / R, 1}
+// (a warp's 32 rows x 32 columns), 64-byte swizzle; rows past the sequence are clipped.
+bool make_y_map(CUtensorMap* m, const ScanArgs& a) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || a.R > 32) return false;
+  const cuuint64_t dims[5] = {(cuuint64_t)kP, (cuuint64_t)a.R, (cuuint64_t)a.nheads, (cuuint64_t)a.seqlen,
+                              (cuuint64_t)a.batch};
+  const cuuint64_t e = 2;
+  const cuuint64_t strides[4] = {e * kP, e * kP * a.R, e * kP * a.R * a.nheads, e * kP * a.R * a.nheads * a.seqlen};
+  const cuuint32_t box[5] = {32, (cuuint32_t)a.R, 1, (cuuint32_t)(32 / a.R), 1};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.y, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 template <int N, int R>
 int launch_nr(const ScanArgs& a, cudaStream_t s) {
-  using K = Cfg<N, R>;
+  using K = Cfg<N, R, kPlain>;  // (Q does not depend on the variant)
+  const int var = a.bcnorm ? kBCNorm : (a.A_t ? kTimeA : kPlain);
+  const int smem_alloc = var == kBCNorm ? Cfg<N, R, kBCNorm>::SMEM_ALLOC
+                                        : (var == kTimeA ? Cfg<N, R, kTimeA>::SMEM_ALLOC : K::SMEM_ALLOC);
+  const int ybuf = var == kBCNorm ? Cfg<N, R, kBCNorm>::YBUF : (var == kTimeA ? Cfg<N, R, kTimeA>::YBUF : K::YBUF);
   CUtensorMap tmB, tmC, tmX, tmT;
   if (!make_map(&tmB, a.B, N, a.ngroups, a, K::Q) || !make_map(&tmC, a.C, N, a.ngroups, a, K::Q) ||
       !make_map(&tmX, a.x, kP, a.nheads, a, K::Q) ||
@@ -950,7 +1034,9 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
   TcParams prm;
   prm.a = a;
   prm.nchunks = (a.seqlen + K::Q - 1) / K::Q;
-  CUtensorMap tmD, tmL, tmA;
+  CUtensorMap tmD, tmL, tmA, tmY;
+  memset(&tmY, 0, sizeof(tmY));
+  if (ybuf > 0 && !make_y_map(&tmY, a)) return MAMBA3_ERR_CUDA;
   memset(&tmD, 0, sizeof(tmD));
   memset(&tmL, 0, sizeof(tmL));
   memset(&tmA, 0, sizeof(tmA));
@@ -960,10 +1046,11 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
     prm.at_tma = prm.dl_tma && !a.bcnorm && make_dl_map(&tmA, a.A_t, a, K::Q);
     if (!prm.at_tma) prm.dl_tma = 0;
   }
-  auto kern = a.bcnorm ? scan_tc_kernel<N, R, kBCNorm> : (a.A_t ? scan_tc_kernel<N, R, kTimeA> : scan_tc_kernel<N, R, kPlain>);
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM_ALLOC) != cudaSuccess)
+  auto kern = var == kBCNorm ? scan_tc_kernel<N, R, kBCNorm>
+                             : (var == kTimeA ? scan_tc_kernel<N, R, kTimeA> : scan_tc_kernel<N, R, kPlain>);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_alloc) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
-  kern<<<a.batch * a.nheads, kThreads, K::SMEM_ALLOC, s>>>(tmB, tmC, tmX, tmT, tmD, tmL, tmA, prm);
+  kern<<<a.batch * a.nheads, kThreads, smem_alloc, s>>>(tmB, tmC, tmX, tmT, tmD, tmL, tmA, tmY, prm);
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 
