@@ -62,7 +62,9 @@ struct GCfg {
   static constexpr int OFF_X = NKB * kTile;             // X, then X_w in place
   static constexpr int OFF_TH = OFF_X + kTile;
   static constexpr int STAGE = OFF_TH + ((TH_BYTES + 1023) & ~1023);
-  static constexpr int TAIL = 1024;                     // final angle, sums, barriers, misc
+  // final angle, sums, barriers, misc, and the per-token scalars of two chunks
+  // ([2][3][Q + 1] floats: dt, lam, A_t of the chunk's tokens and the next one)
+  static constexpr int TAIL = (K2 * 4 + 64 + 2 * 5 * 8 + 16 + 24 * (Q + 1) + 64 + 1023) & ~1023;
   static constexpr int fit(int st) { return st * STAGE + TAIL + 1024; }
   static constexpr int CPS = fit(3) <= 233472 / 2 - 1024 ? 2 : 1;  // CTAs per SM
   static constexpr int NST = CPS == 2 ? 3 : (fit(5) <= 232448 ? 5 : (fit(4) <= 232448 ? 4 : (fit(3) <= 232448 ? 3 : 2)));
@@ -71,7 +73,8 @@ struct GCfg {
   static constexpr int OFF_RED = OFF_PHI + K2 * 4;      // [8] warp sums
   static constexpr int OFF_BAR = (OFF_RED + 64 + 7) & ~7;  // full[NST], mma[NST]
   static constexpr int OFF_MISC = OFF_BAR + 2 * NST * 8;
-  static constexpr int SMEM = OFF_MISC + 16;
+  static constexpr int OFF_SCL = OFF_MISC + 16;
+  static constexpr int SMEM = OFF_SCL + 24 * (Q + 1);
   static constexpr int SMEM_ALLOC = SMEM + 1024;
   static_assert(SMEM - OFF_PHI <= TAIL && SMEM_ALLOC <= 232448 && NST >= 2, "shared memory");
 };
@@ -156,25 +159,45 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
   // its MMA.  Every warp keeps the decay carry and its groups' running angles.
   constexpr int TPL = Q / 32, GPW = NG / (kThreads / 32);
   static_assert(TPL >= 1 && Q % 32 == 0 && TPL * R == 4 && GPW >= 1 && NG % (kThreads / 32) == 0, "lanes and warps");
-  float p_dt[TPL + 1], p_lm[TPL + 1], p_at[TPL];  // this lane's tokens of the next chunk (+ the one after)
-  auto load_scalars = [&](int c) {
+  // dt, lam (and A_t) of a chunk's tokens and the next one: warp 0 loads chunk c + 2's
+  // into registers while chunk c is prepared and stores them into buffer c & 1 ... of
+  // chunk c + 1 at its end, so that every warp reads them from shared memory (one set of
+  // global loads instead of one per warp, and no warp waits on them)
+  constexpr int E = (Q + 1 + 31) / 32;
+  float* scl = reinterpret_cast<float*>(smem + K::OFF_SCL);  // [2][3][Q + 1]
+  float e_dt[E], e_lm[E], e_at[E];
+  auto load_pre = [&](int c) {
 #pragma unroll
-    for (int i = 0; i <= TPL; ++i) {
-      const int t = c * Q + lane * TPL + i;
-      p_dt[i] = 0.f;
-      p_lm[i] = 1.f;
-      if (i < TPL) p_at[i] = Ah;
-      if (t < L) {
+    for (int e = 0; e < E; ++e) {
+      const int k = lane + 32 * e, t = c * Q + k;
+      e_dt[e] = 0.f;
+      e_lm[e] = 1.f;
+      e_at[e] = Ah;
+      if (k <= Q && t < L) {
         const size_t ti = tok(t);
-        p_dt[i] = __bfloat162float(DT[ti]);
-        p_lm[i] = __bfloat162float(LM[ti]);
-        if constexpr (TVA) {
-          if (i < TPL) p_at[i] = __bfloat162float(AT[ti]);
-        }
+        e_dt[e] = __bfloat162float(DT[ti]);
+        e_lm[e] = __bfloat162float(LM[ti]);
+        if constexpr (TVA) e_at[e] = __bfloat162float(AT[ti]);
       }
     }
   };
-  load_scalars(0);
+  auto store_pre = [&](int buf) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int k = lane + 32 * e;
+      if (k <= Q) {
+        scl[(buf * 3 + 0) * (Q + 1) + k] = e_dt[e];
+        scl[(buf * 3 + 1) * (Q + 1) + k] = e_lm[e];
+        scl[(buf * 3 + 2) * (Q + 1) + k] = e_at[e];
+      }
+    }
+  };
+  if (warp == 0) {
+    load_pre(0);
+    store_pre(0);
+    load_pre(1);
+  }
+  __syncthreads();
   float carry = 0.f;       // log2 decay through the end of the previous chunk
   float phw[GPW][4];       // running angle of this warp's pair groups
 #pragma unroll
@@ -187,13 +210,15 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
     const int s = c % NST;
     uint8_t* st = smem + s * K::STAGE;
     float dt[TPL + 1], lm[TPL + 1], at[TPL];
+    {
+      const float* sb = scl + (c & 1) * 3 * (Q + 1);
 #pragma unroll
-    for (int i = 0; i <= TPL; ++i) {
-      dt[i] = p_dt[i];
-      lm[i] = p_lm[i];
-      if (i < TPL) at[i] = p_at[i];
+      for (int i = 0; i <= TPL; ++i) {
+        dt[i] = sb[lane * TPL + i];
+        lm[i] = sb[(Q + 1) + lane * TPL + i];
+        if (i < TPL) at[i] = TVA ? sb[2 * (Q + 1) + lane * TPL + i] : Ah;
+      }
     }
-    load_scalars(c + 1);
     // decay prefix over the chunk (lane-local, then a warp scan) and the X_w weight f
     float f[TPL];
     {
@@ -325,6 +350,10 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
       *reinterpret_cast<uint4*>(xw + swz(row, cc)) =
           make_uint4(pack_bf16(fsel * f0.x, fsel * f0.y), pack_bf16(fsel * f1.x, fsel * f1.y),
                      pack_bf16(fsel * f2.x, fsel * f2.y), pack_bf16(fsel * f3.x, fsel * f3.y));
+    }
+    if (warp == 0) {  // chunk c + 1's scalars for the next iteration; chunk c + 2's in flight
+      store_pre((c + 1) & 1);
+      load_pre(c + 2);
     }
     fence_proxy_async_smem();
     if (__syncthreads_or(*abort_flag != 0)) {
