@@ -66,8 +66,8 @@ struct GCfg {
   // ([2][3][Q + 1] floats: dt, lam, A_t of the chunk's tokens and the next one)
   static constexpr int TAIL = (K2 * 4 + 64 + 2 * 5 * 8 + 16 + 24 * (Q + 1) + 64 + 1023) & ~1023;
   static constexpr int fit(int st) { return st * STAGE + TAIL + 1024; }
-  static constexpr int CPS = fit(3) <= 233472 / 2 - 1024 ? 2 : 1;  // CTAs per SM
-  static constexpr int NST = CPS == 2 ? 3 : (fit(5) <= 232448 ? 5 : (fit(4) <= 232448 ? 4 : (fit(3) <= 232448 ? 3 : 2)));
+  static constexpr int CPS = fit(2) <= 233472 / 3 - 1024 ? 3 : (fit(3) <= 233472 / 2 - 1024 ? 2 : 1);  // CTAs per SM
+  static constexpr int NST = CPS == 3 ? 2 : (CPS == 2 ? 3 : (fit(5) <= 232448 ? 5 : (fit(4) <= 232448 ? 4 : (fit(3) <= 232448 ? 3 : 2))));
   static constexpr int D = NST - 1;                     // chunks loaded ahead
   static constexpr int OFF_PHI = NST * STAGE;           // final angle [K2]
   static constexpr int OFF_RED = OFF_PHI + K2 * 4;      // [8] warp sums
