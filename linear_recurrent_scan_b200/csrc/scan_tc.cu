@@ -545,8 +545,16 @@ __device__ __forceinline__ void store_hbar_bf16(const float (&hb)[32], uint8_t* 
   }
 }
 
+// one 32-byte store (256-bit global store, sm_100): 8 packed words to a 32-byte aligned address
+__device__ __forceinline__ void st_global_32b(void* p, const uint32_t (&v)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 // y rows of one chunk from its Y and Yi accumulators: y = Y + e^{cum_t} Yi
-// (this thread's 32 columns of row m); rows past the sequence are not stored
+// (this thread's 32 columns of row m, 32 bytes per store); rows past the sequence
+// are not stored
 __device__ __forceinline__ void store_y(const ScanArgs& a, uint32_t tY, uint32_t tYi, float e, int b, int hh, int tg,
                                         int rm, int R, int ch) {
   uint4* yr = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) +
@@ -559,16 +567,10 @@ __device__ __forceinline__ void store_y(const ScanArgs& a, uint32_t tY, uint32_t
     tmem_ld16(tYi + 32 * ch + 16 * half, yi);
     tmem_ld_wait();
     if (tg < a.seqlen) {
+      uint32_t w[8];
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
-        const int o = 8 * q2;
-        uint4 q;
-        q.x = pack_bf16(yv[o + 0] + e * yi[o + 0], yv[o + 1] + e * yi[o + 1]);
-        q.y = pack_bf16(yv[o + 2] + e * yi[o + 2], yv[o + 3] + e * yi[o + 3]);
-        q.z = pack_bf16(yv[o + 4] + e * yi[o + 4], yv[o + 5] + e * yi[o + 5]);
-        q.w = pack_bf16(yv[o + 6] + e * yi[o + 6], yv[o + 7] + e * yi[o + 7]);
-        yr[2 * half + q2] = q;
-      }
+      for (int i = 0; i < 8; ++i) w[i] = pack_bf16(yv[2 * i] + e * yi[2 * i], yv[2 * i + 1] + e * yi[2 * i + 1]);
+      st_global_32b(yr + 2 * half, w);
     }
   }
 }
@@ -771,16 +773,11 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
         tmem_ld16(tmem + lane_base + kColYi + 32 * ch + 16 * half, yi);
         tmem_ld_wait();
         if (tg < L) {
+          uint32_t w[8];
 #pragma unroll
-          for (int q2 = 0; q2 < 2; ++q2) {
-            const int o = 8 * q2;
-            uint4 q;
-            q.x = pack_bf16(yv[o + 0] + my_e * yi[o + 0], yv[o + 1] + my_e * yi[o + 1]);
-            q.y = pack_bf16(yv[o + 2] + my_e * yi[o + 2], yv[o + 3] + my_e * yi[o + 3]);
-            q.z = pack_bf16(yv[o + 4] + my_e * yi[o + 4], yv[o + 5] + my_e * yi[o + 5]);
-            q.w = pack_bf16(yv[o + 6] + my_e * yi[o + 6], yv[o + 7] + my_e * yi[o + 7]);
-            yr[2 * half + q2] = q;
-          }
+          for (int i = 0; i < 8; ++i)
+            w[i] = pack_bf16(yv[2 * i] + my_e * yi[2 * i], yv[2 * i + 1] + my_e * yi[2 * i + 1]);
+          st_global_32b(yr + 2 * half, w);
         }
       }
       }
