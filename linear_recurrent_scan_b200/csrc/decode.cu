@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(kSThreads) decode_stream_kernel(DecodeArgs a) 
       const int r = i / K2, k = i % K2;
       const float phi = wrap_angle(ang[k] + dt * ld1(THs + k));
       float sn, cs;
-      sincosf(phi, &sn, &cs);
+      __sincosf(phi, &sn, &cs);  // |phi| <= pi
       float b0 = ld1(Bs + r * N + 2 * k), b1 = ld1(Bs + r * N + 2 * k + 1);
       float c0 = ld1(Cs + r * N + 2 * k), c1 = ld1(Cs + r * N + 2 * k + 1);
       if constexpr (BCN) {  // normalised row times the head's weight, plus its bias
