@@ -176,11 +176,13 @@ struct Cfg {
   static constexpr int OFF_DL = (OFF_MISC + 16 + 127) & ~127;
   static constexpr int OFF_SINK = OFF_DL + 2 * DL_PAD;  // [Q] floats: consumes the tile reads
   // fused B/C normalisation (V = kBCNorm): w_B, bias_B, w_C, bias_C of this head,
-  // [R][N] floats each; time-varying decay by TMA (V = kTimeA): the A_t tile [Q][8]
-  // bf16 (refilled with theta); nothing for the plain variant
+  // [R][N] floats each, then 1 / RMS of the chunk's raw B and C rows [2][128];
+  // time-varying decay by TMA (V = kTimeA): the A_t tile [Q][8] bf16 (refilled with
+  // theta); nothing for the plain variant
   static constexpr int OFF_NRM = (OFF_SINK + Q * 4 + 127) & ~127;
   static constexpr int AT_BYTES = Q * 16;
-  static constexpr int NRM_BYTES = V == kBCNorm ? 4 * R * N * 4 : (V == kTimeA ? AT_BYTES : 0);
+  static constexpr int OFF_RINV = OFF_NRM + 4 * R * N * 4;
+  static constexpr int NRM_BYTES = V == kBCNorm ? 4 * R * N * 4 + 2 * kM * 4 : (V == kTimeA ? AT_BYTES : 0);
   // y staging where shared memory allows (N = 64; N = 128 with R = 4 except the
   // fused norm): per epilogue warp one or two
   // 32-row x 64-byte tiles (64-byte swizzle) that the warp writes out with a TMA store
@@ -366,6 +368,30 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
     if (prep_sync_any(*abort_flag != 0)) return;  // barrier 1: one decision for all prep threads
 
     // ---- phase B: scalars, prefix of the angle, RoPE ----
+    float* rinv = reinterpret_cast<float*>(smem + K::OFF_RINV);
+    if constexpr (BCN) {
+      // 1 / RMS of every raw row of the chunk, thread = row (B rows: pt < 128, C rows:
+      // the rest): 16-byte reads of the whole row, no cross-lane reduction; an
+      // all-zero row with eps = 0 (e.g. the padding past the sequence end) gives 0
+      const int row = pt & (kM - 1);
+      const uint8_t* tile = st + (pt < kM ? K::OFF_B : K::OFF_C);
+      float ss = 0.f;
+#pragma unroll
+      for (int kb = 0; kb < K::NKB; ++kb)
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const uint4 q = *reinterpret_cast<const uint4*>(tile + kb * kTile + swz(row, c8));
+          const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = unpack_bf16(qw[k]);
+            ss += f.x * f.x + f.y * f.y;
+          }
+        }
+      const float vr = ss * (1.f / N) + a.neps;
+      rinv[pt] = vr > 0.f ? rsqrtf(vr) : 0.f;
+      prep_sync();
+    }
     for (int w = 0; w < (pt >> 5); ++w) v += warp_tot[w];
     if (pt < Q) {
       const float gam = s_lm * s_dt;
@@ -423,26 +449,16 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
         const uint32_t cw[4] = {cq[j].x, cq[j].y, cq[j].z, cq[j].w};
         uint32_t bo[4], co[4];
         if constexpr (BCN) {
-          // raw row (t, r): RMS over N (its NG groups sit in NG consecutive
-          // lanes), weight and bias, then the rotation
-          float bv[8], cv[8], ssb = 0.f, ssc = 0.f;
+          // raw row (t, r): its 1 / RMS from the pass above, weight and bias, then the rotation
+          float bv[8], cv[8];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const float2 b2 = unpack_bf16(bw[k]), c2v = unpack_bf16(cw[k]);
             bv[2 * k] = b2.x; bv[2 * k + 1] = b2.y;
             cv[2 * k] = c2v.x; cv[2 * k + 1] = c2v.y;
-            ssb += b2.x * b2.x + b2.y * b2.y;
-            ssc += c2v.x * c2v.x + c2v.y * c2v.y;
           }
-#pragma unroll
-          for (int o = 1; o < NG; o <<= 1) {
-            ssb += __shfl_xor_sync(0xffffffffu, ssb, o);
-            ssc += __shfl_xor_sync(0xffffffffu, ssc, o);
-          }
-          // an all-zero row with eps = 0 (e.g. the padding past the sequence end)
-          // normalises to 0 instead of 0/0
-          const float vb = ssb * (1.f / N) + a.neps, vc = ssc * (1.f / N) + a.neps;
-          const float ib = vb > 0.f ? rsqrtf(vb) : 0.f, ic = vc > 0.f ? rsqrtf(vc) : 0.f;
+          const int rowi = t * R + r;
+          const float ib = rinv[rowi], ic = rinv[kM + rowi];
           const float* wB = nrm + r * N + 8 * g;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {

@@ -62,7 +62,9 @@ def test_bf16_shapes(shape):
     check_state(fin, fr, TOL[torch.bfloat16])
 
 
-@pytest.mark.parametrize("shape", [(2, 200, 148, 64, 128, 2), (5, 200, 40, 64, 128, 2), (2, 300, 100, 64, 128, 1)])
+@pytest.mark.parametrize("shape", [(2, 200, 148, 64, 128, 2), (5, 200, 40, 64, 128, 2), (2, 300, 100, 64, 128, 1),
+                                   # y written through the epilogue warps' TMA stores (N = 64; N = 128 with R = 4)
+                                   (2, 300, 100, 64, 128, 4), (3, 250, 64, 64, 64, 1)])
 def test_repeated_launches_are_identical_and_match(shape):
     """Many units in flight, launched repeatedly: every launch must match the
     oracle and reproduce the first launch bit for bit (a race between a shared
