@@ -43,31 +43,31 @@ BACKWARD_KERNEL = "bwd_state_kernel + bwd_chunk_kernel (tcgen05, TMA)"
 # capture).  A kernel whose sources no longer hash to the recorded value gets
 # traffic null, since its counters are out of date.
 TRAFFIC = {
-    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "2fd97fd6842377ca6cf13ed5c1b3cd2a97413f5709f879c78f99af04d68faa60",
-                811786240 + 137171712, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
-    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "2fd97fd6842377ca6cf13ed5c1b3cd2a97413f5709f879c78f99af04d68faa60",
-                               5648931584 + 1067155968, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "9e8c0af09abae135f3370d8437840fb2425658b1f546a1fb309f0a6882f2a2ff",
+                811691008 + 138072832, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "9e8c0af09abae135f3370d8437840fb2425658b1f546a1fb309f0a6882f2a2ff",
+                               5647990528 + 1066386944, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     # the segmented prefill: seg_state_kernel + seg_combine_kernel + scan_tc_kernel of one call
-    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "705af9f8899b1ee571690894152745f2d22aeed7f8344fdb02df534021916253",
-                             4591036416 + 36303104 + 38104064 + 295168 + 6773899264 + 2128042240,
+    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "25cbcd2e13032cb9b0645382caa30c4da83b8388029fa0e11190c6025d726407",
+                             4590474752 + 36340736 + 38103296 + 185088 + 6773025792 + 2127789568,
                              "profiles/segmented_prefill_mimo4_b1_l65536.txt"),
-    "siso_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "58dce3e3e41c8eba0c285f96d096107466bc9c65f7d641819e2f6d0619616490",
-                         283193088 + 220056320, "profiles/decode_stream_b128_traffic_and_counters.txt"),
-    "mimo4_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "58dce3e3e41c8eba0c285f96d096107466bc9c65f7d641819e2f6d0619616490",
-                          317806848 + 240501504, "profiles/decode_stream_b128_traffic_and_counters.txt"),
-    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "2fd97fd6842377ca6cf13ed5c1b3cd2a97413f5709f879c78f99af04d68faa60",
-                        284051712 + 114322944, "profiles/grouped_bc_prefill_decode_traffic.txt"),
-    "grouped_decode": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "58dce3e3e41c8eba0c285f96d096107466bc9c65f7d641819e2f6d0619616490",
-                       279064576 + 219895040, "profiles/grouped_bc_prefill_decode_traffic.txt"),
+    "siso_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
+                         283177728 + 219681280, "profiles/decode_stream_b128_traffic_and_counters.txt"),
+    "mimo4_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
+                          317789952 + 241042432, "profiles/decode_stream_b128_traffic_and_counters.txt"),
+    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "9e8c0af09abae135f3370d8437840fb2425658b1f546a1fb309f0a6882f2a2ff",
+                        284561920 + 119342848, "profiles/grouped_bc_prefill_decode_traffic.txt"),
+    "grouped_decode": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
+                       279047936 + 219645952, "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "backward": (('scan_bwd_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "9c8ecf6ec0fbc08bb3233640edb7629a98d0dbddec756d39bef072514d4d24b8",
-                 541858816 + 240333824 + 1219140096 + 787908096,
+                 541950208 + 240395520 + 1218947840 + 788487424,
                  "profiles/scan_bwd_tc_siso_b8_l2048_traffic_and_counters.txt"),
     "mimo_proj_up": (('mimo_proj.cu', 'sm100_ptx.cuh', 'common.cuh'), "c2a412f8cf230533471e6093ea6ca476f1bedd003f0d0f0a07475de750bfd4e2",
-                     406654208 + 1016409088, "profiles/mimo_proj_b4_l8192_traffic.txt"),
+                     406625280 + 1016199424, "profiles/mimo_proj_b4_l8192_traffic.txt"),
     "mimo_proj_down_gated": (('mimo_proj.cu', 'sm100_ptx.cuh', 'common.cuh'), "c2a412f8cf230533471e6093ea6ca476f1bedd003f0d0f0a07475de750bfd4e2",
-                             1480559616 + 246832128, "profiles/mimo_proj_b4_l8192_traffic.txt"),
+                             1480475392 + 247016704, "profiles/mimo_proj_b4_l8192_traffic.txt"),
     "gated_norm_per_head": (('gated_norm.cu', 'common.cuh'), "eb90ad7d72a2607cc062684461d599cc86e5eea7058c9d970afd24eac530e380",
-                            268548608 + 103126784, "profiles/gated_norm_b8_l2048_traffic_and_counters.txt"),
+                            268478976 + 101627392, "profiles/gated_norm_b8_l2048_traffic_and_counters.txt"),
 }
 
 
