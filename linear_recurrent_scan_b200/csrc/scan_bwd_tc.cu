@@ -448,8 +448,8 @@ struct CCfg : BCfg<N, R> {
   static constexpr int OFF_SC = OFF_PHT + B::K2 * QP * 4;
   static constexpr int PART_FLOATS = (NPA > NPART2 ? NPA : NPART2) * B::K2;
   static constexpr int OFF_PART = OFF_SC + kNScal * kScalStride * 4;
-  static constexpr int OFF_SANG = OFF_PART + PART_FLOATS * 4;  // angle gradient from the end [K2]
-  static constexpr int OFF_RED = OFF_SANG + B::K2 * 4;         // block sums [32]
+  static constexpr int OFF_SANG = OFF_PART + PART_FLOATS * 4;  // angle gradient from the end [2][K2] (by chunk parity)
+  static constexpr int OFF_RED = OFF_SANG + 2 * B::K2 * 4;     // block sums [32]
   static constexpr int OFF_BAR = OFF_RED + 128;                // full0, full1, mma1, mma2
   static constexpr int OFF_MISC = OFF_BAR + 64;                // tmem slot, abort flag
   static constexpr int SMEM = OFF_MISC + 16;
@@ -1027,25 +1027,54 @@ __global__ void __launch_bounds__(kCThreads, 1)
     // ---- the angle gradient summed from the end: dtheta = dt S, and sum_k theta S per token ----
     {
       const int k = tid % K2, part = tid / K2;
-      const int tb = part * TPP2, te = (tb + TPP2 < Q) ? tb + TPP2 : Q;
+      const int tb = part * TPP2;
       float ps = 0.f;
-      for (int t = tb; t < te; ++t) ps += dphi_s[dphi_at(t, k)];
+#pragma unroll
+      for (int i = 0; i < TPP2; ++i)
+        if (tb + i < Q) ps += dphi_s[dphi_at(tb + i, k)];
       part_sum[part * K2 + k] = ps;
       __syncthreads();
-      float S = sang[k];
+      // running sum from the end of the sequence, double-buffered by chunk parity
+      float S = sang[(r & 1) * K2 + k];
       for (int p2 = part + 1; p2 < NPART2; ++p2) S += part_sum[p2 * K2 + k];
-      __syncthreads();  // every thread has read sang[k]
-      for (int t = te - 1; t >= tb; --t) {
-        S += dphi_s[dphi_at(t, k)];
-        const float dtv = sc[sDt * kScalStride + t];
-        const int tg = t0 + t;
-        if (tg < L) dTHg[tok_index(a, b, tg, hh) * K2 + k] = __float2bfloat16_rn(dtv * S);
-        float v = __bfloat162float(th[t * K2 + k]) * S;
+      float v[TPP2];  // theta S of this thread's pair at each of its tokens
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) atomicAdd(&sc[sDth * kScalStride + t], v);
+      for (int i = TPP2 - 1; i >= 0; --i) {
+        const int t = tb + i;
+        v[i] = 0.f;
+        if (t < Q) {
+          S += dphi_s[dphi_at(t, k)];
+          const float dtv = sc[sDt * kScalStride + t];
+          const int tg = t0 + t;
+          if (tg < L) dTHg[tok_index(a, b, tg, hh) * K2 + k] = __float2bfloat16_rn(dtv * S);
+          v[i] = __bfloat162float(th[t * K2 + k]) * S;
+        }
       }
-      if (part == 0) sang[k] = S;
+      // the sums over the warp's 32 pairs of all TPP2 tokens at once: each butterfly
+      // step halves the values a lane holds (it keeps the half its lane bit selects
+      // and adds the partner's copy of it), then the last steps reduce the one left
+      constexpr int HB = TPP2 >= 16 ? 4 : (TPP2 >= 8 ? 3 : (TPP2 >= 4 ? 2 : (TPP2 >= 2 ? 1 : 0)));
+      static_assert((1 << HB) == TPP2, "tokens per part: a power of two");
+#pragma unroll
+      for (int st2 = 0; st2 < HB; ++st2) {
+        const int off = 16 >> st2, hlf = TPP2 >> (st2 + 1);
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < TPP2 / 2; ++i)
+          if (i < hlf) {
+            const float send = up ? v[i] : v[i + hlf];
+            const float keep = up ? v[i + hlf] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+          }
+      }
+#pragma unroll
+      for (int off = 16 >> HB; off > 0; off >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+      int j = 0;  // the token whose sum this lane holds
+#pragma unroll
+      for (int st2 = 0; st2 < HB; ++st2)
+        if (lane & (16 >> st2)) j += TPP2 >> (st2 + 1);
+      if ((lane & ((32 >> HB) - 1)) == 0 && tb + j < Q) atomicAdd(&sc[sDth * kScalStride + tb + j], v[0]);
+      if (part == 0) sang[((r + 1) & 1) * K2 + k] = S;
     }
     __syncthreads();
 
@@ -1181,7 +1210,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
           for (int nn = 0; nn < N; ++nn) s2 += Gs[nn * kP + pp] * a.bprev0[((size_t)unit * R + rr) * N + nn];
         g.dxprev0[(size_t)unit * R * kP + i] = mu1 * s2;
       }
-      for (int k = tid; k < K2; k += kCThreads) g.dangle0[(size_t)unit * K2 + k] = sang[k];
+      for (int k = tid; k < K2; k += kCThreads) g.dangle0[(size_t)unit * K2 + k] = sang[(nchunks & 1) * K2 + k];
     }
   }
   tc_fence_before();
