@@ -59,8 +59,8 @@ TRAFFIC = {
                         284561920 + 119342848, "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "grouped_decode": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                        279047936 + 219645952, "profiles/grouped_bc_prefill_decode_traffic.txt"),
-    "backward": (('scan_bwd_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "9c8ecf6ec0fbc08bb3233640edb7629a98d0dbddec756d39bef072514d4d24b8",
-                 541950208 + 240395520 + 1218947840 + 788487424,
+    "backward": (('scan_bwd_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "4e0c7c64d7cdf0641dc3706bae97f8049f27d153a1436da0552077c3f5ea4781",
+                 541800448 + 240511488 + 1218752768 + 787912960,
                  "profiles/scan_bwd_tc_siso_b8_l2048_traffic_and_counters.txt"),
     "mimo_proj_up": (('mimo_proj.cu', 'sm100_ptx.cuh', 'common.cuh'), "c2a412f8cf230533471e6093ea6ca476f1bedd003f0d0f0a07475de750bfd4e2",
                      406625280 + 1016199424, "profiles/mimo_proj_b4_l8192_traffic.txt"),
