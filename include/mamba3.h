@@ -121,6 +121,31 @@ MAMBA3_API int mamba3_scan_fwd(const mamba3_dims* dims, const void* x, const voi
                     void* stream);
 
 /*
+ * The prefill from host buffers (mamba3_scan_fwd with x, B, C, theta, dt, lam and
+ * y in host memory; page-locked memory lets the copies run asynchronously).  The
+ * batch is cut into up to 8 sub-batches that cycle through two slots of `stage`:
+ * while sub-batch i is computed on `stream`, the inputs of sub-batch i + 1 are
+ * copied in and y of sub-batch i - 1 is copied out on two streams of the call's
+ * own, so that both copy directions and the kernels overlap.  Every batch row is
+ * an independent set of (b, h) units, so the result equals mamba3_scan_fwd's.
+ *   A, D, init, final_state   device memory, as for mamba3_scan_fwd.
+ *   stage        device memory of at least mamba3_scan_fwd_host_stage_bytes(dims)
+ *                (16-byte aligned); its first 256 bytes are the status word
+ *                (mamba3_device_status), reset by this call.
+ *   stream       the call's work, including the last copy of y into host memory,
+ *                is ordered on `stream`: synchronising it makes y readable.
+ * Errors are reported before anything is enqueued, except MAMBA3_ERR_CUDA.
+ * Host arrays are read and y written asynchronously: they must stay valid and
+ * unmodified until `stream` has passed this call.  Section 1.1-1.3 as above.
+ */
+MAMBA3_API size_t mamba3_scan_fwd_host_stage_bytes(const mamba3_dims* dims);
+MAMBA3_API int mamba3_scan_fwd_host(const mamba3_dims* dims, const void* x, const void* B, const void* C,
+                                    const void* theta, const void* dt, const void* lam, const float* A,
+                                    const float* D, const mamba3_state* init, void* y,
+                                    const mamba3_state* final_state, void* stage, size_t stage_bytes,
+                                    void* stream);
+
+/*
  * One decode step for every (batch, head), in place on `state`
  * (section 1.3: the state is streamed once; the rank-R update and readout
  * happen in registers).  Per-token inputs have no seqlen axis:

@@ -124,6 +124,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba3_test_set_segments.restype = i
     lib.mamba3_library_status.argtypes = [vp]
     lib.mamba3_library_status.restype = i
+    lib.mamba3_scan_fwd_host_stage_bytes.argtypes = [ctypes.POINTER(Dims)]
+    lib.mamba3_scan_fwd_host_stage_bytes.restype = sz
+    lib.mamba3_scan_fwd_host.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, vp, vp, vp, vp,
+                                         ctypes.POINTER(_CState), vp, ctypes.POINTER(_CState), vp, sz, vp]
+    lib.mamba3_scan_fwd_host.restype = i
     lib.mamba3_mimo_up.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp]
     lib.mamba3_mimo_up.restype = i
     lib.mamba3_mimo_down.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, ctypes.c_float, vp, vp]
@@ -244,6 +249,40 @@ def mamba3_scan_fwd(x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = 
                              ctypes.byref(cf) if cf is not None else None, _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "mamba3_scan_fwd")
+    return y
+
+
+def mamba3_scan_fwd_host_stage_bytes(dims: Dims) -> int:
+    """Device stage bytes mamba3_scan_fwd_host needs for ``dims``."""
+    return int(load_library().mamba3_scan_fwd_host_stage_bytes(ctypes.byref(dims)))
+
+
+def mamba3_scan_fwd_host(x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = None,
+                         y: Optional[torch.Tensor] = None, final_state: Optional[State] = None,
+                         stage: Optional[torch.Tensor] = None, stream=None):
+    """The prefill from host tensors (x .. lam on the CPU, page-locked for
+    asynchronous copies; the shapes of mamba3_scan_fwd): the library copies
+    sub-batches in, runs them and copies y out on overlapping streams.  A, D, init,
+    final_state and ``stage`` are device tensors. Returns the host y (allocated,
+    page-locked, if not given); it is complete once ``stream`` is synchronised."""
+    lib = load_library()
+    _check_inputs(x, B, C, theta, dt, lam, A, D, decode=False)
+    if x.device.type != "cpu":
+        raise ValueError("mamba3_scan_fwd_host takes host tensors; use mamba3_scan_fwd for device tensors")
+    dims = make_dims(x, B)
+    if y is None:
+        y = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    if y.device.type != "cpu" or y.shape != x.shape or y.dtype != x.dtype or not y.is_contiguous():
+        raise ValueError("y must be a contiguous host tensor shaped like x")
+    if stage is None:
+        stage = torch.empty(mamba3_scan_fwd_host_stage_bytes(dims), dtype=torch.uint8, device=A.device)
+    ci = init._c() if init is not None else None
+    cf = final_state._c() if final_state is not None else None
+    rc = lib.mamba3_scan_fwd_host(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam),
+                                  _ptr(A), _ptr(D), ctypes.byref(ci) if ci is not None else None, _ptr(y),
+                                  ctypes.byref(cf) if cf is not None else None, _ptr(stage),
+                                  stage.numel() * stage.element_size(), _stream(stream))
+    _check(rc, "mamba3_scan_fwd_host")
     return y
 
 
@@ -557,7 +596,8 @@ def mamba3_test_withhold_loads(on: bool) -> None:
 
 __all__ = [
     "Dims", "State", "BCNorm", "Mamba3Error", "load_library", "make_dims",
-    "mamba3_scan_workspace_bytes", "mamba3_scan_segmented_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc", "mamba3_decode_step",
+    "mamba3_scan_workspace_bytes", "mamba3_scan_segmented_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc",
+    "mamba3_scan_fwd_host_stage_bytes", "mamba3_scan_fwd_host", "mamba3_decode_step",
     "mamba3_scan_fwd_bcnorm", "mamba3_decode_step_bcnorm", "mamba3_scan_fwd_at", "mamba3_decode_step_at",
     "mamba3_scan_bwd_workspace_bytes", "mamba3_scan_bwd", "mamba3_scan_bwd_at", "mamba3_gated_norm",
     "mamba3_device_status", "mamba3_library_status", "mamba3_mimo_up", "mamba3_mimo_down", "mamba3_set_wait_limit", "mamba3_test_withhold_loads", "mamba3_test_set_segments",

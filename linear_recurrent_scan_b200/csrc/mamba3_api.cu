@@ -428,3 +428,159 @@ int mamba3_gated_norm(const mamba3_dims* d, int groups, const void* y, const voi
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- the prefill from host buffers
+namespace {
+
+constexpr int kHostSplits = 8;  // sub-batches the host prefill cycles through the stage
+
+size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// The sub-batches of mamba3_scan_fwd_host (bs batch rows each, nb of them) and the
+// device stage: the status word, then two slots of one sub-batch's x, y, B, C,
+// theta, dt and lam.
+struct HostLayout {
+  int nb, bs;
+  size_t x_row, bc_row, th_row, dl_row;  // bytes of one batch row of x (and y), B (and C), theta, dt (and lam)
+  size_t x, bc, th, dl;                  // aligned bytes of one sub-batch of each
+  size_t slot, total;
+};
+
+HostLayout host_layout(const mamba3_dims* d) {
+  HostLayout l;
+  l.nb = d->batch < kHostSplits ? d->batch : kHostSplits;
+  l.bs = (d->batch + l.nb - 1) / l.nb;
+  l.nb = (d->batch + l.bs - 1) / l.bs;
+  const size_t es = d->in_dtype == MAMBA3_BF16 ? 2 : 4;
+  const size_t L = d->seqlen, H = d->nheads, R = d->rank, P = d->headdim, N = d->dstate, G = bc_groups(d);
+  l.x_row = L * H * R * P * es;
+  l.bc_row = L * G * R * N * es;
+  l.th_row = L * H * (N / 2) * es;
+  l.dl_row = L * H * es;
+  l.x = align256(l.bs * l.x_row);
+  l.bc = align256(l.bs * l.bc_row);
+  l.th = align256(l.bs * l.th_row);
+  l.dl = align256(l.bs * l.dl_row);
+  l.slot = 2 * l.x + 2 * l.bc + l.th + 2 * l.dl;
+  l.total = kStatusBytes + 2 * l.slot;
+  return l;
+}
+
+// Streams and events of one call (created per call, so that calls on different
+// streams never share them; destroying them does not wait for their work).
+struct HostPipe {
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t start = nullptr, in[2] = {nullptr, nullptr}, done[2] = {nullptr, nullptr}, out[2] = {nullptr, nullptr};
+  bool ok = true;
+  HostPipe() {
+    const unsigned f = cudaEventDisableTiming;
+    ok = cudaStreamCreateWithFlags(&up, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&down, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaEventCreateWithFlags(&start, f) == cudaSuccess;
+    for (int i = 0; ok && i < 2; ++i)
+      ok = cudaEventCreateWithFlags(&in[i], f) == cudaSuccess && cudaEventCreateWithFlags(&done[i], f) == cudaSuccess &&
+           cudaEventCreateWithFlags(&out[i], f) == cudaSuccess;
+  }
+  ~HostPipe() {
+    for (int i = 0; i < 2; ++i) {
+      if (in[i]) cudaEventDestroy(in[i]);
+      if (done[i]) cudaEventDestroy(done[i]);
+      if (out[i]) cudaEventDestroy(out[i]);
+    }
+    if (start) cudaEventDestroy(start);
+    if (up) cudaStreamDestroy(up);
+    if (down) cudaStreamDestroy(down);
+  }
+};
+
+mamba3_state state_rows(const mamba3_state* s, const mamba3_dims* d, int r0) {
+  mamba3_state o;
+  const size_t H = d->nheads, N = d->dstate, P = d->headdim, R = d->rank;
+  o.h = s->h + r0 * H * N * P;
+  o.b_prev = s->b_prev + r0 * H * R * N;
+  o.x_prev = s->x_prev + r0 * H * R * P;
+  o.angle = s->angle + r0 * H * (N / 2);
+  return o;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mamba3_scan_fwd_host_stage_bytes(const mamba3_dims* d) {
+  if (check_dims(d, true) != MAMBA3_OK) return 0;
+  return host_layout(d).total;
+}
+
+int mamba3_scan_fwd_host(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                         const void* dt, const void* lam, const float* A, const float* D, const mamba3_state* init,
+                         void* y, const mamba3_state* final_state, void* stage, size_t stage_bytes, void* stream) {
+  int rc = check_dims(d, true);
+  if (rc) return rc;
+  if (!A || !aligned4(A) || (D && !aligned4(D))) return MAMBA3_ERR_INVALID;
+  if ((rc = check_state(init)) || (rc = check_state(final_state))) return rc;
+  if (!stage || !aligned16(stage)) return MAMBA3_ERR_WORKSPACE;
+  const HostLayout l = host_layout(d);
+  if (stage_bytes < l.total) return MAMBA3_ERR_WORKSPACE;
+  if (d->seqlen == 0)  // nothing to copy: the state passes through as in the device call
+    return scan_fwd_impl(d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, A, nullptr, D, nullptr, init,
+                         nullptr, final_state, stage, stage_bytes, stream);
+  if (!x || !B || !C || !theta || !dt || !lam || !y) return MAMBA3_ERR_INVALID;
+  // the kernel family for the whole problem (every sub-batch takes the same one)
+  uint8_t* base = static_cast<uint8_t*>(stage);
+  m3::ScanArgs probe = scan_args(d, base, base, base, base, base, base, A, D, init);
+  const bool use_tc = m3::tc_scan_supported(probe) == MAMBA3_OK;
+  if (!use_tc && (rc = m3::simt_scan_supported(probe))) return rc;
+
+  HostPipe p;
+  if (!p.ok) return MAMBA3_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaMemcpyKind h2d = cudaMemcpyHostToDevice, d2h = cudaMemcpyDeviceToHost;
+  bool ok = cudaMemsetAsync(stage, 0, sizeof(m3::DeviceStatus), s) == cudaSuccess &&
+            cudaEventRecord(p.start, s) == cudaSuccess && cudaStreamWaitEvent(p.up, p.start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(p.down, p.start, 0) == cudaSuccess;
+  for (int i = 0; ok && i < l.nb; ++i) {
+    const int r0 = i * l.bs, rows = (d->batch - r0) < l.bs ? (d->batch - r0) : l.bs, slot = i & 1;
+    uint8_t* sx = base + kStatusBytes + slot * l.slot;
+    uint8_t* sy = sx + l.x;
+    uint8_t* sB = sy + l.x;
+    uint8_t* sC = sB + l.bc;
+    uint8_t* sth = sC + l.bc;
+    uint8_t* sdt = sth + l.th;
+    uint8_t* slm = sdt + l.dl;
+    // inputs of sub-batch i into the slot once the prefill of sub-batch i - 2 has read it
+    if (i >= 2) ok = cudaStreamWaitEvent(p.up, p.done[slot], 0) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(sx, static_cast<const uint8_t*>(x) + r0 * l.x_row, rows * l.x_row, h2d, p.up) == cudaSuccess &&
+         cudaMemcpyAsync(sB, static_cast<const uint8_t*>(B) + r0 * l.bc_row, rows * l.bc_row, h2d, p.up) == cudaSuccess &&
+         cudaMemcpyAsync(sC, static_cast<const uint8_t*>(C) + r0 * l.bc_row, rows * l.bc_row, h2d, p.up) == cudaSuccess &&
+         cudaMemcpyAsync(sth, static_cast<const uint8_t*>(theta) + r0 * l.th_row, rows * l.th_row, h2d, p.up) == cudaSuccess &&
+         cudaMemcpyAsync(sdt, static_cast<const uint8_t*>(dt) + r0 * l.dl_row, rows * l.dl_row, h2d, p.up) == cudaSuccess &&
+         cudaMemcpyAsync(slm, static_cast<const uint8_t*>(lam) + r0 * l.dl_row, rows * l.dl_row, h2d, p.up) == cudaSuccess &&
+         cudaEventRecord(p.in[slot], p.up) == cudaSuccess && cudaStreamWaitEvent(s, p.in[slot], 0) == cudaSuccess;
+    // its y buffer once the copy-out of sub-batch i - 2 has read it
+    if (ok && i >= 2) ok = cudaStreamWaitEvent(s, p.out[slot], 0) == cudaSuccess;
+    if (!ok) break;
+    mamba3_dims ds = *d;
+    ds.batch = rows;
+    mamba3_state is, fs;
+    if (init) is = state_rows(init, d, r0);
+    if (final_state) fs = state_rows(final_state, d, r0);
+    m3::ScanArgs a = scan_args(&ds, sx, sB, sC, sth, sdt, slm, A, D, init ? &is : nullptr);
+    a.y = sy;
+    if (final_state) {
+      a.h_out = fs.h; a.bprev_out = fs.b_prev; a.xprev_out = fs.x_prev; a.angle_out = fs.angle;
+    }
+    a.workspace = stage;
+    a.workspace_bytes = kStatusBytes;
+    if ((rc = use_tc ? m3::launch_scan_tc(a, s) : m3::launch_scan_simt(a, s)) != MAMBA3_OK) return rc;
+    ok = cudaEventRecord(p.done[slot], s) == cudaSuccess && cudaStreamWaitEvent(p.down, p.done[slot], 0) == cudaSuccess &&
+         cudaMemcpyAsync(static_cast<uint8_t*>(y) + r0 * l.x_row, sy, rows * l.x_row, d2h, p.down) == cudaSuccess &&
+         cudaEventRecord(p.out[slot], p.down) == cudaSuccess;
+  }
+  // the caller's stream resumes after the last copies out
+  for (int i = l.nb - 2; ok && i < l.nb; ++i)
+    if (i >= 0) ok = cudaStreamWaitEvent(s, p.out[i & 1], 0) == cudaSuccess;
+  return ok ? MAMBA3_OK : MAMBA3_ERR_CUDA;
+}
+
+}  // extern "C"

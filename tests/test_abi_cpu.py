@@ -336,3 +336,40 @@ def test_mimo_projection_host_validation(lib):
 def test_mimo_projection_valid_call_without_device_is_a_cuda_error(lib):
     assert proj_up(lib, dims(rank=4, headdim=64)) == m3.MAMBA3_ERR_CUDA
     assert proj_down(lib, dims(rank=2, headdim=64), z=FAKE, w=FAKE) == m3.MAMBA3_ERR_CUDA
+
+
+def host_scan(lib, d, ptrs=None, init=None, final=None, stage=FAKE, stage_bytes=1 << 30):
+    p = dict(x=FAKE, B=FAKE, C=FAKE, theta=FAKE, dt=FAKE, lam=FAKE, A=FAKE, D=None, y=FAKE)
+    p.update(ptrs or {})
+    return lib.mamba3_scan_fwd_host(ctypes.byref(d) if d is not None else None, p["x"], p["B"], p["C"], p["theta"],
+                                    p["dt"], p["lam"], p["A"], p["D"], init, p["y"], final, stage, stage_bytes,
+                                    None)
+
+
+def test_host_stage_bytes(lib):
+    """The status word, then two slots of one sub-batch (here one batch row of two)
+    of x, y, B, C, theta, dt and lam, each 256-byte aligned."""
+    es, L, H, R, P, N = 2, 64, 3, 1, 16, 16
+    al = lambda v: (v + 255) // 256 * 256
+    slot = 2 * al(L * H * R * P * es) + 2 * al(L * H * R * N * es) + al(L * H * (N // 2) * es) + 2 * al(L * H * es)
+    assert lib.mamba3_scan_fwd_host_stage_bytes(ctypes.byref(dims())) == 256 + 2 * slot
+    # batch 20: 8 sub-batches of 3 rows (the last one 2), slots sized for 3 rows
+    slot3 = 2 * al(3 * L * H * R * P * es) + 2 * al(3 * L * H * R * N * es) + al(3 * L * H * (N // 2) * es) + \
+        2 * al(3 * L * H * es)
+    assert lib.mamba3_scan_fwd_host_stage_bytes(ctypes.byref(dims(batch=20))) == 256 + 2 * slot3
+    assert lib.mamba3_scan_fwd_host_stage_bytes(ctypes.byref(dims(batch=0))) == 0
+
+
+@pytest.mark.parametrize("name", ["x", "B", "C", "theta", "dt", "lam", "A", "y"])
+def test_host_scan_rejects_null_pointer(lib, name):
+    assert host_scan(lib, dims(), {name: None}) == m3.MAMBA3_ERR_INVALID
+
+
+def test_host_scan_rejects_stage_and_dims(lib):
+    d = dims()
+    need = lib.mamba3_scan_fwd_host_stage_bytes(ctypes.byref(d))
+    assert host_scan(lib, d, stage_bytes=need - 1) == m3.MAMBA3_ERR_WORKSPACE
+    assert host_scan(lib, d, stage=FAKE + 8) == m3.MAMBA3_ERR_WORKSPACE
+    assert host_scan(lib, d, stage=None) == m3.MAMBA3_ERR_WORKSPACE
+    assert host_scan(lib, dims(rank=3)) == m3.MAMBA3_ERR_INVALID
+    assert host_scan(lib, None) == m3.MAMBA3_ERR_INVALID
