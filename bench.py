@@ -268,7 +268,7 @@ def run_prefill(m3, args, world, rank, clk):
     y = torch.empty_like(inp["x"])
     fin = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
     dims = m3.make_dims(inp["x"], inp["B"])
-    ws = torch.zeros(m3.mamba3_scan_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(m3.mamba3_scan_fwd_workspace_bytes(dims), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -355,8 +355,9 @@ def run_prefill_plain(m3, w: wl.Workload, rank, steps, warmup, fused_norm=False,
     y = torch.empty_like(inp["x"])
     fin = m3.State.zeros(w.batch, w.nheads, w.headdim, w.dstate, w.rank, device=dev)
     dims = m3.make_dims(inp["x"], inp["B"])
-    # the workspace size with which a long sequence over few units runs in segments
-    ws = torch.zeros(max(256, m3.mamba3_scan_segmented_workspace_bytes(dims)), dtype=torch.uint8, device=dev)
+    # the workspace of the library's best schedule (segments for a long sequence over
+    # few units, else the split last wave)
+    ws = torch.zeros(m3.mamba3_scan_fwd_workspace_bytes(dims), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def launch():

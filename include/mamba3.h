@@ -310,6 +310,34 @@ MAMBA3_API size_t mamba3_scan_segmented_workspace_bytes(const mamba3_dims* dims)
  */
 MAMBA3_API int mamba3_test_set_segments(int S);
 
+/*
+ * The workspace with which mamba3_scan_fwd (and its _at and _bcnorm forms) runs
+ * its best schedule for `dims`: the segmented prefill where that applies (then
+ * equal to mamba3_scan_segmented_workspace_bytes), otherwise the status block
+ * plus what the tensor-core prefill needs to split its last wave.  With U = b H
+ * units on the 148 SMs, the last of ceil(U / 148) waves of one CTA per unit holds
+ * only U mod 148 units; the library instead runs k units in two CTAs, chunks
+ * [0, c1) in the first wave and [c1, n) in the last, the second continuing from
+ * the carried state and the accumulated angle that the first hands over in the
+ * workspace (the chunk recurrence of "Mamba-3: 2x smaller state ..." (MarkTechPost,
+ * Korean translation), sections 1.1-1.2, crosses a chunk boundary the same way
+ * inside one CTA, so y and the final state are those of the unsplit prefill bit
+ * for bit).  The space is 256 bytes of status, k 4-byte flags rounded up to 256
+ * bytes, and k (N P + N/2) floats, k < 148 + 32; 256 when the shape gains nothing
+ * from a split (U a multiple of 148, U <= 148, or no tensor-core path).  0 for
+ * invalid dims.  Any workspace of at least mamba3_scan_workspace_bytes works: a
+ * smaller one than this runs without the split.
+ */
+MAMBA3_API size_t mamba3_scan_fwd_workspace_bytes(const mamba3_dims* dims);
+
+/*
+ * For testing the split last wave only: k > 0 splits units 0 .. k-1 after c1
+ * chunks whenever k <= b H and 1 <= c1 < the number of chunks (otherwise no
+ * split); k < 0 never splits; k = 0 restores the library's plan.  Returns
+ * MAMBA3_ERR_INVALID for k > 0 with c1 < 1.  Process-wide.
+ */
+MAMBA3_API int mamba3_test_set_split(int k, int c1);
+
 /* Synchronises `stream`, then returns the device status word that the last
  * mamba3_scan_fwd on `workspace` left (MAMBA3_OK or MAMBA3_ERR_TIMEOUT), or
  * MAMBA3_ERR_CUDA / MAMBA3_ERR_INVALID. */

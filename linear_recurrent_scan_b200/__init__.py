@@ -122,6 +122,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba3_scan_segmented_workspace_bytes.restype = sz
     lib.mamba3_test_set_segments.argtypes = [i]
     lib.mamba3_test_set_segments.restype = i
+    lib.mamba3_scan_fwd_workspace_bytes.argtypes = [ctypes.POINTER(Dims)]
+    lib.mamba3_scan_fwd_workspace_bytes.restype = sz
+    lib.mamba3_test_set_split.argtypes = [i, i]
+    lib.mamba3_test_set_split.restype = i
     lib.mamba3_library_status.argtypes = [vp]
     lib.mamba3_library_status.restype = i
     lib.mamba3_scan_fwd_host_stage_bytes.argtypes = [ctypes.POINTER(Dims)]
@@ -202,6 +206,12 @@ def mamba3_scan_workspace_bytes(dims: Dims) -> int:
     return int(load_library().mamba3_scan_workspace_bytes(ctypes.byref(dims)))
 
 
+def mamba3_scan_fwd_workspace_bytes(dims: Dims) -> int:
+    """Workspace with which mamba3_scan_fwd runs its best schedule (segments for
+    few long sequences, else the split last wave; the minimum when neither applies)."""
+    return int(load_library().mamba3_scan_fwd_workspace_bytes(ctypes.byref(dims)))
+
+
 def mamba3_scan_segmented_workspace_bytes(dims: Dims) -> int:
     """Workspace with which a long sequence over few (batch, head) units runs in
     segments (mamba3_scan_workspace_bytes when the dims do not qualify)."""
@@ -241,7 +251,7 @@ def mamba3_scan_fwd(x, B, C, theta, dt, lam, A, D=None, init: Optional[State] = 
     if y is None:
         y = torch.empty_like(x)
     if workspace is None:
-        workspace = torch.empty(mamba3_scan_segmented_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
+        workspace = torch.empty(mamba3_scan_fwd_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
     ci = init._c() if init is not None else None
     cf = final_state._c() if final_state is not None else None
     rc = lib.mamba3_scan_fwd(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam),
@@ -358,7 +368,7 @@ def mamba3_scan_fwd_bcnorm(x, B_raw, C_raw, theta, dt, lam, A, D=None, norm: Opt
     if y is None:
         y = torch.empty_like(x)
     if workspace is None:
-        workspace = torch.empty(mamba3_scan_segmented_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
+        workspace = torch.empty(mamba3_scan_fwd_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
     ci = init._c() if init is not None else None
     cf = final_state._c() if final_state is not None else None
     rc = lib.mamba3_scan_fwd_bcnorm(ctypes.byref(dims), _ptr(x), _ptr(B_raw), _ptr(C_raw), _ptr(theta), _ptr(dt),
@@ -406,7 +416,7 @@ def mamba3_scan_fwd_at(x, B, C, theta, dt, lam, A_t, D=None, init: Optional[Stat
     if y is None:
         y = torch.empty_like(x)
     if workspace is None:
-        workspace = torch.empty(mamba3_scan_segmented_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
+        workspace = torch.empty(mamba3_scan_fwd_workspace_bytes(dims), dtype=torch.uint8, device=x.device)
     ci = init._c() if init is not None else None
     cf = final_state._c() if final_state is not None else None
     rc = lib.mamba3_scan_fwd_at(ctypes.byref(dims), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt), _ptr(lam),
@@ -582,6 +592,12 @@ def mamba3_set_wait_limit(cycles: int) -> None:
     _check(load_library().mamba3_set_wait_limit(int(cycles)), "mamba3_set_wait_limit")
 
 
+def mamba3_test_set_split(k: int, c1: int = 0) -> None:
+    """Testing only: split units 0..k-1 after c1 chunks (k > 0), never split (k < 0),
+    or restore the library's plan (k = 0)."""
+    _check(load_library().mamba3_test_set_split(int(k), int(c1)), "mamba3_test_set_split")
+
+
 def mamba3_test_set_segments(S: int) -> None:
     """Testing the segmented prefill only: S >= 2 segments whenever S divides the
     sequence length; 0 restores the library's choice."""
@@ -596,10 +612,10 @@ def mamba3_test_withhold_loads(on: bool) -> None:
 
 __all__ = [
     "Dims", "State", "BCNorm", "Mamba3Error", "load_library", "make_dims",
-    "mamba3_scan_workspace_bytes", "mamba3_scan_segmented_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc",
+    "mamba3_scan_workspace_bytes", "mamba3_scan_segmented_workspace_bytes", "mamba3_scan_fwd_workspace_bytes", "mamba3_scan_fwd", "mamba3_scan_fwd_noalloc",
     "mamba3_scan_fwd_host_stage_bytes", "mamba3_scan_fwd_host", "mamba3_decode_step",
     "mamba3_scan_fwd_bcnorm", "mamba3_decode_step_bcnorm", "mamba3_scan_fwd_at", "mamba3_decode_step_at",
     "mamba3_scan_bwd_workspace_bytes", "mamba3_scan_bwd", "mamba3_scan_bwd_at", "mamba3_gated_norm",
-    "mamba3_device_status", "mamba3_library_status", "mamba3_mimo_up", "mamba3_mimo_down", "mamba3_set_wait_limit", "mamba3_test_withhold_loads", "mamba3_test_set_segments",
+    "mamba3_device_status", "mamba3_library_status", "mamba3_mimo_up", "mamba3_mimo_down", "mamba3_set_wait_limit", "mamba3_test_withhold_loads", "mamba3_test_set_segments", "mamba3_test_set_split",
     "mamba3_status_string",
 ]

@@ -29,6 +29,8 @@ struct ScanArgs {
   long long wait_limit;
   int test_withhold;  // testing the timeout path only: issue no input loads
   float* decay_out;   // segment aggregates: sum of dt * A over each sequence [b, H], or null
+  int split;          // the tensor-core prefill may split its last wave (the workspace holds
+                      // tc_split_bytes after the status block, the first bytes zeroed)
 };
 
 struct DecodeArgs {
@@ -133,6 +135,21 @@ bool make_theta_map(CUtensorMap* m, const ScanArgs& a, int Q, bool swizzle = fal
 // (0 = run unsegmented), the workspace they need after the status word, and the
 // segmented prefill.
 constexpr int kSMs = 148;
+// the device status block at the start of every prefill workspace
+constexpr size_t kStatusBlockBytes = 256;
+
+// The tensor-core prefill's split last wave (scan_tc.cu): units that run in two
+// CTAs and where they split (k = 0: none), the workspace it needs after the
+// status block (0 without a split) and the part of it that must be zero before
+// the launch; tc_force_split(k, c1) fixes the plan for tests (k = 0: the
+// library's plan, k < 0: never split).
+struct SplitPlan {
+  int k, c1;
+};
+SplitPlan tc_split_plan(const ScanArgs& a);
+size_t tc_split_bytes(const ScanArgs& a);
+size_t tc_split_zero_bytes(const ScanArgs& a);
+void tc_force_split(int k, int c1);
 int seg_count(const ScanArgs& a, int sms);
 // CTAs of the segment-state kernel that share an SM for these sizes (1 or 2)
 int seg_state_ctas_per_sm(const ScanArgs& a);

@@ -9,7 +9,7 @@
 
 namespace {
 
-constexpr size_t kStatusBytes = 256;
+constexpr size_t kStatusBytes = m3::kStatusBlockBytes;
 
 // Process-wide settings of the bounded device waits (mamba3_set_wait_limit,
 // mamba3_test_withhold_loads), read at every launch.
@@ -158,12 +158,23 @@ int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
   if (!use_tc && (rc = m3::simt_scan_supported(a))) return rc;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
   if (use_tc) {  // a long sequence over few units runs in segments when the workspace allows it
     const int S = g_test_segments ? forced_segments(a) : m3::seg_count(a, m3::kSMs);
-    if (S > 0 && workspace_bytes >= kStatusBytes + m3::seg_workspace_bytes(a, S))
+    if (S > 0 && workspace_bytes >= kStatusBytes + m3::seg_workspace_bytes(a, S)) {
+      if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
       return m3::launch_scan_segmented(a, S, s);
+    }
   }
+  // otherwise the tensor-core prefill splits its last wave when the workspace allows it
+  size_t zero = sizeof(m3::DeviceStatus);
+  if (use_tc && d->seqlen > 0) {
+    const size_t sb = m3::tc_split_bytes(a);
+    if (sb > 0 && workspace_bytes >= kStatusBytes + sb) {
+      a.split = 1;
+      zero = m3::tc_split_zero_bytes(a);
+    }
+  }
+  if (cudaMemsetAsync(workspace, 0, zero, s) != cudaSuccess) return MAMBA3_ERR_CUDA;
   return use_tc ? m3::launch_scan_tc(a, s) : m3::launch_scan_simt(a, s);
 }
 
@@ -307,6 +318,20 @@ size_t mamba3_scan_segmented_workspace_bytes(const mamba3_dims* d) {
   m3::ScanArgs a = scan_args(d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
   const int S = g_test_segments ? forced_segments(a) : m3::seg_count(a, m3::kSMs);
   return kStatusBytes + m3::seg_workspace_bytes(a, S);
+}
+
+size_t mamba3_scan_fwd_workspace_bytes(const mamba3_dims* d) {
+  if (check_dims(d, true) != MAMBA3_OK) return 0;
+  m3::ScanArgs a = scan_args(d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  const int S = g_test_segments ? forced_segments(a) : m3::seg_count(a, m3::kSMs);
+  if (S > 0) return kStatusBytes + m3::seg_workspace_bytes(a, S);
+  return kStatusBytes + (d->seqlen > 0 ? m3::tc_split_bytes(a) : 0);
+}
+
+int mamba3_test_set_split(int k, int c1) {
+  if (k > 0 && c1 < 1) return MAMBA3_ERR_INVALID;
+  m3::tc_force_split(k, c1);
+  return MAMBA3_OK;
 }
 
 int mamba3_test_set_segments(int S) {

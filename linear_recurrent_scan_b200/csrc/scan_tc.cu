@@ -47,6 +47,12 @@
 #include <cuda.h>
 #include <string.h>
 
+#include <map>
+#include <mutex>
+#include <queue>
+#include <utility>
+#include <vector>
+
 #include "common.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
@@ -135,7 +141,9 @@ constexpr uint32_t kTmemCols = 512;
 // the epilogue writes y of chunk c while the MMAs of chunk c + 1 run.
 constexpr uint32_t kColS = 0, kColP = 128, kColY = 192, kColYi = 256, kColH = 320, kColYBuf = 192;
 
-enum Tag { kTagEmpty = 1, kTagFull, kTagPrep1, kTagSFull, kTagAcc, kTagEpiDone, kTagP, kTagY, kTagDrain, kTagTh };
+enum Tag {
+  kTagEmpty = 1, kTagFull, kTagPrep1, kTagSFull, kTagAcc, kTagEpiDone, kTagP, kTagY, kTagDrain, kTagTh, kTagHand, kTagXw
+};
 
 // kernel variants: the plain recurrence, the fused B/C norm, the time-varying decay A_t
 enum Variant { kPlain = 0, kBCNorm = 1, kTimeA = 2 };
@@ -152,6 +160,10 @@ struct Cfg {
   // y one chunk late (double-buffered Y, Yi): shortens the epilogue's chain;
   // measured faster for R = 1 only
   static constexpr bool DEFER_Y = (R == 1);
+  // X_w written by the epilogue warps (R = 1): prep bounds the chunk there, and the
+  // epilogue computes X_w while the S MMA runs; with R > 1 the epilogue is the
+  // longer role and prep keeps it
+  static constexpr bool XW_EPI = (R == 1);
   static constexpr int STAGE_BYTES = (2 * NKB + 1) * kTile;  // B, C, X
   static constexpr int TMA_BYTES = STAGE_BYTES;
   static constexpr int OFF_B = 0, OFF_C = NKB * kTile, OFF_X = 2 * NKB * kTile;
@@ -167,7 +179,7 @@ struct Cfg {
   static constexpr int OFF_PHI = OFF_PART + NPART * K2 * 4;            // running base angle [K2]
   static constexpr int OFF_WARP = OFF_PHI + K2 * 4;                     // scan scratch [8]
   static constexpr int OFF_BAR = (OFF_WARP + 32 + 7) & ~7;
-  static constexpr int NBAR = 16;
+  static constexpr int NBAR = 17;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
   // dt and lam of tokens [t0, t0 + Q] for the 8 heads of this head's 16-byte
   // group (TMA tiles [Q + 1][8] bf16, single buffer, refilled with theta)
@@ -198,7 +210,7 @@ struct Cfg {
 // barrier slots
 enum Bar {
   bFull0 = 0, bFull1, bEmptyBC0, bEmptyBC1, bPrep0, bPrep1, bSFull, bAcc, bEpiDone, bPReady, bYFull, bDone,
-  bThFull, bThFree, bEmptyX0, bEmptyX1
+  bThFull, bThFree, bEmptyX0, bEmptyX1, bXw
 };
 
 struct TcParams {
@@ -206,7 +218,24 @@ struct TcParams {
   int nchunks;
   int dl_tma;  // dt and lam arrive by TMA with theta (else: global loads one chunk ahead)
   int at_tma;  // a time-varying decay A_t arrives by TMA with theta (needs dl_tma)
+  // split last wave (split_k > 0): units 0 .. split_k - 1 run in two CTAs, chunks
+  // [0, split_c1) and [split_c1, nchunks); a CTA's work comes from a ticket
+  // (tickets 0 .. k-1: first parts; k .. U-1: whole units; U .. U+k-1: second parts)
+  int split_k, split_c1;
+  int* ticket;  // zeroed before the launch
+  int* flags;   // [split_k], zeroed: set once a first part has handed over
+  float* hand;  // [split_k][N P + N/2]: the carried state hbar and the angle at chunk split_c1
 };
+
+// acquire / release accesses of the hand-over flags (gpu scope)
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 __device__ __forceinline__ size_t tok_index(const ScanArgs& a, int b, int t, int h) {
   return ((size_t)b * a.seqlen + t) * a.nheads + h;
@@ -239,6 +268,32 @@ __device__ __forceinline__ bool prep_sync_any(bool v) {
 }
 __device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
+// X_w = diag(wsc) X of one chunk: thread i of 256 scales 16-byte chunks i, i + 256,
+// i + 512, i + 768 of the swizzled x tile (row = token rank row, wsc per token)
+template <int R>
+__device__ __forceinline__ void write_xw(uint8_t* xw, const uint8_t* x, const float* wsc, int i0) {
+  uint4 xq[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = i0 + 256 * i;
+    xq[i] = *reinterpret_cast<const uint4*>(x + swz(idx >> 3, idx & 7));
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = i0 + 256 * i;
+    const int row = idx >> 3, cc = idx & 7;
+    const float f = wsc[row / R];
+    const float2 f0 = unpack_bf16(xq[i].x), f1 = unpack_bf16(xq[i].y), f2 = unpack_bf16(xq[i].z),
+                 f3 = unpack_bf16(xq[i].w);
+    uint4 o;
+    o.x = pack_bf16(f * f0.x, f * f0.y);
+    o.y = pack_bf16(f * f1.x, f * f1.y);
+    o.z = pack_bf16(f * f2.x, f * f2.y);
+    o.w = pack_bf16(f * f3.x, f * f3.y);
+    *reinterpret_cast<uint4*>(xw + swz(row, cc)) = o;
+  }
+}
+
 // ------------------------------------------------------------------ prep warps
 // Thread pt in [0,256).  Per chunk: decay scalars (thread = token), accumulated
 // angles (thread = group g of 4 pairs x token part) and RoPE of B and C in
@@ -247,7 +302,8 @@ __device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 256;" ::
 // ahead into registers; theta arrives by TMA.
 template <int N, int R, int V>
 __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int dl_tma, int b, int hh,
-                                          float Ah, uint64_t* bars, volatile int* abort_flag, DeviceStatus* status) {
+                                          int c0, const float* hand_in, float* hand_out, float Ah, uint64_t* bars,
+                                          volatile int* abort_flag, DeviceStatus* status) {
   constexpr bool BCN = V == kBCNorm, TVA = V == kTimeA;
   using K = Cfg<N, R, V>;
   constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, TPP = K::TPP, TB = K::TB, NPART = K::NPART;
@@ -265,14 +321,17 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
   const __nv_bfloat16* LMu = static_cast<const __nv_bfloat16*>(a.lam) + (size_t)b * L * H + hh;
 
 
-  if (pt < K2) phi[pt] = a.angle0 ? a.angle0[unit * K2 + pt] : 0.f;
+  if (pt < K2) phi[pt] = hand_in ? __ldcg(hand_in + N * kP + pt) : (a.angle0 ? a.angle0[unit * K2 + pt] : 0.f);
+  // (this CTA's chunks start at chunk c0 of the sequence; only a part that ends the
+  // sequence exports the final state, a first part hands hbar and phi over instead)
+  const int t_last = (hand_out == nullptr && a.bprev_out != nullptr) ? L - 1 - c0 * Q : -1;
 
   // prefetched per chunk: (scan threads) dt, lam of token pt and of the next
   // token, and its decay rate (A_t, else A); (angle threads) dt of this part's tokens
   float s_dt, s_lm, s_dtn, s_lmn, s_at, p_dt[TPP];
   auto load_scalars = [&](int cc, float& o_dt, float& o_lm, float& o_dtn, float& o_lmn, float& o_at,
                           float (&o_pdt)[TPP]) {
-    const int tc0 = cc * Q;
+    const int tc0 = (c0 + cc) * Q;
     const int tg = tc0 + pt;
     const bool ok = pt < Q && cc < nchunks;
     o_at = Ah;
@@ -444,7 +503,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       for (int j = 0; j < TB * R; ++j) {
         const int jt = j / R, r = j % R;
         const int t = part * TPP + i0 + jt;
-        const bool export_row = last_chunk && (t0 + t == L - 1) && a.bprev_out != nullptr;
+        const bool export_row = last_chunk && (t0 + t == t_last);
         const uint32_t bw[4] = {bq[j].x, bq[j].y, bq[j].z, bq[j].w};
         const uint32_t cw[4] = {cq[j].x, cq[j].y, cq[j].z, cq[j].w};
         uint32_t bo[4], co[4];
@@ -498,8 +557,12 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
     if (part == NPART - 1) {  // the last part's running angle is the chunk's end angle
       *reinterpret_cast<float4*>(phi + 4 * g) =
           make_float4(wrap_angle(run[0]), wrap_angle(run[1]), wrap_angle(run[2]), wrap_angle(run[3]));
-      if (last_chunk && a.angle_out)
-        for (int k = 0; k < 4; ++k) a.angle_out[unit * K2 + 4 * g + k] = wrap_angle(run[k]);
+      if (last_chunk) {
+        float* ad = hand_out ? hand_out + N * kP : (a.angle_out ? a.angle_out + unit * K2 : nullptr);
+        if (ad)
+          for (int k = 0; k < 4; ++k) ad[4 * g + k] = wrap_angle(run[k]);
+        if (hand_out) __threadfence();
+      }
     }
     prep_sync();  // barrier 2: scalars complete, every part has read phi
 
@@ -512,34 +575,15 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       const int tj = j / R, tref = (32 * qq) / R;
       colf[pt] = ex2(c2[tref] - c2[tj]) * wv[tj];
     }
-    if (c > 0) mbar_wait(&bars[bAcc], (c - 1) & 1, abort_flag, status, kTagAcc, a.wait_limit);
-    if (prep_sync_any(*abort_flag != 0)) return;  // barrier 3: wsc visible, X_w free
-    {
-      uint4 xq[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int idx = pt + kNPrep * i;
-        xq[i] = *reinterpret_cast<const uint4*>(st + K::OFF_X + swz(idx >> 3, idx & 7));
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int idx = pt + kNPrep * i;
-        const int row = idx >> 3, cc = idx & 7;
-        const float f = wsc[row / R];
-        const float2 f0 = unpack_bf16(xq[i].x), f1 = unpack_bf16(xq[i].y), f2 = unpack_bf16(xq[i].z),
-                     f3 = unpack_bf16(xq[i].w);
-        uint4 o;
-        o.x = pack_bf16(f * f0.x, f * f0.y);
-        o.y = pack_bf16(f * f1.x, f * f1.y);
-        o.z = pack_bf16(f * f2.x, f * f2.y);
-        o.w = pack_bf16(f * f3.x, f * f3.y);
-        *reinterpret_cast<uint4*>(smem + K::OFF_XW + swz(row, cc)) = o;
-      }
+    if constexpr (!K::XW_EPI) {
+      if (c > 0) mbar_wait(&bars[bAcc], (c - 1) & 1, abort_flag, status, kTagAcc, a.wait_limit);
+      if (prep_sync_any(*abort_flag != 0)) return;  // barrier 3: wsc visible, X_w free
+      write_xw<R>(smem + K::OFF_XW, st + K::OFF_X, wsc, pt);
     }
     fence_proxy_async_smem();
-    mbar_arrive(&bars[bPrep0 + s]);
+    mbar_arrive(&bars[bPrep0 + s]);  // (releases wsc and the mask factors to the epilogue)
 
-    if (last_chunk && a.xprev_out && L > 0) {
+    if (last_chunk && hand_out == nullptr && a.xprev_out && L > 0) {
       const __nv_bfloat16* xl =
           static_cast<const __nv_bfloat16*>(a.x) + tok_index(a, b, L - 1, hh) * R * kP;
       for (int i = pt; i < R * kP; i += kNPrep) a.xprev_out[unit * R * kP + i] = __bfloat162float(xl[i]);
@@ -632,9 +676,10 @@ __device__ __forceinline__ void store_y_tma(const CUtensorMap* tmY, uint8_t* stg
 // half ch).  Row m of S, P, Y, Yi; state row n of Hacc / hbar (for N = 64 the
 // M = 64 accumulator uses lanes 0..15 of each 32-lane quadrant).
 template <int N, int R, int V>
-__device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh,
-                                         uint64_t* bars, volatile int* abort_flag, DeviceStatus* status,
-                                         uint32_t tmem, const CUtensorMap* tmY) {
+__device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh, int c0,
+                                         const float* hand_in, float* hand_out, uint64_t* bars,
+                                         volatile int* abort_flag, DeviceStatus* status, uint32_t tmem,
+                                         const CUtensorMap* tmY) {
   using K = Cfg<N, R, V>;
   constexpr int Q = K::Q;
   const int et = threadIdx.x - kEpi0;
@@ -659,7 +704,11 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
   float hb[32];
 #pragma unroll
   for (int p = 0; p < 32; ++p) hb[p] = 0.f;
-  if (n >= 0 && a.h0 != nullptr) {
+  if (n >= 0 && hand_in != nullptr) {  // a second part: hbar as the first part left it
+    const float* hi = hand_in + n * kP + 32 * ch;
+#pragma unroll
+    for (int p = 0; p < 32; ++p) hb[p] = __ldcg(hi + p);
+  } else if (n >= 0 && a.h0 != nullptr) {
     const size_t i0 = tok_index(a, b, 0, hh);
     const float mu1 = (1.f - __bfloat162float(static_cast<const __nv_bfloat16*>(a.lam)[i0])) *
                       __bfloat162float(static_cast<const __nv_bfloat16*>(a.dt)[i0]);
@@ -681,12 +730,20 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
   float e_prev = 0.f;  // (deferred y) e^{cum} of row m in the previous chunk
   for (int c = 0; c < nchunks; ++c) {
     const int s = c & 1, u = c >> 1;
-    const int t0 = c * Q;
+    const int t0 = (c0 + c) * Q;
     const float* sc = reinterpret_cast<const float*>(smem + K::OFF_SC) + s * K::SC_PER_STAGE;
     const float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *colf = sc + 4 * Q + colf_off;
 
-    // ---- S -> P (bf16, into TMEM) ----
     mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1, a.wait_limit);
+    if constexpr (K::XW_EPI) {
+      // ---- X_w of this chunk (the buffer's last reader, the previous chunk's state
+      // MMA, completed before this thread's previous state update), while S runs ----
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
+      write_xw<R>(smem + K::OFF_XW, smem + s * K::STAGE_BYTES + K::OFF_X, sc + 3 * Q, et);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[bXw]);
+    }
+    // ---- S -> P (bf16, into TMEM) ----
     mbar_wait(&bars[bSFull], c & 1, abort_flag, status, kTagSFull, a.wait_limit);
     if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
     tc_fence_after();
@@ -751,11 +808,12 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
       for (int p = 0; p < 16; ++p) hb[16 * half + p] = e_end * hb[16 * half + p] + acc[p];
     }
     store_hbar_bf16(hb, Hs, n, ch);
-    if (c == nchunks - 1 && a.h_out != nullptr && n >= 0) {
-      float* ho = a.h_out + (unit * N + n) * kP + 32 * ch;
+    if (c == nchunks - 1 && n >= 0 && (hand_out != nullptr || a.h_out != nullptr)) {
+      float* ho = hand_out ? hand_out + n * kP + 32 * ch : a.h_out + (unit * N + n) * kP + 32 * ch;
 #pragma unroll
       for (int p = 0; p < 32; p += 4)
         *reinterpret_cast<float4*>(ho + p) = make_float4(hb[p], hb[p + 1], hb[p + 2], hb[p + 3]);
+      if (hand_out) __threadfence();
     }
 
     // ---- y = Y + e^{cum_t} Yi ----
@@ -809,10 +867,11 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     const int cl = nchunks - 1;
     if constexpr (K::YBUF > 0)
       store_y_tma<K::YBUF - 1>(tmY, ystg + (cl % K::YBUF) * K::Y_TILE, tmem + lane_base + kColY + (cl & 1) * kColYBuf,
-                               tmem + lane_base + kColYi + (cl & 1) * kColYBuf, e_prev, b, hh, cl * Q + trow, ch, lane);
+                               tmem + lane_base + kColYi + (cl & 1) * kColYBuf, e_prev, b, hh, (c0 + cl) * Q + trow, ch,
+                               lane);
     else
       store_y(a, tmem + lane_base + kColY + (cl & 1) * kColYBuf, tmem + lane_base + kColYi + (cl & 1) * kColYBuf,
-              e_prev, b, hh, cl * Q + tm, rm, R, ch);
+              e_prev, b, hh, (c0 + cl) * Q + tm, rm, R, ch);
     tc_fence_before();
   }
 }
@@ -832,14 +891,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const ScanArgs& a = prm.a;
-  const int nchunks = prm.nchunks;
-  const int unit = blockIdx.x;
-  const int b = unit / a.nheads, hh = unit % a.nheads;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + K::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::OFF_MISC + 4);
+  volatile int* item_slot = reinterpret_cast<volatile int*>(smem + K::OFF_MISC + 8);
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.workspace);
+  const int units = a.batch * a.nheads;
 
   if (tid == 0) {
     mbar_init(&bars[bFull0], 1);
@@ -858,6 +916,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[bDone], 1);
     mbar_init(&bars[bThFull], 1);
     mbar_init(&bars[bThFree], kNPrep);
+    mbar_init(&bars[bXw], kNEpi);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmB);
@@ -869,6 +928,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmL);
     }
     if (prm.at_tma) prefetch_tmap(&tmA);
+    // this CTA's work: a whole unit (blockIdx), or with a split last wave the next
+    // ticket; a second part first waits (bounded) for its first part's hand-over
+    int item = blockIdx.x;
+    if (prm.split_k > 0) {
+      item = atomicAdd(prm.ticket, 1);
+      if (item >= units) {
+        const int* f = prm.flags + (item - units);
+        const long long t_start = clock64();
+        while (ld_acquire_gpu(f) == 0) {
+          if (clock64() - t_start > a.wait_limit) {
+            *abort_flag = 1;
+            report_timeout(status, kTagHand);
+            break;
+          }
+          __nanosleep(256);
+        }
+      }
+    }
+    *item_slot = item;
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -878,8 +956,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int item = *item_slot;
+  const bool skip = *abort_flag != 0;  // the hand-over never came: compute nothing
+  int unit = item, c0 = 0, nchunks = prm.nchunks;
+  const float* hand_in = nullptr;
+  float* hand_out = nullptr;
+  if (prm.split_k > 0) {
+    const size_t slot_floats = (size_t)N * kP + N / 2;
+    if (item < prm.split_k) {  // first part: chunks [0, c1), hands hbar and phi over
+      nchunks = prm.split_c1;
+      hand_out = prm.hand + (size_t)item * slot_floats;
+    } else if (item >= units) {  // second part: chunks [c1, n) from the hand-over
+      unit = item - units;
+      c0 = prm.split_c1;
+      nchunks -= c0;
+      hand_in = prm.hand + (size_t)unit * slot_floats;
+    }
+  }
+  const int b = unit / a.nheads, hh = unit % a.nheads;
 
-  if (warp == 0) {
+  if (skip) {
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       // Three refill streams, each issued as soon as its buffer is free:
@@ -896,7 +993,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (!a.test_withhold && (cx < nchunks || ct < nchunks)) {
         bool progress = false;
         if (cb < nchunks && mbar_test(&bars[bEmptyBC0 + (cb & 1)], ((cb >> 1) & 1) ^ 1)) {
-          const int s = cb & 1, t0 = cb * Q;
+          const int s = cb & 1, t0 = (c0 + cb) * Q;
           uint8_t* st = smem + s * K::STAGE_BYTES;
           mbar_arrive_expect_tx(&bars[bFull0 + s], K::TMA_BYTES);  // B, C and x of chunk cb
 #pragma unroll
@@ -909,12 +1006,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (cx < cb && mbar_test(&bars[bEmptyX0 + (cx & 1)], ((cx >> 1) & 1) ^ 1)) {
           const int s = cx & 1;
-          tma_load_5d(smem + s * K::STAGE_BYTES + K::OFF_X, &tmX, &bars[bFull0 + s], 0, 0, hh, cx * Q, b);
+          tma_load_5d(smem + s * K::STAGE_BYTES + K::OFF_X, &tmX, &bars[bFull0 + s], 0, 0, hh, (c0 + cx) * Q, b);
           ++cx;
           progress = true;
         }
         if (ct < nchunks && (ct == 0 || mbar_test(&bars[bThFree], (ct - 1) & 1))) {
-          const int t0 = ct * Q;
+          const int t0 = (c0 + ct) * Q;
           mbar_arrive_expect_tx(&bars[bThFull], th_bytes);
           tma_load_4d(smem + K::OFF_TH, &tmT, &bars[bThFull], 0, hh, t0, b);
           if (prm.dl_tma) {
@@ -941,7 +1038,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // stage whose x load was never issued (abort) gets it now, so that its
       // full barrier can complete.
       for (; cx < cb; ++cx)
-        tma_load_5d(smem + (cx & 1) * K::STAGE_BYTES + K::OFF_X, &tmX, &bars[bFull0 + (cx & 1)], 0, 0, hh, cx * Q, b);
+        tma_load_5d(smem + (cx & 1) * K::STAGE_BYTES + K::OFF_X, &tmX, &bars[bFull0 + (cx & 1)], 0, 0, hh,
+                    (c0 + cx) * Q, b);
       for (int c = cb - 2; c < cb; ++c)
         if (c >= 0 && !mbar_wait_drain(&bars[bFull0 + (c & 1)], (c >> 1) & 1)) report_timeout(status, kTagDrain);
       if (ct > 0 && !mbar_wait_drain(&bars[bThFull], (ct - 1) & 1)) report_timeout(status, kTagDrain);
@@ -976,6 +1074,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16_ss(tmem + kColYi + ybuf, smem_desc_sw128(cC + offa, 16, 1024),
                       smem_desc_sw128(sbase + K::OFF_H + kk * 2048, N * 128, 1024), iYi, kk > 0);
         }
+        if constexpr (K::XW_EPI) {  // X_w comes from the epilogue warps
+          if (!mbar_wait(&bars[bXw], c & 1, abort_flag, status, kTagXw, a.wait_limit)) break;
+          tc_fence_after();
+        }
 #pragma unroll
         for (int kk = 0; kk < kM / 16; ++kk) {
           mma_bf16_ss(tmem + kColH, smem_desc_sw128(cB + kk * 2048, kTile, 1024),
@@ -1000,9 +1102,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_drain(&bars[bDone], 0)) report_timeout(status, kTagDrain);
     }
   } else if (tid < kEpi0) {
-    prep_role<N, R, V>(smem, a, nchunks, prm.dl_tma, b, hh, a.A ? a.A[hh] : 0.f, bars, abort_flag, status);
+    prep_role<N, R, V>(smem, a, nchunks, prm.dl_tma, b, hh, c0, hand_in, hand_out, a.A ? a.A[hh] : 0.f, bars,
+                       abort_flag, status);
   } else {
-    epi_role<N, R, V>(smem, a, nchunks, b, hh, bars, abort_flag, status, tmem, &tmY);
+    epi_role<N, R, V>(smem, a, nchunks, b, hh, c0, hand_in, hand_out, bars, abort_flag, status, tmem, &tmY);
     // the y stores issued by this warp have read their staging tiles (and completed)
     if (K::YBUF > 0 && (tid & 31) == 0) bulk_wait_all();
   }
@@ -1012,6 +1115,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  // a first part releases its hand-over (written and fenced by the prep and
+  // epilogue threads before the barrier above), also after an abort, so that the
+  // second part never waits for a CTA that has ended
+  if (tid == 0 && hand_out != nullptr) {
+    __threadfence();
+    st_release_gpu(prm.flags + item, 1);
   }
 }
 
@@ -1031,6 +1141,75 @@ bool make_y_map(CUtensorMap* m, const ScanArgs& a) {
              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
+
+// ------------------------------------------------------------------ split last wave
+// U units on S SMs (one CTA each) run in ceil(U / S) waves, the last holding only
+// U mod S of them while the other SMs idle.  k units can instead run in two CTAs:
+// chunks [0, c1) early (tickets 0 .. k-1, ahead of the whole units) and [c1, n)
+// last (tickets U .. U+k-1), the second continuing from the carried state and
+// angle the first hands over, so the result is the one-CTA result bit for bit.
+// The plan minimises the makespan of the tickets' list schedule: a CTA takes its
+// chunks plus kFillChunks, and a second part starts no earlier than its first part
+// ends.  Plans are cached by (U, n).
+constexpr double kFillChunks = 2.0;  // pipeline fill and drain of a CTA, in chunk times
+constexpr size_t kSplitFlagBytes = 4;
+constexpr size_t kSplitRegion = kStatusBlockBytes;  // the split's flags and hand-over slots start here
+
+double split_makespan(int U, int n, int S, int k, int c1) {
+  std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+  for (int i = 0; i < S; ++i) free_at.push(0.0);
+  std::vector<double> first_end((size_t)k);
+  double span = 0.0;
+  auto run = [&](double ready, int chunks) {
+    double t = free_at.top();
+    free_at.pop();
+    if (t < ready) t = ready;
+    const double e = t + kFillChunks + chunks;
+    free_at.push(e);
+    if (e > span) span = e;
+    return e;
+  };
+  for (int i = 0; i < k; ++i) first_end[(size_t)i] = run(0.0, c1);
+  for (int i = k; i < U; ++i) run(0.0, n);
+  for (int i = 0; i < k; ++i) run(first_end[(size_t)i], n - c1);
+  return span;
+}
+
+SplitPlan plan_split(int U, int n, int S) {
+  SplitPlan best{0, 0};
+  if (U <= S || n < 2 || U % S == 0) return best;
+  const double base = split_makespan(U, n, S, 0, 0);
+  double best_span = base;
+  const int r = U % S;
+  const int dk[] = {0, 2, 4, 8, 12, 16, 24, 32};
+  const int step = n > 32 ? n / 32 : 1;
+  for (int d : dk) {
+    const int k = r + d;
+    if (k > U) break;
+    for (int c1 = step; c1 < n; c1 += step) {
+      const double span = split_makespan(U, n, S, k, c1);
+      if (span < best_span - 1e-9) {
+        best_span = span;
+        best = SplitPlan{k, c1};
+      }
+    }
+  }
+  // not worth two more CTAs' fill for less than 2 %
+  if (best_span > 0.98 * base) best = SplitPlan{0, 0};
+  return best;
+}
+
+std::mutex g_plan_mu;
+std::map<std::pair<int, int>, SplitPlan> g_plans;
+int g_force_k = 0, g_force_c1 = 0;
+
+int tc_chunks(const ScanArgs& a) {
+  const int Q = kM / a.R;
+  return (a.seqlen + Q - 1) / Q;
+}
+
+size_t split_slot_bytes(const ScanArgs& a) { return ((size_t)a.N * kP + a.N / 2) * sizeof(float); }
+size_t split_flag_region(int k) { return ((size_t)k * kSplitFlagBytes + 255) & ~(size_t)255; }
 
 template <int N, int R>
 int launch_nr(const ScanArgs& a, cudaStream_t s) {
@@ -1059,11 +1238,25 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
     prm.at_tma = prm.dl_tma && !a.bcnorm && make_dl_map(&tmA, a.A_t, a, K::Q);
     if (!prm.at_tma) prm.dl_tma = 0;
   }
+  prm.split_k = prm.split_c1 = 0;
+  prm.ticket = prm.flags = nullptr;
+  prm.hand = nullptr;
+  if (a.split) {  // the caller zeroed the ticket and the flags
+    const SplitPlan sp = tc_split_plan(a);
+    if (sp.k > 0) {
+      uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+      prm.split_k = sp.k;
+      prm.split_c1 = sp.c1;
+      prm.ticket = reinterpret_cast<int*>(ws + sizeof(DeviceStatus));
+      prm.flags = reinterpret_cast<int*>(ws + kSplitRegion);
+      prm.hand = reinterpret_cast<float*>(ws + kSplitRegion + split_flag_region(sp.k));
+    }
+  }
   auto kern = var == kBCNorm ? scan_tc_kernel<N, R, kBCNorm>
                              : (var == kTimeA ? scan_tc_kernel<N, R, kTimeA> : scan_tc_kernel<N, R, kPlain>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_alloc) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
-  kern<<<a.batch * a.nheads, kThreads, smem_alloc, s>>>(tmB, tmC, tmX, tmT, tmD, tmL, tmA, tmY, prm);
+  kern<<<a.batch * a.nheads + prm.split_k, kThreads, smem_alloc, s>>>(tmB, tmC, tmX, tmT, tmD, tmL, tmA, tmY, prm);
   return cudaGetLastError() == cudaSuccess ? MAMBA3_OK : MAMBA3_ERR_CUDA;
 }
 
@@ -1076,6 +1269,38 @@ int tc_scan_supported(const ScanArgs& a) {
   if (a.R != 1 && a.R != 2 && a.R != 4) return MAMBA3_ERR_UNSUPPORTED;
   if (a.Q != 0 && a.Q != kM / a.R) return MAMBA3_ERR_UNSUPPORTED;
   return MAMBA3_OK;
+}
+
+SplitPlan tc_split_plan(const ScanArgs& a) {
+  const int U = a.batch * a.nheads, n = tc_chunks(a);
+  std::lock_guard<std::mutex> lock(g_plan_mu);
+  if (g_force_k < 0) return SplitPlan{0, 0};
+  if (g_force_k > 0)  // a forced plan that does not fit the shape means no split
+    return (g_force_k <= U && g_force_c1 >= 1 && g_force_c1 < n) ? SplitPlan{g_force_k, g_force_c1} : SplitPlan{0, 0};
+  const auto key = std::make_pair(U, n);
+  auto it = g_plans.find(key);
+  if (it != g_plans.end()) return it->second;
+  const SplitPlan p = plan_split(U, n, kSMs);
+  g_plans[key] = p;
+  return p;
+}
+
+size_t tc_split_bytes(const ScanArgs& a) {
+  if (tc_scan_supported(a) != MAMBA3_OK) return 0;
+  const SplitPlan p = tc_split_plan(a);
+  if (p.k == 0) return 0;
+  return split_flag_region(p.k) + (size_t)p.k * split_slot_bytes(a);
+}
+
+size_t tc_split_zero_bytes(const ScanArgs& a) {
+  const SplitPlan p = tc_split_plan(a);
+  return kSplitRegion + split_flag_region(p.k);
+}
+
+void tc_force_split(int k, int c1) {
+  std::lock_guard<std::mutex> lock(g_plan_mu);
+  g_force_k = k;
+  g_force_c1 = c1;
 }
 
 int launch_scan_tc(const ScanArgs& a, cudaStream_t s) {
