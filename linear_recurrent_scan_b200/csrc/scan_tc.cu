@@ -754,10 +754,13 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     const float my_e = ex2(my_c2);
     const float e_end = ex2(c2[Q - 1]);
     const float rowf = ex2(my_c2 - c2[tref]);
+    // the two warps of a lane quadrant take alternate 16-column pieces (piece k of
+    // this warp: columns 32 k + 16 ch ..), so that each converts one half of the
+    // diagonal block, the costly one, and half of every other block
 #pragma unroll 1
     for (int k = 0; k < 4; ++k) {
-      const int cb = 2 * ch + (k >> 1);  // 32-column block of S
-      const int j0 = 32 * cb + 16 * (k & 1);  // first of this piece's 16 columns
+      const int cb = k;                  // 32-column block of S
+      const int j0 = 32 * cb + 16 * ch;  // first of this piece's 16 columns
       uint32_t pk[8];
       if (cb > quad) {  // warp-uniform: every column is a later token
 #pragma unroll
@@ -776,14 +779,16 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
             sv[4 * j4 + 3] *= cf.w * rowf;
           }
         } else {  // diagonal block: causal mask, trapezoid weights, D on the diagonal
+          // one factor per column token (the piece's 16 columns are 16 / R tokens of R ranks)
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int j = j0 + jj;
-            const int tj = j / R;
-            float kf = 0.f;
-            if (tj < tm) kf = ex2(my_c2 - c2[tj]) * wv[tj];
-            else if (tj == tm) kf = my_gam;
-            sv[jj] = sv[jj] * kf + (j == m ? Dh : 0.f);
+          for (int q = 0; q < 16 / R; ++q) {
+            const int tj = j0 / R + q;
+            const float kf = tj < tm ? ex2(my_c2 - c2[tj]) * wv[tj] : (tj == tm ? my_gam : 0.f);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              const int jj = q * R + r;
+              sv[jj] = sv[jj] * kf + (j0 + jj == m ? Dh : 0.f);
+            }
           }
         }
 #pragma unroll
