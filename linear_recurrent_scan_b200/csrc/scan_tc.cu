@@ -27,15 +27,17 @@
 //                of a stage are refilled once the state MMAs have read them, X
 //                once the Y MMA has; theta (+ dt, lam) into single tiles.
 //   warp 1       TMEM allocator and single-thread MMA issuer.
-//   warps 2..9   prep: decay scalars and the rank-1 decay factors of the mask,
-//                X_w = diag(e^{cum_end - cum_t} w_t) X, accumulated angles
-//                (wrapped) and RoPE of B and C in place, 16 bytes per access.
-//                Prep runs up to two chunks ahead of the MMAs.
-//   warps 10..17 epilogue, two warps per TMEM lane quadrant (column halves):
-//                S -> P (bf16, back into TMEM), hbar update and its bf16 copy
-//                for the next chunk's inter-chunk MMA, y = Y + e^{cum} Yi
-//                (with R = 1 for the previous chunk, so that the Y MMA's
-//                latency is off the epilogue's path).
+//   warps 2..9   prep: decay scalars, the row scale of X_w and the rank-1 decay
+//                factors of the mask, accumulated angles (wrapped) and RoPE of
+//                B and C in place, 16 bytes per access.  Prep bounds the chunk.
+//   warps 10..17 epilogue, two warps per TMEM lane quadrant: X_w =
+//                diag(e^{cum_end - cum_t} w_t) X while the S MMA runs, S -> P
+//                (bf16, back into TMEM; the two warps take alternate 16-column
+//                pieces), hbar update (column halves) and its bf16 copy for the
+//                next chunk's inter-chunk MMA, y = Y + e^{cum} Yi (with R = 1 for
+//                the previous chunk, so that the Y MMA's latency is off the
+//                epilogue's path).
+// With more units than SMs the last wave can be split (see the split plan below).
 // MMAs per chunk: S = C~ B~^T; Yi = C~ hbar_in; Hacc = B~^T X_w (smem operands);
 // Y = P X (P from TMEM).  TMEM columns: S [0,128), P [128,192) (bf16 pairs),
 // Y [192,256), Yi [256,320), Hacc [320,384); with R = 1 a second Y, Yi buffer at
@@ -160,10 +162,6 @@ struct Cfg {
   // y one chunk late (double-buffered Y, Yi): shortens the epilogue's chain;
   // measured faster for R = 1 only
   static constexpr bool DEFER_Y = (R == 1);
-  // X_w written by the epilogue warps (R = 1): prep bounds the chunk there, and the
-  // epilogue computes X_w while the S MMA runs; with R > 1 the epilogue is the
-  // longer role and prep keeps it
-  static constexpr bool XW_EPI = (R == 1);
   static constexpr int STAGE_BYTES = (2 * NKB + 1) * kTile;  // B, C, X
   static constexpr int TMA_BYTES = STAGE_BYTES;
   static constexpr int OFF_B = 0, OFF_C = NKB * kTile, OFF_X = 2 * NKB * kTile;
@@ -575,11 +573,6 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       const int tj = j / R, tref = (32 * qq) / R;
       colf[pt] = ex2(c2[tref] - c2[tj]) * wv[tj];
     }
-    if constexpr (!K::XW_EPI) {
-      if (c > 0) mbar_wait(&bars[bAcc], (c - 1) & 1, abort_flag, status, kTagAcc, a.wait_limit);
-      if (prep_sync_any(*abort_flag != 0)) return;  // barrier 3: wsc visible, X_w free
-      write_xw<R>(smem + K::OFF_XW, st + K::OFF_X, wsc, pt);
-    }
     fence_proxy_async_smem();
     mbar_arrive(&bars[bPrep0 + s]);  // (releases wsc and the mask factors to the epilogue)
 
@@ -735,7 +728,7 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     const float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *colf = sc + 4 * Q + colf_off;
 
     mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1, a.wait_limit);
-    if constexpr (K::XW_EPI) {
+    {
       // ---- X_w of this chunk (the buffer's last reader, the previous chunk's state
       // MMA, completed before this thread's previous state update), while S runs ----
       if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
@@ -1079,10 +1072,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16_ss(tmem + kColYi + ybuf, smem_desc_sw128(cC + offa, 16, 1024),
                       smem_desc_sw128(sbase + K::OFF_H + kk * 2048, N * 128, 1024), iYi, kk > 0);
         }
-        if constexpr (K::XW_EPI) {  // X_w comes from the epilogue warps
-          if (!mbar_wait(&bars[bXw], c & 1, abort_flag, status, kTagXw, a.wait_limit)) break;
-          tc_fence_after();
-        }
+        // X_w comes from the epilogue warps
+        if (!mbar_wait(&bars[bXw], c & 1, abort_flag, status, kTagXw, a.wait_limit)) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kM / 16; ++kk) {
           mma_bf16_ss(tmem + kColH, smem_desc_sw128(cB + kk * 2048, kTile, 1024),
