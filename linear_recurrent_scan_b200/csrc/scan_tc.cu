@@ -144,7 +144,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColP = 128, kColY = 192, kColYi = 256, kColH = 320, kColYBuf = 192;
 
 enum Tag {
-  kTagEmpty = 1, kTagFull, kTagPrep1, kTagSFull, kTagAcc, kTagEpiDone, kTagP, kTagY, kTagDrain, kTagTh, kTagHand, kTagXw
+  kTagEmpty = 1, kTagFull, kTagPrep1, kTagSFull, kTagAcc, kTagEpiDone, kTagP, kTagY, kTagDrain, kTagTh, kTagHand, kTagXw,
+  kTagNorm
 };
 
 // kernel variants: the plain recurrence, the fused B/C norm, the time-varying decay A_t
@@ -177,7 +178,7 @@ struct Cfg {
   static constexpr int OFF_PHI = OFF_PART + NPART * K2 * 4;            // running base angle [K2]
   static constexpr int OFF_WARP = OFF_PHI + K2 * 4;                     // scan scratch [8]
   static constexpr int OFF_BAR = (OFF_WARP + 32 + 7) & ~7;
-  static constexpr int NBAR = 17;
+  static constexpr int NBAR = 19;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
   // dt and lam of tokens [t0, t0 + Q] for the 8 heads of this head's 16-byte
   // group (TMA tiles [Q + 1][8] bf16, single buffer, refilled with theta)
@@ -186,13 +187,19 @@ struct Cfg {
   static constexpr int OFF_DL = (OFF_MISC + 16 + 127) & ~127;
   static constexpr int OFF_SINK = OFF_DL + 2 * DL_PAD;  // [Q] floats: consumes the tile reads
   // fused B/C normalisation (V = kBCNorm): w_B, bias_B, w_C, bias_C of this head,
-  // [R][N] floats each, then 1 / RMS of the chunk's raw B and C rows [2][128];
+  // [R][N] floats each;
   // time-varying decay by TMA (V = kTimeA): the A_t tile [Q][8] bf16 (refilled with
   // theta); nothing for the plain variant
   static constexpr int OFF_NRM = (OFF_SINK + Q * 4 + 127) & ~127;
   static constexpr int AT_BYTES = Q * 16;
+  // (R = 1: the epilogue warps normalise the raw rows in place two chunks ahead; R > 1,
+  // where the epilogue has no time to spare: prep applies the norm in its rotation,
+  // from 1 / RMS of every raw row [2][128] computed first)
+  static constexpr bool EPI_NORM = V == kBCNorm && R == 1;
+  static constexpr bool PREP_NORM = V == kBCNorm && R > 1;
   static constexpr int OFF_RINV = OFF_NRM + 4 * R * N * 4;
-  static constexpr int NRM_BYTES = V == kBCNorm ? 4 * R * N * 4 + 2 * kM * 4 : (V == kTimeA ? AT_BYTES : 0);
+  static constexpr int NRM_BYTES = V == kBCNorm ? 4 * R * N * 4 + (PREP_NORM ? 2 * kM * 4 : 0)
+                                                : (V == kTimeA ? AT_BYTES : 0);
   // y staging where shared memory allows (N = 64; N = 128 with R = 4 except the
   // fused norm): per epilogue warp one or two
   // 32-row x 64-byte tiles (64-byte swizzle) that the warp writes out with a TMA store
@@ -208,7 +215,7 @@ struct Cfg {
 // barrier slots
 enum Bar {
   bFull0 = 0, bFull1, bEmptyBC0, bEmptyBC1, bPrep0, bPrep1, bSFull, bAcc, bEpiDone, bPReady, bYFull, bDone,
-  bThFull, bThFree, bEmptyX0, bEmptyX1, bXw
+  bThFull, bThFree, bEmptyX0, bEmptyX1, bXw, bNorm0, bNorm1
 };
 
 struct TcParams {
@@ -361,7 +368,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
   const __nv_bfloat16* lms = reinterpret_cast<const __nv_bfloat16*>(smem + K::OFF_DL + K::DL_PAD) + (hh & 7);
   float* sink = reinterpret_cast<float*>(smem + K::OFF_SINK);
   const float* nrm = reinterpret_cast<const float*>(smem + K::OFF_NRM);
-  if constexpr (BCN) {  // this head's normalisation weights and biases, [4][R][N]
+  if constexpr (K::PREP_NORM) {  // this head's normalisation weights and biases, [4][R][N]
     float* nw = reinterpret_cast<float*>(smem + K::OFF_NRM);
     const size_t base = (size_t)hh * R * N;
     for (int i = pt; i < R * N; i += kNPrep) {
@@ -422,11 +429,13 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
     mbar_arrive(&bars[bThFree]);
     const float4 base = *reinterpret_cast<const float4*>(phi + 4 * g);
     mbar_wait(&bars[bFull0 + s], u & 1, abort_flag, status, kTagFull, a.wait_limit);
+    // (fused norm) the epilogue warps have normalised this chunk's raw B and C rows in place
+    if constexpr (K::EPI_NORM) mbar_wait(&bars[bNorm0 + s], u & 1, abort_flag, status, kTagNorm, a.wait_limit);
     if (prep_sync_any(*abort_flag != 0)) return;  // barrier 1: one decision for all prep threads
 
     // ---- phase B: scalars, prefix of the angle, RoPE ----
     float* rinv = reinterpret_cast<float*>(smem + K::OFF_RINV);
-    if constexpr (BCN) {
+    if constexpr (K::PREP_NORM) {
       // 1 / RMS of every raw row of the chunk, thread = row (B rows: pt < 128, C rows:
       // the rest): 16-byte reads of the whole row, no cross-lane reduction; an
       // all-zero row with eps = 0 (e.g. the padding past the sequence end) gives 0
@@ -505,7 +514,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
         const uint32_t bw[4] = {bq[j].x, bq[j].y, bq[j].z, bq[j].w};
         const uint32_t cw[4] = {cq[j].x, cq[j].y, cq[j].z, cq[j].w};
         uint32_t bo[4], co[4];
-        if constexpr (BCN) {
+        if constexpr (K::PREP_NORM) {
           // raw row (t, r): its 1 / RMS from the pass above, weight and bias, then the rotation
           float bv[8], cv[8];
 #pragma unroll
@@ -664,6 +673,54 @@ __device__ __forceinline__ void store_y_tma(const CUtensorMap* tmY, uint8_t* stg
   }
 }
 
+// Fused B/C norm of one chunk in place (raw -> w * row / RMS(row) + bias, bf16):
+// thread et of the 256 epilogue threads owns row et of B (et < 128) or row et - 128
+// of C, reads it whole in 16-byte pieces for its sum of squares (no cross-lane
+// reduction), then rewrites it; all lanes of a warp read the same weights (R = 1)
+// or R of them, so those reads are broadcasts.  An all-zero row with eps = 0 (the
+// padding past the sequence end) gives 1 / RMS = 0.
+template <int N, int R, int V>
+__device__ __forceinline__ void bc_normalise(uint8_t* st, const float* nw, float eps, int et) {
+  using K = Cfg<N, R, V>;
+  const int row = et & (kM - 1);
+  const bool is_c = et >= kM;
+  uint8_t* tile = st + (is_c ? K::OFF_C : K::OFF_B);
+  const float* w = nw + (is_c ? 2 : 0) * R * N + (row % R) * N;  // weight [n]; bias at + R N
+  float ss = 0.f;
+#pragma unroll
+  for (int kb = 0; kb < K::NKB; ++kb)
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+      const uint4 q = *reinterpret_cast<const uint4*>(tile + kb * kTile + swz(row, c8));
+      const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = unpack_bf16(qw[k]);
+        ss += f.x * f.x + f.y * f.y;
+      }
+    }
+  const float vr = ss * (1.f / N) + eps;
+  const float ri = vr > 0.f ? rsqrtf(vr) : 0.f;
+#pragma unroll 2
+  for (int kb = 0; kb < K::NKB; ++kb)
+#pragma unroll 2
+    for (int c8 = 0; c8 < 8; ++c8) {
+      uint4* p = reinterpret_cast<uint4*>(tile + kb * kTile + swz(row, c8));
+      const uint4 q = *p;
+      const int n0 = kb * 64 + c8 * 8;
+      const float4 w0 = *reinterpret_cast<const float4*>(w + n0), w1 = *reinterpret_cast<const float4*>(w + n0 + 4);
+      const float4 b0 = *reinterpret_cast<const float4*>(w + R * N + n0),
+                   b1 = *reinterpret_cast<const float4*>(w + R * N + n0 + 4);
+      const float2 f0 = unpack_bf16(q.x), f1 = unpack_bf16(q.y), f2 = unpack_bf16(q.z), f3 = unpack_bf16(q.w);
+      uint4 o;
+      o.x = pack_bf16(f0.x * ri * w0.x + b0.x, f0.y * ri * w0.y + b0.y);
+      o.y = pack_bf16(f1.x * ri * w0.z + b0.z, f1.y * ri * w0.w + b0.w);
+      o.z = pack_bf16(f2.x * ri * w1.x + b1.x, f2.y * ri * w1.y + b1.y);
+      o.w = pack_bf16(f3.x * ri * w1.z + b1.z, f3.y * ri * w1.w + b1.w);
+      *p = o;
+    }
+}
+
 // ------------------------------------------------------------------ epilogue warps
 // Two warps per TMEM lane quadrant: thread = (row m = 32 quad + lane, column
 // half ch).  Row m of S, P, Y, Yi; state row n of Hacc / hbar (for N = 64 the
@@ -719,6 +776,30 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
   store_hbar_bf16(hb, Hs, n, ch);
   fence_proxy_async_smem();
   mbar_arrive(&bars[bEpiDone]);
+
+  // (fused norm, R = 1) this head's weights and biases [4][R][N], then chunks 0 and 1;
+  // chunk c + 2 follows at the end of chunk c, in the time the epilogue would wait for prep
+  float* nw = reinterpret_cast<float*>(smem + K::OFF_NRM);
+  auto normalise = [&](int cn) -> bool {
+    const int sn = cn & 1;
+    if (!mbar_wait(&bars[bFull0 + sn], (cn >> 1) & 1, abort_flag, status, kTagFull, a.wait_limit)) return false;
+    bc_normalise<N, R, V>(smem + sn * K::STAGE_BYTES, nw, a.neps, et);
+    fence_proxy_async_smem();  // the stage is refilled by TMA later
+    mbar_arrive(&bars[bNorm0 + sn]);
+    return true;
+  };
+  if constexpr (K::EPI_NORM) {
+    const size_t base = (size_t)hh * R * N;
+    for (int i = et; i < R * N; i += kNEpi) {
+      nw[i] = a.nw_B ? a.nw_B[base + i] : 1.f;
+      nw[R * N + i] = a.nb_B ? a.nb_B[base + i] : 0.f;
+      nw[2 * R * N + i] = a.nw_C ? a.nw_C[base + i] : 1.f;
+      nw[3 * R * N + i] = a.nb_C ? a.nb_C[base + i] : 0.f;
+    }
+    asm volatile("bar.sync 2, 256;" ::: "memory");  // the epilogue warps' named barrier
+    for (int cn = 0; cn < 2 && cn < nchunks; ++cn)
+      if (!normalise(cn)) return;
+  }
 
   float e_prev = 0.f;  // (deferred y) e^{cum} of row m in the previous chunk
   for (int c = 0; c < nchunks; ++c) {
@@ -857,6 +938,9 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     tc_fence_before();
     fence_proxy_async_smem();  // hbar (bf16) is read by the next chunk's MMA
     mbar_arrive(&bars[bEpiDone]);
+    if constexpr (K::EPI_NORM) {
+      if (c + 2 < nchunks && !normalise(c + 2)) return;
+    }
   }
   if constexpr (K::DEFER_Y) {  // y of the last chunk (the Y barrier is committed for it alone)
     mbar_wait(&bars[bYFull], 0, abort_flag, status, kTagY, a.wait_limit);
@@ -915,6 +999,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[bThFull], 1);
     mbar_init(&bars[bThFree], kNPrep);
     mbar_init(&bars[bXw], kNEpi);
+    mbar_init(&bars[bNorm0], kNEpi);
+    mbar_init(&bars[bNorm1], kNEpi);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmB);
