@@ -110,7 +110,9 @@ MAMBA3_API size_t mamba3_scan_workspace_bytes(const mamba3_dims* dims);
  *                non-null.  It may alias `init` (in-place continuation).
  *   workspace    device memory of at least mamba3_scan_workspace_bytes(dims);
  *                its status word is reset by this call and read back with
- *                mamba3_device_status.
+ *                mamba3_device_status.  With mamba3_scan_fwd_workspace_bytes(dims)
+ *                the call also runs its long-sequence segments or its split
+ *                last wave (declared below), which give the same y and state.
  * Numerics: float32 arithmetic and state; bf16 inputs feed bf16 tensor-core
  * products with float32 accumulation.  y is written in in_dtype.
  */
