@@ -113,6 +113,10 @@ MAMBA3_API size_t mamba3_scan_workspace_bytes(const mamba3_dims* dims);
  *                mamba3_device_status.  With mamba3_scan_fwd_workspace_bytes(dims)
  *                the call also runs its long-sequence segments or its split
  *                last wave (declared below), which give the same y and state.
+ *                A workspace serves one call at a time: calls that overlap on
+ *                the GPU need workspaces of their own (a split launch that
+ *                draws a ticket past its range, which only a shared workspace
+ *                causes, computes nothing and reports MAMBA3_ERR_TIMEOUT).
  * Numerics: float32 arithmetic and state; bf16 inputs feed bf16 tensor-core
  * products with float32 accumulation.  y is written in in_dtype.
  */
@@ -428,7 +432,9 @@ MAMBA3_API int mamba3_test_withhold_loads(int on);
  *  - Every call on a device shares the same scratch and it keeps the last
  *    call's contents; the parts that must start at zero (the device status
  *    word) are cleared by each call on its stream.  Calls that overlap on the
- *    GPU (different streams without ordering between them) race on it.
+ *    GPU (different streams without ordering between them) race on it.  For
+ *    that reason this entry point never splits the last wave (see
+ *    mamba3_scan_fwd_workspace_bytes).
  *  - The device status word stays in the library's scratch: use
  *    mamba3_scan_fwd with a caller workspace when mamba3_device_status is needed.
  */

@@ -150,6 +150,14 @@ SplitPlan tc_split_plan(const ScanArgs& a);
 size_t tc_split_bytes(const ScanArgs& a);
 size_t tc_split_zero_bytes(const ScanArgs& a);
 void tc_force_split(int k, int c1);
+
+// mamba3_scan_fwd on a scratch that every call on the device shares (the no-alloc
+// entry point): never splits the last wave, whose tickets and hand-over flags would
+// then be shared by overlapping calls (mamba3_api.cu).
+int scan_fwd_shared_scratch(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                            const void* dt, const void* lam, const float* A, const float* D,
+                            const mamba3_state* init, void* y, const mamba3_state* final_state, void* scratch,
+                            size_t scratch_bytes, void* stream);
 int seg_count(const ScanArgs& a, int sms);
 // CTAs of the segment-state kernel that share an SM for these sizes (1 or 2)
 int seg_state_ctas_per_sm(const ScanArgs& a);

@@ -132,7 +132,8 @@ m3::ScanArgs scan_args(const mamba3_dims* d, const void* x, const void* B, const
 int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
                   const void* dt, const void* lam, const float* A, const void* A_t, const float* D,
                   const mamba3_bc_norm* norm, const mamba3_state* init, void* y,
-                  const mamba3_state* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+                  const mamba3_state* final_state, void* workspace, size_t workspace_bytes, void* stream,
+                  bool allow_split = true) {
   int rc = check_dims(d, true);
   if (rc) return rc;
   const float* A_chk = A ? A : static_cast<const float*>(A_t);  // the rate array that must be present
@@ -167,7 +168,7 @@ int scan_fwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
   }
   // otherwise the tensor-core prefill splits its last wave when the workspace allows it
   size_t zero = sizeof(m3::DeviceStatus);
-  if (use_tc && d->seqlen > 0) {
+  if (use_tc && allow_split && d->seqlen > 0) {
     const size_t sb = m3::tc_split_bytes(a);
     if (sb > 0 && workspace_bytes >= kStatusBytes + sb) {
       a.split = 1;
@@ -217,6 +218,20 @@ int mamba3_scan_fwd(const mamba3_dims* d, const void* x, const void* B, const vo
   return scan_fwd_impl(d, x, B, C, theta, dt, lam, A, nullptr, D, nullptr, init, y, final_state, workspace,
                        workspace_bytes, stream);
 }
+
+}  // extern "C"
+
+namespace m3 {
+int scan_fwd_shared_scratch(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
+                            const void* dt, const void* lam, const float* A, const float* D,
+                            const mamba3_state* init, void* y, const mamba3_state* final_state, void* scratch,
+                            size_t scratch_bytes, void* stream) {
+  return scan_fwd_impl(d, x, B, C, theta, dt, lam, A, nullptr, D, nullptr, init, y, final_state, scratch,
+                       scratch_bytes, stream, /*allow_split=*/false);
+}
+}  // namespace m3
+
+extern "C" {
 
 int mamba3_scan_fwd_at(const mamba3_dims* d, const void* x, const void* B, const void* C, const void* theta,
                        const void* dt, const void* lam, const void* A_t, const float* D, const mamba3_state* init,

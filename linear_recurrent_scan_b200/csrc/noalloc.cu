@@ -4,6 +4,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "internal.h"
 
 namespace {
 
@@ -43,6 +44,6 @@ extern "C" int mamba3_scan_fwd_noalloc(const mamba3_dims* dims, const void* x, c
   const int rc = scratch_for_current_device(&scratch);
   if (rc != MAMBA3_OK) return rc;
   // mamba3_scan_fwd clears the status word on `stream` before its kernels run
-  return mamba3_scan_fwd(dims, x, B, C, theta, dt, lam, A, D, init, y, final_state, scratch,
-                         MAMBA3_NOALLOC_SCRATCH_BYTES, stream);
+  return m3::scan_fwd_shared_scratch(dims, x, B, C, theta, dt, lam, A, D, init, y, final_state, scratch,
+                                     MAMBA3_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -145,7 +145,7 @@ constexpr uint32_t kColS = 0, kColP = 128, kColY = 192, kColYi = 256, kColH = 32
 
 enum Tag {
   kTagEmpty = 1, kTagFull, kTagPrep1, kTagSFull, kTagAcc, kTagEpiDone, kTagP, kTagY, kTagDrain, kTagTh, kTagHand, kTagXw,
-  kTagNorm
+  kTagNorm, kTagTicket
 };
 
 // kernel variants: the plain recurrence, the fused B/C norm, the time-varying decay A_t
@@ -1017,7 +1017,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int item = blockIdx.x;
     if (prm.split_k > 0) {
       item = atomicAdd(prm.ticket, 1);
-      if (item >= units) {
+      if (item >= units + prm.split_k) {
+        // a ticket past this launch's range: another launch shares the workspace
+        // (overlapping calls on one workspace race); compute nothing, touch no slot
+        *abort_flag = 1;
+        report_timeout(status, kTagTicket);
+        item = 0;
+      } else if (item >= units) {
         const int* f = prm.flags + (item - units);
         const long long t_start = clock64();
         while (ld_acquire_gpu(f) == 0) {
@@ -1045,7 +1051,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int unit = item, c0 = 0, nchunks = prm.nchunks;
   const float* hand_in = nullptr;
   float* hand_out = nullptr;
-  if (prm.split_k > 0) {
+  if (prm.split_k > 0 && !skip) {
     const size_t slot_floats = (size_t)N * kP + N / 2;
     if (item < prm.split_k) {  // first part: chunks [0, c1), hands hbar and phi over
       nchunks = prm.split_c1;
