@@ -305,8 +305,8 @@ __device__ __forceinline__ void write_xw(uint8_t* xw, const uint8_t* x, const fl
 // place (16 bytes per shared-memory access, 2 rows in flight), the rank-1
 // column factors of the mask and X_w.  dt and lam are prefetched one chunk
 // ahead into registers; theta arrives by TMA.
-template <int N, int R, int V>
-__device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int dl_tma, int b, int hh,
+template <int N, int R, int V, bool dl_tma>
+__device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int nchunks, int b, int hh,
                                           int c0, const float* hand_in, float* hand_out, float Ah, uint64_t* bars,
                                           volatile int* abort_flag, DeviceStatus* status) {
   constexpr bool BCN = V == kBCNorm, TVA = V == kTimeA;
@@ -354,7 +354,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       o_pdt[i] = (cc < nchunks && tp < L) ? __bfloat162float(DTu[(size_t)tp * H]) : 0.f;
     }
   };
-  if (dl_tma) {
+  if constexpr (dl_tma) {
     s_dt = s_dtn = 0.f;
     s_lm = s_lmn = 1.f;
     s_at = Ah;
@@ -390,7 +390,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
 
     // ---- phase A (no shared state): in-warp scan of dt*A*log2(e); theta of this part ----
     mbar_wait(&bars[bThFull], c & 1, abort_flag, status, kTagTh, a.wait_limit);
-    if (dl_tma) {  // this chunk's dt and lam from the tile (rows past the sequence read 0)
+    if constexpr (dl_tma) {  // this chunk's dt and lam from the tile (rows past the sequence read 0)
       if (pt < Q) {
         s_dt = __bfloat162float(dts[pt * 8]);
         s_lm = __bfloat162float(lms[pt * 8]);
@@ -484,7 +484,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
 #pragma unroll
     for (int i = 0; i < TPP; ++i) pdt_cur[i] = p_dt[i];
     // next chunk's scalars, in flight during the rotation (unless they come by TMA)
-    if (!dl_tma) load_scalars(c + 1, s_dt, s_lm, s_dtn, s_lmn, s_at, p_dt);
+    if constexpr (!dl_tma) load_scalars(c + 1, s_dt, s_lm, s_dtn, s_lmn, s_at, p_dt);
 #pragma unroll
     for (int i0 = 0; i0 < TPP; i0 += TB) {
       float sn[TB][4], cs[TB][4];
@@ -958,7 +958,9 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
   }
 }
 
-template <int N, int R, int V>
+// DL: dt and lam arrive by TMA with theta (a compile-time choice, so that the
+// global-load path's prefetch registers are not live in the TMA kernel's rotation)
+template <int N, int R, int V, bool DL>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
@@ -1007,7 +1009,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmC);
     prefetch_tmap(&tmX);
     prefetch_tmap(&tmT);
-    if (prm.dl_tma) {
+    if (DL) {
       prefetch_tmap(&tmD);
       prefetch_tmap(&tmL);
     }
@@ -1078,7 +1080,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int gh = hh / (prm.a.nheads / prm.a.ngroups);  // the B/C row this head reads
       long long t_last = clock64();
       const uint32_t th_bytes =
-          K::TH_BYTES + (prm.dl_tma ? 2u * K::DL_BYTES : 0u) + (prm.at_tma ? (uint32_t)K::AT_BYTES : 0u);
+          K::TH_BYTES + (DL ? 2u * K::DL_BYTES : 0u) + (prm.at_tma ? (uint32_t)K::AT_BYTES : 0u);
       // (test_withhold: issue nothing, so that every wait on a load must time out)
       while (!a.test_withhold && (cx < nchunks || ct < nchunks)) {
         bool progress = false;
@@ -1104,7 +1106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t0 = (c0 + ct) * Q;
           mbar_arrive_expect_tx(&bars[bThFull], th_bytes);
           tma_load_4d(smem + K::OFF_TH, &tmT, &bars[bThFull], 0, hh, t0, b);
-          if (prm.dl_tma) {
+          if (DL) {
             tma_load_3d(smem + K::OFF_DL, &tmD, &bars[bThFull], hh & ~7, t0, b);
             tma_load_3d(smem + K::OFF_DL + K::DL_PAD, &tmL, &bars[bThFull], hh & ~7, t0, b);
           }
@@ -1191,7 +1193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_drain(&bars[bDone], 0)) report_timeout(status, kTagDrain);
     }
   } else if (tid < kEpi0) {
-    prep_role<N, R, V>(smem, a, nchunks, prm.dl_tma, b, hh, c0, hand_in, hand_out, a.A ? a.A[hh] : 0.f, bars,
+    prep_role<N, R, V, DL>(smem, a, nchunks, b, hh, c0, hand_in, hand_out, a.A ? a.A[hh] : 0.f, bars,
                        abort_flag, status);
   } else {
     epi_role<N, R, V>(smem, a, nchunks, b, hh, c0, hand_in, hand_out, bars, abort_flag, status, tmem, &tmY);
@@ -1341,8 +1343,12 @@ int launch_nr(const ScanArgs& a, cudaStream_t s) {
       prm.hand = reinterpret_cast<float*>(ws + kSplitRegion + split_flag_region(sp.k));
     }
   }
-  auto kern = var == kBCNorm ? scan_tc_kernel<N, R, kBCNorm>
-                             : (var == kTimeA ? scan_tc_kernel<N, R, kTimeA> : scan_tc_kernel<N, R, kPlain>);
+  auto kern = prm.dl_tma ? (var == kBCNorm ? scan_tc_kernel<N, R, kBCNorm, true>
+                                           : (var == kTimeA ? scan_tc_kernel<N, R, kTimeA, true>
+                                                            : scan_tc_kernel<N, R, kPlain, true>))
+                        : (var == kBCNorm ? scan_tc_kernel<N, R, kBCNorm, false>
+                                          : (var == kTimeA ? scan_tc_kernel<N, R, kTimeA, false>
+                                                           : scan_tc_kernel<N, R, kPlain, false>));
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_alloc) != cudaSuccess)
     return MAMBA3_ERR_CUDA;
   kern<<<a.batch * a.nheads + prm.split_k, kThreads, smem_alloc, s>>>(tmB, tmC, tmX, tmT, tmD, tmL, tmA, tmY, prm);
