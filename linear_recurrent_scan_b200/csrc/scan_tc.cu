@@ -196,6 +196,11 @@ struct Cfg {
   // where the epilogue has no time to spare: prep applies the norm in its rotation,
   // from 1 / RMS of every raw row [2][128] computed first)
   static constexpr bool EPI_NORM = V == kBCNorm && R == 1;
+  // the exported B~ of the last token computed after the rotation loop (fewer live
+  // registers in the loop) rather than inside it: measured faster for N = 128 with
+  // R = 1 and N = 64 with R = 4 (2 % each), slower for the other shapes (register
+  // allocation differs); never with the epilogue-side norm (the raw row is gone)
+  static constexpr bool EXPORT_AFTER = !EPI_NORM && ((N == 128 && R == 1) || (N == 64 && R == 4));
   static constexpr bool PREP_NORM = V == kBCNorm && R > 1;
   static constexpr int OFF_RINV = OFF_NRM + 4 * R * N * 4;
   static constexpr int NRM_BYTES = V == kBCNorm ? 4 * R * N * 4 + (PREP_NORM ? 2 * kM * 4 : 0)
@@ -510,7 +515,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       for (int j = 0; j < TB * R; ++j) {
         const int jt = j / R, r = j % R;
         const int t = part * TPP + i0 + jt;
-        const bool export_row = last_chunk && (t0 + t == t_last);
+        const bool export_row = !K::EXPORT_AFTER && last_chunk && (t0 + t == t_last);
         const uint32_t bw[4] = {bq[j].x, bq[j].y, bq[j].z, bq[j].w};
         const uint32_t cw[4] = {cq[j].x, cq[j].y, cq[j].z, cq[j].w};
         uint32_t bo[4], co[4];
@@ -559,6 +564,40 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
         const uint32_t off = kb * kTile + swz(t * R + r, c8);
         *reinterpret_cast<uint4*>(st + K::OFF_B + off) = make_uint4(bo[0], bo[1], bo[2], bo[3]);
         *reinterpret_cast<uint4*>(st + K::OFF_C + off) = make_uint4(co[0], co[1], co[2], co[3]);
+      }
+    }
+    if (K::EXPORT_AFTER && last_chunk && t_last >= t0 && t_last < t0 + Q && (t_last - t0) / TPP == part) {
+      // B~ of the sequence's last token in fp32 for the exported state: the part's
+      // running angle is that token's (padding tokens add dt = 0), and its raw row
+      // is read again from global memory, rotated with the loop's arithmetic
+      const int tl = t_last - t0;
+      const int gh = hh / (H / a.ngroups);
+      float snl[4], csl[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) __sincosf(run[k], &snl[k], &csl[k]);
+      const __nv_bfloat16* brow = static_cast<const __nv_bfloat16*>(a.B) +
+                                  (((size_t)b * L + (size_t)(c0 * Q + t_last)) * a.ngroups + gh) * R * N + 8 * g;
+      for (int r = 0; r < R; ++r) {
+        const uint4 q = *reinterpret_cast<const uint4*>(brow + r * N);
+        const uint32_t bw[4] = {q.x, q.y, q.z, q.w};
+        float bv[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = unpack_bf16(bw[k]);
+          bv[2 * k] = f.x;
+          bv[2 * k + 1] = f.y;
+        }
+        if constexpr (K::PREP_NORM) {  // as in the loop: 1 / RMS of the row, weight and bias
+          const float ib = reinterpret_cast<const float*>(smem + K::OFF_RINV)[tl * R + r];
+          const float* wB = nrm + r * N + 8 * g;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) bv[e] = bv[e] * ib * wB[e] + wB[R * N + e];
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k] = csl[k] * bv[2 * k] + snl[k] * bv[2 * k + 1];
+          a.bprev_out[(unit * R + r) * N + 8 * g + 2 * k + 1] = csl[k] * bv[2 * k + 1] - snl[k] * bv[2 * k];
+        }
       }
     }
     if (part == NPART - 1) {  // the last part's running angle is the chunk's end angle
