@@ -1415,6 +1415,7 @@ SplitPlan tc_split_plan(const ScanArgs& a) {
   auto it = g_plans.find(key);
   if (it != g_plans.end()) return it->second;
   const SplitPlan p = plan_split(U, n, kSMs);
+  if (g_plans.size() >= 4096) g_plans.clear();  // (bounded: callers with ever-new shapes)
   g_plans[key] = p;
   return p;
 }

@@ -75,3 +75,21 @@ def test_host_prefill_back_to_back_reuses_the_stage():
         y_d = m3.mamba3_scan_fwd(*(inp[n] for n in NAMES), inp["A"], inp["D"])
         torch.cuda.synchronize()
         assert torch.equal(y_h, y_d.cpu())
+
+
+def test_host_prefill_of_no_tokens_passes_the_state_through():
+    """seqlen 0: nothing is copied; the final state is the initial one."""
+    b, H, P, N, R = 2, 4, 64, 128, 1
+    inp = small_inputs(b, 1, H, P, N, R, torch.bfloat16, seed=8400)
+    host = {n: inp[n][:, :0].cpu().contiguous().pin_memory() for n in NAMES}
+    init = rand_state(b, H, P, N, R, 8401)
+    fin = m3.State.zeros(b, H, P, N, R)
+    dims = m3.make_dims(host["x"], host["B"])
+    stage = torch.zeros(m3.mamba3_scan_fwd_host_stage_bytes(dims), dtype=torch.uint8, device="cuda")
+    y = m3.mamba3_scan_fwd_host(*(host[n] for n in NAMES), inp["A"], inp["D"], init=init, final_state=fin,
+                                stage=stage)
+    torch.cuda.synchronize()
+    assert y.shape[1] == 0
+    assert m3.mamba3_device_status(stage) == m3.MAMBA3_OK
+    for n in ("h", "b_prev", "x_prev", "angle"):
+        assert torch.equal(getattr(fin, n), getattr(init, n)), n
