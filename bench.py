@@ -43,20 +43,20 @@ BACKWARD_KERNEL = "bwd_state_kernel + bwd_chunk_kernel (tcgen05, TMA)"
 # capture).  A kernel whose sources no longer hash to the recorded value gets
 # traffic null, since its counters are out of date.
 TRAFFIC = {
-    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "a95a7e3ec365e6f4892dc9f7331e01d5518982a9e6115a2084d83a5287c15348",
-                814220288 + 135966464, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
-    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "a95a7e3ec365e6f4892dc9f7331e01d5518982a9e6115a2084d83a5287c15348",
-                               5655534080 + 1071639040, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "d08afa02947a8903c6a1b21fa1875530b6e18ed495eb8c36c0bb19a1bfaf216c",
+                813621248 + 136253440, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "d08afa02947a8903c6a1b21fa1875530b6e18ed495eb8c36c0bb19a1bfaf216c",
+                               5652974336 + 1069713920, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     # the segmented prefill: seg_state_kernel + seg_combine_kernel + scan_tc_kernel of one call
-    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "46c99dcbcd395dbb31d7bebbecb905e0cdc5781fb312090acc5f4d9541a23123",
-                             4590971392 + 36402688 + 38102016 + 426752 + 6772917504 + 2122883840,
+    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "7e93e46f4e00c13aa1be9329b305ad1424fc02bb0601f6c26c9ce1f5ac4cd504",
+                             4590874880 + 36291840 + 38103296 + 108544 + 6772763648 + 2123679744,
                              "profiles/segmented_prefill_mimo4_b1_l65536.txt"),
     "siso_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                          283177728 + 219681280, "profiles/decode_stream_b128_traffic_and_counters.txt"),
     "mimo4_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                           317789952 + 241042432, "profiles/decode_stream_b128_traffic_and_counters.txt"),
-    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "a95a7e3ec365e6f4892dc9f7331e01d5518982a9e6115a2084d83a5287c15348",
-                        284614656 + 121699072, "profiles/grouped_bc_prefill_decode_traffic.txt"),
+    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "d08afa02947a8903c6a1b21fa1875530b6e18ed495eb8c36c0bb19a1bfaf216c",
+                        284710656 + 121127424, "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "grouped_decode": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                        279047936 + 219645952, "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "backward": (('scan_bwd_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "4e0c7c64d7cdf0641dc3706bae97f8049f27d153a1436da0552077c3f5ea4781",
