@@ -250,6 +250,15 @@ MAMBA3_API int mamba3_decode_step_at(const mamba3_dims* dims, const mamba3_state
  *                 Q = 32 / rank tokens, N P + N/2 floats; with grouped B/C then
  *                 the same fp32 group sums (2 * batch * seqlen * ngroups * rank *
  *                 dstate floats; each head adds its share with atomics).
+ *                 With more (b, h) units than the 148 SMs the tensor-core path
+ *                 also splits the last wave of its reverse sweep (as the prefill
+ *                 does, see mamba3_scan_fwd_workspace_bytes): the CTA that sweeps
+ *                 a unit's end hands the adjoint of the carried state, the running
+ *                 angle-gradient sum and one token's pending dt, lam gradient share
+ *                 over to the CTA that sweeps its start; mamba3_scan_bwd_workspace_bytes
+ *                 includes that region (256 bytes, then k + 1 counters rounded up to
+ *                 256 bytes and k (N P + N/2 + 4) floats), and a workspace of the
+ *                 size above without it runs unsplit.
  * Products on the tensor cores take bf16 operands with float32 accumulation;
  * everything else is float32.  Returns MAMBA3_ERR_UNSUPPORTED for N, P whose
  * per-chunk tiles exceed shared memory.

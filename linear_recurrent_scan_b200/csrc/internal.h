@@ -60,6 +60,7 @@ struct BwdArgs {
   void* dA_t;  // with f.A_t: the decay-rate gradient per token (layout of dt, dtype of x); dA null
   float *dh0, *dbprev0, *dxprev0, *dangle0;                      // all null = not wanted
   float* ckpt;  // [units][chunks][N*P + N/2]: hbar and Phi at every chunk start
+  int split;         // the tensor-core backward may split its last wave (bwd_tc_split_bytes fit)
   float *dBh, *dCh;  // grouped B, C: fp32 scratch for their gradients (SIMT path: per head
                      // [b, L, H, R, N], summed afterwards; tensor-core path: the group sums
                      // [b, L, G, R, N] themselves); null with one row per head
@@ -147,6 +148,12 @@ struct SplitPlan {
   int k, c1;
 };
 SplitPlan tc_split_plan(const ScanArgs& a);
+// the cached plan for `units` units of `nchunks` chunks each (tc_force_split applies;
+// c1 counts the chunks of the kernel that asks)
+SplitPlan split_plan(int units, int nchunks);
+// the backward chunk kernel's split (scan_bwd_tc.cu): workspace after the checkpoints
+// and group sums, 0 without a split
+size_t bwd_tc_split_bytes(const ScanArgs& a);
 size_t tc_split_bytes(const ScanArgs& a);
 size_t tc_split_zero_bytes(const ScanArgs& a);
 void tc_force_split(int k, int c1);

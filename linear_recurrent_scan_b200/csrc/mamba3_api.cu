@@ -406,6 +406,9 @@ int scan_bwd_impl(const mamba3_dims* d, const void* x, const void* B, const void
   g.ckpt = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_tc) {
+    // the chunk kernel splits its last wave when the workspace holds the hand-over
+    const size_t sb = d->seqlen > 0 ? m3::bwd_tc_split_bytes(sizes) : 0;
+    g.split = sb > 0 && workspace_bytes >= kStatusBytes + need + sb;
     if (cudaMemsetAsync(workspace, 0, sizeof(m3::DeviceStatus), s) != cudaSuccess) return MAMBA3_ERR_CUDA;
     return m3::launch_scan_bwd_tc(g, s);
   }
@@ -423,7 +426,8 @@ extern "C" {
 size_t mamba3_scan_bwd_workspace_bytes(const mamba3_dims* d) {
   if (check_dims(d, true) != MAMBA3_OK) return 0;
   const m3::ScanArgs a = scan_args(d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
-  if (m3::bwd_tc_supported(a) == MAMBA3_OK) return kStatusBytes + m3::bwd_tc_workspace_bytes(a);
+  if (m3::bwd_tc_supported(a) == MAMBA3_OK)  // (with the split last wave's hand-over where it applies)
+    return kStatusBytes + m3::bwd_tc_workspace_bytes(a) + (d->seqlen > 0 ? m3::bwd_tc_split_bytes(a) : 0);
   return kStatusBytes + m3::bwd_checkpoint_bytes(a) + m3::bwd_group_bytes(a);
 }
 

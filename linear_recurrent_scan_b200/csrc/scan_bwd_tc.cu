@@ -59,7 +59,24 @@ constexpr int kBlk = 8192;    // one 64-row x 128-byte swizzled tile
 constexpr int kNScal = 16;    // per-token scalar arrays
 constexpr int kScalStride = 80;  // >= Q + 1
 
-enum Tag { kTagFull = 21, kTagMma1, kTagMma2, kTagDrain2 };
+enum Tag { kTagFull = 21, kTagMma1, kTagMma2, kTagDrain2, kTagHand2, kTagTicket2 };
+
+// split last wave of the chunk kernel (k = 0: one CTA per unit)
+struct BwdSplit {
+  int k, c1;
+  int* ticket;  // zeroed before the launch
+  int* flags;   // [k], zeroed
+  float* hand;  // [k][N P + N/2 + 4]
+};
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 // byte offset of 16-byte chunk c (0..7) of row `row` inside a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t swz(int row, int c) { return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4)); }
@@ -467,7 +484,8 @@ template <int N, int R, bool TVA, bool GRP>
 __global__ void __launch_bounds__(kCThreads, 1)
     bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                      const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDY,
-                     const __grid_constant__ CUtensorMap tmT, const BwdArgs g, const uint8_t* ckpt, int nchunks) {
+                     const __grid_constant__ CUtensorMap tmT, const BwdArgs g, const uint8_t* ckpt, int nchunks,
+                     const BwdSplit sp) {
   using K = CCfg<N, R>;
   constexpr int Q = K::Q, K2 = K::K2, NG = K::NG, NPA = K::NPA, TPP = K::TPP, NKB = K::NKB;
   constexpr int NPART2 = K::NPART2, TPP2 = K::TPP2, QP = K::QP;
@@ -476,14 +494,62 @@ __global__ void __launch_bounds__(kCThreads, 1)
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const ScanArgs& a = g.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int unit = blockIdx.x;
-  const int b = unit / a.nheads, hh = unit % a.nheads;
-  const int L = a.seqlen;
-  const int gh = hh / (a.nheads / a.ngroups);
+  const int units = a.batch * a.nheads;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + K::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::OFF_MISC + 4);
+  volatile int* item_slot = reinterpret_cast<volatile int*>(smem + K::OFF_MISC + 8);
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.workspace);
+  // this CTA's work: a whole unit (blockIdx), or with a split last wave the next
+  // ticket (0..k-1: the end of units 0..k-1, chunks [c1, n), marched first; k..U-1:
+  // whole units; U..U+k-1: chunks [0, c1) of units 0..k-1, from the hand-over of the
+  // adjoint state, the running angle-gradient sum and the pending token)
+  if (tid == 0) {
+    *abort_flag = 0;
+    int item = blockIdx.x;
+    if (sp.k > 0) {
+      item = atomicAdd(sp.ticket, 1);
+      if (item >= units + sp.k) {  // only a workspace shared by overlapping calls gives one
+        *abort_flag = 1;
+        report_timeout(status, kTagTicket2);
+        item = 0;
+      } else if (item >= units) {
+        const int* f = sp.flags + (item - units);
+        const long long t_start = clock64();
+        while (ld_acquire_gpu(f) == 0) {
+          if (clock64() - t_start > a.wait_limit) {
+            *abort_flag = 1;
+            report_timeout(status, kTagHand2);
+            break;
+          }
+          __nanosleep(256);
+        }
+      }
+    }
+    *item_slot = item;
+  }
+  __syncthreads();
+  const int item = *item_slot;
+  const bool skip = *abort_flag != 0;
+  int unit = item, c_top = nchunks - 1, r_end = nchunks;
+  const float* hand_in = nullptr;
+  float* hand_out = nullptr;
+  constexpr int kSlot = N * kP + K::K2 + 4;  // G, the angle-gradient sum, the pending ddt and dlam
+  if (sp.k > 0 && !skip) {
+    if (item < sp.k) {  // the end of the sequence: chunks [c1, n), then the hand-over
+      r_end = nchunks - sp.c1;
+      hand_out = sp.hand + (size_t)item * kSlot;
+    } else if (item >= units) {  // chunks [0, c1) from the hand-over
+      unit = item - units;
+      c_top = sp.c1 - 1;
+      r_end = sp.c1;
+      hand_in = sp.hand + (size_t)unit * kSlot;
+    }
+  }
+  if (skip) r_end = 0;
+  const int b = unit / a.nheads, hh = unit % a.nheads;
+  const int L = a.seqlen;
+  const int gh = hh / (a.nheads / a.ngroups);
   float* sc = reinterpret_cast<float*>(smem + K::OFF_SC);
   float* part_sum = reinterpret_cast<float*>(smem + K::OFF_PART);
   float* sang = reinterpret_cast<float*>(smem + K::OFF_SANG);
@@ -507,11 +573,10 @@ __global__ void __launch_bounds__(kCThreads, 1)
   const float Ah = TVA ? 0.f : a.A[hh];
   const float Dh = a.D ? a.D[hh] : 0.f;
   const size_t ck_unit = (size_t)unit * nchunks;
-  const float* ckphi = reinterpret_cast<const float*>(ckpt + (size_t)gridDim.x * nchunks * K::HB_BYTES);
+  const float* ckphi = reinterpret_cast<const float*>(ckpt + (size_t)units * nchunks * K::HB_BYTES);
 
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
-    *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmC);
@@ -523,7 +588,8 @@ __global__ void __launch_bounds__(kCThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (tid < K2) sang[tid] = g.dangle_out ? g.dangle_out[(size_t)unit * K2 + tid] : 0.f;
+  if (tid < K2)
+    sang[tid] = hand_in ? __ldcg(hand_in + N * kP + tid) : (g.dangle_out ? g.dangle_out[(size_t)unit * K2 + tid] : 0.f);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -544,7 +610,10 @@ __global__ void __launch_bounds__(kCThreads, 1)
   float G[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) G[i] = 0.f;
-  if (n >= 0 && g.dh_out) {
+  if (n >= 0 && hand_in) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) G[i] = __ldcg(hand_in + n * kP + p0 + i);
+  } else if (n >= 0 && g.dh_out) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) G[i] = g.dh_out[((size_t)unit * N + n) * kP + p0 + i];
   }
@@ -562,9 +631,9 @@ __global__ void __launch_bounds__(kCThreads, 1)
   };
   store_G();
 
-  // loads of chunk c (reverse index r = nchunks - 1 - c: stage r & 1, phase (r >> 1) & 1)
+  // loads of chunk c (reverse index r = c_top - c: stage r & 1, phase (r >> 1) & 1)
   auto issue = [&](int c) {
-    const int r = nchunks - 1 - c, s = r & 1;
+    const int r = c_top - c, s = r & 1;
     uint8_t* st = smem + s * K::STAGE;
     const int t0 = c * Q;
     mbar_arrive_expect_tx(&bars[s], (uint32_t)K::LOAD_BYTES);
@@ -591,21 +660,26 @@ __global__ void __launch_bounds__(kCThreads, 1)
     }
   };
   int issued = 0;  // chunks (in reverse order) whose loads were issued
-  if (tid == 0 && !a.test_withhold) { issue(nchunks - 1); issued = 1; }
-  load_scalars(nchunks - 1);
+  if (tid == 0 && !a.test_withhold && r_end > 0) { issue(c_top); issued = 1; }
+  load_scalars(c_top);
   // pending (thread 0): ddt, dlam of the first token of the chunk processed last,
   // without its lagged share, which the next chunk processed (the one before it) supplies
   float pend_ddt = 0.f, pend_dlm = 0.f, dA_acc = 0.f, dD_acc = 0.f;
   int pend_t = -1;
+  if (hand_in && tid == 0) {  // the first token after this part waits for its lagged share
+    pend_t = (c_top + 1) * Q;
+    pend_ddt = __ldcg(hand_in + N * kP + K2);
+    pend_dlm = __ldcg(hand_in + N * kP + K2 + 1);
+  }
   int abort_r = -1, abort_stage = 0;  // where an abort happened (0: loads, 1: batch 1, 2: batch 2)
   const int ag = tid % NG, apart = tid / NG;   // angle scan: 4-pair group, token part
   const int akb = ag / 8, ac8 = ag % 8;
 
-  for (int r = 0; r < nchunks; ++r) {
-    const int c = nchunks - 1 - r, s = r & 1;
+  for (int r = 0; r < r_end; ++r) {
+    const int c = c_top - r, s = r & 1;
     uint8_t* st = smem + s * K::STAGE;
     const int t0 = c * Q;
-    if (tid == 0 && c >= 1 && !a.test_withhold) {
+    if (tid == 0 && r + 1 < r_end && !a.test_withhold) {
       fence_proxy_async_smem();  // the stage's previous generic reads before the TMA refill
       issue(c - 1);
       issued = r + 2;
@@ -1146,7 +1220,9 @@ __global__ void __launch_bounds__(kCThreads, 1)
     __syncthreads();
   }
 
-  if (abort_r >= 0) {
+  if (skip) {
+    // (no ticket in range, or the hand-over never came: nothing was issued)
+  } else if (abort_r >= 0) {
     if (tid == 0) {
       // let what was issued land before TMEM is freed and the CTA exits: the
       // loads not yet waited for and the MMA batch the abort interrupted
@@ -1155,6 +1231,27 @@ __global__ void __launch_bounds__(kCThreads, 1)
       if (abort_stage > 0 && !mbar_wait_drain(&bars[1 + abort_stage], abort_r & 1))
         report_timeout(status, kTagDrain2);
     }
+  } else if (hand_out) {
+    // ---- the end of a split unit: its dA and dD shares into the globals; G, the
+    // running angle-gradient sum and the pending token's ddt, dlam to the hand-over ----
+    if (tid < 4) red[1 + tid] = 0.f;
+    __syncthreads();
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, o);
+    if (lane == 0) atomicAdd(&red[2], dD_acc);
+    if (n >= 0) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) hand_out[n * kP + p0 + i] = G[i];
+    }
+    for (int k = tid; k < K2; k += kCThreads) hand_out[N * kP + k] = sang[(r_end & 1) * K2 + k];
+    __syncthreads();
+    if (tid == 0) {
+      hand_out[N * kP + K2] = pend_ddt;
+      hand_out[N * kP + K2 + 1] = pend_dlm;
+      if (!TVA) atomicAdd(g.dA + hh, dA_acc);
+      if (g.dD) atomicAdd(g.dD + hh, red[2]);
+    }
+    __threadfence();
   } else {
     // ---- the initial state: hbar_in of the first chunk = h_0 + mu1 sum_r b_prev0[r]^T x_prev0[r] ----
     float* Gs = reinterpret_cast<float*>(smem);  // [N][P] f32 in the stage buffers (no loads pending)
@@ -1210,7 +1307,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
           for (int nn = 0; nn < N; ++nn) s2 += Gs[nn * kP + pp] * a.bprev0[((size_t)unit * R + rr) * N + nn];
         g.dxprev0[(size_t)unit * R * kP + i] = mu1 * s2;
       }
-      for (int k = tid; k < K2; k += kCThreads) g.dangle0[(size_t)unit * K2 + k] = sang[(nchunks & 1) * K2 + k];
+      for (int k = tid; k < K2; k += kCThreads) g.dangle0[(size_t)unit * K2 + k] = sang[(r_end & 1) * K2 + k];
     }
   }
   tc_fence_before();
@@ -1218,6 +1315,12 @@ __global__ void __launch_bounds__(kCThreads, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+  // the end of a split unit releases its hand-over (also after an abort, so that the
+  // CTA of the unit's start never waits for one that has ended)
+  if (tid == 0 && hand_out != nullptr) {
+    __threadfence();
+    st_release_gpu(sp.flags + item, 1);
   }
 }
 
@@ -1254,7 +1357,22 @@ int launch_nr(const BwdArgs& g, cudaStream_t s) {
     return MAMBA3_ERR_CUDA;
   ks<<<units, kSThreads, SK::SMEM_ALLOC, s>>>(tmB, tmX, tmT, a, ckpt, nchunks);
   if (cudaGetLastError() != cudaSuccess) return MAMBA3_ERR_CUDA;
-  kc<<<units, kCThreads, CK::SMEM_ALLOC, s>>>(tmB, tmC, tmX, tmDY, tmT, g, ckpt, nchunks);
+  BwdSplit sp;
+  memset(&sp, 0, sizeof(sp));
+  if (g.split) {  // the region after the checkpoints and group sums (bwd_tc_split_bytes)
+    const SplitPlan p = split_plan(units, nchunks);
+    if (p.k > 0) {
+      uint8_t* region = static_cast<uint8_t*>(a.workspace) + 256 + ((bwd_tc_workspace_bytes(a) + 255) & ~(size_t)255);
+      const size_t flag_bytes = ((size_t)(p.k + 1) * 4 + 255) & ~(size_t)255;
+      sp.k = p.k;
+      sp.c1 = p.c1;
+      sp.ticket = reinterpret_cast<int*>(region);
+      sp.flags = sp.ticket + 1;
+      sp.hand = reinterpret_cast<float*>(region + flag_bytes);
+      if (cudaMemsetAsync(region, 0, flag_bytes, s) != cudaSuccess) return MAMBA3_ERR_CUDA;
+    }
+  }
+  kc<<<units + sp.k, kCThreads, CK::SMEM_ALLOC, s>>>(tmB, tmC, tmX, tmDY, tmT, g, ckpt, nchunks, sp);
   if (cudaGetLastError() != cudaSuccess) return MAMBA3_ERR_CUDA;
   if (GRP) {
     const long long total4 = (long long)a.batch * a.seqlen * a.ngroups * R * N / 4;
@@ -1282,6 +1400,15 @@ int bwd_tc_supported(const ScanArgs& a) {
   if (a.R != 1 && a.R != 2 && a.R != 4) return MAMBA3_ERR_UNSUPPORTED;
   if (a.nheads % a.ngroups != 0) return MAMBA3_ERR_INVALID;
   return MAMBA3_OK;
+}
+
+size_t bwd_tc_split_bytes(const ScanArgs& a) {
+  if (bwd_tc_supported(a) != MAMBA3_OK) return 0;
+  const int Q = 64 / a.R, nchunks = (a.seqlen + Q - 1) / Q;
+  const SplitPlan p = split_plan(a.batch * a.nheads, nchunks);
+  if (p.k == 0) return 0;
+  const size_t slot = ((size_t)a.N * kP + a.N / 2 + 4) * sizeof(float);
+  return 256 + (((size_t)(p.k + 1) * 4 + 255) & ~(size_t)255) + (size_t)p.k * slot;  // (256: alignment)
 }
 
 size_t bwd_tc_workspace_bytes(const ScanArgs& a) {

@@ -1405,8 +1405,9 @@ int tc_scan_supported(const ScanArgs& a) {
   return MAMBA3_OK;
 }
 
-SplitPlan tc_split_plan(const ScanArgs& a) {
-  const int U = a.batch * a.nheads, n = tc_chunks(a);
+SplitPlan tc_split_plan(const ScanArgs& a) { return split_plan(a.batch * a.nheads, tc_chunks(a)); }
+
+SplitPlan split_plan(int U, int n) {
   std::lock_guard<std::mutex> lock(g_plan_mu);
   if (g_force_k < 0) return SplitPlan{0, 0};
   if (g_force_k > 0)  // a forced plan that does not fit the shape means no split
