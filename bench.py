@@ -43,24 +43,24 @@ BACKWARD_KERNEL = "bwd_state_kernel + bwd_chunk_kernel (tcgen05, TMA)"
 # capture).  A kernel whose sources no longer hash to the recorded value gets
 # traffic null, since its counters are out of date.
 TRAFFIC = {
-    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "d08afa02947a8903c6a1b21fa1875530b6e18ed495eb8c36c0bb19a1bfaf216c",
-                813621248 + 136253440, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
-    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "d08afa02947a8903c6a1b21fa1875530b6e18ed495eb8c36c0bb19a1bfaf216c",
-                               5652974336 + 1069713920, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "4b5b269d3c8df1587116e4af8a91b2ba36333bfcf25926e3b609ca78939b1341",
+                813646080 + 136545536, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "4b5b269d3c8df1587116e4af8a91b2ba36333bfcf25926e3b609ca78939b1341",
+                               5653630208 + 1070447872, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     # the segmented prefill: seg_state_kernel + seg_combine_kernel + scan_tc_kernel of one call
-    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "7e93e46f4e00c13aa1be9329b305ad1424fc02bb0601f6c26c9ce1f5ac4cd504",
-                             4590874880 + 36291840 + 38103296 + 108544 + 6772763648 + 2123679744,
+    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "aab0626961fb70866e1ad0f8392560a6f1c44650cce669e3188aa04ce8412bc7",
+                             4591002880 + 36278016 + 38109440 + 381696 + 6773376256 + 2123267072,
                              "profiles/segmented_prefill_mimo4_b1_l65536.txt"),
     "siso_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                          283177728 + 219681280, "profiles/decode_stream_b128_traffic_and_counters.txt"),
     "mimo4_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                           317789952 + 241042432, "profiles/decode_stream_b128_traffic_and_counters.txt"),
-    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "d08afa02947a8903c6a1b21fa1875530b6e18ed495eb8c36c0bb19a1bfaf216c",
-                        284710656 + 121127424, "profiles/grouped_bc_prefill_decode_traffic.txt"),
+    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "4b5b269d3c8df1587116e4af8a91b2ba36333bfcf25926e3b609ca78939b1341",
+                        284955648 + 121807104, "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "grouped_decode": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                        279047936 + 219645952, "profiles/grouped_bc_prefill_decode_traffic.txt"),
-    "backward": (('scan_bwd_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "4e0c7c64d7cdf0641dc3706bae97f8049f27d153a1436da0552077c3f5ea4781",
-                 541800448 + 240511488 + 1218752768 + 787912960,
+    "backward": (('scan_bwd_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "58bdeb0f1b41cb82988d2c19c9a1ca646f603380d204215b052a7ef1a9d4bf3b",
+                 542074880 + 240609280 + 1223284992 + 785020160,
                  "profiles/scan_bwd_tc_siso_b8_l2048_traffic_and_counters.txt"),
     "mimo_proj_up": (('mimo_proj.cu', 'sm100_ptx.cuh', 'common.cuh'), "c2a412f8cf230533471e6093ea6ca476f1bedd003f0d0f0a07475de750bfd4e2",
                      406625280 + 1016199424, "profiles/mimo_proj_b4_l8192_traffic.txt"),
