@@ -196,6 +196,9 @@ struct Cfg {
   // where the epilogue has no time to spare: prep applies the norm in its rotation,
   // from 1 / RMS of every raw row [2][128] computed first)
   static constexpr bool EPI_NORM = V == kBCNorm && R == 1;
+  // X_w by the epilogue warps, except with the epilogue-side norm, which leaves the
+  // epilogue the longer role: then prep writes it (after the previous state MMA)
+  static constexpr bool XW_PREP = EPI_NORM;
   // the exported B~ of the last token computed after the rotation loop (fewer live
   // registers in the loop) rather than inside it: measured faster for N = 128 with
   // R = 1 and N = 64 with R = 4 (2 % each), slower for the other shapes (register
@@ -621,6 +624,13 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
       const int tj = j / R, tref = (32 * qq) / R;
       colf[pt] = ex2(c2[tref] - c2[tj]) * wv[tj];
     }
+    if constexpr (K::XW_PREP) {
+      if (c > 0) mbar_wait(&bars[bAcc], (c - 1) & 1, abort_flag, status, kTagAcc, a.wait_limit);
+      if (prep_sync_any(*abort_flag != 0)) return;  // wsc visible, X_w free
+      write_xw<R>(smem + K::OFF_XW, st + K::OFF_X, wsc, pt);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[bXw]);
+    }
     fence_proxy_async_smem();
     mbar_arrive(&bars[bPrep0 + s]);  // (releases wsc and the mask factors to the epilogue)
 
@@ -848,7 +858,7 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
     const float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *colf = sc + 4 * Q + colf_off;
 
     mbar_wait(&bars[bPrep0 + s], u & 1, abort_flag, status, kTagPrep1, a.wait_limit);
-    {
+    if constexpr (!K::XW_PREP) {
       // ---- X_w of this chunk (the buffer's last reader, the previous chunk's state
       // MMA, completed before this thread's previous state update), while S runs ----
       if (__any_sync(0xffffffffu, *abort_flag != 0)) return;
