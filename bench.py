@@ -43,24 +43,24 @@ BACKWARD_KERNEL = "bwd_state_kernel + bwd_chunk_kernel (tcgen05, TMA)"
 # capture).  A kernel whose sources no longer hash to the recorded value gets
 # traffic null, since its counters are out of date.
 TRAFFIC = {
-    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "4b5b269d3c8df1587116e4af8a91b2ba36333bfcf25926e3b609ca78939b1341",
-                813646080 + 136545536, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
-    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "4b5b269d3c8df1587116e4af8a91b2ba36333bfcf25926e3b609ca78939b1341",
-                               5653630208 + 1070447872, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "3b9a2962b96e1b1c16aeeb51b2236b60fb9c7920234041f4f35107e7f24011b4",
+                813935104 + 136358144, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "3b9a2962b96e1b1c16aeeb51b2236b60fb9c7920234041f4f35107e7f24011b4",
+                               5655001856 + 1070696448, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     # the segmented prefill: seg_state_kernel + seg_combine_kernel + scan_tc_kernel of one call
-    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "aab0626961fb70866e1ad0f8392560a6f1c44650cce669e3188aa04ce8412bc7",
-                             4591002880 + 36278016 + 38109440 + 381696 + 6773376256 + 2123267072,
+    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "e2579662912f23b06257e6fce771729caa05e8090e5236f7351108ba21b69ee7",
+                             4590568448 + 36562944 + 38102784 + 131072 + 6774374912 + 2123151872,
                              "profiles/segmented_prefill_mimo4_b1_l65536.txt"),
     "siso_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                          283177728 + 219681280, "profiles/decode_stream_b128_traffic_and_counters.txt"),
     "mimo4_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                           317789952 + 241042432, "profiles/decode_stream_b128_traffic_and_counters.txt"),
-    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "4b5b269d3c8df1587116e4af8a91b2ba36333bfcf25926e3b609ca78939b1341",
-                        284955648 + 121807104, "profiles/grouped_bc_prefill_decode_traffic.txt"),
+    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "3b9a2962b96e1b1c16aeeb51b2236b60fb9c7920234041f4f35107e7f24011b4",
+                        284650496 + 121850368, "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "grouped_decode": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                        279047936 + 219645952, "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "backward": (('scan_bwd_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "58bdeb0f1b41cb82988d2c19c9a1ca646f603380d204215b052a7ef1a9d4bf3b",
-                 542074880 + 240609280 + 1223284992 + 785020160,
+                 541825792 + 240689408 + 1223041280 + 784799232,
                  "profiles/scan_bwd_tc_siso_b8_l2048_traffic_and_counters.txt"),
     "mimo_proj_up": (('mimo_proj.cu', 'sm100_ptx.cuh', 'common.cuh'), "c2a412f8cf230533471e6093ea6ca476f1bedd003f0d0f0a07475de750bfd4e2",
                      406625280 + 1016199424, "profiles/mimo_proj_b4_l8192_traffic.txt"),
