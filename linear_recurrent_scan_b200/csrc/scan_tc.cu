@@ -22,7 +22,7 @@
 //
 // Design: one CTA per (batch, head) marches over its chunks; the state stays on
 // chip, in fp32 registers of the epilogue warps.  18 warps:
-//   warp 0       TMA producer: B, C, X tiles of chunk c into a 2-stage ring
+//   warp 0       TMA producer: B, C, X tiles of chunk c into a 2-stage ring (3 for N = 64)
 //                (128-byte swizzle, the layout the MMA descriptors read); B and C
 //                of a stage are refilled once the state MMAs have read them, X
 //                once the Y MMA has; theta (+ dt, lam) into single tiles.
@@ -132,7 +132,6 @@ using namespace ptx;
 constexpr int kP = 64;          // head dim handled by this kernel
 constexpr int kM = 128;         // rows per chunk (MMA M)
 constexpr int kTile = 16384;    // one 128-row x 128-byte swizzled tile
-constexpr int kStages = 2;
 constexpr int kThreads = 576;   // 18 warps
 constexpr int kPrep0 = 64;      // first prep thread
 constexpr int kNPrep = 256;
@@ -164,9 +163,12 @@ struct Cfg {
   // measured faster for R = 1 only
   static constexpr bool DEFER_Y = (R == 1);
   static constexpr int STAGE_BYTES = (2 * NKB + 1) * kTile;  // B, C, X
+  // input stages: three where they fit (N = 64: 48 KB each), so that a stage's
+  // refill has a chunk more of lead time; two for N = 128 (80 KB each)
+  static constexpr int NST = N == 64 ? 3 : 2;
   static constexpr int TMA_BYTES = STAGE_BYTES;
   static constexpr int OFF_B = 0, OFF_C = NKB * kTile, OFF_X = 2 * NKB * kTile;
-  static constexpr int OFF_XW = kStages * STAGE_BYTES;   // X_w (single buffer)
+  static constexpr int OFF_XW = NST * STAGE_BYTES;      // X_w (single buffer)
   static constexpr int OFF_TH = OFF_XW + kTile;          // theta tile [Q][N/2] bf16 (single buffer)
   static constexpr int TH_BYTES = Q * K2 * 2;
   static constexpr int OFF_H = OFF_TH + ((TH_BYTES + 1023) & ~1023);  // hbar bf16, N rows x 128 bytes
@@ -174,11 +176,11 @@ struct Cfg {
   // per stage (floats): c2[Q] (log2 of the chunk-local decay), gam[Q], wv[Q],
   // wsc[Q] (X_w row scale), colf[192] (rank-1 column factors of the mask)
   static constexpr int SC_PER_STAGE = 4 * Q + 192;
-  static constexpr int OFF_PART = OFF_SC + kStages * SC_PER_STAGE * 4;  // angle partials [NPART][K2]
+  static constexpr int OFF_PART = OFF_SC + NST * SC_PER_STAGE * 4;  // angle partials [NPART][K2]
   static constexpr int OFF_PHI = OFF_PART + NPART * K2 * 4;            // running base angle [K2]
   static constexpr int OFF_WARP = OFF_PHI + K2 * 4;                     // scan scratch [8]
   static constexpr int OFF_BAR = (OFF_WARP + 32 + 7) & ~7;
-  static constexpr int NBAR = 19;
+  static constexpr int NBAR = 24;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
   // dt and lam of tokens [t0, t0 + Q] for the 8 heads of this head's 16-byte
   // group (TMA tiles [Q + 1][8] bf16, single buffer, refilled with theta)
@@ -222,8 +224,8 @@ struct Cfg {
 
 // barrier slots
 enum Bar {
-  bFull0 = 0, bFull1, bEmptyBC0, bEmptyBC1, bPrep0, bPrep1, bSFull, bAcc, bEpiDone, bPReady, bYFull, bDone,
-  bThFull, bThFree, bEmptyX0, bEmptyX1, bXw, bNorm0, bNorm1
+  bFull0 = 0, bEmptyBC0 = 3, bPrep0 = 6, bEmptyX0 = 9, bNorm0 = 12,  // one per stage (up to 3)
+  bSFull = 15, bAcc, bEpiDone, bPReady, bYFull, bDone, bThFull, bThFree, bXw
 };
 
 struct TcParams {
@@ -253,6 +255,13 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
 __device__ __forceinline__ size_t tok_index(const ScanArgs& a, int b, int t, int h) {
   return ((size_t)b * a.seqlen + t) * a.nheads + h;
 }
+
+// stage of chunk c in an NST-stage ring and the ring's round (for the mbarrier
+// parity); unsigned, so that a two-stage ring compiles to a mask and a shift
+template <int NST>
+__device__ __forceinline__ int stage_of(int c) { return (int)((unsigned)c % NST); }
+template <int NST>
+__device__ __forceinline__ int round_of(int c) { return (int)((unsigned)c / NST); }
 
 // byte offset of 16-byte chunk `c` (0..7) of row `row` inside a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t swz(int row, int c) { return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4)); }
@@ -389,7 +398,7 @@ __device__ __forceinline__ void prep_role(uint8_t* smem, const ScanArgs& a, int 
   prep_sync();
 
   for (int c = 0; c < nchunks; ++c) {
-    const int s = c & 1, u = c >> 1;
+    const int s = stage_of<K::NST>(c), u = round_of<K::NST>(c);
     const int t0 = c * Q;
     float* sc = reinterpret_cast<float*>(smem + K::OFF_SC) + s * K::SC_PER_STAGE;
     float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *wsc = sc + 3 * Q, *colf = sc + 4 * Q;
@@ -830,8 +839,8 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
   // chunk c + 2 follows at the end of chunk c, in the time the epilogue would wait for prep
   float* nw = reinterpret_cast<float*>(smem + K::OFF_NRM);
   auto normalise = [&](int cn) -> bool {
-    const int sn = cn & 1;
-    if (!mbar_wait(&bars[bFull0 + sn], (cn >> 1) & 1, abort_flag, status, kTagFull, a.wait_limit)) return false;
+    const int sn = stage_of<K::NST>(cn);
+    if (!mbar_wait(&bars[bFull0 + sn], round_of<K::NST>(cn) & 1, abort_flag, status, kTagFull, a.wait_limit)) return false;
     bc_normalise<N, R, V>(smem + sn * K::STAGE_BYTES, nw, a.neps, et);
     fence_proxy_async_smem();  // the stage is refilled by TMA later
     mbar_arrive(&bars[bNorm0 + sn]);
@@ -852,7 +861,7 @@ __device__ __forceinline__ void epi_role(uint8_t* smem, const ScanArgs& a, int n
 
   float e_prev = 0.f;  // (deferred y) e^{cum} of row m in the previous chunk
   for (int c = 0; c < nchunks; ++c) {
-    const int s = c & 1, u = c >> 1;
+    const int s = stage_of<K::NST>(c), u = round_of<K::NST>(c);
     const int t0 = (c0 + c) * Q;
     const float* sc = reinterpret_cast<const float*>(smem + K::OFF_SC) + s * K::SC_PER_STAGE;
     const float *c2 = sc, *gm = sc + Q, *wv = sc + 2 * Q, *colf = sc + 4 * Q + colf_off;
@@ -1033,14 +1042,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int units = a.batch * a.nheads;
 
   if (tid == 0) {
-    mbar_init(&bars[bFull0], 1);
-    mbar_init(&bars[bFull1], 1);
-    mbar_init(&bars[bEmptyBC0], 1);
-    mbar_init(&bars[bEmptyBC1], 1);
-    mbar_init(&bars[bEmptyX0], 1);
-    mbar_init(&bars[bEmptyX1], 1);
-    mbar_init(&bars[bPrep0], kNPrep);
-    mbar_init(&bars[bPrep1], kNPrep);
+    for (int i = 0; i < K::NST; ++i) {
+      mbar_init(&bars[bFull0 + i], 1);
+      mbar_init(&bars[bEmptyBC0 + i], 1);
+      mbar_init(&bars[bEmptyX0 + i], 1);
+      mbar_init(&bars[bPrep0 + i], kNPrep);
+      mbar_init(&bars[bNorm0 + i], kNEpi);
+    }
     mbar_init(&bars[bSFull], 1);
     mbar_init(&bars[bAcc], 1);
     mbar_init(&bars[bEpiDone], kNEpi);
@@ -1050,8 +1058,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[bThFull], 1);
     mbar_init(&bars[bThFree], kNPrep);
     mbar_init(&bars[bXw], kNEpi);
-    mbar_init(&bars[bNorm0], kNEpi);
-    mbar_init(&bars[bNorm1], kNEpi);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmB);
@@ -1133,8 +1139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (test_withhold: issue nothing, so that every wait on a load must time out)
       while (!a.test_withhold && (cx < nchunks || ct < nchunks)) {
         bool progress = false;
-        if (cb < nchunks && mbar_test(&bars[bEmptyBC0 + (cb & 1)], ((cb >> 1) & 1) ^ 1)) {
-          const int s = cb & 1, t0 = (c0 + cb) * Q;
+        if (cb < nchunks && mbar_test(&bars[bEmptyBC0 + stage_of<K::NST>(cb)], (round_of<K::NST>(cb) & 1) ^ 1)) {
+          const int s = stage_of<K::NST>(cb), t0 = (c0 + cb) * Q;
           uint8_t* st = smem + s * K::STAGE_BYTES;
           mbar_arrive_expect_tx(&bars[bFull0 + s], K::TMA_BYTES);  // B, C and x of chunk cb
 #pragma unroll
@@ -1145,8 +1151,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++cb;
           progress = true;
         }
-        if (cx < cb && mbar_test(&bars[bEmptyX0 + (cx & 1)], ((cx >> 1) & 1) ^ 1)) {
-          const int s = cx & 1;
+        if (cx < cb && mbar_test(&bars[bEmptyX0 + stage_of<K::NST>(cx)], (round_of<K::NST>(cx) & 1) ^ 1)) {
+          const int s = stage_of<K::NST>(cx);
           tma_load_5d(smem + s * K::STAGE_BYTES + K::OFF_X, &tmX, &bars[bFull0 + s], 0, 0, hh, (c0 + cx) * Q, b);
           ++cx;
           progress = true;
@@ -1179,10 +1185,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // stage whose x load was never issued (abort) gets it now, so that its
       // full barrier can complete.
       for (; cx < cb; ++cx)
-        tma_load_5d(smem + (cx & 1) * K::STAGE_BYTES + K::OFF_X, &tmX, &bars[bFull0 + (cx & 1)], 0, 0, hh,
-                    (c0 + cx) * Q, b);
-      for (int c = cb - 2; c < cb; ++c)
-        if (c >= 0 && !mbar_wait_drain(&bars[bFull0 + (c & 1)], (c >> 1) & 1)) report_timeout(status, kTagDrain);
+        tma_load_5d(smem + stage_of<K::NST>(cx) * K::STAGE_BYTES + K::OFF_X, &tmX,
+                    &bars[bFull0 + stage_of<K::NST>(cx)], 0, 0, hh, (c0 + cx) * Q, b);
+      for (int c = cb - K::NST; c < cb; ++c)
+        if (c >= 0 && !mbar_wait_drain(&bars[bFull0 + stage_of<K::NST>(c)], round_of<K::NST>(c) & 1))
+          report_timeout(status, kTagDrain);
       if (ct > 0 && !mbar_wait_drain(&bars[bThFull], (ct - 1) & 1)) report_timeout(status, kTagDrain);
     }
   } else if (warp == 1) {
@@ -1194,7 +1201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t iY = idesc_bf16(kM, kP, 0, 1);     // Y = P X            (A in TMEM)
       const uint32_t sbase = smem_u32(smem);
       for (int c = 0; c < nchunks; ++c) {
-        const int s = c & 1, u = c >> 1;
+        const int s = stage_of<K::NST>(c), u = round_of<K::NST>(c);
         const uint32_t st = sbase + s * K::STAGE_BYTES;
         const uint32_t cB = st + K::OFF_B, cC = st + K::OFF_C, cX = st + K::OFF_X, cXw = sbase + K::OFF_XW;
         const uint32_t ybuf = K::DEFER_Y ? (c & 1) * kColYBuf : 0u;  // Y, Yi buffer of this chunk
