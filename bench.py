@@ -43,24 +43,24 @@ BACKWARD_KERNEL = "bwd_state_kernel + bwd_chunk_kernel (tcgen05, TMA)"
 # capture).  A kernel whose sources no longer hash to the recorded value gets
 # traffic null, since its counters are out of date.
 TRAFFIC = {
-    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "3b9a2962b96e1b1c16aeeb51b2236b60fb9c7920234041f4f35107e7f24011b4",
-                813935104 + 136358144, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
-    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "3b9a2962b96e1b1c16aeeb51b2236b60fb9c7920234041f4f35107e7f24011b4",
-                               5655001856 + 1070696448, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "448664d301f10051f82172c25f0f7e4448a777edacd6cfbf54b425df8bab2511",
+                813574656 + 137644800, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
+    "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "448664d301f10051f82172c25f0f7e4448a777edacd6cfbf54b425df8bab2511",
+                               5653950464 + 1070973184, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     # the segmented prefill: seg_state_kernel + seg_combine_kernel + scan_tc_kernel of one call
-    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "e2579662912f23b06257e6fce771729caa05e8090e5236f7351108ba21b69ee7",
-                             4590568448 + 36562944 + 38102784 + 131072 + 6774374912 + 2123151872,
+    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "93bd244499048d0f57c7c5bf5bd5a499401dd7e7327ef4732a82edf40c42fca3",
+                             4590572544 + 36198400 + 38102784 + 128512 + 6772852224 + 2121991424,
                              "profiles/segmented_prefill_mimo4_b1_l65536.txt"),
     "siso_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                          283177728 + 219681280, "profiles/decode_stream_b128_traffic_and_counters.txt"),
     "mimo4_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                           317789952 + 241042432, "profiles/decode_stream_b128_traffic_and_counters.txt"),
-    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "3b9a2962b96e1b1c16aeeb51b2236b60fb9c7920234041f4f35107e7f24011b4",
-                        284650496 + 121850368, "profiles/grouped_bc_prefill_decode_traffic.txt"),
+    "grouped_prefill": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "448664d301f10051f82172c25f0f7e4448a777edacd6cfbf54b425df8bab2511",
+                        284654080 + 121231616, "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "grouped_decode": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                        279047936 + 219645952, "profiles/grouped_bc_prefill_decode_traffic.txt"),
     "backward": (('scan_bwd_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "58bdeb0f1b41cb82988d2c19c9a1ca646f603380d204215b052a7ef1a9d4bf3b",
-                 541825792 + 240689408 + 1223041280 + 784799232,
+                 541811456 + 241067776 + 1223138304 + 785098240,
                  "profiles/scan_bwd_tc_siso_b8_l2048_traffic_and_counters.txt"),
     "mimo_proj_up": (('mimo_proj.cu', 'sm100_ptx.cuh', 'common.cuh'), "c2a412f8cf230533471e6093ea6ca476f1bedd003f0d0f0a07475de750bfd4e2",
                      406625280 + 1016199424, "profiles/mimo_proj_b4_l8192_traffic.txt"),
