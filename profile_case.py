@@ -110,7 +110,9 @@ def main():
         dims = m3.make_dims(inp["x"], inp["B"])
         ws = torch.empty(m3.mamba3_scan_bwd_workspace_bytes(dims), dtype=torch.uint8, device=dev)
         grads = None
+        flush = torch.ones(256 << 20, dtype=torch.uint8, device=dev)  # read before each pass: L2 cold
         for i in range(args.reps):
+            flush.sum()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             grads = m3.mamba3_scan_bwd(*(inp[n] for n in NAMES), inp["A"], inp["D"], dy, grads=grads, workspace=ws)
