@@ -35,6 +35,11 @@ constexpr int kP = 64;
 constexpr int kM = 128;          // rows per chunk
 constexpr int kTile = 16384;     // 128 rows x 128 bytes, 128-byte swizzle
 constexpr int kThreads = 256;
+// Besides its share of every chunk's preparation, one lane issues the TMA loads (warp
+// 7), one warp loads the next chunks' scalars (warp 6) and one lane issues the MMAs
+// (thread 0), so that no warp carries more than one of these to the chunk's barrier.
+constexpr int kLoader = kThreads - 32;  // lane 0 of warp 7
+constexpr int kScalarWarp = 6;
 
 enum Tag { kTagFull = 41, kTagMma, kTagDrain };
 
@@ -133,8 +138,8 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
     tma_load_5d(st + K::OFF_X, &tmX, &bars[s], 0, 0, hh, t0, b);
     tma_load_4d(st + K::OFF_TH, &tmT, &bars[s], 0, hh, t0, b);
   };
-  int issued = 0;
-  if (tid == 0 && !a.test_withhold)
+  int issued = 0;  // (the loader's) chunks whose loads were issued
+  if (tid == kLoader && !a.test_withhold)
     for (; issued < D && issued < nchunks; ++issued) issue(issued);
 
   // the segment's total log2 decay (block reduction over its tokens)
@@ -159,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
   // its MMA.  Every warp keeps the decay carry and its groups' running angles.
   constexpr int TPL = Q / 32, GPW = NG / (kThreads / 32);
   static_assert(TPL >= 1 && Q % 32 == 0 && TPL * R == 4 && GPW >= 1 && NG % (kThreads / 32) == 0, "lanes and warps");
-  // dt, lam (and A_t) of a chunk's tokens and the next one: warp 0 loads chunk c + 2's
+  // dt, lam (and A_t) of a chunk's tokens and the next one: one warp loads chunk c + 2's
   // into registers while chunk c is prepared and stores them into buffer c & 1 ... of
   // chunk c + 1 at its end, so that every warp reads them from shared memory (one set of
   // global loads instead of one per warp, and no warp waits on them)
@@ -192,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
       }
     }
   };
-  if (warp == 0) {
+  if (warp == kScalarWarp) {
     load_pre(0);
     store_pre(0);
     load_pre(1);
@@ -321,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
       }
     }
     // load chunk c + D into the stage of chunk c - 1 once that chunk's MMA has read it
-    if (tid == 0 && c + D < nchunks && !a.test_withhold) {
+    if (tid == kLoader && c + D < nchunks && !a.test_withhold) {
       const int prev = c + D - NST;
       if (prev < 0 ||
           mbar_wait(&bars[NST + prev % NST], (prev / NST) & 1, abort_flag, status, kTagMma, a.wait_limit)) {
@@ -351,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
           make_uint4(pack_bf16(fsel * f0.x, fsel * f0.y), pack_bf16(fsel * f1.x, fsel * f1.y),
                      pack_bf16(fsel * f2.x, fsel * f2.y), pack_bf16(fsel * f3.x, fsel * f3.y));
     }
-    if (warp == 0) {  // chunk c + 1's scalars for the next iteration; chunk c + 2's in flight
+    if (warp == kScalarWarp) {  // chunk c + 1's scalars for the next iteration; chunk c + 2's in flight
       store_pre((c + 1) & 1);
       load_pre(c + 2);
     }
@@ -386,14 +391,15 @@ __global__ void __launch_bounds__(kThreads, GCfg<N, R>::CPS) seg_state_kernel(co
     if (abort_c < 0 && nchunks > 0)
       mbar_wait(&bars[NST + (nchunks - 1) % NST], ((nchunks - 1) / NST) & 1, abort_flag, status, kTagMma,
                 a.wait_limit);
-    if (*abort_flag) {
-      // let the copies and MMAs issued land before TMEM is freed and the CTA exits
-      for (int c2 = abort_c >= 0 ? abort_c : nchunks; c2 < issued; ++c2)
-        if (!mbar_wait_drain(&bars[c2 % NST], (c2 / NST) & 1)) report_timeout(status, kTagDrain);
-      if (mma_issued > 0 &&
-          !mbar_wait_drain(&bars[NST + (mma_issued - 1) % NST], ((mma_issued - 1) / NST) & 1))
-        report_timeout(status, kTagDrain);
-    }
+    // after an abort, let the MMAs issued land before TMEM is freed and the CTA exits
+    if (*abort_flag && mma_issued > 0 &&
+        !mbar_wait_drain(&bars[NST + (mma_issued - 1) % NST], ((mma_issued - 1) / NST) & 1))
+      report_timeout(status, kTagDrain);
+  }
+  __syncthreads();  // the abort flag as thread 0 left it
+  if (tid == kLoader && *abort_flag) {  // and the copies issued land before the CTA exits
+    for (int c2 = abort_c >= 0 ? abort_c : nchunks; c2 < issued; ++c2)
+      if (!mbar_wait_drain(&bars[c2 % NST], (c2 / NST) & 1)) report_timeout(status, kTagDrain);
   }
   if (__syncthreads_or(*abort_flag != 0)) {
     // aborted: outputs undefined, the status word says so

@@ -70,3 +70,26 @@ def test_decode_timeout_is_reported_and_context_survives():
     assert m3.mamba3_library_status() == m3.MAMBA3_OK
     yr, _ = oracle_scan(pre)
     assert rel_err(y.float().cpu().double().numpy(), yr[:, 0]) < TOL[torch.bfloat16]
+
+
+def test_segmented_prefill_timeout_is_reported_and_context_survives():
+    """The segmented path (segment end states, their chaining, the prefill of the
+    segments) with every input copy withheld: the segment-state pass and the prefill
+    pass give up, the status says so, and the next call is correct."""
+    b, L, H, P, N, R = 1, 512, 2, 64, 64, 4
+    inp = small_inputs(b, L, H, P, N, R, torch.bfloat16, seed=5300)
+    dims = m3.make_dims(inp["x"], inp["B"])
+    m3.mamba3_test_set_segments(4)
+    try:
+        need = m3.mamba3_scan_segmented_workspace_bytes(dims)
+        assert need > m3.mamba3_scan_workspace_bytes(dims)  # the segmented path is taken
+        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        y = torch.empty_like(inp["x"])
+        _starved(lambda: m3.mamba3_scan_fwd(*(inp[n] for n in NAMES), inp["A"], inp["D"], y=y, workspace=ws))
+        assert m3.mamba3_device_status(ws) == m3.MAMBA3_ERR_TIMEOUT
+        y = m3.mamba3_scan_fwd(*(inp[n] for n in NAMES), inp["A"], inp["D"], y=y, workspace=ws)
+        assert m3.mamba3_device_status(ws) == m3.MAMBA3_OK
+    finally:
+        m3.mamba3_test_set_segments(0)
+    yr, _ = oracle_scan(inp)
+    assert rel_err(y.float().cpu().double().numpy(), yr) < TOL[torch.bfloat16]
