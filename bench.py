@@ -48,8 +48,8 @@ TRAFFIC = {
     "mimo4_prefill_b4_l8192": (('scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "448664d301f10051f82172c25f0f7e4448a777edacd6cfbf54b425df8bab2511",
                                5653950464 + 1070973184, "profiles/scan_tc_prefill_traffic_and_counters.txt"),
     # the segmented prefill: seg_state_kernel + seg_combine_kernel + scan_tc_kernel of one call
-    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "93bd244499048d0f57c7c5bf5bd5a499401dd7e7327ef4732a82edf40c42fca3",
-                             4590572544 + 36198400 + 38102784 + 128512 + 6772852224 + 2121991424,
+    "mimo4_long_b1_l65536": (('seg_state.cu', 'scan_seg.cu', 'scan_tc.cu', 'sm100_ptx.cuh', 'common.cuh'), "887c8a24ebd2ffc028fa17604efd17f2226f4deff7eb31d43698c2c8b2f2e9ee",
+                             4590757632 + 36491776 + 38109696 + 322304 + 6772821504 + 2121624832,
                              "profiles/segmented_prefill_mimo4_b1_l65536.txt"),
     "siso_decode_b128": (('decode.cu', 'sm100_ptx.cuh', 'common.cuh'), "9209a603433cf2acc54a602e33acfa286eefb362ab1303717af46b2effb2b96c",
                          283177728 + 219681280, "profiles/decode_stream_b128_traffic_and_counters.txt"),
